@@ -1,0 +1,31 @@
+"""B200-native 1.5-entmax ("AdaSplash") attention.
+
+Multi-head attention whose softmax is replaced by Tsallis 1.5-entmax: per query row,
+tau solves sum_j max(0, (S_ij - tau)/2)^2 = 1 by bisection, A = max(0, (S - tau)/2)^2 has exact
+zeros, O = A V; the backward pass uses the closed-form Jacobian.  The work runs in hand-written
+sm_100a kernels (tcgen05 tensor cores, TMEM, TMA) behind the C ABI in include/entmax_attn.h;
+this package is its thin Python binding.
+"""
+from ._binding import (  # noqa: F401
+    ENTMAX_BF16,
+    ENTMAX_ERR_ARG,
+    ENTMAX_ERR_CUDA,
+    ENTMAX_ERR_TIMEOUT,
+    ENTMAX_ERR_UNSUPPORTED,
+    ENTMAX_ERR_WORKSPACE,
+    ENTMAX_F32,
+    ENTMAX_OK,
+    EXPORTED,
+    LIB_PATH,
+    EntmaxAttention,
+    EntmaxError,
+    entmax_attn_bwd,
+    entmax_attn_bwd_workspace_size,
+    entmax_attn_device_status,
+    entmax_attn_fwd,
+    entmax_attn_last_cuda_error,
+    entmax_attn_set_wait_timeout_ns,
+    lib,
+    strerror,
+    version,
+)

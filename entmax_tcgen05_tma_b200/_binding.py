@@ -1,0 +1,211 @@
+"""ctypes binding of libentmax_attn.so (include/entmax_attn.h).
+
+Argument marshalling only: checks tensor placement/dtype/contiguity, allocates outputs with
+torch when the caller gives none, passes raw device pointers and the current CUDA stream, and
+turns status codes into exceptions.  All arithmetic runs in the library's CUDA kernels; there is
+no CPU path.  A missing or unloadable library raises at import.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libentmax_attn.so"
+
+ENTMAX_OK = 0
+ENTMAX_ERR_ARG = -1
+ENTMAX_ERR_UNSUPPORTED = -2
+ENTMAX_ERR_CUDA = -3
+ENTMAX_ERR_TIMEOUT = -4
+ENTMAX_ERR_WORKSPACE = -5
+ENTMAX_BF16 = 0
+ENTMAX_F32 = 1
+
+EXPORTED = (
+    "entmax_attn_fwd",
+    "entmax_attn_bwd_workspace_size",
+    "entmax_attn_bwd",
+    "entmax_attn_strerror",
+    "entmax_attn_device_status",
+    "entmax_attn_last_cuda_error",
+    "entmax_attn_set_wait_timeout_ns",
+    "entmax_attn_version",
+)
+
+
+class EntmaxError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (what, strerror(status), status))
+
+
+def _load_library() -> ctypes.CDLL:
+    if not LIB_PATH.exists():
+        raise ImportError(
+            "libentmax_attn.so is not built (%s); run `python -m entmax_tcgen05_tma_b200.build`" % LIB_PATH)
+    lib = ctypes.CDLL(str(LIB_PATH))
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.entmax_attn_fwd.restype = i
+    lib.entmax_attn_fwd.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, i, vp, vp]
+    lib.entmax_attn_bwd_workspace_size.restype = sz
+    lib.entmax_attn_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.entmax_attn_bwd.restype = i
+    lib.entmax_attn_bwd.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.entmax_attn_strerror.restype = ctypes.c_char_p
+    lib.entmax_attn_strerror.argtypes = [i]
+    lib.entmax_attn_device_status.restype = i
+    lib.entmax_attn_device_status.argtypes = [vp]
+    lib.entmax_attn_last_cuda_error.restype = i
+    lib.entmax_attn_last_cuda_error.argtypes = []
+    lib.entmax_attn_set_wait_timeout_ns.restype = None
+    lib.entmax_attn_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+    lib.entmax_attn_version.restype = i
+    lib.entmax_attn_version.argtypes = []
+    return lib
+
+
+lib = _load_library()
+
+
+def strerror(status: int) -> str:
+    return lib.entmax_attn_strerror(int(status)).decode()
+
+
+def version() -> int:
+    return lib.entmax_attn_version()
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ENTMAX_BF16
+    if t.dtype == torch.float32:
+        return ENTMAX_F32
+    raise TypeError("inputs must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _check_input(name: str, t: torch.Tensor, shape, dtype=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def _mask_ptr(key_mask, B: int, L: int, device) -> int | None:
+    if key_mask is None:
+        return None
+    _check_input("key_mask", key_mask, (B, L))
+    if key_mask.dtype not in (torch.uint8, torch.bool):
+        raise TypeError("key_mask must be uint8 or bool")
+    if key_mask.device != device:
+        raise ValueError("key_mask must be on the same device as Q")
+    return key_mask.data_ptr()
+
+
+def entmax_attn_fwd(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
+                    O=None, tau=None, stream=None):
+    """1.5-entmax attention forward.  Q, K, V: [B,H,L,64] bf16 or fp32 CUDA tensors.
+
+    Returns (O, tau): O [B,H,L,64] in ``out_dtype``; tau [B,H,L] fp32 thresholds.
+    """
+    B, H, L, D = Q.shape
+    _check_input("Q", Q, (B, H, L, D))
+    _check_input("K", K, (B, H, L, D), Q.dtype)
+    _check_input("V", V, (B, H, L, D), Q.dtype)
+    if scale is None:
+        scale = D ** -0.5
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be bfloat16 or float32")
+    if O is None:
+        O = torch.empty((B, H, L, D), dtype=out_dtype, device=Q.device)
+    else:
+        _check_input("O", O, (B, H, L, D), out_dtype)
+    if tau is None:
+        tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
+    else:
+        _check_input("tau", tau, (B, H, L), torch.float32)
+    st = lib.entmax_attn_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
+                             _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale),
+                             B, H, L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16,
+                             tau.data_ptr(), _stream_handle(stream))
+    if st != ENTMAX_OK:
+        raise EntmaxError(st, "entmax_attn_fwd")
+    return O, tau
+
+
+def entmax_attn_bwd_workspace_size(B: int, H: int, L: int, D: int = 64) -> int:
+    return int(lib.entmax_attn_bwd_workspace_size(B, H, L, D))
+
+
+def entmax_attn_bwd(Q, K, V, tau, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None, dK=None,
+                    dV=None, workspace=None, stream=None):
+    """Closed-form backward.  Returns (dQ, dK, dV), fp32 [B,H,L,64]."""
+    B, H, L, D = Q.shape
+    _check_input("Q", Q, (B, H, L, D))
+    _check_input("K", K, (B, H, L, D), Q.dtype)
+    _check_input("V", V, (B, H, L, D), Q.dtype)
+    _check_input("dO", dO, (B, H, L, D), Q.dtype)
+    _check_input("tau", tau, (B, H, L), torch.float32)
+    if scale is None:
+        scale = D ** -0.5
+    outs = []
+    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        if t is None:
+            t = torch.empty((B, H, L, D), dtype=torch.float32, device=Q.device)
+        else:
+            _check_input(name, t, (B, H, L, D), torch.float32)
+        outs.append(t)
+    ws_bytes = entmax_attn_bwd_workspace_size(B, H, L, D)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=Q.device)
+    st = lib.entmax_attn_bwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
+                             _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale),
+                             B, H, L, D, tau.data_ptr(), dO.data_ptr(), outs[0].data_ptr(), outs[1].data_ptr(),
+                             outs[2].data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream_handle(stream))
+    if st != ENTMAX_OK:
+        raise EntmaxError(st, "entmax_attn_bwd")
+    return tuple(outs)
+
+
+def entmax_attn_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(lib.entmax_attn_device_status(_stream_handle(stream)))
+
+
+def entmax_attn_set_wait_timeout_ns(ns: int) -> None:
+    lib.entmax_attn_set_wait_timeout_ns(int(ns))
+
+
+def entmax_attn_last_cuda_error() -> int:
+    return int(lib.entmax_attn_last_cuda_error())
+
+
+class EntmaxAttention(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run in the library's kernels."""
+
+    @staticmethod
+    def forward(ctx, Q, K, V, key_mask=None, causal=False, window=0, scale=None):
+        O, tau = entmax_attn_fwd(Q, K, V, key_mask, causal, window, scale)
+        ctx.save_for_backward(Q, K, V, tau, key_mask if key_mask is not None else torch.empty(0))
+        ctx.cfg = (key_mask is not None, causal, window, scale)
+        return O
+
+    @staticmethod
+    def backward(ctx, dO):
+        Q, K, V, tau, km = ctx.saved_tensors
+        has_mask, causal, window, scale = ctx.cfg
+        dQ, dK, dV = entmax_attn_bwd(Q, K, V, tau, dO.to(Q.dtype).contiguous(), km if has_mask else None, causal,
+                                     window, scale)
+        return dQ.to(Q.dtype), dK.to(K.dtype), dV.to(V.dtype), None, None, None, None

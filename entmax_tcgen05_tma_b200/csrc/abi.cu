@@ -1,0 +1,252 @@
+// abi.cu -- the extern "C" entry points of libentmax_attn.so: argument checks, tensor maps,
+// the device status word, fp32-input conversion, and kernel launches.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+#include "../../include/entmax_attn.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace entmax {
+
+namespace {
+
+__device__ int g_device_status;  // ENTMAX_OK or the first device-side error since the last read
+
+constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;
+unsigned long long g_timeout_ns = DEFAULT_TIMEOUT_NS;
+int g_last_cuda_error = 0;
+constexpr int MAX_DEVICES = 64;
+int* g_status_ptr[MAX_DEVICES] = {};
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int record(cudaError_t e) {
+    if (e == cudaSuccess) return ENTMAX_OK;
+    g_last_cuda_error = (int)e;
+    return ENTMAX_ERR_CUDA;
+}
+
+cudaError_t status_ptr(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_status);
+        if (e != cudaSuccess) return e;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    *out = g_status_ptr[dev];
+    return cudaSuccess;
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (; i < n; i += stride) dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_common(const void* Q, const void* K, const void* V, int in_dtype, int causal, int window, float scale,
+                 int B, int H, int L, int D) {
+    if (B < 0 || H < 0 || L < 0) return ENTMAX_ERR_ARG;
+    if (in_dtype != ENTMAX_BF16 && in_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return ENTMAX_ERR_ARG;
+    if (window < 0 || (causal != 0 && causal != 1)) return ENTMAX_ERR_ARG;
+    if (D != HEAD_DIM) return ENTMAX_ERR_UNSUPPORTED;
+    if (window > 0 && !causal) return ENTMAX_ERR_UNSUPPORTED;
+    if (L > MAX_L) return ENTMAX_ERR_UNSUPPORTED;
+    if ((long long)B * H > 65535) return ENTMAX_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
+    if (!Q || !K || !V) return ENTMAX_ERR_ARG;
+    if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16)) return ENTMAX_ERR_ARG;
+    return ENTMAX_OK;
+}
+
+// bf16 copies of fp32 inputs, in stream-ordered temporaries.
+struct Bf16Copies {
+    void* buf = nullptr;
+    cudaStream_t stream = nullptr;
+    ~Bf16Copies() {
+        if (buf) cudaFreeAsync(buf, stream);
+    }
+};
+
+cudaError_t convert_inputs(const void* const* src, const void** dst, int count, size_t n_each, Bf16Copies& tmp,
+                           cudaStream_t stream) {
+    tmp.stream = stream;
+    const size_t bytes_each = n_each * 2;
+    const size_t pitch = (bytes_each + 255) & ~size_t(255);
+    cudaError_t e = cudaMallocAsync(&tmp.buf, pitch * count, stream);
+    if (e != cudaSuccess) {
+        tmp.buf = nullptr;
+        return e;
+    }
+    for (int k = 0; k < count; ++k) {
+        void* d = static_cast<uint8_t*>(tmp.buf) + pitch * k;
+        e = launch_f32_to_bf16(static_cast<const float*>(src[k]), d, n_each, stream);
+        if (e != cudaSuccess) return e;
+        dst[k] = d;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, cudaStream_t stream) {
+    const int threads = 256;
+    const size_t blocks = std::min<size_t>((n + threads - 1) / threads, 148 * 16);
+    f32_to_bf16_kernel<<<(unsigned)std::max<size_t>(blocks, 1), threads, 0, stream>>>(
+        src, static_cast<__nv_bfloat16*>(dst), n);
+    return cudaGetLastError();
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes, int slot) {
+    static bool done[8][MAX_DEVICES] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= MAX_DEVICES || slot < 0 || slot >= 8) return cudaErrorInvalidValue;
+    if (done[slot][dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[slot][dev] = true;
+    return e;
+}
+
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+            if (e != cudaSuccess) return e;
+            if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)HEAD_DIM, (cuuint64_t)L, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)HEAD_DIM * 2, (cuuint64_t)L * HEAD_DIM * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)HEAD_DIM, (cuuint32_t)TILE, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace entmax
+
+using namespace entmax;
+
+extern "C" {
+
+int entmax_attn_version(void) { return 100; }
+
+const char* entmax_attn_strerror(int status) {
+    switch (status) {
+        case ENTMAX_OK: return "ok";
+        case ENTMAX_ERR_ARG: return "invalid argument";
+        case ENTMAX_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ENTMAX_ERR_CUDA: return "CUDA error";
+        case ENTMAX_ERR_TIMEOUT: return "device wait timed out";
+        case ENTMAX_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int entmax_attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+void entmax_attn_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns = ns ? ns : DEFAULT_TIMEOUT_NS; }
+
+int entmax_attn_device_status(cudaStream_t stream) {
+    int* p = nullptr;
+    int rc = record(status_ptr(&p));
+    if (rc) return rc;
+    rc = record(cudaStreamSynchronize(stream));
+    if (rc) return rc;
+    int v = 0;
+    rc = record(cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost));
+    if (rc) return rc;
+    const int zero = 0;
+    rc = record(cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice));
+    if (rc) return rc;
+    return v;
+}
+
+int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+                    int window, float scale, int B, int H, int L, int D, void* O, int out_dtype, float* tau,
+                    cudaStream_t stream) {
+    int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
+    if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
+    if (!O || !tau) return ENTMAX_ERR_ARG;
+    if (!aligned(O, 8) || !aligned(tau, 4)) return ENTMAX_ERR_ARG;
+    int* status = nullptr;
+    rc = record(status_ptr(&status));
+    if (rc) return rc;
+
+    const size_t n = (size_t)B * H * L * HEAD_DIM;
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    Bf16Copies tmp;
+    if (in_dtype == ENTMAX_F32) {
+        const void* src[3] = {Q, K, V};
+        const void* dst[3];
+        rc = record(convert_inputs(src, dst, 3, n, tmp, stream));
+        if (rc) return rc;
+        a.Q = dst[0];
+        a.K = dst[1];
+        a.V = dst[2];
+    }
+    FwdOut o{O, out_dtype == ENTMAX_F32, tau};
+    return record(launch_fwd(a, o, stream));
+}
+
+size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D) {
+    (void)D;
+    if (B <= 0 || H <= 0 || L <= 0) return 0;
+    return (((size_t)B * H * L * sizeof(float)) + 255) & ~size_t(255);
+}
+
+int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+                    int window, float scale, int B, int H, int L, int D, const float* tau, const void* dO, float* dQ,
+                    float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
+    if (!tau || !dO || !dQ || !dK || !dV) return ENTMAX_ERR_ARG;
+    if (!aligned(dO, 16) || !aligned(dQ, 8) || !aligned(dK, 8) || !aligned(dV, 8) || !aligned(tau, 4))
+        return ENTMAX_ERR_ARG;
+    if (!workspace || ws_bytes < entmax_attn_bwd_workspace_size(B, H, L, D)) return ENTMAX_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return ENTMAX_ERR_ARG;
+    int* status = nullptr;
+    rc = record(status_ptr(&status));
+    if (rc) return rc;
+
+    const size_t n = (size_t)B * H * L * HEAD_DIM;
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    BwdIO io{tau, dO, dQ, dK, dV, static_cast<float*>(workspace)};
+    Bf16Copies tmp;
+    if (in_dtype == ENTMAX_F32) {
+        const void* src[4] = {Q, K, V, dO};
+        const void* dst[4];
+        rc = record(convert_inputs(src, dst, 4, n, tmp, stream));
+        if (rc) return rc;
+        a.Q = dst[0];
+        a.K = dst[1];
+        a.V = dst[2];
+        io.dO = dst[3];
+    }
+    return record(launch_bwd(a, io, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,129 @@
+/*
+ * entmax_attn.h -- C ABI of the B200 (sm_100a) 1.5-entmax attention library.
+ *
+ * Operation (page "svd-sst2-roberta-adasplash", sections 2.2-2.4 and 3; model cards
+ * "roberta-base-adasplash" and "distilbert-sst2-adasplash", "Mathematical Formulation"):
+ * multi-head attention whose softmax is replaced by Tsallis 1.5-entmax.  For each batch b,
+ * head h and query row i:
+ *
+ *   S_ij   = scale * <Q_i, K_j>                      for the allowed keys j,
+ *   tau_i  : the unique root of sum_j max(0, (S_ij - tau_i)/2)^2 = 1   (Theorem 1),
+ *            found by bisection on [max_j S_ij - 2, max_j S_ij - 2/sqrt(n_i)] (Theorem 2 and the
+ *            model cards' bracket; n_i = number of allowed keys), at most 25 halvings,
+ *   A_ij   = max(0, (S_ij - tau_i)/2)^2  (exact zeros off the support),
+ *   O_i    = sum_j A_ij V_j.
+ *
+ * Allowed keys (section 3, "Structural Masking Stage"): key j is allowed for query i iff
+ *   key_mask[b, j] != 0 (key padding; NULL means every key is valid),
+ *   and, if causal, j <= i,
+ *   and, if window > 0, j >= i - window + 1 (a causal sliding window of `window` keys
+ *   including the query itself; window requires causal).
+ * Masked keys are excluded, not filled with a large negative value.  A row with no allowed
+ * key gets O_i = 0, tau_i = +inf and zero gradients.
+ *
+ * Layout: Q, K, V, dO, O, dQ, dK, dV are contiguous row-major [B, H, L, D] tensors; tau is
+ * [B, H, L]; key_mask is [B, L] bytes.  D must be 64.  All pointers are DEVICE pointers owned
+ * by the caller; the library keeps no reference after a call returns.  Every call is
+ * asynchronous on `stream` (0 = the legacy default stream).
+ *
+ * Errors: arguments are checked on the host before any launch; a bad argument returns a
+ * negative status and launches nothing.  Problems found on the device (a bounded wait that
+ * timed out) are recorded in a device status word; entmax_attn_device_status() reads it.
+ */
+#ifndef ENTMAX_ATTN_H
+#define ENTMAX_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define ENTMAX_API __attribute__((visibility("default")))
+#else
+#define ENTMAX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ENTMAX_OK = 0,
+    ENTMAX_ERR_ARG = -1,          /* null pointer, bad size, bad dtype, misaligned pointer, scale <= 0 */
+    ENTMAX_ERR_UNSUPPORTED = -2,  /* D != 64, L > 16384, B*H > 65535, window without causal */
+    ENTMAX_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed (see entmax_attn_last_cuda_error) */
+    ENTMAX_ERR_TIMEOUT = -4,      /* a device-side bounded wait expired */
+    ENTMAX_ERR_WORKSPACE = -5     /* workspace missing or smaller than entmax_attn_bwd_workspace_size */
+} entmax_status;
+
+typedef enum {
+    ENTMAX_BF16 = 0,
+    ENTMAX_F32 = 1
+} entmax_dtype;
+
+/*
+ * Forward pass.
+ *   Q, K, V   [B,H,L,D] in `in_dtype`.  ENTMAX_F32 inputs are rounded to bf16 (round to
+ *             nearest even) on the device before use; the arithmetic is bf16 x bf16 products
+ *             with fp32 accumulation either way.  16-byte aligned.
+ *   key_mask  [B,L] uint8, 1 = valid key; NULL = all valid.
+ *   causal    0/1.   window: keys per row including the query (0 = off; > 0 needs causal).
+ *   scale     > 0, multiplies Q.K (1/sqrt(D) on the pages' encoders).
+ *   O         [B,H,L,D] in `out_dtype` (bf16 or fp32), 8-byte aligned.
+ *   tau       [B,H,L] fp32, the threshold in score units: A_ij = max(0,(S_ij - tau_i)/2)^2.
+ *             Needed by the backward pass.
+ * Returns ENTMAX_OK once the work is queued on `stream`.  B, H or L equal to 0 is a no-op.
+ */
+ENTMAX_API int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype,
+                    const uint8_t* key_mask, int causal, int window, float scale,
+                    int B, int H, int L, int D,
+                    void* O, int out_dtype, float* tau, cudaStream_t stream);
+
+/* Bytes of device workspace entmax_attn_bwd needs: one float per query row (the row
+ * scalar u_i passed from the dQ kernel to the dK/dV kernel), rounded up to 256 bytes.
+ * 0 when B, H or L is 0. */
+ENTMAX_API size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D);
+
+/*
+ * Backward pass for the loss gradient dO = dL/dO, by the closed-form Jacobian of section 2.4
+ * (page "svd-sst2-roberta-adasplash"; model card "roberta-base-adasplash", section 2):
+ *   dA_ij = <dO_i, V_j>,  sp_ij = sqrt(A_ij),  u_i = sum_j sp_ij dA_ij / sum_j sp_ij,
+ *   dS_ij = sp_ij (dA_ij - u_i),
+ *   dQ_i = scale sum_j dS_ij K_j,  dK_j = scale sum_i dS_ij Q_i,  dV_j = sum_i A_ij dO_i.
+ *   Q, K, V, dO  [B,H,L,D] in `in_dtype` (fp32 inputs are rounded to bf16 first).
+ *   tau          [B,H,L] from entmax_attn_fwd with the same Q, K, masks and scale.
+ *   dQ, dK, dV   [B,H,L,D] fp32, fully overwritten.  8-byte aligned.
+ *   workspace    device buffer of at least entmax_attn_bwd_workspace_size(B,H,L,D) bytes,
+ *                16-byte aligned, owned by the caller; its contents need no initialisation.
+ * fp32 inputs additionally use stream-ordered temporaries (cudaMallocAsync) for their bf16
+ * copies; bf16 inputs allocate nothing.
+ */
+ENTMAX_API int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype,
+                    const uint8_t* key_mask, int causal, int window, float scale,
+                    int B, int H, int L, int D,
+                    const float* tau, const void* dO,
+                    float* dQ, float* dK, float* dV,
+                    void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Static description of a status code. */
+ENTMAX_API const char* entmax_attn_strerror(int status);
+
+/* Synchronises `stream`, then returns and clears the device status word of the current device:
+ * ENTMAX_OK, or ENTMAX_ERR_TIMEOUT if a kernel's bounded wait expired since the last read. */
+ENTMAX_API int entmax_attn_device_status(cudaStream_t stream);
+
+/* cudaError_t value of the most recent failed CUDA call inside the library (0 if none). */
+ENTMAX_API int entmax_attn_last_cuda_error(void);
+
+/* Bound on each device-side wait, in nanoseconds; 0 restores the default (2 s).  Affects
+ * launches made after the call.  Intended for tests of the timeout path. */
+ENTMAX_API void entmax_attn_set_wait_timeout_ns(unsigned long long ns);
+
+/* Library version, major*10000 + minor*100 + patch. */
+ENTMAX_API int entmax_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENTMAX_ATTN_H */

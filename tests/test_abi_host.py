@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI: the library loads, exports every function include/*.h
+declares, and rejects bad arguments before touching the GPU.  No compute call is made: every
+call here fails validation (or is a documented no-op) before any CUDA API is reached, and the
+pointers passed are never dereferenced on the host."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import entmax_tcgen05_tma_b200 as E
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def _declared():
+    names = set()
+    for h in (ROOT / "include").glob("*.h"):
+        for m in re.finditer(r"ENTMAX_API\s+[\w\s\*]+?\b(entmax_\w+)\s*\(", h.read_text()):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_abi():
+    assert set(_declared()) == set(E.EXPORTED)
+
+
+@pytest.mark.parametrize("name", _declared())
+def test_library_exports(name):
+    lib = ctypes.CDLL(str(E.LIB_PATH))
+    assert hasattr(lib, name)
+
+
+def test_strerror_and_version():
+    assert E.strerror(0) == "ok"
+    for code in (-1, -2, -3, -4, -5):
+        assert E.strerror(code) != "unknown status"
+    assert E.strerror(12345) == "unknown status"
+    assert E.version() >= 100
+
+
+def test_workspace_size():
+    assert E.entmax_attn_bwd_workspace_size(0, 12, 128) == 0
+    n = E.entmax_attn_bwd_workspace_size(4, 12, 4096)
+    assert n >= 4 * 12 * 4096 * 4 and n % 256 == 0
+
+
+P = 0x10000  # fake, 16-byte aligned device address: never dereferenced by these calls
+
+
+def _fwd(**kw):
+    a = dict(Q=P, K=P, V=P, in_dtype=0, mask=None, causal=0, window=0, scale=0.125, B=1, H=1, L=64, D=64,
+             O=P, out_dtype=0, tau=P, stream=None)
+    a.update(kw)
+    return E.lib.entmax_attn_fwd(a["Q"], a["K"], a["V"], a["in_dtype"], a["mask"], a["causal"], a["window"],
+                                 a["scale"], a["B"], a["H"], a["L"], a["D"], a["O"], a["out_dtype"], a["tau"],
+                                 a["stream"])
+
+
+def _bwd(**kw):
+    a = dict(Q=P, K=P, V=P, in_dtype=0, mask=None, causal=0, window=0, scale=0.125, B=1, H=1, L=64, D=64, tau=P,
+             dO=P, dQ=P, dK=P, dV=P, ws=P, ws_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return E.lib.entmax_attn_bwd(a["Q"], a["K"], a["V"], a["in_dtype"], a["mask"], a["causal"], a["window"],
+                                 a["scale"], a["B"], a["H"], a["L"], a["D"], a["tau"], a["dO"], a["dQ"], a["dK"],
+                                 a["dV"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=32), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(D=128), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(L=16385), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(B=300, H=300), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(window=32, causal=0), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(window=-1, causal=1), E.ENTMAX_ERR_ARG),
+    (dict(causal=2), E.ENTMAX_ERR_ARG),
+    (dict(in_dtype=7), E.ENTMAX_ERR_ARG),
+    (dict(out_dtype=3), E.ENTMAX_ERR_ARG),
+    (dict(scale=0.0), E.ENTMAX_ERR_ARG),
+    (dict(scale=-0.125), E.ENTMAX_ERR_ARG),
+    (dict(scale=float("nan")), E.ENTMAX_ERR_ARG),
+    (dict(scale=float("inf")), E.ENTMAX_ERR_ARG),
+    (dict(Q=None), E.ENTMAX_ERR_ARG),
+    (dict(V=None), E.ENTMAX_ERR_ARG),
+    (dict(O=None), E.ENTMAX_ERR_ARG),
+    (dict(tau=None), E.ENTMAX_ERR_ARG),
+    (dict(K=P + 8), E.ENTMAX_ERR_ARG),
+    (dict(O=P + 4), E.ENTMAX_ERR_ARG),
+    (dict(B=-1), E.ENTMAX_ERR_ARG),
+    (dict(B=0), E.ENTMAX_OK),
+    (dict(L=0, Q=None, K=None, V=None, O=None, tau=None), E.ENTMAX_OK),
+])
+def test_fwd_argument_checks(kw, code):
+    assert _fwd(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=16), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(window=4), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(tau=None), E.ENTMAX_ERR_ARG),
+    (dict(dO=None), E.ENTMAX_ERR_ARG),
+    (dict(dQ=None), E.ENTMAX_ERR_ARG),
+    (dict(dV=None), E.ENTMAX_ERR_ARG),
+    (dict(dO=P + 2), E.ENTMAX_ERR_ARG),
+    (dict(dK=P + 4), E.ENTMAX_ERR_ARG),
+    (dict(ws=None), E.ENTMAX_ERR_WORKSPACE),
+    (dict(ws_bytes=64 * 4 - 1), E.ENTMAX_ERR_WORKSPACE),
+    (dict(ws=P + 4), E.ENTMAX_ERR_ARG),
+    (dict(B=0), E.ENTMAX_OK),
+])
+def test_bwd_argument_checks(kw, code):
+    assert _bwd(**kw) == code
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+
+    x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        E.entmax_attn_fwd(x, x, x)

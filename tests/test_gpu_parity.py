@@ -1,0 +1,200 @@
+"""GPU (sm_100a kernels through the C ABI) vs the fp64 oracle, element by element.
+
+Small shapes span several 128-row tiles and ragged tails and are compared in full; the five
+workloads at full size run in the launch configuration bench.py times and are compared on
+sampled rows (forward) and sampled heads (backward).  Tolerances: tests/gpu_helpers.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from entmax_tcgen05_tma_b200 import entmax_attn_bwd, entmax_attn_device_status, entmax_attn_fwd
+from entmax_tcgen05_tma_b200.workloads import WORKLOADS, Workload, make_inputs
+from oracle import oracle as orc
+from tests.gpu_helpers import GRAD_TOL, O_TOL, check_rows, inputs_f64, to64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _gpu_fwd(inp, w: Workload, out_dtype=torch.float32):
+    Q, K, V = (inp[k].to(DEV) for k in ("Q", "K", "V"))
+    km = None if inp["key_mask"] is None else inp["key_mask"].to(DEV)
+    O, tau = entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, out_dtype=out_dtype)
+    assert entmax_attn_device_status() == 0
+    return O, tau, (Q, K, V, km)
+
+
+def _gpu_bwd(dev_inp, tau, dO, w: Workload):
+    Q, K, V, km = dev_inp
+    dQ, dK, dV = entmax_attn_bwd(Q, K, V, tau, dO.to(DEV), km, w.causal, w.window, w.scale)
+    assert entmax_attn_device_status() == 0
+    return dQ, dK, dV
+
+
+def _mask_np(inp):
+    return None if inp["key_mask"] is None else inp["key_mask"].numpy()
+
+
+SMALL = [
+    # B, H, L, scale, causal, window, len_range
+    (1, 2, 64, 1 / 8, False, 0, None),
+    (2, 2, 1, 1 / 8, False, 0, None),
+    (2, 3, 17, 1 / 8, False, 0, None),
+    (1, 2, 127, 1 / 8, False, 0, None),
+    (1, 2, 128, 1 / 8, False, 0, None),
+    (2, 1, 129, 1 / 8, False, 0, None),
+    (3, 2, 300, 1 / 8, False, 0, (1, 300)),
+    (2, 2, 300, 2 / 8, False, 0, None),
+    (2, 2, 300, 1 / 8, True, 0, None),
+    (2, 2, 300, 1 / 8, True, 32, None),
+    (1, 2, 513, 1 / 8, True, 0, (200, 513)),
+    (1, 1, 700, 2 / 8, True, 5, None),
+]
+
+
+@pytest.mark.parametrize("B,H,L,scale,causal,window,lens", SMALL)
+def test_small_fwd_bwd_full_parity(B, H, L, scale, causal, window, lens):
+    w = Workload(0, "small", B, H, L, 64, scale, causal, window, lens)
+    inp = make_inputs(w, seed=7 + L + B + window)
+    d = inputs_f64(inp, False)
+    km = _mask_np(inp)
+    O, tau, dev = _gpu_fwd(inp, w)
+    O_ref, tau_ref = orc.attn_fwd(d["Q"], d["K"], d["V"], km, causal, window, scale)
+    Og, tg = to64(O), to64(tau)
+    finite = np.isfinite(tau_ref)
+    assert np.array_equal(np.isfinite(tg), finite)
+    assert np.max(np.abs(Og - O_ref)) <= O_TOL
+    ids = np.arange(B * H * L)
+    check_rows(d["Q"], d["K"], ids, tg.reshape(-1), tau_ref.reshape(-1), km, causal, window, scale, H, L)
+    # backward
+    dQ, dK, dV = _gpu_bwd(dev, tau, inp["dO"], w)
+    rQ, rK, rV = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], km, causal, window, scale)
+    for name, g, r in (("dQ", dQ, rQ), ("dK", dK, rK), ("dV", dV, rV)):
+        err = np.max(np.abs(to64(g) - r))
+        assert err <= GRAD_TOL, (name, err)
+
+
+def test_fp32_inputs_bf16_output_workload1():
+    """Workload 1: fp32 inputs rounded to bf16 at the boundary; bf16 output."""
+    w = WORKLOADS[1]
+    inp = make_inputs(w)
+    d = inputs_f64(inp, True)
+    O, tau, _ = _gpu_fwd(inp, w, out_dtype=torch.bfloat16)
+    O_ref, tau_ref = orc.attn_fwd(d["Q"], d["K"], d["V"], None, False, 0, w.scale)
+    tol = O_TOL + np.abs(O_ref) * 2.0 ** -9
+    assert np.all(np.abs(to64(O) - O_ref) <= tol)
+    assert np.max(np.abs(to64(tau) - tau_ref)) <= 1e-3
+    # and the fp32-input backward path
+    w2 = w.with_shape()
+    Q, K, V = (inp[k].to(DEV) for k in ("Q", "K", "V"))
+    dQ, dK, dV = entmax_attn_bwd(Q, K, V, tau, inp["dO"].to(DEV), None, False, 0, w.scale)
+    assert entmax_attn_device_status() == 0
+    rQ, rK, rV = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], None, False, 0, w2.scale)
+    for g, r in ((dQ, rQ), (dK, rK), (dV, rV)):
+        assert np.max(np.abs(to64(g) - r)) <= GRAD_TOL
+
+
+def _sample_rows(w: Workload, inp, rng, n=192):
+    L, BH = w.L, w.B * w.H
+    ids = set(rng.integers(0, BH * L, size=n).tolist())
+    for bh in (0, BH - 1):
+        for i in (0, 1, L // 2, L - 1):
+            ids.add(bh * L + i)
+    if inp["lengths"] is not None:
+        b = int(torch.argmin(inp["lengths"]))
+        for i in (0, L - 1):
+            ids.add((b * w.H) * L + i)
+    return np.array(sorted(ids), dtype=np.int64)
+
+
+@pytest.mark.parametrize("wid", [2, 3, 4, 5])
+def test_full_size_workloads(wid):
+    """Full-size workloads in the bench launch configuration (bf16 in/out, as timed)."""
+    w = WORKLOADS[wid]
+    inp = make_inputs(w)
+    d = inputs_f64(inp, False)
+    km = _mask_np(inp)
+    O, tau, dev = _gpu_fwd(inp, w, out_dtype=torch.bfloat16)
+    rng = np.random.default_rng(wid)
+    ids = _sample_rows(w, inp, rng)
+    O_ref, tau_ref = orc.attn_fwd_rows(d["Q"], d["K"], d["V"], ids, km, w.causal, w.window, w.scale)
+    Og = to64(O).reshape(-1, w.D)[ids]
+    tol = O_TOL + np.abs(O_ref) * 2.0 ** -9
+    assert np.all(np.abs(Og - O_ref) <= tol), np.max(np.abs(Og - O_ref))
+    check_rows(d["Q"], d["K"], ids, to64(tau).reshape(-1)[ids], tau_ref, km, w.causal, w.window, w.scale, w.H, w.L)
+    # every row: finite tau (no row is empty in these workloads), O finite
+    assert torch.isfinite(tau).all() and torch.isfinite(O.float()).all()
+    if not w.backward:
+        return
+    dQ, dK, dV = _gpu_bwd(dev, tau, inp["dO"], w)
+    heads = [0, w.B * w.H - 1] if wid != 4 else [5]
+    rQ, rK, rV = orc.attn_bwd_heads(d["Q"], d["K"], d["V"], d["dO"], heads, km, w.causal, w.window, w.scale)
+    for name, g, r in (("dQ", dQ, rQ), ("dK", dK, rK), ("dV", dV, rV)):
+        gh = to64(g).reshape(w.B * w.H, w.L, w.D)[heads]
+        err = np.max(np.abs(gh - r))
+        assert err <= GRAD_TOL, (name, err)
+    for g in (dQ, dK, dV):
+        assert torch.isfinite(g).all()
+
+
+def test_empty_rows_and_masked_batches():
+    """A batch whose keys are all padding: O = 0, tau = +inf, zero gradients."""
+    w = Workload(0, "empty", 2, 2, 200, 64, 1 / 8, len_range=(50, 50))
+    inp = make_inputs(w, seed=3)
+    inp["key_mask"][1] = 0
+    O, tau, dev = _gpu_fwd(inp, w)
+    assert torch.all(O[1] == 0) and torch.all(torch.isinf(tau[1]))
+    dQ, dK, dV = _gpu_bwd(dev, tau, inp["dO"], w)
+    assert torch.all(dQ[1] == 0) and torch.all(dK[1] == 0) and torch.all(dV[1] == 0)
+    d = inputs_f64(inp, False)
+    rQ, rK, rV = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], inp["key_mask"].numpy(), False, 0, w.scale)
+    assert np.max(np.abs(to64(dK) - rK)) <= GRAD_TOL
+
+
+@pytest.mark.parametrize("L", [100, 300, 1000])
+def test_uniform_rows_take_the_exact_redo_path(L):
+    """Q = 0 makes every allowed score equal: the support is the whole row, larger than the
+    candidate capacity once L > 128, so the rows are redone exactly on CUDA cores.  O is the
+    plain mean of V and tau = -2/sqrt(n)."""
+    w = Workload(0, "uniform", 1, 2, L, 64, 1 / 8)
+    inp = make_inputs(w, seed=11)
+    inp["Q"].zero_()
+    O, tau, dev = _gpu_fwd(inp, w)
+    V = to64(inp["V"])
+    np.testing.assert_allclose(to64(O), np.broadcast_to(V.mean(axis=2, keepdims=True), V.shape), atol=1e-4)
+    np.testing.assert_allclose(to64(tau), -2 / math.sqrt(L), atol=1e-6)
+    dQ, dK, dV = _gpu_bwd(dev, tau, inp["dO"], w)
+    d = inputs_f64(inp, False)
+    rQ, rK, rV = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], None, False, 0, w.scale)
+    for g, r in ((dQ, rQ), (dK, rK), (dV, rV)):
+        assert np.max(np.abs(to64(g) - r)) <= GRAD_TOL
+
+
+def test_one_hot_rows():
+    """A key aligned with every query and far above the rest takes all the weight."""
+    w = Workload(0, "onehot", 1, 1, 256, 64, 1.0)
+    inp = make_inputs(w, seed=5)
+    inp["Q"] = torch.zeros_like(inp["Q"])
+    inp["K"] = torch.zeros_like(inp["K"])
+    inp["Q"][..., 0] = 1.0
+    inp["K"][0, 0, 77, 0] = 8.0
+    O, tau, _ = _gpu_fwd(inp, w)
+    V = to64(inp["V"])
+    np.testing.assert_allclose(to64(O)[0, 0], np.broadcast_to(V[0, 0, 77], (256, 64)), atol=1e-6)
+    np.testing.assert_allclose(to64(tau), 6.0, atol=1e-6)
+
+
+def test_repeat_calls_are_deterministic():
+    w = WORKLOADS[3].with_shape(B=2)
+    inp = make_inputs(w)
+    O1, t1, dev = _gpu_fwd(inp, w)
+    O2, t2, _ = _gpu_fwd(inp, w)
+    assert torch.equal(O1, O2) and torch.equal(t1, t2)
+    g1 = _gpu_bwd(dev, t1, inp["dO"], w)
+    g2 = _gpu_bwd(dev, t1, inp["dO"], w)
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
