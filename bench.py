@@ -1,0 +1,466 @@
+#!/usr/bin/env python3
+"""Benchmark of 1.5-entmax attention forward+backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload {2,3,4,5}] [--impl {b200,reference}]
+
+One step = entmax_attn_fwd + entmax_attn_bwd (all kernels of the hot path) over one batch of
+synthetic inputs resident in HBM.  Prints ONE JSON line (rank 0).
+
+Metric: dense-equivalent TFLOP/s = 14 * d * P / t_step (fwd+bwd; 4 * d * P for forward-only
+workloads), where P counts the (query, key) pairs the masks allow -- entmax zeros are never
+subtracted.  ms_per_step is reported beside it.  Default workload: 4 (B=4, H=12, L=4096, d=64,
+scale 2/8, no mask), the tensor-bound fwd+bwd configuration.
+
+Multi-GPU: the operation does not shard (every (b, h) is independent and the workloads fit one
+GPU), so --gpus N runs N independent replicas, one per rank, with no data-path collective;
+value = total work of all ranks / max step time over ranks ("scaling": "weak").
+
+--impl reference times the fp64 CPU oracle on the host cores (bounded sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+if str(ROOT) not in sys.path:
+    sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+from entmax_tcgen05_tma_b200.workloads import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+METRIC = "1.5-entmax attn fwd+bwd ms & dense-equiv TFLOP/s vs bf16 peak, 1 B200"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def allowed_pairs(w: Workload, key_mask) -> int:
+    """(query, key) pairs allowed by key padding, causal and window, over all (b, h)."""
+    L = w.L
+    i = torch.arange(L).unsqueeze(1)
+    j = torch.arange(L).unsqueeze(0)
+    band = torch.ones(L, L, dtype=torch.bool)
+    if w.causal:
+        band &= j <= i
+    if w.window > 0:
+        band &= j >= i - w.window + 1
+    if key_mask is None:
+        per_b = torch.full((w.B,), int(band.sum()), dtype=torch.int64)
+    else:
+        per_b = (band.unsqueeze(0) & key_mask.bool().unsqueeze(1)).sum(dim=(1, 2))
+    return int(per_b.sum()) * w.H
+
+
+def dense_equiv_flops(w: Workload, pairs: int) -> float:
+    return (14.0 if w.backward else 4.0) * w.D * pairs
+
+
+def workload_desc(w: Workload) -> str:
+    s = "%s: B=%d H=%d L=%d d=%d scale=%g" % (w.name, w.B, w.H, w.L, w.D, w.scale)
+    if w.len_range:
+        s += " key-padding len U[%d,%d]" % w.len_range
+    if w.causal:
+        s += " causal"
+    if w.window:
+        s += " window=%d" % w.window
+    return s
+
+
+def load_peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            for line in Path(self.path).read_text().splitlines():
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        finally:
+            if self.path:
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        smax = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: int = 64) -> dict:
+    """Time the fp64 oracle (as it stands) on whole heads of the workload until ~budget_s."""
+    from oracle import oracle as orc
+
+    f64 = {k: inp[k].to(torch.float64).numpy() for k in ("Q", "K", "V", "dO")}
+    km = None if inp["key_mask"] is None else inp["key_mask"].numpy()
+    pairs_per_head = []
+    full_pairs = allowed_pairs(w, inp["key_mask"])
+    BH = w.B * w.H
+    heads = 0
+    t0 = time.perf_counter()
+    while heads < min(max_heads, BH) and time.perf_counter() - t0 < budget_s:
+        bh = (heads * 7919) % BH
+        b = bh // w.H
+        L = w.L
+        rows = bh * L + torch.arange(L).numpy()
+        orc.attn_fwd_rows(f64["Q"], f64["K"], f64["V"], rows, km, w.causal, w.window, w.scale)
+        if w.backward:
+            orc.attn_bwd_heads(f64["Q"], f64["K"], f64["V"], f64["dO"], [bh], km, w.causal, w.window, w.scale)
+        sub = w.with_shape(B=1)
+        pairs_per_head.append(allowed_pairs(sub.with_shape(H=1), None if km is None else inp["key_mask"][b:b + 1]))
+        heads += 1
+    dt = time.perf_counter() - t0
+    flops = dense_equiv_flops(w, sum(pairs_per_head))
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": "%d of %d heads (fwd%s) of the workload, %.1f s" % (heads, BH, "+bwd" if w.backward else "", dt),
+            "seconds": dt, "heads": heads, "full_job_seconds_est": dt * full_pairs / max(1, sum(pairs_per_head))}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def measured_sparsity(w: Workload, Q, K, tau, km) -> float:
+    """Fraction of allowed pairs with A = 0 (scores recomputed in fp32 with torch, outside the timed
+    region; only for reporting)."""
+    zeros = 0
+    allowed = 0
+    L = w.L
+    i = torch.arange(L, device=Q.device).unsqueeze(1)
+    j = torch.arange(L, device=Q.device).unsqueeze(0)
+    band = torch.ones(L, L, dtype=torch.bool, device=Q.device)
+    if w.causal:
+        band &= j <= i
+    if w.window:
+        band &= j >= i - w.window + 1
+    for b in range(w.B):
+        a = band if km is None else band & km[b].bool().unsqueeze(0)
+        for h in range(w.H):
+            S = w.scale * (Q[b, h].float() @ K[b, h].float().T)
+            supp = (S > tau[b, h].unsqueeze(1)) & a
+            allowed += int(a.sum())
+            zeros += int(a.sum()) - int(supp.sum())
+    return zeros / max(1, allowed)
+
+
+def run_gpu(args, rank: int, world: int) -> dict | None:
+    import entmax_tcgen05_tma_b200 as E
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = make_inputs(w)
+    pairs = allowed_pairs(w, inp["key_mask"])
+    flops = dense_equiv_flops(w, pairs)
+    Q, K, V, dO = (inp[k].to(dev) for k in ("Q", "K", "V", "dO"))
+    km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
+    B, H, L, D = w.B, w.H, w.L, w.D
+    O = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
+    tau = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    dQ, dK, dV = (torch.empty((B, H, L, D), dtype=torch.float32, device=dev) for _ in range(3))
+    ws = torch.empty((E.entmax_attn_bwd_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 1 + (2 if w.backward else 0)
+
+    def step():
+        E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+        if w.backward:
+            E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    st = E.entmax_attn_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after warm-up" % st)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        wall0 = time.perf_counter()
+        for k in range(args.steps):
+            flush.fill_(float(k))  # evict L2 between steps (outside the timed events)
+            ev[k][0].record(stream)
+            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+            ev[k][1].record(stream)
+            if w.backward:
+                E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV,
+                                  workspace=ws)
+            ev[k][2].record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    dist_barrier(world)
+    clocks = clk.summary()
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    total_ms = sum(step_ms)
+    total_ms = dist_max(total_ms, world, dev)
+    st = E.entmax_attn_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after the timed steps" % st)
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    host_in = {k: inp[k].pin_memory() for k in ("Q", "K", "V", "dO")}
+    host_km = None if inp["key_mask"] is None else inp["key_mask"].pin_memory()
+    host_out = {"O": torch.empty(O.shape, dtype=O.dtype).pin_memory(),
+                "tau": torch.empty(tau.shape, dtype=tau.dtype).pin_memory()}
+    if w.backward:
+        for name in ("dQ", "dK", "dV"):
+            host_out[name] = torch.empty((B, H, L, D), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + (
+        0 if host_km is None else host_km.numel())
+    if not w.backward:
+        h2d -= host_in["dO"].numel() * host_in["dO"].element_size()
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    e2e_steps = max(3, min(args.steps, 20))
+    dQe, dKe, dVe = dQ, dK, dV
+
+    def e2e_step():
+        Qd = host_in["Q"].to(dev, non_blocking=True)
+        Kd = host_in["K"].to(dev, non_blocking=True)
+        Vd = host_in["V"].to(dev, non_blocking=True)
+        kmd = None if host_km is None else host_km.to(dev, non_blocking=True)
+        Oo, to = E.entmax_attn_fwd(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale)
+        host_out["O"].copy_(Oo, non_blocking=True)
+        host_out["tau"].copy_(to, non_blocking=True)
+        if w.backward:
+            dOd = host_in["dO"].to(dev, non_blocking=True)
+            g = E.entmax_attn_bwd(Qd, Kd, Vd, to, dOd, kmd, w.causal, w.window, w.scale, dQ=dQe, dK=dKe, dV=dVe,
+                                  workspace=ws)
+            for name, t in zip(("dQ", "dK", "dV"), g):
+                host_out[name].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = dist_max(e0.elapsed_time(e1), world, dev) / e2e_steps
+    if E.entmax_attn_device_status() != 0:
+        raise RuntimeError("device status after the end-to-end steps")
+
+    if rank != 0:
+        return None
+
+    # ---- dominant kernel roofline (forward kernel: one launch per entmax_attn_fwd call)
+    peaks = load_peaks()
+    sparsity = measured_sparsity(w, Q, K, tau, km)
+    supp_pairs = (1.0 - sparsity) * pairs
+    fwd_alg_flops = 2.0 * D * pairs + 2.0 * D * supp_pairs
+    fwd_mean = statistics.mean(fwd_ms)
+    bwd_mean = statistics.mean(bwd_ms) if w.backward else 0.0
+    ms_per_step = total_ms / args.steps
+    roof = {
+        "kernel": "entmax_fwd_kernel",
+        "bound": "tensor",
+        "achieved": fwd_alg_flops / (fwd_mean * 1e-3) / 1e12,
+        "peak": peaks["bf16_tflops_sustained"],
+        "unit": "TFLOP/s",
+        "traffic": None,
+        "peak_source": "%s bf16 sustained (MEASURED_PEAKS.json)" % peaks["source"],
+        "algorithmic_flops_per_launch": fwd_alg_flops,
+    }
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = ROOT / "profiles" / ("traffic_workload%d.json" % w.wid)
+    if tr.exists():
+        t = json.loads(tr.read_text())
+        if t.get("kernel") == "entmax_fwd_kernel" and t.get("source_hash") == source_hash():
+            roof["traffic"] = t["bytes_per_launch"]
+
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded i.i.d. N(0,1), bf16; stands in for GLUE SST-2 batches)",
+        "config": {
+            "workload": workload_desc(w),
+            "workload_id": w.wid,
+            "allowed_pairs": pairs,
+            "dense_equiv_gflop_per_step": flops / 1e9,
+            "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+        },
+        "fwd_ms": round(fwd_mean, 4),
+        "bwd_ms": round(bwd_mean, 4),
+        "step_ms_median": round(statistics.median(step_ms), 4),
+        "wall_ms_per_step_incl_flush": round(wall * 1e3 / args.steps, 4),
+        "sparsity": round(sparsity, 4),
+        "roofline": roof,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cb = oracle_baseline(w, inp, budget_s=args.cpu_seconds)
+        out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    return out
+
+
+def source_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for p in sorted((ROOT / "entmax_tcgen05_tma_b200" / "csrc").glob("*")):
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def run_reference(args) -> dict:
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    per = []
+    cb = None
+    for k in range(args.warmup + args.steps):
+        cb = oracle_baseline(w, inp, budget_s=args.ref_step_seconds, max_heads=1 if k < args.warmup else 64)
+        if k >= args.warmup:
+            per.append(cb)
+    secs = sum(c["seconds"] for c in per)
+    value = sum(c["value"] * c["seconds"] for c in per) / secs
+    pairs = allowed_pairs(w, inp["key_mask"])
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": 0,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * dense_equiv_flops(w, pairs) / (value * 1e12), 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded i.i.d. N(0,1), bf16-rounded)",
+        "config": {"workload": workload_desc(w), "workload_id": w.wid,
+                   "note": "each step times the fp64 CPU oracle on a bounded sample of whole heads; "
+                           "ms_per_step extrapolates to the full workload"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
+                         "sample": "%d steps, each %s" % (args.steps, per[-1]["sample"])},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- dist helpers
+def dist_barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def dist_max(x: float, world: int, dev) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out = run_gpu(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -24,18 +24,21 @@
 namespace entmax {
 namespace {
 
-constexpr int CAP = 128;
+constexpr int CAP = 128;              // support entries per row (or key), split between the warpgroups
+constexpr int CAPW = CAP / NUM_EPI_WG;
 
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + TILE_BYTES;
 constexpr int OFF_CV = OFF_B + NSTAGE * BLK_BYTES;     // float [CAP][TILE]: sp
 constexpr int OFF_CJ = OFF_CV + CAP * TILE * 4;        // u16   [CAP][TILE]: partner index
-constexpr int OFF_BITS = OFF_CJ + CAP * TILE * 2;      // u32   [MASK_WORDS]
+constexpr int OFF_STAGE = OFF_CJ + CAP * TILE * 2;     // float [NUM_EPI][32]
+constexpr int OFF_BITS = OFF_STAGE + STAGE_FLOATS * 4; // u32   [MASK_WORDS]
 constexpr int OFF_BLK = OFF_BITS + MASK_WORDS * 4;     // u16   [MAX_BLOCKS]
-constexpr int OFF_CNT = OFF_BLK + MAX_BLOCKS * 2;      // int   [TILE]: entries (-1: redo)
-constexpr int OFF_TBUF = OFF_CNT + TILE * 4;           // float [2][TILE]: column thresholds
-constexpr int OFF_RED = OFF_TBUF + 2 * TILE * 4;       // float [256]
-constexpr int OFF_CTL = OFF_RED + 256 * 4;
+constexpr int OFF_CNT = OFF_BLK + MAX_BLOCKS * 2;      // int   [NUM_EPI_WG][TILE]: entries (-1: redo)
+constexpr int OFF_TBUF = OFF_CNT + NUM_EPI_WG * TILE * 4;  // float [NBUF][TILE]: column thresholds
+constexpr int OFF_RED = OFF_TBUF + NBUF * TILE * 4;    // float [NUM_THREADS]
+constexpr int OFF_FLAGS = OFF_RED + NUM_THREADS * 4;   // u32   [TILE/32] rows (keys) redone on CUDA cores
+constexpr int OFF_CTL = OFF_FLAGS + 16;
 constexpr int SMEM_USED = OFF_CTL + (int)sizeof(PipeCtl);
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 constexpr int OFF_SCRATCH = 0;                          // reused after the S pass
@@ -43,10 +46,9 @@ constexpr int SCRATCH_FLOATS = OFF_CV / 4;
 static_assert(CAP * TILE <= SCRATCH_FLOATS, "dA scratch must fit the S-pass buffers");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
-constexpr int EPI_BARRIER = 1;  // named barrier among the 4 epilogue warps
-
-__device__ __forceinline__ void epi_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(EPI_BARRIER), "n"(128) : "memory");
+// Named barrier among the 4 warps of epilogue warpgroup g (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void wg_sync(int g) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(128) : "memory");
 }
 
 struct ListState {
@@ -54,14 +56,18 @@ struct ListState {
     int ovf;
 };
 
-__device__ __forceinline__ void push_entry(ListState& st, float sp, int idx, float* cv, uint16_t* cj, int r) {
-    if (st.n == CAP) {
+// Lists support entry (partner idx, sp) and prefetches into L2 the two rows its gather will read.
+__device__ __forceinline__ void push_entry(ListState& st, float sp, int idx, float* cv, uint16_t* cj, int r,
+                                           const __nv_bfloat16* X1, const __nv_bfloat16* X2) {
+    if (st.n == CAPW) {
         st.ovf = 1;
         return;
     }
     cv[st.n * TILE + r] = sp;
     cj[st.n * TILE + r] = (uint16_t)idx;
     ++st.n;
+    prefetch_l2(X1 + (size_t)idx * HEAD_DIM);
+    prefetch_l2(X2 + (size_t)idx * HEAD_DIM);
 }
 
 __device__ __forceinline__ float block_sum(float a, float* red) {
@@ -72,7 +78,7 @@ __device__ __forceinline__ float block_sum(float a, float* red) {
     __syncthreads();
     float s = 0.f;
 #pragma unroll
-    for (int w = 0; w < NUM_THREADS / 32; ++w) s += red[w];
+    for (int w = 0; w < NUM_WARPS; ++w) s += red[w];
     return s;
 }
 
@@ -140,9 +146,10 @@ __device__ __noinline__ void rows_fallback(const AttnArgs& a, const BwdIO& io, c
         if (sp > 0.f) sbuf[e] = sp * (dot64_f32_bf16(gf, V + head + (size_t)(lo + e) * HEAD_DIM) - u);
     }
     __syncthreads();
-    const int d = tid & (HEAD_DIM - 1), ph = tid >> 6;
+    constexpr int PH = NUM_THREADS / HEAD_DIM;
+    const int d = tid % HEAD_DIM, ph = tid / HEAD_DIM;
     float acc = 0.f;
-    for (int e = ph; e < span; e += NUM_THREADS / HEAD_DIM) {
+    for (int e = ph; e < span; e += PH) {
         const float ds = sbuf[e];
         if (ds != 0.f) acc = fmaf(ds, __bfloat162float(K[head + (size_t)(lo + e) * HEAD_DIM + d]), acc);
     }
@@ -150,7 +157,10 @@ __device__ __noinline__ void rows_fallback(const AttnArgs& a, const BwdIO& io, c
     red[tid] = acc;
     __syncthreads();
     if (tid < HEAD_DIM) {
-        io.dQ[head + (size_t)i * HEAD_DIM + tid] = a.scale * (red[tid] + red[tid + 64] + red[tid + 128] + red[tid + 192]);
+        float q = 0.f;
+#pragma unroll
+        for (int p = 0; p < PH; ++p) q += red[tid + p * HEAD_DIM];
+        io.dQ[head + (size_t)i * HEAD_DIM + tid] = a.scale * q;
         if (tid == 0) io.u[(size_t)bh * L + i] = u;
     }
     __syncthreads();
@@ -174,7 +184,8 @@ __device__ __noinline__ void keys_fallback(const AttnArgs& a, const BwdIO& io, f
     __syncthreads();
     int qlo, qhi;
     col_query_range(j, L, a.causal, a.window, qlo, qhi);
-    const int d = tid & (HEAD_DIM - 1), ph = tid >> 6;
+    constexpr int PH = NUM_THREADS / HEAD_DIM;
+    const int d = tid % HEAD_DIM, ph = tid / HEAD_DIM;
     float accK = 0.f, accV = 0.f;
     constexpr int CHUNK = SCRATCH_FLOATS / 2;
     float* pbuf = sbuf;           // p_ij
@@ -191,7 +202,7 @@ __device__ __noinline__ void keys_fallback(const AttnArgs& a, const BwdIO& io, f
             dsbuf[e] = ds;
         }
         __syncthreads();
-        for (int e = ph; e < cn; e += NUM_THREADS / HEAD_DIM) {
+        for (int e = ph; e < cn; e += PH) {
             const float p = pbuf[e];
             if (p > 0.f) {
                 const size_t row = head + (size_t)(c0 + e) * HEAD_DIM + d;
@@ -204,13 +215,19 @@ __device__ __noinline__ void keys_fallback(const AttnArgs& a, const BwdIO& io, f
     red[tid] = accK;
     __syncthreads();
     float k_out = 0.f;
-    if (tid < HEAD_DIM) k_out = red[tid] + red[tid + 64] + red[tid + 128] + red[tid + 192];
+    if (tid < HEAD_DIM) {
+#pragma unroll
+        for (int p = 0; p < PH; ++p) k_out += red[tid + p * HEAD_DIM];
+    }
     __syncthreads();
     red[tid] = accV;
     __syncthreads();
     if (tid < HEAD_DIM) {
+        float v_out = 0.f;
+#pragma unroll
+        for (int p = 0; p < PH; ++p) v_out += red[tid + p * HEAD_DIM];
         io.dK[head + (size_t)j * HEAD_DIM + tid] = a.scale * k_out;
-        io.dV[head + (size_t)j * HEAD_DIM + tid] = red[tid] + red[tid + 64] + red[tid + 128] + red[tid + 192];
+        io.dV[head + (size_t)j * HEAD_DIM + tid] = v_out;
     }
     __syncthreads();
 }
@@ -220,11 +237,13 @@ struct Smem {
     uint8_t* b;
     float* cv;
     uint16_t* cj;
+    float* stage;
     uint32_t* bits;
     uint16_t* blk;
     int* cnt;
     float* tbuf;
     float* red;
+    uint32_t* redo;
     float* scratch;
     PipeCtl* ctl;
 };
@@ -236,11 +255,13 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     m.b = s + OFF_B;
     m.cv = reinterpret_cast<float*>(s + OFF_CV);
     m.cj = reinterpret_cast<uint16_t*>(s + OFF_CJ);
+    m.stage = reinterpret_cast<float*>(s + OFF_STAGE);
     m.bits = reinterpret_cast<uint32_t*>(s + OFF_BITS);
     m.blk = reinterpret_cast<uint16_t*>(s + OFF_BLK);
     m.cnt = reinterpret_cast<int*>(s + OFF_CNT);
     m.tbuf = reinterpret_cast<float*>(s + OFF_TBUF);
     m.red = reinterpret_cast<float*>(s + OFF_RED);
+    m.redo = reinterpret_cast<uint32_t*>(s + OFF_FLAGS);
     m.scratch = reinterpret_cast<float*>(s + OFF_SCRATCH);
     m.ctl = reinterpret_cast<PipeCtl*>(s + OFF_CTL);
     return m;
@@ -253,7 +274,8 @@ __device__ __forceinline__ void setup_cta(const Smem& sm, const CUtensorMap* ma,
         prefetch_tmap(ma);
         prefetch_tmap(mb);
     }
-    if (warp == 4) {
+    if (tid < TILE / 32) sm.redo[tid] = 0u;
+    if (warp == WARP_PRODUCER) {
         tmem_alloc(smem_u32(&sm.ctl->tmem_base), TMEM_COLS);
         tmem_relinquish();
     }
@@ -262,7 +284,7 @@ __device__ __forceinline__ void setup_cta(const Smem& sm, const CUtensorMap* ma,
 __device__ __forceinline__ void finish_cta(const Smem& sm) {
     tc_fence_before();
     __syncthreads();
-    if ((threadIdx.x >> 5) == 4) {
+    if ((threadIdx.x >> 5) == WARP_PRODUCER) {
         tc_fence_after();
         tmem_dealloc(sm.ctl->tmem_base, TMEM_COLS);
     }
@@ -283,64 +305,59 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
     setup_cta(sm, &map_q, &map_k);
     build_key_bitmap(sm.bits, a.key_mask, b, L);
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {
         const int i_last = min(i0 + TILE - 1, L - 1);
-        int klo = 0, khi = L - 1;
-        if (a.window > 0) klo = max(0, i0 - a.window + 1);
-        if (a.causal) khi = i_last;
-        int nb = 0;
-        for (int kb = klo / BLK; kb <= khi / BLK; ++kb) {
-            bool any = false;
-            for (int w = kb * (BLK / 32); w < (kb + 1) * (BLK / 32) && w * 32 <= khi; ++w)
-                any |= (sm.bits[w] & range_bits(w * 32, klo, khi)) != 0u;
-            if (any) sm.blk[nb++] = (uint16_t)kb;
-        }
-        ctl->nblk = nb;
+        const int klo = a.window > 0 ? max(0, i0 - a.window + 1) : 0;
+        const int khi = a.causal ? i_last : L - 1;
+        const int nb = build_block_list(sm.blk, sm.bits, klo, khi, i0, i_last, a.causal, a.window);
+        if (lane == 0) ctl->nblk = nb;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
     const float scale = a.scale;
+    const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue row and warpgroup
     ListState st{0, 0};
-    if (warp == 4) {
+    if (warp == WARP_PRODUCER) {
         if (lane == 0) role_producer(ctl, wc, &map_q, &map_k, bh, i0, sm.blk, sm.a, sm.b);
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == WARP_MMA) {
         if (lane == 0) role_mma(ctl, wc, sm.a, sm.b);
         __syncwarp();
-    } else if (warp < 4) {
-        const int r = tid, i = i0 + r;
+    } else {
+        const int i = i0 + r;
         int rlo, rhi;
         row_key_range(i, L, a.causal, a.window, rlo, rhi);
         const float tau = i < L ? io.tau[(size_t)bh * L + i] : INFINITY;
-        const float t = tau / scale;  // raw-score threshold
+        const float t = tau / scale;  // raw-score threshold: support iff raw score > t
         const float half_scale = 0.5f * scale;
-        const uint32_t lane_base = ctl->tmem_base + ((uint32_t)(warp * 32) << 16);
+        const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(a.V) + (size_t)bh * L * HEAD_DIM;
+        const __nv_bfloat16* Kh = reinterpret_cast<const __nv_bfloat16*>(a.K) + (size_t)bh * L * HEAD_DIM;
+        float* pcv = sm.cv + g * CAPW * TILE;
+        uint16_t* pcj = sm.cj + g * CAPW * TILE;
         const int nblk = ctl->nblk;
-        for (int n = 0; n < nblk; ++n) {
+        for (int n = g; n < nblk; n += NUM_EPI_WG) {
             if (!epi_wait_scores(ctl, wc, n)) break;
-            const int j0 = (int)sm.blk[n] * BLK;
-#pragma unroll 1
-            for (int c = 0; c < BLK / 32; ++c) {
-                float v[32];
-                tmem_ld32(lane_base + (uint32_t)((n & 1) * BLK + c * 32), v);
-                tmem_wait_ld();
-                if (c == BLK / 32 - 1) epi_release_scores(ctl, n);
+            const int j0 = (int)(sm.blk[n] & ~FULL_BLOCK) * BLK;
+            const bool full = (sm.blk[n] & FULL_BLOCK) && i < L;
+            for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
                 const int jc = j0 + c * 32;
-                const uint32_t vm = (jc < L && i < L) ? (sm.bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
-                if (vm == 0xffffffffu) {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (v[k] > t) push_entry(st, half_scale * (v[k] - t), jc + k, sm.cv, sm.cj, r);
-                } else if (vm != 0u) {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (((vm >> k) & 1u) && v[k] > t) push_entry(st, half_scale * (v[k] - t), jc + k, sm.cv, sm.cj, r);
+                const uint32_t vm = full ? 0xffffffffu
+                                         : (jc < L && i < L) ? (sm.bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
+                uint32_t hits = hit_bits(cur, t) & __brev(vm);
+                if (hits) {
+                    stage_chunk(sm.stage, cur);
+                    do {
+                        const int k = __clz(hits);
+                        hits &= ~(0x80000000u >> k);
+                        push_entry(st, half_scale * (staged(sm.stage, k) - t), jc + k, pcv, pcj, r, Vh, Kh);
+                    } while (hits);
                 }
-            }
+            });
         }
-        sm.cnt[r] = st.ovf ? -1 : st.n;
+        sm.cnt[g * TILE + r] = st.ovf ? 0 : st.n;
+        if (st.ovf) atomicOr(&sm.redo[r >> 5], 1u << (r & 31));
     }
     tc_fence_before();
     __syncthreads();
@@ -352,53 +369,57 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
         const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(a.V);
         const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
         const size_t head = (size_t)bh * L * HEAD_DIM;
-        float* dAbuf = sm.scratch;  // [CAP][TILE]
-        for (int r = warp; r < TILE; r += NUM_THREADS / 32) {
-            const int i = i0 + r;
-            const int k = sm.cnt[r];
-            if (i >= L || k < 0) continue;
+        float* dAbuf = sm.scratch;  // [CAP][TILE], same slots as the entry lists
+        for (int rr = warp; rr < TILE; rr += NUM_WARPS) {
+            const int i = i0 + rr;
+            const int k0 = sm.cnt[rr], k1 = sm.cnt[TILE + rr];
+            if (i >= L || ((sm.redo[rr >> 5] >> (rr & 31)) & 1u)) continue;
             const uint32_t gw = reinterpret_cast<const uint32_t*>(dO + head + (size_t)i * HEAD_DIM)[lane];
             const float g0 = bf16lo(gw), g1 = bf16hi(gw);
+            // dA_e = <dO_i, V_j> for every entry, eight gathered rows in flight
             float rs = 0.f, ws = 0.f;
-            int e = 0;
-            for (; e + 2 <= k; e += 2) {
-                const int ja = sm.cj[e * TILE + r], jb = sm.cj[(e + 1) * TILE + r];
-                const uint32_t va = reinterpret_cast<const uint32_t*>(V + head + (size_t)ja * HEAD_DIM)[lane];
-                const uint32_t vb = reinterpret_cast<const uint32_t*>(V + head + (size_t)jb * HEAD_DIM)[lane];
-                float da = fmaf(g0, bf16lo(va), g1 * bf16hi(va));
-                float db = fmaf(g0, bf16lo(vb), g1 * bf16hi(vb));
+            for (int q = 0; q < NUM_EPI_WG; ++q) {
+                const int base = q * CAPW, end = base + (q == 0 ? k0 : k1);
+                for (int e = base; e < end; e += 8) {
+                    uint32_t x[8];
+                    float pd[8];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    da += __shfl_xor_sync(0xffffffffu, da, o);
-                    db += __shfl_xor_sync(0xffffffffu, db, o);
+                    for (int u8 = 0; u8 < 8; ++u8) {
+                        const bool ok = e + u8 < end;
+                        const int j = ok ? (int)sm.cj[(e + u8) * TILE + rr] : 0;
+                        x[u8] = ok ? __ldg(reinterpret_cast<const uint32_t*>(V + head + (size_t)j * HEAD_DIM) + lane) : 0u;
+                    }
+#pragma unroll
+                    for (int u8 = 0; u8 < 8; ++u8) pd[u8] = fmaf(g0, bf16lo(x[u8]), g1 * bf16hi(x[u8]));
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+                        for (int u8 = 0; u8 < 8; ++u8) pd[u8] += __shfl_xor_sync(0xffffffffu, pd[u8], o);
+                    }
+#pragma unroll
+                    for (int u8 = 0; u8 < 8; ++u8) {
+                        if (e + u8 < end) {
+                            const float sp = sm.cv[(e + u8) * TILE + rr];
+                            rs += sp;
+                            ws = fmaf(sp, pd[u8], ws);
+                            if (lane == 0) dAbuf[(e + u8) * TILE + rr] = pd[u8];
+                        }
+                    }
                 }
-                const float spa = sm.cv[e * TILE + r], spb = sm.cv[(e + 1) * TILE + r];
-                rs += spa + spb;
-                ws = fmaf(spa, da, fmaf(spb, db, ws));
-                if (lane == 0) {
-                    dAbuf[e * TILE + r] = da;
-                    dAbuf[(e + 1) * TILE + r] = db;
-                }
-            }
-            if (e < k) {
-                const int ja = sm.cj[e * TILE + r];
-                const uint32_t va = reinterpret_cast<const uint32_t*>(V + head + (size_t)ja * HEAD_DIM)[lane];
-                const float da = warp_sum(fmaf(g0, bf16lo(va), g1 * bf16hi(va)));
-                const float spa = sm.cv[e * TILE + r];
-                rs += spa;
-                ws = fmaf(spa, da, ws);
-                if (lane == 0) dAbuf[e * TILE + r] = da;
             }
             const float u = rs > 0.f ? ws / rs : 0.f;
             __syncwarp();
-            float q0 = 0.f, q1 = 0.f;
-            for (e = 0; e < k; ++e) {
-                const int j = sm.cj[e * TILE + r];
-                const float ds = sm.cv[e * TILE + r] * (dAbuf[e * TILE + r] - u);
-                const uint32_t kw = reinterpret_cast<const uint32_t*>(K + head + (size_t)j * HEAD_DIM)[lane];
-                q0 = fmaf(ds, bf16lo(kw), q0);
-                q1 = fmaf(ds, bf16hi(kw), q1);
+            // dS_e = sp_e (dA_e - u), written over dA, then dQ_i = scale sum_e dS_e K_j
+            for (int q = 0; q < NUM_EPI_WG; ++q) {
+                const int base = q * CAPW, end = base + (q == 0 ? k0 : k1);
+                for (int e = base + lane; e < end; e += 32)
+                    dAbuf[e * TILE + rr] = sm.cv[e * TILE + rr] * (dAbuf[e * TILE + rr] - u);
             }
+            __syncwarp();
+            float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
+            gather_accumulate2(K + head, sm.cj, dAbuf, rr, 0, k0, rr, CAPW, CAPW + k1, lane, q0, q1, q2, q3);
+            q0 += q2;
+            q1 += q3;
             *reinterpret_cast<float2*>(io.dQ + head + (size_t)i * HEAD_DIM + 2 * lane) =
                 make_float2(scale * q0, scale * q1);
             if (lane == 0) io.u[(size_t)bh * L + i] = u;
@@ -406,9 +427,13 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
     }
     __syncthreads();
     if (!aborted) {
-        for (int r = 0; r < TILE; ++r) {
-            if (sm.cnt[r] >= 0) continue;
-            rows_fallback(a, io, sm.bits, sm.scratch, sm.red, bh, i0 + r);
+        for (int wd = 0; wd < TILE / 32; ++wd) {
+            uint32_t mask = sm.redo[wd];  // uniform across the CTA
+            while (mask) {
+                const int rr = wd * 32 + __ffs(mask) - 1;
+                mask &= mask - 1;
+                rows_fallback(a, io, sm.bits, sm.scratch, sm.red, bh, i0 + rr);
+            }
         }
     }
     finish_cta(sm);
@@ -446,41 +471,39 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
     tc_fence_after();
 
     const float scale = a.scale;
+    const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue key and warpgroup
     ListState st{0, 0};
-    if (warp == 4) {
+    if (warp == WARP_PRODUCER) {
         if (lane == 0) role_producer(ctl, wc, &map_k, &map_q, bh, j0, sm.blk, sm.a, sm.b);
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == WARP_MMA) {
         if (lane == 0) role_mma(ctl, wc, sm.a, sm.b);
         __syncwarp();
-    } else if (warp < 4) {
-        const int r = tid, j = j0 + r;
+    } else {
+        const int j = j0 + r;
         const bool key_ok = j < L && ((sm.bits[j >> 5] >> (j & 31)) & 1u);
         int qlo, qhi;
         col_query_range(j, L, a.causal, a.window, qlo, qhi);
         const float half_scale = 0.5f * scale;
-        const uint32_t lane_base = ctl->tmem_base + ((uint32_t)(warp * 32) << 16);
+        const __nv_bfloat16* dOh = reinterpret_cast<const __nv_bfloat16*>(io.dO) + (size_t)bh * L * HEAD_DIM;
+        const __nv_bfloat16* Qh = reinterpret_cast<const __nv_bfloat16*>(a.Q) + (size_t)bh * L * HEAD_DIM;
+        float* pcv = sm.cv + g * CAPW * TILE;
+        uint16_t* pcj = sm.cj + g * CAPW * TILE;
         const int nblk = ctl->nblk;
-        bool live = true;  // every epilogue warp runs all nblk iterations: the named barrier counts match
-        for (int n = 0; n < nblk; ++n) {
+        bool live = true;  // each warpgroup runs all its iterations so its named-barrier counts match
+        for (int n = g; n < nblk; n += NUM_EPI_WG) {
             const int q0 = (int)sm.blk[n] * BLK;
-            float* tb = sm.tbuf + (n & 1) * TILE;
+            float* tb = sm.tbuf + (n % NBUF) * TILE;
             {
                 const int i = q0 + r;
                 tb[r] = i < L ? io.tau[(size_t)bh * L + i] / scale : INFINITY;
             }
-            epi_sync();
+            wg_sync(g);
             if (live) live = epi_wait_scores(ctl, wc, n);
             if (!live) continue;
-#pragma unroll 1
-            for (int c = 0; c < BLK / 32; ++c) {
-                float v[32];
-                tmem_ld32(lane_base + (uint32_t)((n & 1) * BLK + c * 32), v);
-                tmem_wait_ld();
-                if (c == BLK / 32 - 1) epi_release_scores(ctl, n);
+            for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
                 const int qc = q0 + c * 32;
                 const uint32_t vm = key_ok ? range_bits(qc, qlo, qhi) : 0u;
-                if (vm == 0u) continue;
                 float t[32];
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {
@@ -490,12 +513,19 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
                     t[4 * k4 + 2] = t4.z;
                     t[4 * k4 + 3] = t4.w;
                 }
-#pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    if (((vm >> k) & 1u) && v[k] > t[k]) push_entry(st, half_scale * (v[k] - t[k]), qc + k, sm.cv, sm.cj, r);
-            }
+                uint32_t hits = hit_bits(cur, t) & __brev(vm);
+                if (hits) {
+                    stage_chunk(sm.stage, cur);
+                    do {
+                        const int k = __clz(hits);
+                        hits &= ~(0x80000000u >> k);
+                        push_entry(st, half_scale * (staged(sm.stage, k) - tb[c * 32 + k]), qc + k, pcv, pcj, r, dOh, Qh);
+                    } while (hits);
+                }
+            });
         }
-        sm.cnt[r] = st.ovf ? -1 : st.n;
+        sm.cnt[g * TILE + r] = st.ovf ? 0 : st.n;
+        if (st.ovf) atomicOr(&sm.redo[r >> 5], 1u << (r & 31));
     }
     tc_fence_before();
     __syncthreads();
@@ -507,36 +537,59 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
         const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(a.V);
         const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
         const size_t head = (size_t)bh * L * HEAD_DIM;
-        for (int r = warp; r < TILE; r += NUM_THREADS / 32) {
-            const int j = j0 + r;
-            const int k = sm.cnt[r];
-            if (j >= L || k < 0) continue;
+        for (int rr = warp; rr < TILE; rr += NUM_WARPS) {
+            const int j = j0 + rr;
+            const int k0 = sm.cnt[rr], k1 = sm.cnt[TILE + rr];
+            if (j >= L || ((sm.redo[rr >> 5] >> (rr & 31)) & 1u)) continue;
             const uint32_t vw = reinterpret_cast<const uint32_t*>(V + head + (size_t)j * HEAD_DIM)[lane];
             const float v0 = bf16lo(vw), v1 = bf16hi(vw);
-            float k0 = 0.f, k1 = 0.f, w0 = 0.f, w1 = 0.f;
-            for (int e = 0; e < k; ++e) {
-                const int i = sm.cj[e * TILE + r];
-                const float sp = sm.cv[e * TILE + r];
-                const uint32_t gw = reinterpret_cast<const uint32_t*>(dO + head + (size_t)i * HEAD_DIM)[lane];
-                const uint32_t qw = reinterpret_cast<const uint32_t*>(Q + head + (size_t)i * HEAD_DIM)[lane];
-                const float g0 = bf16lo(gw), g1 = bf16hi(gw);
-                const float dA = warp_sum(fmaf(g0, v0, g1 * v1));
-                const float ds = sp * (dA - io.u[(size_t)bh * L + i]);
-                const float p = sp * sp;
-                w0 = fmaf(p, g0, w0);
-                w1 = fmaf(p, g1, w1);
-                k0 = fmaf(ds, bf16lo(qw), k0);
-                k1 = fmaf(ds, bf16hi(qw), k1);
+            float kk0 = 0.f, kk1 = 0.f, w0 = 0.f, w1 = 0.f;
+            const float* ub = io.u + (size_t)bh * L;
+            for (int q = 0; q < NUM_EPI_WG; ++q) {
+                const int base = q * CAPW, end = base + (q == 0 ? k0 : k1);
+                for (int e = base; e < end; e += 8) {
+                    uint32_t gw[8], qw[8];
+                    float uu[8], sp[8], pd[8];
+#pragma unroll
+                    for (int u8 = 0; u8 < 8; ++u8) {
+                        const bool ok = e + u8 < end;
+                        const int i = ok ? (int)sm.cj[(e + u8) * TILE + rr] : 0;
+                        sp[u8] = ok ? sm.cv[(e + u8) * TILE + rr] : 0.f;
+                        gw[u8] = ok ? __ldg(reinterpret_cast<const uint32_t*>(dO + head + (size_t)i * HEAD_DIM) + lane) : 0u;
+                        qw[u8] = ok ? __ldg(reinterpret_cast<const uint32_t*>(Q + head + (size_t)i * HEAD_DIM) + lane) : 0u;
+                        uu[u8] = ok ? __ldg(ub + i) : 0.f;
+                    }
+#pragma unroll
+                    for (int u8 = 0; u8 < 8; ++u8) pd[u8] = fmaf(bf16lo(gw[u8]), v0, bf16hi(gw[u8]) * v1);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+                        for (int u8 = 0; u8 < 8; ++u8) pd[u8] += __shfl_xor_sync(0xffffffffu, pd[u8], o);
+                    }
+#pragma unroll
+                    for (int u8 = 0; u8 < 8; ++u8) {
+                        const float ds = sp[u8] * (pd[u8] - uu[u8]);
+                        const float p = sp[u8] * sp[u8];
+                        w0 = fmaf(p, bf16lo(gw[u8]), w0);
+                        w1 = fmaf(p, bf16hi(gw[u8]), w1);
+                        kk0 = fmaf(ds, bf16lo(qw[u8]), kk0);
+                        kk1 = fmaf(ds, bf16hi(qw[u8]), kk1);
+                    }
+                }
             }
-            *reinterpret_cast<float2*>(io.dK + head + (size_t)j * HEAD_DIM + 2 * lane) = make_float2(scale * k0, scale * k1);
+            *reinterpret_cast<float2*>(io.dK + head + (size_t)j * HEAD_DIM + 2 * lane) = make_float2(scale * kk0, scale * kk1);
             *reinterpret_cast<float2*>(io.dV + head + (size_t)j * HEAD_DIM + 2 * lane) = make_float2(w0, w1);
         }
     }
     __syncthreads();
     if (!aborted) {
-        for (int r = 0; r < TILE; ++r) {
-            if (sm.cnt[r] >= 0) continue;
-            keys_fallback(a, io, sm.scratch, sm.red, bh, j0 + r);
+        for (int wd = 0; wd < TILE / 32; ++wd) {
+            uint32_t mask = sm.redo[wd];  // uniform across the CTA
+            while (mask) {
+                const int rr = wd * 32 + __ffs(mask) - 1;
+                mask &= mask - 1;
+                keys_fallback(a, io, sm.scratch, sm.red, bh, j0 + rr);
+            }
         }
     }
     finish_cta(sm);

@@ -3,13 +3,14 @@
 //
 // Score pipeline ("S pass"): one CTA owns a fixed 128-row tile (the A operand) and streams
 // 128-row blocks of the other operand (B).  For every streamed block the tensor core computes
-// the 128x128 fp32 tile A.B^T into one of two TMEM buffers; epilogue warps read it back with
-// tcgen05.ld (TMEM lane = row of A) while the next block's MMA runs.
+// the 128x128 fp32 tile A.B^T into one of four TMEM buffers (block n -> buffer n % 4); two
+// epilogue warpgroups read them back with tcgen05.ld (TMEM lane = row of A), warpgroup g taking
+// the blocks n = g (mod 2), while later blocks' MMAs run.
 //
-//   warp 4 (lane 0) : TMA producer  -- A tile once, B blocks through an NSTAGE ring
-//   warp 5 (lane 0) : MMA issuer    -- 4 x (M128 N128 K16) per block, commit to mbarriers
-//   warps 0-3       : epilogue      -- one thread per A row, consumes TMEM buffers
-//   warp 4          : TMEM allocation / release
+//   warps 0-3, 4-7  : epilogue warpgroups 0 and 1 -- thread (g, r) serves A row r
+//   warp 8 (lane 0) : TMA producer  -- A tile once, B blocks through an NSTAGE ring
+//   warp 9 (lane 0) : MMA issuer    -- 4 x (M128 N128 K16) per block, commit to mbarriers
+//   warp 8          : TMEM allocation / release
 //
 // Every wait is bounded: on timeout the CTA records ENTMAX_ERR_TIMEOUT in the device status
 // word, raises a CTA-local abort flag that all roles poll, waits (again bounded) for its own
@@ -24,11 +25,18 @@ namespace entmax {
 constexpr int HEAD_DIM = 64;            // d, the only head size the kernels take
 constexpr int TILE = 128;               // rows of the fixed tile == MMA M
 constexpr int BLK = 128;                // rows of a streamed block == MMA N
-constexpr int NSTAGE = 3;               // streamed-block ring depth
+constexpr int NSTAGE = 4;               // streamed-block ring depth
 constexpr int TILE_BYTES = TILE * HEAD_DIM * 2;  // 16 KiB, bf16 rows of 128 B
 constexpr int BLK_BYTES = BLK * HEAD_DIM * 2;    // 16 KiB
-constexpr int NUM_THREADS = 256;
-constexpr int TMEM_COLS = 2 * BLK;      // two fp32 score buffers
+constexpr int NUM_EPI_WG = 2;           // epilogue warpgroups
+constexpr int NUM_EPI = NUM_EPI_WG * 128;
+constexpr int NBUF = 4;                 // TMEM score buffers
+constexpr int NUM_THREADS = NUM_EPI + 64;  // + producer warp + MMA warp
+constexpr int NUM_WARPS = NUM_THREADS / 32;
+constexpr int WARP_PRODUCER = NUM_EPI / 32;
+constexpr int WARP_MMA = WARP_PRODUCER + 1;
+constexpr int TMEM_COLS = NBUF * BLK;   // four fp32 score buffers = all 512 columns
+constexpr int STAGE_FLOATS = NUM_EPI * 32;  // per-thread staging of one 32-value chunk
 constexpr int MAX_L = 16384;            // longest sequence the kernels take
 constexpr int MASK_WORDS = MAX_L / 32;
 constexpr int MAX_BLOCKS = MAX_L / BLK;
@@ -43,8 +51,8 @@ struct PipeCtl {
     uint64_t full_a;               // A tile landed
     uint64_t full_b[NSTAGE];       // B block landed
     uint64_t empty_b[NSTAGE];      // B stage consumed by the MMA
-    uint64_t s_full[2];            // score buffer written
-    uint64_t s_empty[2];           // score buffer read by the epilogue warps
+    uint64_t s_full[NBUF];         // score buffer written
+    uint64_t s_empty[NBUF];        // score buffer read by its epilogue warpgroup
     uint32_t tmem_base;
     int abort_flag;
     int nblk;                      // streamed blocks this CTA visits
@@ -126,6 +134,42 @@ __device__ __forceinline__ uint32_t range_bits(int jc, int lo, int hi) {
     return upper & ~((1u << lb) - 1u);
 }
 
+// Streamed key blocks a query tile (rows [i0, i_last]) visits: blocks kb in [klo/BLK, khi/BLK]
+// holding at least one valid key in [klo, khi].  Entry = block index | FULL_BLOCK when every key
+// of the block is valid and allowed for every row of the tile (no per-row mask work needed).
+// Built by warp 0 (one lane per candidate block, ballot + prefix count); returns the count.
+constexpr uint16_t FULL_BLOCK = 0x8000u;
+__device__ __forceinline__ int build_block_list(uint16_t* list, const uint32_t* bits, int klo, int khi, int i0,
+                                                int i_last, int causal, int window) {
+    const int lane = threadIdx.x & 31;
+    const int kb0 = klo / BLK, kb1 = khi / BLK;
+    int nb = 0;
+    for (int base = kb0; base <= kb1; base += 32) {
+        const int kb = base + lane;
+        bool any = false, full = kb <= kb1;
+        if (kb <= kb1) {
+#pragma unroll
+            for (int q = 0; q < BLK / 32; ++q) {
+                const int w = kb * (BLK / 32) + q;
+                const uint32_t word = w * 32 <= khi ? bits[w] : 0u;
+                if (w * 32 <= khi) any |= (word & range_bits(w * 32, klo, khi)) != 0u;
+                full &= word == 0xffffffffu;
+            }
+            const int j0 = kb * BLK, j1 = j0 + BLK - 1;
+            if (causal) full &= j1 <= i0;
+            if (window > 0) full &= j0 >= i_last - window + 1;
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, any);
+        if (any) list[nb + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(kb | (full ? FULL_BLOCK : 0));
+        nb += __popc(bal);
+    }
+    return nb;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ------------------------------------------------------- TMA producer role
 // Loads the fixed A tile (rows a_row0.. of head bh) and then the streamed B blocks listed in
 // blk_list (block index -> rows blk*BLK..) through the NSTAGE ring.
@@ -141,7 +185,7 @@ __device__ __forceinline__ void role_producer(PipeCtl* ctl, const WaitCfg& wc, c
         const uint32_t ph = (uint32_t)(n / NSTAGE) & 1u;
         if (!wait_bounded(smem_u32(&ctl->empty_b[s]), ph ^ 1u, ctl, wc)) break;
         mbar_arrive_expect_tx(smem_u32(&ctl->full_b[s]), BLK_BYTES);
-        tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)blk_list[n] * BLK, bh,
+        tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[n] & ~FULL_BLOCK) * BLK, bh,
                     smem_u32(&ctl->full_b[s]));
         ++issued;
     }
@@ -163,9 +207,9 @@ __device__ __forceinline__ void role_mma(PipeCtl* ctl, const WaitCfg& wc, const 
         tc_fence_after();
         const uint64_t da = umma_desc_kmajor_sw128(smem_u32(smem_a));
         for (int n = 0; n < nblk; ++n) {
-            const int s = n % NSTAGE, buf = n & 1;
+            const int s = n % NSTAGE, buf = n % NBUF;
             if (!wait_bounded(smem_u32(&ctl->full_b[s]), (uint32_t)(n / NSTAGE) & 1u, ctl, wc)) break;
-            if (!wait_bounded(smem_u32(&ctl->s_empty[buf]), ((uint32_t)(n >> 1) & 1u) ^ 1u, ctl, wc)) break;
+            if (!wait_bounded(smem_u32(&ctl->s_empty[buf]), ((uint32_t)(n / NBUF) & 1u) ^ 1u, ctl, wc)) break;
             tc_fence_after();
             const uint64_t db = umma_desc_kmajor_sw128(smem_u32(smem_b + s * BLK_BYTES));
             const uint32_t d_tmem = ctl->tmem_base + (uint32_t)(buf * BLK);
@@ -179,7 +223,7 @@ __device__ __forceinline__ void role_mma(PipeCtl* ctl, const WaitCfg& wc, const 
     }
     if (cta_aborted(ctl) && issued > 0) {
         const int n = issued - 1;  // the last commit covers every earlier MMA
-        wait_drain(smem_u32(&ctl->s_full[n & 1]), (uint32_t)(n >> 1) & 1u);
+        wait_drain(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u);
     }
 }
 
@@ -189,9 +233,9 @@ __device__ __forceinline__ void init_pipe(PipeCtl* ctl) {
         mbar_init(smem_u32(&ctl->full_b[s]), 1);
         mbar_init(smem_u32(&ctl->empty_b[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
         mbar_init(smem_u32(&ctl->s_full[b]), 1);
-        mbar_init(smem_u32(&ctl->s_empty[b]), 4);  // one arrival per epilogue warp
+        mbar_init(smem_u32(&ctl->s_empty[b]), 4);  // one arrival per warp of the owning warpgroup
     }
     ctl->abort_flag = 0;
     fence_barrier_init();
@@ -199,7 +243,7 @@ __device__ __forceinline__ void init_pipe(PipeCtl* ctl) {
 
 // Epilogue side: wait for score buffer of streamed block n; false on abort.
 __device__ __forceinline__ bool epi_wait_scores(PipeCtl* ctl, const WaitCfg& wc, int n) {
-    const bool ok = wait_bounded(smem_u32(&ctl->s_full[n & 1]), (uint32_t)(n >> 1) & 1u, ctl, wc);
+    const bool ok = wait_bounded(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u, ctl, wc);
     tc_fence_after();
     return ok;
 }
@@ -208,11 +252,132 @@ __device__ __forceinline__ bool epi_wait_scores(PipeCtl* ctl, const WaitCfg& wc,
 __device__ __forceinline__ void epi_release_scores(PipeCtl* ctl, int n) {
     tc_fence_before();
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&ctl->s_empty[n & 1]));
+    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&ctl->s_empty[n % NBUF]));
 }
+
+// TMEM address of lane quarter (warp % 4), buffer of block n, 32-column chunk c.
+__device__ __forceinline__ uint32_t epi_taddr(const PipeCtl* ctl, int n, int c) {
+    const int warp = threadIdx.x >> 5;
+    return ctl->tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((n % NBUF) * BLK + c * 32);
+}
+
+// Reads the four 32-column chunks of score block n, double-buffered in registers, and calls
+// f(v, c) for chunk c.  The buffer is released to the MMA warp once its last chunk is loaded.
+template <class F>
+__device__ __forceinline__ void for_each_chunk(PipeCtl* ctl, int n, F&& f) {
+    static_assert(BLK == 128, "four chunks per block");
+    float va[32], vb[32];
+    tmem_ld32(epi_taddr(ctl, n, 0), va);
+    tmem_wait_ld(va);
+    tmem_ld32(epi_taddr(ctl, n, 1), vb);
+    f(va, 0);
+    tmem_wait_ld(vb);
+    tmem_ld32(epi_taddr(ctl, n, 2), va);
+    f(vb, 1);
+    tmem_wait_ld(va);
+    tmem_ld32(epi_taddr(ctl, n, 3), vb);
+    f(va, 2);
+    tmem_wait_ld(vb);
+    epi_release_scores(ctl, n);
+    f(vb, 3);
+}
+
+// ------------------------------------------------------------ hit filtering
+// Bit (31 - k) of the result is set iff v[k] > t: the sign bit of t - v[k] funnel-shifted into
+// four independent 8-bit chains (two instructions per value, no branches).
+__device__ __forceinline__ uint32_t hit_bits(const float (&v)[32], float t) {
+    uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        h0 = __funnelshift_l(__float_as_uint(t - v[k]), h0, 1);
+        h1 = __funnelshift_l(__float_as_uint(t - v[8 + k]), h1, 1);
+        h2 = __funnelshift_l(__float_as_uint(t - v[16 + k]), h2, 1);
+        h3 = __funnelshift_l(__float_as_uint(t - v[24 + k]), h3, 1);
+    }
+    return (h0 << 24) | (h1 << 16) | (h2 << 8) | h3;
+}
+
+// Same with a per-value threshold t[k].
+__device__ __forceinline__ uint32_t hit_bits(const float (&v)[32], const float (&t)[32]) {
+    uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        h0 = __funnelshift_l(__float_as_uint(t[k] - v[k]), h0, 1);
+        h1 = __funnelshift_l(__float_as_uint(t[8 + k] - v[8 + k]), h1, 1);
+        h2 = __funnelshift_l(__float_as_uint(t[16 + k] - v[16 + k]), h2, 1);
+        h3 = __funnelshift_l(__float_as_uint(t[24 + k] - v[24 + k]), h3, 1);
+    }
+    return (h0 << 24) | (h1 << 16) | (h2 << 8) | h3;
+}
+
+// Per-thread staging of a 32-value chunk in shared memory (16-byte groups XOR-swizzled by the
+// thread index, so a warp's 128-bit stores are conflict-free), read back by dynamic index.
+__device__ __forceinline__ void stage_chunk(float* stage, const float (&v)[32]) {
+    float* row = stage + (threadIdx.x % NUM_EPI) * 32;
+    const int sw = threadIdx.x & 7;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(row + ((c ^ sw) << 2)) = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
+__device__ __forceinline__ float staged(const float* stage, int k) {
+    return stage[(threadIdx.x % NUM_EPI) * 32 + ((((k >> 2) ^ (threadIdx.x & 7))) << 2) + (k & 3)];
+}
+
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// acc += sum over list slots e in [e0, e1) of w[e] * X[j[e]][2 lane .. 2 lane + 1], where the
+// slot arrays are [slot][TILE] with column `col`.  Loads go out eight rows at a time so a warp
+// keeps eight independent global reads in flight.
+__device__ __forceinline__ void gather_accumulate(const __nv_bfloat16* __restrict__ X, const uint16_t* cj,
+                                                  const float* cw, int col, int e0, int e1, int lane, float& acc0,
+                                                  float& acc1) {
+    for (int e = e0; e < e1; e += 8) {
+        uint32_t x[8];
+        float w[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const bool ok = e + u < e1;
+            const int j = ok ? (int)cj[(e + u) * TILE + col] : 0;
+            w[u] = ok ? cw[(e + u) * TILE + col] : 0.f;
+            x[u] = ok ? __ldg(reinterpret_cast<const uint32_t*>(X + (size_t)j * HEAD_DIM) + lane) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            acc0 = fmaf(w[u], bf16lo(x[u]), acc0);
+            acc1 = fmaf(w[u], bf16hi(x[u]), acc1);
+        }
+    }
+}
+
+// Two lists at once (columns ca, cb), so a warp keeps sixteen gathered rows in flight.
+__device__ __forceinline__ void gather_accumulate2(const __nv_bfloat16* __restrict__ X, const uint16_t* cj,
+                                                   const float* cw, int ca, int ea0, int ea1, int cb, int eb0,
+                                                   int eb1, int lane, float& a0, float& a1, float& b0, float& b1) {
+    for (int ea = ea0, eb = eb0; ea < ea1 || eb < eb1; ea += 8, eb += 8) {
+        uint32_t xa[8], xb[8];
+        float wa[8], wb[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const bool oka = ea + u < ea1, okb = eb + u < eb1;
+            const int ja = oka ? (int)cj[(ea + u) * TILE + ca] : 0;
+            const int jb = okb ? (int)cj[(eb + u) * TILE + cb] : 0;
+            wa[u] = oka ? cw[(ea + u) * TILE + ca] : 0.f;
+            wb[u] = okb ? cw[(eb + u) * TILE + cb] : 0.f;
+            xa[u] = oka ? __ldg(reinterpret_cast<const uint32_t*>(X + (size_t)ja * HEAD_DIM) + lane) : 0u;
+            xb[u] = okb ? __ldg(reinterpret_cast<const uint32_t*>(X + (size_t)jb * HEAD_DIM) + lane) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            a0 = fmaf(wa[u], bf16lo(xa[u]), a0);
+            a1 = fmaf(wa[u], bf16hi(xa[u]), a1);
+            b0 = fmaf(wb[u], bf16lo(xb[u]), b0);
+            b1 = fmaf(wb[u], bf16hi(xb[u]), b1);
+        }
+    }
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -12,13 +12,13 @@
 //     lower bound t of tau (max - 2, tightened to the exact threshold of the row's top four
 //     scores whenever the list fills).  A score at or below any lower bound of tau is outside
 //     the support, so the support is a subset of the candidates.
-//  2. tau solve per row on the candidate list: the pages' bisection, where candidates already
-//     known to lie above the bracket are folded into running moments and those below it are
-//     dropped; once no candidate lies strictly inside the bracket the support is fixed and the
-//     root of the now-quadratic constraint is taken in closed form.  If 25 halvings leave the
-//     support undecided the final midpoint is used, as on the pages.
+//  2. tau solve per row on the candidate list: the pages' 25 halvings of the bracket
+//     [max - 2, max - 2/sqrt(n)], with g(mid) summed over the candidates (held in registers by two
+//     threads per row), then the root of sum_S (S_ij - tau)^2 = 4 in closed form on the support
+//     S = {S_ij > final midpoint}, kept if it lies in the final bracket (else the midpoint).
 //  3. O_i = sum p_ij V_j over the support (typically 5-40 keys) with one warp per row: lane l
-//     accumulates dimensions 2l, 2l+1 from V rows gathered out of L2.
+//     accumulates dimensions 2l, 2l+1 from V rows gathered out of L2 (prefetched into L2 when the
+//     candidate was listed).
 //  4. Rows whose candidates exceed the list capacity are redone exactly by the whole CTA on
 //     CUDA cores (scores into shared memory, bisection with block reductions).
 #include <cuda_bf16.h>
@@ -29,19 +29,24 @@
 namespace entmax {
 namespace {
 
-constexpr int CAP = 128;  // candidates per row
+constexpr int CAP = 128;              // candidates per row, split between the two warpgroups
+constexpr int CAPW = CAP / NUM_EPI_WG;
+constexpr int REG_CAND = 32;          // candidates per thread held in registers by the tau solve
 
 // shared-memory layout (bytes from the 1024-aligned base)
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + TILE_BYTES;
 constexpr int OFF_CV = OFF_B + NSTAGE * BLK_BYTES;     // float [CAP][TILE]
 constexpr int OFF_CJ = OFF_CV + CAP * TILE * 4;        // u16   [CAP][TILE]
-constexpr int OFF_BITS = OFF_CJ + CAP * TILE * 2;      // u32   [MASK_WORDS]
+constexpr int OFF_STAGE = OFF_CJ + CAP * TILE * 2;     // float [NUM_EPI][32]
+constexpr int OFF_BITS = OFF_STAGE + STAGE_FLOATS * 4; // u32   [MASK_WORDS]
 constexpr int OFF_BLK = OFF_BITS + MASK_WORDS * 4;     // u16   [MAX_BLOCKS]
-constexpr int OFF_SUPP = OFF_BLK + MAX_BLOCKS * 2;     // int   [TILE]  support size (or -1: redo)
-constexpr int OFF_NALLOW = OFF_SUPP + TILE * 4;        // int   [TILE]
-constexpr int OFF_RED = OFF_NALLOW + TILE * 4;         // float [256]   reductions / fallback q
-constexpr int OFF_CTL = OFF_RED + 256 * 4;
+constexpr int OFF_SUPP = OFF_BLK + MAX_BLOCKS * 2;     // int   [2][TILE] support size per partition
+constexpr int OFF_ROWS = OFF_SUPP + 2 * TILE * 4;      // RowOut[2][TILE] per-warpgroup row state
+constexpr int OFF_RED = OFF_ROWS + 2 * TILE * 32;      // float [NUM_THREADS]
+constexpr int OFF_FLAGS = OFF_RED + NUM_THREADS * 4;   // u32   [TILE/32] rows redone by the fallback
+constexpr int OFF_TSHARE = OFF_FLAGS + 16;             // float [2][2][TILE] bounds exchanged per block pair
+constexpr int OFF_CTL = OFF_TSHARE + 4 * TILE * 4;
 constexpr int SMEM_USED = OFF_CTL + (int)sizeof(PipeCtl);
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 // scratch reused after the S pass: per-row undecided candidates, then fallback score rows
@@ -52,101 +57,125 @@ static_assert(MAX_L * 4 <= SCRATCH_BYTES, "fallback score row must fit the S-pas
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 struct RowState {
-    float t;        // raw-score lower bound of tau (scores <= t are never in the support)
-    float m;        // running max raw score
-    int n;          // candidates stored
-    int nallow;     // allowed keys seen
-    int ovf;        // list overflowed: row is redone by the fallback
+    float t;                 // raw-score lower bound of tau (scores <= t are never in the support)
+    float a0, a1, a2, a3;    // four largest raw scores seen by this warpgroup (a0 = running max)
+    int n;                   // candidates stored in this warpgroup's partition
+    int nallow;              // allowed keys seen
+    int ovf;                 // partition overflowed: row is redone by the fallback
 };
 
-// Exact threshold (raw units, constraint sum (v - t)^2 = c4) of the four largest candidates:
-// a valid lower bound of the row's tau, used to prune a full list.
-__device__ __noinline__ void prune_list(RowState& st, float* cv, uint16_t* cj, int r, float c4) {
-    float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-    for (int c = 0; c < st.n; ++c) {
-        const float v = cv[c * TILE + r];
-        if (v > a3) {
-            if (v > a2) {
-                a3 = a2;
-                if (v > a1) {
-                    a2 = a1;
-                    if (v > a0) { a1 = a0; a0 = v; } else { a1 = v; }
-                } else {
-                    a2 = v;
-                }
-            } else {
-                a3 = v;
-            }
-        }
-    }
+struct __align__(16) RowOut {
+    float a0, a1, a2, a3;
+    float t;
+    int n, nallow, ovf;
+};
+
+// Exact threshold (raw units: sum (v - t)^2 = c4 over the kept values) of the set {a0..a3}
+// (a0 >= a1 >= a2 >= a3, missing values -inf), lowered by a rounding margin.  Any subset of a
+// row gives a lower bound of the row's tau: adding scores can only raise the threshold.
+__device__ __forceinline__ float top4_bound(float a0, float a1, float a2, float a3, float c4) {
     const float z[4] = {a0, a1, a2, a3};
+    const float inv[4] = {1.f, 0.5f, 1.f / 3.f, 0.25f};
     float sum = 0.f, sq = 0.f, bound = a0 - sqrtf(c4);
 #pragma unroll
-    for (int k = 1; k <= 4; ++k) {
-        sum += z[k - 1];
-        sq = fmaf(z[k - 1], z[k - 1], sq);
-        const float mu = sum / k;
-        const float delta = c4 / k - (sq / k - mu * mu);
+    for (int k = 0; k < 4; ++k) {
+        sum += z[k];
+        sq = fmaf(z[k], z[k], sq);
+        const float mu = sum * inv[k];
+        const float delta = fmaf(c4 - sq, inv[k], mu * mu);
         if (delta >= 0.f) {
             const float tk = mu - sqrtf(delta);
-            if (tk <= z[k - 1]) bound = tk;
+            if (tk <= z[k]) bound = tk;
         }
     }
-    st.t = fmaxf(st.t, bound);
+    return bound - 1e-5f * sqrtf(c4);
+}
+
+__device__ __forceinline__ void top4_insert(float v, float& a0, float& a1, float& a2, float& a3) {
+    if (v > a3) {
+        if (v > a2) {
+            a3 = a2;
+            if (v > a1) {
+                a2 = a1;
+                if (v > a0) { a1 = a0; a0 = v; } else { a1 = v; }
+            } else {
+                a2 = v;
+            }
+        } else {
+            a3 = v;
+        }
+    }
+}
+
+// Drops the partition's candidates at or below the bound t; returns the new count.
+__device__ __noinline__ int compact_list(float t, int n, float* cv, uint16_t* cj, int r) {
     int w = 0;
-    for (int c = 0; c < st.n; ++c) {
+    for (int c = 0; c < n; ++c) {
         const float v = cv[c * TILE + r];
-        if (v > st.t) {
+        if (v > t) {
             cv[w * TILE + r] = v;
             cj[w * TILE + r] = cj[c * TILE + r];
             ++w;
         }
     }
-    st.n = w;
+    return w;
 }
 
-__device__ __forceinline__ void push_candidate(RowState& st, float v, int j, float* cv, uint16_t* cj, int r,
-                                               float c4, float two_over_scale) {
-    if (st.n == CAP) {
-        prune_list(st, cv, cj, r, c4);
-        if (st.n == CAP) {
+// Append candidate v (key j) to this warpgroup's partition (cv/cj already offset to it), prefetch
+// its V row into L2 for the output gather, and keep the warpgroup's four largest scores.  Returns
+// true when v entered the top four (the caller then tightens the bound once per chunk).
+__device__ __forceinline__ bool push_candidate(RowState& st, float v, int j, float* cv, uint16_t* cj, int r,
+                                               const __nv_bfloat16* Vh) {
+    if (!(v > st.t)) return false;  // the bound rose since the chunk was filtered
+    if (st.n == CAPW) {
+        st.n = compact_list(st.t, st.n, cv, cj, r);
+        if (st.n == CAPW) {
             st.ovf = 1;
             st.t = INFINITY;
-            return;
+            return false;
         }
-        if (!(v > st.t)) return;
     }
     cv[st.n * TILE + r] = v;
     cj[st.n * TILE + r] = (uint16_t)j;
     ++st.n;
-    if (v > st.m) {
-        st.m = v;
-        st.t = fmaxf(st.t, v - two_over_scale);
+    prefetch_l2(Vh + (size_t)j * HEAD_DIM);
+    if (v > st.a3) {
+        top4_insert(v, st.a0, st.a1, st.a2, st.a3);
+        return true;
     }
+    return false;
 }
 
-// Phase 2: tau of one row from its candidate list.  Works in shifted, scaled units
-// x = scale * v - ms (ms = scale * max), bracket [-2, -2/sqrt(nallow)].  Rewrites the list
-// in place as the support: cv <- p_ij, cj <- j.  Returns tau_x; *supp = support size.
-__device__ float solve_row(float* cv, uint16_t* cj, float* U, int r, int n, float scale, float ms, int nallow,
-                           int* supp) {
+// Named barrier over the 8 epilogue warps (id 3; 0 is __syncthreads).
+__device__ __forceinline__ void epi_pair_sync() {
+    asm volatile("bar.sync 3, %0;" ::"n"(NUM_EPI) : "memory");
+}
+
+// Slow path of phase 2 (a partition keeps more than REG_CAND candidates above the bound): the same
+// bisection by one thread over the candidate list in shared memory, with candidates already known
+// to be in the support folded into running moments and those below the bracket dropped.  Writes the
+// support compactly from slot 0: cv <- p_ij, cj <- j.  Returns tau_x; *supp = support size.
+__device__ __noinline__ float solve_row_smem(float* cv, uint16_t* cj, float* U, int r, int n0, int n1, float scale,
+                                             float ms, int nallow, int* supp) {
     float lo = -2.f, hi = -2.f / sqrtf((float)nallow);
-    float K = 0.f, S1 = 0.f, S2 = 0.f;  // moments of candidates known to be in the support
-    int u = 0;                          // undecided candidates (strictly inside the bracket)
-    for (int c = 0; c < n; ++c) {
-        const float x = fmaf(scale, cv[c * TILE + r], -ms);
-        if (x >= hi) {
-            K += 1.f;
-            S1 += x;
-            S2 = fmaf(x, x, S2);
-        } else if (x > lo) {
-            U[u * TILE + r] = x;
-            ++u;
+    float K = 0.f, S1 = 0.f, S2 = 0.f;
+    int u = 0;
+    for (int q = 0; q < NUM_EPI_WG; ++q) {
+        const int n = q == 0 ? n0 : n1;
+        for (int c = q * CAPW; c < q * CAPW + n; ++c) {
+            const float x = fmaf(scale, cv[c * TILE + r], -ms);
+            if (x >= hi) {
+                K += 1.f;
+                S1 += x;
+                S2 = fmaf(x, x, S2);
+            } else if (x > lo) {
+                U[u * TILE + r] = x;
+                ++u;
+            }
         }
     }
     for (int it = 0; it < 25 && u > 0; ++it) {
         const float mid = 0.5f * (lo + hi);
-        // g(mid) = sum over the support side of ((x - mid)/2)^2
         float g = 0.25f * fmaf(mid * K, mid, fmaf(-2.f * mid, S1, S2));
         float ka = 0.f, s1a = 0.f, s2a = 0.f;
         for (int e = 0; e < u; ++e) {
@@ -160,7 +189,7 @@ __device__ float solve_row(float* cv, uint16_t* cj, float* U, int r, int n, floa
             }
         }
         int w = 0;
-        if (g > 1.f) {  // root lies right of mid
+        if (g > 1.f) {
             lo = mid;
             for (int e = 0; e < u; ++e) {
                 const float x = U[e * TILE + r];
@@ -180,7 +209,6 @@ __device__ float solve_row(float* cv, uint16_t* cj, float* U, int r, int n, floa
     }
     float tau_x;
     if (u == 0 && K > 0.f) {
-        // support fixed: sum_S (x - tau)^2 = 4, smaller root
         const float mu = S1 / K;
         const float var = fmaxf(S2 / K - mu * mu, 0.f);
         tau_x = mu - sqrtf(fmaxf(4.f / K - var, 0.f));
@@ -189,20 +217,23 @@ __device__ float solve_row(float* cv, uint16_t* cj, float* U, int r, int n, floa
         tau_x = 0.5f * (lo + hi);
     }
     int s = 0;
-    for (int c = 0; c < n; ++c) {
-        const float x = fmaf(scale, cv[c * TILE + r], -ms);
-        if (x > tau_x) {
-            const float h = 0.5f * (x - tau_x);
-            cv[s * TILE + r] = h * h;
-            cj[s * TILE + r] = cj[c * TILE + r];
-            ++s;
+    for (int q = 0; q < NUM_EPI_WG; ++q) {
+        const int n = q == 0 ? n0 : n1;
+        for (int c = q * CAPW; c < q * CAPW + n; ++c) {
+            const float x = fmaf(scale, cv[c * TILE + r], -ms);
+            if (x > tau_x) {
+                const float h = 0.5f * (x - tau_x);
+                cv[s * TILE + r] = h * h;
+                cj[s * TILE + r] = cj[c * TILE + r];
+                ++s;
+            }
         }
     }
     *supp = s;
     return tau_x;
 }
 
-// Block-wide sum of two floats (all NUM_THREADS threads call it).
+// Block-wide sum of two floats (all NUM_THREADS threads call it).  red: >= 64 floats.
 __device__ __forceinline__ float2 block_sum2(float a, float b, float* red) {
     a = warp_sum(a);
     b = warp_sum(b);
@@ -210,14 +241,14 @@ __device__ __forceinline__ float2 block_sum2(float a, float b, float* red) {
     __syncthreads();
     if (lane == 0) {
         red[warp] = a;
-        red[8 + warp] = b;
+        red[16 + warp] = b;
     }
     __syncthreads();
     float sa = 0.f, sb = 0.f;
 #pragma unroll
-    for (int w = 0; w < NUM_THREADS / 32; ++w) {
+    for (int w = 0; w < NUM_WARPS; ++w) {
         sa += red[w];
-        sb += red[8 + w];
+        sb += red[16 + w];
     }
     return make_float2(sa, sb);
 }
@@ -227,11 +258,11 @@ __device__ __forceinline__ float block_max(float a, float* red) {
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     __syncthreads();
-    if (lane == 0) red[16 + warp] = a;
+    if (lane == 0) red[32 + warp] = a;
     __syncthreads();
     float m = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NUM_THREADS / 32; ++w) m = fmaxf(m, red[16 + w]);
+    for (int w = 0; w < NUM_WARPS; ++w) m = fmaxf(m, red[32 + w]);
     return m;
 }
 
@@ -324,9 +355,10 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         t = 0.5f * (blo + bhi);
     }
     // O_i: thread -> (dimension d, key phase ph)
-    const int d = tid & (HEAD_DIM - 1), ph = tid >> 6;
+    constexpr int PH = NUM_THREADS / HEAD_DIM;
+    const int d = tid % HEAD_DIM, ph = tid / HEAD_DIM;
     float acc = 0.f;
-    for (int e = ph; e < span; e += NUM_THREADS / HEAD_DIM) {
+    for (int e = ph; e < span; e += PH) {
         const float s = sbuf[e];
         if (s > t) {
             const float h = 0.5f * (s - t);
@@ -337,7 +369,9 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
     red[tid] = acc;
     __syncthreads();
     if (tid < HEAD_DIM) {
-        const float o = red[tid] + red[tid + 64] + red[tid + 128] + red[tid + 192];
+        float o = 0.f;
+#pragma unroll
+        for (int p = 0; p < PH; ++p) o += red[tid + p * HEAD_DIM];
         const size_t oi = head + (size_t)i * HEAD_DIM + tid;
         if (out_f32) reinterpret_cast<float*>(O)[oi] = o;
         else reinterpret_cast<__nv_bfloat16*>(O)[oi] = __float2bfloat16_rn(o);
@@ -355,11 +389,14 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     uint8_t* smem_b = smem + OFF_B;
     float* cv = reinterpret_cast<float*>(smem + OFF_CV);
     uint16_t* cj = reinterpret_cast<uint16_t*>(smem + OFF_CJ);
+    float* stage = reinterpret_cast<float*>(smem + OFF_STAGE);
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + OFF_BITS);
     uint16_t* blk_list = reinterpret_cast<uint16_t*>(smem + OFF_BLK);
     int* supp_cnt = reinterpret_cast<int*>(smem + OFF_SUPP);
-    int* nallow_s = reinterpret_cast<int*>(smem + OFF_NALLOW);
+    RowOut* rows = reinterpret_cast<RowOut*>(smem + OFF_ROWS);
     float* red = reinterpret_cast<float*>(smem + OFF_RED);
+    uint32_t* redo = reinterpret_cast<uint32_t*>(smem + OFF_FLAGS);
+    float* tshare = reinterpret_cast<float*>(smem + OFF_TSHARE);
     float* scratch = reinterpret_cast<float*>(smem + OFF_SCRATCH);
     PipeCtl* ctl = reinterpret_cast<PipeCtl*>(smem + OFF_CTL);
 
@@ -369,141 +406,227 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int b = bh / args.H;
     const int i0 = tile * TILE;
     const WaitCfg wc{args.status, args.timeout_ns};
+    const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(args.V) + (size_t)bh * L * HEAD_DIM;
 
     if (tid == 0) {
         init_pipe(ctl);
         prefetch_tmap(&map_q);
         prefetch_tmap(&map_k);
     }
-    if (warp == 4) {
+    if (tid < TILE / 32) redo[tid] = 0u;
+    if (warp == WARP_PRODUCER) {
         tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
         tmem_relinquish();
     }
     build_key_bitmap(bits, args.key_mask, b, L);
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {
         // key blocks that hold at least one key some row of this tile may attend to
         const int i_last = min(i0 + TILE - 1, L - 1);
-        int klo = 0, khi = L - 1;
-        if (args.window > 0) klo = max(0, i0 - args.window + 1);
-        if (args.causal) khi = i_last;
-        int nb = 0;
-        for (int kb = klo / BLK; kb <= khi / BLK; ++kb) {
-            bool any = false;
-            for (int w = kb * (BLK / 32); w < (kb + 1) * (BLK / 32) && w * 32 <= khi; ++w)
-                any |= (bits[w] & range_bits(w * 32, klo, khi)) != 0u;
-            if (any) blk_list[nb++] = (uint16_t)kb;
-        }
-        ctl->nblk = nb;
+        const int klo = args.window > 0 ? max(0, i0 - args.window + 1) : 0;
+        const int khi = args.causal ? i_last : L - 1;
+        const int nb = build_block_list(blk_list, bits, klo, khi, i0, i_last, args.causal, args.window);
+        if (lane == 0) ctl->nblk = nb;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
     const float scale = args.scale;
-    const float two_over_scale = 2.f / scale;
     const float c4 = 4.f / (scale * scale);
-    RowState st{-INFINITY, -INFINITY, 0, 0, 0};
+    const float two_over_scale = 2.f / scale;
 
-    if (warp == 4) {
+    if (warp == WARP_PRODUCER) {
         if (lane == 0) role_producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b);
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == WARP_MMA) {
         if (lane == 0) role_mma(ctl, wc, smem_a, smem_b);
         __syncwarp();
-    } else if (warp < 4) {
-        // ---------------- phase 1: candidate filter (thread r = query row i0 + r)
-        const int r = tid;
+    } else {
+        // ---------------- phase 1: candidate filter (thread (g, r): row i0 + r, blocks n = g mod 2)
+        const int r = tid & (TILE - 1), g = tid >> 7;
+        RowState st{-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, 0, 0, 0};
         const int i = i0 + r;
         int rlo, rhi;
         row_key_range(i, L, args.causal, args.window, rlo, rhi);
-        const uint32_t lane_base = ctl->tmem_base + ((uint32_t)(warp * 32) << 16);
+        float* pcv = cv + g * CAPW * TILE;
+        uint16_t* pcj = cj + g * CAPW * TILE;
         const int nblk = ctl->nblk;
-        for (int n = 0; n < nblk; ++n) {
-            if (!epi_wait_scores(ctl, wc, n)) break;
-            const int j0 = (int)blk_list[n] * BLK;
-#pragma unroll 1
-            for (int c = 0; c < BLK / 32; ++c) {
-                float v[32];
-                tmem_ld32(lane_base + (uint32_t)((n & 1) * BLK + c * 32), v);
-                tmem_wait_ld();
-                if (c == BLK / 32 - 1) epi_release_scores(ctl, n);
-                const int jc = j0 + c * 32;
-                const uint32_t vm = (jc < L) ? (bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
-                if (i >= L) continue;
-                st.nallow += __popc(vm);
-                if (vm == 0xffffffffu) {
+        bool live = true;
+        // the two warpgroups take blocks 2k and 2k+1, then swap bounds: the other warpgroup's bound
+        // is a lower bound of tau as well (any subset of a row), and exchanging it at fixed points
+        // keeps the candidate sets, hence the results, independent of timing
+        for (int k = 0; 2 * k < nblk; ++k) {
+            const int n = 2 * k + g;
+            if (n < nblk && live) live = epi_wait_scores(ctl, wc, n);
+            if (n < nblk && live) {
+                const int j0 = (int)(blk_list[n] & ~FULL_BLOCK) * BLK;
+                const bool full = (blk_list[n] & FULL_BLOCK) && i < L;
+                for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
+                    const int jc = j0 + c * 32;
+                    const uint32_t vm = full ? 0xffffffffu
+                                             : (jc < L && i < L) ? (bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
+                    st.nallow += __popc(vm);
+                    if (st.t == -INFINITY && vm != 0u) {
+                        // first allowed scores of this row: start from (max - 2) of the chunk
+                        float mx = -INFINITY;
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (v[k] > st.t) push_candidate(st, v[k], jc + k, cv, cj, r, c4, two_over_scale);
-                } else if (vm != 0u) {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (((vm >> k) & 1u) && v[k] > st.t) push_candidate(st, v[k], jc + k, cv, cj, r, c4, two_over_scale);
-                }
+                        for (int q = 0; q < 32; ++q) mx = fmaxf(mx, ((vm >> q) & 1u) ? cur[q] : -INFINITY);
+                        st.t = mx - two_over_scale;
+                    }
+                    uint32_t hits = hit_bits(cur, st.t) & __brev(vm);
+                    if (hits) {
+                        stage_chunk(stage, cur);
+                        bool grew = false;
+                        do {
+                            const int q = __clz(hits);
+                            hits &= ~(0x80000000u >> q);
+                            grew |= push_candidate(st, staged(stage, q), jc + q, pcv, pcj, r, Vh);
+                        } while (hits);
+                        // early in the row the bound moves fast: tighten it after every chunk of the
+                        // first block, later once per block pair (below)
+                        if (grew && k == 0) st.t = fmaxf(st.t, top4_bound(st.a0, st.a1, st.a2, st.a3, c4));
+                    }
+                });
             }
+            if (k > 0) st.t = fmaxf(st.t, top4_bound(st.a0, st.a1, st.a2, st.a3, c4));
+            float* tx = tshare + (k & 1) * 2 * TILE;
+            tx[g * TILE + r] = st.t;
+            epi_pair_sync();
+            st.t = fmaxf(st.t, tx[(g ^ 1) * TILE + r]);
         }
+        rows[g * TILE + r] = RowOut{st.a0, st.a1, st.a2, st.a3, st.t, st.n, st.nallow, st.ovf};
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const bool aborted = cta_aborted(ctl);
 
-    // ---------------- phase 2: tau per row (scratch reuses the S-pass buffers)
-    if (!aborted && warp < 4) {
-        const int r = tid, i = i0 + r;
-        int supp = 0;
-        if (i < L) {
-            if (st.nallow == 0) {
-                out.tau[(size_t)bh * L + i] = INFINITY;  // no allowed key: O_i = 0
-            } else if (st.ovf) {
-                supp = -1;
-            } else {
-                const float ms = scale * st.m;
-                const float tau_x = solve_row(cv, cj, scratch, r, st.n, scale, ms, st.nallow, &supp);
-                out.tau[(size_t)bh * L + i] = ms + tau_x;
+    // ---------------- phase 2: tau per row, two threads per row (one per partition)
+    if (!aborted && tid < NUM_EPI) {
+        const int r = (warp << 4) | (lane >> 1), h = lane & 1;
+        const int i = i0 + r;
+        const RowOut s0 = rows[r], s1 = rows[TILE + r];
+        const int nallow = s0.nallow + s1.nallow;
+        const int ovf = s0.ovf | s1.ovf;
+        // merged bound: the four largest scores of the whole row
+        float a0 = s0.a0, a1 = s0.a1, a2 = s0.a2, a3 = s0.a3;
+        top4_insert(s1.a0, a0, a1, a2, a3);
+        top4_insert(s1.a1, a0, a1, a2, a3);
+        top4_insert(s1.a2, a0, a1, a2, a3);
+        top4_insert(s1.a3, a0, a1, a2, a3);
+        const float tf = fmaxf(fmaxf(s0.t, s1.t), top4_bound(a0, a1, a2, a3, c4));
+        const float ms = scale * a0;  // scaled row max
+        int mode = 0;                 // 0: registers, 1: slow path, 2: fallback, 3: no key
+        if (i >= L || nallow == 0) mode = 3;
+        else if (ovf) mode = 2;
+        int nh = h == 0 ? s0.n : s1.n;
+        float* pcv = cv + h * CAPW * TILE;
+        uint16_t* pcj = cj + h * CAPW * TILE;
+        if (mode == 0 && nh > REG_CAND) nh = compact_list(tf, nh, pcv, pcj, r);
+        // every lane takes part in the pair shuffles below (rows of one warp may differ in mode)
+        const int nh_other = __shfl_xor_sync(0xffffffffu, nh, 1);
+        if (mode == 0 && (nh > REG_CAND || nh_other > REG_CAND)) mode = 1;
+        float x[REG_CAND];
+#pragma unroll
+        for (int k = 0; k < REG_CAND; ++k) {
+            const float v = (mode == 0 && k < nh) ? pcv[k * TILE + r] : -INFINITY;
+            x[k] = v > tf ? fmaf(scale, v, -ms) : -INFINITY;
+        }
+        float lo = -2.f, hi = -2.f / sqrtf((float)max(nallow, 1));
+        for (int it = 0; it < 25; ++it) {
+            const float mid = 0.5f * (lo + hi);
+            float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
+#pragma unroll
+            for (int k = 0; k < REG_CAND; k += 4) {
+                const float d0 = fmaxf(x[k] - mid, 0.f), d1 = fmaxf(x[k + 1] - mid, 0.f);
+                const float d2 = fmaxf(x[k + 2] - mid, 0.f), d3 = fmaxf(x[k + 3] - mid, 0.f);
+                g0 = fmaf(d0, d0, g0);
+                g1 = fmaf(d1, d1, g1);
+                g2 = fmaf(d2, d2, g2);
+                g3 = fmaf(d3, d3, g3);
+            }
+            float gs = (g0 + g1) + (g2 + g3);
+            gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+            if (0.25f * gs > 1.f) lo = mid;
+            else hi = mid;
+        }
+        // support fixed by the final bracket: closed-form root of sum_S (x - tau)^2 = 4
+        const float mid = 0.5f * (lo + hi);
+        float K = 0.f, S1 = 0.f, S2 = 0.f;
+#pragma unroll
+        for (int k = 0; k < REG_CAND; ++k) {
+            if (x[k] > mid) {
+                K += 1.f;
+                S1 += x[k];
+                S2 = fmaf(x[k], x[k], S2);
             }
         }
-        supp_cnt[r] = supp;
-        nallow_s[r] = st.nallow;
+        K += __shfl_xor_sync(0xffffffffu, K, 1);
+        S1 += __shfl_xor_sync(0xffffffffu, S1, 1);
+        S2 += __shfl_xor_sync(0xffffffffu, S2, 1);
+        float tau_x = mid;
+        if (K > 0.f) {
+            const float mu = S1 / K;
+            const float var = fmaxf(S2 / K - mu * mu, 0.f);
+            const float tc = mu - sqrtf(fmaxf(4.f / K - var, 0.f));
+            if (tc >= lo && tc <= hi) tau_x = tc;
+        }
+        if (mode == 0) {
+            // this thread's partition of the support: cv <- p_ij, cj <- j (in place)
+            int sn = 0;
+            for (int k = 0; k < nh; ++k) {
+                const float xv = fmaf(scale, pcv[k * TILE + r], -ms);
+                if (xv > tau_x) {
+                    const float hh = 0.5f * (xv - tau_x);
+                    pcv[sn * TILE + r] = hh * hh;
+                    pcj[sn * TILE + r] = pcj[k * TILE + r];
+                    ++sn;
+                }
+            }
+            supp_cnt[h * TILE + r] = sn;
+            if (h == 0) out.tau[(size_t)bh * L + i] = ms + tau_x;
+        } else if (mode == 1) {
+            if (h == 0) {
+                int sn = 0;
+                // counts after this pair's compaction (h = 0 holds partition 0, its partner partition 1)
+                const float tx = solve_row_smem(cv, cj, scratch, r, nh, nh_other, scale, ms, nallow, &sn);
+                supp_cnt[r] = sn;
+                supp_cnt[TILE + r] = 0;
+                out.tau[(size_t)bh * L + i] = ms + tx;
+            }
+        } else if (mode == 2) {
+            if (h == 0) atomicOr(&redo[r >> 5], 1u << (r & 31));
+            supp_cnt[h * TILE + r] = 0;
+        } else {
+            supp_cnt[h * TILE + r] = 0;
+            if (h == 0 && i < L) out.tau[(size_t)bh * L + i] = INFINITY;  // no allowed key: O_i = 0
+        }
     }
     __syncthreads();
 
-    // ---------------- phase 3: O_i = sum_j p_ij V_j, one warp per row
+    // ---------------- phase 3: O_i = sum_j p_ij V_j, one warp per row, two rows in flight
     if (!aborted) {
-        const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(args.V);
-        const size_t head = (size_t)bh * L * HEAD_DIM;
-        for (int r = warp; r < TILE; r += NUM_THREADS / 32) {
-            const int i = i0 + r;
-            const int k = supp_cnt[r];
-            if (i >= L || k < 0) continue;
+        for (int ra = warp; ra < TILE; ra += 2 * NUM_WARPS) {
+            const int rb = ra + NUM_WARPS;
+            const bool okb = rb < TILE;
             float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-            int e = 0;
-            for (; e + 2 <= k; e += 2) {
-                const int j0 = cj[e * TILE + r], j1 = cj[(e + 1) * TILE + r];
-                const float p0 = cv[e * TILE + r], p1 = cv[(e + 1) * TILE + r];
-                const uint32_t w0 = reinterpret_cast<const uint32_t*>(V + head + (size_t)j0 * HEAD_DIM)[lane];
-                const uint32_t w1 = reinterpret_cast<const uint32_t*>(V + head + (size_t)j1 * HEAD_DIM)[lane];
-                a0 = fmaf(p0, bf16lo(w0), a0);
-                a1 = fmaf(p0, bf16hi(w0), a1);
-                b0 = fmaf(p1, bf16lo(w1), b0);
-                b1 = fmaf(p1, bf16hi(w1), b1);
-            }
-            if (e < k) {
-                const int j0 = cj[e * TILE + r];
-                const float p0 = cv[e * TILE + r];
-                const uint32_t w0 = reinterpret_cast<const uint32_t*>(V + head + (size_t)j0 * HEAD_DIM)[lane];
-                a0 = fmaf(p0, bf16lo(w0), a0);
-                a1 = fmaf(p0, bf16hi(w0), a1);
-            }
-            a0 += b0;
-            a1 += b1;
-            const size_t oi = head + (size_t)i * HEAD_DIM + 2 * lane;
-            if (out.out_f32) {
-                *reinterpret_cast<float2*>(reinterpret_cast<float*>(out.O) + oi) = make_float2(a0, a1);
-            } else {
-                __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-                *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out.O) + oi) = h;
+            const int na0 = supp_cnt[ra], na1 = supp_cnt[TILE + ra];
+            const int nb0 = okb ? supp_cnt[rb] : 0, nb1 = okb ? supp_cnt[TILE + rb] : 0;
+            gather_accumulate2(Vh, cj, cv, ra, 0, na0, okb ? rb : ra, 0, nb0, lane, a0, a1, b0, b1);
+            gather_accumulate2(Vh, cj, cv, ra, CAPW, CAPW + na1, okb ? rb : ra, CAPW, CAPW + nb1, lane, a0, a1, b0, b1);
+            for (int q = 0; q < 2; ++q) {
+                const int rr = q == 0 ? ra : rb;
+                const int i = i0 + rr;
+                if ((q == 1 && !okb) || i >= L || ((redo[rr >> 5] >> (rr & 31)) & 1u)) continue;
+                const float o0 = q == 0 ? a0 : b0, o1 = q == 0 ? a1 : b1;
+                const size_t oi = ((size_t)bh * L + i) * HEAD_DIM + 2 * lane;
+                if (out.out_f32) {
+                    *reinterpret_cast<float2*>(reinterpret_cast<float*>(out.O) + oi) = make_float2(o0, o1);
+                } else {
+                    *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out.O) + oi) =
+                        __floats2bfloat162_rn(o0, o1);
+                }
             }
         }
     }
@@ -511,17 +634,22 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 
     // ---------------- phase 4: exact redo of overflowed rows
     if (!aborted) {
-        for (int r = 0; r < TILE; ++r) {
-            if (supp_cnt[r] >= 0) continue;  // uniform across the CTA
-            fallback_row(reinterpret_cast<const __nv_bfloat16*>(args.Q), reinterpret_cast<const __nv_bfloat16*>(args.K),
-                         reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, bh, i0 + r, L,
-                         args.causal, args.window, scale, nallow_s[r], out.O, out.out_f32, out.tau);
+        for (int wd = 0; wd < TILE / 32; ++wd) {
+            uint32_t mask = redo[wd];  // uniform across the CTA
+            while (mask) {
+                const int rr = wd * 32 + __ffs(mask) - 1;
+                mask &= mask - 1;
+                fallback_row(reinterpret_cast<const __nv_bfloat16*>(args.Q), reinterpret_cast<const __nv_bfloat16*>(args.K),
+                             reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, bh, i0 + rr, L,
+                             args.causal, args.window, scale, rows[rr].nallow + rows[TILE + rr].nallow, out.O,
+                             out.out_f32, out.tau);
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == WARP_PRODUCER) {
         tc_fence_after();
         tmem_dealloc(ctl->tmem_base, TMEM_COLS);
     }

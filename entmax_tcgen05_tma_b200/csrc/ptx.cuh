@@ -120,6 +120,19 @@ __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Waits for this thread's outstanding tcgen05.ld and ties the destination registers to the wait,
+// so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld(float (&v)[32]) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+          "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]),
+          "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]),
+          "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+        :
+        : "memory");
+}
+
 // ------------------------------------------------- UMMA operand descriptors
 // Shared-memory matrix descriptor for a K-major operand stored as rows of 128 bytes
 // (64 bf16) in the 128-byte swizzle pattern TMA writes: 8-row groups 1024 bytes apart.
