@@ -316,7 +316,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "algorithmic_flops_per_launch": fwd_alg_flops,
     }
     roof["frac"] = roof["achieved"] / roof["peak"]
-    tr = ROOT / "profiles" / ("traffic_workload%d.json" % w.wid)
+    tr = ROOT / "profiles" / ("traffic_workload%d.txt" % w.wid)
     if tr.exists():
         t = json.loads(tr.read_text())
         if t.get("kernel") == "entmax_fwd_kernel" and t.get("source_hash") == source_hash():

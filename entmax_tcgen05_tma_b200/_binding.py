@@ -3,7 +3,7 @@
 Argument marshalling only: checks tensor placement/dtype/contiguity, allocates outputs with
 torch when the caller gives none, passes raw device pointers and the current CUDA stream, and
 turns status codes into exceptions.  All arithmetic runs in the library's CUDA kernels; there is
-no CPU path.  A missing or unloadable library raises at import.
+no CPU path.  A missing or unloadable library raises ImportError at the first call.
 """
 from __future__ import annotations
 
@@ -67,7 +67,19 @@ def _load_library() -> ctypes.CDLL:
     return lib
 
 
-lib = _load_library()
+class _LazyLibrary:
+    """Loads libentmax_attn.so on first use, so the package (and its build module) imports without
+    the library; any call into the library raises ImportError if it has not been built."""
+
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _LazyLibrary._cdll is None:
+            _LazyLibrary._cdll = _load_library()
+        return getattr(_LazyLibrary._cdll, name)
+
+
+lib = _LazyLibrary()
 
 
 def strerror(status: int) -> str:

@@ -250,3 +250,4 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
 }
 
 }  // extern "C"
+
