@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     EntmaxAttention,
     EntmaxError,
     entmax_attn_bwd,
+    entmax_attn_bwd_noalloc,
     entmax_attn_bwd_workspace_size,
     entmax_attn_device_status,
     entmax_attn_fwd,

@@ -28,6 +28,7 @@ EXPORTED = (
     "entmax_attn_fwd",
     "entmax_attn_bwd_workspace_size",
     "entmax_attn_bwd",
+    "entmax_attn_bwd_noalloc",
     "entmax_attn_strerror",
     "entmax_attn_device_status",
     "entmax_attn_last_cuda_error",
@@ -54,6 +55,8 @@ def _load_library() -> ctypes.CDLL:
     lib.entmax_attn_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.entmax_attn_bwd.restype = i
     lib.entmax_attn_bwd.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.entmax_attn_bwd_noalloc.restype = i
+    lib.entmax_attn_bwd_noalloc.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp]
     lib.entmax_attn_strerror.restype = ctypes.c_char_p
     lib.entmax_attn_strerror.argtypes = [i]
     lib.entmax_attn_device_status.restype = i
@@ -188,6 +191,34 @@ def entmax_attn_bwd(Q, K, V, tau, dO, key_mask=None, causal=False, window=0, sca
                              _stream_handle(stream))
     if st != ENTMAX_OK:
         raise EntmaxError(st, "entmax_attn_bwd")
+    return tuple(outs)
+
+
+def entmax_attn_bwd_noalloc(Q, K, V, tau, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None, dK=None,
+                            dV=None, stream=None):
+    """Backward pass without a workspace argument: the library's own fixed device scratch is used
+    (bf16 inputs, at most 2**20 query rows; calls must not overlap on the GPU).  Returns (dQ, dK, dV)."""
+    B, H, L, D = Q.shape
+    _check_input("Q", Q, (B, H, L, D))
+    _check_input("K", K, (B, H, L, D), Q.dtype)
+    _check_input("V", V, (B, H, L, D), Q.dtype)
+    _check_input("dO", dO, (B, H, L, D), Q.dtype)
+    _check_input("tau", tau, (B, H, L), torch.float32)
+    if scale is None:
+        scale = D ** -0.5
+    outs = []
+    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        if t is None:
+            t = torch.empty((B, H, L, D), dtype=torch.float32, device=Q.device)
+        else:
+            _check_input(name, t, (B, H, L, D), torch.float32)
+        outs.append(t)
+    st = lib.entmax_attn_bwd_noalloc(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
+                                     _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window),
+                                     float(scale), B, H, L, D, tau.data_ptr(), dO.data_ptr(), outs[0].data_ptr(),
+                                     outs[1].data_ptr(), outs[2].data_ptr(), _stream_handle(stream))
+    if st != ENTMAX_OK:
+        raise EntmaxError(st, "entmax_attn_bwd_noalloc")
     return tuple(outs)
 
 

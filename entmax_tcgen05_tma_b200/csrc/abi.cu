@@ -251,3 +251,59 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------------------------
+// Allocation-free backward.  Same computation and kernels as entmax_attn_bwd; the per-row scratch
+// (one float per query row) lives in a fixed device array owned by this library instead of a
+// caller-provided workspace.
+namespace entmax {
+
+constexpr long long NOALLOC_MAX_ROWS = 1ll << 20;  // B*H*L limit: 4 MiB of scratch per device
+
+// File-scope device scratch, present on every GPU that loads the library until the process exits.
+static __device__ __align__(256) float g_noalloc_scratch[NOALLOC_MAX_ROWS];
+
+namespace {
+float* g_noalloc_ptr[MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device.  Looked up once per device (host code
+// may not use the array's symbol as an address); the lookup allocates nothing.
+cudaError_t noalloc_scratch(float** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+}  // namespace entmax
+
+extern "C" int entmax_attn_bwd_noalloc(const void* Q, const void* K, const void* V, int in_dtype,
+                                       const uint8_t* key_mask, int causal, int window, float scale, int B, int H,
+                                       int L, int D, const float* tau, const void* dO, float* dQ, float* dK,
+                                       float* dV, cudaStream_t stream) {
+    int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    if (in_dtype != ENTMAX_BF16) return ENTMAX_ERR_UNSUPPORTED;  // fp32 inputs would need bf16 copies
+    if ((long long)B * H * L > NOALLOC_MAX_ROWS) return ENTMAX_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
+    if (!tau || !dO || !dQ || !dK || !dV) return ENTMAX_ERR_ARG;
+    if (!aligned(dO, 16) || !aligned(dQ, 8) || !aligned(dK, 8) || !aligned(dV, 8) || !aligned(tau, 4))
+        return ENTMAX_ERR_ARG;
+    int* status = nullptr;
+    rc = record(status_ptr(&status));
+    if (rc) return rc;
+    float* scratch = nullptr;
+    rc = record(noalloc_scratch(&scratch));
+    if (rc) return rc;
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    BwdIO io{tau, dO, dQ, dK, dV, scratch};
+    return record(launch_bwd(a, io, stream));
+}

@@ -105,6 +105,31 @@ ENTMAX_API int entmax_attn_bwd(const void* Q, const void* K, const void* V, int 
                     float* dQ, float* dK, float* dV,
                     void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * Allocation-free variant of entmax_attn_bwd (no counterpart in the AdaSplash pages; it exists for
+ * this library's users).  Some callers cannot allocate device memory at the point where they run
+ * the backward pass: engines that plan all memory ahead of time and forbid allocation inside their
+ * execution callbacks, code running while a stream is being captured, or latency-critical loops
+ * where an allocator call would synchronise the device.  This entry point takes the same arguments
+ * as entmax_attn_bwd minus the workspace: its per-row scratch (one float per query row) is a fixed
+ * array inside the library, 4 MiB on every GPU that loads the library, held until the process exits.
+ *   - B*H*L must not exceed 1,048,576 (1 << 20) rows: larger problems return ENTMAX_ERR_UNSUPPORTED
+ *     (use entmax_attn_bwd with a caller workspace instead).
+ *   - Inputs must be bf16 (ENTMAX_F32 returns ENTMAX_ERR_UNSUPPORTED: converting them would need
+ *     temporary memory).
+ *   - It calls no allocation routine.  The first call on a device looks up the array's device
+ *     address (cudaGetSymbolAddress) for that device; make that first call before any stream
+ *     capture.
+ *   - All calls share the one array, which keeps the previous call's contents (every value a call
+ *     reads it writes first).  Calls whose execution overlaps on the GPU, e.g. on two streams,
+ *     race on it: serialise them.
+ */
+ENTMAX_API int entmax_attn_bwd_noalloc(const void* Q, const void* K, const void* V, int in_dtype,
+                                       const uint8_t* key_mask, int causal, int window, float scale,
+                                       int B, int H, int L, int D,
+                                       const float* tau, const void* dO,
+                                       float* dQ, float* dK, float* dV, cudaStream_t stream);
+
 /* Static description of a status code. */
 ENTMAX_API const char* entmax_attn_strerror(int status);
 
