@@ -3,8 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload {2,3,4,5}] [--impl {b200,reference}]
 
-One step = entmax_attn_fwd + entmax_attn_bwd (all kernels of the hot path) over one batch of
-synthetic inputs resident in HBM.  Prints ONE JSON line (rank 0).
+One step = entmax_attn_fwd_train + entmax_attn_bwd_saved (the training path: forward with saved
+supports, then the closed-form backward from them) over one batch of synthetic inputs resident in
+HBM; forward-only workloads run entmax_attn_fwd.  Prints ONE JSON line (rank 0).
 
 Metric: dense-equivalent TFLOP/s = 14 * d * P / t_step (fwd+bwd; 4 * d * P for forward-only
 workloads), where P counts the (query, key) pairs the masks allow -- entmax zeros are never
@@ -204,15 +205,26 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     O = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
     tau = torch.empty((B, H, L), dtype=torch.float32, device=dev)
     dQ, dK, dV = (torch.empty((B, H, L, D), dtype=torch.float32, device=dev) for _ in range(3))
-    ws = torch.empty((E.entmax_attn_bwd_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
+    saved = torch.empty((E.entmax_attn_saved_bytes(B, H, L, D),), dtype=torch.uint8, device=dev)
+    ws = torch.empty((E.entmax_attn_bwd_saved_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 1 + (2 if w.backward else 0)
+    launches_per_step = 1 + (4 if w.backward else 0)
+
+    def fwd_call():
+        if w.backward:
+            E.entmax_attn_fwd_train(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau, saved=saved)
+        else:
+            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+
+    def bwd_call():
+        E.entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV,
+                                workspace=ws)
 
     def step():
-        E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+        fwd_call()
         if w.backward:
-            E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV, workspace=ws)
+            bwd_call()
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -231,11 +243,10 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         for k in range(args.steps):
             flush.fill_(float(k))  # evict L2 between steps (outside the timed events)
             ev[k][0].record(stream)
-            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+            fwd_call()
             ev[k][1].record(stream)
             if w.backward:
-                E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV,
-                                  workspace=ws)
+                bwd_call()
             ev[k][2].record(stream)
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - wall0
@@ -271,13 +282,16 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         Kd = host_in["K"].to(dev, non_blocking=True)
         Vd = host_in["V"].to(dev, non_blocking=True)
         kmd = None if host_km is None else host_km.to(dev, non_blocking=True)
-        Oo, to = E.entmax_attn_fwd(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale)
+        if w.backward:
+            Oo, to, sv = E.entmax_attn_fwd_train(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale, saved=saved)
+        else:
+            Oo, to = E.entmax_attn_fwd(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale)
         host_out["O"].copy_(Oo, non_blocking=True)
         host_out["tau"].copy_(to, non_blocking=True)
         if w.backward:
             dOd = host_in["dO"].to(dev, non_blocking=True)
-            g = E.entmax_attn_bwd(Qd, Kd, Vd, to, dOd, kmd, w.causal, w.window, w.scale, dQ=dQe, dK=dKe, dV=dVe,
-                                  workspace=ws)
+            g = E.entmax_attn_bwd_saved(Qd, Kd, Vd, to, sv, dOd, kmd, w.causal, w.window, w.scale, dQ=dQe, dK=dKe,
+                                        dV=dVe, workspace=ws)
             for name, t in zip(("dQ", "dK", "dV"), g):
                 host_out[name].copy_(t, non_blocking=True)
 

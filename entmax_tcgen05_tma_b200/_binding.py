@@ -29,6 +29,10 @@ EXPORTED = (
     "entmax_attn_bwd_workspace_size",
     "entmax_attn_bwd",
     "entmax_attn_bwd_noalloc",
+    "entmax_attn_saved_bytes",
+    "entmax_attn_bwd_saved_workspace_size",
+    "entmax_attn_fwd_train",
+    "entmax_attn_bwd_saved",
     "entmax_attn_strerror",
     "entmax_attn_device_status",
     "entmax_attn_last_cuda_error",
@@ -57,6 +61,15 @@ def _load_library() -> ctypes.CDLL:
     lib.entmax_attn_bwd.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.entmax_attn_bwd_noalloc.restype = i
     lib.entmax_attn_bwd_noalloc.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp]
+    lib.entmax_attn_saved_bytes.restype = sz
+    lib.entmax_attn_saved_bytes.argtypes = [i, i, i, i]
+    lib.entmax_attn_bwd_saved_workspace_size.restype = sz
+    lib.entmax_attn_bwd_saved_workspace_size.argtypes = [i, i, i, i]
+    lib.entmax_attn_fwd_train.restype = i
+    lib.entmax_attn_fwd_train.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, i, vp, vp, sz, vp]
+    lib.entmax_attn_bwd_saved.restype = i
+    lib.entmax_attn_bwd_saved.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, sz, vp, vp, vp, vp, vp, sz,
+                                          vp]
     lib.entmax_attn_strerror.restype = ctypes.c_char_p
     lib.entmax_attn_strerror.argtypes = [i]
     lib.entmax_attn_device_status.restype = i
@@ -222,6 +235,84 @@ def entmax_attn_bwd_noalloc(Q, K, V, tau, dO, key_mask=None, causal=False, windo
     return tuple(outs)
 
 
+def entmax_attn_saved_bytes(B: int, H: int, L: int, D: int = 64) -> int:
+    return int(lib.entmax_attn_saved_bytes(B, H, L, D))
+
+
+def entmax_attn_bwd_saved_workspace_size(B: int, H: int, L: int, D: int = 64) -> int:
+    return int(lib.entmax_attn_bwd_saved_workspace_size(B, H, L, D))
+
+
+def _byte_buffer(t, nbytes: int, device, name: str):
+    if t is None:
+        return torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=device)
+    if not t.is_cuda or t.numel() * t.element_size() < nbytes:
+        raise ValueError("%s must be a CUDA buffer of at least %d bytes" % (name, nbytes))
+    return t
+
+
+def entmax_attn_fwd_train(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
+                          O=None, tau=None, saved=None, stream=None):
+    """Forward pass that also saves each row's support for entmax_attn_bwd_saved.
+
+    Returns (O, tau, saved); ``saved`` is an opaque uint8 device buffer."""
+    B, H, L, D = Q.shape
+    _check_input("Q", Q, (B, H, L, D))
+    _check_input("K", K, (B, H, L, D), Q.dtype)
+    _check_input("V", V, (B, H, L, D), Q.dtype)
+    if scale is None:
+        scale = D ** -0.5
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be bfloat16 or float32")
+    if O is None:
+        O = torch.empty((B, H, L, D), dtype=out_dtype, device=Q.device)
+    else:
+        _check_input("O", O, (B, H, L, D), out_dtype)
+    if tau is None:
+        tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
+    else:
+        _check_input("tau", tau, (B, H, L), torch.float32)
+    nbytes = entmax_attn_saved_bytes(B, H, L, D)
+    saved = _byte_buffer(saved, nbytes, Q.device, "saved")
+    st = lib.entmax_attn_fwd_train(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
+                                   _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale),
+                                   B, H, L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16,
+                                   tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(),
+                                   _stream_handle(stream))
+    if st != ENTMAX_OK:
+        raise EntmaxError(st, "entmax_attn_fwd_train")
+    return O, tau, saved
+
+
+def entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None,
+                          dK=None, dV=None, workspace=None, stream=None):
+    """Backward pass from the supports saved by entmax_attn_fwd_train.  Returns (dQ, dK, dV) fp32."""
+    B, H, L, D = Q.shape
+    _check_input("Q", Q, (B, H, L, D))
+    _check_input("K", K, (B, H, L, D), Q.dtype)
+    _check_input("V", V, (B, H, L, D), Q.dtype)
+    _check_input("dO", dO, (B, H, L, D), Q.dtype)
+    _check_input("tau", tau, (B, H, L), torch.float32)
+    if scale is None:
+        scale = D ** -0.5
+    outs = []
+    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        if t is None:
+            t = torch.empty((B, H, L, D), dtype=torch.float32, device=Q.device)
+        else:
+            _check_input(name, t, (B, H, L, D), torch.float32)
+        outs.append(t)
+    ws = _byte_buffer(workspace, entmax_attn_bwd_saved_workspace_size(B, H, L, D), Q.device, "workspace")
+    st = lib.entmax_attn_bwd_saved(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
+                                   _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale),
+                                   B, H, L, D, tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(),
+                                   dO.data_ptr(), outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(),
+                                   ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
+    if st != ENTMAX_OK:
+        raise EntmaxError(st, "entmax_attn_bwd_saved")
+    return tuple(outs)
+
+
 def entmax_attn_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(lib.entmax_attn_device_status(_stream_handle(stream)))
@@ -240,15 +331,15 @@ class EntmaxAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, Q, K, V, key_mask=None, causal=False, window=0, scale=None):
-        O, tau = entmax_attn_fwd(Q, K, V, key_mask, causal, window, scale)
-        ctx.save_for_backward(Q, K, V, tau, key_mask if key_mask is not None else torch.empty(0))
+        O, tau, saved = entmax_attn_fwd_train(Q, K, V, key_mask, causal, window, scale)
+        ctx.save_for_backward(Q, K, V, tau, saved, key_mask if key_mask is not None else torch.empty(0))
         ctx.cfg = (key_mask is not None, causal, window, scale)
         return O
 
     @staticmethod
     def backward(ctx, dO):
-        Q, K, V, tau, km = ctx.saved_tensors
+        Q, K, V, tau, saved, km = ctx.saved_tensors
         has_mask, causal, window, scale = ctx.cfg
-        dQ, dK, dV = entmax_attn_bwd(Q, K, V, tau, dO.to(Q.dtype).contiguous(), km if has_mask else None, causal,
-                                     window, scale)
+        dQ, dK, dV = entmax_attn_bwd_saved(Q, K, V, tau, saved, dO.to(Q.dtype).contiguous(),
+                                           km if has_mask else None, causal, window, scale)
         return dQ.to(Q.dtype), dK.to(K.dtype), dV.to(V.dtype), None, None, None, None

@@ -207,7 +207,7 @@ int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, c
         a.K = dst[1];
         a.V = dst[2];
     }
-    FwdOut o{O, out_dtype == ENTMAX_F32, tau};
+    FwdOut o{O, out_dtype == ENTMAX_F32, tau, SavedSupport{}};
     return record(launch_fwd(a, o, stream));
 }
 
@@ -247,6 +247,95 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
         io.dO = dst[3];
     }
     return record(launch_bwd(a, io, stream));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Training path: the forward saves each row's support, the backward works from those lists.
+extern "C" {
+
+size_t entmax_attn_saved_bytes(int B, int H, int L, int D) {
+    (void)D;
+    if (B <= 0 || H <= 0 || L <= 0) return 0;
+    return saved_support_bytes((long long)B * H * L);
+}
+
+size_t entmax_attn_bwd_saved_workspace_size(int B, int H, int L, int D) {
+    (void)D;
+    if (B <= 0 || H <= 0 || L <= 0) return 0;
+    return saved_bwd_ws_bytes((long long)B * H * L);
+}
+
+int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                          int causal, int window, float scale, int B, int H, int L, int D, void* O, int out_dtype,
+                          float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
+    int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
+    if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
+    if (!O || !tau) return ENTMAX_ERR_ARG;
+    if (!aligned(O, 8) || !aligned(tau, 4)) return ENTMAX_ERR_ARG;
+    const long long R = (long long)B * H * L;
+    if (!saved || saved_bytes < saved_support_bytes(R)) return ENTMAX_ERR_WORKSPACE;
+    if (!aligned(saved, 256)) return ENTMAX_ERR_ARG;
+    int* status = nullptr;
+    rc = record(status_ptr(&status));
+    if (rc) return rc;
+    const SavedSupport sv = carve_saved(saved, R);
+    rc = record(cudaMemsetAsync(sv.key_cnt, 0, sizeof(int) * (size_t)R, stream));
+    if (rc) return rc;
+    rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
+    if (rc) return rc;
+    const size_t n = (size_t)R * HEAD_DIM;
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    Bf16Copies tmp;
+    if (in_dtype == ENTMAX_F32) {
+        const void* src[3] = {Q, K, V};
+        const void* dst[3];
+        rc = record(convert_inputs(src, dst, 3, n, tmp, stream));
+        if (rc) return rc;
+        a.Q = dst[0];
+        a.K = dst[1];
+        a.V = dst[2];
+    }
+    FwdOut o{O, out_dtype == ENTMAX_F32, tau, sv};
+    return record(launch_fwd(a, o, stream));
+}
+
+int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                          int causal, int window, float scale, int B, int H, int L, int D, const float* tau,
+                          const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV,
+                          void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
+    if (!tau || !dO || !dQ || !dK || !dV) return ENTMAX_ERR_ARG;
+    if (!aligned(dO, 16) || !aligned(dQ, 8) || !aligned(dK, 8) || !aligned(dV, 8) || !aligned(tau, 4))
+        return ENTMAX_ERR_ARG;
+    const long long R = (long long)B * H * L;
+    if (!saved || saved_bytes < saved_support_bytes(R)) return ENTMAX_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < saved_bwd_ws_bytes(R)) return ENTMAX_ERR_WORKSPACE;
+    if (!aligned(saved, 256) || !aligned(workspace, 256)) return ENTMAX_ERR_ARG;
+    int* status = nullptr;
+    rc = record(status_ptr(&status));
+    if (rc) return rc;
+    const size_t n = (size_t)R * HEAD_DIM;
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    BwdIO io{tau, dO, dQ, dK, dV, nullptr};
+    Bf16Copies tmp;
+    if (in_dtype == ENTMAX_F32) {
+        const void* src[4] = {Q, K, V, dO};
+        const void* dst[4];
+        rc = record(convert_inputs(src, dst, 4, n, tmp, stream));
+        if (rc) return rc;
+        a.Q = dst[0];
+        a.K = dst[1];
+        a.V = dst[2];
+        io.dO = dst[3];
+    }
+    return record(launch_bwd_saved(a, io, carve_saved(const_cast<void*>(saved), R), carve_saved_bwd_ws(workspace, R),
+                                   stream));
 }
 
 }  // extern "C"

@@ -146,6 +146,34 @@ __device__ __forceinline__ bool push_candidate(RowState& st, float v, int j, flo
     return false;
 }
 
+// Writes row r's support (both partitions, p_ij in cv) to the saved lists as (j, sqrt(p_ij)) and
+// counts each key once per row that holds it.  Run by the row's two threads (h = 0, 1) after phase 2;
+// rows redone on CUDA cores (mode 2) or with more than SAVE_CAP entries are marked unsaved.
+__device__ __forceinline__ void save_row_support(const SavedSupport& sv, const float* cv, const uint16_t* cj,
+                                                 const int* supp_cnt, int r, int h, int mode, size_t head_row0,
+                                                 int i, int L) {
+    const int s0 = supp_cnt[r], s1 = supp_cnt[TILE + r];
+    const bool saved = mode != 2 && s0 + s1 <= SAVE_CAP;
+    if (i >= L) return;
+    const size_t row = head_row0 + i;
+    if (!saved) {
+        if (h == 0) {
+            sv.row_cnt[row] = -1;
+            sv.unsaved_rows[atomicAdd(sv.unsaved_cnt, 1)] = (int)row;
+        }
+        return;
+    }
+    if (h == 0) sv.row_cnt[row] = s0 + s1;
+    const int n = h == 0 ? s0 : s1, base = h == 0 ? 0 : s0;
+    const int slot0 = h * CAPW;
+    for (int e = 0; e < n; ++e) {
+        const int j = cj[(slot0 + e) * TILE + r];
+        sv.row_j[row * SAVE_CAP + base + e] = (uint16_t)j;
+        sv.row_sp[row * SAVE_CAP + base + e] = sqrtf(cv[(slot0 + e) * TILE + r]);
+        atomicAdd(sv.key_cnt + head_row0 + j, 1);
+    }
+}
+
 // Named barrier over the 8 epilogue warps (id 3; 0 is __syncthreads).
 __device__ __forceinline__ void epi_pair_sync() {
     asm volatile("bar.sync 3, %0;" ::"n"(NUM_EPI) : "memory");
@@ -602,6 +630,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             supp_cnt[h * TILE + r] = 0;
             if (h == 0 && i < L) out.tau[(size_t)bh * L + i] = INFINITY;  // no allowed key: O_i = 0
         }
+        __syncwarp();  // the slow path's counts (written by h = 0) are read by both threads of the pair
+        if (out.save.row_cnt) save_row_support(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, i, L);
     }
     __syncthreads();
 

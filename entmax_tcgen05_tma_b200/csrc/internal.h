@@ -20,11 +20,29 @@ struct AttnArgs {
     unsigned long long timeout_ns;
 };
 
+// Saved support of the forward pass, consumed by the support-list backward.  R = B*H*L rows.
+constexpr int SAVE_CAP = 64;  // support entries kept per row
+struct SavedSupport {
+    int* row_cnt;            // [R] entries of row, or -1 when the row's support was not saved
+    uint16_t* row_j;         // [R][SAVE_CAP] key index of each entry
+    float* row_sp;           // [R][SAVE_CAP] sqrt(p_ij) = (S_ij - tau_i)/2 of each entry
+    int* key_cnt;            // [R] rows whose support holds key j (zeroed before the forward)
+    int* unsaved_cnt;        // [1] rows whose support was not saved (zeroed before the forward)
+    int* unsaved_rows;       // [R] their row ids
+};
+
 struct FwdOut {
     void* O;                 // [B,H,L,64] bf16 or fp32
     int out_f32;
     float* tau;              // [B,H,L]
+    SavedSupport save;       // row_cnt == nullptr: nothing saved
 };
+
+// Carves a caller buffer of entmax_attn_saved_bytes() into its arrays.
+size_t saved_support_bytes(long long R);
+SavedSupport carve_saved(void* base, long long R);
+
+
 
 struct BwdIO {
     const float* tau;        // [B,H,L] from the forward
@@ -34,6 +52,19 @@ struct BwdIO {
     float* dV;
     float* u;                // workspace [B,H,L]: u_i = sum_j sqrt(p_ij) dA_ij / sum_j sqrt(p_ij)
 };
+
+// Workspace of the support-list backward.
+struct SavedBwdWs {
+    int* key_off;            // [R] head-local start of key j's bucket
+    int* key_cur;            // [R] fill cursor
+    uint32_t* bucket_i;      // [R * SAVE_CAP] query row of each (key, row) entry (head-local)
+    float* bucket_sp;        // [R * SAVE_CAP] sqrt(p_ij)
+    float* bucket_ds;        // [R * SAVE_CAP] dS_ij
+};
+size_t saved_bwd_ws_bytes(long long R);
+SavedBwdWs carve_saved_bwd_ws(void* base, long long R);
+cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv, const SavedBwdWs& ws,
+                             cudaStream_t stream);
 
 // Tensor map over a [B*H, L, 64] bf16 tensor, 128-row boxes, 128-byte swizzle.
 cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L);

@@ -106,6 +106,35 @@ ENTMAX_API int entmax_attn_bwd(const void* Q, const void* K, const void* V, int 
                     void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Training path.  entmax_attn_fwd_train computes exactly what entmax_attn_fwd computes and also saves
+ * each row's support {(j, sqrt(A_ij)) : A_ij > 0} (up to 64 entries per row; rows with more, and rows
+ * the forward had to redo exactly on CUDA cores, are marked and recomputed by the backward) plus, per
+ * key, how many rows hold it.  entmax_attn_bwd_saved then evaluates the same closed-form gradients as
+ * entmax_attn_bwd from those lists without forming Q K^T again: its cost scales with the number of
+ * support entries.  (Page "svd-sst2-roberta-adasplash", section 2.4: the gradient is zero off the
+ * support, and the support is what the forward's tau already fixed.)
+ *   saved      device buffer of entmax_attn_saved_bytes(B,H,L,D) bytes, 256-byte aligned, written by
+ *              entmax_attn_fwd_train and read by entmax_attn_bwd_saved for the same Q, K, masks and
+ *              scale; owned by the caller.
+ *   workspace  device buffer of entmax_attn_bwd_saved_workspace_size(B,H,L,D) bytes, 256-byte aligned.
+ * dK and dV are summed in an order that depends on scheduling (last-bit differences between runs);
+ * dQ, O and tau are deterministic.
+ */
+ENTMAX_API size_t entmax_attn_saved_bytes(int B, int H, int L, int D);
+ENTMAX_API size_t entmax_attn_bwd_saved_workspace_size(int B, int H, int L, int D);
+ENTMAX_API int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dtype,
+                                     const uint8_t* key_mask, int causal, int window, float scale,
+                                     int B, int H, int L, int D,
+                                     void* O, int out_dtype, float* tau,
+                                     void* saved, size_t saved_bytes, cudaStream_t stream);
+ENTMAX_API int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dtype,
+                                     const uint8_t* key_mask, int causal, int window, float scale,
+                                     int B, int H, int L, int D,
+                                     const float* tau, const void* saved, size_t saved_bytes,
+                                     const void* dO, float* dQ, float* dK, float* dV,
+                                     void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Allocation-free variant of entmax_attn_bwd (no counterpart in the AdaSplash pages; it exists for
  * this library's users).  Some callers cannot allocate device memory at the point where they run
  * the backward pass: engines that plan all memory ahead of time and forbid allocation inside their

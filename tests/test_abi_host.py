@@ -118,3 +118,28 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         E.entmax_attn_fwd(x, x, x)
+
+
+def test_training_path_argument_checks():
+    R = 64
+    need = E.entmax_attn_saved_bytes(1, 1, R)
+    assert need > R * 64 * 6 and E.entmax_attn_saved_bytes(0, 1, R) == 0
+    assert E.entmax_attn_bwd_saved_workspace_size(1, 1, R) > R * 64 * 12
+    f = E.lib.entmax_attn_fwd_train
+    args = [P, P, P, 0, None, 0, 0, 0.125, 1, 1, R, 64, P, 0, P, P, need, None]
+    assert f(*args[:16], need - 1, None) == E.ENTMAX_ERR_WORKSPACE
+    assert f(*args[:15], None, need, None) == E.ENTMAX_ERR_WORKSPACE
+    assert f(*args[:15], P + 16, need, None) == E.ENTMAX_ERR_ARG  # not 256-byte aligned
+    bad = list(args)
+    bad[11] = 32
+    assert f(*bad) == E.ENTMAX_ERR_UNSUPPORTED
+    b = E.lib.entmax_attn_bwd_saved
+    ws = E.entmax_attn_bwd_saved_workspace_size(1, 1, R)
+    bargs = [P, P, P, 0, None, 0, 0, 0.125, 1, 1, R, 64, P, P, need, P, P, P, P, P, ws, None]
+    assert b(*bargs[:20], ws - 1, None) == E.ENTMAX_ERR_WORKSPACE
+    nb = list(bargs)
+    nb[13] = None
+    assert b(*nb) == E.ENTMAX_ERR_WORKSPACE
+    nb = list(bargs)
+    nb[16] = P + 4
+    assert b(*nb) == E.ENTMAX_ERR_ARG

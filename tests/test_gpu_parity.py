@@ -10,7 +10,13 @@ import numpy as np
 import pytest
 import torch
 
-from entmax_tcgen05_tma_b200 import entmax_attn_bwd, entmax_attn_device_status, entmax_attn_fwd
+from entmax_tcgen05_tma_b200 import (
+    entmax_attn_bwd,
+    entmax_attn_bwd_saved,
+    entmax_attn_device_status,
+    entmax_attn_fwd,
+    entmax_attn_fwd_train,
+)
 from entmax_tcgen05_tma_b200.workloads import WORKLOADS, Workload, make_inputs
 from oracle import oracle as orc
 from tests.gpu_helpers import GRAD_TOL, O_TOL, check_rows, inputs_f64, to64
@@ -198,3 +204,73 @@ def test_repeat_calls_are_deterministic():
     g2 = _gpu_bwd(dev, t1, inp["dO"], w)
     for a, b in zip(g1, g2):
         assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------------------------- training path
+def _gpu_train(inp, w: Workload, out_dtype=torch.float32):
+    Q, K, V, dO = (inp[k].to(DEV) for k in ("Q", "K", "V", "dO"))
+    km = None if inp["key_mask"] is None else inp["key_mask"].to(DEV)
+    O, tau, saved = entmax_attn_fwd_train(Q, K, V, km, w.causal, w.window, w.scale, out_dtype=out_dtype)
+    dQ, dK, dV = entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale)
+    assert entmax_attn_device_status() == 0
+    return O, tau, (dQ, dK, dV)
+
+
+@pytest.mark.parametrize("B,H,L,scale,causal,window,lens", SMALL)
+def test_training_path_small_full_parity(B, H, L, scale, causal, window, lens):
+    """entmax_attn_fwd_train + entmax_attn_bwd_saved against the oracle, every element."""
+    w = Workload(0, "small", B, H, L, 64, scale, causal, window, lens)
+    inp = make_inputs(w, seed=7 + L + B + window)
+    d = inputs_f64(inp, False)
+    km = _mask_np(inp)
+    O, tau, grads = _gpu_train(inp, w)
+    O_ref, tau_ref = orc.attn_fwd(d["Q"], d["K"], d["V"], km, causal, window, scale)
+    assert np.max(np.abs(to64(O) - O_ref)) <= O_TOL
+    # the training forward computes exactly what the plain forward computes
+    O2, tau2, _ = _gpu_fwd(inp, w)
+    assert torch.equal(O, O2) and torch.equal(tau, tau2)
+    rQ, rK, rV = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], km, causal, window, scale)
+    for name, g, r in (("dQ", grads[0], rQ), ("dK", grads[1], rK), ("dV", grads[2], rV)):
+        err = np.max(np.abs(to64(g) - r))
+        assert err <= GRAD_TOL, (name, err)
+
+
+@pytest.mark.parametrize("wid", [3, 4, 5])
+def test_training_path_full_size_workloads(wid):
+    w = WORKLOADS[wid]
+    inp = make_inputs(w)
+    d = inputs_f64(inp, False)
+    km = _mask_np(inp)
+    O, tau, grads = _gpu_train(inp, w, out_dtype=torch.bfloat16)
+    heads = [0, w.B * w.H - 1] if wid != 4 else [7]
+    rQ, rK, rV = orc.attn_bwd_heads(d["Q"], d["K"], d["V"], d["dO"], heads, km, w.causal, w.window, w.scale)
+    for name, g, r in (("dQ", grads[0], rQ), ("dK", grads[1], rK), ("dV", grads[2], rV)):
+        gh = to64(g).reshape(w.B * w.H, w.L, w.D)[heads]
+        err = np.max(np.abs(gh - r))
+        assert err <= GRAD_TOL, (name, err)
+    for g in grads:
+        assert torch.isfinite(g).all()
+
+
+@pytest.mark.parametrize("L", [100, 300])
+def test_training_path_unsaved_rows(L):
+    """Uniform rows (Q = 0) have supports larger than the saved lists once L > 64: the backward's
+    exact pass recomputes them and adds their dK/dV terms."""
+    w = Workload(0, "uniform", 1, 2, L, 64, 1 / 8)
+    inp = make_inputs(w, seed=11)
+    inp["Q"].zero_()
+    O, tau, grads = _gpu_train(inp, w)
+    d = inputs_f64(inp, False)
+    rQ, rK, rV = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], None, False, 0, w.scale)
+    for g, r in zip(grads, (rQ, rK, rV)):
+        assert np.max(np.abs(to64(g) - r)) <= GRAD_TOL
+
+
+def test_training_path_empty_batch():
+    w = Workload(0, "empty", 2, 2, 200, 64, 1 / 8, len_range=(50, 50))
+    inp = make_inputs(w, seed=3)
+    inp["key_mask"][1] = 0
+    O, tau, grads = _gpu_train(inp, w)
+    assert torch.all(O[1] == 0) and torch.all(torch.isinf(tau[1]))
+    for g in grads:
+        assert torch.all(g[1] == 0)
