@@ -44,7 +44,10 @@ EXPORTED = (
 class EntmaxError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__("%s failed: %s (%d)" % (what, strerror(status), status))
+        msg = "%s failed: %s (%d)" % (what, strerror(status), status)
+        if status == ENTMAX_ERR_CUDA:
+            msg += ", cudaError %d" % lib.entmax_attn_last_cuda_error()
+        super().__init__(msg)
 
 
 def _load_library() -> ctypes.CDLL:

@@ -121,7 +121,7 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, int slot) {
     return e;
 }
 
-cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L) {
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L, int box_rows) {
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!g_encode) {
@@ -135,7 +135,7 @@ cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L) {
     }
     const cuuint64_t dims[3] = {(cuuint64_t)HEAD_DIM, (cuuint64_t)L, (cuuint64_t)BH};
     const cuuint64_t strides[2] = {(cuuint64_t)HEAD_DIM * 2, (cuuint64_t)L * HEAD_DIM * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)HEAD_DIM, (cuuint32_t)TILE, 1};
+    const cuuint32_t box[3] = {(cuuint32_t)HEAD_DIM, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -24,6 +24,14 @@
 namespace entmax {
 namespace {
 
+using P = Pipe<128, 4, 4, 2>;  // 128-key blocks, 4-deep ring, 4 TMEM buffers, 2 epilogue warpgroups
+using PipeCtl = P::Ctl;
+constexpr int BLK = P::BLK, NSTAGE = P::NSTAGE, NBUF = P::NBUF, NUM_EPI_WG = P::NUM_EPI_WG;
+constexpr int NUM_EPI = P::NUM_EPI, NUM_THREADS = P::NUM_THREADS, NUM_WARPS = P::NUM_WARPS;
+constexpr int WARP_PRODUCER = P::WARP_PRODUCER, WARP_MMA = P::WARP_MMA;
+constexpr int BLK_BYTES = P::BLK_BYTES, TMEM_COLS = P::TMEM_COLS, MAX_BLOCKS = P::MAX_BLOCKS;
+constexpr int STAGE_FLOATS = NUM_EPI * 32;  // per-thread staging of one 32-value chunk
+
 constexpr int CAP = 128;              // support entries per row (or key), split between the warpgroups
 constexpr int CAPW = CAP / NUM_EPI_WG;
 
@@ -270,7 +278,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
 __device__ __forceinline__ void setup_cta(const Smem& sm, const CUtensorMap* ma, const CUtensorMap* mb) {
     const int tid = threadIdx.x, warp = tid >> 5;
     if (tid == 0) {
-        init_pipe(sm.ctl);
+        P::init(sm.ctl);
         prefetch_tmap(ma);
         prefetch_tmap(mb);
     }
@@ -309,7 +317,7 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
         const int i_last = min(i0 + TILE - 1, L - 1);
         const int klo = a.window > 0 ? max(0, i0 - a.window + 1) : 0;
         const int khi = a.causal ? i_last : L - 1;
-        const int nb = build_block_list(sm.blk, sm.bits, klo, khi, i0, i_last, a.causal, a.window);
+        const int nb = P::build_block_list(sm.blk, sm.bits, klo, khi, i0, i_last, a.causal, a.window);
         if (lane == 0) ctl->nblk = nb;
     }
     tc_fence_before();
@@ -320,10 +328,10 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
     const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue row and warpgroup
     ListState st{0, 0};
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) role_producer(ctl, wc, &map_q, &map_k, bh, i0, sm.blk, sm.a, sm.b);
+        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, sm.blk, sm.a, sm.b);
         __syncwarp();
     } else if (warp == WARP_MMA) {
-        if (lane == 0) role_mma(ctl, wc, sm.a, sm.b);
+        if (lane == 0) P::mma(ctl, wc, sm.a, sm.b);
         __syncwarp();
     } else {
         const int i = i0 + r;
@@ -338,20 +346,20 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
         uint16_t* pcj = sm.cj + g * CAPW * TILE;
         const int nblk = ctl->nblk;
         for (int n = g; n < nblk; n += NUM_EPI_WG) {
-            if (!epi_wait_scores(ctl, wc, n)) break;
+            if (!P::wait_scores(ctl, wc, n)) break;
             const int j0 = (int)(sm.blk[n] & ~FULL_BLOCK) * BLK;
             const bool full = (sm.blk[n] & FULL_BLOCK) && i < L;
-            for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
+            P::for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
                 const int jc = j0 + c * 32;
                 const uint32_t vm = full ? 0xffffffffu
                                          : (jc < L && i < L) ? (sm.bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
                 uint32_t hits = hit_bits(cur, t) & __brev(vm);
                 if (hits) {
-                    stage_chunk(sm.stage, cur);
+                    stage_chunk(sm.stage, threadIdx.x % NUM_EPI, cur);
                     do {
                         const int k = __clz(hits);
                         hits &= ~(0x80000000u >> k);
-                        push_entry(st, half_scale * (staged(sm.stage, k) - t), jc + k, pcv, pcj, r, Vh, Kh);
+                        push_entry(st, half_scale * (staged(sm.stage, threadIdx.x % NUM_EPI, k) - t), jc + k, pcv, pcj, r, Vh, Kh);
                     } while (hits);
                 }
             });
@@ -362,7 +370,7 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const bool aborted = cta_aborted(ctl);
+    const bool aborted = P::aborted(ctl);
 
     if (!aborted) {
         const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(a.K);
@@ -474,10 +482,10 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
     const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue key and warpgroup
     ListState st{0, 0};
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) role_producer(ctl, wc, &map_k, &map_q, bh, j0, sm.blk, sm.a, sm.b);
+        if (lane == 0) P::producer(ctl, wc, &map_k, &map_q, bh, j0, sm.blk, sm.a, sm.b);
         __syncwarp();
     } else if (warp == WARP_MMA) {
-        if (lane == 0) role_mma(ctl, wc, sm.a, sm.b);
+        if (lane == 0) P::mma(ctl, wc, sm.a, sm.b);
         __syncwarp();
     } else {
         const int j = j0 + r;
@@ -499,9 +507,9 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
                 tb[r] = i < L ? io.tau[(size_t)bh * L + i] / scale : INFINITY;
             }
             wg_sync(g);
-            if (live) live = epi_wait_scores(ctl, wc, n);
+            if (live) live = P::wait_scores(ctl, wc, n);
             if (!live) continue;
-            for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
+            P::for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
                 const int qc = q0 + c * 32;
                 const uint32_t vm = key_ok ? range_bits(qc, qlo, qhi) : 0u;
                 float t[32];
@@ -515,11 +523,11 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
                 }
                 uint32_t hits = hit_bits(cur, t) & __brev(vm);
                 if (hits) {
-                    stage_chunk(sm.stage, cur);
+                    stage_chunk(sm.stage, threadIdx.x % NUM_EPI, cur);
                     do {
                         const int k = __clz(hits);
                         hits &= ~(0x80000000u >> k);
-                        push_entry(st, half_scale * (staged(sm.stage, k) - tb[c * 32 + k]), qc + k, pcv, pcj, r, dOh, Qh);
+                        push_entry(st, half_scale * (staged(sm.stage, threadIdx.x % NUM_EPI, k) - tb[c * 32 + k]), qc + k, pcv, pcj, r, dOh, Qh);
                     } while (hits);
                 }
             });
@@ -530,7 +538,7 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const bool aborted = cta_aborted(ctl);
+    const bool aborted = P::aborted(ctl);
 
     if (!aborted) {
         const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.Q);
@@ -602,9 +610,9 @@ size_t bwd_keys_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream) {
     CUtensorMap mq, mk;
-    cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L);
+    cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L, TILE);
     if (e != cudaSuccess) return e;
-    e = make_tile_map(&mk, a.K, a.B * a.H, a.L);
+    e = make_tile_map(&mk, a.K, a.B * a.H, a.L, BLK);
     if (e != cudaSuccess) return e;
     e = ensure_smem_attr(reinterpret_cast<const void*>(entmax_bwd_rows_kernel), SMEM_BYTES, 1);
     if (e != cudaSuccess) return e;

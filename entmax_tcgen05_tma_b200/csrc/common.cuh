@@ -1,16 +1,16 @@
 // common.cuh -- tile geometry, bounded waits, mask bitmaps and the TMA/tcgen05 score
 // pipeline shared by the forward and backward kernels.
 //
-// Score pipeline ("S pass"): one CTA owns a fixed 128-row tile (the A operand) and streams
-// 128-row blocks of the other operand (B).  For every streamed block the tensor core computes
-// the 128x128 fp32 tile A.B^T into one of four TMEM buffers (block n -> buffer n % 4); two
-// epilogue warpgroups read them back with tcgen05.ld (TMEM lane = row of A), warpgroup g taking
-// the blocks n = g (mod 2), while later blocks' MMAs run.
+// Score pipeline ("S pass"), Pipe<BLK, NSTAGE, NBUF, NWG>: one CTA owns a fixed 128-row tile (the
+// A operand) and streams BLK-row blocks of the other operand (B).  For every streamed block the
+// tensor core computes the 128 x BLK fp32 tile A.B^T into one of NBUF TMEM buffers (block n ->
+// buffer n % NBUF); NWG epilogue warpgroups read them back with tcgen05.ld (TMEM lane = row of A),
+// warpgroup g taking the blocks n = g (mod NWG), while later blocks' MMAs run.
 //
-//   warps 0-3, 4-7  : epilogue warpgroups 0 and 1 -- thread (g, r) serves A row r
-//   warp 8 (lane 0) : TMA producer  -- A tile once, B blocks through an NSTAGE ring
-//   warp 9 (lane 0) : MMA issuer    -- 4 x (M128 N128 K16) per block, commit to mbarriers
-//   warp 8          : TMEM allocation / release
+//   warps 0 .. 4 NWG - 1 : epilogue warpgroups -- thread (g, r) serves A row r
+//   next warp (lane 0)   : TMA producer -- A tile once, B blocks through an NSTAGE ring
+//   next warp (lane 0)   : MMA issuer   -- 4 x (M128 N=BLK K16) per block, commit to mbarriers
+//   producer warp        : TMEM allocation / release
 //
 // Every wait is bounded: on timeout the CTA records ENTMAX_ERR_TIMEOUT in the device status
 // word, raises a CTA-local abort flag that all roles poll, waits (again bounded) for its own
@@ -24,66 +24,41 @@ namespace entmax {
 
 constexpr int HEAD_DIM = 64;            // d, the only head size the kernels take
 constexpr int TILE = 128;               // rows of the fixed tile == MMA M
-constexpr int BLK = 128;                // rows of a streamed block == MMA N
-constexpr int NSTAGE = 4;               // streamed-block ring depth
 constexpr int TILE_BYTES = TILE * HEAD_DIM * 2;  // 16 KiB, bf16 rows of 128 B
-constexpr int BLK_BYTES = BLK * HEAD_DIM * 2;    // 16 KiB
-constexpr int NUM_EPI_WG = 2;           // epilogue warpgroups
-constexpr int NUM_EPI = NUM_EPI_WG * 128;
-constexpr int NBUF = 4;                 // TMEM score buffers
-constexpr int NUM_THREADS = NUM_EPI + 64;  // + producer warp + MMA warp
-constexpr int NUM_WARPS = NUM_THREADS / 32;
-constexpr int WARP_PRODUCER = NUM_EPI / 32;
-constexpr int WARP_MMA = WARP_PRODUCER + 1;
-constexpr int TMEM_COLS = NBUF * BLK;   // four fp32 score buffers = all 512 columns
-constexpr int STAGE_FLOATS = NUM_EPI * 32;  // per-thread staging of one 32-value chunk
 constexpr int MAX_L = 16384;            // longest sequence the kernels take
 constexpr int MASK_WORDS = MAX_L / 32;
-constexpr int MAX_BLOCKS = MAX_L / BLK;
 constexpr uint64_t TEARDOWN_TIMEOUT_NS = 2000000000ull;  // bound for draining in-flight copies
+constexpr uint16_t FULL_BLOCK = 0x8000u;  // block-list flag: every key allowed for every row
 
 // device status codes (mirror entmax_status in include/entmax_attn.h)
 constexpr int STATUS_OK = 0;
 constexpr int STATUS_TIMEOUT = -4;
-
-// Control block shared by all roles of a CTA (lives in shared memory).
-struct PipeCtl {
-    uint64_t full_a;               // A tile landed
-    uint64_t full_b[NSTAGE];       // B block landed
-    uint64_t empty_b[NSTAGE];      // B stage consumed by the MMA
-    uint64_t s_full[NBUF];         // score buffer written
-    uint64_t s_empty[NBUF];        // score buffer read by its epilogue warpgroup
-    uint32_t tmem_base;
-    int abort_flag;
-    int nblk;                      // streamed blocks this CTA visits
-    int pad_;
-};
 
 struct WaitCfg {
     int* status;                   // device status word (global)
     uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ bool cta_aborted(const PipeCtl* ctl) {
-    return *reinterpret_cast<const volatile int*>(&ctl->abort_flag) != 0;
+__device__ __forceinline__ bool flag_set(const int* abort_flag) {
+    return *reinterpret_cast<const volatile int*>(abort_flag) != 0;
 }
 
-static __device__ __noinline__ void raise_timeout(PipeCtl* ctl, const WaitCfg& wc) {
-    *reinterpret_cast<volatile int*>(&ctl->abort_flag) = 1;
+static __device__ __noinline__ void raise_timeout(int* abort_flag, const WaitCfg& wc) {
+    *reinterpret_cast<volatile int*>(abort_flag) = 1;
     if (wc.status) atomicExch(wc.status, STATUS_TIMEOUT);
 }
 
 // Bounded wait on an mbarrier phase.  Returns false if the CTA aborted (this wait timed out,
 // or another role already raised the abort flag).
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, PipeCtl* ctl, const WaitCfg& wc) {
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, int* abort_flag, const WaitCfg& wc) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 127u) == 0) {
-            if (cta_aborted(ctl)) return false;
+            if (flag_set(abort_flag)) return false;
             if (globaltimer_ns() - t0 > wc.timeout_ns) {
-                raise_timeout(ctl, wc);
+                raise_timeout(abort_flag, wc);
                 return false;
             }
         }
@@ -104,7 +79,7 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ void build_key_bitmap(uint32_t* bits, const uint8_t* key_mask, int b, int L) {
     const int nwords = (L + 31) / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int w = warp; w < nwords; w += NUM_THREADS / 32) {
+    for (int w = warp; w < nwords; w += blockDim.x / 32) {
         const int j = w * 32 + lane;
         bool valid = j < L;
         if (valid && key_mask) valid = key_mask[(size_t)b * L + j] != 0;
@@ -134,153 +109,205 @@ __device__ __forceinline__ uint32_t range_bits(int jc, int lo, int hi) {
     return upper & ~((1u << lb) - 1u);
 }
 
-// Streamed key blocks a query tile (rows [i0, i_last]) visits: blocks kb in [klo/BLK, khi/BLK]
-// holding at least one valid key in [klo, khi].  Entry = block index | FULL_BLOCK when every key
-// of the block is valid and allowed for every row of the tile (no per-row mask work needed).
-// Built by warp 0 (one lane per candidate block, ballot + prefix count); returns the count.
-constexpr uint16_t FULL_BLOCK = 0x8000u;
-__device__ __forceinline__ int build_block_list(uint16_t* list, const uint32_t* bits, int klo, int khi, int i0,
-                                                int i_last, int causal, int window) {
-    const int lane = threadIdx.x & 31;
-    const int kb0 = klo / BLK, kb1 = khi / BLK;
-    int nb = 0;
-    for (int base = kb0; base <= kb1; base += 32) {
-        const int kb = base + lane;
-        bool any = false, full = kb <= kb1;
-        if (kb <= kb1) {
-#pragma unroll
-            for (int q = 0; q < BLK / 32; ++q) {
-                const int w = kb * (BLK / 32) + q;
-                const uint32_t word = w * 32 <= khi ? bits[w] : 0u;
-                if (w * 32 <= khi) any |= (word & range_bits(w * 32, klo, khi)) != 0u;
-                full &= word == 0xffffffffu;
-            }
-            const int j0 = kb * BLK, j1 = j0 + BLK - 1;
-            if (causal) full &= j1 <= i0;
-            if (window > 0) full &= j0 >= i_last - window + 1;
-        }
-        const uint32_t bal = __ballot_sync(0xffffffffu, any);
-        if (any) list[nb + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(kb | (full ? FULL_BLOCK : 0));
-        nb += __popc(bal);
-    }
-    return nb;
-}
-
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// ------------------------------------------------------- TMA producer role
-// Loads the fixed A tile (rows a_row0.. of head bh) and then the streamed B blocks listed in
-// blk_list (block index -> rows blk*BLK..) through the NSTAGE ring.
-__device__ __forceinline__ void role_producer(PipeCtl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
-                                              const CUtensorMap* map_b, int bh, int a_row0,
-                                              const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b) {
-    const int nblk = ctl->nblk;
-    mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
-    tma_load_3d(smem_u32(smem_a), map_a, 0, a_row0, bh, smem_u32(&ctl->full_a));
-    int issued = 0;
-    for (int n = 0; n < nblk; ++n) {
-        const int s = n % NSTAGE;
-        const uint32_t ph = (uint32_t)(n / NSTAGE) & 1u;
-        if (!wait_bounded(smem_u32(&ctl->empty_b[s]), ph ^ 1u, ctl, wc)) break;
-        mbar_arrive_expect_tx(smem_u32(&ctl->full_b[s]), BLK_BYTES);
-        tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[n] & ~FULL_BLOCK) * BLK, bh,
-                    smem_u32(&ctl->full_b[s]));
-        ++issued;
-    }
-    if (cta_aborted(ctl)) {
-        // drain: every load issued must land before the CTA's shared memory is released
-        wait_drain(smem_u32(&ctl->full_a), 0);
-        for (int n = max(0, issued - NSTAGE); n < issued; ++n)
-            wait_drain(smem_u32(&ctl->full_b[n % NSTAGE]), (uint32_t)(n / NSTAGE) & 1u);
-    }
-}
+// ------------------------------------------------------------------ score pipeline
+template <int kBlk, int kNStage, int kNBuf, int kNumEpiWg>
+struct Pipe {
+    static constexpr int BLK = kBlk;             // rows of a streamed block == MMA N
+    static constexpr int NSTAGE = kNStage;       // streamed-block ring depth
+    static constexpr int NBUF = kNBuf;           // TMEM score buffers
+    static constexpr int NUM_EPI_WG = kNumEpiWg;
+    static constexpr int NUM_EPI = NUM_EPI_WG * 128;
+    static constexpr int NUM_THREADS = NUM_EPI + 64;  // + producer warp + MMA warp
+    static constexpr int NUM_WARPS = NUM_THREADS / 32;
+    static constexpr int WARP_PRODUCER = NUM_EPI / 32;
+    static constexpr int WARP_MMA = WARP_PRODUCER + 1;
+    static constexpr int BLK_BYTES = BLK * HEAD_DIM * 2;
+    static constexpr int TMEM_COLS = NBUF * BLK;
+    static constexpr int CHUNKS = BLK / 32;       // 32-column chunks per block
+    static constexpr int MAX_BLOCKS = MAX_L / BLK;
+    static_assert(BLK % 32 == 0 && BLK >= 32 && BLK <= 256, "MMA N");
+    static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation");
+    static_assert(NBUF % NUM_EPI_WG == 0, "each warpgroup owns whole buffers");
 
-// ------------------------------------------------------------ MMA issuer role
-__device__ __forceinline__ void role_mma(PipeCtl* ctl, const WaitCfg& wc, const uint8_t* smem_a,
-                                         const uint8_t* smem_b) {
-    const int nblk = ctl->nblk;
-    constexpr uint32_t idesc = umma_idesc_bf16_f32(TILE, BLK);
-    int issued = 0;
-    if (wait_bounded(smem_u32(&ctl->full_a), 0, ctl, wc)) {
-        tc_fence_after();
-        const uint64_t da = umma_desc_kmajor_sw128(smem_u32(smem_a));
-        for (int n = 0; n < nblk; ++n) {
-            const int s = n % NSTAGE, buf = n % NBUF;
-            if (!wait_bounded(smem_u32(&ctl->full_b[s]), (uint32_t)(n / NSTAGE) & 1u, ctl, wc)) break;
-            if (!wait_bounded(smem_u32(&ctl->s_empty[buf]), ((uint32_t)(n / NBUF) & 1u) ^ 1u, ctl, wc)) break;
-            tc_fence_after();
-            const uint64_t db = umma_desc_kmajor_sw128(smem_u32(smem_b + s * BLK_BYTES));
-            const uint32_t d_tmem = ctl->tmem_base + (uint32_t)(buf * BLK);
+    // Control block shared by all roles of a CTA (lives in shared memory).
+    struct Ctl {
+        uint64_t full_a;               // A tile landed
+        uint64_t full_b[NSTAGE];       // B block landed
+        uint64_t empty_b[NSTAGE];      // B stage consumed by the MMA
+        uint64_t s_full[NBUF];         // score buffer written
+        uint64_t s_empty[NBUF];        // score buffer read by its epilogue warpgroup
+        uint32_t tmem_base;
+        int abort_flag;
+        int nblk;                      // streamed blocks this CTA visits
+        int pad_;
+    };
+
+    static __device__ __forceinline__ bool aborted(const Ctl* ctl) { return flag_set(&ctl->abort_flag); }
+
+    static __device__ __forceinline__ void init(Ctl* ctl) {
+        mbar_init(smem_u32(&ctl->full_a), 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(smem_u32(&ctl->full_b[s]), 1);
+            mbar_init(smem_u32(&ctl->empty_b[s]), 1);
+        }
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(smem_u32(&ctl->s_full[b]), 1);
+            mbar_init(smem_u32(&ctl->s_empty[b]), 4);  // one arrival per warp of the owning warpgroup
+        }
+        ctl->abort_flag = 0;
+        fence_barrier_init();
+    }
+
+    // Streamed blocks a query tile (rows [i0, i_last]) visits: blocks kb in [klo/BLK, khi/BLK]
+    // holding at least one valid key in [klo, khi].  Entry = block index | FULL_BLOCK when every key
+    // of the block is valid and allowed for every row of the tile (no per-row mask work needed).
+    // Built by one warp (one lane per candidate block, ballot + prefix count); returns the count.
+    static __device__ __forceinline__ int build_block_list(uint16_t* list, const uint32_t* bits, int klo, int khi,
+                                                           int i0, int i_last, int causal, int window) {
+        const int lane = threadIdx.x & 31;
+        const int kb0 = klo / BLK, kb1 = khi / BLK;
+        int nb = 0;
+        for (int base = kb0; base <= kb1; base += 32) {
+            const int kb = base + lane;
+            bool any = false, full = kb <= kb1;
+            if (kb <= kb1) {
 #pragma unroll
-            for (int k = 0; k < HEAD_DIM / 16; ++k)  // 16 bf16 = 32 B = 2 descriptor units per step
-                tc_mma_bf16(d_tmem, da + 2u * k, db + 2u * k, idesc, k > 0 ? 1u : 0u);
-            tc_commit(smem_u32(&ctl->empty_b[s]));
-            tc_commit(smem_u32(&ctl->s_full[buf]));
+                for (int q = 0; q < CHUNKS; ++q) {
+                    const int w = kb * CHUNKS + q;
+                    const uint32_t word = w * 32 <= khi ? bits[w] : 0u;
+                    if (w * 32 <= khi) any |= (word & range_bits(w * 32, klo, khi)) != 0u;
+                    full &= word == 0xffffffffu;
+                }
+                const int j0 = kb * BLK, j1 = j0 + BLK - 1;
+                if (causal) full &= j1 <= i0;
+                if (window > 0) full &= j0 >= i_last - window + 1;
+            }
+            const uint32_t bal = __ballot_sync(0xffffffffu, any);
+            if (any) list[nb + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(kb | (full ? FULL_BLOCK : 0));
+            nb += __popc(bal);
+        }
+        return nb;
+    }
+
+    // TMA producer: the fixed A tile (rows a_row0.. of head bh), then the streamed B blocks listed
+    // in blk_list through the NSTAGE ring.
+    static __device__ __forceinline__ void producer(Ctl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
+                                                    const CUtensorMap* map_b, int bh, int a_row0,
+                                                    const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b) {
+        const int nblk = ctl->nblk;
+        mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
+        tma_load_3d(smem_u32(smem_a), map_a, 0, a_row0, bh, smem_u32(&ctl->full_a));
+        int issued = 0;
+        for (int n = 0; n < nblk; ++n) {
+            const int s = n % NSTAGE;
+            const uint32_t ph = (uint32_t)(n / NSTAGE) & 1u;
+            if (!wait_bounded(smem_u32(&ctl->empty_b[s]), ph ^ 1u, &ctl->abort_flag, wc)) break;
+            mbar_arrive_expect_tx(smem_u32(&ctl->full_b[s]), BLK_BYTES);
+            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[n] & ~FULL_BLOCK) * BLK, bh,
+                        smem_u32(&ctl->full_b[s]));
             ++issued;
         }
+        if (aborted(ctl)) {
+            // drain: every load issued must land before the CTA's shared memory is released
+            wait_drain(smem_u32(&ctl->full_a), 0);
+            for (int n = max(0, issued - NSTAGE); n < issued; ++n)
+                wait_drain(smem_u32(&ctl->full_b[n % NSTAGE]), (uint32_t)(n / NSTAGE) & 1u);
+        }
     }
-    if (cta_aborted(ctl) && issued > 0) {
-        const int n = issued - 1;  // the last commit covers every earlier MMA
-        wait_drain(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u);
+
+    // MMA issuer (one thread).
+    static __device__ __forceinline__ void mma(Ctl* ctl, const WaitCfg& wc, const uint8_t* smem_a,
+                                               const uint8_t* smem_b) {
+        const int nblk = ctl->nblk;
+        constexpr uint32_t idesc = umma_idesc_bf16_f32(TILE, BLK);
+        int issued = 0;
+        if (wait_bounded(smem_u32(&ctl->full_a), 0, &ctl->abort_flag, wc)) {
+            tc_fence_after();
+            const uint64_t da = umma_desc_kmajor_sw128(smem_u32(smem_a));
+            for (int n = 0; n < nblk; ++n) {
+                const int s = n % NSTAGE, buf = n % NBUF;
+                if (!wait_bounded(smem_u32(&ctl->full_b[s]), (uint32_t)(n / NSTAGE) & 1u, &ctl->abort_flag, wc)) break;
+                if (!wait_bounded(smem_u32(&ctl->s_empty[buf]), ((uint32_t)(n / NBUF) & 1u) ^ 1u, &ctl->abort_flag, wc))
+                    break;
+                tc_fence_after();
+                const uint64_t db = umma_desc_kmajor_sw128(smem_u32(smem_b + s * BLK_BYTES));
+                const uint32_t d_tmem = ctl->tmem_base + (uint32_t)(buf * BLK);
+#pragma unroll
+                for (int k = 0; k < HEAD_DIM / 16; ++k)  // 16 bf16 = 32 B = 2 descriptor units per step
+                    tc_mma_bf16(d_tmem, da + 2u * k, db + 2u * k, idesc, k > 0 ? 1u : 0u);
+                tc_commit(smem_u32(&ctl->empty_b[s]));
+                tc_commit(smem_u32(&ctl->s_full[buf]));
+                ++issued;
+            }
+        }
+        if (aborted(ctl) && issued > 0) {
+            const int n = issued - 1;  // the last commit covers every earlier MMA
+            wait_drain(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u);
+        }
     }
-}
 
-__device__ __forceinline__ void init_pipe(PipeCtl* ctl) {
-    mbar_init(smem_u32(&ctl->full_a), 1);
-    for (int s = 0; s < NSTAGE; ++s) {
-        mbar_init(smem_u32(&ctl->full_b[s]), 1);
-        mbar_init(smem_u32(&ctl->empty_b[s]), 1);
+    // Epilogue side: wait for the score buffer of streamed block n; false on abort.
+    static __device__ __forceinline__ bool wait_scores(Ctl* ctl, const WaitCfg& wc, int n) {
+        const bool ok = wait_bounded(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u, &ctl->abort_flag, wc);
+        tc_fence_after();
+        return ok;
     }
-    for (int b = 0; b < NBUF; ++b) {
-        mbar_init(smem_u32(&ctl->s_full[b]), 1);
-        mbar_init(smem_u32(&ctl->s_empty[b]), 4);  // one arrival per warp of the owning warpgroup
+
+    // Epilogue side: this warp finished reading the score buffer of block n.
+    static __device__ __forceinline__ void release_scores(Ctl* ctl, int n) {
+        tc_fence_before();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&ctl->s_empty[n % NBUF]));
     }
-    ctl->abort_flag = 0;
-    fence_barrier_init();
-}
 
-// Epilogue side: wait for score buffer of streamed block n; false on abort.
-__device__ __forceinline__ bool epi_wait_scores(PipeCtl* ctl, const WaitCfg& wc, int n) {
-    const bool ok = wait_bounded(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u, ctl, wc);
-    tc_fence_after();
-    return ok;
-}
+    // TMEM address of lane quarter (warp % 4), buffer of block n, 32-column chunk c.
+    static __device__ __forceinline__ uint32_t taddr(const Ctl* ctl, int n, int c) {
+        const int warp = threadIdx.x >> 5;
+        return ctl->tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((n % NBUF) * BLK + c * 32);
+    }
 
-// Epilogue side: this warp finished reading score buffer of block n.
-__device__ __forceinline__ void epi_release_scores(PipeCtl* ctl, int n) {
-    tc_fence_before();
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&ctl->s_empty[n % NBUF]));
-}
+    // Reads the 32-column chunks of score block n one at a time (for kernels with enough epilogue
+    // warps per SM sub-partition to hide the TMEM load latency) and calls f(v, c) for chunk c.  The
+    // buffer goes back to the MMA warp once its last chunk is in registers.
+    template <class F>
+    static __device__ __forceinline__ void for_each_chunk_single(Ctl* ctl, int n, F&& f) {
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+            float v[32];
+            tmem_ld32(taddr(ctl, n, c), v);
+            tmem_wait_ld(v);
+            if (c == CHUNKS - 1) release_scores(ctl, n);
+            f(v, c);
+        }
+    }
 
-// TMEM address of lane quarter (warp % 4), buffer of block n, 32-column chunk c.
-__device__ __forceinline__ uint32_t epi_taddr(const PipeCtl* ctl, int n, int c) {
-    const int warp = threadIdx.x >> 5;
-    return ctl->tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((n % NBUF) * BLK + c * 32);
-}
-
-// Reads the four 32-column chunks of score block n, double-buffered in registers, and calls
-// f(v, c) for chunk c.  The buffer is released to the MMA warp once its last chunk is loaded.
-template <class F>
-__device__ __forceinline__ void for_each_chunk(PipeCtl* ctl, int n, F&& f) {
-    static_assert(BLK == 128, "four chunks per block");
-    float va[32], vb[32];
-    tmem_ld32(epi_taddr(ctl, n, 0), va);
-    tmem_wait_ld(va);
-    tmem_ld32(epi_taddr(ctl, n, 1), vb);
-    f(va, 0);
-    tmem_wait_ld(vb);
-    tmem_ld32(epi_taddr(ctl, n, 2), va);
-    f(vb, 1);
-    tmem_wait_ld(va);
-    tmem_ld32(epi_taddr(ctl, n, 3), vb);
-    f(va, 2);
-    tmem_wait_ld(vb);
-    epi_release_scores(ctl, n);
-    f(vb, 3);
-}
+    // Reads the 32-column chunks of score block n (the next chunk's load in flight while f runs)
+    // and calls f(v, c) for chunk c.  The buffer goes back to the MMA warp once its last chunk is in
+    // registers.
+    template <class F>
+    static __device__ __forceinline__ void for_each_chunk(Ctl* ctl, int n, F&& f) {
+        float va[32], vb[32];
+        tmem_ld32(taddr(ctl, n, 0), va);
+        tmem_wait_ld(va);
+#pragma unroll
+        for (int c = 0; c < CHUNKS; c += 2) {
+            if (c + 1 < CHUNKS) tmem_ld32(taddr(ctl, n, c + 1), vb);
+            else release_scores(ctl, n);
+            f(va, c);
+            if (c + 1 < CHUNKS) {
+                tmem_wait_ld(vb);
+                if (c + 2 < CHUNKS) tmem_ld32(taddr(ctl, n, c + 2), va);
+                else release_scores(ctl, n);
+                f(vb, c + 1);
+                if (c + 2 < CHUNKS) tmem_wait_ld(va);
+            }
+        }
+    }
+};
 
 // ------------------------------------------------------------ hit filtering
 // Bit (31 - k) of the result is set iff v[k] > t: the sign bit of t - v[k] funnel-shifted into
@@ -312,18 +339,33 @@ __device__ __forceinline__ uint32_t hit_bits(const float (&v)[32], const float (
 
 // Per-thread staging of a 32-value chunk in shared memory (16-byte groups XOR-swizzled by the
 // thread index, so a warp's 128-bit stores are conflict-free), read back by dynamic index.
-__device__ __forceinline__ void stage_chunk(float* stage, const float (&v)[32]) {
-    float* row = stage + (threadIdx.x % NUM_EPI) * 32;
-    const int sw = threadIdx.x & 7;
+// `slot` = the thread's epilogue index.
+__device__ __forceinline__ void stage_chunk(float* stage, int slot, const float (&v)[32]) {
+    float* row = stage + slot * 32;
+    const int sw = slot & 7;
 #pragma unroll
     for (int c = 0; c < 8; ++c)
         *reinterpret_cast<float4*>(row + ((c ^ sw) << 2)) = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
 }
 
-__device__ __forceinline__ float staged(const float* stage, int k) {
-    return stage[(threadIdx.x % NUM_EPI) * 32 + ((((k >> 2) ^ (threadIdx.x & 7))) << 2) + (k & 3)];
+__device__ __forceinline__ float staged(const float* stage, int slot, int k) {
+    return stage[slot * 32 + ((((k >> 2) ^ (slot & 7))) << 2) + (k & 3)];
 }
 
+// Half-chunk variants (16 values: chunk values [16 half, 16 half + 16)).
+__device__ __forceinline__ void stage_half(float* stage, int slot, const float (&v)[32], int half) {
+    float* row = stage + slot * 16;
+    const int sw = slot & 3;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int b = 16 * half + 4 * c;
+        *reinterpret_cast<float4*>(row + ((c ^ sw) << 2)) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
+    }
+}
+
+__device__ __forceinline__ float staged_half(const float* stage, int slot, int k16) {
+    return stage[slot * 16 + ((((k16 >> 2) ^ (slot & 3))) << 2) + (k16 & 3)];
+}
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

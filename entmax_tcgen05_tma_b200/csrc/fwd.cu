@@ -29,6 +29,14 @@
 namespace entmax {
 namespace {
 
+using P = Pipe<128, 4, 4, 2>;  // 128-key blocks, 4-deep ring, 4 TMEM buffers, 2 epilogue warpgroups
+using PipeCtl = P::Ctl;
+constexpr int BLK = P::BLK, NSTAGE = P::NSTAGE, NUM_EPI_WG = P::NUM_EPI_WG;
+constexpr int NUM_EPI = P::NUM_EPI, NUM_THREADS = P::NUM_THREADS, NUM_WARPS = P::NUM_WARPS;
+constexpr int WARP_PRODUCER = P::WARP_PRODUCER, WARP_MMA = P::WARP_MMA;
+constexpr int BLK_BYTES = P::BLK_BYTES, TMEM_COLS = P::TMEM_COLS, MAX_BLOCKS = P::MAX_BLOCKS;
+constexpr int STAGE_FLOATS = NUM_EPI * 32;  // per-thread staging of one 32-value chunk
+
 constexpr int CAP = 128;              // candidates per row, split between the two warpgroups
 constexpr int CAPW = CAP / NUM_EPI_WG;
 constexpr int REG_CAND = 32;          // candidates per thread held in registers by the tau solve
@@ -437,7 +445,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(args.V) + (size_t)bh * L * HEAD_DIM;
 
     if (tid == 0) {
-        init_pipe(ctl);
+        P::init(ctl);
         prefetch_tmap(&map_q);
         prefetch_tmap(&map_k);
     }
@@ -453,7 +461,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const int i_last = min(i0 + TILE - 1, L - 1);
         const int klo = args.window > 0 ? max(0, i0 - args.window + 1) : 0;
         const int khi = args.causal ? i_last : L - 1;
-        const int nb = build_block_list(blk_list, bits, klo, khi, i0, i_last, args.causal, args.window);
+        const int nb = P::build_block_list(blk_list, bits, klo, khi, i0, i_last, args.causal, args.window);
         if (lane == 0) ctl->nblk = nb;
     }
     tc_fence_before();
@@ -465,10 +473,10 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const float two_over_scale = 2.f / scale;
 
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) role_producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b);
+        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b);
         __syncwarp();
     } else if (warp == WARP_MMA) {
-        if (lane == 0) role_mma(ctl, wc, smem_a, smem_b);
+        if (lane == 0) P::mma(ctl, wc, smem_a, smem_b);
         __syncwarp();
     } else {
         // ---------------- phase 1: candidate filter (thread (g, r): row i0 + r, blocks n = g mod 2)
@@ -486,11 +494,11 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // keeps the candidate sets, hence the results, independent of timing
         for (int k = 0; 2 * k < nblk; ++k) {
             const int n = 2 * k + g;
-            if (n < nblk && live) live = epi_wait_scores(ctl, wc, n);
+            if (n < nblk && live) live = P::wait_scores(ctl, wc, n);
             if (n < nblk && live) {
                 const int j0 = (int)(blk_list[n] & ~FULL_BLOCK) * BLK;
                 const bool full = (blk_list[n] & FULL_BLOCK) && i < L;
-                for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
+                P::for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
                     const int jc = j0 + c * 32;
                     const uint32_t vm = full ? 0xffffffffu
                                              : (jc < L && i < L) ? (bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
@@ -504,12 +512,12 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     }
                     uint32_t hits = hit_bits(cur, st.t) & __brev(vm);
                     if (hits) {
-                        stage_chunk(stage, cur);
+                        stage_chunk(stage, threadIdx.x % NUM_EPI, cur);
                         bool grew = false;
                         do {
                             const int q = __clz(hits);
                             hits &= ~(0x80000000u >> q);
-                            grew |= push_candidate(st, staged(stage, q), jc + q, pcv, pcj, r, Vh);
+                            grew |= push_candidate(st, staged(stage, threadIdx.x % NUM_EPI, q), jc + q, pcv, pcj, r, Vh);
                         } while (hits);
                         // early in the row the bound moves fast: tighten it after every chunk of the
                         // first block, later once per block pair (below)
@@ -528,7 +536,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const bool aborted = cta_aborted(ctl);
+    const bool aborted = P::aborted(ctl);
 
     // ---------------- phase 2: tau per row, two threads per row (one per partition)
     if (!aborted && tid < NUM_EPI) {
@@ -691,9 +699,9 @@ size_t fwd_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream) {
     CUtensorMap mq, mk;
-    cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L);
+    cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L, TILE);
     if (e != cudaSuccess) return e;
-    e = make_tile_map(&mk, a.K, a.B * a.H, a.L);
+    e = make_tile_map(&mk, a.K, a.B * a.H, a.L, BLK);
     if (e != cudaSuccess) return e;
     e = ensure_smem_attr(reinterpret_cast<const void*>(entmax_fwd_kernel), SMEM_BYTES, 0);
     if (e != cudaSuccess) return e;

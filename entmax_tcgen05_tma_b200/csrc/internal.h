@@ -66,8 +66,8 @@ SavedBwdWs carve_saved_bwd_ws(void* base, long long R);
 cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv, const SavedBwdWs& ws,
                              cudaStream_t stream);
 
-// Tensor map over a [B*H, L, 64] bf16 tensor, 128-row boxes, 128-byte swizzle.
-cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L);
+// Tensor map over a [B*H, L, 64] bf16 tensor, boxes of box_rows rows, 128-byte swizzle.
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L, int box_rows);
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
 cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
