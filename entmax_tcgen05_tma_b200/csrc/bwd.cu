@@ -328,10 +328,10 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
     const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue row and warpgroup
     ListState st{0, 0};
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, sm.blk, sm.a, sm.b);
+        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, sm.blk, sm.a, sm.b, ctl->nblk);
         __syncwarp();
     } else if (warp == WARP_MMA) {
-        if (lane == 0) P::mma(ctl, wc, sm.a, sm.b);
+        if (lane == 0) P::mma(ctl, wc, sm.a, sm.b, ctl->nblk);
         __syncwarp();
     } else {
         const int i = i0 + r;
@@ -482,10 +482,10 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
     const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue key and warpgroup
     ListState st{0, 0};
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) P::producer(ctl, wc, &map_k, &map_q, bh, j0, sm.blk, sm.a, sm.b);
+        if (lane == 0) P::producer(ctl, wc, &map_k, &map_q, bh, j0, sm.blk, sm.a, sm.b, ctl->nblk);
         __syncwarp();
     } else if (warp == WARP_MMA) {
-        if (lane == 0) P::mma(ctl, wc, sm.a, sm.b);
+        if (lane == 0) P::mma(ctl, wc, sm.a, sm.b, ctl->nblk);
         __syncwarp();
     } else {
         const int j = j0 + r;

@@ -193,21 +193,24 @@ struct Pipe {
         return nb;
     }
 
-    // TMA producer: the fixed A tile (rows a_row0.. of head bh), then the streamed B blocks listed
-    // in blk_list through the NSTAGE ring.
+    // TMA producer: the fixed A tile (rows a_row0.. of head bh), then njobs streamed B blocks through
+    // the NSTAGE ring, job n loading listed block n mod nblk (njobs <= 2 nblk: a second pass re-streams
+    // the list).
     static __device__ __forceinline__ void producer(Ctl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
                                                     const CUtensorMap* map_b, int bh, int a_row0,
-                                                    const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b) {
+                                                    const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b,
+                                                    int njobs) {
         const int nblk = ctl->nblk;
         mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
         tma_load_3d(smem_u32(smem_a), map_a, 0, a_row0, bh, smem_u32(&ctl->full_a));
         int issued = 0;
-        for (int n = 0; n < nblk; ++n) {
+        for (int n = 0; n < njobs; ++n) {
             const int s = n % NSTAGE;
             const uint32_t ph = (uint32_t)(n / NSTAGE) & 1u;
             if (!wait_bounded(smem_u32(&ctl->empty_b[s]), ph ^ 1u, &ctl->abort_flag, wc)) break;
+            const int e = n < nblk ? n : n - nblk;
             mbar_arrive_expect_tx(smem_u32(&ctl->full_b[s]), BLK_BYTES);
-            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[n] & ~FULL_BLOCK) * BLK, bh,
+            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[e] & ~FULL_BLOCK) * BLK, bh,
                         smem_u32(&ctl->full_b[s]));
             ++issued;
         }
@@ -221,14 +224,13 @@ struct Pipe {
 
     // MMA issuer (one thread).
     static __device__ __forceinline__ void mma(Ctl* ctl, const WaitCfg& wc, const uint8_t* smem_a,
-                                               const uint8_t* smem_b) {
-        const int nblk = ctl->nblk;
+                                               const uint8_t* smem_b, int njobs) {
         constexpr uint32_t idesc = umma_idesc_bf16_f32(TILE, BLK);
         int issued = 0;
         if (wait_bounded(smem_u32(&ctl->full_a), 0, &ctl->abort_flag, wc)) {
             tc_fence_after();
             const uint64_t da = umma_desc_kmajor_sw128(smem_u32(smem_a));
-            for (int n = 0; n < nblk; ++n) {
+            for (int n = 0; n < njobs; ++n) {
                 const int s = n % NSTAGE, buf = n % NBUF;
                 if (!wait_bounded(smem_u32(&ctl->full_b[s]), (uint32_t)(n / NSTAGE) & 1u, &ctl->abort_flag, wc)) break;
                 if (!wait_bounded(smem_u32(&ctl->s_empty[buf]), ((uint32_t)(n / NBUF) & 1u) ^ 1u, &ctl->abort_flag, wc))
@@ -286,9 +288,9 @@ struct Pipe {
     }
 
     // Reads the 32-column chunks of score block n (the next chunk's load in flight while f runs)
-    // and calls f(v, c) for chunk c.  The buffer goes back to the MMA warp once its last chunk is in
-    // registers.
-    template <class F>
+    // and calls f(v, c) for chunk c.  With kRelease the buffer goes back to the MMA warp once its
+    // last chunk is in registers; without, it stays readable for a later pass.
+    template <bool kRelease = true, class F>
     static __device__ __forceinline__ void for_each_chunk(Ctl* ctl, int n, F&& f) {
         float va[32], vb[32];
         tmem_ld32(taddr(ctl, n, 0), va);
@@ -296,12 +298,12 @@ struct Pipe {
 #pragma unroll
         for (int c = 0; c < CHUNKS; c += 2) {
             if (c + 1 < CHUNKS) tmem_ld32(taddr(ctl, n, c + 1), vb);
-            else release_scores(ctl, n);
+            else if (kRelease) release_scores(ctl, n);
             f(va, c);
             if (c + 1 < CHUNKS) {
                 tmem_wait_ld(vb);
                 if (c + 2 < CHUNKS) tmem_ld32(taddr(ctl, n, c + 2), va);
-                else release_scores(ctl, n);
+                else if (kRelease) release_scores(ctl, n);
                 f(vb, c + 1);
                 if (c + 2 < CHUNKS) tmem_wait_ld(va);
             }

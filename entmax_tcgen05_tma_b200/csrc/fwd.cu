@@ -7,20 +7,21 @@
 //   O_i = sum_j max(0, (S_ij - tau_i)/2)^2 V_j.
 //
 // One CTA per 128-query tile.  Phases:
-//  1. S pass (common.cuh): QK^T on tcgen05, 128 keys per block, fp32 scores in TMEM.  Each
-//     epilogue thread owns one query row and keeps only *candidates*: scores above a running
-//     lower bound t of tau (max - 2, tightened to the exact threshold of the row's top four
-//     scores whenever the list fills).  A score at or below any lower bound of tau is outside
-//     the support, so the support is a subset of the candidates.
-//  2. tau solve per row on the candidate list: the pages' 25 halvings of the bracket
-//     [max - 2, max - 2/sqrt(n)], with g(mid) summed over the candidates (held in registers by two
-//     threads per row), then the root of sum_S (S_ij - tau)^2 = 4 in closed form on the support
-//     S = {S_ij > final midpoint}, kept if it lies in the final bracket (else the midpoint).
-//  3. O_i = sum p_ij V_j over the support (typically 5-40 keys) with one warp per row: lane l
-//     accumulates dimensions 2l, 2l+1 from V rows gathered out of L2 (prefetched into L2 when the
-//     candidate was listed).
-//  4. Rows whose candidates exceed the list capacity are redone exactly by the whole CTA on
-//     CUDA cores (scores into shared memory, bisection with block reductions).
+//  1. Score passes (common.cuh pipeline): QK^T on tcgen05, 128 keys per block, fp32 scores in TMEM.
+//     Pass A reduces every row to its maximum m_i over the allowed keys.  Pass B keeps the row's
+//     *candidates*, the scores above m_i - 2 (scaled units) -- the bisection's lower bracket end,
+//     so the support is a subset of them -- as (score, key) lists in shared memory.  When the
+//     tile's key blocks fit in TMEM at once (at most four blocks: L <= 512, or a causal window)
+//     the scores are computed once and read twice ("resident"); otherwise the blocks are streamed
+//     twice, the second time recomputing the scores.
+//  2. tau per row on the candidate list (two threads per row, candidates in registers): halvings
+//     of [m-2, m-2/sqrt(n)] until no candidate is left strictly inside the bracket (at most 25),
+//     then the root of sum_S (S_ij - tau)^2 = 4 in closed form on the support S so fixed.
+//  3. O_i = sum p_ij V_j over the support with one warp per row: lane l accumulates dimensions
+//     2l, 2l+1.  Resident tiles gather V rows from shared memory (TMA-loaded during phase 2);
+//     streamed tiles gather them from L2 (prefetched when the candidate was listed).
+//  4. Rows with more candidates than a list holds are redone exactly by the whole CTA on CUDA
+//     cores (scores into shared memory, bisection with block reductions).
 #include <cuda_bf16.h>
 #include <math.h>
 #include "common.cuh"
@@ -31,53 +32,49 @@ namespace {
 
 using P = Pipe<128, 4, 4, 2>;  // 128-key blocks, 4-deep ring, 4 TMEM buffers, 2 epilogue warpgroups
 using PipeCtl = P::Ctl;
-constexpr int BLK = P::BLK, NSTAGE = P::NSTAGE, NUM_EPI_WG = P::NUM_EPI_WG;
+constexpr int BLK = P::BLK, NSTAGE = P::NSTAGE, NBUF = P::NBUF;
 constexpr int NUM_EPI = P::NUM_EPI, NUM_THREADS = P::NUM_THREADS, NUM_WARPS = P::NUM_WARPS;
 constexpr int WARP_PRODUCER = P::WARP_PRODUCER, WARP_MMA = P::WARP_MMA;
 constexpr int BLK_BYTES = P::BLK_BYTES, TMEM_COLS = P::TMEM_COLS, MAX_BLOCKS = P::MAX_BLOCKS;
 constexpr int STAGE_FLOATS = NUM_EPI * 32;  // per-thread staging of one 32-value chunk
+static_assert(NSTAGE >= NBUF, "a resident tile's V blocks are staged in the streamed-block ring");
 
 constexpr int CAP = 128;              // candidates per row, split between the two warpgroups
-constexpr int CAPW = CAP / NUM_EPI_WG;
-constexpr int REG_CAND = 32;          // candidates per thread held in registers by the tau solve
+constexpr int CAPW = CAP / 2;
 
 // shared-memory layout (bytes from the 1024-aligned base)
 constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + TILE_BYTES;
-constexpr int OFF_CV = OFF_B + NSTAGE * BLK_BYTES;     // float [CAP][TILE]
-constexpr int OFF_CJ = OFF_CV + CAP * TILE * 4;        // u16   [CAP][TILE]
-constexpr int OFF_STAGE = OFF_CJ + CAP * TILE * 2;     // float [NUM_EPI][32]
-constexpr int OFF_BITS = OFF_STAGE + STAGE_FLOATS * 4; // u32   [MASK_WORDS]
-constexpr int OFF_BLK = OFF_BITS + MASK_WORDS * 4;     // u16   [MAX_BLOCKS]
-constexpr int OFF_SUPP = OFF_BLK + MAX_BLOCKS * 2;     // int   [2][TILE] support size per partition
-constexpr int OFF_ROWS = OFF_SUPP + 2 * TILE * 4;      // RowOut[2][TILE] per-warpgroup row state
-constexpr int OFF_RED = OFF_ROWS + 2 * TILE * 32;      // float [NUM_THREADS]
-constexpr int OFF_FLAGS = OFF_RED + NUM_THREADS * 4;   // u32   [TILE/32] rows redone by the fallback
-constexpr int OFF_TSHARE = OFF_FLAGS + 16;             // float [2][2][TILE] bounds exchanged per block pair
-constexpr int OFF_CTL = OFF_TSHARE + 4 * TILE * 4;
+constexpr int OFF_B = OFF_A + TILE_BYTES;               // K ring; V blocks of a resident tile in phase 3
+constexpr int OFF_CV = OFF_B + NSTAGE * BLK_BYTES;      // float [CAP][TILE]
+constexpr int OFF_CJ = OFF_CV + CAP * TILE * 4;         // u16   [CAP][TILE]
+constexpr int OFF_STAGE = OFF_CJ + CAP * TILE * 2;      // float [NUM_EPI][32]
+constexpr int OFF_BITS = OFF_STAGE + STAGE_FLOATS * 4;  // u32   [MASK_WORDS]
+constexpr int OFF_BLK = OFF_BITS + MASK_WORDS * 4;      // u16   [MAX_BLOCKS]
+constexpr int OFF_VSLOT = OFF_BLK + MAX_BLOCKS * 2;     // u8    [MAX_BLOCKS] ring slot of key block kb's V rows
+constexpr int OFF_SUPP = OFF_VSLOT + MAX_BLOCKS;        // int   [2][TILE] support size per partition
+constexpr int OFF_ROWS = OFF_SUPP + 2 * TILE * 4;       // RowOut[2][TILE] per-warpgroup row state
+constexpr int OFF_RED = OFF_ROWS + 2 * TILE * 32;       // float [NUM_THREADS]
+constexpr int OFF_FLAGS = OFF_RED + NUM_THREADS * 4;    // u32   [TILE/32] rows redone by the fallback
+constexpr int OFF_VBAR = OFF_FLAGS + 16;                // u64   mbarrier: V blocks landed
+constexpr int OFF_CTL = OFF_VBAR + 16;
 constexpr int SMEM_USED = OFF_CTL + (int)sizeof(PipeCtl);
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
-// scratch reused after the S pass: per-row undecided candidates, then fallback score rows
+// scratch reused by the fallback after phase 3: one score row
 constexpr int OFF_SCRATCH = 0;
 constexpr int SCRATCH_BYTES = OFF_CV;
-static_assert(CAP * TILE * 4 <= SCRATCH_BYTES, "undecided-candidate scratch must fit the S-pass buffers");
-static_assert(MAX_L * 4 <= SCRATCH_BYTES, "fallback score row must fit the S-pass buffers");
+static_assert(MAX_L * 4 <= SCRATCH_BYTES, "fallback score row must fit the score-pass buffers");
+static_assert(OFF_SUPP % 16 == 0 && OFF_ROWS % 16 == 0 && OFF_VBAR % 8 == 0, "alignment");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
-struct RowState {
-    float t;                 // raw-score lower bound of tau (scores <= t are never in the support)
-    float a0, a1, a2, a3;    // four largest raw scores seen by this warpgroup (a0 = running max)
-    int n;                   // candidates stored in this warpgroup's partition
-    int nallow;              // allowed keys seen
-    int ovf;                 // partition overflowed: row is redone by the fallback
-};
-
+// Per-warpgroup row state: pass-A four largest scores and allowed-key count over the warpgroup's
+// keys, pass-B candidate count of its partition and overflow flag.
 struct __align__(16) RowOut {
     float a0, a1, a2, a3;
-    float t;
-    int n, nallow, ovf;
+    int nallow;
+    int n;
+    int ovf;
+    int pad_;
 };
-
 // Exact threshold (raw units: sum (v - t)^2 = c4 over the kept values) of the set {a0..a3}
 // (a0 >= a1 >= a2 >= a3, missing values -inf), lowered by a rounding margin.  Any subset of a
 // row gives a lower bound of the row's tau: adding scores can only raise the threshold.
@@ -115,43 +112,203 @@ __device__ __forceinline__ void top4_insert(float v, float& a0, float& a1, float
     }
 }
 
-// Drops the partition's candidates at or below the bound t; returns the new count.
-__device__ __noinline__ int compact_list(float t, int n, float* cv, uint16_t* cj, int r) {
-    int w = 0;
-    for (int c = 0; c < n; ++c) {
-        const float v = cv[c * TILE + r];
-        if (v > t) {
-            cv[w * TILE + r] = v;
-            cj[w * TILE + r] = cj[c * TILE + r];
-            ++w;
-        }
-    }
-    return w;
+
+// Named barrier over the 8 epilogue warps (id 3; 0 is __syncthreads).
+__device__ __forceinline__ void epi_sync() {
+    asm volatile("bar.sync 3, %0;" ::"n"(NUM_EPI) : "memory");
 }
 
-// Append candidate v (key j) to this warpgroup's partition (cv/cj already offset to it), prefetch
-// its V row into L2 for the output gather, and keep the warpgroup's four largest scores.  Returns
-// true when v entered the top four (the caller then tightens the bound once per chunk).
-__device__ __forceinline__ bool push_candidate(RowState& st, float v, int j, float* cv, uint16_t* cj, int r,
-                                               const __nv_bfloat16* Vh) {
-    if (!(v > st.t)) return false;  // the bound rose since the chunk was filtered
-    if (st.n == CAPW) {
-        st.n = compact_list(st.t, st.n, cv, cj, r);
-        if (st.n == CAPW) {
-            st.ovf = 1;
-            st.t = INFINITY;
-            return false;
+// Bounded mbarrier wait whose outcome the whole warp shares (the warp-collective tcgen05 loads
+// that follow must be executed by all lanes or none).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* abort_flag, const WaitCfg& wc) {
+    return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, wc));
+}
+
+// Maximum of the chunk values whose bit (k) is set in vm (bit k <-> value k), -inf if none.
+__device__ __forceinline__ float masked_max(const float (&v)[32], uint32_t vm) {
+    float a = -INFINITY, b = -INFINITY, c = -INFINITY, d = -INFINITY;
+    if (vm == 0xffffffffu) {
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+            a = fmaxf(a, v[k]);
+            b = fmaxf(b, v[k + 1]);
+            c = fmaxf(c, v[k + 2]);
+            d = fmaxf(d, v[k + 3]);
+        }
+    } else if (vm != 0u) {
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+            a = fmaxf(a, ((vm >> k) & 1u) ? v[k] : -INFINITY);
+            b = fmaxf(b, ((vm >> (k + 1)) & 1u) ? v[k + 1] : -INFINITY);
+            c = fmaxf(c, ((vm >> (k + 2)) & 1u) ? v[k + 2] : -INFINITY);
+            d = fmaxf(d, ((vm >> (k + 3)) & 1u) ? v[k + 3] : -INFINITY);
         }
     }
-    cv[st.n * TILE + r] = v;
-    cj[st.n * TILE + r] = (uint16_t)j;
-    ++st.n;
-    prefetch_l2(Vh + (size_t)j * HEAD_DIM);
-    if (v > st.a3) {
-        top4_insert(v, st.a0, st.a1, st.a2, st.a3);
-        return true;
+    return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// Reads chunks 2 half and 2 half + 1 of the (resident) score buffer of block n and calls f(v, c).
+template <class F>
+__device__ __forceinline__ void for_half_block(const PipeCtl* ctl, int n, int half, F&& f) {
+    float va[32], vb[32];
+    tmem_ld32(P::taddr(ctl, n, 2 * half), va);
+    tmem_ld32(P::taddr(ctl, n, 2 * half + 1), vb);
+    tmem_wait_ld(va);
+    tmem_wait_ld(vb);
+    f(va, 2 * half);
+    f(vb, 2 * half + 1);
+}
+
+// tau of one row in shifted scaled units (x = scale * S - scale * m, so the row max is 0), from the
+// candidates of the two partitions held by a lane pair (NC registers each, -inf where unused).
+// Bisection of [-2, -2/sqrt(n)] (g(-2) >= 1 from the max alone, g(-2/sqrt n) <= 1); every four
+// halvings the warp stops if no lane pair has a candidate strictly inside its bracket: the support
+// is then fixed and the closed-form root on it is exact.  Returns tau_x.
+template <int NC>
+__device__ __forceinline__ float solve_tau(const float* pcv, int r, int nh, float scale, float ms, int nallow) {
+    float x[NC];
+#pragma unroll
+    for (int k = 0; k < NC; ++k) x[k] = k < nh ? fmaf(scale, pcv[k * TILE + r], -ms) : -INFINITY;
+    float lo = -2.f, hi = -2.f / sqrtf((float)max(nallow, 1));
+    bool settled = false;
+    for (int it = 0; it < 25; ++it) {
+        const float mid = 0.5f * (lo + hi);
+        float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
+#pragma unroll
+        for (int k = 0; k < NC; k += 4) {
+            const float d0 = fmaxf(x[k] - mid, 0.f), d1 = fmaxf(x[k + 1] - mid, 0.f);
+            const float d2 = fmaxf(x[k + 2] - mid, 0.f), d3 = fmaxf(x[k + 3] - mid, 0.f);
+            g0 = fmaf(d0, d0, g0);
+            g1 = fmaf(d1, d1, g1);
+            g2 = fmaf(d2, d2, g2);
+            g3 = fmaf(d3, d3, g3);
+        }
+        float gs = (g0 + g1) + (g2 + g3);
+        gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+        if (0.25f * gs > 1.f) lo = mid;
+        else hi = mid;
+        if ((it & 3) == 3 || it == 24) {
+            int und = 0;
+#pragma unroll
+            for (int k = 0; k < NC; ++k) und += (x[k] > lo && x[k] < hi) ? 1 : 0;
+            und += __shfl_xor_sync(0xffffffffu, und, 1);
+            settled = und == 0;
+            if (__all_sync(0xffffffffu, settled)) break;
+        }
     }
-    return false;
+    // closed-form root of sum_S (x - tau)^2 = 4 on S = {x > final midpoint}
+    const float mid = 0.5f * (lo + hi);
+    float K = 0.f, S1 = 0.f, S2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+        if (x[k] > mid) {
+            K += 1.f;
+            S1 += x[k];
+            S2 = fmaf(x[k], x[k], S2);
+        }
+    }
+    K += __shfl_xor_sync(0xffffffffu, K, 1);
+    S1 += __shfl_xor_sync(0xffffffffu, S1, 1);
+    S2 += __shfl_xor_sync(0xffffffffu, S2, 1);
+    float tau_x = mid;
+    if (K > 0.f) {
+        const float mu = S1 / K;
+        const float var = fmaxf(S2 / K - mu * mu, 0.f);
+        const float tc = mu - sqrtf(fmaxf(4.f / K - var, 0.f));
+        // with the support settled the root lies in the bracket (clamp only absorbs rounding);
+        // otherwise keep it only if it does
+        if (settled) tau_x = fminf(fmaxf(tc, lo), hi);
+        else if (tc >= lo && tc <= hi) tau_x = tc;
+    }
+    return tau_x;
+}
+
+// Support entry e of row r (partition 0 holds entries [0, n0), partition 1 the rest): key j and
+// weight p_ij from the [slot][TILE] lists.
+__device__ __forceinline__ void support_entry(const uint16_t* cj, const float* cw, int r, int n0, int e, int& j,
+                                              float& w) {
+    const int sl = e < n0 ? e : CAPW + (e - n0);
+    j = cj[sl * TILE + r];
+    w = cw[sl * TILE + r];
+}
+
+__device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4& x) {
+    const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        acc[2 * k] = fmaf(w, bf16lo(u[k]), acc[2 * k]);
+        acc[2 * k + 1] = fmaf(w, bf16hi(u[k]), acc[2 * k + 1]);
+    }
+}
+
+// O rows ra and rb (rb < 0: none) = sum over their support of p_ij V_j, one warp: lane = 8 grp + sub,
+// group grp takes every fourth entry, lane sub the 16-byte column chunk (dimensions 8 sub .. 8 sub + 7).
+// V rows come from the shared-memory ring (kSmem: 128-byte swizzled blocks of BLK keys, block kb in
+// slot vslot[kb]) or from global memory.  The four groups' sums are reduced with shuffles; the
+// result is valid in lanes 0..7 (acc index = dimension - 8 sub).
+template <bool kSmem>
+__device__ __forceinline__ void gather_rows(const uint8_t* vring, const uint8_t* vslot, const __nv_bfloat16* Vh,
+                                            const uint16_t* cj, const float* cw, int ra, int na0, int na1, int rb,
+                                            int nb0, int nb1, int lane, float (&oa)[8], float (&ob)[8]) {
+    const int grp = lane >> 3, sub = lane & 7;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) oa[k] = ob[k] = 0.f;
+    const int na = na0 + na1, nb = rb >= 0 ? nb0 + nb1 : 0;
+    auto load = [&](int j) -> uint4 {
+        if (kSmem) {
+            const uint32_t row = (uint32_t)j & (BLK - 1);
+            const uint8_t* p = vring + vslot[j / BLK] * BLK_BYTES + row * 128u + (((uint32_t)sub ^ (row & 7u)) << 4);
+            return *reinterpret_cast<const uint4*>(p);
+        } else {
+            return __ldg(reinterpret_cast<const uint4*>(Vh + (size_t)j * HEAD_DIM) + sub);
+        }
+    };
+    for (int e = grp; e < na || e < nb; e += 8) {
+        uint4 x[4];
+        float w[4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int ea = e + 4 * u;
+            int j;
+            w[u] = w[2 + u] = 0.f;
+            x[u] = x[2 + u] = make_uint4(0u, 0u, 0u, 0u);
+            if (ea < na) {
+                support_entry(cj, cw, ra, na0, ea, j, w[u]);
+                x[u] = load(j);
+            }
+            if (ea < nb) {
+                support_entry(cj, cw, rb, nb0, ea, j, w[2 + u]);
+                x[2 + u] = load(j);
+            }
+        }
+        fma_bf16x8(oa, w[0], x[0]);
+        fma_bf16x8(oa, w[1], x[1]);
+        fma_bf16x8(ob, w[2], x[2]);
+        fma_bf16x8(ob, w[3], x[3]);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        oa[k] += __shfl_xor_sync(0xffffffffu, oa[k], 8);
+        ob[k] += __shfl_xor_sync(0xffffffffu, ob[k], 8);
+        oa[k] += __shfl_xor_sync(0xffffffffu, oa[k], 16);
+        ob[k] += __shfl_xor_sync(0xffffffffu, ob[k], 16);
+    }
+}
+
+// Lanes 0..7 store their 8 dimensions of O row i.
+__device__ __forceinline__ void store_o_row(const FwdOut& out, size_t row, int lane, const float (&o)[8]) {
+    if (lane >= 8) return;
+    const size_t oi = row * HEAD_DIM + 8 * lane;
+    if (out.out_f32) {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out.O) + oi);
+        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+    } else {
+        __nv_bfloat162 h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) h[k] = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
+        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out.O) + oi) = *reinterpret_cast<const uint4*>(h);
+    }
 }
 
 // Writes row r's support (both partitions, p_ij in cv) to the saved lists as (j, sqrt(p_ij)) and
@@ -180,93 +337,6 @@ __device__ __forceinline__ void save_row_support(const SavedSupport& sv, const f
         sv.row_sp[row * SAVE_CAP + base + e] = sqrtf(cv[(slot0 + e) * TILE + r]);
         atomicAdd(sv.key_cnt + head_row0 + j, 1);
     }
-}
-
-// Named barrier over the 8 epilogue warps (id 3; 0 is __syncthreads).
-__device__ __forceinline__ void epi_pair_sync() {
-    asm volatile("bar.sync 3, %0;" ::"n"(NUM_EPI) : "memory");
-}
-
-// Slow path of phase 2 (a partition keeps more than REG_CAND candidates above the bound): the same
-// bisection by one thread over the candidate list in shared memory, with candidates already known
-// to be in the support folded into running moments and those below the bracket dropped.  Writes the
-// support compactly from slot 0: cv <- p_ij, cj <- j.  Returns tau_x; *supp = support size.
-__device__ __noinline__ float solve_row_smem(float* cv, uint16_t* cj, float* U, int r, int n0, int n1, float scale,
-                                             float ms, int nallow, int* supp) {
-    float lo = -2.f, hi = -2.f / sqrtf((float)nallow);
-    float K = 0.f, S1 = 0.f, S2 = 0.f;
-    int u = 0;
-    for (int q = 0; q < NUM_EPI_WG; ++q) {
-        const int n = q == 0 ? n0 : n1;
-        for (int c = q * CAPW; c < q * CAPW + n; ++c) {
-            const float x = fmaf(scale, cv[c * TILE + r], -ms);
-            if (x >= hi) {
-                K += 1.f;
-                S1 += x;
-                S2 = fmaf(x, x, S2);
-            } else if (x > lo) {
-                U[u * TILE + r] = x;
-                ++u;
-            }
-        }
-    }
-    for (int it = 0; it < 25 && u > 0; ++it) {
-        const float mid = 0.5f * (lo + hi);
-        float g = 0.25f * fmaf(mid * K, mid, fmaf(-2.f * mid, S1, S2));
-        float ka = 0.f, s1a = 0.f, s2a = 0.f;
-        for (int e = 0; e < u; ++e) {
-            const float x = U[e * TILE + r];
-            if (x >= mid) {
-                const float d = x - mid;
-                g = fmaf(0.25f * d, d, g);
-                ka += 1.f;
-                s1a += x;
-                s2a = fmaf(x, x, s2a);
-            }
-        }
-        int w = 0;
-        if (g > 1.f) {
-            lo = mid;
-            for (int e = 0; e < u; ++e) {
-                const float x = U[e * TILE + r];
-                if (x > mid) U[w++ * TILE + r] = x;
-            }
-        } else {
-            hi = mid;
-            K += ka;
-            S1 += s1a;
-            S2 += s2a;
-            for (int e = 0; e < u; ++e) {
-                const float x = U[e * TILE + r];
-                if (x < mid) U[w++ * TILE + r] = x;
-            }
-        }
-        u = w;
-    }
-    float tau_x;
-    if (u == 0 && K > 0.f) {
-        const float mu = S1 / K;
-        const float var = fmaxf(S2 / K - mu * mu, 0.f);
-        tau_x = mu - sqrtf(fmaxf(4.f / K - var, 0.f));
-        tau_x = fminf(fmaxf(tau_x, lo), hi);
-    } else {
-        tau_x = 0.5f * (lo + hi);
-    }
-    int s = 0;
-    for (int q = 0; q < NUM_EPI_WG; ++q) {
-        const int n = q == 0 ? n0 : n1;
-        for (int c = q * CAPW; c < q * CAPW + n; ++c) {
-            const float x = fmaf(scale, cv[c * TILE + r], -ms);
-            if (x > tau_x) {
-                const float h = 0.5f * (x - tau_x);
-                cv[s * TILE + r] = h * h;
-                cj[s * TILE + r] = cj[c * TILE + r];
-                ++s;
-            }
-        }
-    }
-    *supp = s;
-    return tau_x;
 }
 
 // Block-wide sum of two floats (all NUM_THREADS threads call it).  red: >= 64 floats.
@@ -418,7 +488,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                  const AttnArgs args, const FwdOut out) {
+                  const __grid_constant__ CUtensorMap map_v, const AttnArgs args, const FwdOut out) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* smem_a = smem + OFF_A;
@@ -428,11 +498,12 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     float* stage = reinterpret_cast<float*>(smem + OFF_STAGE);
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + OFF_BITS);
     uint16_t* blk_list = reinterpret_cast<uint16_t*>(smem + OFF_BLK);
+    uint8_t* vslot = smem + OFF_VSLOT;
     int* supp_cnt = reinterpret_cast<int*>(smem + OFF_SUPP);
     RowOut* rows = reinterpret_cast<RowOut*>(smem + OFF_ROWS);
     float* red = reinterpret_cast<float*>(smem + OFF_RED);
     uint32_t* redo = reinterpret_cast<uint32_t*>(smem + OFF_FLAGS);
-    float* tshare = reinterpret_cast<float*>(smem + OFF_TSHARE);
+    uint64_t* vbar = reinterpret_cast<uint64_t*>(smem + OFF_VBAR);
     float* scratch = reinterpret_cast<float*>(smem + OFF_SCRATCH);
     PipeCtl* ctl = reinterpret_cast<PipeCtl*>(smem + OFF_CTL);
 
@@ -445,9 +516,11 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(args.V) + (size_t)bh * L * HEAD_DIM;
 
     if (tid == 0) {
-        P::init(ctl);
+        mbar_init(smem_u32(vbar), 1);
+        P::init(ctl);  // ends with the barrier-init fence
         prefetch_tmap(&map_q);
         prefetch_tmap(&map_k);
+        prefetch_tmap(&map_v);
     }
     if (tid < TILE / 32) redo[tid] = 0u;
     if (warp == WARP_PRODUCER) {
@@ -462,6 +535,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const int klo = args.window > 0 ? max(0, i0 - args.window + 1) : 0;
         const int khi = args.causal ? i_last : L - 1;
         const int nb = P::build_block_list(blk_list, bits, klo, khi, i0, i_last, args.causal, args.window);
+        __syncwarp();
+        if (nb <= NBUF && lane < nb) vslot[blk_list[lane] & ~FULL_BLOCK] = (uint8_t)lane;
         if (lane == 0) ctl->nblk = nb;
     }
     tc_fence_before();
@@ -469,74 +544,140 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     tc_fence_after();
 
     const float scale = args.scale;
-    const float c4 = 4.f / (scale * scale);
     const float two_over_scale = 2.f / scale;
+    const float c4 = 4.f / (scale * scale);
+    const int nblk = ctl->nblk;
+    const bool resident = nblk <= NBUF;
+    const int njobs = resident ? nblk : 2 * nblk;
 
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b);
+        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs);
         __syncwarp();
     } else if (warp == WARP_MMA) {
-        if (lane == 0) P::mma(ctl, wc, smem_a, smem_b);
+        if (lane == 0) P::mma(ctl, wc, smem_a, smem_b, njobs);
         __syncwarp();
     } else {
-        // ---------------- phase 1: candidate filter (thread (g, r): row i0 + r, blocks n = g mod 2)
+        // thread (g, r): query row i0 + r; warpgroup g takes half g of every block (resident) or
+        // every other block (streamed)
         const int r = tid & (TILE - 1), g = tid >> 7;
-        RowState st{-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, 0, 0, 0};
         const int i = i0 + r;
         int rlo, rhi;
         row_key_range(i, L, args.causal, args.window, rlo, rhi);
+        auto allowed = [&](int n, int jc) -> uint32_t {
+            const bool full = (blk_list[n] & FULL_BLOCK) && i < L;
+            return full ? 0xffffffffu : (jc < L && i < L) ? (bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
+        };
+        bool live = true;
+
+        // ---------------- pass A: four largest scores and allowed-key count
+        // Only scores above th = max(a3, a0 - 2/scale) can change the top four in a way that matters:
+        // scores at or below a0 - 2/scale never enter the support, so leaving them out of the top
+        // four only weakens bounds that max - 2 already dominates.
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+        float th = -INFINITY;
+        int nallow = 0;
+        const int slot = threadIdx.x % NUM_EPI;
+        auto pass_a = [&](int n) {
+            const int j0 = (int)(blk_list[n] & ~FULL_BLOCK) * BLK;
+            return [&, n, j0](const float (&cur)[32], int c) {
+                const uint32_t vm = allowed(n, j0 + c * 32);
+                nallow += __popc(vm);
+                if (a0 == -INFINITY && vm != 0u) th = masked_max(cur, vm) - two_over_scale;
+                uint32_t hits = hit_bits(cur, th) & __brev(vm);
+                if (hits) {
+                    stage_chunk(stage, slot, cur);
+                    do {
+                        const int q = __clz(hits);
+                        hits &= ~(0x80000000u >> q);
+                        top4_insert(staged(stage, slot, q), a0, a1, a2, a3);
+                    } while (hits);
+                    th = fmaxf(a3, a0 - two_over_scale);
+                }
+            };
+        };
+        if (resident) {
+            for (int n = 0; n < nblk; ++n) {
+                if (live) live = warp_wait(smem_u32(&ctl->s_full[n]), 0u, &ctl->abort_flag, wc);
+                tc_fence_after();
+                if (live) for_half_block(ctl, n, g, pass_a(n));
+            }
+        } else {
+            for (int n = g; n < nblk; n += 2) {
+                if (live) live = __all_sync(0xffffffffu, P::wait_scores(ctl, wc, n));
+                if (live) P::for_each_chunk(ctl, n, pass_a(n));
+            }
+        }
+        {
+            RowOut& mine = rows[g * TILE + r];
+            mine.a0 = a0;
+            mine.a1 = a1;
+            mine.a2 = a2;
+            mine.a3 = a3;
+            mine.nallow = nallow;
+        }
+        epi_sync();
+        {
+            const RowOut& other = rows[(g ^ 1) * TILE + r];
+            top4_insert(other.a0, a0, a1, a2, a3);
+            top4_insert(other.a1, a0, a1, a2, a3);
+            top4_insert(other.a2, a0, a1, a2, a3);
+            top4_insert(other.a3, a0, a1, a2, a3);
+        }
+        // scores at or below t are outside the support: max - 2 (scaled), raised to the exact
+        // threshold of the row's four largest scores (any subset's threshold is at most tau)
+        const float t = fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
+
+        // ---------------- pass B: candidates s > m - 2 (scaled) into this warpgroup's partition
         float* pcv = cv + g * CAPW * TILE;
         uint16_t* pcj = cj + g * CAPW * TILE;
-        const int nblk = ctl->nblk;
-        bool live = true;
-        // the two warpgroups take blocks 2k and 2k+1, then swap bounds: the other warpgroup's bound
-        // is a lower bound of tau as well (any subset of a row), and exchanging it at fixed points
-        // keeps the candidate sets, hence the results, independent of timing
-        for (int k = 0; 2 * k < nblk; ++k) {
-            const int n = 2 * k + g;
-            if (n < nblk && live) live = P::wait_scores(ctl, wc, n);
-            if (n < nblk && live) {
-                const int j0 = (int)(blk_list[n] & ~FULL_BLOCK) * BLK;
-                const bool full = (blk_list[n] & FULL_BLOCK) && i < L;
-                P::for_each_chunk(ctl, n, [&](const float (&cur)[32], int c) {
-                    const int jc = j0 + c * 32;
-                    const uint32_t vm = full ? 0xffffffffu
-                                             : (jc < L && i < L) ? (bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
-                    st.nallow += __popc(vm);
-                    if (st.t == -INFINITY && vm != 0u) {
-                        // first allowed scores of this row: start from (max - 2) of the chunk
-                        float mx = -INFINITY;
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) mx = fmaxf(mx, ((vm >> q) & 1u) ? cur[q] : -INFINITY);
-                        st.t = mx - two_over_scale;
-                    }
-                    uint32_t hits = hit_bits(cur, st.t) & __brev(vm);
-                    if (hits) {
-                        stage_chunk(stage, threadIdx.x % NUM_EPI, cur);
-                        bool grew = false;
-                        do {
-                            const int q = __clz(hits);
-                            hits &= ~(0x80000000u >> q);
-                            grew |= push_candidate(st, staged(stage, threadIdx.x % NUM_EPI, q), jc + q, pcv, pcj, r, Vh);
-                        } while (hits);
-                        // early in the row the bound moves fast: tighten it after every chunk of the
-                        // first block, later once per block pair (below)
-                        if (grew && k == 0) st.t = fmaxf(st.t, top4_bound(st.a0, st.a1, st.a2, st.a3, c4));
-                    }
-                });
+        int nc = 0;
+        auto pass_b = [&](int e) {
+            const int j0 = (int)(blk_list[e] & ~FULL_BLOCK) * BLK;
+            return [&, e, j0](const float (&cur)[32], int c) {
+                const int jc = j0 + c * 32;
+                uint32_t hits = hit_bits(cur, t) & __brev(allowed(e, jc));
+                if (hits) {
+                    stage_chunk(stage, slot, cur);
+                    do {
+                        const int q = __clz(hits);
+                        hits &= ~(0x80000000u >> q);
+                        if (nc < CAPW) {
+                            pcv[nc * TILE + r] = staged(stage, slot, q);
+                            pcj[nc * TILE + r] = (uint16_t)(jc + q);
+                            if (!resident) prefetch_l2(Vh + (size_t)(jc + q) * HEAD_DIM);
+                        }
+                        ++nc;
+                    } while (hits);
+                }
+            };
+        };
+        if (resident) {
+            tc_fence_after();
+            if (live) {
+                for (int n = 0; n < nblk; ++n) for_half_block(ctl, n, g, pass_b(n));
             }
-            if (k > 0) st.t = fmaxf(st.t, top4_bound(st.a0, st.a1, st.a2, st.a3, c4));
-            float* tx = tshare + (k & 1) * 2 * TILE;
-            tx[g * TILE + r] = st.t;
-            epi_pair_sync();
-            st.t = fmaxf(st.t, tx[(g ^ 1) * TILE + r]);
+        } else {
+            for (int n = nblk + ((g ^ nblk) & 1); n < njobs; n += 2) {
+                if (live) live = __all_sync(0xffffffffu, P::wait_scores(ctl, wc, n));
+                if (live) P::for_each_chunk(ctl, n, pass_b(n - nblk));
+            }
         }
-        rows[g * TILE + r] = RowOut{st.a0, st.a1, st.a2, st.a3, st.t, st.n, st.nallow, st.ovf};
+        rows[g * TILE + r].n = min(nc, CAPW);
+        rows[g * TILE + r].ovf = nc > CAPW ? 1 : 0;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const bool aborted = P::aborted(ctl);
+    const bool v_staged = resident && !aborted;
+
+    // V blocks of a resident tile into the (now idle) ring, overlapping phase 2
+    if (warp == WARP_PRODUCER && lane == 0 && v_staged) {
+        mbar_arrive_expect_tx(smem_u32(vbar), (uint32_t)(nblk * BLK_BYTES));
+        for (int s = 0; s < nblk; ++s)
+            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), &map_v, 0, (int)(blk_list[s] & ~FULL_BLOCK) * BLK, bh,
+                        smem_u32(vbar));
+    }
 
     // ---------------- phase 2: tau per row, two threads per row (one per partition)
     if (!aborted && tid < NUM_EPI) {
@@ -544,70 +685,18 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const int i = i0 + r;
         const RowOut s0 = rows[r], s1 = rows[TILE + r];
         const int nallow = s0.nallow + s1.nallow;
-        const int ovf = s0.ovf | s1.ovf;
-        // merged bound: the four largest scores of the whole row
-        float a0 = s0.a0, a1 = s0.a1, a2 = s0.a2, a3 = s0.a3;
-        top4_insert(s1.a0, a0, a1, a2, a3);
-        top4_insert(s1.a1, a0, a1, a2, a3);
-        top4_insert(s1.a2, a0, a1, a2, a3);
-        top4_insert(s1.a3, a0, a1, a2, a3);
-        const float tf = fmaxf(fmaxf(s0.t, s1.t), top4_bound(a0, a1, a2, a3, c4));
-        const float ms = scale * a0;  // scaled row max
-        int mode = 0;                 // 0: registers, 1: slow path, 2: fallback, 3: no key
+        const float ms = scale * fmaxf(s0.a0, s1.a0);  // scaled row max
+        int mode = 0;                                 // 0: solved here, 2: fallback, 3: no key
         if (i >= L || nallow == 0) mode = 3;
-        else if (ovf) mode = 2;
-        int nh = h == 0 ? s0.n : s1.n;
+        else if (s0.ovf | s1.ovf) mode = 2;
+        const int nh = mode == 0 ? (h == 0 ? s0.n : s1.n) : 0;
         float* pcv = cv + h * CAPW * TILE;
         uint16_t* pcj = cj + h * CAPW * TILE;
-        if (mode == 0 && nh > REG_CAND) nh = compact_list(tf, nh, pcv, pcj, r);
-        // every lane takes part in the pair shuffles below (rows of one warp may differ in mode)
-        const int nh_other = __shfl_xor_sync(0xffffffffu, nh, 1);
-        if (mode == 0 && (nh > REG_CAND || nh_other > REG_CAND)) mode = 1;
-        float x[REG_CAND];
-#pragma unroll
-        for (int k = 0; k < REG_CAND; ++k) {
-            const float v = (mode == 0 && k < nh) ? pcv[k * TILE + r] : -INFINITY;
-            x[k] = v > tf ? fmaf(scale, v, -ms) : -INFINITY;
-        }
-        float lo = -2.f, hi = -2.f / sqrtf((float)max(nallow, 1));
-        for (int it = 0; it < 25; ++it) {
-            const float mid = 0.5f * (lo + hi);
-            float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
-#pragma unroll
-            for (int k = 0; k < REG_CAND; k += 4) {
-                const float d0 = fmaxf(x[k] - mid, 0.f), d1 = fmaxf(x[k + 1] - mid, 0.f);
-                const float d2 = fmaxf(x[k + 2] - mid, 0.f), d3 = fmaxf(x[k + 3] - mid, 0.f);
-                g0 = fmaf(d0, d0, g0);
-                g1 = fmaf(d1, d1, g1);
-                g2 = fmaf(d2, d2, g2);
-                g3 = fmaf(d3, d3, g3);
-            }
-            float gs = (g0 + g1) + (g2 + g3);
-            gs += __shfl_xor_sync(0xffffffffu, gs, 1);
-            if (0.25f * gs > 1.f) lo = mid;
-            else hi = mid;
-        }
-        // support fixed by the final bracket: closed-form root of sum_S (x - tau)^2 = 4
-        const float mid = 0.5f * (lo + hi);
-        float K = 0.f, S1 = 0.f, S2 = 0.f;
-#pragma unroll
-        for (int k = 0; k < REG_CAND; ++k) {
-            if (x[k] > mid) {
-                K += 1.f;
-                S1 += x[k];
-                S2 = fmaf(x[k], x[k], S2);
-            }
-        }
-        K += __shfl_xor_sync(0xffffffffu, K, 1);
-        S1 += __shfl_xor_sync(0xffffffffu, S1, 1);
-        S2 += __shfl_xor_sync(0xffffffffu, S2, 1);
-        float tau_x = mid;
-        if (K > 0.f) {
-            const float mu = S1 / K;
-            const float var = fmaxf(S2 / K - mu * mu, 0.f);
-            const float tc = mu - sqrtf(fmaxf(4.f / K - var, 0.f));
-            if (tc >= lo && tc <= hi) tau_x = tc;
-        }
+        // every lane takes part in the pair shuffles (rows of one warp may differ in mode)
+        const int nmax = __reduce_max_sync(0xffffffffu, nh);
+        const float tau_x = nmax <= 16   ? solve_tau<16>(pcv, r, nh, scale, ms, nallow)
+                            : nmax <= 32 ? solve_tau<32>(pcv, r, nh, scale, ms, nallow)
+                                         : solve_tau<CAPW>(pcv, r, nh, scale, ms, nallow);
         if (mode == 0) {
             // this thread's partition of the support: cv <- p_ij, cj <- j (in place)
             int sn = 0;
@@ -622,15 +711,6 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             }
             supp_cnt[h * TILE + r] = sn;
             if (h == 0) out.tau[(size_t)bh * L + i] = ms + tau_x;
-        } else if (mode == 1) {
-            if (h == 0) {
-                int sn = 0;
-                // counts after this pair's compaction (h = 0 holds partition 0, its partner partition 1)
-                const float tx = solve_row_smem(cv, cj, scratch, r, nh, nh_other, scale, ms, nallow, &sn);
-                supp_cnt[r] = sn;
-                supp_cnt[TILE + r] = 0;
-                out.tau[(size_t)bh * L + i] = ms + tx;
-            }
         } else if (mode == 2) {
             if (h == 0) atomicOr(&redo[r >> 5], 1u << (r & 31));
             supp_cnt[h * TILE + r] = 0;
@@ -638,40 +718,32 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             supp_cnt[h * TILE + r] = 0;
             if (h == 0 && i < L) out.tau[(size_t)bh * L + i] = INFINITY;  // no allowed key: O_i = 0
         }
-        __syncwarp();  // the slow path's counts (written by h = 0) are read by both threads of the pair
+        __syncwarp();
         if (out.save.row_cnt) save_row_support(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, i, L);
     }
     __syncthreads();
 
     // ---------------- phase 3: O_i = sum_j p_ij V_j, one warp per row, two rows in flight
-    if (!aborted) {
+    bool v_ok = true;
+    if (v_staged) v_ok = warp_wait(smem_u32(vbar), 0u, &ctl->abort_flag, wc);
+    if (!aborted && v_ok) {
         for (int ra = warp; ra < TILE; ra += 2 * NUM_WARPS) {
-            const int rb = ra + NUM_WARPS;
-            const bool okb = rb < TILE;
-            float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+            const int rb = ra + NUM_WARPS < TILE ? ra + NUM_WARPS : -1;
+            float oa[8], ob[8];
             const int na0 = supp_cnt[ra], na1 = supp_cnt[TILE + ra];
-            const int nb0 = okb ? supp_cnt[rb] : 0, nb1 = okb ? supp_cnt[TILE + rb] : 0;
-            gather_accumulate2(Vh, cj, cv, ra, 0, na0, okb ? rb : ra, 0, nb0, lane, a0, a1, b0, b1);
-            gather_accumulate2(Vh, cj, cv, ra, CAPW, CAPW + na1, okb ? rb : ra, CAPW, CAPW + nb1, lane, a0, a1, b0, b1);
-            for (int q = 0; q < 2; ++q) {
-                const int rr = q == 0 ? ra : rb;
-                const int i = i0 + rr;
-                if ((q == 1 && !okb) || i >= L || ((redo[rr >> 5] >> (rr & 31)) & 1u)) continue;
-                const float o0 = q == 0 ? a0 : b0, o1 = q == 0 ? a1 : b1;
-                const size_t oi = ((size_t)bh * L + i) * HEAD_DIM + 2 * lane;
-                if (out.out_f32) {
-                    *reinterpret_cast<float2*>(reinterpret_cast<float*>(out.O) + oi) = make_float2(o0, o1);
-                } else {
-                    *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out.O) + oi) =
-                        __floats2bfloat162_rn(o0, o1);
-                }
-            }
+            const int nb0 = rb >= 0 ? supp_cnt[rb] : 0, nb1 = rb >= 0 ? supp_cnt[TILE + rb] : 0;
+            if (v_staged) gather_rows<true>(smem_b, vslot, Vh, cj, cv, ra, na0, na1, rb, nb0, nb1, lane, oa, ob);
+            else gather_rows<false>(smem_b, vslot, Vh, cj, cv, ra, na0, na1, rb, nb0, nb1, lane, oa, ob);
+            const int ia = i0 + ra, ib = i0 + rb;
+            if (ia < L && !((redo[ra >> 5] >> (ra & 31)) & 1u)) store_o_row(out, (size_t)bh * L + ia, lane, oa);
+            if (rb >= 0 && ib < L && !((redo[rb >> 5] >> (rb & 31)) & 1u)) store_o_row(out, (size_t)bh * L + ib, lane, ob);
         }
     }
+    if (v_staged && warp == WARP_PRODUCER && lane == 0 && !v_ok) wait_drain(smem_u32(vbar), 0u);
     __syncthreads();
 
     // ---------------- phase 4: exact redo of overflowed rows
-    if (!aborted) {
+    if (!P::aborted(ctl)) {
         for (int wd = 0; wd < TILE / 32; ++wd) {
             uint32_t mask = redo[wd];  // uniform across the CTA
             while (mask) {
@@ -698,15 +770,17 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 size_t fwd_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream) {
-    CUtensorMap mq, mk;
+    CUtensorMap mq, mk, mv;
     cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L, TILE);
     if (e != cudaSuccess) return e;
     e = make_tile_map(&mk, a.K, a.B * a.H, a.L, BLK);
     if (e != cudaSuccess) return e;
+    e = make_tile_map(&mv, a.V, a.B * a.H, a.L, BLK);
+    if (e != cudaSuccess) return e;
     e = ensure_smem_attr(reinterpret_cast<const void*>(entmax_fwd_kernel), SMEM_BYTES, 0);
     if (e != cudaSuccess) return e;
     dim3 grid((a.L + TILE - 1) / TILE, a.B * a.H);
-    entmax_fwd_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, a, o);
+    entmax_fwd_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, a, o);
     return cudaGetLastError();
 }
 
