@@ -1,0 +1,69 @@
+"""Host-side logic of bench.py's multi-GPU replicas, on CPU with two gloo ranks.
+
+The operation has no exchange step, so N GPUs run N independent replicas; the only cross-rank work
+is the barrier around the timed region and the max of the step time over ranks, which these tests
+exercise without a GPU.
+"""
+import os
+import socket
+import sys
+from pathlib import Path
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, out_dir: str):
+    sys.path.insert(0, str(ROOT))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+
+        bench.dist_barrier(world)
+        # each rank reports its own step time; every rank must see the slowest one
+        mine = 10.0 + 5.0 * rank
+        worst = bench.dist_max(mine, world, torch.device("cpu"))
+        value = bench.aggregate_value(1e12, world, worst)
+        Path(out_dir, "r%d.txt" % rank).write_text("%r %r" % (worst, value))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_max_over_ranks_and_whole_job_value(tmp_path, world):
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, str(tmp_path))) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = [Path(tmp_path, "r%d.txt" % r).read_text().split() for r in range(world)]
+    slowest = 10.0 + 5.0 * (world - 1)
+    for worst, value in got:
+        assert float(worst) == slowest
+        # whole-job throughput: every rank's work over the slowest rank's time (TFLOP/s)
+        assert abs(float(value) - world * 1e12 / (slowest * 1e-3) / 1e12) < 1e-9
+
+
+def test_single_process_helpers_need_no_process_group():
+    sys.path.insert(0, str(ROOT))
+    import bench
+
+    bench.dist_barrier(1)
+    assert bench.dist_max(3.5, 1, torch.device("cpu")) == 3.5
+    assert bench.aggregate_value(2e12, 1, 1000.0) == pytest.approx(2.0)
