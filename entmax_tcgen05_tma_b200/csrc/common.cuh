@@ -148,7 +148,9 @@ struct Pipe {
 
     static __device__ __forceinline__ bool aborted(const Ctl* ctl) { return flag_set(&ctl->abort_flag); }
 
-    static __device__ __forceinline__ void init(Ctl* ctl) {
+    // empty_arrivals: warps that release each score buffer (4: the owning warpgroup; NUM_EPI / 32
+    // when every epilogue warp reads a share of every block).
+    static __device__ __forceinline__ void init(Ctl* ctl, uint32_t empty_arrivals = 4) {
         mbar_init(smem_u32(&ctl->full_a), 1);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(smem_u32(&ctl->full_b[s]), 1);
@@ -156,7 +158,7 @@ struct Pipe {
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(smem_u32(&ctl->s_full[b]), 1);
-            mbar_init(smem_u32(&ctl->s_empty[b]), 4);  // one arrival per warp of the owning warpgroup
+            mbar_init(smem_u32(&ctl->s_empty[b]), empty_arrivals);
         }
         ctl->abort_flag = 0;
         fence_barrier_init();
@@ -312,6 +314,24 @@ struct Pipe {
 };
 
 // ------------------------------------------------------------ hit filtering
+// Three-input maximum (one sm_100 instruction).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Maximum of a 32-value chunk: a tree of three-input maxima (16 instructions, depth 4).
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+    float m[11];
+#pragma unroll
+    for (int k = 0; k < 10; ++k) m[k] = fmax3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
+    m[10] = fmaxf(v[30], v[31]);
+    const float a = fmax3(m[0], m[1], m[2]), b = fmax3(m[3], m[4], m[5]), c = fmax3(m[6], m[7], m[8]);
+    const float d = fmaxf(m[9], m[10]);
+    return fmaxf(fmax3(a, b, c), d);
+}
+
 // Bit (31 - k) of the result is set iff v[k] > t: the sign bit of t - v[k] funnel-shifted into
 // four independent 8-bit chains (two instructions per value, no branches).
 __device__ __forceinline__ uint32_t hit_bits(const float (&v)[32], float t) {

@@ -8,7 +8,8 @@
 //
 // One CTA per 128-query tile.  Phases:
 //  1. Score passes (common.cuh pipeline): QK^T on tcgen05, 128 keys per block, fp32 scores in TMEM.
-//     Pass A reduces every row to its maximum m_i over the allowed keys.  Pass B keeps the row's
+//     Pass A reduces every row to its maximum m_i over the allowed keys and the four largest
+//     maxima of its 32-key chunks (branch-free: three-input max trees).  Pass B keeps the row's
 //     *candidates*, the scores above m_i - 2 (scaled units) -- the bisection's lower bracket end,
 //     so the support is a subset of them -- as (score, key) lists in shared memory.  When the
 //     tile's key blocks fit in TMEM at once (at most four blocks: L <= 512, or a causal window)
@@ -569,30 +570,29 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         };
         bool live = true;
 
-        // ---------------- pass A: four largest scores and allowed-key count
-        // Only scores above th = max(a3, a0 - 2/scale) can change the top four in a way that matters:
-        // scores at or below a0 - 2/scale never enter the support, so leaving them out of the top
-        // four only weakens bounds that max - 2 already dominates.
+        // ---------------- pass A: row max, the four largest 32-key chunk maxima, allowed-key count
+        // Branch-free: a chunk costs a tree of three-input maxima and a min/max insertion network.
+        // The chunk maxima are scores of the row, so the exact threshold of the four largest is a
+        // lower bound of tau (a subset's threshold never exceeds the row's).
         float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-        float th = -INFINITY;
         int nallow = 0;
         const int slot = threadIdx.x % NUM_EPI;
         auto pass_a = [&](int n) {
             const int j0 = (int)(blk_list[n] & ~FULL_BLOCK) * BLK;
             return [&, n, j0](const float (&cur)[32], int c) {
                 const uint32_t vm = allowed(n, j0 + c * 32);
-                nallow += __popc(vm);
-                if (a0 == -INFINITY && vm != 0u) th = masked_max(cur, vm) - two_over_scale;
-                uint32_t hits = hit_bits(cur, th) & __brev(vm);
-                if (hits) {
-                    stage_chunk(stage, slot, cur);
-                    do {
-                        const int q = __clz(hits);
-                        hits &= ~(0x80000000u >> q);
-                        top4_insert(staged(stage, slot, q), a0, a1, a2, a3);
-                    } while (hits);
-                    th = fmaxf(a3, a0 - two_over_scale);
+                float cm;
+                if (vm == 0xffffffffu) {
+                    nallow += 32;
+                    cm = max32(cur);
+                } else {
+                    nallow += __popc(vm);
+                    cm = masked_max(cur, vm);
                 }
+                a3 = fmaxf(a3, fminf(a2, cm));
+                a2 = fmaxf(a2, fminf(a1, cm));
+                a1 = fmaxf(a1, fminf(a0, cm));
+                a0 = fmaxf(a0, cm);
             };
         };
         if (resident) {
@@ -624,7 +624,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             top4_insert(other.a3, a0, a1, a2, a3);
         }
         // scores at or below t are outside the support: max - 2 (scaled), raised to the exact
-        // threshold of the row's four largest scores (any subset's threshold is at most tau)
+        // threshold of the row's four largest chunk maxima (any subset's threshold is at most tau)
         const float t = fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
 
         // ---------------- pass B: candidates s > m - 2 (scaled) into this warpgroup's partition
