@@ -162,15 +162,15 @@ __device__ __forceinline__ void for_half_block(const PipeCtl* ctl, int n, int ha
 
 // tau of one row in shifted scaled units (x = scale * S - scale * m, so the row max is 0), from the
 // candidates of the two partitions held by a lane pair (NC registers each, -inf where unused).
-// Bisection of [-2, -2/sqrt(n)] (g(-2) >= 1 from the max alone, g(-2/sqrt n) <= 1); every four
+// Bisection of [lo, hi], a sub-bracket of [-2, -2/sqrt(n)] that still holds the root (the caller's
+// bounds: g(lo) >= 1, g(hi) <= 1; g(-2) >= 1 from the max alone, g(-2/sqrt n) <= 1); every four
 // halvings the warp stops if no lane pair has a candidate strictly inside its bracket: the support
 // is then fixed and the closed-form root on it is exact.  Returns tau_x.
 template <int NC>
-__device__ __forceinline__ float solve_tau(const float* pcv, int r, int nh, float scale, float ms, int nallow) {
+__device__ __forceinline__ float solve_tau(const float* pcv, int r, int nh, float scale, float ms, float lo, float hi) {
     float x[NC];
 #pragma unroll
     for (int k = 0; k < NC; ++k) x[k] = k < nh ? fmaf(scale, pcv[k * TILE + r], -ms) : -INFINITY;
-    float lo = -2.f, hi = -2.f / sqrtf((float)max(nallow, 1));
     bool settled = false;
     for (int it = 0; it < 25; ++it) {
         const float mid = 0.5f * (lo + hi);
@@ -224,91 +224,12 @@ __device__ __forceinline__ float solve_tau(const float* pcv, int r, int nh, floa
     return tau_x;
 }
 
-// Support entry e of row r (partition 0 holds entries [0, n0), partition 1 the rest): key j and
-// weight p_ij from the [slot][TILE] lists.
-__device__ __forceinline__ void support_entry(const uint16_t* cj, const float* cw, int r, int n0, int e, int& j,
-                                              float& w) {
-    const int sl = e < n0 ? e : CAPW + (e - n0);
-    j = cj[sl * TILE + r];
-    w = cw[sl * TILE + r];
-}
-
 __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4& x) {
     const uint32_t u[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         acc[2 * k] = fmaf(w, bf16lo(u[k]), acc[2 * k]);
         acc[2 * k + 1] = fmaf(w, bf16hi(u[k]), acc[2 * k + 1]);
-    }
-}
-
-// O rows ra and rb (rb < 0: none) = sum over their support of p_ij V_j, one warp: lane = 8 grp + sub,
-// group grp takes every fourth entry, lane sub the 16-byte column chunk (dimensions 8 sub .. 8 sub + 7).
-// V rows come from the shared-memory ring (kSmem: 128-byte swizzled blocks of BLK keys, block kb in
-// slot vslot[kb]) or from global memory.  The four groups' sums are reduced with shuffles; the
-// result is valid in lanes 0..7 (acc index = dimension - 8 sub).
-template <bool kSmem>
-__device__ __forceinline__ void gather_rows(const uint8_t* vring, const uint8_t* vslot, const __nv_bfloat16* Vh,
-                                            const uint16_t* cj, const float* cw, int ra, int na0, int na1, int rb,
-                                            int nb0, int nb1, int lane, float (&oa)[8], float (&ob)[8]) {
-    const int grp = lane >> 3, sub = lane & 7;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) oa[k] = ob[k] = 0.f;
-    const int na = na0 + na1, nb = rb >= 0 ? nb0 + nb1 : 0;
-    auto load = [&](int j) -> uint4 {
-        if (kSmem) {
-            const uint32_t row = (uint32_t)j & (BLK - 1);
-            const uint8_t* p = vring + vslot[j / BLK] * BLK_BYTES + row * 128u + (((uint32_t)sub ^ (row & 7u)) << 4);
-            return *reinterpret_cast<const uint4*>(p);
-        } else {
-            return __ldg(reinterpret_cast<const uint4*>(Vh + (size_t)j * HEAD_DIM) + sub);
-        }
-    };
-    for (int e = grp; e < na || e < nb; e += 8) {
-        uint4 x[4];
-        float w[4];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int ea = e + 4 * u;
-            int j;
-            w[u] = w[2 + u] = 0.f;
-            x[u] = x[2 + u] = make_uint4(0u, 0u, 0u, 0u);
-            if (ea < na) {
-                support_entry(cj, cw, ra, na0, ea, j, w[u]);
-                x[u] = load(j);
-            }
-            if (ea < nb) {
-                support_entry(cj, cw, rb, nb0, ea, j, w[2 + u]);
-                x[2 + u] = load(j);
-            }
-        }
-        fma_bf16x8(oa, w[0], x[0]);
-        fma_bf16x8(oa, w[1], x[1]);
-        fma_bf16x8(ob, w[2], x[2]);
-        fma_bf16x8(ob, w[3], x[3]);
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        oa[k] += __shfl_xor_sync(0xffffffffu, oa[k], 8);
-        ob[k] += __shfl_xor_sync(0xffffffffu, ob[k], 8);
-        oa[k] += __shfl_xor_sync(0xffffffffu, oa[k], 16);
-        ob[k] += __shfl_xor_sync(0xffffffffu, ob[k], 16);
-    }
-}
-
-// Lanes 0..7 store their 8 dimensions of O row i.
-__device__ __forceinline__ void store_o_row(const FwdOut& out, size_t row, int lane, const float (&o)[8]) {
-    if (lane >= 8) return;
-    const size_t oi = row * HEAD_DIM + 8 * lane;
-    if (out.out_f32) {
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out.O) + oi);
-        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
-    } else {
-        __nv_bfloat162 h[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) h[k] = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
-        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out.O) + oi) = *reinterpret_cast<const uint4*>(h);
     }
 }
 
@@ -693,10 +614,22 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         float* pcv = cv + h * CAPW * TILE;
         uint16_t* pcj = cj + h * CAPW * TILE;
         // every lane takes part in the pair shuffles (rows of one warp may differ in mode)
+        // Bracket (shifted scaled units, row max = 0): lo = the bound the candidates were cut at (the
+        // exact threshold of the four largest chunk maxima, or max - 2), g(lo) >= g(tau) = 1; hi =
+        // -2/sqrt(k) with k = the candidates listed, a superset of the support, so
+        // g(hi) <= k (1/sqrt k)^2 = 1.  Both lie inside the pages' bracket [-2, -2/sqrt(n)].
+        float b0 = s0.a0, b1 = s0.a1, b2 = s0.a2, b3 = s0.a3;
+        top4_insert(s1.a0, b0, b1, b2, b3);
+        top4_insert(s1.a1, b0, b1, b2, b3);
+        top4_insert(s1.a2, b0, b1, b2, b3);
+        top4_insert(s1.a3, b0, b1, b2, b3);
+        const float t_cut = fmaxf(b0 - two_over_scale, top4_bound(b0, b1, b2, b3, c4));
+        const float hi = -2.f / sqrtf((float)max(s0.n + s1.n, 1));
+        const float lo = fminf(fmaxf(-2.f, fmaf(scale, t_cut, -ms)), hi);
         const int nmax = __reduce_max_sync(0xffffffffu, nh);
-        const float tau_x = nmax <= 16   ? solve_tau<16>(pcv, r, nh, scale, ms, nallow)
-                            : nmax <= 32 ? solve_tau<32>(pcv, r, nh, scale, ms, nallow)
-                                         : solve_tau<CAPW>(pcv, r, nh, scale, ms, nallow);
+        const float tau_x = nmax <= 16   ? solve_tau<16>(pcv, r, nh, scale, ms, lo, hi)
+                            : nmax <= 32 ? solve_tau<32>(pcv, r, nh, scale, ms, lo, hi)
+                                         : solve_tau<CAPW>(pcv, r, nh, scale, ms, lo, hi);
         if (mode == 0) {
             // this thread's partition of the support: cv <- p_ij, cj <- j (in place)
             int sn = 0;
@@ -720,27 +653,61 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         __syncwarp();
         if (out.save.row_cnt) save_row_support(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, i, L);
-    }
-    __syncthreads();
 
-    // ---------------- phase 3: O_i = sum_j p_ij V_j, one warp per row, two rows in flight
-    bool v_ok = true;
-    if (v_staged) v_ok = warp_wait(smem_u32(vbar), 0u, &ctl->abort_flag, wc);
-    if (!aborted && v_ok) {
-        for (int ra = warp; ra < TILE; ra += 2 * NUM_WARPS) {
-            const int rb = ra + NUM_WARPS < TILE ? ra + NUM_WARPS : -1;
-            float oa[8], ob[8];
-            const int na0 = supp_cnt[ra], na1 = supp_cnt[TILE + ra];
-            const int nb0 = rb >= 0 ? supp_cnt[rb] : 0, nb1 = rb >= 0 ? supp_cnt[TILE + rb] : 0;
-            if (v_staged) gather_rows<true>(smem_b, vslot, Vh, cj, cv, ra, na0, na1, rb, nb0, nb1, lane, oa, ob);
-            else gather_rows<false>(smem_b, vslot, Vh, cj, cv, ra, na0, na1, rb, nb0, nb1, lane, oa, ob);
-            const int ia = i0 + ra, ib = i0 + rb;
-            if (ia < L && !((redo[ra >> 5] >> (ra & 31)) & 1u)) store_o_row(out, (size_t)bh * L + ia, lane, oa);
-            if (rb >= 0 && ib < L && !((redo[rb >> 5] >> (rb & 31)) & 1u)) store_o_row(out, (size_t)bh * L + ib, lane, ob);
+        // ---------------- phase 3: O_i = sum_j p_ij V_j over the row's whole support (both
+        // partitions); thread h of the pair accumulates dimensions [32 h, 32 h + 32) in registers
+        const bool v_ok = !v_staged || warp_wait(smem_u32(vbar), 0u, &ctl->abort_flag, wc);
+        if (v_ok && mode != 2 && i < L) {
+            const int n0 = supp_cnt[r], n1 = supp_cnt[TILE + r];
+            float acc[4][8];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[c][k] = 0.f;
+            for (int e = 0; e < n0 + n1; ++e) {
+                const int sl = e < n0 ? e : CAPW + (e - n0);
+                const int j = cj[sl * TILE + r];
+                const float p = cv[sl * TILE + r];
+                uint4 x[4];
+                if (v_staged) {
+                    // 128-byte swizzled V block in ring slot vslot[j / BLK]: 16-byte chunk c of row
+                    // `row` sits at chunk position c ^ (row & 7)
+                    const uint32_t row = (uint32_t)j & (BLK - 1);
+                    const uint8_t* base = smem_b + vslot[j / BLK] * BLK_BYTES + row * 128u;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        x[c] = *reinterpret_cast<const uint4*>(base + ((((uint32_t)(4 * h + c)) ^ (row & 7u)) << 4));
+                } else {
+                    const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)j * HEAD_DIM) + 4 * h;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) x[c] = __ldg(src + c);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) fma_bf16x8(acc[c], p, x[c]);
+            }
+            const size_t oi = ((size_t)bh * L + i) * HEAD_DIM + 32 * h;
+            if (out.out_f32) {
+                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out.O) + oi);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    dst[2 * c] = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+                    dst[2 * c + 1] = make_float4(acc[c][4], acc[c][5], acc[c][6], acc[c][7]);
+                }
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out.O) + oi);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    __nv_bfloat162 hv[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) hv[k] = __floats2bfloat162_rn(acc[c][2 * k], acc[c][2 * k + 1]);
+                    dst[c] = *reinterpret_cast<const uint4*>(hv);
+                }
+            }
         }
     }
-    if (v_staged && warp == WARP_PRODUCER && lane == 0 && !v_ok) wait_drain(smem_u32(vbar), 0u);
     __syncthreads();
+    // a V wait that gave up raised the abort flag: the staged copies must land before exit
+    if (v_staged && warp == WARP_PRODUCER && lane == 0 && P::aborted(ctl)) wait_drain(smem_u32(vbar), 0u);
 
     // ---------------- phase 4: exact redo of overflowed rows
     if (!P::aborted(ctl)) {
