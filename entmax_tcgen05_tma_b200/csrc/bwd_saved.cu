@@ -8,10 +8,11 @@
 // so no QK^T is formed again: the work is proportional to the number of support entries.
 //
 //  1. key_scan:   per head, exclusive scan of the per-key support counts -> bucket offsets.
-//  2. rows:       one warp per query row.  dA_ij with one support entry per lane (each lane reads a
-//                 whole V row, 8 x 16-byte loads), u_i, dS_ij, dQ_i (lanes over dimensions), and the
+//  2. rows:       four query rows per warp, eight lanes per row (each lane owns eight dimensions, so
+//                 a gathered row is one 16-byte load per lane): dA_ij, u_i, dS_ij, dQ_i, and the
 //                 entries (i, sp_ij, dS_ij) scattered into per-key buckets.
-//  3. keys:       one warp per key: dK_j and dV_j from its bucket (gathered Q_i, dO_i rows).
+//  3. keys:       four keys per warp, eight lanes per key: dK_j and dV_j from its bucket (gathered
+//                 Q_i, dO_i rows).
 //  4. unsaved:    rows whose support was not saved (redone on CUDA cores in the forward, or with more
 //                 than SAVE_CAP entries) are recomputed exactly by a whole CTA each; their dK/dV terms
 //                 are added with atomics after step 3.
@@ -26,28 +27,6 @@ namespace entmax {
 namespace {
 
 constexpr int ROW_WARPS = 8;  // warps per CTA of the rows / keys kernels
-
-__device__ __forceinline__ float dot64_smem(const float* g, const __nv_bfloat16* row) {
-    const uint4* p = reinterpret_cast<const uint4*>(row);
-    uint4 w[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) w[c] = __ldg(p + c);
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const float4 ga = reinterpret_cast<const float4*>(g)[2 * c];
-        const float4 gb = reinterpret_cast<const float4*>(g)[2 * c + 1];
-        acc0 = fmaf(ga.x, bf16lo(w[c].x), acc0);
-        acc1 = fmaf(ga.y, bf16hi(w[c].x), acc1);
-        acc0 = fmaf(ga.z, bf16lo(w[c].y), acc0);
-        acc1 = fmaf(ga.w, bf16hi(w[c].y), acc1);
-        acc0 = fmaf(gb.x, bf16lo(w[c].z), acc0);
-        acc1 = fmaf(gb.y, bf16hi(w[c].z), acc1);
-        acc0 = fmaf(gb.z, bf16lo(w[c].w), acc0);
-        acc1 = fmaf(gb.w, bf16hi(w[c].w), acc1);
-    }
-    return acc0 + acc1;
-}
 
 __global__ void __launch_bounds__(1024) key_scan_kernel(const int* __restrict__ key_cnt, int* __restrict__ key_off,
                                                         int* __restrict__ key_cur, int L) {
@@ -85,130 +64,207 @@ __global__ void __launch_bounds__(1024) key_scan_kernel(const int* __restrict__ 
     }
 }
 
+constexpr int RPW = 4;  // rows (keys) per warp: eight lanes each, lane s of a group owns dimensions 8s .. 8s+7
+
+__device__ __forceinline__ void unpack8(const uint4& x, float (&v)[8]) {
+    const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        v[2 * k] = bf16lo(u[k]);
+        v[2 * k + 1] = bf16hi(u[k]);
+    }
+}
+
+// Sum over the eight lanes of a group (lanes 8q .. 8q + 7).
+__device__ __forceinline__ float group8_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    return v;
+}
+
+// Four query rows per warp, eight lanes per row.  The row's saved list is staged in shared memory;
+// dA_e = dO_i . V_je takes one 16-byte load of V_je per lane and a three-step group reduction, two
+// entries in flight; then u_i, dS_e, the bucket entries, and dQ_i (one 16-byte load of K_je per lane
+// per entry).
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
-    __shared__ __align__(16) float gsm[ROW_WARPS][HEAD_DIM];
+    __shared__ uint16_t lj[ROW_WARPS][RPW][SAVE_CAP];
+    __shared__ float lsp[ROW_WARPS][RPW][SAVE_CAP];
+    __shared__ float lds[ROW_WARPS][RPW][SAVE_CAP];  // dA, then dS
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = lane >> 3, sd = lane & 7;
     const int L = a.L;
     const long long R = (long long)a.B * a.H * L;
     const size_t cap = (size_t)L * SAVE_CAP;
     const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(a.K);
     const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(a.V);
     const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
-    float* gs = gsm[warp];
-    for (long long row = (long long)blockIdx.x * ROW_WARPS + warp; row < R; row += (long long)gridDim.x * ROW_WARPS) {
-        const int cnt = sv.row_cnt[row];
-        if (cnt < 0) continue;  // not saved: the exact pass handles this row
-        const long long bh = row / L;
+    uint16_t* mj = lj[warp][q];
+    float* msp = lsp[warp][q];
+    float* mds = lds[warp][q];
+    for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
+        const long long row = grp * RPW + q;
+        const int cnt = row < R ? sv.row_cnt[row] : -1;  // -1: no row, or not saved (the exact pass handles it)
+        const long long bh = row < R ? row / L : 0;
         const int i = (int)(row - bh * L);
         const size_t head = (size_t)bh * L * HEAD_DIM;
-        const uint32_t gw = reinterpret_cast<const uint32_t*>(dO + (size_t)row * HEAD_DIM)[lane];
-        gs[2 * lane] = bf16lo(gw);
-        gs[2 * lane + 1] = bf16hi(gw);
+        for (int e = sd; e < cnt; e += 8) {
+            mj[e] = sv.row_j[(size_t)row * SAVE_CAP + e];
+            msp[e] = sv.row_sp[(size_t)row * SAVE_CAP + e];
+        }
+        float g[8];
+        {
+            const uint4 x = cnt >= 0 ? __ldg(reinterpret_cast<const uint4*>(dO + (size_t)row * HEAD_DIM) + sd)
+                                     : make_uint4(0u, 0u, 0u, 0u);
+            unpack8(x, g);
+        }
+        const int maxc = __reduce_max_sync(0xffffffffu, max(cnt, 0));
         __syncwarp();
-        // dA_ij: one support entry per lane
-        int jj[2] = {0, 0};
-        float sp[2] = {0.f, 0.f}, dA[2] = {0.f, 0.f};
+        // dA_e, two entries in flight
+        for (int e = 0; e < maxc; e += 2) {
+            uint4 x[2];
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            if (b * 32 < cnt) {  // uniform
-                const int e = b * 32 + lane;
-                if (e < cnt) {
-                    jj[b] = sv.row_j[(size_t)row * SAVE_CAP + e];
-                    sp[b] = sv.row_sp[(size_t)row * SAVE_CAP + e];
-                    dA[b] = dot64_smem(gs, V + head + (size_t)jj[b] * HEAD_DIM);
-                }
+            for (int u = 0; u < 2; ++u) {
+                const bool ok = e + u < cnt;
+                const int j = ok ? mj[e + u] : 0;
+                x[u] = ok ? __ldg(reinterpret_cast<const uint4*>(V + head + (size_t)j * HEAD_DIM) + sd)
+                          : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                float v[8];
+                unpack8(x[u], v);
+                float part = 0.f;
+#pragma unroll
+                for (int d = 0; d < 8; ++d) part = fmaf(g[d], v[d], part);
+                part = group8_sum(part);
+                if (sd == 0 && e + u < cnt) mds[e + u] = part;
             }
         }
-        const float rs = warp_sum(sp[0] + sp[1]);
-        const float wsum = warp_sum(fmaf(sp[0], dA[0], sp[1] * dA[1]));
-        const float u = rs > 0.f ? wsum / rs : 0.f;
-        const float ds[2] = {sp[0] * (dA[0] - u), sp[1] * (dA[1] - u)};
-        // dQ_i = scale sum_e dS_e K_je, lanes over dimensions, eight gathered rows in flight
-        float q0 = 0.f, q1 = 0.f;
-        for (int e0 = 0; e0 < cnt; e0 += 8) {
-            uint32_t kw[8];
-            float dsv[8];
+        __syncwarp();
+        // u_i = sum sp dA / sum sp over the row's entries
+        float r1 = 0.f, w1 = 0.f;
+        for (int e = sd; e < cnt; e += 8) {
+            const float sp = msp[e];
+            r1 += sp;
+            w1 = fmaf(sp, mds[e], w1);
+        }
+        r1 = group8_sum(r1);
+        w1 = group8_sum(w1);
+        const float uu = r1 > 0.f ? w1 / r1 : 0.f;
+        __syncwarp();
+        // dS_e, and (i, sp, dS) into key j's bucket
+        for (int e = sd; e < cnt; e += 8) {
+            const float sp = msp[e];
+            const float ds = sp * (mds[e] - uu);
+            mds[e] = ds;
+            const size_t key = (size_t)bh * L + mj[e];
+            const size_t at = (size_t)bh * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
+            ws.bucket_i[at] = (uint32_t)i;
+            ws.bucket_sp[at] = sp;
+            ws.bucket_ds[at] = ds;
+        }
+        __syncwarp();
+        // dQ_i = scale sum_e dS_e K_je, two entries in flight
+        float acc[8];
 #pragma unroll
-            for (int u8 = 0; u8 < 8; ++u8) {
-                const int e = e0 + u8;
-                const int b = e >> 5;  // uniform
-                const int j = __shfl_sync(0xffffffffu, b == 0 ? jj[0] : jj[1], e & 31);
-                const float d = __shfl_sync(0xffffffffu, b == 0 ? ds[0] : ds[1], e & 31);
-                const bool ok = e < cnt;
-                dsv[u8] = ok ? d : 0.f;
-                kw[u8] = ok ? __ldg(reinterpret_cast<const uint32_t*>(K + head + (size_t)j * HEAD_DIM) + lane) : 0u;
+        for (int d = 0; d < 8; ++d) acc[d] = 0.f;
+        for (int e = 0; e < maxc; e += 2) {
+            uint4 x[2];
+            float dsv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const bool ok = e + u < cnt;
+                const int j = ok ? mj[e + u] : 0;
+                dsv[u] = ok ? mds[e + u] : 0.f;
+                x[u] = ok ? __ldg(reinterpret_cast<const uint4*>(K + head + (size_t)j * HEAD_DIM) + sd)
+                          : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
-            for (int u8 = 0; u8 < 8; ++u8) {
-                q0 = fmaf(dsv[u8], bf16lo(kw[u8]), q0);
-                q1 = fmaf(dsv[u8], bf16hi(kw[u8]), q1);
+            for (int u = 0; u < 2; ++u) {
+                float v[8];
+                unpack8(x[u], v);
+#pragma unroll
+                for (int d = 0; d < 8; ++d) acc[d] = fmaf(dsv[u], v[d], acc[d]);
             }
         }
-        *reinterpret_cast<float2*>(io.dQ + (size_t)row * HEAD_DIM + 2 * lane) = make_float2(a.scale * q0, a.scale * q1);
-        // (i, sp, dS) into key j's bucket
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            const int e = b * 32 + lane;
-            if (e < cnt) {
-                const size_t key = (size_t)bh * L + jj[b];
-                const size_t at = (size_t)bh * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
-                ws.bucket_i[at] = (uint32_t)i;
-                ws.bucket_sp[at] = sp[b];
-                ws.bucket_ds[at] = ds[b];
-            }
+        if (cnt >= 0) {
+            float4* dst = reinterpret_cast<float4*>(io.dQ + (size_t)row * HEAD_DIM + 8 * sd);
+            dst[0] = make_float4(a.scale * acc[0], a.scale * acc[1], a.scale * acc[2], a.scale * acc[3]);
+            dst[1] = make_float4(a.scale * acc[4], a.scale * acc[5], a.scale * acc[6], a.scale * acc[7]);
         }
-        __syncwarp();  // gs is rewritten for the next row
+        __syncwarp();  // the lists are rewritten for the next rows
     }
 }
 
+// Four keys per warp, eight lanes per key: dK_j = scale sum dS Q_i and dV_j = sum p dO_i over key j's
+// bucket, lane s of the group loading entry e0 + s and the group sharing it by shuffles; two
+// entries (four 16-byte row loads per lane) in flight.
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = lane >> 3, sd = lane & 7, g0 = lane & ~7;
     const int L = a.L;
     const long long R = (long long)a.B * a.H * L;
     const size_t cap = (size_t)L * SAVE_CAP;
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.Q);
     const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
-    for (long long key = (long long)blockIdx.x * ROW_WARPS + warp; key < R; key += (long long)gridDim.x * ROW_WARPS) {
-        const int n = sv.key_cnt[key];
-        const long long bh = key / L;
+    for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
+        const long long key = grp * RPW + q;
+        const bool kv = key < R;
+        const int n = kv ? sv.key_cnt[key] : 0;
+        const long long bh = kv ? key / L : 0;
         const size_t head = (size_t)bh * L * HEAD_DIM;
-        const size_t b0 = (size_t)bh * cap + (size_t)ws.key_off[key];
-        float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
-        for (int e0 = 0; e0 < n; e0 += 32) {
-            const int e = e0 + lane;
-            const bool valid = e < n;
-            const uint32_t ii = valid ? ws.bucket_i[b0 + e] : 0u;
-            const float sp = valid ? ws.bucket_sp[b0 + e] : 0.f;
-            const float ds = valid ? ws.bucket_ds[b0 + e] : 0.f;
-            const int m = min(32, n - e0);
-            for (int t0 = 0; t0 < m; t0 += 8) {
-                uint32_t gw[8], qw[8];
-                float pv[8], dv[8];
+        const size_t b0 = (size_t)bh * cap + (size_t)(kv ? ws.key_off[key] : 0);
+        const int maxn = __reduce_max_sync(0xffffffffu, n);
+        float ak[8], av[8];
 #pragma unroll
-                for (int u8 = 0; u8 < 8; ++u8) {
-                    const int t = t0 + u8;
-                    const uint32_t it = __shfl_sync(0xffffffffu, ii, t & 31);
-                    const float st = __shfl_sync(0xffffffffu, sp, t & 31);
-                    const float dt = __shfl_sync(0xffffffffu, ds, t & 31);
-                    const bool ok = t < m;
-                    pv[u8] = ok ? st * st : 0.f;
-                    dv[u8] = ok ? dt : 0.f;
-                    gw[u8] = ok ? __ldg(reinterpret_cast<const uint32_t*>(dO + head + (size_t)it * HEAD_DIM) + lane) : 0u;
-                    qw[u8] = ok ? __ldg(reinterpret_cast<const uint32_t*>(Q + head + (size_t)it * HEAD_DIM) + lane) : 0u;
+        for (int d = 0; d < 8; ++d) ak[d] = av[d] = 0.f;
+        for (int e0 = 0; e0 < maxn; e0 += 8) {
+            const bool mine = e0 + sd < n;
+            const uint32_t ei = mine ? ws.bucket_i[b0 + e0 + sd] : 0u;
+            const float esp = mine ? ws.bucket_sp[b0 + e0 + sd] : 0.f;
+            const float eds = mine ? ws.bucket_ds[b0 + e0 + sd] : 0.f;
+#pragma unroll
+            for (int t = 0; t < 8; t += 2) {
+                uint4 xg[2], xq[2];
+                float pv[2], dv[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int src = g0 | (t + u);
+                    const uint32_t it = __shfl_sync(0xffffffffu, ei, src);
+                    const float st = __shfl_sync(0xffffffffu, esp, src);
+                    const float dt = __shfl_sync(0xffffffffu, eds, src);
+                    const bool ok = e0 + t + u < n;
+                    pv[u] = ok ? st * st : 0.f;
+                    dv[u] = ok ? dt : 0.f;
+                    xg[u] = ok ? __ldg(reinterpret_cast<const uint4*>(dO + head + (size_t)it * HEAD_DIM) + sd)
+                               : make_uint4(0u, 0u, 0u, 0u);
+                    xq[u] = ok ? __ldg(reinterpret_cast<const uint4*>(Q + head + (size_t)it * HEAD_DIM) + sd)
+                               : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
-                for (int u8 = 0; u8 < 8; ++u8) {
-                    v0 = fmaf(pv[u8], bf16lo(gw[u8]), v0);
-                    v1 = fmaf(pv[u8], bf16hi(gw[u8]), v1);
-                    k0 = fmaf(dv[u8], bf16lo(qw[u8]), k0);
-                    k1 = fmaf(dv[u8], bf16hi(qw[u8]), k1);
+                for (int u = 0; u < 2; ++u) {
+                    float vg[8], vq[8];
+                    unpack8(xg[u], vg);
+                    unpack8(xq[u], vq);
+#pragma unroll
+                    for (int d = 0; d < 8; ++d) {
+                        av[d] = fmaf(pv[u], vg[d], av[d]);
+                        ak[d] = fmaf(dv[u], vq[d], ak[d]);
+                    }
                 }
             }
         }
-        *reinterpret_cast<float2*>(io.dK + (size_t)key * HEAD_DIM + 2 * lane) = make_float2(a.scale * k0, a.scale * k1);
-        *reinterpret_cast<float2*>(io.dV + (size_t)key * HEAD_DIM + 2 * lane) = make_float2(v0, v1);
+        if (kv) {
+            float4* dk = reinterpret_cast<float4*>(io.dK + (size_t)key * HEAD_DIM + 8 * sd);
+            float4* dv4 = reinterpret_cast<float4*>(io.dV + (size_t)key * HEAD_DIM + 8 * sd);
+            dk[0] = make_float4(a.scale * ak[0], a.scale * ak[1], a.scale * ak[2], a.scale * ak[3]);
+            dk[1] = make_float4(a.scale * ak[4], a.scale * ak[5], a.scale * ak[6], a.scale * ak[7]);
+            dv4[0] = make_float4(av[0], av[1], av[2], av[3]);
+            dv4[1] = make_float4(av[4], av[5], av[6], av[7]);
+        }
     }
 }
 
