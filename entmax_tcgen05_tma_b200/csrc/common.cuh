@@ -196,13 +196,17 @@ struct Pipe {
     }
 
     // TMA producer: the fixed A tile (rows a_row0.. of head bh), then njobs streamed B blocks through
-    // the NSTAGE ring, job n loading listed block n mod nblk (njobs <= 2 nblk: a second pass re-streams
-    // the list).
+    // the NSTAGE ring.  Job n < n1 loads listed block n * s1 (a first pass over every s1-th block);
+    // job n >= n1 loads listed block n - n1 (a second pass over the whole list).  n1 < 0 means
+    // n1 = nblk, s1 = 1.
     static __device__ __forceinline__ void producer(Ctl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
                                                     const CUtensorMap* map_b, int bh, int a_row0,
                                                     const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b,
-                                                    int njobs) {
-        const int nblk = ctl->nblk;
+                                                    int njobs, int n1 = -1, int s1 = 1) {
+        if (n1 < 0) {
+            n1 = ctl->nblk;
+            s1 = 1;
+        }
         mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
         tma_load_3d(smem_u32(smem_a), map_a, 0, a_row0, bh, smem_u32(&ctl->full_a));
         int issued = 0;
@@ -210,7 +214,7 @@ struct Pipe {
             const int s = n % NSTAGE;
             const uint32_t ph = (uint32_t)(n / NSTAGE) & 1u;
             if (!wait_bounded(smem_u32(&ctl->empty_b[s]), ph ^ 1u, &ctl->abort_flag, wc)) break;
-            const int e = n < nblk ? n : n - nblk;
+            const int e = n < n1 ? n * s1 : n - n1;
             mbar_arrive_expect_tx(smem_u32(&ctl->full_b[s]), BLK_BYTES);
             tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[e] & ~FULL_BLOCK) * BLK, bh,
                         smem_u32(&ctl->full_b[s]));

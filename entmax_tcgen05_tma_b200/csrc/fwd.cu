@@ -470,10 +470,13 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const float c4 = 4.f / (scale * scale);
     const int nblk = ctl->nblk;
     const bool resident = nblk <= NBUF;
-    const int njobs = resident ? nblk : 2 * nblk;
+    // Streamed tiles run pass A on every other listed block only (any subset of a row bounds tau
+    // from below); pass B visits them all.
+    const int nA = resident ? nblk : (nblk + 1) / 2;
+    const int njobs = resident ? nblk : nA + nblk;
 
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs);
+        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs, nA, resident ? 1 : 2);
         __syncwarp();
     } else if (warp == WARP_MMA) {
         if (lane == 0) P::mma(ctl, wc, smem_a, smem_b, njobs);
@@ -491,10 +494,11 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         };
         bool live = true;
 
-        // ---------------- pass A: row max, the four largest 32-key chunk maxima, allowed-key count
-        // Branch-free: a chunk costs a tree of three-input maxima and a min/max insertion network.
-        // The chunk maxima are scores of the row, so the exact threshold of the four largest is a
-        // lower bound of tau (a subset's threshold never exceeds the row's).
+        // ---------------- pass A: the four largest 32-key chunk maxima (of every block, or of every
+        // other block on a streamed tile).  Branch-free: a chunk costs a tree of three-input maxima
+        // and a min/max insertion network.  The chunk maxima are scores of the row, so the exact
+        // threshold of the four largest is a lower bound of tau (a subset's threshold never exceeds
+        // the row's).
         float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
         int nallow = 0;
         const int slot = threadIdx.x % NUM_EPI;
@@ -502,14 +506,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             const int j0 = (int)(blk_list[n] & ~FULL_BLOCK) * BLK;
             return [&, n, j0](const float (&cur)[32], int c) {
                 const uint32_t vm = allowed(n, j0 + c * 32);
-                float cm;
-                if (vm == 0xffffffffu) {
-                    nallow += 32;
-                    cm = max32(cur);
-                } else {
-                    nallow += __popc(vm);
-                    cm = masked_max(cur, vm);
-                }
+                const float cm = vm == 0xffffffffu ? max32(cur) : masked_max(cur, vm);
                 a3 = fmaxf(a3, fminf(a2, cm));
                 a2 = fmaxf(a2, fminf(a1, cm));
                 a1 = fmaxf(a1, fminf(a0, cm));
@@ -523,9 +520,9 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 if (live) for_half_block(ctl, n, g, pass_a(n));
             }
         } else {
-            for (int n = g; n < nblk; n += 2) {
+            for (int n = g; n < nA; n += 2) {
                 if (live) live = __all_sync(0xffffffffu, P::wait_scores(ctl, wc, n));
-                if (live) P::for_each_chunk(ctl, n, pass_a(n));
+                if (live) P::for_each_chunk(ctl, n, pass_a(2 * n));
             }
         }
         {
@@ -534,7 +531,6 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             mine.a1 = a1;
             mine.a2 = a2;
             mine.a3 = a3;
-            mine.nallow = nallow;
         }
         epi_sync();
         {
@@ -544,8 +540,9 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             top4_insert(other.a2, a0, a1, a2, a3);
             top4_insert(other.a3, a0, a1, a2, a3);
         }
-        // scores at or below t are outside the support: max - 2 (scaled), raised to the exact
-        // threshold of the row's four largest chunk maxima (any subset's threshold is at most tau)
+        // scores at or below t are outside the support: the largest chunk maximum seen minus 2
+        // (scaled), raised to the exact threshold of the four largest chunk maxima seen (any
+        // subset's threshold is at most tau)
         const float t = fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
 
         // ---------------- pass B: candidates s > m - 2 (scaled) into this warpgroup's partition
@@ -556,7 +553,9 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             const int j0 = (int)(blk_list[e] & ~FULL_BLOCK) * BLK;
             return [&, e, j0](const float (&cur)[32], int c) {
                 const int jc = j0 + c * 32;
-                uint32_t hits = hit_bits(cur, t) & __brev(allowed(e, jc));
+                const uint32_t vm = allowed(e, jc);
+                nallow += __popc(vm);
+                uint32_t hits = hit_bits(cur, t) & __brev(vm);
                 if (hits) {
                     stage_chunk(stage, slot, cur);
                     do {
@@ -578,11 +577,12 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 for (int n = 0; n < nblk; ++n) for_half_block(ctl, n, g, pass_b(n));
             }
         } else {
-            for (int n = nblk + ((g ^ nblk) & 1); n < njobs; n += 2) {
+            for (int n = nA + ((g ^ nA) & 1); n < njobs; n += 2) {
                 if (live) live = __all_sync(0xffffffffu, P::wait_scores(ctl, wc, n));
-                if (live) P::for_each_chunk(ctl, n, pass_b(n - nblk));
+                if (live) P::for_each_chunk(ctl, n, pass_b(n - nA));
             }
         }
+        rows[g * TILE + r].nallow = nallow;
         rows[g * TILE + r].n = min(nc, CAPW);
         rows[g * TILE + r].ovf = nc > CAPW ? 1 : 0;
     }
@@ -606,13 +606,22 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const int i = i0 + r;
         const RowOut s0 = rows[r], s1 = rows[TILE + r];
         const int nallow = s0.nallow + s1.nallow;
-        const float ms = scale * fmaxf(s0.a0, s1.a0);  // scaled row max
-        int mode = 0;                                 // 0: solved here, 2: fallback, 3: no key
+        int mode = 0;  // 0: solved here, 2: fallback, 3: no key
         if (i >= L || nallow == 0) mode = 3;
         else if (s0.ovf | s1.ovf) mode = 2;
         const int nh = mode == 0 ? (h == 0 ? s0.n : s1.n) : 0;
         float* pcv = cv + h * CAPW * TILE;
         uint16_t* pcj = cj + h * CAPW * TILE;
+        // Row max: pass A saw every block of a resident tile, so its largest chunk maximum is the max;
+        // on a streamed tile take the largest candidate (the max exceeds every lower bound of tau, so
+        // it is always listed).
+        float cmax = fmaxf(s0.a0, s1.a0);
+        if (!resident) {
+            cmax = -INFINITY;
+            for (int k = 0; k < nh; ++k) cmax = fmaxf(cmax, pcv[k * TILE + r]);
+            cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
+        }
+        const float ms = scale * cmax;  // scaled row max
         // every lane takes part in the pair shuffles (rows of one warp may differ in mode)
         // Bracket (shifted scaled units, row max = 0): lo = the bound the candidates were cut at (the
         // exact threshold of the four largest chunk maxima, or max - 2), g(lo) >= g(tau) = 1; hi =
