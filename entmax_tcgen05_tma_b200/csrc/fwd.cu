@@ -673,26 +673,40 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             for (int c = 0; c < 4; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) acc[c][k] = 0.f;
-            for (int e = 0; e < n0 + n1; ++e) {
-                const int sl = e < n0 ? e : CAPW + (e - n0);
-                const int j = cj[sl * TILE + r];
-                const float p = cv[sl * TILE + r];
-                uint4 x[4];
-                if (v_staged) {
+            const int ns = n0 + n1;
+            if (v_staged) {
+                for (int e = 0; e < ns; ++e) {
+                    const int sl = e < n0 ? e : CAPW + (e - n0);
+                    const int j = cj[sl * TILE + r];
+                    const float p = cv[sl * TILE + r];
                     // 128-byte swizzled V block in ring slot vslot[j / BLK]: 16-byte chunk c of row
                     // `row` sits at chunk position c ^ (row & 7)
                     const uint32_t row = (uint32_t)j & (BLK - 1);
                     const uint8_t* base = smem_b + vslot[j / BLK] * BLK_BYTES + row * 128u;
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        x[c] = *reinterpret_cast<const uint4*>(base + ((((uint32_t)(4 * h + c)) ^ (row & 7u)) << 4));
-                } else {
-                    const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)j * HEAD_DIM) + 4 * h;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) x[c] = __ldg(src + c);
+                        fma_bf16x8(acc[c], p, *reinterpret_cast<const uint4*>(base + ((((uint32_t)(4 * h + c)) ^ (row & 7u)) << 4)));
                 }
+            } else {
+                // V rows from L2, two support entries per step (eight 16-byte loads in flight; a missing
+                // second entry repeats the first with weight 0)
+                for (int e = 0; e < ns; e += 2) {
+                    uint4 x[2][4];
+                    float pw[2];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) fma_bf16x8(acc[c], p, x[c]);
+                    for (int u = 0; u < 2; ++u) {
+                        const int ee = e + u < ns ? e + u : e;
+                        const int sl = ee < n0 ? ee : CAPW + (ee - n0);
+                        const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)cj[sl * TILE + r] * HEAD_DIM) + 4 * h;
+                        pw[u] = e + u < ns ? cv[sl * TILE + r] : 0.f;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) x[u][c] = __ldg(src + c);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) fma_bf16x8(acc[c], pw[u], x[u][c]);
+                }
             }
             const size_t oi = ((size_t)bh * L + i) * HEAD_DIM + 32 * h;
             if (out.out_f32) {
