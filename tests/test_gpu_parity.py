@@ -274,3 +274,46 @@ def test_training_path_empty_batch():
     assert torch.all(O[1] == 0) and torch.all(torch.isinf(tau[1]))
     for g in grads:
         assert torch.all(g[1] == 0)
+
+
+# ----------------------------------------------------------------------------------- size limits
+@pytest.mark.parametrize("causal,window,scale", [(False, 0, 2 / 8), (True, 32, 1 / 8)])
+def test_maximum_sequence_length(causal, window, scale):
+    """L = 16384, the longest sequence the library takes (128 streamed key blocks per query tile):
+    forward on sampled rows, both backward paths on the whole head."""
+    w = Workload(0, "max-L", 1, 1, 16384, 64, scale, causal=causal, window=window)
+    inp = make_inputs(w, seed=21)
+    d = inputs_f64(inp, False)
+    O, tau, dev = _gpu_fwd(inp, w, out_dtype=torch.float32)
+    rng = np.random.default_rng(21)
+    ids = np.unique(np.concatenate([rng.integers(0, w.L, size=96), [0, 1, 127, 128, w.L // 2, w.L - 1]]))
+    O_ref, tau_ref = orc.attn_fwd_rows(d["Q"], d["K"], d["V"], ids, None, causal, window, scale)
+    assert np.max(np.abs(to64(O).reshape(-1, w.D)[ids] - O_ref)) <= O_TOL
+    check_rows(d["Q"], d["K"], ids, to64(tau).reshape(-1)[ids], tau_ref, None, causal, window, scale, w.H, w.L)
+    rQ, rK, rV = orc.attn_bwd_heads(d["Q"], d["K"], d["V"], d["dO"], [0], None, causal, window, scale)
+    grads = [_gpu_bwd(dev, tau, inp["dO"], w)]
+    _, _, g_saved = _gpu_train(inp, w)
+    grads.append(g_saved)
+    for g in grads:
+        for name, x, r in zip(("dQ", "dK", "dV"), g, (rQ, rK, rV)):
+            err = np.max(np.abs(to64(x).reshape(1, w.L, w.D) - r))
+            assert err <= GRAD_TOL, (name, err)
+
+
+def test_maximum_head_count():
+    """B * H = 65535 heads (the grid's limit), two rows each, with key padding down to one key."""
+    w = Workload(0, "max-heads", 65535, 1, 2, 64, 1 / 8, len_range=(1, 2))
+    inp = make_inputs(w, seed=22)
+    d = inputs_f64(inp, False)
+    km = inp["key_mask"].numpy()
+    O, tau, dev = _gpu_fwd(inp, w, out_dtype=torch.float32)
+    ids = np.array(sorted({0, 1, 2, 3, 65533 * 2, 65534 * 2, 65534 * 2 + 1} | set(range(40000, 40040))), dtype=np.int64)
+    O_ref, tau_ref = orc.attn_fwd_rows(d["Q"], d["K"], d["V"], ids, km, False, 0, w.scale)
+    assert np.max(np.abs(to64(O).reshape(-1, w.D)[ids] - O_ref)) <= O_TOL
+    check_rows(d["Q"], d["K"], ids, to64(tau).reshape(-1)[ids], tau_ref, km, False, 0, w.scale, w.H, w.L)
+    heads = [0, 1, 20000, 65534]
+    rQ, rK, rV = orc.attn_bwd_heads(d["Q"], d["K"], d["V"], d["dO"], heads, km, False, 0, w.scale)
+    for g in (_gpu_bwd(dev, tau, inp["dO"], w), _gpu_train(inp, w)[2]):
+        for name, x, r in zip(("dQ", "dK", "dV"), g, (rQ, rK, rV)):
+            err = np.max(np.abs(to64(x).reshape(-1, w.L, w.D)[heads] - r))
+            assert err <= GRAD_TOL, (name, err)
