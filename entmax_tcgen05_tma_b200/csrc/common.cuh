@@ -336,16 +336,34 @@ __device__ __forceinline__ float max32(const float (&v)[32]) {
     return fmaxf(fmax3(a, b, c), d);
 }
 
-// Bit (31 - k) of the result is set iff v[k] > t: the sign bit of t - v[k] funnel-shifted into
-// four independent 8-bit chains (two instructions per value, no branches).
+// t - (a, b) for two values at once (one packed sm_100 subtraction).
+__device__ __forceinline__ void sub2(float t, float a, float b, float& da, float& db) {
+    uint64_t ab, tt, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ab) : "f"(a), "f"(b));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(tt) : "f"(t));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(tt), "l"(ab));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(da), "=f"(db) : "l"(r));
+}
+
+// Bit (31 - k) of the result is set iff v[k] > t: the sign bit of t - v[k] (packed subtractions,
+// two values each) funnel-shifted into four independent 8-bit chains (no branches).
 __device__ __forceinline__ uint32_t hit_bits(const float (&v)[32], float t) {
     uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        h0 = __funnelshift_l(__float_as_uint(t - v[k]), h0, 1);
-        h1 = __funnelshift_l(__float_as_uint(t - v[8 + k]), h1, 1);
-        h2 = __funnelshift_l(__float_as_uint(t - v[16 + k]), h2, 1);
-        h3 = __funnelshift_l(__float_as_uint(t - v[24 + k]), h3, 1);
+    for (int k = 0; k < 8; k += 2) {
+        float d[8];
+        sub2(t, v[k], v[k + 1], d[0], d[1]);
+        sub2(t, v[8 + k], v[9 + k], d[2], d[3]);
+        sub2(t, v[16 + k], v[17 + k], d[4], d[5]);
+        sub2(t, v[24 + k], v[25 + k], d[6], d[7]);
+        h0 = __funnelshift_l(__float_as_uint(d[0]), h0, 1);
+        h1 = __funnelshift_l(__float_as_uint(d[2]), h1, 1);
+        h2 = __funnelshift_l(__float_as_uint(d[4]), h2, 1);
+        h3 = __funnelshift_l(__float_as_uint(d[6]), h3, 1);
+        h0 = __funnelshift_l(__float_as_uint(d[1]), h0, 1);
+        h1 = __funnelshift_l(__float_as_uint(d[3]), h1, 1);
+        h2 = __funnelshift_l(__float_as_uint(d[5]), h2, 1);
+        h3 = __funnelshift_l(__float_as_uint(d[7]), h3, 1);
     }
     return (h0 << 24) | (h1 << 16) | (h2 << 8) | h3;
 }

@@ -34,8 +34,14 @@ namespace {
 using P = Pipe<128, 4, 4, 2>;  // 128-key blocks, 4-deep ring, 4 TMEM buffers, 2 epilogue warpgroups
 using PipeCtl = P::Ctl;
 constexpr int BLK = P::BLK, NSTAGE = P::NSTAGE, NBUF = P::NBUF;
-constexpr int NUM_EPI = P::NUM_EPI, NUM_THREADS = P::NUM_THREADS, NUM_WARPS = P::NUM_WARPS;
+constexpr int NUM_EPI = P::NUM_EPI;
+// Two producer/MMA warp pairs: on a streamed tile pair p feeds epilogue warpgroup p alone (its own
+// K-ring stages 2p, 2p + 1 and TMEM buffers p, p + 2), so the warpgroups never wait on each other's
+// MMAs; on a resident tile pair 0 feeds both.
 constexpr int WARP_PRODUCER = P::WARP_PRODUCER, WARP_MMA = P::WARP_MMA;
+constexpr int WARP_PRODUCER2 = WARP_MMA + 1, WARP_MMA2 = WARP_MMA + 2;
+constexpr int NUM_THREADS = P::NUM_THREADS + 64, NUM_WARPS = NUM_THREADS / 32;
+static_assert(NSTAGE == 4 && NBUF == 4, "two pipelines of two stages and two buffers each");
 constexpr int BLK_BYTES = P::BLK_BYTES, TMEM_COLS = P::TMEM_COLS, MAX_BLOCKS = P::MAX_BLOCKS;
 constexpr int STAGE_FLOATS = NUM_EPI * 32;  // per-thread staging of one 32-value chunk
 static_assert(NSTAGE >= NBUF, "a resident tile's V blocks are staged in the streamed-block ring");
@@ -408,6 +414,66 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
     __syncthreads();
 }
 
+// Streamed tile, pipeline p: local job m loads and multiplies listed block half_block(p, m) -- first
+// the pass-A blocks 2k (k < nA, k = p mod 2), then the pass-B blocks k = p mod 2 -- through K-ring
+// stage 2p + (m & 1) into TMEM buffer p + 2 (m & 1); both alternate, so their completion parity is
+// (m >> 1) & 1.
+__device__ __forceinline__ int half_block(int p, int m, int mA) { return m < mA ? 2 * (p + 2 * m) : p + 2 * (m - mA); }
+
+__device__ __noinline__ void produce_half(PipeCtl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
+                                          const CUtensorMap* map_b, int bh, int a_row0, const uint16_t* blk_list,
+                                          uint8_t* smem_a, uint8_t* smem_b, int p, int mA, int mB) {
+    if (p == 0) {
+        mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
+        tma_load_3d(smem_u32(smem_a), map_a, 0, a_row0, bh, smem_u32(&ctl->full_a));
+    }
+    int issued = 0;
+    for (int m = 0; m < mA + mB; ++m) {
+        const int st = 2 * p + (m & 1);
+        const uint32_t ph = (uint32_t)(m >> 1) & 1u;
+        if (!wait_bounded(smem_u32(&ctl->empty_b[st]), ph ^ 1u, &ctl->abort_flag, wc)) break;
+        mbar_arrive_expect_tx(smem_u32(&ctl->full_b[st]), BLK_BYTES);
+        tma_load_3d(smem_u32(smem_b + st * BLK_BYTES), map_b, 0, (int)(blk_list[half_block(p, m, mA)] & ~FULL_BLOCK) * BLK,
+                    bh, smem_u32(&ctl->full_b[st]));
+        ++issued;
+    }
+    if (P::aborted(ctl)) {
+        // drain: every copy issued must land before the CTA's shared memory is released
+        if (p == 0) wait_drain(smem_u32(&ctl->full_a), 0);
+        for (int m = max(0, issued - 2); m < issued; ++m)
+            wait_drain(smem_u32(&ctl->full_b[2 * p + (m & 1)]), (uint32_t)(m >> 1) & 1u);
+    }
+}
+
+__device__ __noinline__ void mma_half(PipeCtl* ctl, const WaitCfg& wc, const uint8_t* smem_a, const uint8_t* smem_b,
+                                      int p, int njobs) {
+    constexpr uint32_t idesc = umma_idesc_bf16_f32(TILE, BLK);
+    int issued = 0;
+    if (wait_bounded(smem_u32(&ctl->full_a), 0, &ctl->abort_flag, wc)) {
+        tc_fence_after();
+        const uint64_t da = umma_desc_kmajor_sw128(smem_u32(smem_a));
+        for (int m = 0; m < njobs; ++m) {
+            const int st = 2 * p + (m & 1), buf = p + 2 * (m & 1);
+            const uint32_t ph = (uint32_t)(m >> 1) & 1u;
+            if (!wait_bounded(smem_u32(&ctl->full_b[st]), ph, &ctl->abort_flag, wc)) break;
+            if (!wait_bounded(smem_u32(&ctl->s_empty[buf]), ph ^ 1u, &ctl->abort_flag, wc)) break;
+            tc_fence_after();
+            const uint64_t db = umma_desc_kmajor_sw128(smem_u32(smem_b + st * BLK_BYTES));
+            const uint32_t d_tmem = ctl->tmem_base + (uint32_t)(buf * BLK);
+#pragma unroll
+            for (int k = 0; k < HEAD_DIM / 16; ++k)  // 16 bf16 = 32 B = 2 descriptor units per step
+                tc_mma_bf16(d_tmem, da + 2u * k, db + 2u * k, idesc, k > 0 ? 1u : 0u);
+            tc_commit(smem_u32(&ctl->empty_b[st]));
+            tc_commit(smem_u32(&ctl->s_full[buf]));
+            ++issued;
+        }
+    }
+    if (P::aborted(ctl) && issued > 0) {
+        const int m = issued - 1;  // the last commit covers every earlier MMA of this thread
+        wait_drain(smem_u32(&ctl->s_full[p + 2 * (m & 1)]), (uint32_t)(m >> 1) & 1u);
+    }
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const AttnArgs args, const FwdOut out) {
@@ -475,11 +541,28 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int nA = resident ? nblk : (nblk + 1) / 2;
     const int njobs = resident ? nblk : nA + nblk;
 
-    if (warp == WARP_PRODUCER) {
-        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs, nA, resident ? 1 : 2);
+    // per-warpgroup job counts of a streamed tile: pass-A blocks 2k (k < nA, k = g mod 2), then
+    // pass-B blocks k = g mod 2
+    const int mA0 = (nA + 1) >> 1, mA1 = nA >> 1, mB0 = (nblk + 1) >> 1, mB1 = nblk >> 1;
+    if (warp == WARP_PRODUCER || warp == WARP_PRODUCER2) {
+        const int p = warp == WARP_PRODUCER ? 0 : 1;
+        if (lane == 0) {
+            if (resident) {
+                if (p == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs);
+            } else {
+                produce_half(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, p, p ? mA1 : mA0, p ? mB1 : mB0);
+            }
+        }
         __syncwarp();
-    } else if (warp == WARP_MMA) {
-        if (lane == 0) P::mma(ctl, wc, smem_a, smem_b, njobs);
+    } else if (warp == WARP_MMA || warp == WARP_MMA2) {
+        const int p = warp == WARP_MMA ? 0 : 1;
+        if (lane == 0) {
+            if (resident) {
+                if (p == 0) P::mma(ctl, wc, smem_a, smem_b, njobs);
+            } else {
+                mma_half(ctl, wc, smem_a, smem_b, p, p ? mA1 + mB1 : mA0 + mB0);
+            }
+        }
         __syncwarp();
     } else {
         // thread (g, r): query row i0 + r; warpgroup g takes half g of every block (resident) or
@@ -520,9 +603,13 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 if (live) for_half_block(ctl, n, g, pass_a(n));
             }
         } else {
-            for (int n = g; n < nA; n += 2) {
-                if (live) live = __all_sync(0xffffffffu, P::wait_scores(ctl, wc, n));
-                if (live) P::for_each_chunk(ctl, n, pass_a(2 * n));
+            // this warpgroup's pipeline: local job m in TMEM buffer g + 2 (m & 1), parity (m >> 1) & 1
+            const int mA = g ? mA1 : mA0;
+            for (int m = 0; m < mA; ++m) {
+                const int buf = g + 2 * (m & 1);
+                if (live) live = warp_wait(smem_u32(&ctl->s_full[buf]), (uint32_t)(m >> 1) & 1u, &ctl->abort_flag, wc);
+                tc_fence_after();
+                if (live) P::for_each_chunk(ctl, buf, pass_a(half_block(g, m, mA)));
             }
         }
         {
@@ -577,9 +664,12 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 for (int n = 0; n < nblk; ++n) for_half_block(ctl, n, g, pass_b(n));
             }
         } else {
-            for (int n = nA + ((g ^ nA) & 1); n < njobs; n += 2) {
-                if (live) live = __all_sync(0xffffffffu, P::wait_scores(ctl, wc, n));
-                if (live) P::for_each_chunk(ctl, n, pass_b(n - nA));
+            const int mA = g ? mA1 : mA0, mB = g ? mB1 : mB0;
+            for (int m = mA; m < mA + mB; ++m) {
+                const int buf = g + 2 * (m & 1);
+                if (live) live = warp_wait(smem_u32(&ctl->s_full[buf]), (uint32_t)(m >> 1) & 1u, &ctl->abort_flag, wc);
+                tc_fence_after();
+                if (live) P::for_each_chunk(ctl, buf, pass_b(half_block(g, m, mA)));
             }
         }
         rows[g * TILE + r].nallow = nallow;
