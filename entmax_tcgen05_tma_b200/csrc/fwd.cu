@@ -167,16 +167,21 @@ __device__ __forceinline__ void for_half_block(const PipeCtl* ctl, int n, int ha
 }
 
 // tau of one row in shifted scaled units (x = scale * S - scale * m, so the row max is 0), from the
-// candidates of the two partitions held by a lane pair (NC registers each, -inf where unused).
+// row's candidates (both partitions, partition 0 first) split evenly over a lane pair: lane h holds
+// entries h, h + 2, ... (NC registers, -inf where unused).
 // Bisection of [lo, hi], a sub-bracket of [-2, -2/sqrt(n)] that still holds the root (the caller's
 // bounds: g(lo) >= 1, g(hi) <= 1; g(-2) >= 1 from the max alone, g(-2/sqrt n) <= 1); every four
 // halvings the warp stops if no lane pair has a candidate strictly inside its bracket: the support
 // is then fixed and the closed-form root on it is exact.  Returns tau_x.
 template <int NC>
-__device__ __forceinline__ float solve_tau(const float* pcv, int r, int nh, float scale, float ms, float lo, float hi) {
+__device__ __forceinline__ float solve_tau(const float* lcv, int r, int h, int nh, int n0, float scale, float ms,
+                                           float lo, float hi) {
     float x[NC];
 #pragma unroll
-    for (int k = 0; k < NC; ++k) x[k] = k < nh ? fmaf(scale, pcv[k * TILE + r], -ms) : -INFINITY;
+    for (int k = 0; k < NC; ++k) {
+        const int e = 2 * k + h;  // entry e of the row's two lists, partition 0's n0 entries first
+        x[k] = k < nh ? fmaf(scale, lcv[(e < n0 ? e : CAPW + (e - n0)) * TILE + r], -ms) : -INFINITY;
+    }
     bool settled = false;
     for (int it = 0; it < 25; ++it) {
         const float mid = 0.5f * (lo + hi);
@@ -725,10 +730,22 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const float t_cut = fmaxf(b0 - two_over_scale, top4_bound(b0, b1, b2, b3, c4));
         const float hi = -2.f / sqrtf((float)max(s0.n + s1.n, 1));
         const float lo = fminf(fmaxf(-2.f, fmaf(scale, t_cut, -ms)), hi);
-        const int nmax = __reduce_max_sync(0xffffffffu, nh);
-        const float tau_x = nmax <= 16   ? solve_tau<16>(pcv, r, nh, scale, ms, lo, hi)
-                            : nmax <= 32 ? solve_tau<32>(pcv, r, nh, scale, ms, lo, hi)
-                                         : solve_tau<CAPW>(pcv, r, nh, scale, ms, lo, hi);
+        // the row's candidates split evenly over its two threads; registers: the warp's largest share
+        // rounded up to a multiple of eight
+        const int ns = mode == 0 ? (s0.n + s1.n + 1 - h) >> 1 : 0;
+        const int nmax = __reduce_max_sync(0xffffffffu, ns);
+        float tau_x;
+        switch ((nmax + 7) >> 3) {
+            case 0:
+            case 1: tau_x = solve_tau<8>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            case 2: tau_x = solve_tau<16>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            case 3: tau_x = solve_tau<24>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            case 4: tau_x = solve_tau<32>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            case 5: tau_x = solve_tau<40>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            case 6: tau_x = solve_tau<48>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            case 7: tau_x = solve_tau<56>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            default: tau_x = solve_tau<CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+        }
         if (mode == 0) {
             // this thread's partition of the support: cv <- p_ij, cj <- j (in place)
             int sn = 0;
