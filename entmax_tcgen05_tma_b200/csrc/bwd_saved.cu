@@ -83,10 +83,169 @@ __device__ __forceinline__ float group8_sum(float v) {
     return v;
 }
 
-// Four query rows per warp, eight lanes per row.  The row's saved list is staged in shared memory;
-// dA_e = dO_i . V_je takes one 16-byte load of V_je per lane and a three-step group reduction, two
-// entries in flight; then u_i, dS_e, the bucket entries, and dQ_i (one 16-byte load of K_je per lane
-// per entry).
+// Gathered 128-byte rows of one head's [L, 64] slab: lane sd's 16-byte piece of row j.
+struct GlobalRows {
+    const __nv_bfloat16* x;  // [L, 64] slab of one head
+    __device__ __forceinline__ uint4 get(int j, int sd) const {
+        return __ldg(reinterpret_cast<const uint4*>(x + (size_t)j * HEAD_DIM) + sd);
+    }
+};
+// One query row per group of eight lanes (lane sd owns dimensions 8 sd .. 8 sd + 7), row list
+// staged in shared memory (mj, msp; mds holds dA, then dS).  dA_e = dO_i . V_je with one 16-byte
+// piece of V_je per lane and a three-step group reduction, two entries in flight; then u_i, dS_e,
+// the bucket entries, and dQ_i (one 16-byte piece of K_je per lane per entry).  cnt < 0: no row, or
+// a row the exact pass handles.
+template <class Rows>
+__device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
+                                           const SavedBwdWs& ws, long long row, int cnt, int bh, int i, const Rows& Vr,
+                                           const Rows& Kr, uint16_t* mj, float* msp, float* mds, int sd) {
+    const int L = a.L;
+    const size_t cap = (size_t)L * SAVE_CAP;
+    const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
+    for (int e = sd; e < cnt; e += 8) {
+        mj[e] = sv.row_j[(size_t)row * SAVE_CAP + e];
+        msp[e] = sv.row_sp[(size_t)row * SAVE_CAP + e];
+    }
+    float g[8];
+    {
+        const uint4 x = cnt >= 0 ? __ldg(reinterpret_cast<const uint4*>(dO + (size_t)row * HEAD_DIM) + sd)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+        unpack8(x, g);
+    }
+    const int maxc = __reduce_max_sync(0xffffffffu, max(cnt, 0));
+    __syncwarp();
+    // dA_e, two entries in flight
+    for (int e = 0; e < maxc; e += 2) {
+        uint4 x[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const bool ok = e + u < cnt;
+            x[u] = ok ? Vr.get(mj[e + u], sd) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            float v[8];
+            unpack8(x[u], v);
+            float part = 0.f;
+#pragma unroll
+            for (int d = 0; d < 8; ++d) part = fmaf(g[d], v[d], part);
+            part = group8_sum(part);
+            if (sd == 0 && e + u < cnt) mds[e + u] = part;
+        }
+    }
+    __syncwarp();
+    // u_i = sum sp dA / sum sp over the row's entries
+    float r1 = 0.f, w1 = 0.f;
+    for (int e = sd; e < cnt; e += 8) {
+        const float sp = msp[e];
+        r1 += sp;
+        w1 = fmaf(sp, mds[e], w1);
+    }
+    r1 = group8_sum(r1);
+    w1 = group8_sum(w1);
+    const float uu = r1 > 0.f ? w1 / r1 : 0.f;
+    __syncwarp();
+    // dS_e, and (i, sp, dS) into key j's bucket
+    for (int e = sd; e < cnt; e += 8) {
+        const float sp = msp[e];
+        const float ds = sp * (mds[e] - uu);
+        mds[e] = ds;
+        const size_t key = (size_t)bh * L + mj[e];
+        const size_t at = (size_t)bh * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
+        ws.bucket_i[at] = (uint32_t)i;
+        ws.bucket_sp[at] = sp;
+        ws.bucket_ds[at] = ds;
+    }
+    __syncwarp();
+    // dQ_i = scale sum_e dS_e K_je, two entries in flight
+    float acc[8];
+#pragma unroll
+    for (int d = 0; d < 8; ++d) acc[d] = 0.f;
+    for (int e = 0; e < maxc; e += 2) {
+        uint4 x[2];
+        float dsv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const bool ok = e + u < cnt;
+            dsv[u] = ok ? mds[e + u] : 0.f;
+            x[u] = ok ? Kr.get(mj[e + u], sd) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            float v[8];
+            unpack8(x[u], v);
+#pragma unroll
+            for (int d = 0; d < 8; ++d) acc[d] = fmaf(dsv[u], v[d], acc[d]);
+        }
+    }
+    if (cnt >= 0) {
+        float4* dst = reinterpret_cast<float4*>(io.dQ + (size_t)row * HEAD_DIM + 8 * sd);
+        dst[0] = make_float4(a.scale * acc[0], a.scale * acc[1], a.scale * acc[2], a.scale * acc[3]);
+        dst[1] = make_float4(a.scale * acc[4], a.scale * acc[5], a.scale * acc[6], a.scale * acc[7]);
+    }
+    __syncwarp();  // the lists are rewritten for the next rows
+}
+
+// One key per group of eight lanes: dK_j = scale sum dS Q_i and dV_j = sum p dO_i over key j's bucket,
+// lane sd of the group loading entry e0 + sd and the group sharing it by shuffles; two entries (two
+// 16-byte pieces each per lane) in flight.  valid = false: no key (the group still takes part).
+template <class Rows>
+__device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
+                                           const SavedBwdWs& ws, long long key, bool valid, int bh, const Rows& Qr,
+                                           const Rows& Gr, int sd, int g0) {
+    const int L = a.L;
+    const size_t cap = (size_t)L * SAVE_CAP;
+    const int n = valid ? sv.key_cnt[key] : 0;
+    const size_t b0 = (size_t)bh * cap + (size_t)(valid ? ws.key_off[key] : 0);
+    const int maxn = __reduce_max_sync(0xffffffffu, n);
+    float ak[8], av[8];
+#pragma unroll
+    for (int d = 0; d < 8; ++d) ak[d] = av[d] = 0.f;
+    for (int e0 = 0; e0 < maxn; e0 += 8) {
+        const bool mine = e0 + sd < n;
+        const uint32_t ei = mine ? ws.bucket_i[b0 + e0 + sd] : 0u;
+        const float esp = mine ? ws.bucket_sp[b0 + e0 + sd] : 0.f;
+        const float eds = mine ? ws.bucket_ds[b0 + e0 + sd] : 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; t += 2) {
+            uint4 xg[2], xq[2];
+            float pv[2], dv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int src = g0 | (t + u);
+                const uint32_t it = __shfl_sync(0xffffffffu, ei, src);
+                const float st = __shfl_sync(0xffffffffu, esp, src);
+                const float dt = __shfl_sync(0xffffffffu, eds, src);
+                const bool ok = e0 + t + u < n;
+                pv[u] = ok ? st * st : 0.f;
+                dv[u] = ok ? dt : 0.f;
+                xg[u] = ok ? Gr.get((int)it, sd) : make_uint4(0u, 0u, 0u, 0u);
+                xq[u] = ok ? Qr.get((int)it, sd) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                float vg[8], vq[8];
+                unpack8(xg[u], vg);
+                unpack8(xq[u], vq);
+#pragma unroll
+                for (int d = 0; d < 8; ++d) {
+                    av[d] = fmaf(pv[u], vg[d], av[d]);
+                    ak[d] = fmaf(dv[u], vq[d], ak[d]);
+                }
+            }
+        }
+    }
+    if (valid) {
+        float4* dk = reinterpret_cast<float4*>(io.dK + (size_t)key * HEAD_DIM + 8 * sd);
+        float4* dv4 = reinterpret_cast<float4*>(io.dV + (size_t)key * HEAD_DIM + 8 * sd);
+        dk[0] = make_float4(a.scale * ak[0], a.scale * ak[1], a.scale * ak[2], a.scale * ak[3]);
+        dk[1] = make_float4(a.scale * ak[4], a.scale * ak[5], a.scale * ak[6], a.scale * ak[7]);
+        dv4[0] = make_float4(av[0], av[1], av[2], av[3]);
+        dv4[1] = make_float4(av[4], av[5], av[6], av[7]);
+    }
+}
+
+// Four query rows per warp (eight lanes each), rows of K and V gathered from L2.
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     __shared__ uint16_t lj[ROW_WARPS][RPW][SAVE_CAP];
@@ -96,175 +255,33 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
     const int q = lane >> 3, sd = lane & 7;
     const int L = a.L;
     const long long R = (long long)a.B * a.H * L;
-    const size_t cap = (size_t)L * SAVE_CAP;
-    const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(a.K);
-    const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(a.V);
-    const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
-    uint16_t* mj = lj[warp][q];
-    float* msp = lsp[warp][q];
-    float* mds = lds[warp][q];
     for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long row = grp * RPW + q;
-        const int cnt = row < R ? sv.row_cnt[row] : -1;  // -1: no row, or not saved (the exact pass handles it)
-        const long long bh = row < R ? row / L : 0;
-        const int i = (int)(row - bh * L);
+        const int cnt = row < R ? sv.row_cnt[row] : -1;
+        const int bh = row < R ? (int)(row / L) : 0;
+        const int i = (int)(row - (long long)bh * L);
         const size_t head = (size_t)bh * L * HEAD_DIM;
-        for (int e = sd; e < cnt; e += 8) {
-            mj[e] = sv.row_j[(size_t)row * SAVE_CAP + e];
-            msp[e] = sv.row_sp[(size_t)row * SAVE_CAP + e];
-        }
-        float g[8];
-        {
-            const uint4 x = cnt >= 0 ? __ldg(reinterpret_cast<const uint4*>(dO + (size_t)row * HEAD_DIM) + sd)
-                                     : make_uint4(0u, 0u, 0u, 0u);
-            unpack8(x, g);
-        }
-        const int maxc = __reduce_max_sync(0xffffffffu, max(cnt, 0));
-        __syncwarp();
-        // dA_e, two entries in flight
-        for (int e = 0; e < maxc; e += 2) {
-            uint4 x[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const bool ok = e + u < cnt;
-                const int j = ok ? mj[e + u] : 0;
-                x[u] = ok ? __ldg(reinterpret_cast<const uint4*>(V + head + (size_t)j * HEAD_DIM) + sd)
-                          : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                float v[8];
-                unpack8(x[u], v);
-                float part = 0.f;
-#pragma unroll
-                for (int d = 0; d < 8; ++d) part = fmaf(g[d], v[d], part);
-                part = group8_sum(part);
-                if (sd == 0 && e + u < cnt) mds[e + u] = part;
-            }
-        }
-        __syncwarp();
-        // u_i = sum sp dA / sum sp over the row's entries
-        float r1 = 0.f, w1 = 0.f;
-        for (int e = sd; e < cnt; e += 8) {
-            const float sp = msp[e];
-            r1 += sp;
-            w1 = fmaf(sp, mds[e], w1);
-        }
-        r1 = group8_sum(r1);
-        w1 = group8_sum(w1);
-        const float uu = r1 > 0.f ? w1 / r1 : 0.f;
-        __syncwarp();
-        // dS_e, and (i, sp, dS) into key j's bucket
-        for (int e = sd; e < cnt; e += 8) {
-            const float sp = msp[e];
-            const float ds = sp * (mds[e] - uu);
-            mds[e] = ds;
-            const size_t key = (size_t)bh * L + mj[e];
-            const size_t at = (size_t)bh * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
-            ws.bucket_i[at] = (uint32_t)i;
-            ws.bucket_sp[at] = sp;
-            ws.bucket_ds[at] = ds;
-        }
-        __syncwarp();
-        // dQ_i = scale sum_e dS_e K_je, two entries in flight
-        float acc[8];
-#pragma unroll
-        for (int d = 0; d < 8; ++d) acc[d] = 0.f;
-        for (int e = 0; e < maxc; e += 2) {
-            uint4 x[2];
-            float dsv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const bool ok = e + u < cnt;
-                const int j = ok ? mj[e + u] : 0;
-                dsv[u] = ok ? mds[e + u] : 0.f;
-                x[u] = ok ? __ldg(reinterpret_cast<const uint4*>(K + head + (size_t)j * HEAD_DIM) + sd)
-                          : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                float v[8];
-                unpack8(x[u], v);
-#pragma unroll
-                for (int d = 0; d < 8; ++d) acc[d] = fmaf(dsv[u], v[d], acc[d]);
-            }
-        }
-        if (cnt >= 0) {
-            float4* dst = reinterpret_cast<float4*>(io.dQ + (size_t)row * HEAD_DIM + 8 * sd);
-            dst[0] = make_float4(a.scale * acc[0], a.scale * acc[1], a.scale * acc[2], a.scale * acc[3]);
-            dst[1] = make_float4(a.scale * acc[4], a.scale * acc[5], a.scale * acc[6], a.scale * acc[7]);
-        }
-        __syncwarp();  // the lists are rewritten for the next rows
+        const GlobalRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head};
+        const GlobalRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head};
+        rows_group(a, io, sv, ws, row, cnt, bh, i, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd);
     }
 }
 
-// Four keys per warp, eight lanes per key: dK_j = scale sum dS Q_i and dV_j = sum p dO_i over key j's
-// bucket, lane s of the group loading entry e0 + s and the group sharing it by shuffles; two
-// entries (four 16-byte row loads per lane) in flight.
+// Four keys per warp (eight lanes each), rows of Q and dO gathered from L2.
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = lane >> 3, sd = lane & 7, g0 = lane & ~7;
     const int L = a.L;
     const long long R = (long long)a.B * a.H * L;
-    const size_t cap = (size_t)L * SAVE_CAP;
-    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.Q);
-    const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
     for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long key = grp * RPW + q;
         const bool kv = key < R;
-        const int n = kv ? sv.key_cnt[key] : 0;
-        const long long bh = kv ? key / L : 0;
+        const int bh = kv ? (int)(key / L) : 0;
         const size_t head = (size_t)bh * L * HEAD_DIM;
-        const size_t b0 = (size_t)bh * cap + (size_t)(kv ? ws.key_off[key] : 0);
-        const int maxn = __reduce_max_sync(0xffffffffu, n);
-        float ak[8], av[8];
-#pragma unroll
-        for (int d = 0; d < 8; ++d) ak[d] = av[d] = 0.f;
-        for (int e0 = 0; e0 < maxn; e0 += 8) {
-            const bool mine = e0 + sd < n;
-            const uint32_t ei = mine ? ws.bucket_i[b0 + e0 + sd] : 0u;
-            const float esp = mine ? ws.bucket_sp[b0 + e0 + sd] : 0.f;
-            const float eds = mine ? ws.bucket_ds[b0 + e0 + sd] : 0.f;
-#pragma unroll
-            for (int t = 0; t < 8; t += 2) {
-                uint4 xg[2], xq[2];
-                float pv[2], dv[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int src = g0 | (t + u);
-                    const uint32_t it = __shfl_sync(0xffffffffu, ei, src);
-                    const float st = __shfl_sync(0xffffffffu, esp, src);
-                    const float dt = __shfl_sync(0xffffffffu, eds, src);
-                    const bool ok = e0 + t + u < n;
-                    pv[u] = ok ? st * st : 0.f;
-                    dv[u] = ok ? dt : 0.f;
-                    xg[u] = ok ? __ldg(reinterpret_cast<const uint4*>(dO + head + (size_t)it * HEAD_DIM) + sd)
-                               : make_uint4(0u, 0u, 0u, 0u);
-                    xq[u] = ok ? __ldg(reinterpret_cast<const uint4*>(Q + head + (size_t)it * HEAD_DIM) + sd)
-                               : make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    float vg[8], vq[8];
-                    unpack8(xg[u], vg);
-                    unpack8(xq[u], vq);
-#pragma unroll
-                    for (int d = 0; d < 8; ++d) {
-                        av[d] = fmaf(pv[u], vg[d], av[d]);
-                        ak[d] = fmaf(dv[u], vq[d], ak[d]);
-                    }
-                }
-            }
-        }
-        if (kv) {
-            float4* dk = reinterpret_cast<float4*>(io.dK + (size_t)key * HEAD_DIM + 8 * sd);
-            float4* dv4 = reinterpret_cast<float4*>(io.dV + (size_t)key * HEAD_DIM + 8 * sd);
-            dk[0] = make_float4(a.scale * ak[0], a.scale * ak[1], a.scale * ak[2], a.scale * ak[3]);
-            dk[1] = make_float4(a.scale * ak[4], a.scale * ak[5], a.scale * ak[6], a.scale * ak[7]);
-            dv4[0] = make_float4(av[0], av[1], av[2], av[3]);
-            dv4[1] = make_float4(av[4], av[5], av[6], av[7]);
-        }
+        const GlobalRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q) + head};
+        const GlobalRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO) + head};
+        keys_group(a, io, sv, ws, key, kv, bh, Qr, Gr, sd, g0);
     }
 }
 
