@@ -33,6 +33,9 @@ EXPORTED = (
     "entmax_attn_bwd_saved_workspace_size",
     "entmax_attn_fwd_train",
     "entmax_attn_bwd_saved",
+    "entmax_attn_fwd_gqa",
+    "entmax_attn_fwd_train_gqa",
+    "entmax_attn_bwd_saved_gqa",
     "entmax_attn_strerror",
     "entmax_attn_device_status",
     "entmax_attn_last_cuda_error",
@@ -73,6 +76,13 @@ def _load_library() -> ctypes.CDLL:
     lib.entmax_attn_bwd_saved.restype = i
     lib.entmax_attn_bwd_saved.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, sz, vp, vp, vp, vp, vp, sz,
                                           vp]
+    lib.entmax_attn_fwd_gqa.restype = i
+    lib.entmax_attn_fwd_gqa.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, i, vp, i, vp, vp]
+    lib.entmax_attn_fwd_train_gqa.restype = i
+    lib.entmax_attn_fwd_train_gqa.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, i, vp, i, vp, vp, sz, vp]
+    lib.entmax_attn_bwd_saved_gqa.restype = i
+    lib.entmax_attn_bwd_saved_gqa.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, i, vp, vp, sz, vp, vp, vp, vp,
+                                              vp, sz, vp]
     lib.entmax_attn_strerror.restype = ctypes.c_char_p
     lib.entmax_attn_strerror.argtypes = [i]
     lib.entmax_attn_device_status.restype = i
@@ -144,16 +154,25 @@ def _mask_ptr(key_mask, B: int, L: int, device) -> int | None:
     return key_mask.data_ptr()
 
 
-def entmax_attn_fwd(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
-                    O=None, tau=None, stream=None):
-    """1.5-entmax attention forward.  Q, K, V: [B,H,L,64] bf16 or fp32 CUDA tensors.
+def _kv_heads(Q, K, grouped: bool) -> int:
+    """Key/value head count: K.shape[1] for the grouped calls, which must divide H; H otherwise."""
+    H = Q.shape[1]
+    if not grouped:
+        return H
+    if K.dim() != 4:
+        raise ValueError("K must be [B,H_kv,L,D]")
+    Hkv = K.shape[1]
+    if Hkv < 1 or H % Hkv != 0:
+        raise ValueError("H (%d) must be a multiple of K's head count (%d)" % (H, Hkv))
+    return Hkv
 
-    Returns (O, tau): O [B,H,L,64] in ``out_dtype``; tau [B,H,L] fp32 thresholds.
-    """
+
+def _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, grouped):
     B, H, L, D = Q.shape
+    Hkv = _kv_heads(Q, K, grouped)
     _check_input("Q", Q, (B, H, L, D))
-    _check_input("K", K, (B, H, L, D), Q.dtype)
-    _check_input("V", V, (B, H, L, D), Q.dtype)
+    _check_input("K", K, (B, Hkv, L, D), Q.dtype)
+    _check_input("V", V, (B, Hkv, L, D), Q.dtype)
     if scale is None:
         scale = D ** -0.5
     if out_dtype not in (torch.bfloat16, torch.float32):
@@ -166,13 +185,31 @@ def entmax_attn_fwd(Q, K, V, key_mask=None, causal=False, window=0, scale=None, 
         tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
     else:
         _check_input("tau", tau, (B, H, L), torch.float32)
-    st = lib.entmax_attn_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
-                             _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale),
-                             B, H, L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16,
-                             tau.data_ptr(), _stream_handle(stream))
+    args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
+            int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
+            L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(),
+            _stream_handle(stream))
+    name = "entmax_attn_fwd_gqa" if grouped else "entmax_attn_fwd"
+    st = getattr(lib, name)(*args)
     if st != ENTMAX_OK:
-        raise EntmaxError(st, "entmax_attn_fwd")
+        raise EntmaxError(st, name)
     return O, tau
+
+
+def entmax_attn_fwd(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
+                    O=None, tau=None, stream=None):
+    """1.5-entmax attention forward.  Q, K, V: [B,H,L,64] bf16 or fp32 CUDA tensors.
+
+    Returns (O, tau): O [B,H,L,64] in ``out_dtype``; tau [B,H,L] fp32 thresholds.
+    """
+    return _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, False)
+
+
+def entmax_attn_fwd_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
+                        O=None, tau=None, stream=None):
+    """Grouped-query forward: Q [B,H,L,64], K and V [B,H_kv,L,64] bf16 with H % H_kv == 0; query
+    head h uses key/value head h // (H // H_kv).  Returns (O, tau) as entmax_attn_fwd."""
+    return _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, True)
 
 
 def entmax_attn_bwd_workspace_size(B: int, H: int, L: int, D: int = 64) -> int:
@@ -254,15 +291,12 @@ def _byte_buffer(t, nbytes: int, device, name: str):
     return t
 
 
-def entmax_attn_fwd_train(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
-                          O=None, tau=None, saved=None, stream=None):
-    """Forward pass that also saves each row's support for entmax_attn_bwd_saved.
-
-    Returns (O, tau, saved); ``saved`` is an opaque uint8 device buffer."""
+def _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, grouped):
     B, H, L, D = Q.shape
+    Hkv = _kv_heads(Q, K, grouped)
     _check_input("Q", Q, (B, H, L, D))
-    _check_input("K", K, (B, H, L, D), Q.dtype)
-    _check_input("V", V, (B, H, L, D), Q.dtype)
+    _check_input("K", K, (B, Hkv, L, D), Q.dtype)
+    _check_input("V", V, (B, Hkv, L, D), Q.dtype)
     if scale is None:
         scale = D ** -0.5
     if out_dtype not in (torch.bfloat16, torch.float32):
@@ -277,43 +311,74 @@ def entmax_attn_fwd_train(Q, K, V, key_mask=None, causal=False, window=0, scale=
         _check_input("tau", tau, (B, H, L), torch.float32)
     nbytes = entmax_attn_saved_bytes(B, H, L, D)
     saved = _byte_buffer(saved, nbytes, Q.device, "saved")
-    st = lib.entmax_attn_fwd_train(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
-                                   _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale),
-                                   B, H, L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16,
-                                   tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(),
-                                   _stream_handle(stream))
+    args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
+            int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
+            L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(),
+            saved.data_ptr(), saved.numel() * saved.element_size(), _stream_handle(stream))
+    name = "entmax_attn_fwd_train_gqa" if grouped else "entmax_attn_fwd_train"
+    st = getattr(lib, name)(*args)
     if st != ENTMAX_OK:
-        raise EntmaxError(st, "entmax_attn_fwd_train")
+        raise EntmaxError(st, name)
     return O, tau, saved
 
 
-def entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None,
-                          dK=None, dV=None, workspace=None, stream=None):
-    """Backward pass from the supports saved by entmax_attn_fwd_train.  Returns (dQ, dK, dV) fp32."""
+def entmax_attn_fwd_train(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
+                          O=None, tau=None, saved=None, stream=None):
+    """Forward pass that also saves each row's support for entmax_attn_bwd_saved.
+
+    Returns (O, tau, saved); ``saved`` is an opaque uint8 device buffer."""
+    return _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, False)
+
+
+def entmax_attn_fwd_train_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=None,
+                              out_dtype=torch.bfloat16, O=None, tau=None, saved=None, stream=None):
+    """Grouped-query training forward (K, V [B,H_kv,L,64] bf16).  Returns (O, tau, saved)."""
+    return _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, True)
+
+
+def _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK, dV, workspace, stream, grouped):
     B, H, L, D = Q.shape
+    Hkv = _kv_heads(Q, K, grouped)
     _check_input("Q", Q, (B, H, L, D))
-    _check_input("K", K, (B, H, L, D), Q.dtype)
-    _check_input("V", V, (B, H, L, D), Q.dtype)
+    _check_input("K", K, (B, Hkv, L, D), Q.dtype)
+    _check_input("V", V, (B, Hkv, L, D), Q.dtype)
     _check_input("dO", dO, (B, H, L, D), Q.dtype)
     _check_input("tau", tau, (B, H, L), torch.float32)
     if scale is None:
         scale = D ** -0.5
     outs = []
-    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+    for name, t, heads in (("dQ", dQ, H), ("dK", dK, Hkv), ("dV", dV, Hkv)):
         if t is None:
-            t = torch.empty((B, H, L, D), dtype=torch.float32, device=Q.device)
+            t = torch.empty((B, heads, L, D), dtype=torch.float32, device=Q.device)
         else:
-            _check_input(name, t, (B, H, L, D), torch.float32)
+            _check_input(name, t, (B, heads, L, D), torch.float32)
         outs.append(t)
     ws = _byte_buffer(workspace, entmax_attn_bwd_saved_workspace_size(B, H, L, D), Q.device, "workspace")
-    st = lib.entmax_attn_bwd_saved(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
-                                   _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale),
-                                   B, H, L, D, tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(),
-                                   dO.data_ptr(), outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(),
-                                   ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
+    args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
+            int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
+            L, D, tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(), dO.data_ptr(),
+            outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(), ws.data_ptr(),
+            ws.numel() * ws.element_size(), _stream_handle(stream))
+    name = "entmax_attn_bwd_saved_gqa" if grouped else "entmax_attn_bwd_saved"
+    st = getattr(lib, name)(*args)
     if st != ENTMAX_OK:
-        raise EntmaxError(st, "entmax_attn_bwd_saved")
+        raise EntmaxError(st, name)
     return tuple(outs)
+
+
+def entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None,
+                          dK=None, dV=None, workspace=None, stream=None):
+    """Backward pass from the supports saved by entmax_attn_fwd_train.  Returns (dQ, dK, dV) fp32."""
+    return _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK, dV, workspace, stream,
+                      False)
+
+
+def entmax_attn_bwd_saved_gqa(Q, K, V, tau, saved, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None,
+                              dK=None, dV=None, workspace=None, stream=None):
+    """Grouped-query backward from entmax_attn_fwd_train_gqa's supports.  Returns dQ [B,H,L,64] and
+    dK, dV [B,H_kv,L,64] (fp32), each key/value head's gradient summed over the query heads sharing it."""
+    return _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK, dV, workspace, stream,
+                      True)
 
 
 def entmax_attn_device_status(stream=None) -> int:
@@ -334,15 +399,17 @@ class EntmaxAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, Q, K, V, key_mask=None, causal=False, window=0, scale=None):
-        O, tau, saved = entmax_attn_fwd_train(Q, K, V, key_mask, causal, window, scale)
+        grouped = K.shape[1] != Q.shape[1]  # K, V with fewer heads than Q: grouped-query attention
+        O, tau, saved = _fwd_train(Q, K, V, key_mask, causal, window, scale, torch.bfloat16, None, None, None, None,
+                                   grouped)
         ctx.save_for_backward(Q, K, V, tau, saved, key_mask if key_mask is not None else torch.empty(0))
-        ctx.cfg = (key_mask is not None, causal, window, scale)
+        ctx.cfg = (key_mask is not None, causal, window, scale, grouped)
         return O
 
     @staticmethod
     def backward(ctx, dO):
         Q, K, V, tau, saved, km = ctx.saved_tensors
-        has_mask, causal, window, scale = ctx.cfg
-        dQ, dK, dV = entmax_attn_bwd_saved(Q, K, V, tau, saved, dO.to(Q.dtype).contiguous(),
-                                           km if has_mask else None, causal, window, scale)
+        has_mask, causal, window, scale, grouped = ctx.cfg
+        dQ, dK, dV = _bwd_saved(Q, K, V, tau, saved, dO.to(Q.dtype).contiguous(), km if has_mask else None, causal,
+                                window, scale, None, None, None, None, None, grouped)
         return dQ.to(Q.dtype), dK.to(K.dtype), dV.to(V.dtype), None, None, None, None

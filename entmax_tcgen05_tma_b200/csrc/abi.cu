@@ -182,10 +182,25 @@ int entmax_attn_device_status(cudaStream_t stream) {
     return v;
 }
 
-int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-                    int window, float scale, int B, int H, int L, int D, void* O, int out_dtype, float* tau,
-                    cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+// Key/value head count check of the grouped-query entry points.  Grouped inputs must be bf16 (fp32
+// inputs would need per-tensor conversion sizes).
+int check_kv_heads(int H, int Hkv, int in_dtype) {
+    if (Hkv < 0) return ENTMAX_ERR_ARG;
+    if (H == 0 || Hkv == 0) return H == Hkv ? ENTMAX_OK : ENTMAX_ERR_ARG;
+    if (H % Hkv != 0) return ENTMAX_ERR_ARG;
+    if (Hkv != H && in_dtype != ENTMAX_BF16) return ENTMAX_ERR_UNSUPPORTED;
+    return ENTMAX_OK;
+}
+
+int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+             int window, float scale, int B, int H, int Hkv, int L, int D, void* O, int out_dtype, float* tau,
+             cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
     if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
@@ -196,7 +211,7 @@ int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, c
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -209,6 +224,21 @@ int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, c
     }
     FwdOut o{O, out_dtype == ENTMAX_F32, tau, SavedSupport{}};
     return record(launch_fwd(a, o, stream));
+}
+}  // namespace
+
+extern "C" {
+
+int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+                    int window, float scale, int B, int H, int L, int D, void* O, int out_dtype, float* tau,
+                    cudaStream_t stream) {
+    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, H, L, D, O, out_dtype, tau, stream);
+}
+
+int entmax_attn_fwd_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                        int causal, int window, float scale, int B, int H, int Hkv, int L, int D, void* O,
+                        int out_dtype, float* tau, cudaStream_t stream) {
+    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, Hkv, L, D, O, out_dtype, tau, stream);
 }
 
 size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D) {
@@ -233,7 +263,7 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H};
     BwdIO io{tau, dO, dQ, dK, dV, static_cast<float*>(workspace)};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -267,10 +297,15 @@ size_t entmax_attn_bwd_saved_workspace_size(int B, int H, int L, int D) {
     return saved_bwd_ws_bytes((long long)B * H * L);
 }
 
-int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
-                          int causal, int window, float scale, int B, int H, int L, int D, void* O, int out_dtype,
-                          float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+                   int window, float scale, int B, int H, int Hkv, int L, int D, void* O, int out_dtype, float* tau,
+                   void* saved, size_t saved_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
     if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
@@ -288,7 +323,7 @@ int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dt
     rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -303,11 +338,13 @@ int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dt
     return record(launch_fwd(a, o, stream));
 }
 
-int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
-                          int causal, int window, float scale, int B, int H, int L, int D, const float* tau,
-                          const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV,
-                          void* workspace, size_t ws_bytes, cudaStream_t stream) {
+int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+                   int window, float scale, int B, int H, int Hkv, int L, int D, const float* tau, const void* saved,
+                   size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV, void* workspace,
+                   size_t ws_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
     if (!tau || !dO || !dQ || !dK || !dV) return ENTMAX_ERR_ARG;
@@ -321,7 +358,7 @@ int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dt
     rc = record(status_ptr(&status));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv};
     BwdIO io{tau, dO, dQ, dK, dV, nullptr};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -336,6 +373,39 @@ int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dt
     }
     return record(launch_bwd_saved(a, io, carve_saved(const_cast<void*>(saved), R), carve_saved_bwd_ws(workspace, R),
                                    stream));
+}
+}  // namespace
+
+extern "C" {
+
+int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                          int causal, int window, float scale, int B, int H, int L, int D, void* O, int out_dtype,
+                          float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, H, L, D, O, out_dtype, tau, saved,
+                          saved_bytes, stream);
+}
+
+int entmax_attn_fwd_train_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                              int causal, int window, float scale, int B, int H, int Hkv, int L, int D, void* O,
+                              int out_dtype, float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, Hkv, L, D, O, out_dtype, tau,
+                          saved, saved_bytes, stream);
+}
+
+int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                          int causal, int window, float scale, int B, int H, int L, int D, const float* tau,
+                          const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV,
+                          void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, H, L, D, tau, saved, saved_bytes,
+                          dO, dQ, dK, dV, workspace, ws_bytes, stream);
+}
+
+int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                              int causal, int window, float scale, int B, int H, int Hkv, int L, int D,
+                              const float* tau, const void* saved, size_t saved_bytes, const void* dO, float* dQ,
+                              float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, Hkv, L, D, tau, saved,
+                          saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -392,7 +462,7 @@ extern "C" int entmax_attn_bwd_noalloc(const void* Q, const void* K, const void*
     float* scratch = nullptr;
     rc = record(noalloc_scratch(&scratch));
     if (rc) return rc;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H};
     BwdIO io{tau, dO, dQ, dK, dV, scratch};
     return record(launch_bwd(a, io, stream));
 }

@@ -97,10 +97,10 @@ struct GlobalRows {
 // a row the exact pass handles.
 template <class Rows>
 __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
-                                           const SavedBwdWs& ws, long long row, int cnt, int bh, int i, const Rows& Vr,
+                                           const SavedBwdWs& ws, long long row, int cnt, int bhk, const Rows& Vr,
                                            const Rows& Kr, uint16_t* mj, float* msp, float* mds, int sd) {
     const int L = a.L;
-    const size_t cap = (size_t)L * SAVE_CAP;
+    const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
     const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
     for (int e = sd; e < cnt; e += 8) {
         mj[e] = sv.row_j[(size_t)row * SAVE_CAP + e];
@@ -150,9 +150,9 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
         const float sp = msp[e];
         const float ds = sp * (mds[e] - uu);
         mds[e] = ds;
-        const size_t key = (size_t)bh * L + mj[e];
-        const size_t at = (size_t)bh * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
-        ws.bucket_i[at] = (uint32_t)i;
+        const size_t key = (size_t)bhk * L + mj[e];
+        const size_t at = (size_t)bhk * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
+        ws.bucket_i[at] = (uint32_t)row;
         ws.bucket_sp[at] = sp;
         ws.bucket_ds[at] = ds;
     }
@@ -191,12 +191,12 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
 // 16-byte pieces each per lane) in flight.  valid = false: no key (the group still takes part).
 template <class Rows>
 __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
-                                           const SavedBwdWs& ws, long long key, bool valid, int bh, const Rows& Qr,
+                                           const SavedBwdWs& ws, long long key, bool valid, int bhk, const Rows& Qr,
                                            const Rows& Gr, int sd, int g0) {
     const int L = a.L;
-    const size_t cap = (size_t)L * SAVE_CAP;
+    const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
     const int n = valid ? sv.key_cnt[key] : 0;
-    const size_t b0 = (size_t)bh * cap + (size_t)(valid ? ws.key_off[key] : 0);
+    const size_t b0 = (size_t)bhk * cap + (size_t)(valid ? ws.key_off[key] : 0);
     const int maxn = __reduce_max_sync(0xffffffffu, n);
     float ak[8], av[8];
 #pragma unroll
@@ -258,12 +258,11 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
     for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long row = grp * RPW + q;
         const int cnt = row < R ? sv.row_cnt[row] : -1;
-        const int bh = row < R ? (int)(row / L) : 0;
-        const int i = (int)(row - (long long)bh * L);
-        const size_t head = (size_t)bh * L * HEAD_DIM;
+        const int bhk = row < R ? kv_head_of((int)(row / L), a.H, a.Hkv) : 0;
+        const size_t head = (size_t)bhk * L * HEAD_DIM;
         const GlobalRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head};
         const GlobalRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head};
-        rows_group(a, io, sv, ws, row, cnt, bh, i, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd);
+        rows_group(a, io, sv, ws, row, cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd);
     }
 }
 
@@ -273,15 +272,15 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnAr
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = lane >> 3, sd = lane & 7, g0 = lane & ~7;
     const int L = a.L;
-    const long long R = (long long)a.B * a.H * L;
-    for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
+    const long long Rk = (long long)a.B * a.Hkv * L;  // keys
+    // bucket entries name their query row by its global index, so Q and dO are read from the base
+    const GlobalRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q)};
+    const GlobalRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO)};
+    for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < Rk; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long key = grp * RPW + q;
-        const bool kv = key < R;
-        const int bh = kv ? (int)(key / L) : 0;
-        const size_t head = (size_t)bh * L * HEAD_DIM;
-        const GlobalRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q) + head};
-        const GlobalRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO) + head};
-        keys_group(a, io, sv, ws, key, kv, bh, Qr, Gr, sd, g0);
+        const bool kv = key < Rk;
+        const int bhk = kv ? (int)(key / L) : 0;
+        keys_group(a, io, sv, ws, key, kv, bhk, Qr, Gr, sd, g0);
     }
 }
 
@@ -334,7 +333,8 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
         const long long bh = row / L;
         const int i = (int)(row - bh * L);
         const int b = (int)(bh / a.H);
-        const size_t head = (size_t)bh * L * HEAD_DIM;
+        const int bhk = kv_head_of((int)bh, a.H, a.Hkv);
+        const size_t head = (size_t)bhk * L * HEAD_DIM;  // K and V rows of the row's KV head
         __syncthreads();
         if (tid < HEAD_DIM) {
             qf[tid] = __bfloat162float(Q[(size_t)row * HEAD_DIM + tid]);
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
         for (int e = ph; e < span; e += PH) {
             const float sp = sbuf[e];
             if (sp > 0.f) {
-                const size_t key = (size_t)bh * L + lo + e;
+                const size_t key = (size_t)bhk * L + lo + e;
                 const float ds = sp * (sbuf[L + e] - u);
                 acc = fmaf(ds, __bfloat162float(K[key * HEAD_DIM + d]), acc);
                 atomicAdd(io.dK + key * HEAD_DIM + d, a.scale * ds * qf[d]);
@@ -439,7 +439,7 @@ SavedBwdWs carve_saved_bwd_ws(void* base, long long R) {
 cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv, const SavedBwdWs& ws,
                              cudaStream_t stream) {
     const long long R = (long long)a.B * a.H * a.L;
-    key_scan_kernel<<<a.B * a.H, 1024, 0, stream>>>(sv.key_cnt, ws.key_off, ws.key_cur, a.L);
+    key_scan_kernel<<<a.B * a.Hkv, 1024, 0, stream>>>(sv.key_cnt, ws.key_off, ws.key_cur, a.L);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -449,7 +449,9 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
     saved_rows_kernel<<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    saved_keys_kernel<<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    const long long Rk = (long long)a.B * a.Hkv * a.L;
+    const unsigned kgrid = (unsigned)std::max<long long>(1, std::min<long long>((Rk + ROW_WARPS * RPW - 1) / (ROW_WARPS * RPW), (long long)sms * 8));
+    saved_keys_kernel<<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int smem = 2 * a.L * (int)sizeof(float);

@@ -202,7 +202,8 @@ struct Pipe {
     static __device__ __forceinline__ void producer(Ctl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
                                                     const CUtensorMap* map_b, int bh, int a_row0,
                                                     const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b,
-                                                    int njobs, int n1 = -1, int s1 = 1) {
+                                                    int njobs, int n1 = -1, int s1 = 1, int bh_b = -1) {
+        if (bh_b < 0) bh_b = bh;  // head (third coordinate) of the streamed operand
         if (n1 < 0) {
             n1 = ctl->nblk;
             s1 = 1;
@@ -216,7 +217,7 @@ struct Pipe {
             if (!wait_bounded(smem_u32(&ctl->empty_b[s]), ph ^ 1u, &ctl->abort_flag, wc)) break;
             const int e = n < n1 ? n * s1 : n - n1;
             mbar_arrive_expect_tx(smem_u32(&ctl->full_b[s]), BLK_BYTES);
-            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[e] & ~FULL_BLOCK) * BLK, bh,
+            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[e] & ~FULL_BLOCK) * BLK, bh_b,
                         smem_u32(&ctl->full_b[s]));
             ++issued;
         }

@@ -249,7 +249,7 @@ __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4
 // rows redone on CUDA cores (mode 2) or with more than SAVE_CAP entries are marked unsaved.
 __device__ __forceinline__ void save_row_support(const SavedSupport& sv, const float* cv, const uint16_t* cj,
                                                  const int* supp_cnt, int r, int h, int mode, size_t head_row0,
-                                                 int i, int L) {
+                                                 size_t key_row0, int i, int L) {
     const int s0 = supp_cnt[r], s1 = supp_cnt[TILE + r];
     const bool saved = mode != 2 && s0 + s1 <= SAVE_CAP;
     if (i >= L) return;
@@ -268,7 +268,7 @@ __device__ __forceinline__ void save_row_support(const SavedSupport& sv, const f
         const int j = cj[(slot0 + e) * TILE + r];
         sv.row_j[row * SAVE_CAP + base + e] = (uint16_t)j;
         sv.row_sp[row * SAVE_CAP + base + e] = sqrtf(cv[(slot0 + e) * TILE + r]);
-        atomicAdd(sv.key_cnt + head_row0 + j, 1);
+        atomicAdd(sv.key_cnt + key_row0 + j, 1);
     }
 }
 
@@ -308,11 +308,11 @@ __device__ __forceinline__ float block_max(float a, float* red) {
 // Phase 4: the whole CTA recomputes one row exactly on CUDA cores.
 __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                                           const __nv_bfloat16* __restrict__ V, const uint32_t* bits, float* sbuf,
-                                          float* red, int bh, int i, int L, int causal, int window, float scale,
+                                          float* red, int bh, int bhk, int i, int L, int causal, int window, float scale,
                                           int nallow, void* O, int out_f32, float* tau) {
     const int tid = threadIdx.x;
     float* qf = red + 64;  // 64 floats (red[0..63] holds reduction partials)
-    const size_t head = (size_t)bh * L * HEAD_DIM;
+    const size_t head = (size_t)bh * L * HEAD_DIM, kv_head = (size_t)bhk * L * HEAD_DIM;
     __syncthreads();
     if (tid < HEAD_DIM) qf[tid] = __bfloat162float(Q[head + (size_t)i * HEAD_DIM + tid]);
     __syncthreads();
@@ -324,7 +324,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         const int j = lo + e;
         float s = -INFINITY;
         if ((bits[j >> 5] >> (j & 31)) & 1u) {
-            const uint4* kr = reinterpret_cast<const uint4*>(K + head + (size_t)j * HEAD_DIM);
+            const uint4* kr = reinterpret_cast<const uint4*>(K + kv_head + (size_t)j * HEAD_DIM);
             float acc = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -401,7 +401,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         const float s = sbuf[e];
         if (s > t) {
             const float h = 0.5f * (s - t);
-            acc = fmaf(h * h, __bfloat162float(V[head + (size_t)(lo + e) * HEAD_DIM + d]), acc);
+            acc = fmaf(h * h, __bfloat162float(V[kv_head + (size_t)(lo + e) * HEAD_DIM + d]), acc);
         }
     }
     __syncthreads();
@@ -426,7 +426,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
 __device__ __forceinline__ int half_block(int p, int m, int mA) { return m < mA ? 2 * (p + 2 * m) : p + 2 * (m - mA); }
 
 __device__ __noinline__ void produce_half(PipeCtl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
-                                          const CUtensorMap* map_b, int bh, int a_row0, const uint16_t* blk_list,
+                                          const CUtensorMap* map_b, int bh, int bhk, int a_row0, const uint16_t* blk_list,
                                           uint8_t* smem_a, uint8_t* smem_b, int p, int mA, int mB) {
     if (p == 0) {
         mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
@@ -439,7 +439,7 @@ __device__ __noinline__ void produce_half(PipeCtl* ctl, const WaitCfg& wc, const
         if (!wait_bounded(smem_u32(&ctl->empty_b[st]), ph ^ 1u, &ctl->abort_flag, wc)) break;
         mbar_arrive_expect_tx(smem_u32(&ctl->full_b[st]), BLK_BYTES);
         tma_load_3d(smem_u32(smem_b + st * BLK_BYTES), map_b, 0, (int)(blk_list[half_block(p, m, mA)] & ~FULL_BLOCK) * BLK,
-                    bh, smem_u32(&ctl->full_b[st]));
+                    bhk, smem_u32(&ctl->full_b[st]));
         ++issued;
     }
     if (P::aborted(ctl)) {
@@ -504,9 +504,10 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int L = args.L;
     const int tile = blockIdx.x, bh = blockIdx.y;
     const int b = bh / args.H;
+    const int bhk = kv_head_of(bh, args.H, args.Hkv);  // K/V head
     const int i0 = tile * TILE;
     const WaitCfg wc{args.status, args.timeout_ns};
-    const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(args.V) + (size_t)bh * L * HEAD_DIM;
+    const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(args.V) + (size_t)bhk * L * HEAD_DIM;
 
     if (tid == 0) {
         mbar_init(smem_u32(vbar), 1);
@@ -553,9 +554,9 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const int p = warp == WARP_PRODUCER ? 0 : 1;
         if (lane == 0) {
             if (resident) {
-                if (p == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs);
+                if (p == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs, -1, 1, bhk);
             } else {
-                produce_half(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, p, p ? mA1 : mA0, p ? mB1 : mB0);
+                produce_half(ctl, wc, &map_q, &map_k, bh, bhk, i0, blk_list, smem_a, smem_b, p, p ? mA1 : mA0, p ? mB1 : mB0);
             }
         }
         __syncwarp();
@@ -691,7 +692,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     if (warp == WARP_PRODUCER && lane == 0 && v_staged) {
         mbar_arrive_expect_tx(smem_u32(vbar), (uint32_t)(nblk * BLK_BYTES));
         for (int s = 0; s < nblk; ++s)
-            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), &map_v, 0, (int)(blk_list[s] & ~FULL_BLOCK) * BLK, bh,
+            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), &map_v, 0, (int)(blk_list[s] & ~FULL_BLOCK) * BLK, bhk,
                         smem_u32(vbar));
     }
 
@@ -768,7 +769,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             if (h == 0 && i < L) out.tau[(size_t)bh * L + i] = INFINITY;  // no allowed key: O_i = 0
         }
         __syncwarp();
-        if (out.save.row_cnt) save_row_support(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, i, L);
+        if (out.save.row_cnt)
+            save_row_support(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, (size_t)bhk * L, i, L);
 
         // ---------------- phase 3: O_i = sum_j p_ij V_j over the row's whole support (both
         // partitions); thread h of the pair accumulates dimensions [32 h, 32 h + 32) in registers
@@ -847,7 +849,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 const int rr = wd * 32 + __ffs(mask) - 1;
                 mask &= mask - 1;
                 fallback_row(reinterpret_cast<const __nv_bfloat16*>(args.Q), reinterpret_cast<const __nv_bfloat16*>(args.K),
-                             reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, bh, i0 + rr, L,
+                             reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, bh, bhk, i0 + rr, L,
                              args.causal, args.window, scale, rows[rr].nallow + rows[TILE + rr].nallow, out.O,
                              out.out_f32, out.tau);
             }
@@ -870,9 +872,9 @@ cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream) 
     CUtensorMap mq, mk, mv;
     cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L, TILE);
     if (e != cudaSuccess) return e;
-    e = make_tile_map(&mk, a.K, a.B * a.H, a.L, BLK);
+    e = make_tile_map(&mk, a.K, a.B * a.Hkv, a.L, BLK);
     if (e != cudaSuccess) return e;
-    e = make_tile_map(&mv, a.V, a.B * a.H, a.L, BLK);
+    e = make_tile_map(&mv, a.V, a.B * a.Hkv, a.L, BLK);
     if (e != cudaSuccess) return e;
     e = ensure_smem_attr(reinterpret_cast<const void*>(entmax_fwd_kernel), SMEM_BYTES, 0);
     if (e != cudaSuccess) return e;

@@ -10,7 +10,7 @@ namespace entmax {
 
 struct AttnArgs {
     const void* Q;           // [B,H,L,64] bf16
-    const void* K;
+    const void* K;           // [B,Hkv,L,64] bf16
     const void* V;
     const uint8_t* key_mask; // [B,L] or null
     int B, H, L;
@@ -18,7 +18,12 @@ struct AttnArgs {
     float scale;
     int* status;             // device status word
     unsigned long long timeout_ns;
+    int Hkv;                 // key/value heads (H % Hkv == 0); query head h of batch b reads KV head
+                             // b * Hkv + h / (H / Hkv) -- grouped-query attention when Hkv < H
 };
+
+// Key/value head of query head bh = b * H + h.
+__host__ __device__ __forceinline__ int kv_head_of(int bh, int H, int Hkv) { return (bh / H) * Hkv + (bh % H) / (H / Hkv); }
 
 // Saved support of the forward pass, consumed by the support-list backward.  R = B*H*L rows.
 constexpr int SAVE_CAP = 64;  // support entries kept per row
@@ -26,7 +31,7 @@ struct SavedSupport {
     int* row_cnt;            // [R] entries of row, or -1 when the row's support was not saved
     uint16_t* row_j;         // [R][SAVE_CAP] key index of each entry
     float* row_sp;           // [R][SAVE_CAP] sqrt(p_ij) = (S_ij - tau_i)/2 of each entry
-    int* key_cnt;            // [R] rows whose support holds key j (zeroed before the forward)
+    int* key_cnt;            // [B*Hkv*L] rows whose support holds key j of a KV head (zeroed before the forward)
     int* unsaved_cnt;        // [1] rows whose support was not saved (zeroed before the forward)
     int* unsaved_rows;       // [R] their row ids
 };

@@ -33,6 +33,11 @@ class Workload:
     len_range: tuple[int, int] | None = None  # key-padding valid length U[lo, hi]
     backward: bool = True
     fp32_inputs: bool = False
+    H_kv: int | None = None  # key/value heads (grouped-query attention); None: H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.H_kv is None else self.H_kv
 
     def with_shape(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -53,16 +58,16 @@ WORKLOADS: dict[int, Workload] = {
 def make_inputs(w: Workload, seed: int | None = None) -> dict:
     """Draw the workload's tensors on the CPU.
 
-    Returns a dict with Q, K, V, dO (bf16, or fp32 for fp32-input workloads),
+    Returns a dict with Q, dO [B,H,L,D] and K, V [B,H_kv,L,D] (bf16, or fp32 for fp32-input workloads),
     ``lengths`` (int64 [B] or None) and ``key_mask`` (uint8 [B, L] or None).
     """
     gen = torch.Generator(device="cpu")
     gen.manual_seed(1000 + w.wid if seed is None else seed)
-    shape = (w.B, w.H, w.L, w.D)
     dt = torch.float32 if w.fp32_inputs else torch.bfloat16
     out = {}
     for name in ("Q", "K", "V", "dO"):
-        out[name] = torch.randn(shape, generator=gen, dtype=torch.float32).to(dt)
+        heads = w.kv_heads if name in ("K", "V") else w.H
+        out[name] = torch.randn((w.B, heads, w.L, w.D), generator=gen, dtype=torch.float32).to(dt)
     if w.len_range is not None:
         lo, hi = w.len_range
         lengths = torch.randint(lo, hi + 1, (w.B,), generator=gen, dtype=torch.int64)

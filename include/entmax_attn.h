@@ -135,6 +135,39 @@ ENTMAX_API int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V
                                      void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Grouped-query attention.  The page "svd-sst2-roberta-adasplash" (section 3, the step-by-step
+ * tensor trace, and the attention layer's forward in section 4) projects keys and values to H_kv
+ * heads and repeats each of them H/H_kv times before the scores, so query head h of batch b attends
+ * with key/value head b*H_kv + h/(H/H_kv).  These three entry points compute exactly what
+ * entmax_attn_fwd, entmax_attn_fwd_train and entmax_attn_bwd_saved compute on the repeated K and V,
+ * without materialising the repeat:
+ *   K, V       [B, H_kv, L, 64] bf16 (in_dtype must be ENTMAX_BF16 when H_kv < H;
+ *              ENTMAX_F32 returns ENTMAX_ERR_UNSUPPORTED there).
+ *   Q, O, tau, dO, dQ, saved: as in the non-grouped calls, over B*H query rows.
+ *   dK, dV     [B, H_kv, L, 64] fp32: the gradient of each key/value head, i.e. the sum over the
+ *              H/H_kv query heads that share it.
+ *   H_kv       1 <= H_kv <= H and H % H_kv == 0, else ENTMAX_ERR_ARG (H_kv = H is the plain
+ *              multi-head case; H = 0 requires H_kv = 0).
+ *   saved / workspace sizes: entmax_attn_saved_bytes(B,H,L,D) and
+ *              entmax_attn_bwd_saved_workspace_size(B,H,L,D) with the QUERY head count H.
+ */
+ENTMAX_API int entmax_attn_fwd_gqa(const void* Q, const void* K, const void* V, int in_dtype,
+                                   const uint8_t* key_mask, int causal, int window, float scale,
+                                   int B, int H, int H_kv, int L, int D,
+                                   void* O, int out_dtype, float* tau, cudaStream_t stream);
+ENTMAX_API int entmax_attn_fwd_train_gqa(const void* Q, const void* K, const void* V, int in_dtype,
+                                         const uint8_t* key_mask, int causal, int window, float scale,
+                                         int B, int H, int H_kv, int L, int D,
+                                         void* O, int out_dtype, float* tau,
+                                         void* saved, size_t saved_bytes, cudaStream_t stream);
+ENTMAX_API int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const void* V, int in_dtype,
+                                         const uint8_t* key_mask, int causal, int window, float scale,
+                                         int B, int H, int H_kv, int L, int D,
+                                         const float* tau, const void* saved, size_t saved_bytes,
+                                         const void* dO, float* dQ, float* dK, float* dV,
+                                         void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Allocation-free variant of entmax_attn_bwd (no counterpart in the AdaSplash pages; it exists for
  * this library's users).  Some callers cannot allocate device memory at the point where they run
  * the backward pass: engines that plan all memory ahead of time and forbid allocation inside their

@@ -209,3 +209,46 @@ def attn_bwd(Q, K, V, dO, key_mask=None, causal=False, window=0, scale=0.125):
     B, H, L, D = np.shape(Q)
     dQ, dK, dV = attn_bwd_heads(Q, K, V, dO, np.arange(B * H), key_mask, causal, window, scale)
     return dQ.reshape(B, H, L, D), dK.reshape(B, H, L, D), dV.reshape(B, H, L, D)
+
+
+# --------------------------------------------------------------------------
+# grouped-query attention
+# --------------------------------------------------------------------------
+def repeat_kv(X, n_rep: int) -> np.ndarray:
+    """[B, H_kv, L, D] -> [B, H_kv*n_rep, L, D]: each key/value head copied n_rep times in a row, so
+    query head h reads key/value head h // n_rep.  Page "svd-sst2-roberta-adasplash", section 3 (the
+    grouped-query repeat step of the tensor trace, taken before the scores) and section 4 (the
+    attention layer's forward repeats k and v by H // H_kv)."""
+    X = _f64(X)
+    return np.repeat(X, int(n_rep), axis=1)
+
+
+def _n_rep(Q, K) -> int:
+    H, Hkv = np.shape(Q)[1], np.shape(K)[1]
+    if Hkv < 1 or H % Hkv:
+        raise ValueError("query heads (%d) must be a multiple of key/value heads (%d)" % (H, Hkv))
+    return H // Hkv
+
+
+def attn_fwd_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=0.125, tau_method="sort"):
+    """Grouped-query forward: K, V [B,H_kv,L,D] repeated to H heads, then attn_fwd.  (O, tau)."""
+    r = _n_rep(Q, K)
+    return attn_fwd(Q, repeat_kv(K, r), repeat_kv(V, r), key_mask, causal, window, scale, tau_method)
+
+
+def attn_fwd_rows_gqa(Q, K, V, row_ids, key_mask=None, causal=False, window=0, scale=0.125,
+                      tau_method="sort", n_iter=25):
+    """attn_fwd_rows on the repeated K and V (row id = (b*H + h)*L + i over the query heads)."""
+    r = _n_rep(Q, K)
+    return attn_fwd_rows(Q, repeat_kv(K, r), repeat_kv(V, r), row_ids, key_mask, causal, window, scale,
+                         tau_method, n_iter)
+
+
+def attn_bwd_gqa(Q, K, V, dO, key_mask=None, causal=False, window=0, scale=0.125):
+    """Grouped-query backward.  The repeat copies each key/value head to n_rep query heads, so by the
+    chain rule its gradient is the sum of the copies' gradients over those heads.  Returns dQ
+    [B,H,L,D] and dK, dV [B,H_kv,L,D]."""
+    r = _n_rep(Q, K)
+    B, Hkv, L, D = np.shape(K)
+    dQ, dKr, dVr = attn_bwd(Q, repeat_kv(K, r), repeat_kv(V, r), dO, key_mask, causal, window, scale)
+    return dQ, dKr.reshape(B, Hkv, r, L, D).sum(axis=2), dVr.reshape(B, Hkv, r, L, D).sum(axis=2)

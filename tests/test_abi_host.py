@@ -143,3 +143,39 @@ def test_training_path_argument_checks():
     nb = list(bargs)
     nb[16] = P + 4
     assert b(*nb) == E.ENTMAX_ERR_ARG
+
+
+def _gqa_calls(H, Hkv, in_dtype=0, B=1, L=64, D=64):
+    """Status of the three grouped-query entry points for one head configuration."""
+    R = max(B * H * L, 1)
+    need = E.entmax_attn_saved_bytes(1, 1, R)
+    ws = E.entmax_attn_bwd_saved_workspace_size(1, 1, R)
+    f = E.lib.entmax_attn_fwd_gqa(P, P, P, in_dtype, None, 0, 0, 0.125, B, H, Hkv, L, D, P, 0, P, None)
+    t = E.lib.entmax_attn_fwd_train_gqa(P, P, P, in_dtype, None, 0, 0, 0.125, B, H, Hkv, L, D, P, 0, P, P, need,
+                                        None)
+    b = E.lib.entmax_attn_bwd_saved_gqa(P, P, P, in_dtype, None, 0, 0, 0.125, B, H, Hkv, L, D, P, P, need, P, P, P,
+                                        P, P, ws, None)
+    return f, t, b
+
+
+@pytest.mark.parametrize("H,Hkv,in_dtype,B,code", [
+    (4, 3, 0, 1, E.ENTMAX_ERR_ARG),           # H not a multiple of H_kv
+    (4, 0, 0, 1, E.ENTMAX_ERR_ARG),
+    (4, -2, 0, 1, E.ENTMAX_ERR_ARG),
+    (4, 8, 0, 1, E.ENTMAX_ERR_ARG),           # more key/value heads than query heads
+    (0, 1, 0, 1, E.ENTMAX_ERR_ARG),
+    (8, 2, 1, 1, E.ENTMAX_ERR_UNSUPPORTED),   # fp32 inputs with grouped heads
+    (0, 0, 0, 1, E.ENTMAX_OK),
+    (8, 2, 0, 0, E.ENTMAX_OK),                # empty batch: a no-op
+])
+def test_gqa_argument_checks(H, Hkv, in_dtype, B, code):
+    assert _gqa_calls(H, Hkv, in_dtype, B) == (code, code, code)
+
+
+def test_binding_rejects_bad_kv_head_count():
+    import torch
+
+    q = torch.zeros(1, 6, 8, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 4, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        E.entmax_attn_fwd_gqa(q, k, k)

@@ -383,3 +383,71 @@ def test_backward_matches_finite_differences(causal, window, masked):
         if done == 3:
             break
     assert done >= 1
+
+
+# ------------------------------------------------------- grouped-query attention
+def test_gqa_head_mapping_by_constant_values():
+    """V constant per key/value head g -> every output row of a query head reading g equals that
+    constant (the weights sum to one), which fixes the head map h -> h // (H/H_kv) without the oracle."""
+    B, H, Hkv, L, D = 2, 6, 2, 12, 4
+    rng = np.random.default_rng(21)
+    Q = orc.round_bf16(rng.normal(0, 1, (B, H, L, D)).astype(np.float32))
+    K = orc.round_bf16(rng.normal(0, 1, (B, Hkv, L, D)).astype(np.float32))
+    c = np.arange(B * Hkv, dtype=float).reshape(B, Hkv) + 1.0
+    V = np.broadcast_to(c[:, :, None, None], (B, Hkv, L, D)).copy()
+    O, _ = orc.attn_fwd_gqa(Q, K, V, causal=True, scale=0.5)
+    for b in range(B):
+        for h in range(H):
+            np.testing.assert_allclose(O[b, h], c[b, h // (H // Hkv)], atol=1e-13)
+
+
+def test_gqa_single_kv_head_equals_shared_keys():
+    """H_kv = 1: every query head sees the same K and V, as plain attention with K, V broadcast."""
+    B, H, L, D = 1, 3, 10, 8
+    Q, K, V, _ = _rand_qkv(22, B, H, L, D)
+    K1, V1 = K[:, :1], V[:, :1]
+    O, tau = orc.attn_fwd_gqa(Q, K1, V1, scale=0.4)
+    for h in range(H):
+        Oh, th = orc.attn_fwd(Q[:, h:h + 1], K1, V1, scale=0.4)
+        np.testing.assert_array_equal(O[:, h], Oh[:, 0])
+        np.testing.assert_array_equal(tau[:, h], th[:, 0])
+
+
+def test_gqa_backward_matches_finite_differences():
+    """Central differences of <dO, O> w.r.t. the SHARED key/value heads: pins the sum over the group."""
+    B, H, Hkv, L, D = 1, 4, 2, 6, 3
+    scale = 0.7
+    done = 0
+    for seed in range(40):
+        rng = np.random.default_rng(300 + seed)
+        Q = rng.normal(0, 1, (B, H, L, D))
+        K = rng.normal(0, 1, (B, Hkv, L, D))
+        V = rng.normal(0, 1, (B, Hkv, L, D))
+        dO = rng.normal(0, 1, (B, H, L, D))
+        O, tau = orc.attn_fwd_gqa(Q, K, V, None, True, 0, scale)
+        ok = True
+        for h in range(H):
+            S = scale * Q[0, h] @ K[0, h // (H // Hkv)].T
+            a = _allowed(L, True, 0, None)
+            if np.abs(S - tau[0, h][:, None])[a].min() < 1e-3:
+                ok = False
+        if not ok:
+            continue
+        dQ, dK, dV = orc.attn_bwd_gqa(Q, K, V, dO, None, True, 0, scale)
+        assert dK.shape == K.shape and dV.shape == V.shape and dQ.shape == Q.shape
+        eps = 1e-6
+        for X, dX in ((Q, dQ), (K, dK), (V, dV)):
+            num = np.zeros_like(X)
+            for idx in np.ndindex(X.shape):
+                old = X[idx]
+                X[idx] = old + eps
+                Lp = np.sum(dO * orc.attn_fwd_gqa(Q, K, V, None, True, 0, scale)[0])
+                X[idx] = old - eps
+                Lm = np.sum(dO * orc.attn_fwd_gqa(Q, K, V, None, True, 0, scale)[0])
+                X[idx] = old
+                num[idx] = (Lp - Lm) / (2 * eps)
+            np.testing.assert_allclose(dX, num, atol=2e-6)
+        done += 1
+        if done == 2:
+            break
+    assert done >= 1
