@@ -17,7 +17,13 @@
  *   backward: closed-form Jacobian of section 2.4,
  *     dL/dS_j = 1[j in S] sqrt(p_j) (g_j - sum_k sqrt(p_k) g_k / sum_k sqrt(p_k))
  *
- * tau is obtained two ways:
+ * General alpha in (1, 2] (the pages' alpha-entmax by bisection, page
+ * "svd-sst2-roberta-adasplash", section 4, the entmax_bisect routine): with
+ * a = alpha - 1, p_ij = max(0, a (S_ij - tau_i))^(1/a), sum_j p_ij = 1 (tau in
+ * score units; alpha = 1.5 gives the formula above), and the Jacobian
+ * dp_i/ds_j = w_i (delta_ij - w_j / sum_k w_k) with w = p^(2 - alpha).
+ *
+ * tau (alpha = 1.5) is obtained two ways:
  *   - eo_tau_sort:   exact, from the closed form on a sorted row (on a support
  *                    of size k, sum (z_i - tau)^2 = 4 is a quadratic in tau);
  *   - eo_tau_bisect: the pages' bisection (Theorem 2), 25 halvings of a
@@ -189,6 +195,103 @@ void eo_entmax15_jvp(const double* p, const double* g, int n, double* ds)
 }
 
 /* ------------------------------------------------------------------------ */
+/* alpha-entmax, alpha in (1, 2].  a = alpha - 1.                            */
+/*   g_alpha(tau) = sum_i max(0, a (s_i - tau))^(1/a)                         */
+/* is continuous and strictly decreasing where positive, so g_alpha = 1 has  */
+/* one root.  The max alone gives g_alpha(max - 1/a) >= 1; n equal terms of  */
+/* 1/n give g_alpha(max - n^(-a)/a) <= 1 (every term is at most 1/n there).  */
+/* The root is found by halving that bracket until the midpoint no longer    */
+/* changes in fp64 (at most 2000 halvings): the exact root to rounding.      */
+/* ------------------------------------------------------------------------ */
+double eo_g_alpha(const double* s, int n, double tau, double alpha)
+{
+    const double a = alpha - 1.0;
+    double acc = 0.0;
+    for (int i = 0; i < n; ++i) {
+        double t = a * (s[i] - tau);
+        if (t > 0.0) acc += pow(t, 1.0 / a);
+    }
+    return acc;
+}
+
+double eo_tau_alpha(const double* s, int n, double alpha)
+{
+    if (n <= 0) return INFINITY;
+    const double a = alpha - 1.0;
+    double m = s[0];
+    for (int i = 1; i < n; ++i) if (s[i] > m) m = s[i];
+    double lo = m - 1.0 / a, hi = m - pow((double)n, -a) / a;
+    for (int it = 0; it < 2000; ++it) {
+        double mid = 0.5 * (lo + hi);
+        if (mid <= lo || mid >= hi) break;
+        if (eo_g_alpha(s, n, mid, alpha) > 1.0) lo = mid;
+        else hi = mid;
+    }
+    return 0.5 * (lo + hi);
+}
+
+/* The pages' procedure for general alpha on the same bracket: n_iter halvings, final midpoint. */
+double eo_tau_alpha_bisect(const double* s, int n, double alpha, int n_iter)
+{
+    if (n <= 0) return INFINITY;
+    const double a = alpha - 1.0;
+    double m = s[0];
+    for (int i = 1; i < n; ++i) if (s[i] > m) m = s[i];
+    double lo = m - 1.0 / a, hi = m - pow((double)n, -a) / a;
+    for (int it = 0; it < n_iter; ++it) {
+        double mid = 0.5 * (lo + hi);
+        if (eo_g_alpha(s, n, mid, alpha) > 1.0) lo = mid;
+        else hi = mid;
+    }
+    return 0.5 * (lo + hi);
+}
+
+/* p_i = max(0, a (s_i - tau))^(1/a). */
+void eo_entmax_alpha(const double* s, int n, double tau, double alpha, double* p)
+{
+    const double a = alpha - 1.0;
+    for (int i = 0; i < n; ++i) {
+        double t = a * (s[i] - tau);
+        p[i] = t > 0.0 ? pow(t, 1.0 / a) : 0.0;
+    }
+}
+
+/* Jacobian-vector product of alpha-entmax: w_j = p_j^(2 - alpha) on the    */
+/* support, ds_j = w_j (g_j - sum_k w_k g_k / sum_k w_k).                   */
+void eo_entmax_alpha_jvp(const double* p, const double* g, int n, double alpha, double* ds)
+{
+    double r = 0.0, acc = 0.0;
+    for (int k = 0; k < n; ++k) {
+        if (p[k] <= 0.0) continue;
+        double w = pow(p[k], 2.0 - alpha);
+        r += w;
+        acc += w * g[k];
+    }
+    double u = r > 0.0 ? acc / r : 0.0;
+    for (int j = 0; j < n; ++j) ds[j] = p[j] > 0.0 ? pow(p[j], 2.0 - alpha) * (g[j] - u) : 0.0;
+}
+
+/* tau and p of one row for any alpha: the closed form (alpha = 1.5, sort)  */
+/* or the converged bisection; tau_method 1 = the pages' n_iter halvings.   */
+static double row_tau(const double* s, int n, double alpha, int tau_method, int n_iter)
+{
+    if (alpha == 1.5) {
+        double tau;
+        if (tau_method == 0) eo_tau_sort(s, n, &tau);
+        else tau = eo_tau_bisect(s, n, n_iter > 0 ? n_iter : 25);
+        return tau;
+    }
+    if (tau_method == 0) return eo_tau_alpha(s, n, alpha);
+    return eo_tau_alpha_bisect(s, n, alpha, n_iter > 0 ? n_iter : 25);
+}
+
+static void row_probs(const double* s, int n, double tau, double alpha, double* p)
+{
+    if (alpha == 1.5) eo_entmax15(s, n, tau, p);
+    else eo_entmax_alpha(s, n, tau, alpha, p);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Attention.  Tensors are [B,H,L,D] row-major fp64; key_mask is [B,L]      */
 /* (1 = valid) or NULL for all valid.                                       */
 /* ------------------------------------------------------------------------ */
@@ -204,7 +307,7 @@ static int allowed(const unsigned char* key_mask, int b, int L, int causal, int 
 /* 1 = bisection (25 iterations unless n_iter > 0 given).  Scratch s, idx   */
 /* and p hold L entries each.                                               */
 static double row_forward(const double* Q, const double* K, const double* V,
-                          const unsigned char* key_mask, int causal, int window, double scale,
+                          const unsigned char* key_mask, int causal, int window, double scale, double alpha,
                           int H, int L, int D, int b, int h, int i, int tau_method, int n_iter,
                           double* s, int* idx, double* p, double* O_row)
 {
@@ -222,10 +325,8 @@ static double row_forward(const double* Q, const double* K, const double* V,
     }
     for (int t = 0; t < D; ++t) O_row[t] = 0.0;
     if (n == 0) return INFINITY;
-    double tau;
-    if (tau_method == 0) eo_tau_sort(s, n, &tau);
-    else tau = eo_tau_bisect(s, n, n_iter > 0 ? n_iter : 25);
-    eo_entmax15(s, n, tau, p);
+    const double tau = row_tau(s, n, alpha, tau_method, n_iter);
+    row_probs(s, n, tau, alpha, p);
     for (int e = 0; e < n; ++e) {
         if (p[e] == 0.0) continue;
         const double* v = V + head + (size_t)idx[e] * D;
@@ -237,7 +338,7 @@ static double row_forward(const double* Q, const double* K, const double* V,
 /* Forward for a list of rows, row id = (b*H + h)*L + i.  O_rows is         */
 /* [nrows, D], tau_rows [nrows].                                            */
 void eo_attn_fwd_rows(const double* Q, const double* K, const double* V,
-                      const unsigned char* key_mask, int causal, int window, double scale,
+                      const unsigned char* key_mask, int causal, int window, double scale, double alpha,
                       int B, int H, int L, int D, const long long* row_ids, long long nrows,
                       int tau_method, int n_iter, double* O_rows, double* tau_rows)
 {
@@ -254,7 +355,7 @@ void eo_attn_fwd_rows(const double* Q, const double* K, const double* V,
             long long bh = id / L;
             int h = (int)(bh % H);
             int b = (int)(bh / H);
-            tau_rows[r] = row_forward(Q, K, V, key_mask, causal, window, scale, H, L, D, b, h, i,
+            tau_rows[r] = row_forward(Q, K, V, key_mask, causal, window, scale, alpha, H, L, D, b, h, i,
                                       tau_method, n_iter, s, idx, p, O_rows + (size_t)r * D);
         }
         free(s);
@@ -265,23 +366,23 @@ void eo_attn_fwd_rows(const double* Q, const double* K, const double* V,
 
 /* Full forward: O [B,H,L,D], tau [B,H,L]. */
 void eo_attn_fwd(const double* Q, const double* K, const double* V,
-                 const unsigned char* key_mask, int causal, int window, double scale,
+                 const unsigned char* key_mask, int causal, int window, double scale, double alpha,
                  int B, int H, int L, int D, int tau_method, double* O, double* tau)
 {
     long long nrows = (long long)B * H * L;
     long long* ids = (long long*)malloc(sizeof(long long) * (size_t)nrows);
     for (long long r = 0; r < nrows; ++r) ids[r] = r;
-    eo_attn_fwd_rows(Q, K, V, key_mask, causal, window, scale, B, H, L, D, ids, nrows,
+    eo_attn_fwd_rows(Q, K, V, key_mask, causal, window, scale, alpha, B, H, L, D, ids, nrows,
                      tau_method, 25, O, tau);
     free(ids);
 }
 
 /* Backward for a list of heads bh = b*H + h (gradients of all rows and keys */
-/* of each listed head).  tau is recomputed here (exact, by sort): the      */
+/* of each listed head).  tau is recomputed here (exact): the              */
 /* oracle takes nothing from the code under test.  dQ, dK, dV are [nheads,  */
 /* L, D] in the order of bh_ids.                                            */
 void eo_attn_bwd_heads(const double* Q, const double* K, const double* V,
-                       const unsigned char* key_mask, int causal, int window, double scale,
+                       const unsigned char* key_mask, int causal, int window, double scale, double alpha,
                        int B, int H, int L, int D, const double* dO,
                        const long long* bh_ids, int nheads,
                        double* dQ, double* dK, double* dV)
@@ -323,9 +424,8 @@ void eo_attn_bwd_heads(const double* Q, const double* K, const double* V,
                     ++n;
                 }
                 if (n == 0) continue;
-                double tau;
-                eo_tau_sort(s, n, &tau);
-                eo_entmax15(s, n, tau, p);
+                const double tau = row_tau(s, n, alpha, 0, 0);
+                row_probs(s, n, tau, alpha, p);
                 /* g_j = dL/dp_ij = <dO_i, V_j> (O_i = sum_j p_ij V_j) */
                 for (int e = 0; e < n; ++e) {
                     const double* v = V + head + (size_t)idx[e] * D;
@@ -333,7 +433,8 @@ void eo_attn_bwd_heads(const double* Q, const double* K, const double* V,
                     for (int t = 0; t < D; ++t) acc += go[t] * v[t];
                     g[e] = acc;
                 }
-                eo_entmax15_jvp(p, g, n, ds);
+                if (alpha == 1.5) eo_entmax15_jvp(p, g, n, ds);
+                else eo_entmax_alpha_jvp(p, g, n, alpha, ds);
                 for (int e = 0; e < n; ++e) {
                     if (p[e] == 0.0) continue;
                     int j = idx[e];

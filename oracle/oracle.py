@@ -67,13 +67,22 @@ def _load():
         lib.eo_entmax15.argtypes = [_dp, ctypes.c_int, ctypes.c_double, _dp]
         lib.eo_entmax15_jvp.argtypes = [_dp, _dp, ctypes.c_int, _dp]
         lib.eo_attn_fwd_rows.argtypes = [_dp, _dp, _dp, _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          _i64p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, _dp, _dp]
         lib.eo_attn_fwd.argtypes = [_dp, _dp, _dp, _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp]
+                                    ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, _dp, _dp]
         lib.eo_attn_bwd_heads.argtypes = [_dp, _dp, _dp, _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp,
-                                          _i64p, ctypes.c_int, _dp, _dp, _dp]
+                                          ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          _dp, _i64p, ctypes.c_int, _dp, _dp, _dp]
+        lib.eo_g_alpha.restype = ctypes.c_double
+        lib.eo_g_alpha.argtypes = [_dp, ctypes.c_int, ctypes.c_double, ctypes.c_double]
+        lib.eo_tau_alpha.restype = ctypes.c_double
+        lib.eo_tau_alpha.argtypes = [_dp, ctypes.c_int, ctypes.c_double]
+        lib.eo_tau_alpha_bisect.restype = ctypes.c_double
+        lib.eo_tau_alpha_bisect.argtypes = [_dp, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+        lib.eo_entmax_alpha.argtypes = [_dp, ctypes.c_int, ctypes.c_double, ctypes.c_double, _dp]
+        lib.eo_entmax_alpha_jvp.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_double, _dp]
         lib.eo_num_threads.restype = ctypes.c_int
         lib.eo_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -152,8 +161,47 @@ def entmax15_jvp(p, gvec) -> np.ndarray:
     return ds
 
 
+def g_alpha(s, tau: float, alpha: float) -> float:
+    """sum_i max(0, (alpha-1)(s_i - tau))^(1/(alpha-1)) (the alpha-entmax constraint function)."""
+    s = _f64(s)
+    return _load().eo_g_alpha(_d(s), s.size, float(tau), float(alpha))
+
+
+def tau_alpha(s, alpha: float) -> float:
+    """alpha-entmax threshold (score units) by bisection run to fp64 convergence on
+    [max - 1/(alpha-1), max - n^(1-alpha)/(alpha-1)] -- the pages' bisection (page
+    "svd-sst2-roberta-adasplash", section 4, entmax_bisect) taken to its limit."""
+    s = _f64(s)
+    return _load().eo_tau_alpha(_d(s), s.size, float(alpha))
+
+
+def tau_alpha_bisect(s, alpha: float, n_iter: int = 25) -> float:
+    """The same bracket halved n_iter times, final midpoint."""
+    s = _f64(s)
+    return _load().eo_tau_alpha_bisect(_d(s), s.size, float(alpha), int(n_iter))
+
+
+def entmax_alpha(s, alpha: float, tau: float | None = None) -> np.ndarray:
+    """p = max(0, (alpha-1)(s - tau))^(1/(alpha-1)), tau from tau_alpha unless given."""
+    s = _f64(s)
+    if tau is None:
+        tau = tau_alpha(s, alpha)
+    p = np.empty_like(s)
+    _load().eo_entmax_alpha(_d(s), s.size, float(tau), float(alpha), _d(p))
+    return p
+
+
+def entmax_alpha_jvp(p, gvec, alpha: float) -> np.ndarray:
+    """dL/ds from dL/dp for alpha-entmax: w = p^(2-alpha), ds = w (g - <w, g>/sum w)."""
+    p = _f64(p)
+    gvec = _f64(gvec)
+    ds = np.empty_like(p)
+    _load().eo_entmax_alpha_jvp(_d(p), _d(gvec), p.size, float(alpha), _d(ds))
+    return ds
+
+
 # --------------------------------------------------------------------------
-# attention
+# attention (alpha = 1.5 unless given; other alpha in (1, 2] use tau_alpha)
 # --------------------------------------------------------------------------
 def _mask_arg(key_mask, B, L):
     if key_mask is None:
@@ -162,20 +210,27 @@ def _mask_arg(key_mask, B, L):
     return m, m.ctypes.data_as(_u8p)
 
 
-def attn_fwd(Q, K, V, key_mask=None, causal=False, window=0, scale=0.125, tau_method="sort"):
+def _alpha_arg(alpha) -> float:
+    a = float(alpha)
+    if not (1.0 < a <= 2.0):
+        raise ValueError("alpha must lie in (1, 2], got %r" % alpha)
+    return a
+
+
+def attn_fwd(Q, K, V, key_mask=None, causal=False, window=0, scale=0.125, tau_method="sort", alpha=1.5):
     """Full forward. Q,K,V: [B,H,L,D] (values already bf16-rounded). Returns (O, tau)."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, H, L, D = Q.shape
     m, mp = _mask_arg(key_mask, B, L)
     O = np.empty_like(Q)
     tau = np.empty((B, H, L), dtype=np.float64)
-    _load().eo_attn_fwd(_d(Q), _d(K), _d(V), mp, int(bool(causal)), int(window), float(scale),
+    _load().eo_attn_fwd(_d(Q), _d(K), _d(V), mp, int(bool(causal)), int(window), float(scale), _alpha_arg(alpha),
                         B, H, L, D, 0 if tau_method == "sort" else 1, _d(O), _d(tau))
     return O, tau
 
 
 def attn_fwd_rows(Q, K, V, row_ids, key_mask=None, causal=False, window=0, scale=0.125,
-                  tau_method="sort", n_iter=25):
+                  tau_method="sort", n_iter=25, alpha=1.5):
     """Forward for selected rows (row id = (b*H + h)*L + i). Returns (O_rows, tau_rows)."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, H, L, D = Q.shape
@@ -184,12 +239,12 @@ def attn_fwd_rows(Q, K, V, row_ids, key_mask=None, causal=False, window=0, scale
     O = np.empty((ids.size, D), dtype=np.float64)
     tau = np.empty((ids.size,), dtype=np.float64)
     _load().eo_attn_fwd_rows(_d(Q), _d(K), _d(V), mp, int(bool(causal)), int(window), float(scale),
-                             B, H, L, D, ids.ctypes.data_as(_i64p), ids.size,
+                             _alpha_arg(alpha), B, H, L, D, ids.ctypes.data_as(_i64p), ids.size,
                              0 if tau_method == "sort" else 1, int(n_iter), _d(O), _d(tau))
     return O, tau
 
 
-def attn_bwd_heads(Q, K, V, dO, bh_ids, key_mask=None, causal=False, window=0, scale=0.125):
+def attn_bwd_heads(Q, K, V, dO, bh_ids, key_mask=None, causal=False, window=0, scale=0.125, alpha=1.5):
     """Gradients (dQ, dK, dV) of <dO, O> for the listed heads bh = b*H + h, each [n, L, D]."""
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
     B, H, L, D = Q.shape
@@ -200,14 +255,15 @@ def attn_bwd_heads(Q, K, V, dO, bh_ids, key_mask=None, causal=False, window=0, s
     dK = np.empty((n, L, D), dtype=np.float64)
     dV = np.empty((n, L, D), dtype=np.float64)
     _load().eo_attn_bwd_heads(_d(Q), _d(K), _d(V), mp, int(bool(causal)), int(window), float(scale),
-                              B, H, L, D, _d(dO), ids.ctypes.data_as(_i64p), n, _d(dQ), _d(dK), _d(dV))
+                              _alpha_arg(alpha), B, H, L, D, _d(dO), ids.ctypes.data_as(_i64p), n, _d(dQ), _d(dK),
+                              _d(dV))
     return dQ, dK, dV
 
 
-def attn_bwd(Q, K, V, dO, key_mask=None, causal=False, window=0, scale=0.125):
+def attn_bwd(Q, K, V, dO, key_mask=None, causal=False, window=0, scale=0.125, alpha=1.5):
     """Full backward; returns dQ, dK, dV shaped [B,H,L,D]."""
     B, H, L, D = np.shape(Q)
-    dQ, dK, dV = attn_bwd_heads(Q, K, V, dO, np.arange(B * H), key_mask, causal, window, scale)
+    dQ, dK, dV = attn_bwd_heads(Q, K, V, dO, np.arange(B * H), key_mask, causal, window, scale, alpha)
     return dQ.reshape(B, H, L, D), dK.reshape(B, H, L, D), dV.reshape(B, H, L, D)
 
 
@@ -230,25 +286,25 @@ def _n_rep(Q, K) -> int:
     return H // Hkv
 
 
-def attn_fwd_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=0.125, tau_method="sort"):
+def attn_fwd_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=0.125, tau_method="sort", alpha=1.5):
     """Grouped-query forward: K, V [B,H_kv,L,D] repeated to H heads, then attn_fwd.  (O, tau)."""
     r = _n_rep(Q, K)
-    return attn_fwd(Q, repeat_kv(K, r), repeat_kv(V, r), key_mask, causal, window, scale, tau_method)
+    return attn_fwd(Q, repeat_kv(K, r), repeat_kv(V, r), key_mask, causal, window, scale, tau_method, alpha)
 
 
 def attn_fwd_rows_gqa(Q, K, V, row_ids, key_mask=None, causal=False, window=0, scale=0.125,
-                      tau_method="sort", n_iter=25):
+                      tau_method="sort", n_iter=25, alpha=1.5):
     """attn_fwd_rows on the repeated K and V (row id = (b*H + h)*L + i over the query heads)."""
     r = _n_rep(Q, K)
     return attn_fwd_rows(Q, repeat_kv(K, r), repeat_kv(V, r), row_ids, key_mask, causal, window, scale,
-                         tau_method, n_iter)
+                         tau_method, n_iter, alpha)
 
 
-def attn_bwd_gqa(Q, K, V, dO, key_mask=None, causal=False, window=0, scale=0.125):
+def attn_bwd_gqa(Q, K, V, dO, key_mask=None, causal=False, window=0, scale=0.125, alpha=1.5):
     """Grouped-query backward.  The repeat copies each key/value head to n_rep query heads, so by the
     chain rule its gradient is the sum of the copies' gradients over those heads.  Returns dQ
     [B,H,L,D] and dK, dV [B,H_kv,L,D]."""
     r = _n_rep(Q, K)
     B, Hkv, L, D = np.shape(K)
-    dQ, dKr, dVr = attn_bwd(Q, repeat_kv(K, r), repeat_kv(V, r), dO, key_mask, causal, window, scale)
+    dQ, dKr, dVr = attn_bwd(Q, repeat_kv(K, r), repeat_kv(V, r), dO, key_mask, causal, window, scale, alpha)
     return dQ, dKr.reshape(B, Hkv, r, L, D).sum(axis=2), dVr.reshape(B, Hkv, r, L, D).sum(axis=2)

@@ -451,3 +451,140 @@ def test_gqa_backward_matches_finite_differences():
         if done == 2:
             break
     assert done >= 1
+
+
+# ------------------------------------------------------------ general alpha
+# alpha-entmax (page "svd-sst2-roberta-adasplash", section 4, the entmax_bisect routine):
+# p = max(0, (alpha-1)(s - tau))^(1/(alpha-1)), sum p = 1, for alpha in (1, 2].
+ALPHAS = (1.1, 1.25, 1.5, 1.75, 2.0)
+
+
+def _sparsemax_textbook(z):
+    """Sparsemax by sorting (Martins & Astudillo 2016, Algorithm 1): k(z) = max{k : 1 + k z_(k) >
+    sum_{j<=k} z_(j)}, tau = (sum_{j<=k} z_(j) - 1) / k, p = max(0, z - tau)."""
+    zs = np.sort(z)[::-1]
+    cs = np.cumsum(zs)
+    ks = np.arange(1, z.size + 1)
+    k = ks[1 + ks * zs > cs][-1]
+    tau = (cs[k - 1] - 1.0) / k
+    return np.clip(z - tau, 0.0, None), tau
+
+
+def test_alpha_two_is_textbook_sparsemax():
+    for s in _rows(31, 200, nmin=1, nmax=40, spread=(0.2, 4.0)):
+        p_ref, t_ref = _sparsemax_textbook(s)
+        assert orc.tau_alpha(s, 2.0) == pytest.approx(t_ref, abs=1e-12)
+        np.testing.assert_allclose(orc.entmax_alpha(s, 2.0), p_ref, atol=1e-12)
+
+
+def test_alpha_one_point_five_matches_closed_form():
+    """The generic solver at alpha = 1.5 against the sorted closed form of Theorem 1."""
+    for s in _rows(32, 200, nmin=1, nmax=60):
+        assert orc.tau_alpha(s, 1.5) == pytest.approx(orc.tau_sort(s)[0], abs=1e-12)
+        np.testing.assert_allclose(orc.entmax_alpha(s, 1.5), orc.entmax15(s), atol=1e-12)
+
+
+def test_alpha_near_one_tends_to_softmax():
+    """alpha -> 1+: alpha-entmax tends to softmax (the pages fall back to softmax at alpha = 1)."""
+    rng = np.random.default_rng(33)
+    for _ in range(20):
+        s = rng.normal(0, 1.0, size=12)
+        sm = np.exp(s - s.max())
+        sm /= sm.sum()
+        np.testing.assert_allclose(orc.entmax_alpha(s, 1.0 + 1e-4), sm, atol=2e-3)
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.75, 2.0])
+def test_alpha_argmax_definition_by_optimiser(alpha):
+    """alpha-entmax(s) = argmax_{p in simplex} p.s + sum (p - p^alpha) / (alpha (alpha - 1))
+    (the Tsallis-entropy definition of which section 2.1 is the alpha = 1.5 case)."""
+    c = 1.0 / (alpha * (alpha - 1.0))
+    for s in _rows(34, 25, nmin=2, nmax=6, spread=(0.3, 2.5)):
+        n = s.size
+
+        def neg(p):
+            p = np.clip(p, 0.0, None)
+            return -(p @ s + c * np.sum(p - p ** alpha))
+
+        best = None
+        for x0 in (np.full(n, 1.0 / n), np.eye(n)[int(np.argmax(s))] * 0.9 + 0.1 / n):
+            r = optimize.minimize(neg, x0, method="SLSQP", bounds=[(0, 1)] * n,
+                                  constraints=[{"type": "eq", "fun": lambda p: p.sum() - 1.0}],
+                                  options={"ftol": 1e-14, "maxiter": 500})
+            if best is None or r.fun < best.fun:
+                best = r
+        np.testing.assert_allclose(orc.entmax_alpha(s, alpha), np.clip(best.x, 0, None), atol=3e-4)
+
+
+@pytest.mark.parametrize("alpha", ALPHAS)
+def test_alpha_invariants_and_bisection_bound(alpha):
+    """Simplex, shift invariance, max-gap one-hot (gap >= 1/(alpha-1)), and the pages' 25 halvings
+    within half the final bracket of the converged root."""
+    a = alpha - 1.0
+    for s in _rows(35, 100, nmin=1, nmax=30):
+        p = orc.entmax_alpha(s, alpha)
+        assert np.all(p >= 0) and abs(p.sum() - 1.0) < 1e-10
+        np.testing.assert_allclose(orc.entmax_alpha(s + 3.7, alpha), p, atol=1e-11)
+        t = orc.tau_alpha(s, alpha)
+        width = (1.0 - s.size ** (-a)) / a
+        assert abs(orc.tau_alpha_bisect(s, alpha, 25) - t) <= width / 2 ** 26 + 1e-12
+    s = np.array([0.0, -1.0 / a, -1.0 / a - 0.5, -3.0 / a])
+    np.testing.assert_allclose(orc.entmax_alpha(s, alpha), [1.0, 0.0, 0.0, 0.0], atol=1e-12)
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.75, 2.0])
+def test_alpha_jvp_matches_finite_differences(alpha):
+    rng = np.random.default_rng(36)
+    checked = 0
+    for s in _rows(37, 120, nmin=2, nmax=10, spread=(0.5, 3.0)):
+        t = orc.tau_alpha(s, alpha)
+        if np.min(np.abs(s - t)) < 1e-3:
+            continue
+        h = 1e-6
+        J = np.empty((s.size, s.size))
+        for j in range(s.size):
+            e = np.zeros(s.size)
+            e[j] = h
+            J[:, j] = (orc.entmax_alpha(s + e, alpha) - orc.entmax_alpha(s - e, alpha)) / (2 * h)
+        gv = rng.normal(size=s.size)
+        ds = orc.entmax_alpha_jvp(orc.entmax_alpha(s, alpha), gv, alpha)
+        np.testing.assert_allclose(ds, J.T @ gv, atol=2e-6)
+        checked += 1
+    assert checked > 50
+
+
+@pytest.mark.parametrize("alpha", [1.25, 2.0])
+def test_alpha_attention_backward_matches_finite_differences(alpha):
+    B, H, L, D = 1, 1, 6, 4
+    scale = 0.6
+    done = 0
+    for seed in range(60):
+        Q, K, V, dO = _rand_qkv(400 + seed, B, H, L, D)
+        O, tau = orc.attn_fwd(Q, K, V, None, True, 0, scale, alpha=alpha)
+        S = scale * Q[0, 0] @ K[0, 0].T
+        a = _allowed(L, True, 0, None)
+        if np.abs(S - tau[0, 0][:, None])[a].min() < 1e-3:
+            continue
+        # forward against the scalar root finder, row by row
+        for i in range(L):
+            s = S[i, a[i]]
+            f = lambda t: np.sum(np.clip((alpha - 1) * (s - t), 0, None) ** (1 / (alpha - 1))) - 1.0
+            assert tau[0, 0, i] == pytest.approx(optimize.brentq(f, s.max() - 1 / (alpha - 1) - 1, s.max(),
+                                                                 xtol=1e-15), abs=1e-10)
+        dQ, dK, dV = orc.attn_bwd(Q, K, V, dO, None, True, 0, scale, alpha=alpha)
+        eps = 1e-6
+        for X, dX in ((Q, dQ), (K, dK), (V, dV)):
+            num = np.zeros_like(X)
+            for idx in np.ndindex(X.shape):
+                old = X[idx]
+                X[idx] = old + eps
+                Lp = np.sum(dO * orc.attn_fwd(Q, K, V, None, True, 0, scale, alpha=alpha)[0])
+                X[idx] = old - eps
+                Lm = np.sum(dO * orc.attn_fwd(Q, K, V, None, True, 0, scale, alpha=alpha)[0])
+                X[idx] = old
+                num[idx] = (Lp - Lm) / (2 * eps)
+            np.testing.assert_allclose(dX, num, atol=3e-6)
+        done += 1
+        if done == 2:
+            break
+    assert done >= 1
