@@ -22,11 +22,13 @@ from ._binding import (  # noqa: F401
     entmax_attn_bwd,
     entmax_attn_bwd_noalloc,
     entmax_attn_bwd_saved,
+    entmax_attn_bwd_saved_ex,
     entmax_attn_bwd_saved_gqa,
     entmax_attn_bwd_saved_workspace_size,
     entmax_attn_bwd_workspace_size,
     entmax_attn_device_status,
     entmax_attn_fwd,
+    entmax_attn_fwd_ex,
     entmax_attn_fwd_gqa,
     entmax_attn_fwd_train,
     entmax_attn_fwd_train_gqa,

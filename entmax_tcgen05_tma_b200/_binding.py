@@ -36,6 +36,8 @@ EXPORTED = (
     "entmax_attn_fwd_gqa",
     "entmax_attn_fwd_train_gqa",
     "entmax_attn_bwd_saved_gqa",
+    "entmax_attn_fwd_ex",
+    "entmax_attn_bwd_saved_ex",
     "entmax_attn_strerror",
     "entmax_attn_device_status",
     "entmax_attn_last_cuda_error",
@@ -83,6 +85,11 @@ def _load_library() -> ctypes.CDLL:
     lib.entmax_attn_bwd_saved_gqa.restype = i
     lib.entmax_attn_bwd_saved_gqa.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, i, vp, vp, sz, vp, vp, vp, vp,
                                               vp, sz, vp]
+    lib.entmax_attn_fwd_ex.restype = i
+    lib.entmax_attn_fwd_ex.argtypes = [vp, vp, vp, i, vp, i, i, f, f, i, i, i, i, i, vp, i, vp, vp, sz, vp]
+    lib.entmax_attn_bwd_saved_ex.restype = i
+    lib.entmax_attn_bwd_saved_ex.argtypes = [vp, vp, vp, i, vp, i, i, f, f, i, i, i, i, i, vp, vp, sz, vp, vp, vp,
+                                             vp, vp, sz, vp]
     lib.entmax_attn_strerror.restype = ctypes.c_char_p
     lib.entmax_attn_strerror.argtypes = [i]
     lib.entmax_attn_device_status.restype = i
@@ -167,9 +174,9 @@ def _kv_heads(Q, K, grouped: bool) -> int:
     return Hkv
 
 
-def _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, grouped):
+def _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, grouped, alpha=None):
     B, H, L, D = Q.shape
-    Hkv = _kv_heads(Q, K, grouped)
+    Hkv = _kv_heads(Q, K, grouped or alpha is not None)
     _check_input("Q", Q, (B, H, L, D))
     _check_input("K", K, (B, Hkv, L, D), Q.dtype)
     _check_input("V", V, (B, Hkv, L, D), Q.dtype)
@@ -185,11 +192,18 @@ def _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, gr
         tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
     else:
         _check_input("tau", tau, (B, H, L), torch.float32)
-    args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
-            int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
-            L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(),
-            _stream_handle(stream))
-    name = "entmax_attn_fwd_gqa" if grouped else "entmax_attn_fwd"
+    if alpha is not None:
+        args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
+                int(bool(causal)), int(window), float(scale), float(alpha), B, H, Hkv, L, D, O.data_ptr(),
+                ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(), None, 0,
+                _stream_handle(stream))
+        name = "entmax_attn_fwd_ex"
+    else:
+        args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
+                int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
+                L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(),
+                _stream_handle(stream))
+        name = "entmax_attn_fwd_gqa" if grouped else "entmax_attn_fwd"
     st = getattr(lib, name)(*args)
     if st != ENTMAX_OK:
         raise EntmaxError(st, name)
@@ -291,9 +305,9 @@ def _byte_buffer(t, nbytes: int, device, name: str):
     return t
 
 
-def _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, grouped):
+def _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, grouped, alpha=None):
     B, H, L, D = Q.shape
-    Hkv = _kv_heads(Q, K, grouped)
+    Hkv = _kv_heads(Q, K, grouped or alpha is not None)
     _check_input("Q", Q, (B, H, L, D))
     _check_input("K", K, (B, Hkv, L, D), Q.dtype)
     _check_input("V", V, (B, Hkv, L, D), Q.dtype)
@@ -311,11 +325,18 @@ def _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, save
         _check_input("tau", tau, (B, H, L), torch.float32)
     nbytes = entmax_attn_saved_bytes(B, H, L, D)
     saved = _byte_buffer(saved, nbytes, Q.device, "saved")
-    args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
-            int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
-            L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(),
-            saved.data_ptr(), saved.numel() * saved.element_size(), _stream_handle(stream))
-    name = "entmax_attn_fwd_train_gqa" if grouped else "entmax_attn_fwd_train"
+    if alpha is not None:
+        args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
+                int(bool(causal)), int(window), float(scale), float(alpha), B, H, Hkv, L, D, O.data_ptr(),
+                ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(), saved.data_ptr(),
+                saved.numel() * saved.element_size(), _stream_handle(stream))
+        name = "entmax_attn_fwd_ex"
+    else:
+        args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
+                int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
+                L, D, O.data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(),
+                saved.data_ptr(), saved.numel() * saved.element_size(), _stream_handle(stream))
+        name = "entmax_attn_fwd_train_gqa" if grouped else "entmax_attn_fwd_train"
     st = getattr(lib, name)(*args)
     if st != ENTMAX_OK:
         raise EntmaxError(st, name)
@@ -336,9 +357,10 @@ def entmax_attn_fwd_train_gqa(Q, K, V, key_mask=None, causal=False, window=0, sc
     return _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, True)
 
 
-def _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK, dV, workspace, stream, grouped):
+def _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK, dV, workspace, stream, grouped,
+               alpha=None):
     B, H, L, D = Q.shape
-    Hkv = _kv_heads(Q, K, grouped)
+    Hkv = _kv_heads(Q, K, grouped or alpha is not None)
     _check_input("Q", Q, (B, H, L, D))
     _check_input("K", K, (B, Hkv, L, D), Q.dtype)
     _check_input("V", V, (B, Hkv, L, D), Q.dtype)
@@ -354,12 +376,14 @@ def _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK,
             _check_input(name, t, (B, heads, L, D), torch.float32)
         outs.append(t)
     ws = _byte_buffer(workspace, entmax_attn_bwd_saved_workspace_size(B, H, L, D), Q.device, "workspace")
+    head = (float(alpha), B, H, Hkv) if alpha is not None else (B, H, Hkv) if grouped else (B, H)
     args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
-            int(bool(causal)), int(window), float(scale), B, H) + ((Hkv,) if grouped else ()) + (
+            int(bool(causal)), int(window), float(scale)) + head + (
             L, D, tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(), dO.data_ptr(),
             outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(), ws.data_ptr(),
             ws.numel() * ws.element_size(), _stream_handle(stream))
-    name = "entmax_attn_bwd_saved_gqa" if grouped else "entmax_attn_bwd_saved"
+    name = ("entmax_attn_bwd_saved_ex" if alpha is not None else
+            "entmax_attn_bwd_saved_gqa" if grouped else "entmax_attn_bwd_saved")
     st = getattr(lib, name)(*args)
     if st != ENTMAX_OK:
         raise EntmaxError(st, name)
@@ -381,6 +405,24 @@ def entmax_attn_bwd_saved_gqa(Q, K, V, tau, saved, dO, key_mask=None, causal=Fal
                       True)
 
 
+def entmax_attn_fwd_ex(Q, K, V, key_mask=None, causal=False, window=0, scale=None, alpha=1.5, save=False,
+                       out_dtype=torch.bfloat16, O=None, tau=None, saved=None, stream=None):
+    """alpha-entmax forward, alpha in (1, 2]; K and V may have fewer heads than Q (H % H_kv == 0).
+
+    Returns (O, tau) or, with ``save=True``, (O, tau, saved) for entmax_attn_bwd_saved_ex."""
+    if save:
+        return _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, True, alpha)
+    return _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, True, alpha)
+
+
+def entmax_attn_bwd_saved_ex(Q, K, V, tau, saved, dO, key_mask=None, causal=False, window=0, scale=None, alpha=1.5,
+                             dQ=None, dK=None, dV=None, workspace=None, stream=None):
+    """Backward of entmax_attn_fwd_ex(save=True) with the same alpha.  Returns dQ [B,H,L,64] and
+    dK, dV [B,H_kv,L,64], fp32."""
+    return _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK, dV, workspace, stream, True,
+                      alpha)
+
+
 def entmax_attn_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(lib.entmax_attn_device_status(_stream_handle(stream)))
@@ -398,18 +440,19 @@ class EntmaxAttention(torch.autograd.Function):
     """Autograd wrapper: forward and backward both run in the library's kernels."""
 
     @staticmethod
-    def forward(ctx, Q, K, V, key_mask=None, causal=False, window=0, scale=None):
+    def forward(ctx, Q, K, V, key_mask=None, causal=False, window=0, scale=None, alpha=1.5):
         grouped = K.shape[1] != Q.shape[1]  # K, V with fewer heads than Q: grouped-query attention
+        a = None if alpha == 1.5 else float(alpha)  # other alpha: the _ex entry points
         O, tau, saved = _fwd_train(Q, K, V, key_mask, causal, window, scale, torch.bfloat16, None, None, None, None,
-                                   grouped)
+                                   grouped, a)
         ctx.save_for_backward(Q, K, V, tau, saved, key_mask if key_mask is not None else torch.empty(0))
-        ctx.cfg = (key_mask is not None, causal, window, scale, grouped)
+        ctx.cfg = (key_mask is not None, causal, window, scale, grouped, a)
         return O
 
     @staticmethod
     def backward(ctx, dO):
         Q, K, V, tau, saved, km = ctx.saved_tensors
-        has_mask, causal, window, scale, grouped = ctx.cfg
+        has_mask, causal, window, scale, grouped, a = ctx.cfg
         dQ, dK, dV = _bwd_saved(Q, K, V, tau, saved, dO.to(Q.dtype).contiguous(), km if has_mask else None, causal,
-                                window, scale, None, None, None, None, None, grouped)
-        return dQ.to(Q.dtype), dK.to(K.dtype), dV.to(V.dtype), None, None, None, None
+                                window, scale, None, None, None, None, None, grouped, a)
+        return dQ.to(Q.dtype), dK.to(K.dtype), dV.to(V.dtype), None, None, None, None, None

@@ -195,10 +195,20 @@ int check_kv_heads(int H, int Hkv, int in_dtype) {
     return ENTMAX_OK;
 }
 
+// alpha of alpha-entmax: (1, 2].  alpha = 1 is softmax attention, which this library does not
+// compute (its supports are dense).
+int check_alpha(float alpha) {
+    if (alpha == 1.f) return ENTMAX_ERR_UNSUPPORTED;
+    if (!(alpha > 1.f && alpha <= 2.f)) return ENTMAX_ERR_ARG;
+    return ENTMAX_OK;
+}
+
 int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-             int window, float scale, int B, int H, int Hkv, int L, int D, void* O, int out_dtype, float* tau,
-             cudaStream_t stream) {
+             int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, void* O, int out_dtype,
+             float* tau, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    rc = check_alpha(alpha);
     if (rc) return rc;
     rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
@@ -211,7 +221,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -232,13 +242,15 @@ extern "C" {
 int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
                     int window, float scale, int B, int H, int L, int D, void* O, int out_dtype, float* tau,
                     cudaStream_t stream) {
-    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, H, L, D, O, out_dtype, tau, stream);
+    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, O, out_dtype, tau,
+                    stream);
 }
 
 int entmax_attn_fwd_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                         int causal, int window, float scale, int B, int H, int Hkv, int L, int D, void* O,
                         int out_dtype, float* tau, cudaStream_t stream) {
-    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, Hkv, L, D, O, out_dtype, tau, stream);
+    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, O, out_dtype, tau,
+                    stream);
 }
 
 size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D) {
@@ -263,7 +275,7 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f};
     BwdIO io{tau, dO, dQ, dK, dV, static_cast<float*>(workspace)};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -301,9 +313,11 @@ size_t entmax_attn_bwd_saved_workspace_size(int B, int H, int L, int D) {
 
 namespace {
 int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-                   int window, float scale, int B, int H, int Hkv, int L, int D, void* O, int out_dtype, float* tau,
-                   void* saved, size_t saved_bytes, cudaStream_t stream) {
+                   int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, void* O, int out_dtype,
+                   float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    rc = check_alpha(alpha);
     if (rc) return rc;
     rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
@@ -323,7 +337,7 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -339,10 +353,12 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
 }
 
 int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-                   int window, float scale, int B, int H, int Hkv, int L, int D, const float* tau, const void* saved,
-                   size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV, void* workspace,
-                   size_t ws_bytes, cudaStream_t stream) {
+                   int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, const float* tau,
+                   const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV,
+                   void* workspace, size_t ws_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
+    if (rc) return rc;
+    rc = check_alpha(alpha);
     if (rc) return rc;
     rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
@@ -358,7 +374,7 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(status_ptr(&status));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f};
     BwdIO io{tau, dO, dQ, dK, dV, nullptr};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -381,30 +397,48 @@ extern "C" {
 int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                           int causal, int window, float scale, int B, int H, int L, int D, void* O, int out_dtype,
                           float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
-    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, H, L, D, O, out_dtype, tau, saved,
-                          saved_bytes, stream);
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, O, out_dtype, tau,
+                          saved, saved_bytes, stream);
 }
 
 int entmax_attn_fwd_train_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                               int causal, int window, float scale, int B, int H, int Hkv, int L, int D, void* O,
                               int out_dtype, float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
-    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, Hkv, L, D, O, out_dtype, tau,
-                          saved, saved_bytes, stream);
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, O, out_dtype,
+                          tau, saved, saved_bytes, stream);
 }
 
 int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                           int causal, int window, float scale, int B, int H, int L, int D, const float* tau,
                           const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV,
                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, H, L, D, tau, saved, saved_bytes,
-                          dO, dQ, dK, dV, workspace, ws_bytes, stream);
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, tau, saved,
+                          saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
 }
 
 int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                               int causal, int window, float scale, int B, int H, int Hkv, int L, int D,
                               const float* tau, const void* saved, size_t saved_bytes, const void* dO, float* dQ,
                               float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, Hkv, L, D, tau, saved,
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, tau, saved,
+                          saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
+}
+
+int entmax_attn_fwd_ex(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+                       int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, void* O,
+                       int out_dtype, float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
+    if (!saved && saved_bytes == 0)
+        return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, O, out_dtype, tau,
+                        stream);
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, O, out_dtype,
+                          tau, saved, saved_bytes, stream);
+}
+
+int entmax_attn_bwd_saved_ex(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                             int causal, int window, float scale, float alpha, int B, int H, int Hkv, int L, int D,
+                             const float* tau, const void* saved, size_t saved_bytes, const void* dO, float* dQ,
+                             float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, tau, saved,
                           saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
 }
 
@@ -462,7 +496,7 @@ extern "C" int entmax_attn_bwd_noalloc(const void* Q, const void* K, const void*
     float* scratch = nullptr;
     rc = record(noalloc_scratch(&scratch));
     if (rc) return rc;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f};
     BwdIO io{tau, dO, dQ, dK, dV, scratch};
     return record(launch_bwd(a, io, stream));
 }

@@ -1,11 +1,14 @@
-// bwd_saved.cu -- backward pass of 1.5-entmax attention from the forward's saved supports.
+// bwd_saved.cu -- backward pass of alpha-entmax attention from the forward's saved supports.
 //
 // Same closed-form Jacobian as bwd.cu (page "svd-sst2-roberta-adasplash", section 2.4):
 //   dA_ij = dO_i . V_j,  sp_ij = sqrt(p_ij),  u_i = sum_j sp_ij dA_ij / sum_j sp_ij,
 //   dS_ij = sp_ij (dA_ij - u_i),  dQ_i = scale sum_j dS_ij K_j,  dK_j = scale sum_i dS_ij Q_i,
-//   dV_j = sum_i p_ij dO_i,
-// but the supports {(j, sp_ij)} come from entmax_attn_fwd_train instead of a recomputed score pass,
-// so no QK^T is formed again: the work is proportional to the number of support entries.
+//   dV_j = sum_i p_ij dO_i.
+// General alpha (p = b^(1/am1), b = am1 (S - tau), am1 = alpha - 1; the pages' entmax_bisect
+// routine): the Jacobian has the same form with the weight w_ij = p_ij^(2 - alpha) = b^(1/am1 - 1) in
+// place of sp_ij (at alpha 1.5, w = b = sqrt(p)).  The saved lists hold b_ij in both cases.
+// The supports {(j, b_ij)} come from the training forward instead of a recomputed score pass, so
+// no QK^T is formed again: the work is proportional to the number of support entries.
 //
 //  1. key_scan:   per head, exclusive scan of the per-key support counts -> bucket offsets.
 //  2. rows:       four query rows per warp, eight lanes per row (each lane owns eight dimensions, so
@@ -95,10 +98,12 @@ struct GlobalRows {
 // piece of V_je per lane and a three-step group reduction, two entries in flight; then u_i, dS_e,
 // the bucket entries, and dQ_i (one 16-byte piece of K_je per lane per entry).  cnt < 0: no row, or
 // a row the exact pass handles.
-template <class Rows>
+// GEN: general alpha, weights w = b^em1 (em1 = 1/am1 - 1) and p = w b; the buckets then hold p
+// instead of b.
+template <bool GEN, class Rows>
 __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
                                            const SavedBwdWs& ws, long long row, int cnt, int bhk, const Rows& Vr,
-                                           const Rows& Kr, uint16_t* mj, float* msp, float* mds, int sd) {
+                                           const Rows& Kr, uint16_t* mj, float* msp, float* mds, int sd, float em1) {
     const int L = a.L;
     const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
     const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
@@ -134,12 +139,12 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
         }
     }
     __syncwarp();
-    // u_i = sum sp dA / sum sp over the row's entries
+    // u_i = sum w dA / sum w over the row's entries (w = sp at alpha 1.5)
     float r1 = 0.f, w1 = 0.f;
     for (int e = sd; e < cnt; e += 8) {
-        const float sp = msp[e];
-        r1 += sp;
-        w1 = fmaf(sp, mds[e], w1);
+        const float w = GEN ? pow_pos(msp[e], em1) : msp[e];
+        r1 += w;
+        w1 = fmaf(w, mds[e], w1);
     }
     r1 = group8_sum(r1);
     w1 = group8_sum(w1);
@@ -148,12 +153,13 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
     // dS_e, and (i, sp, dS) into key j's bucket
     for (int e = sd; e < cnt; e += 8) {
         const float sp = msp[e];
-        const float ds = sp * (mds[e] - uu);
+        const float w = GEN ? pow_pos(sp, em1) : sp;
+        const float ds = w * (mds[e] - uu);
         mds[e] = ds;
         const size_t key = (size_t)bhk * L + mj[e];
         const size_t at = (size_t)bhk * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
         ws.bucket_i[at] = (uint32_t)row;
-        ws.bucket_sp[at] = sp;
+        ws.bucket_sp[at] = GEN ? w * sp : sp;
         ws.bucket_ds[at] = ds;
     }
     __syncwarp();
@@ -189,7 +195,7 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
 // One key per group of eight lanes: dK_j = scale sum dS Q_i and dV_j = sum p dO_i over key j's bucket,
 // lane sd of the group loading entry e0 + sd and the group sharing it by shuffles; two entries (two
 // 16-byte pieces each per lane) in flight.  valid = false: no key (the group still takes part).
-template <class Rows>
+template <bool GEN, class Rows>
 __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
                                            const SavedBwdWs& ws, long long key, bool valid, int bhk, const Rows& Qr,
                                            const Rows& Gr, int sd, int g0) {
@@ -217,7 +223,7 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
                 const float st = __shfl_sync(0xffffffffu, esp, src);
                 const float dt = __shfl_sync(0xffffffffu, eds, src);
                 const bool ok = e0 + t + u < n;
-                pv[u] = ok ? st * st : 0.f;
+                pv[u] = ok ? (GEN ? st : st * st) : 0.f;  // p_ij
                 dv[u] = ok ? dt : 0.f;
                 xg[u] = ok ? Gr.get((int)it, sd) : make_uint4(0u, 0u, 0u, 0u);
                 xq[u] = ok ? Qr.get((int)it, sd) : make_uint4(0u, 0u, 0u, 0u);
@@ -246,6 +252,7 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
 }
 
 // Four query rows per warp (eight lanes each), rows of K and V gathered from L2.
+template <bool GEN>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     __shared__ uint16_t lj[ROW_WARPS][RPW][SAVE_CAP];
@@ -255,6 +262,7 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
     const int q = lane >> 3, sd = lane & 7;
     const int L = a.L;
     const long long R = (long long)a.B * a.H * L;
+    const float em1 = 1.f / a.am1 - 1.f;
     for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long row = grp * RPW + q;
         const int cnt = row < R ? sv.row_cnt[row] : -1;
@@ -262,11 +270,12 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
         const size_t head = (size_t)bhk * L * HEAD_DIM;
         const GlobalRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head};
         const GlobalRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head};
-        rows_group(a, io, sv, ws, row, cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd);
+        rows_group<GEN>(a, io, sv, ws, row, cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd, em1);
     }
 }
 
 // Four keys per warp (eight lanes each), rows of Q and dO gathered from L2.
+template <bool GEN>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -280,7 +289,7 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnAr
         const long long key = grp * RPW + q;
         const bool kv = key < Rk;
         const int bhk = kv ? (int)(key / L) : 0;
-        keys_group(a, io, sv, ws, key, kv, bhk, Qr, Gr, sd, g0);
+        keys_group<GEN>(a, io, sv, ws, key, kv, bhk, Qr, Gr, sd, g0);
     }
 }
 
@@ -316,9 +325,11 @@ __device__ __forceinline__ float dot64_f32(const float* a, const __nv_bfloat16* 
 
 // Rows whose support was not saved: recomputed exactly by one CTA each (scores on CUDA cores), dQ_i
 // stored, dK/dV contributions added with atomics (this kernel runs after saved_keys_kernel).
+template <bool GEN>
 __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                       const SavedSupport sv) {
-    extern __shared__ float sbuf[];  // [L]: sqrt(p_ij); [L, 2L): dA_ij
+    extern __shared__ float sbuf[];  // [L]: b_ij = am1 (S_ij - tau_i) (sqrt(p_ij) at alpha 1.5); [L, 2L): dA_ij
+    const float am1 = a.am1, em1 = 1.f / am1 - 1.f;
     __shared__ float red[UNSAVED_THREADS];
     __shared__ float qf[HEAD_DIM], gf[HEAD_DIM];
     const int tid = threadIdx.x;
@@ -351,13 +362,14 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
             float sp = 0.f;
             if (!a.key_mask || a.key_mask[(size_t)b * L + j]) {
                 const float s = a.scale * dot64_f32(qf, K + head + (size_t)j * HEAD_DIM);
-                sp = fmaxf(0.5f * (s - tau), 0.f);
+                sp = fmaxf((GEN ? am1 : 0.5f) * (s - tau), 0.f);
             }
             float dA = 0.f;
             if (sp > 0.f) {
                 dA = dot64_f32(gf, V + head + (size_t)j * HEAD_DIM);
-                r += sp;
-                w = fmaf(sp, dA, w);
+                const float wt = GEN ? pow_pos(sp, em1) : sp;
+                r += wt;
+                w = fmaf(wt, dA, w);
             }
             sbuf[e] = sp;
             sbuf[L + e] = dA;
@@ -373,10 +385,11 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
             const float sp = sbuf[e];
             if (sp > 0.f) {
                 const size_t key = (size_t)bhk * L + lo + e;
-                const float ds = sp * (sbuf[L + e] - u);
+                const float wt = GEN ? pow_pos(sp, em1) : sp;
+                const float ds = wt * (sbuf[L + e] - u);
                 acc = fmaf(ds, __bfloat162float(K[key * HEAD_DIM + d]), acc);
                 atomicAdd(io.dK + key * HEAD_DIM + d, a.scale * ds * qf[d]);
-                atomicAdd(io.dV + key * HEAD_DIM + d, sp * sp * gf[d]);
+                atomicAdd(io.dV + key * HEAD_DIM + d, wt * sp * gf[d]);
             }
         }
         __syncthreads();
@@ -446,18 +459,24 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>((R + ROW_WARPS - 1) / ROW_WARPS, (long long)sms * 8));
-    saved_rows_kernel<<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    const bool gen = generic_alpha(a);
+    if (gen) saved_rows_kernel<true><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    else saved_rows_kernel<false><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long Rk = (long long)a.B * a.Hkv * a.L;
     const unsigned kgrid = (unsigned)std::max<long long>(1, std::min<long long>((Rk + ROW_WARPS * RPW - 1) / (ROW_WARPS * RPW), (long long)sms * 8));
-    saved_keys_kernel<<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    if (gen) saved_keys_kernel<true><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    else saved_keys_kernel<false><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int smem = 2 * a.L * (int)sizeof(float);
-    e = ensure_smem_attr(reinterpret_cast<const void*>(unsaved_rows_kernel), 2 * MAX_L * (int)sizeof(float), 3);
+    const void* ufn = gen ? reinterpret_cast<const void*>(unsaved_rows_kernel<true>)
+                          : reinterpret_cast<const void*>(unsaved_rows_kernel<false>);
+    e = ensure_smem_attr(ufn, 2 * MAX_L * (int)sizeof(float), gen ? 5 : 3);
     if (e != cudaSuccess) return e;
-    unsaved_rows_kernel<<<(unsigned)sms, UNSAVED_THREADS, smem, stream>>>(a, io, sv);
+    if (gen) unsaved_rows_kernel<true><<<(unsigned)sms, UNSAVED_THREADS, smem, stream>>>(a, io, sv);
+    else unsaved_rows_kernel<false><<<(unsigned)sms, UNSAVED_THREADS, smem, stream>>>(a, io, sv);
     return cudaGetLastError();
 }
 

@@ -412,6 +412,16 @@ __device__ __forceinline__ float staged_half(const float* stage, int slot, int k
     return stage[slot * 16 + ((((k16 >> 2) ^ (slot & 3))) << 2) + (k16 & 3)];
 }
 
+// b^e for b > 0 (0 for b <= 0), as 2^(e log2 b) with the hardware base-2 approximations
+// lg2.approx and ex2.approx (close to fp32 precision; the result's relative error grows with
+// |e log2 b|).
+__device__ __forceinline__ float pow_pos(float b, float e) {
+    float l, r;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(b));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(e * l));
+    return b > 0.f ? r : 0.f;
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

@@ -103,6 +103,15 @@ __device__ __forceinline__ float top4_bound(float a0, float a1, float a2, float 
     return bound - 1e-5f * sqrtf(c4);
 }
 
+// General alpha (am1 = alpha - 1, p = max(0, am1 (x - tau))^(1/am1) in scaled units x = scale S):
+// at tau = z_k - k^(-am1)/(am1 scale) (raw units) each of the k largest scores adds at least 1/k, so
+// the row's tau is at least that for every k.  Lower bound (raw units) from the four largest chunk
+// maxima (missing values -inf), lowered by a rounding margin; wk[k] = (k+1)^(-am1) / (am1 scale).
+__device__ __forceinline__ float gen_bound(float a0, float a1, float a2, float a3, const float (&wk)[4]) {
+    const float b = fmaxf(fmaxf(a0 - wk[0], a1 - wk[1]), fmaxf(a2 - wk[2], a3 - wk[3]));
+    return b - 1e-5f * wk[0];
+}
+
 __device__ __forceinline__ void top4_insert(float v, float& a0, float& a1, float& a2, float& a3) {
     if (v > a3) {
         if (v > a2) {
@@ -235,6 +244,76 @@ __device__ __forceinline__ float solve_tau(const float* lcv, int r, int h, int n
     return tau_x;
 }
 
+// General alpha: tau of one row in units y = am1 (scale S - ms) (row max 0, every p term is
+// (y - t)^e with e = 1/am1), candidates split over a lane pair as in solve_tau.  Bisection of
+// [lo, hi] (g(lo) >= 1 >= g(hi)) with the same every-four-halvings stop once no candidate lies
+// strictly inside the bracket and g(lo) <= 1.5; then Newton's method on the support
+// S = {y > midpoint} so fixed, started at lo: on S, phi(t) = sum (y - t)^e - 1 is convex and
+// decreasing with phi(lo) >= 0, so the iterates rise monotonically to the root without passing it
+// (one step is exact when e = 1).  Far from the root a large e makes Newton crawl (each step
+// closes about 1/e of the gap), hence the g(lo) <= 1.5 condition: from there six steps reach fp32
+// precision for e up to 20.  Not settled after 25 halvings: the final midpoint.  Returns t in y
+// units.
+template <int NC>
+__device__ __forceinline__ float solve_tau_gen(const float* lcv, int r, int h, int nh, int n0, float scale, float ms,
+                                               float am1, float e, float lo, float hi) {
+    float y[NC];
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+        const int en = 2 * k + h;
+        y[k] = k < nh ? am1 * fmaf(scale, lcv[(en < n0 ? en : CAPW + (en - n0)) * TILE + r], -ms) : -INFINITY;
+    }
+    bool settled = false;
+    float glo = INFINITY;  // g(lo), once lo has moved
+    for (int it = 0; it < 25; ++it) {
+        const float mid = 0.5f * (lo + hi);
+        float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
+#pragma unroll
+        for (int k = 0; k < NC; k += 4) {
+            g0 += pow_pos(y[k] - mid, e);
+            g1 += pow_pos(y[k + 1] - mid, e);
+            g2 += pow_pos(y[k + 2] - mid, e);
+            g3 += pow_pos(y[k + 3] - mid, e);
+        }
+        float gs = (g0 + g1) + (g2 + g3);
+        gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+        if (gs > 1.f) {
+            lo = mid;
+            glo = gs;
+        } else {
+            hi = mid;
+        }
+        if ((it & 3) == 3 || it == 24) {
+            int und = 0;
+#pragma unroll
+            for (int k = 0; k < NC; ++k) und += (y[k] > lo && y[k] < hi) ? 1 : 0;
+            und += __shfl_xor_sync(0xffffffffu, und, 1);
+            settled = und == 0 && glo <= 1.5f;
+            if (__all_sync(0xffffffffu, settled)) break;
+        }
+    }
+    const float mid = 0.5f * (lo + hi);
+    float t = lo;
+    const float em1 = e - 1.f;
+#pragma unroll 1
+    for (int step = 0; step < 6; ++step) {
+        float s0 = 0.f, s1 = 0.f;  // sum over S of (y - t)^(e-1) and of (y - t)^e
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+            if (y[k] > mid) {
+                const float b = y[k] - t;
+                const float w = pow_pos(b, em1);
+                s0 += w;
+                s1 = fmaf(w, b, s1);
+            }
+        }
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        if (s0 > 0.f) t += (s1 - 1.f) / (e * s0);
+    }
+    return settled ? fminf(fmaxf(t, lo), hi) : mid;
+}
+
 __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4& x) {
     const uint32_t u[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -244,9 +323,11 @@ __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4
     }
 }
 
-// Writes row r's support (both partitions, p_ij in cv) to the saved lists as (j, sqrt(p_ij)) and
+// Writes row r's support (both partitions, p_ij in cv; b_ij for general alpha) to the saved lists as
+// (j, b_ij), b_ij = am1 (S_ij - tau_i) scaled (= sqrt(p_ij) at alpha 1.5), and
 // counts each key once per row that holds it.  Run by the row's two threads (h = 0, 1) after phase 2;
 // rows redone on CUDA cores (mode 2) or with more than SAVE_CAP entries are marked unsaved.
+template <bool GEN>
 __device__ __forceinline__ void save_row_support(const SavedSupport& sv, const float* cv, const uint16_t* cj,
                                                  const int* supp_cnt, int r, int h, int mode, size_t head_row0,
                                                  size_t key_row0, int i, int L) {
@@ -267,7 +348,8 @@ __device__ __forceinline__ void save_row_support(const SavedSupport& sv, const f
     for (int e = 0; e < n; ++e) {
         const int j = cj[(slot0 + e) * TILE + r];
         sv.row_j[row * SAVE_CAP + base + e] = (uint16_t)j;
-        sv.row_sp[row * SAVE_CAP + base + e] = sqrtf(cv[(slot0 + e) * TILE + r]);
+        const float c = cv[(slot0 + e) * TILE + r];  // p (alpha 1.5) or b = am1 (x - tau) (generic)
+        sv.row_sp[row * SAVE_CAP + base + e] = GEN ? c : sqrtf(c);
         atomicAdd(sv.key_cnt + key_row0 + j, 1);
     }
 }
@@ -305,11 +387,16 @@ __device__ __forceinline__ float block_max(float a, float* red) {
     return m;
 }
 
-// Phase 4: the whole CTA recomputes one row exactly on CUDA cores.
+// Phase 4: the whole CTA recomputes one row exactly on CUDA cores.  alpha 1.5: bisection of
+// [m - 2, m - 2/sqrt(n)] and the closed-form root once the support is fixed.  General alpha
+// (GEN, am1 = alpha - 1): the same in units y = am1 (s - m), bracket [-1, -n^(-am1)], and Newton's
+// method from the lower end on the fixed support once also g(lower end) <= 1.5 (as in
+// solve_tau_gen).
+template <bool GEN>
 __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                                           const __nv_bfloat16* __restrict__ V, const uint32_t* bits, float* sbuf,
                                           float* red, int bh, int bhk, int i, int L, int causal, int window, float scale,
-                                          int nallow, void* O, int out_f32, float* tau) {
+                                          float am1, int nallow, void* O, int out_f32, float* tau) {
     const int tid = threadIdx.x;
     float* qf = red + 64;  // 64 floats (red[0..63] holds reduction partials)
     const size_t head = (size_t)bh * L * HEAD_DIM, kv_head = (size_t)bhk * L * HEAD_DIM;
@@ -342,38 +429,73 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         mloc = fmaxf(mloc, s);
     }
     const float m = block_max(mloc, red);
-    float blo = m - 2.f, bhi = m - 2.f / sqrtf((float)nallow);
+    const float ex = 1.f / am1;
+    // alpha 1.5 works on the scores s, general alpha on y = am1 (s - m)
+    auto unit = [&](float s) { return GEN ? am1 * (s - m) : s; };
+    float blo = GEN ? -1.f : m - 2.f;
+    float bhi = GEN ? -pow_pos((float)nallow, -am1) : m - 2.f / sqrtf((float)nallow);
     bool resolved = false;
+    float glo = INFINITY;  // g(blo) once blo has moved (general alpha: Newton needs g(blo) <= 1.5)
     for (int it = 0; it < 25; ++it) {
         const float mid = 0.5f * (blo + bhi);
         float gl = 0.f, inside = 0.f;
         for (int e = tid; e < span; e += NUM_THREADS) {
-            const float s = sbuf[e];
+            const float s = unit(sbuf[e]);
             if (s > mid) {
-                const float d = 0.5f * (s - mid);
-                gl = fmaf(d, d, gl);
+                if (GEN) {
+                    gl += pow_pos(s - mid, ex);
+                } else {
+                    const float d = 0.5f * (s - mid);
+                    gl = fmaf(d, d, gl);
+                }
             }
             if (s > blo && s < bhi) inside += 1.f;
         }
         const float2 r2 = block_sum2(gl, inside, red);
-        if (r2.y == 0.f) {
+        if (r2.y == 0.f && (!GEN || glo <= 1.5f)) {
             resolved = true;
             break;
         }
-        if (r2.x > 1.f) blo = mid;
-        else bhi = mid;
+        if (r2.x > 1.f) {
+            blo = mid;
+            glo = r2.x;
+        } else {
+            bhi = mid;
+        }
     }
     float t;
     if (!resolved) {
         // one more count: the last halving may have emptied the bracket
         float inside = 0.f;
         for (int e = tid; e < span; e += NUM_THREADS) {
-            const float s = sbuf[e];
+            const float s = unit(sbuf[e]);
             if (s > blo && s < bhi) inside += 1.f;
         }
-        resolved = block_sum2(inside, 0.f, red).x == 0.f;
+        resolved = block_sum2(inside, 0.f, red).x == 0.f && (!GEN || glo <= 1.5f);
     }
-    if (resolved) {
+    if (GEN) {
+        // Newton's method on the fixed support {y >= bhi}, from blo (monotone, see solve_tau_gen)
+        float tt = blo;
+        if (resolved) {
+            for (int step = 0; step < 6; ++step) {
+                float s0 = 0.f, s1 = 0.f;
+                for (int e = tid; e < span; e += NUM_THREADS) {
+                    const float y = unit(sbuf[e]);
+                    if (y >= bhi) {
+                        const float b = y - tt;
+                        const float w = pow_pos(b, ex - 1.f);
+                        s0 += w;
+                        s1 = fmaf(w, b, s1);
+                    }
+                }
+                const float2 sums = block_sum2(s0, s1, red);
+                if (sums.x > 0.f) tt += (sums.y - 1.f) / (ex * sums.x);
+            }
+            t = fminf(fmaxf(tt, blo), bhi);
+        } else {
+            t = 0.5f * (blo + bhi);
+        }
+    } else if (resolved) {
         float k = 0.f, s1 = 0.f, s2 = 0.f;
         for (int e = tid; e < span; e += NUM_THREADS) {
             const float s = sbuf[e];
@@ -398,10 +520,16 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
     const int d = tid % HEAD_DIM, ph = tid / HEAD_DIM;
     float acc = 0.f;
     for (int e = ph; e < span; e += PH) {
-        const float s = sbuf[e];
+        const float s = unit(sbuf[e]);
         if (s > t) {
-            const float h = 0.5f * (s - t);
-            acc = fmaf(h * h, __bfloat162float(V[kv_head + (size_t)(lo + e) * HEAD_DIM + d]), acc);
+            float p;
+            if (GEN) {
+                p = pow_pos(s - t, ex);
+            } else {
+                const float h = 0.5f * (s - t);
+                p = h * h;
+            }
+            acc = fmaf(p, __bfloat162float(V[kv_head + (size_t)(lo + e) * HEAD_DIM + d]), acc);
         }
     }
     __syncthreads();
@@ -414,7 +542,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         const size_t oi = head + (size_t)i * HEAD_DIM + tid;
         if (out_f32) reinterpret_cast<float*>(O)[oi] = o;
         else reinterpret_cast<__nv_bfloat16*>(O)[oi] = __float2bfloat16_rn(o);
-        if (tid == 0) tau[(size_t)bh * L + i] = t;
+        if (tid == 0) tau[(size_t)bh * L + i] = GEN ? m + t * ex : t;
     }
     __syncthreads();
 }
@@ -479,6 +607,7 @@ __device__ __noinline__ void mma_half(PipeCtl* ctl, const WaitCfg& wc, const uin
     }
 }
 
+template <bool GEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const AttnArgs args, const FwdOut out) {
@@ -540,6 +669,12 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const float scale = args.scale;
     const float two_over_scale = 2.f / scale;
     const float c4 = 4.f / (scale * scale);
+    // general alpha: am1 = alpha - 1, p = (y - t)^ex with y = am1 (scaled score - row max);
+    // wk[k] = (k+1)^(-am1) / (am1 scale), the lower-bound offsets of gen_bound
+    const float am1 = args.am1, ex = 1.f / am1;
+    float wk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) wk[k] = GEN ? exp2f(-am1 * log2f((float)(k + 1))) / (am1 * scale) : 0.f;
     const int nblk = ctl->nblk;
     const bool resident = nblk <= NBUF;
     // Streamed tiles run pass A on every other listed block only (any subset of a row bounds tau
@@ -636,7 +771,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // scores at or below t are outside the support: the largest chunk maximum seen minus 2
         // (scaled), raised to the exact threshold of the four largest chunk maxima seen (any
         // subset's threshold is at most tau)
-        const float t = fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
+        const float t = GEN ? gen_bound(a0, a1, a2, a3, wk)
+                            : fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
 
         // ---------------- pass B: candidates s > m - 2 (scaled) into this warpgroup's partition
         float* pcv = cv + g * CAPW * TILE;
@@ -728,31 +864,56 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         top4_insert(s1.a1, b0, b1, b2, b3);
         top4_insert(s1.a2, b0, b1, b2, b3);
         top4_insert(s1.a3, b0, b1, b2, b3);
-        const float t_cut = fmaxf(b0 - two_over_scale, top4_bound(b0, b1, b2, b3, c4));
-        const float hi = -2.f / sqrtf((float)max(s0.n + s1.n, 1));
-        const float lo = fminf(fmaxf(-2.f, fmaf(scale, t_cut, -ms)), hi);
+        const float t_cut = GEN ? gen_bound(b0, b1, b2, b3, wk)
+                                : fmaxf(b0 - two_over_scale, top4_bound(b0, b1, b2, b3, c4));
+        // general alpha, in y units: g(-1) >= 1 from the max alone, g(-k^(-am1)) <= 1 over k candidates
+        const float hi = GEN ? -pow_pos((float)max(s0.n + s1.n, 1), -am1) : -2.f / sqrtf((float)max(s0.n + s1.n, 1));
+        const float lo = GEN ? fminf(fmaxf(-1.f, am1 * fmaf(scale, t_cut, -ms)), hi)
+                             : fminf(fmaxf(-2.f, fmaf(scale, t_cut, -ms)), hi);
         // the row's candidates split evenly over its two threads; registers: the warp's largest share
         // rounded up to a multiple of eight
         const int ns = mode == 0 ? (s0.n + s1.n + 1 - h) >> 1 : 0;
         const int nmax = __reduce_max_sync(0xffffffffu, ns);
-        float tau_x;
-        switch ((nmax + 7) >> 3) {
-            case 0:
-            case 1: tau_x = solve_tau<8>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-            case 2: tau_x = solve_tau<16>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-            case 3: tau_x = solve_tau<24>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-            case 4: tau_x = solve_tau<32>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-            case 5: tau_x = solve_tau<40>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-            case 6: tau_x = solve_tau<48>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-            case 7: tau_x = solve_tau<56>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-            default: tau_x = solve_tau<CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+        float tau_x;  // alpha 1.5: scaled units (row max 0); general alpha: y units
+        if (GEN) {
+            switch ((nmax + 7) >> 3) {
+                case 0:
+                case 1: tau_x = solve_tau_gen<8>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+                case 2: tau_x = solve_tau_gen<16>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+                case 3: tau_x = solve_tau_gen<24>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+                case 4: tau_x = solve_tau_gen<32>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+                case 5: tau_x = solve_tau_gen<40>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+                case 6: tau_x = solve_tau_gen<48>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+                case 7: tau_x = solve_tau_gen<56>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+                default: tau_x = solve_tau_gen<CAPW>(cv, r, h, ns, s0.n, scale, ms, am1, ex, lo, hi); break;
+            }
+        } else {
+            switch ((nmax + 7) >> 3) {
+                case 0:
+                case 1: tau_x = solve_tau<8>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 2: tau_x = solve_tau<16>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 3: tau_x = solve_tau<24>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 4: tau_x = solve_tau<32>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 5: tau_x = solve_tau<40>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 6: tau_x = solve_tau<48>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 7: tau_x = solve_tau<56>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                default: tau_x = solve_tau<CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+            }
         }
         if (mode == 0) {
-            // this thread's partition of the support: cv <- p_ij, cj <- j (in place)
+            // this thread's partition of the support: cv <- p_ij (alpha 1.5) or b_ij = y - t (general
+            // alpha; p = b^ex), cj <- j (in place)
             int sn = 0;
             for (int k = 0; k < nh; ++k) {
                 const float xv = fmaf(scale, pcv[k * TILE + r], -ms);
-                if (xv > tau_x) {
+                if (GEN) {
+                    const float b = am1 * xv - tau_x;
+                    if (b > 0.f) {
+                        pcv[sn * TILE + r] = b;
+                        pcj[sn * TILE + r] = pcj[k * TILE + r];
+                        ++sn;
+                    }
+                } else if (xv > tau_x) {
                     const float hh = 0.5f * (xv - tau_x);
                     pcv[sn * TILE + r] = hh * hh;
                     pcj[sn * TILE + r] = pcj[k * TILE + r];
@@ -760,7 +921,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 }
             }
             supp_cnt[h * TILE + r] = sn;
-            if (h == 0) out.tau[(size_t)bh * L + i] = ms + tau_x;
+            if (h == 0) out.tau[(size_t)bh * L + i] = GEN ? ms + tau_x * ex : ms + tau_x;
         } else if (mode == 2) {
             if (h == 0) atomicOr(&redo[r >> 5], 1u << (r & 31));
             supp_cnt[h * TILE + r] = 0;
@@ -770,7 +931,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         __syncwarp();
         if (out.save.row_cnt)
-            save_row_support(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, (size_t)bhk * L, i, L);
+            save_row_support<GEN>(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, (size_t)bhk * L, i, L);
 
         // ---------------- phase 3: O_i = sum_j p_ij V_j over the row's whole support (both
         // partitions); thread h of the pair accumulates dimensions [32 h, 32 h + 32) in registers
@@ -787,7 +948,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 for (int e = 0; e < ns; ++e) {
                     const int sl = e < n0 ? e : CAPW + (e - n0);
                     const int j = cj[sl * TILE + r];
-                    const float p = cv[sl * TILE + r];
+                    const float p = GEN ? pow_pos(cv[sl * TILE + r], ex) : cv[sl * TILE + r];
                     // 128-byte swizzled V block in ring slot vslot[j / BLK]: 16-byte chunk c of row
                     // `row` sits at chunk position c ^ (row & 7)
                     const uint32_t row = (uint32_t)j & (BLK - 1);
@@ -807,7 +968,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         const int ee = e + u < ns ? e + u : e;
                         const int sl = ee < n0 ? ee : CAPW + (ee - n0);
                         const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)cj[sl * TILE + r] * HEAD_DIM) + 4 * h;
-                        pw[u] = e + u < ns ? cv[sl * TILE + r] : 0.f;
+                        pw[u] = e + u < ns ? (GEN ? pow_pos(cv[sl * TILE + r], ex) : cv[sl * TILE + r]) : 0.f;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) x[u][c] = __ldg(src + c);
                     }
@@ -848,10 +1009,11 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             while (mask) {
                 const int rr = wd * 32 + __ffs(mask) - 1;
                 mask &= mask - 1;
-                fallback_row(reinterpret_cast<const __nv_bfloat16*>(args.Q), reinterpret_cast<const __nv_bfloat16*>(args.K),
-                             reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, bh, bhk, i0 + rr, L,
-                             args.causal, args.window, scale, rows[rr].nallow + rows[TILE + rr].nallow, out.O,
-                             out.out_f32, out.tau);
+                fallback_row<GEN>(reinterpret_cast<const __nv_bfloat16*>(args.Q),
+                                  reinterpret_cast<const __nv_bfloat16*>(args.K),
+                                  reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, bh, bhk, i0 + rr,
+                                  L, args.causal, args.window, scale, am1, rows[rr].nallow + rows[TILE + rr].nallow,
+                                  out.O, out.out_f32, out.tau);
             }
         }
     }
@@ -876,10 +1038,14 @@ cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     e = make_tile_map(&mv, a.V, a.B * a.Hkv, a.L, BLK);
     if (e != cudaSuccess) return e;
-    e = ensure_smem_attr(reinterpret_cast<const void*>(entmax_fwd_kernel), SMEM_BYTES, 0);
+    const bool gen = generic_alpha(a);
+    const void* kfn = gen ? reinterpret_cast<const void*>(entmax_fwd_kernel<true>)
+                          : reinterpret_cast<const void*>(entmax_fwd_kernel<false>);
+    e = ensure_smem_attr(kfn, SMEM_BYTES, gen ? 4 : 0);
     if (e != cudaSuccess) return e;
     dim3 grid((a.L + TILE - 1) / TILE, a.B * a.H);
-    entmax_fwd_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, a, o);
+    if (gen) entmax_fwd_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, a, o);
+    else entmax_fwd_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, a, o);
     return cudaGetLastError();
 }
 

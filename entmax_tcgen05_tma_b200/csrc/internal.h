@@ -20,7 +20,12 @@ struct AttnArgs {
     unsigned long long timeout_ns;
     int Hkv;                 // key/value heads (H % Hkv == 0); query head h of batch b reads KV head
                              // b * Hkv + h / (H / Hkv) -- grouped-query attention when Hkv < H
+    float am1;               // alpha - 1 in (0, 1]: p = max(0, am1 (S - tau))^(1 / am1); 0.5 is 1.5-entmax
 };
+
+// alpha = 1.5 runs the specialised kernels (closed-form tau finish, p = h^2); any other alpha the
+// generic ones.
+__host__ __device__ __forceinline__ bool generic_alpha(const AttnArgs& a) { return a.am1 != 0.5f; }
 
 // Key/value head of query head bh = b * H + h.
 __host__ __device__ __forceinline__ int kv_head_of(int bh, int H, int Hkv) { return (bh / H) * Hkv + (bh % H) / (H / Hkv); }
@@ -30,7 +35,7 @@ constexpr int SAVE_CAP = 64;  // support entries kept per row
 struct SavedSupport {
     int* row_cnt;            // [R] entries of row, or -1 when the row's support was not saved
     uint16_t* row_j;         // [R][SAVE_CAP] key index of each entry
-    float* row_sp;           // [R][SAVE_CAP] sqrt(p_ij) = (S_ij - tau_i)/2 of each entry
+    float* row_sp;           // [R][SAVE_CAP] b_ij = am1 (S_ij - tau_i) of each entry (sqrt(p_ij) at alpha 1.5)
     int* key_cnt;            // [B*Hkv*L] rows whose support holds key j of a KV head (zeroed before the forward)
     int* unsaved_cnt;        // [1] rows whose support was not saved (zeroed before the forward)
     int* unsaved_rows;       // [R] their row ids

@@ -168,6 +168,41 @@ ENTMAX_API int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const voi
                                          void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * alpha-entmax attention for any alpha in (1, 2] (page "svd-sst2-roberta-adasplash", section 4: the
+ * attention layer's entmax_bisect routine solves sum_j max(0, (alpha-1) s_j - tau')^(1/(alpha-1)) = 1
+ * by bisection for alpha in (1, 2]; alpha = 1.5 is the 1.5-entmax of every other entry point, alpha =
+ * 2 is sparsemax).  With a = alpha - 1 and tau in score units (tau' = a tau):
+ *   p_ij = max(0, a (S_ij - tau_i))^(1/a),  sum_j p_ij = 1,  O_i = sum_j p_ij V_j,
+ * and the backward uses the Jacobian w_i (delta_ij - w_j / sum_k w_k), w = p^(2 - alpha).
+ *   alpha      in (1, 2]; alpha = 1 (softmax, dense supports) returns ENTMAX_ERR_UNSUPPORTED, any
+ *              other value (or NaN) ENTMAX_ERR_ARG.  alpha = 1.5 runs exactly the kernels of the
+ *              entry points above; other values run variants whose tau solve ends with Newton's
+ *              method on the settled support instead of the closed form.  Supports grow as alpha
+ *              approaches 1: rows with more candidates than the kernels list are recomputed on CUDA
+ *              cores, so small alpha - 1 is correct but slow.
+ *   H_kv       key/value heads as in the _gqa calls (H_kv = H: plain multi-head attention).
+ *   saved      entmax_attn_fwd_ex: NULL with saved_bytes = 0 computes the forward only
+ *              (entmax_attn_fwd / _gqa); otherwise the training forward (entmax_attn_fwd_train /
+ *              _gqa).  entmax_attn_bwd_saved_ex reads supports written by entmax_attn_fwd_ex with
+ *              the same alpha, Q, K, masks and scale.  Each saved entry holds b_ij = a (S_ij - tau_i)
+ *              (sqrt(p_ij) at alpha = 1.5).
+ *   tau        fp32 [B, H, L], score units for every alpha (+inf for a row with no allowed key).
+ * Other arguments, layouts and errors: as entmax_attn_fwd / _fwd_train / _bwd_saved and their _gqa
+ * forms.
+ */
+ENTMAX_API int entmax_attn_fwd_ex(const void* Q, const void* K, const void* V, int in_dtype,
+                                  const uint8_t* key_mask, int causal, int window, float scale, float alpha,
+                                  int B, int H, int H_kv, int L, int D,
+                                  void* O, int out_dtype, float* tau,
+                                  void* saved, size_t saved_bytes, cudaStream_t stream);
+ENTMAX_API int entmax_attn_bwd_saved_ex(const void* Q, const void* K, const void* V, int in_dtype,
+                                        const uint8_t* key_mask, int causal, int window, float scale,
+                                        float alpha, int B, int H, int H_kv, int L, int D,
+                                        const float* tau, const void* saved, size_t saved_bytes,
+                                        const void* dO, float* dQ, float* dK, float* dV,
+                                        void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Allocation-free variant of entmax_attn_bwd (no counterpart in the AdaSplash pages; it exists for
  * this library's users).  Some callers cannot allocate device memory at the point where they run
  * the backward pass: engines that plan all memory ahead of time and forbid allocation inside their

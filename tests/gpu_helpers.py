@@ -47,8 +47,10 @@ def allowed_matrix(L, causal, window, mask_row):
     return a
 
 
-def check_rows(Qd, Kd, row_ids, tau_gpu_rows, tau_ref_rows, key_mask, causal, window, scale, H, L):
-    """Simplex and support checks for the listed rows, in fp64 from the GPU's tau."""
+def check_rows(Qd, Kd, row_ids, tau_gpu_rows, tau_ref_rows, key_mask, causal, window, scale, H, L, alpha=1.5):
+    """Simplex and support checks for the listed rows, in fp64 from the GPU's tau
+    (p = max(0, (alpha-1)(s - tau))^(1/(alpha-1)); alpha 1.5: ((s - tau)/2)^2)."""
+    a1 = alpha - 1.0
     worst_sum = 0.0
     for r, rid in enumerate(row_ids):
         i = rid % L
@@ -62,7 +64,7 @@ def check_rows(Qd, Kd, row_ids, tau_gpu_rows, tau_ref_rows, key_mask, causal, wi
         s = scale * (Kd[b, h][a] @ Qd[b, h, i])
         tg, tr = tau_gpu_rows[r], tau_ref_rows[r]
         assert abs(tg - tr) <= TAU_TOL, (rid, tg, tr)
-        p = np.clip((s - tg) / 2, 0, None) ** 2
+        p = np.clip(a1 * (s - tg), 0, None) ** (1.0 / a1)
         worst_sum = max(worst_sum, abs(p.sum() - 1.0))
         differ = (s > tg) != (s > tr)
         assert np.all(np.abs(s[differ] - tr) < SUPPORT_BAND), (rid, s[differ], tr)

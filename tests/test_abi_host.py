@@ -179,3 +179,48 @@ def test_binding_rejects_bad_kv_head_count():
     k = torch.zeros(1, 4, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         E.entmax_attn_fwd_gqa(q, k, k)
+
+
+def _ex_calls(alpha, B=1, H=2, Hkv=2, in_dtype=0, saved=P, saved_bytes=None):
+    R = max(B * H * 64, 1)
+    need = E.entmax_attn_saved_bytes(1, 1, R) if saved_bytes is None else saved_bytes
+    ws = E.entmax_attn_bwd_saved_workspace_size(1, 1, R)
+    f = E.lib.entmax_attn_fwd_ex(P, P, P, in_dtype, None, 0, 0, 0.125, alpha, B, H, Hkv, 64, 64, P, 0, P, saved,
+                                 need, None)
+    b = E.lib.entmax_attn_bwd_saved_ex(P, P, P, in_dtype, None, 0, 0, 0.125, alpha, B, H, Hkv, 64, 64, P, P, need,
+                                       P, P, P, P, P, ws, None)
+    return f, b
+
+
+@pytest.mark.parametrize("alpha,code", [
+    (1.0, E.ENTMAX_ERR_UNSUPPORTED),  # softmax
+    (0.5, E.ENTMAX_ERR_ARG),
+    (2.0001, E.ENTMAX_ERR_ARG),
+    (float("nan"), E.ENTMAX_ERR_ARG),
+    (float("inf"), E.ENTMAX_ERR_ARG),
+    (-1.5, E.ENTMAX_ERR_ARG),
+])
+def test_alpha_argument_checks(alpha, code):
+    assert _ex_calls(alpha) == (code, code)
+
+
+def test_ex_entry_points_validate_before_launch():
+    # valid alpha, empty batch: a no-op
+    assert _ex_calls(1.75, B=0) == (E.ENTMAX_OK, E.ENTMAX_OK)
+    assert _ex_calls(2.0, B=0) == (E.ENTMAX_OK, E.ENTMAX_OK)
+    # grouped heads are checked as in the _gqa calls
+    assert _ex_calls(1.25, H=4, Hkv=3) == (E.ENTMAX_ERR_ARG, E.ENTMAX_ERR_ARG)
+    assert _ex_calls(1.25, H=4, Hkv=2, in_dtype=1) == (E.ENTMAX_ERR_UNSUPPORTED, E.ENTMAX_ERR_UNSUPPORTED)
+    # a saved buffer that is too small, or a size without a buffer
+    f, _ = _ex_calls(1.25, saved_bytes=16)
+    assert f == E.ENTMAX_ERR_WORKSPACE
+    f, _ = _ex_calls(1.25, saved=None, saved_bytes=1 << 20)
+    assert f == E.ENTMAX_ERR_WORKSPACE
+
+
+def test_binding_rejects_bad_alpha_before_the_library():
+    import torch
+
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        E.entmax_attn_fwd_ex(q, q, q, alpha=1.5)  # CPU tensors are refused first
