@@ -17,6 +17,10 @@ GPU), so --gpus N runs N independent replicas, one per rank, with no data-path c
 value = total work of all ranks / max step time over ranks ("scaling": "weak").
 
 --impl reference times the fp64 CPU oracle on the host cores (bounded sample per step).
+
+Variants (side measurements, not the headline line): --alpha A runs alpha-entmax for A in (1, 2]
+and --hkv N grouped-query attention with N key/value heads, both through entmax_attn_fwd_ex /
+entmax_attn_bwd_saved_ex; the dense-equivalent FLOP count is unchanged (it counts query heads).
 """
 from __future__ import annotations
 
@@ -137,11 +141,14 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: int = 64) -> dict:
+def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: int = 64, alpha: float = 1.5) -> dict:
     """Time the fp64 oracle (as it stands) on whole heads of the workload until ~budget_s."""
     from oracle import oracle as orc
 
     f64 = {k: inp[k].to(torch.float64).numpy() for k in ("Q", "K", "V", "dO")}
+    if w.kv_heads != w.H:  # grouped heads: the oracle's repeat of K and V (outside the timed loop)
+        for k in ("K", "V"):
+            f64[k] = orc.repeat_kv(f64[k], w.H // w.kv_heads)
     km = None if inp["key_mask"] is None else inp["key_mask"].numpy()
     pairs_per_head = []
     full_pairs = allowed_pairs(w, inp["key_mask"])
@@ -153,9 +160,10 @@ def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: i
         b = bh // w.H
         L = w.L
         rows = bh * L + torch.arange(L).numpy()
-        orc.attn_fwd_rows(f64["Q"], f64["K"], f64["V"], rows, km, w.causal, w.window, w.scale)
+        orc.attn_fwd_rows(f64["Q"], f64["K"], f64["V"], rows, km, w.causal, w.window, w.scale, alpha=alpha)
         if w.backward:
-            orc.attn_bwd_heads(f64["Q"], f64["K"], f64["V"], f64["dO"], [bh], km, w.causal, w.window, w.scale)
+            orc.attn_bwd_heads(f64["Q"], f64["K"], f64["V"], f64["dO"], [bh], km, w.causal, w.window, w.scale,
+                               alpha=alpha)
         sub = w.with_shape(B=1)
         pairs_per_head.append(allowed_pairs(sub.with_shape(H=1), None if km is None else inp["key_mask"][b:b + 1]))
         heads += 1
@@ -180,10 +188,11 @@ def measured_sparsity(w: Workload, Q, K, tau, km) -> float:
         band &= j <= i
     if w.window:
         band &= j >= i - w.window + 1
+    rep = w.H // w.kv_heads
     for b in range(w.B):
         a = band if km is None else band & km[b].bool().unsqueeze(0)
         for h in range(w.H):
-            S = w.scale * (Q[b, h].float() @ K[b, h].float().T)
+            S = w.scale * (Q[b, h].float() @ K[b, h // rep].float().T)
             supp = (S > tau[b, h].unsqueeze(1)) & a
             allowed += int(a.sum())
             zeros += int(a.sum()) - int(supp.sum())
@@ -193,7 +202,9 @@ def measured_sparsity(w: Workload, Q, K, tau, km) -> float:
 def run_gpu(args, rank: int, world: int) -> dict | None:
     import entmax_tcgen05_tma_b200 as E
 
-    w = WORKLOADS[args.workload]
+    w = bench_workload(args)
+    alpha = args.alpha
+    variant = alpha != 1.5 or w.kv_heads != w.H  # the _ex entry points
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     inp = make_inputs(w)
@@ -202,9 +213,11 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     Q, K, V, dO = (inp[k].to(dev) for k in ("Q", "K", "V", "dO"))
     km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
     B, H, L, D = w.B, w.H, w.L, w.D
+    Hkv = w.kv_heads
     O = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
     tau = torch.empty((B, H, L), dtype=torch.float32, device=dev)
-    dQ, dK, dV = (torch.empty((B, H, L, D), dtype=torch.float32, device=dev) for _ in range(3))
+    dQ = torch.empty((B, H, L, D), dtype=torch.float32, device=dev)
+    dK, dV = (torch.empty((B, Hkv, L, D), dtype=torch.float32, device=dev) for _ in range(2))
     saved = torch.empty((E.entmax_attn_saved_bytes(B, H, L, D),), dtype=torch.uint8, device=dev)
     ws = torch.empty((E.entmax_attn_bwd_saved_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
@@ -212,14 +225,21 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     launches_per_step = 1 + (4 if w.backward else 0)
 
     def fwd_call():
-        if w.backward:
+        if variant:
+            E.entmax_attn_fwd_ex(Q, K, V, km, w.causal, w.window, w.scale, alpha=alpha, save=w.backward, O=O, tau=tau,
+                                 saved=saved if w.backward else None)
+        elif w.backward:
             E.entmax_attn_fwd_train(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau, saved=saved)
         else:
             E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
 
     def bwd_call():
-        E.entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV,
-                                workspace=ws)
+        if variant:
+            E.entmax_attn_bwd_saved_ex(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale, alpha=alpha, dQ=dQ,
+                                       dK=dK, dV=dV, workspace=ws)
+        else:
+            E.entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV,
+                                    workspace=ws)
 
     def step():
         fwd_call()
@@ -268,7 +288,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                 "tau": torch.empty(tau.shape, dtype=tau.dtype).pin_memory()}
     if w.backward:
         for name in ("dQ", "dK", "dV"):
-            host_out[name] = torch.empty((B, H, L, D), dtype=torch.float32).pin_memory()
+            host_out[name] = torch.empty((B, H if name == "dQ" else Hkv, L, D), dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + (
         0 if host_km is None else host_km.numel())
     if not w.backward:
@@ -282,7 +302,11 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         Kd = host_in["K"].to(dev, non_blocking=True)
         Vd = host_in["V"].to(dev, non_blocking=True)
         kmd = None if host_km is None else host_km.to(dev, non_blocking=True)
-        if w.backward:
+        if variant:
+            r = E.entmax_attn_fwd_ex(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale, alpha=alpha, save=w.backward,
+                                     saved=saved if w.backward else None)
+            Oo, to, sv = r if w.backward else (r[0], r[1], None)
+        elif w.backward:
             Oo, to, sv = E.entmax_attn_fwd_train(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale, saved=saved)
         else:
             Oo, to = E.entmax_attn_fwd(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale)
@@ -290,8 +314,12 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         host_out["tau"].copy_(to, non_blocking=True)
         if w.backward:
             dOd = host_in["dO"].to(dev, non_blocking=True)
-            g = E.entmax_attn_bwd_saved(Qd, Kd, Vd, to, sv, dOd, kmd, w.causal, w.window, w.scale, dQ=dQe, dK=dKe,
-                                        dV=dVe, workspace=ws)
+            if variant:
+                g = E.entmax_attn_bwd_saved_ex(Qd, Kd, Vd, to, sv, dOd, kmd, w.causal, w.window, w.scale, alpha=alpha,
+                                               dQ=dQe, dK=dKe, dV=dVe, workspace=ws)
+            else:
+                g = E.entmax_attn_bwd_saved(Qd, Kd, Vd, to, sv, dOd, kmd, w.causal, w.window, w.scale, dQ=dQe,
+                                            dK=dKe, dV=dVe, workspace=ws)
             for name, t in zip(("dQ", "dK", "dV"), g):
                 host_out[name].copy_(t, non_blocking=True)
 
@@ -319,7 +347,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     rows = B * H * L
     # Q, K, V read once, O (bf16) and tau written; the training forward also writes each row's
     # saved support: a count and a (u16 key, fp32 sqrt p) pair per entry
-    fwd_alg_bytes = 3.0 * rows * D * 2 + rows * D * 2 + rows * 4
+    kv_rows = B * Hkv * L
+    fwd_alg_bytes = rows * D * 2 + 2.0 * kv_rows * D * 2 + rows * D * 2 + rows * 4
     if w.backward:
         fwd_alg_bytes += rows * 4 + supp_pairs * 6
     fwd_mean = statistics.mean(fwd_ms)
@@ -339,7 +368,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                  "algorithmic_bytes_per_launch": fwd_alg_bytes})
     roof["frac"] = roof["achieved"] / roof["peak"]
     tr = ROOT / "profiles" / ("traffic_workload%d.txt" % w.wid)
-    if tr.exists():
+    if tr.exists() and not variant:
         t = json.loads(tr.read_text())
         if t.get("kernel") == "entmax_fwd_kernel" and t.get("source_hash") == source_hash():
             roof["traffic"] = t["bytes_per_launch"]
@@ -366,6 +395,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "l2": "flushed between timed steps (256 MiB write, outside the step events)",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
+        "variant": {"alpha": alpha, "H_kv": Hkv} if variant else None,
         "fwd_ms": round(fwd_mean, 4),
         "bwd_ms": round(bwd_mean, 4),
         "step_ms_median": round(statistics.median(step_ms), 4),
@@ -378,7 +408,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
-        cb = oracle_baseline(w, inp, budget_s=args.cpu_seconds)
+        cb = oracle_baseline(w, inp, budget_s=args.cpu_seconds, alpha=alpha)
         out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
     return out
 
@@ -392,13 +422,23 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def run_reference(args) -> dict:
+def bench_workload(args) -> Workload:
     w = WORKLOADS[args.workload]
+    if args.hkv:
+        if args.hkv < 1 or w.H % args.hkv:
+            raise SystemExit("--hkv must divide the workload's %d heads" % w.H)
+        w = w.with_shape(H_kv=args.hkv)
+    return w
+
+
+def run_reference(args) -> dict:
+    w = bench_workload(args)
     inp = make_inputs(w)
     per = []
     cb = None
     for k in range(args.warmup + args.steps):
-        cb = oracle_baseline(w, inp, budget_s=args.ref_step_seconds, max_heads=1 if k < args.warmup else 64)
+        cb = oracle_baseline(w, inp, budget_s=args.ref_step_seconds, max_heads=1 if k < args.warmup else 64,
+                             alpha=args.alpha)
         if k >= args.warmup:
             per.append(cb)
     secs = sum(c["seconds"] for c in per)
@@ -460,9 +500,13 @@ def main() -> int:
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--alpha", type=float, default=1.5, help="alpha-entmax variant, alpha in (1, 2]")
+    ap.add_argument("--hkv", type=int, default=0, help="grouped-query variant: key/value heads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if not 1.0 < args.alpha <= 2.0:
+        ap.error("--alpha must lie in (1, 2]")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

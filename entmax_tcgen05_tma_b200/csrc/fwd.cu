@@ -104,11 +104,33 @@ __device__ __forceinline__ float top4_bound(float a0, float a1, float a2, float 
 }
 
 // General alpha (am1 = alpha - 1, p = max(0, am1 (x - tau))^(1/am1) in scaled units x = scale S):
-// at tau = z_k - k^(-am1)/(am1 scale) (raw units) each of the k largest scores adds at least 1/k, so
-// the row's tau is at least that for every k.  Lower bound (raw units) from the four largest chunk
-// maxima (missing values -inf), lowered by a rounding margin; wk[k] = (k+1)^(-am1) / (am1 scale).
-__device__ __forceinline__ float gen_bound(float a0, float a1, float a2, float a3, const float (&wk)[4]) {
-    const float b = fmaxf(fmaxf(a0 - wk[0], a1 - wk[1]), fmaxf(a2 - wk[2], a3 - wk[3]));
+// lower bound (raw units) of the row's tau from the four largest chunk maxima z0 >= .. >= z3 (scores
+// of the row; missing values -inf).  Any subset's threshold is at most the row's.  Start: at
+// tau = z_k - k^(-am1)/(am1 scale) each of the k largest adds at least 1/k, so that is a bound for
+// every k (wk[k] = (k+1)^(-am1) / (am1 scale)).  Then three Newton steps on the four-score
+// constraint g4(t) = sum max(0, u_i - t)^e = 1 (u_i = am1 scale (z_i - z0), e = 1/am1): g4 is
+// convex and decreasing (e >= 1), so from a point with g4 >= 1 the Newton iterates rise towards
+// the four-score threshold without passing it -- each is still a bound.  Lowered by a rounding
+// margin.
+__device__ __forceinline__ float gen_bound(float a0, float a1, float a2, float a3, const float (&wk)[4],
+                                           float am1, float e, float scale) {
+    float b = fmaxf(fmaxf(a0 - wk[0], a1 - wk[1]), fmaxf(a2 - wk[2], a3 - wk[3]));
+    const float c = am1 * scale;  // raw -> y units
+    const float u[4] = {0.f, c * (a1 - a0), c * (a2 - a0), c * (a3 - a0)};
+    float t = c * (b - a0);
+#pragma unroll
+    for (int step = 0; step < 3; ++step) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float d = u[k] - t;
+            const float w = pow_pos(d, e - 1.f);
+            s0 += w;
+            s1 = fmaf(w, fmaxf(d, 0.f), s1);
+        }
+        if (s0 > 0.f) t += fmaxf(s1 - 1.f, 0.f) / (e * s0);
+    }
+    b = fmaxf(b, a0 + t / c);
     return b - 1e-5f * wk[0];
 }
 
@@ -245,7 +267,8 @@ __device__ __forceinline__ float solve_tau(const float* lcv, int r, int h, int n
 }
 
 // General alpha: tau of one row in units y = am1 (scale S - ms) (row max 0, every p term is
-// (y - t)^e with e = 1/am1), candidates split over a lane pair as in solve_tau.  Bisection of
+// (y - t)^e with e = 1/am1), candidates split over a lane pair as in solve_tau.  First Newton's
+// method from lo over all candidates (below); rows of a warp that it has not settled go on with: bisection of
 // [lo, hi] (g(lo) >= 1 >= g(hi)) with the same every-four-halvings stop once no candidate lies
 // strictly inside the bracket and g(lo) <= 1.5; then Newton's method on the support
 // S = {y > midpoint} so fixed, started at lo: on S, phi(t) = sum (y - t)^e - 1 is convex and
@@ -263,8 +286,34 @@ __device__ __forceinline__ float solve_tau_gen(const float* lcv, int r, int h, i
         const int en = 2 * k + h;
         y[k] = k < nh ? am1 * fmaf(scale, lcv[(en < n0 ? en : CAPW + (en - n0)) * TILE + r], -ms) : -INFINITY;
     }
+    // Newton's method from lo on all candidates: g is convex and decreasing (e >= 1), g(lo) >= 1, so
+    // the iterates rise monotonically to the root; stop when every row of the warp moved by less
+    // than 2e-7 (y units).  Rows that have not by then continue with the bisection below from the
+    // raised lower end.
+    bool conv = false;
+    {
+        const float em1 = e - 1.f;
+#pragma unroll 1
+        for (int step = 0; step < 8; ++step) {
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < NC; ++k) {
+                const float d = y[k] - lo;
+                const float w = pow_pos(d, em1);
+                s0 += w;
+                s1 = fmaf(w, fmaxf(d, 0.f), s1);
+            }
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+            const float dt = s0 > 0.f ? fmaxf(s1 - 1.f, 0.f) / (e * s0) : 0.f;
+            lo = fminf(lo + dt, hi);
+            conv = dt <= 2e-7f;
+            if (__all_sync(0xffffffffu, conv)) break;
+        }
+        if (__all_sync(0xffffffffu, conv)) return lo;
+    }
     bool settled = false;
-    float glo = INFINITY;  // g(lo), once lo has moved
+    float glo = conv ? 1.f : INFINITY;  // g(lo), once known (a converged Newton lo is at the root)
     for (int it = 0; it < 25; ++it) {
         const float mid = 0.5f * (lo + hi);
         float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
@@ -771,7 +820,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         // scores at or below t are outside the support: the largest chunk maximum seen minus 2
         // (scaled), raised to the exact threshold of the four largest chunk maxima seen (any
         // subset's threshold is at most tau)
-        const float t = GEN ? gen_bound(a0, a1, a2, a3, wk)
+        const float t = GEN ? gen_bound(a0, a1, a2, a3, wk, am1, ex, scale)
                             : fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
 
         // ---------------- pass B: candidates s > m - 2 (scaled) into this warpgroup's partition
@@ -864,7 +913,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         top4_insert(s1.a1, b0, b1, b2, b3);
         top4_insert(s1.a2, b0, b1, b2, b3);
         top4_insert(s1.a3, b0, b1, b2, b3);
-        const float t_cut = GEN ? gen_bound(b0, b1, b2, b3, wk)
+        const float t_cut = GEN ? gen_bound(b0, b1, b2, b3, wk, am1, ex, scale)
                                 : fmaxf(b0 - two_over_scale, top4_bound(b0, b1, b2, b3, c4));
         // general alpha, in y units: g(-1) >= 1 from the max alone, g(-k^(-am1)) <= 1 over k candidates
         const float hi = GEN ? -pow_pos((float)max(s0.n + s1.n, 1), -am1) : -2.f / sqrtf((float)max(s0.n + s1.n, 1));
