@@ -483,9 +483,30 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
     auto unit = [&](float s) { return GEN ? am1 * (s - m) : s; };
     float blo = GEN ? -1.f : m - 2.f;
     float bhi = GEN ? -pow_pos((float)nallow, -am1) : m - 2.f / sqrtf((float)nallow);
+    // Newton's method from blo (g(blo) >= 1; g convex and decreasing, so the iterates rise to the
+    // root without passing it), at most eight steps; converged: the support is {y > blo} up to
+    // scores within 1e-6 of the root.  Otherwise the bisection below continues from the raised blo.
+    bool conv = false;
+    for (int step = 0; step < 8 && !conv; ++step) {
+        float s0 = 0.f, s1 = 0.f;  // GEN: sum (y-t)^(e-1), sum (y-t)^e; 1.5: sum (s-t), sum (s-t)^2
+        for (int e = tid; e < span; e += NUM_THREADS) {
+            const float d = unit(sbuf[e]) - blo;
+            if (d > 0.f) {
+                const float w = GEN ? pow_pos(d, ex - 1.f) : d;
+                s0 += w;
+                s1 = fmaf(w, d, s1);
+            }
+        }
+        const float2 sums = block_sum2(s0, s1, red);  // uniform across the CTA
+        const float g = GEN ? sums.y : 0.25f * sums.y;
+        const float dg = GEN ? ex * sums.x : 0.5f * sums.x;
+        const float dt = dg > 0.f ? fmaxf(g - 1.f, 0.f) / dg : 0.f;
+        blo = fminf(blo + dt, bhi);
+        conv = dt <= 1e-6f;
+    }
     bool resolved = false;
-    float glo = INFINITY;  // g(blo) once blo has moved (general alpha: Newton needs g(blo) <= 1.5)
-    for (int it = 0; it < 25; ++it) {
+    float glo = conv ? 1.f : INFINITY;  // g(blo) once known (general alpha: Newton needs g(blo) <= 1.5)
+    for (int it = 0; it < (conv ? 0 : 25); ++it) {
         const float mid = 0.5f * (blo + bhi);
         float gl = 0.f, inside = 0.f;
         for (int e = tid; e < span; e += NUM_THREADS) {
@@ -513,7 +534,9 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         }
     }
     float t;
-    if (!resolved) {
+    if (conv) {
+        resolved = true;  // Newton converged: the support is {scores >= blo}
+    } else if (!resolved) {
         // one more count: the last halving may have emptied the bracket
         float inside = 0.f;
         for (int e = tid; e < span; e += NUM_THREADS) {
@@ -522,10 +545,15 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         }
         resolved = block_sum2(inside, 0.f, red).x == 0.f && (!GEN || glo <= 1.5f);
     }
+    // support of the finish: the scores at or above the bracket's upper end once none lies inside
+    // the bracket, or at or above blo after a converged Newton phase
+    const float cut = conv ? blo : bhi;
     if (GEN) {
         // Newton's method on the fixed support {y >= bhi}, from blo (monotone, see solve_tau_gen)
         float tt = blo;
-        if (resolved) {
+        if (conv) {
+            t = blo;
+        } else if (resolved) {
             for (int step = 0; step < 6; ++step) {
                 float s0 = 0.f, s1 = 0.f;
                 for (int e = tid; e < span; e += NUM_THREADS) {
@@ -548,7 +576,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         float k = 0.f, s1 = 0.f, s2 = 0.f;
         for (int e = tid; e < span; e += NUM_THREADS) {
             const float s = sbuf[e];
-            if (s >= bhi) {
+            if (s >= cut) {
                 const float x = s - m;
                 k += 1.f;
                 s1 += x;
