@@ -14,6 +14,8 @@ from ._binding import (  # noqa: F401
     ENTMAX_ERR_UNSUPPORTED,
     ENTMAX_ERR_WORKSPACE,
     ENTMAX_F32,
+    ENTMAX_LAYOUT_BHLD,
+    ENTMAX_LAYOUT_BLHD,
     ENTMAX_OK,
     EXPORTED,
     LIB_PATH,

@@ -23,6 +23,8 @@ ENTMAX_ERR_TIMEOUT = -4
 ENTMAX_ERR_WORKSPACE = -5
 ENTMAX_BF16 = 0
 ENTMAX_F32 = 1
+ENTMAX_LAYOUT_BHLD = 0
+ENTMAX_LAYOUT_BLHD = 1
 
 EXPORTED = (
     "entmax_attn_fwd",
@@ -86,10 +88,10 @@ def _load_library() -> ctypes.CDLL:
     lib.entmax_attn_bwd_saved_gqa.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, i, vp, vp, sz, vp, vp, vp, vp,
                                               vp, sz, vp]
     lib.entmax_attn_fwd_ex.restype = i
-    lib.entmax_attn_fwd_ex.argtypes = [vp, vp, vp, i, vp, i, i, f, f, i, i, i, i, i, vp, i, vp, vp, sz, vp]
+    lib.entmax_attn_fwd_ex.argtypes = [vp, vp, vp, i, vp, i, i, f, f, i, i, i, i, i, i, vp, i, vp, vp, sz, vp]
     lib.entmax_attn_bwd_saved_ex.restype = i
-    lib.entmax_attn_bwd_saved_ex.argtypes = [vp, vp, vp, i, vp, i, i, f, f, i, i, i, i, i, vp, vp, sz, vp, vp, vp,
-                                             vp, vp, sz, vp]
+    lib.entmax_attn_bwd_saved_ex.argtypes = [vp, vp, vp, i, vp, i, i, f, f, i, i, i, i, i, i, vp, vp, sz, vp, vp,
+                                             vp, vp, vp, sz, vp]
     lib.entmax_attn_strerror.restype = ctypes.c_char_p
     lib.entmax_attn_strerror.argtypes = [i]
     lib.entmax_attn_device_status.restype = i
@@ -139,13 +141,15 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError("inputs must be bfloat16 or float32, got %s" % t.dtype)
 
 
-def _check_input(name: str, t: torch.Tensor, shape, dtype=None) -> None:
+def _check_input(name: str, t: torch.Tensor, shape, dtype=None, layout: int = ENTMAX_LAYOUT_BHLD) -> None:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor" % name)
     if tuple(t.shape) != tuple(shape):
         raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
-    if not t.is_contiguous():
+    if layout == ENTMAX_LAYOUT_BHLD and not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
+    if layout == ENTMAX_LAYOUT_BLHD and not t.transpose(1, 2).is_contiguous():
+        raise ValueError("%s must be a [B,H,L,D] view of a contiguous [B,L,H,D] tensor, like Q" % name)
     if dtype is not None and t.dtype != dtype:
         raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
 
@@ -159,6 +163,26 @@ def _mask_ptr(key_mask, B: int, L: int, device) -> int | None:
     if key_mask.device != device:
         raise ValueError("key_mask must be on the same device as Q")
     return key_mask.data_ptr()
+
+
+def _layout_of(Q) -> int:
+    """ENTMAX_LAYOUT_BHLD for a contiguous [B,H,L,D] tensor; ENTMAX_LAYOUT_BLHD for the [B,H,L,D] view
+    (x.transpose(1, 2)) of a contiguous [B,L,H,D] tensor x."""
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be a 4-D [B,H,L,D] tensor")
+    if Q.is_contiguous():
+        return ENTMAX_LAYOUT_BHLD
+    if Q.transpose(1, 2).is_contiguous():
+        return ENTMAX_LAYOUT_BLHD
+    raise ValueError("Q must be contiguous [B,H,L,D], or the transpose(1, 2) view of a contiguous [B,L,H,D]")
+
+
+def _empty(shape, dtype, device, layout: int) -> torch.Tensor:
+    """Output tensor of shape [B,H,L,D] in the given memory layout."""
+    if layout == ENTMAX_LAYOUT_BLHD:
+        B, H, L, D = shape
+        return torch.empty((B, L, H, D), dtype=dtype, device=device).transpose(1, 2)
+    return torch.empty(shape, dtype=dtype, device=device)
 
 
 def _kv_heads(Q, K, grouped: bool) -> int:
@@ -177,24 +201,25 @@ def _kv_heads(Q, K, grouped: bool) -> int:
 def _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, grouped, alpha=None):
     B, H, L, D = Q.shape
     Hkv = _kv_heads(Q, K, grouped or alpha is not None)
-    _check_input("Q", Q, (B, H, L, D))
-    _check_input("K", K, (B, Hkv, L, D), Q.dtype)
-    _check_input("V", V, (B, Hkv, L, D), Q.dtype)
+    lay = _layout_of(Q) if alpha is not None else ENTMAX_LAYOUT_BHLD  # strided inputs: _ex calls only
+    _check_input("Q", Q, (B, H, L, D), None, lay)
+    _check_input("K", K, (B, Hkv, L, D), Q.dtype, lay)
+    _check_input("V", V, (B, Hkv, L, D), Q.dtype, lay)
     if scale is None:
         scale = D ** -0.5
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("out_dtype must be bfloat16 or float32")
     if O is None:
-        O = torch.empty((B, H, L, D), dtype=out_dtype, device=Q.device)
+        O = _empty((B, H, L, D), out_dtype, Q.device, lay)
     else:
-        _check_input("O", O, (B, H, L, D), out_dtype)
+        _check_input("O", O, (B, H, L, D), out_dtype, lay)
     if tau is None:
         tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
     else:
         _check_input("tau", tau, (B, H, L), torch.float32)
     if alpha is not None:
         args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
-                int(bool(causal)), int(window), float(scale), float(alpha), B, H, Hkv, L, D, O.data_ptr(),
+                int(bool(causal)), int(window), float(scale), float(alpha), B, H, Hkv, L, D, lay, O.data_ptr(),
                 ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(), None, 0,
                 _stream_handle(stream))
         name = "entmax_attn_fwd_ex"
@@ -308,17 +333,18 @@ def _byte_buffer(t, nbytes: int, device, name: str):
 def _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, grouped, alpha=None):
     B, H, L, D = Q.shape
     Hkv = _kv_heads(Q, K, grouped or alpha is not None)
-    _check_input("Q", Q, (B, H, L, D))
-    _check_input("K", K, (B, Hkv, L, D), Q.dtype)
-    _check_input("V", V, (B, Hkv, L, D), Q.dtype)
+    lay = _layout_of(Q) if alpha is not None else ENTMAX_LAYOUT_BHLD
+    _check_input("Q", Q, (B, H, L, D), None, lay)
+    _check_input("K", K, (B, Hkv, L, D), Q.dtype, lay)
+    _check_input("V", V, (B, Hkv, L, D), Q.dtype, lay)
     if scale is None:
         scale = D ** -0.5
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("out_dtype must be bfloat16 or float32")
     if O is None:
-        O = torch.empty((B, H, L, D), dtype=out_dtype, device=Q.device)
+        O = _empty((B, H, L, D), out_dtype, Q.device, lay)
     else:
-        _check_input("O", O, (B, H, L, D), out_dtype)
+        _check_input("O", O, (B, H, L, D), out_dtype, lay)
     if tau is None:
         tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
     else:
@@ -327,7 +353,7 @@ def _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, save
     saved = _byte_buffer(saved, nbytes, Q.device, "saved")
     if alpha is not None:
         args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
-                int(bool(causal)), int(window), float(scale), float(alpha), B, H, Hkv, L, D, O.data_ptr(),
+                int(bool(causal)), int(window), float(scale), float(alpha), B, H, Hkv, L, D, lay, O.data_ptr(),
                 ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16, tau.data_ptr(), saved.data_ptr(),
                 saved.numel() * saved.element_size(), _stream_handle(stream))
         name = "entmax_attn_fwd_ex"
@@ -361,25 +387,26 @@ def _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK,
                alpha=None):
     B, H, L, D = Q.shape
     Hkv = _kv_heads(Q, K, grouped or alpha is not None)
-    _check_input("Q", Q, (B, H, L, D))
-    _check_input("K", K, (B, Hkv, L, D), Q.dtype)
-    _check_input("V", V, (B, Hkv, L, D), Q.dtype)
-    _check_input("dO", dO, (B, H, L, D), Q.dtype)
+    lay = _layout_of(Q) if alpha is not None else ENTMAX_LAYOUT_BHLD
+    _check_input("Q", Q, (B, H, L, D), None, lay)
+    _check_input("K", K, (B, Hkv, L, D), Q.dtype, lay)
+    _check_input("V", V, (B, Hkv, L, D), Q.dtype, lay)
+    _check_input("dO", dO, (B, H, L, D), Q.dtype, lay)
     _check_input("tau", tau, (B, H, L), torch.float32)
     if scale is None:
         scale = D ** -0.5
     outs = []
     for name, t, heads in (("dQ", dQ, H), ("dK", dK, Hkv), ("dV", dV, Hkv)):
         if t is None:
-            t = torch.empty((B, heads, L, D), dtype=torch.float32, device=Q.device)
+            t = _empty((B, heads, L, D), torch.float32, Q.device, lay)
         else:
-            _check_input(name, t, (B, heads, L, D), torch.float32)
+            _check_input(name, t, (B, heads, L, D), torch.float32, lay)
         outs.append(t)
     ws = _byte_buffer(workspace, entmax_attn_bwd_saved_workspace_size(B, H, L, D), Q.device, "workspace")
     head = (float(alpha), B, H, Hkv) if alpha is not None else (B, H, Hkv) if grouped else (B, H)
     args = (Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q), _mask_ptr(key_mask, B, L, Q.device),
-            int(bool(causal)), int(window), float(scale)) + head + (
-            L, D, tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(), dO.data_ptr(),
+            int(bool(causal)), int(window), float(scale)) + head + (L, D) + ((lay,) if alpha is not None else ()) + (
+            tau.data_ptr(), saved.data_ptr(), saved.numel() * saved.element_size(), dO.data_ptr(),
             outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(), ws.data_ptr(),
             ws.numel() * ws.element_size(), _stream_handle(stream))
     name = ("entmax_attn_bwd_saved_ex" if alpha is not None else
@@ -409,7 +436,9 @@ def entmax_attn_fwd_ex(Q, K, V, key_mask=None, causal=False, window=0, scale=Non
                        out_dtype=torch.bfloat16, O=None, tau=None, saved=None, stream=None):
     """alpha-entmax forward, alpha in (1, 2]; K and V may have fewer heads than Q (H % H_kv == 0).
 
-    Returns (O, tau) or, with ``save=True``, (O, tau, saved) for entmax_attn_bwd_saved_ex."""
+    Q, K, V are [B,H,L,64] tensors: contiguous, or all three the transpose(1, 2) views of contiguous
+    [B,L,H,64] tensors (then O is returned in that layout too).  Returns (O, tau) or, with
+    ``save=True``, (O, tau, saved) for entmax_attn_bwd_saved_ex."""
     if save:
         return _fwd_train(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, saved, stream, True, alpha)
     return _fwd(Q, K, V, key_mask, causal, window, scale, out_dtype, O, tau, stream, True, alpha)
@@ -418,7 +447,7 @@ def entmax_attn_fwd_ex(Q, K, V, key_mask=None, causal=False, window=0, scale=Non
 def entmax_attn_bwd_saved_ex(Q, K, V, tau, saved, dO, key_mask=None, causal=False, window=0, scale=None, alpha=1.5,
                              dQ=None, dK=None, dV=None, workspace=None, stream=None):
     """Backward of entmax_attn_fwd_ex(save=True) with the same alpha.  Returns dQ [B,H,L,64] and
-    dK, dV [B,H_kv,L,64], fp32."""
+    dK, dV [B,H_kv,L,64], fp32, in the memory layout of Q (dO must share it)."""
     return _bwd_saved(Q, K, V, tau, saved, dO, key_mask, causal, window, scale, dQ, dK, dV, workspace, stream, True,
                       alpha)
 
@@ -442,7 +471,8 @@ class EntmaxAttention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, Q, K, V, key_mask=None, causal=False, window=0, scale=None, alpha=1.5):
         grouped = K.shape[1] != Q.shape[1]  # K, V with fewer heads than Q: grouped-query attention
-        a = None if alpha == 1.5 else float(alpha)  # other alpha: the _ex entry points
+        # other alpha, or [B,L,H,D] memory behind the [B,H,L,D] views: the _ex entry points
+        a = None if alpha == 1.5 and Q.is_contiguous() else float(alpha)
         O, tau, saved = _fwd_train(Q, K, V, key_mask, causal, window, scale, torch.bfloat16, None, None, None, None,
                                    grouped, a)
         ctx.save_for_backward(Q, K, V, tau, saved, key_mask if key_mask is not None else torch.empty(0))
@@ -453,6 +483,11 @@ class EntmaxAttention(torch.autograd.Function):
     def backward(ctx, dO):
         Q, K, V, tau, saved, km = ctx.saved_tensors
         has_mask, causal, window, scale, grouped, a = ctx.cfg
-        dQ, dK, dV = _bwd_saved(Q, K, V, tau, saved, dO.to(Q.dtype).contiguous(), km if has_mask else None, causal,
-                                window, scale, None, None, None, None, None, grouped, a)
+        g = dO.to(Q.dtype)
+        if a is not None and _layout_of(Q) == ENTMAX_LAYOUT_BLHD:
+            g = g.transpose(1, 2).contiguous().transpose(1, 2)  # dO in Q's memory layout
+        else:
+            g = g.contiguous()
+        dQ, dK, dV = _bwd_saved(Q, K, V, tau, saved, g, km if has_mask else None, causal, window, scale, None, None,
+                                None, None, None, grouped, a)
         return dQ.to(Q.dtype), dK.to(K.dtype), dV.to(V.dtype), None, None, None, None, None

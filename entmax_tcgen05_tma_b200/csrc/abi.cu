@@ -121,7 +121,7 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, int slot) {
     return e;
 }
 
-cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L, int box_rows) {
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B, int nh, int L, int box_rows) {
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!g_encode) {
@@ -133,9 +133,12 @@ cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L, int
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
         }
     }
-    const cuuint64_t dims[3] = {(cuuint64_t)HEAD_DIM, (cuuint64_t)L, (cuuint64_t)BH};
-    const cuuint64_t strides[2] = {(cuuint64_t)HEAD_DIM * 2, (cuuint64_t)L * HEAD_DIM * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)HEAD_DIM, (cuuint32_t)box_rows, 1};
+    // layout 0 [B, nh, L, 64]: (d, L, B*nh); layout 1 [B, L, nh, 64]: (d, nh, B*L) -- see HeadRef
+    const cuuint64_t row_bytes = (cuuint64_t)HEAD_DIM * 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)HEAD_DIM, (cuuint64_t)(layout ? nh : L),
+                                (cuuint64_t)(layout ? (long long)B * L : (long long)B * nh)};
+    const cuuint64_t strides[2] = {row_bytes, (layout ? (cuuint64_t)nh : (cuuint64_t)L) * row_bytes};
+    const cuuint32_t box[3] = {(cuuint32_t)HEAD_DIM, layout ? 1u : (cuuint32_t)box_rows, layout ? (cuuint32_t)box_rows : 1u};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -204,12 +207,13 @@ int check_alpha(float alpha) {
 }
 
 int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-             int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, void* O, int out_dtype,
-             float* tau, cudaStream_t stream) {
+             int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, int layout, void* O,
+             int out_dtype, float* tau, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
     rc = check_alpha(alpha);
     if (rc) return rc;
+    if (layout != ENTMAX_LAYOUT_BHLD && layout != ENTMAX_LAYOUT_BLHD) return ENTMAX_ERR_ARG;
     rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
     if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
@@ -221,7 +225,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f, layout};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -242,15 +246,15 @@ extern "C" {
 int entmax_attn_fwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
                     int window, float scale, int B, int H, int L, int D, void* O, int out_dtype, float* tau,
                     cudaStream_t stream) {
-    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, O, out_dtype, tau,
-                    stream);
+    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, 0, O, out_dtype,
+                    tau, stream);
 }
 
 int entmax_attn_fwd_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                         int causal, int window, float scale, int B, int H, int Hkv, int L, int D, void* O,
                         int out_dtype, float* tau, cudaStream_t stream) {
-    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, O, out_dtype, tau,
-                    stream);
+    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, 0, O, out_dtype,
+                    tau, stream);
 }
 
 size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D) {
@@ -275,7 +279,7 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f, 0};
     BwdIO io{tau, dO, dQ, dK, dV, static_cast<float*>(workspace)};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -313,12 +317,13 @@ size_t entmax_attn_bwd_saved_workspace_size(int B, int H, int L, int D) {
 
 namespace {
 int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-                   int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, void* O, int out_dtype,
-                   float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
+                   int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, int layout, void* O,
+                   int out_dtype, float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
     rc = check_alpha(alpha);
     if (rc) return rc;
+    if (layout != ENTMAX_LAYOUT_BHLD && layout != ENTMAX_LAYOUT_BLHD) return ENTMAX_ERR_ARG;
     rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
     if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
@@ -337,7 +342,7 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f, layout};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -353,13 +358,14 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
 }
 
 int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-                   int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, const float* tau,
-                   const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV,
-                   void* workspace, size_t ws_bytes, cudaStream_t stream) {
+                   int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, int layout,
+                   const float* tau, const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK,
+                   float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
     rc = check_alpha(alpha);
     if (rc) return rc;
+    if (layout != ENTMAX_LAYOUT_BHLD && layout != ENTMAX_LAYOUT_BLHD) return ENTMAX_ERR_ARG;
     rc = check_kv_heads(H, Hkv, in_dtype);
     if (rc) return rc;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
@@ -374,7 +380,7 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(status_ptr(&status));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f, layout};
     BwdIO io{tau, dO, dQ, dK, dV, nullptr};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -397,22 +403,22 @@ extern "C" {
 int entmax_attn_fwd_train(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                           int causal, int window, float scale, int B, int H, int L, int D, void* O, int out_dtype,
                           float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
-    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, O, out_dtype, tau,
-                          saved, saved_bytes, stream);
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, 0, O, out_dtype,
+                          tau, saved, saved_bytes, stream);
 }
 
 int entmax_attn_fwd_train_gqa(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                               int causal, int window, float scale, int B, int H, int Hkv, int L, int D, void* O,
                               int out_dtype, float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
-    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, O, out_dtype,
-                          tau, saved, saved_bytes, stream);
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, 0, O,
+                          out_dtype, tau, saved, saved_bytes, stream);
 }
 
 int entmax_attn_bwd_saved(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                           int causal, int window, float scale, int B, int H, int L, int D, const float* tau,
                           const void* saved, size_t saved_bytes, const void* dO, float* dQ, float* dK, float* dV,
                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, tau, saved,
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, 0, tau, saved,
                           saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
 }
 
@@ -420,26 +426,26 @@ int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const void* V, int i
                               int causal, int window, float scale, int B, int H, int Hkv, int L, int D,
                               const float* tau, const void* saved, size_t saved_bytes, const void* dO, float* dQ,
                               float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, tau, saved,
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, Hkv, L, D, 0, tau, saved,
                           saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
 }
 
 int entmax_attn_fwd_ex(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-                       int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, void* O,
+                       int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, int layout, void* O,
                        int out_dtype, float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
     if (!saved && saved_bytes == 0)
-        return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, O, out_dtype, tau,
-                        stream);
-    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, O, out_dtype,
-                          tau, saved, saved_bytes, stream);
+        return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, layout, O,
+                        out_dtype, tau, stream);
+    return fwd_train_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, layout, O,
+                          out_dtype, tau, saved, saved_bytes, stream);
 }
 
 int entmax_attn_bwd_saved_ex(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
                              int causal, int window, float scale, float alpha, int B, int H, int Hkv, int L, int D,
-                             const float* tau, const void* saved, size_t saved_bytes, const void* dO, float* dQ,
-                             float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, tau, saved,
-                          saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
+                             int layout, const float* tau, const void* saved, size_t saved_bytes, const void* dO,
+                             float* dQ, float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    return bwd_saved_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, alpha, B, H, Hkv, L, D, layout, tau,
+                          saved, saved_bytes, dO, dQ, dK, dV, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -496,7 +502,7 @@ extern "C" int entmax_attn_bwd_noalloc(const void* Q, const void* K, const void*
     float* scratch = nullptr;
     rc = record(noalloc_scratch(&scratch));
     if (rc) return rc;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f, 0};
     BwdIO io{tau, dO, dQ, dK, dV, scratch};
     return record(launch_bwd(a, io, stream));
 }

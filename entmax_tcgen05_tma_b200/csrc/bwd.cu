@@ -328,7 +328,9 @@ entmax_bwd_rows_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
     const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue row and warpgroup
     ListState st{0, 0};
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, sm.blk, sm.a, sm.b, ctl->nblk);
+        // [B, H, L, 64] tensors (this path takes layout 0 only)
+        const HeadRef hr{0, bh / a.H, bh % a.H, a.H, a.L};
+        if (lane == 0) P::producer(ctl, wc, &map_q, &map_k, hr, i0, sm.blk, sm.a, sm.b, ctl->nblk, hr);
         __syncwarp();
     } else if (warp == WARP_MMA) {
         if (lane == 0) P::mma(ctl, wc, sm.a, sm.b, ctl->nblk);
@@ -482,7 +484,8 @@ entmax_bwd_keys_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
     const int r = tid & (TILE - 1), g = tid >> 7;  // epilogue key and warpgroup
     ListState st{0, 0};
     if (warp == WARP_PRODUCER) {
-        if (lane == 0) P::producer(ctl, wc, &map_k, &map_q, bh, j0, sm.blk, sm.a, sm.b, ctl->nblk);
+        const HeadRef hr{0, bh / a.H, bh % a.H, a.H, a.L};
+        if (lane == 0) P::producer(ctl, wc, &map_k, &map_q, hr, j0, sm.blk, sm.a, sm.b, ctl->nblk, hr);
         __syncwarp();
     } else if (warp == WARP_MMA) {
         if (lane == 0) P::mma(ctl, wc, sm.a, sm.b, ctl->nblk);
@@ -610,9 +613,9 @@ size_t bwd_keys_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream) {
     CUtensorMap mq, mk;
-    cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L, TILE);
+    cudaError_t e = make_tile_map(&mq, a.Q, 0, a.B, a.H, a.L, TILE);
     if (e != cudaSuccess) return e;
-    e = make_tile_map(&mk, a.K, a.B * a.H, a.L, BLK);
+    e = make_tile_map(&mk, a.K, 0, a.B, a.H, a.L, BLK);
     if (e != cudaSuccess) return e;
     e = ensure_smem_attr(reinterpret_cast<const void*>(entmax_bwd_rows_kernel), SMEM_BYTES, 1);
     if (e != cudaSuccess) return e;

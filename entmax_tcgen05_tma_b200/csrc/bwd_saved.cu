@@ -86,11 +86,12 @@ __device__ __forceinline__ float group8_sum(float v) {
     return v;
 }
 
-// Gathered 128-byte rows of one head's [L, 64] slab: lane sd's 16-byte piece of row j.
+// Gathered 128-byte rows: lane sd's 16-byte piece of row j, at x + j * step elements.
 struct GlobalRows {
-    const __nv_bfloat16* x;  // [L, 64] slab of one head
-    __device__ __forceinline__ uint4 get(int j, int sd) const {
-        return __ldg(reinterpret_cast<const uint4*>(x + (size_t)j * HEAD_DIM) + sd);
+    const __nv_bfloat16* x;  // row 0
+    size_t step;             // elements from one row to the next
+    __device__ __forceinline__ uint4 get(size_t j, int sd) const {
+        return __ldg(reinterpret_cast<const uint4*>(x + j * step) + sd);
     }
 };
 // One query row per group of eight lanes (lane sd owns dimensions 8 sd .. 8 sd + 7), row list
@@ -100,10 +101,12 @@ struct GlobalRows {
 // a row the exact pass handles.
 // GEN: general alpha, weights w = b^em1 (em1 = 1/am1 - 1) and p = w b; the buckets then hold p
 // instead of b.
+// qmem: memory row of query row `row` in Q, dO and dQ (layout); bucket entries name it by qmem.
 template <bool GEN, class Rows>
 __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
-                                           const SavedBwdWs& ws, long long row, int cnt, int bhk, const Rows& Vr,
-                                           const Rows& Kr, uint16_t* mj, float* msp, float* mds, int sd, float em1) {
+                                           const SavedBwdWs& ws, long long row, size_t qmem, int cnt, int bhk,
+                                           const Rows& Vr, const Rows& Kr, uint16_t* mj, float* msp, float* mds,
+                                           int sd, float em1) {
     const int L = a.L;
     const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
     const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
@@ -113,7 +116,7 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
     }
     float g[8];
     {
-        const uint4 x = cnt >= 0 ? __ldg(reinterpret_cast<const uint4*>(dO + (size_t)row * HEAD_DIM) + sd)
+        const uint4 x = cnt >= 0 ? __ldg(reinterpret_cast<const uint4*>(dO + qmem * HEAD_DIM) + sd)
                                  : make_uint4(0u, 0u, 0u, 0u);
         unpack8(x, g);
     }
@@ -158,7 +161,7 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
         mds[e] = ds;
         const size_t key = (size_t)bhk * L + mj[e];
         const size_t at = (size_t)bhk * cap + (size_t)ws.key_off[key] + (size_t)atomicAdd(ws.key_cur + key, 1);
-        ws.bucket_i[at] = (uint32_t)row;
+        ws.bucket_i[at] = (uint32_t)qmem;
         ws.bucket_sp[at] = GEN ? w * sp : sp;
         ws.bucket_ds[at] = ds;
     }
@@ -185,7 +188,7 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
         }
     }
     if (cnt >= 0) {
-        float4* dst = reinterpret_cast<float4*>(io.dQ + (size_t)row * HEAD_DIM + 8 * sd);
+        float4* dst = reinterpret_cast<float4*>(io.dQ + qmem * HEAD_DIM + 8 * sd);
         dst[0] = make_float4(a.scale * acc[0], a.scale * acc[1], a.scale * acc[2], a.scale * acc[3]);
         dst[1] = make_float4(a.scale * acc[4], a.scale * acc[5], a.scale * acc[6], a.scale * acc[7]);
     }
@@ -195,10 +198,11 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
 // One key per group of eight lanes: dK_j = scale sum dS Q_i and dV_j = sum p dO_i over key j's bucket,
 // lane sd of the group loading entry e0 + sd and the group sharing it by shuffles; two entries (two
 // 16-byte pieces each per lane) in flight.  valid = false: no key (the group still takes part).
+// key: logical key row (bhk * L + j); kmem: its memory row in K, V, dK and dV (layout).
 template <bool GEN, class Rows>
 __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
-                                           const SavedBwdWs& ws, long long key, bool valid, int bhk, const Rows& Qr,
-                                           const Rows& Gr, int sd, int g0) {
+                                           const SavedBwdWs& ws, long long key, size_t kmem, bool valid, int bhk,
+                                           const Rows& Qr, const Rows& Gr, int sd, int g0) {
     const int L = a.L;
     const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
     const int n = valid ? sv.key_cnt[key] : 0;
@@ -225,8 +229,8 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
                 const bool ok = e0 + t + u < n;
                 pv[u] = ok ? (GEN ? st : st * st) : 0.f;  // p_ij
                 dv[u] = ok ? dt : 0.f;
-                xg[u] = ok ? Gr.get((int)it, sd) : make_uint4(0u, 0u, 0u, 0u);
-                xq[u] = ok ? Qr.get((int)it, sd) : make_uint4(0u, 0u, 0u, 0u);
+                xg[u] = ok ? Gr.get(it, sd) : make_uint4(0u, 0u, 0u, 0u);
+                xq[u] = ok ? Qr.get(it, sd) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
@@ -242,8 +246,8 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
         }
     }
     if (valid) {
-        float4* dk = reinterpret_cast<float4*>(io.dK + (size_t)key * HEAD_DIM + 8 * sd);
-        float4* dv4 = reinterpret_cast<float4*>(io.dV + (size_t)key * HEAD_DIM + 8 * sd);
+        float4* dk = reinterpret_cast<float4*>(io.dK + kmem * HEAD_DIM + 8 * sd);
+        float4* dv4 = reinterpret_cast<float4*>(io.dV + kmem * HEAD_DIM + 8 * sd);
         dk[0] = make_float4(a.scale * ak[0], a.scale * ak[1], a.scale * ak[2], a.scale * ak[3]);
         dk[1] = make_float4(a.scale * ak[4], a.scale * ak[5], a.scale * ak[6], a.scale * ak[7]);
         dv4[0] = make_float4(av[0], av[1], av[2], av[3]);
@@ -266,11 +270,15 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
     for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < R; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long row = grp * RPW + q;
         const int cnt = row < R ? sv.row_cnt[row] : -1;
-        const int bhk = row < R ? kv_head_of((int)(row / L), a.H, a.Hkv) : 0;
-        const size_t head = (size_t)bhk * L * HEAD_DIM;
-        const GlobalRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head};
-        const GlobalRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head};
-        rows_group<GEN>(a, io, sv, ws, row, cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd, em1);
+        const int bh = row < R ? (int)(row / L) : 0;
+        const int b = bh / a.H, i = (int)(row - (long long)bh * L);
+        const int bhk = kv_head_of(bh, a.H, a.Hkv);
+        const HeadRef hq{a.layout, b, bh - b * a.H, a.H, L}, hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};
+        const size_t head = hkv.row(0) * HEAD_DIM, step = hkv.step() * HEAD_DIM;
+        const GlobalRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head, step};
+        const GlobalRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head, step};
+        rows_group<GEN>(a, io, sv, ws, row, hq.row(i), cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd,
+                        em1);
     }
 }
 
@@ -282,14 +290,16 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnAr
     const int q = lane >> 3, sd = lane & 7, g0 = lane & ~7;
     const int L = a.L;
     const long long Rk = (long long)a.B * a.Hkv * L;  // keys
-    // bucket entries name their query row by its global index, so Q and dO are read from the base
-    const GlobalRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q)};
-    const GlobalRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO)};
+    // bucket entries name their query row by its memory row, so Q and dO are read from the base
+    const GlobalRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q), HEAD_DIM};
+    const GlobalRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO), HEAD_DIM};
     for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < Rk; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long key = grp * RPW + q;
         const bool kv = key < Rk;
         const int bhk = kv ? (int)(key / L) : 0;
-        keys_group<GEN>(a, io, sv, ws, key, kv, bhk, Qr, Gr, sd, g0);
+        const int b = bhk / a.Hkv;
+        const HeadRef hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};
+        keys_group<GEN>(a, io, sv, ws, key, hkv.row((int)(key - (long long)bhk * L)), kv, bhk, Qr, Gr, sd, g0);
     }
 }
 
@@ -345,11 +355,13 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
         const int i = (int)(row - bh * L);
         const int b = (int)(bh / a.H);
         const int bhk = kv_head_of((int)bh, a.H, a.Hkv);
-        const size_t head = (size_t)bhk * L * HEAD_DIM;  // K and V rows of the row's KV head
+        const HeadRef hq{a.layout, b, (int)bh - b * a.H, a.H, L};            // rows of Q, dO, dQ
+        const HeadRef hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};          // rows of K, V, dK, dV
+        const size_t qmem = hq.row(i);
         __syncthreads();
         if (tid < HEAD_DIM) {
-            qf[tid] = __bfloat162float(Q[(size_t)row * HEAD_DIM + tid]);
-            gf[tid] = __bfloat162float(dO[(size_t)row * HEAD_DIM + tid]);
+            qf[tid] = __bfloat162float(Q[qmem * HEAD_DIM + tid]);
+            gf[tid] = __bfloat162float(dO[qmem * HEAD_DIM + tid]);
         }
         __syncthreads();
         const float tau = io.tau[row];
@@ -361,12 +373,12 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
             const int j = lo + e;
             float sp = 0.f;
             if (!a.key_mask || a.key_mask[(size_t)b * L + j]) {
-                const float s = a.scale * dot64_f32(qf, K + head + (size_t)j * HEAD_DIM);
+                const float s = a.scale * dot64_f32(qf, K + hkv.row(j) * HEAD_DIM);
                 sp = fmaxf((GEN ? am1 : 0.5f) * (s - tau), 0.f);
             }
             float dA = 0.f;
             if (sp > 0.f) {
-                dA = dot64_f32(gf, V + head + (size_t)j * HEAD_DIM);
+                dA = dot64_f32(gf, V + hkv.row(j) * HEAD_DIM);
                 const float wt = GEN ? pow_pos(sp, em1) : sp;
                 r += wt;
                 w = fmaf(wt, dA, w);
@@ -384,7 +396,7 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
         for (int e = ph; e < span; e += PH) {
             const float sp = sbuf[e];
             if (sp > 0.f) {
-                const size_t key = (size_t)bhk * L + lo + e;
+                const size_t key = hkv.row(lo + e);  // memory row of K, V, dK, dV
                 const float wt = GEN ? pow_pos(sp, em1) : sp;
                 const float ds = wt * (sbuf[L + e] - u);
                 acc = fmaf(ds, __bfloat162float(K[key * HEAD_DIM + d]), acc);
@@ -399,7 +411,7 @@ __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const Att
             float q = 0.f;
 #pragma unroll
             for (int p = 0; p < PH; ++p) q += red[tid + p * HEAD_DIM];
-            io.dQ[(size_t)row * HEAD_DIM + tid] = a.scale * q;
+            io.dQ[qmem * HEAD_DIM + tid] = a.scale * q;
         }
     }
 }

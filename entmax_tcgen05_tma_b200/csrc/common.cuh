@@ -19,6 +19,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 #include "ptx.cuh"
+#include "internal.h"
 
 namespace entmax {
 
@@ -195,21 +196,20 @@ struct Pipe {
         return nb;
     }
 
-    // TMA producer: the fixed A tile (rows a_row0.. of head bh), then njobs streamed B blocks through
-    // the NSTAGE ring.  Job n < n1 loads listed block n * s1 (a first pass over every s1-th block);
-    // job n >= n1 loads listed block n - n1 (a second pass over the whole list).  n1 < 0 means
-    // n1 = nblk, s1 = 1.
+    // TMA producer: the fixed A tile (rows a_row0.. of head ha), then njobs streamed B blocks of head
+    // hb through the NSTAGE ring.  Job n < n1 loads listed block n * s1 (a first pass over every
+    // s1-th block); job n >= n1 loads listed block n - n1 (a second pass over the whole list).
+    // n1 < 0 means n1 = nblk, s1 = 1.
     static __device__ __forceinline__ void producer(Ctl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
-                                                    const CUtensorMap* map_b, int bh, int a_row0,
+                                                    const CUtensorMap* map_b, const HeadRef& ha, int a_row0,
                                                     const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b,
-                                                    int njobs, int n1 = -1, int s1 = 1, int bh_b = -1) {
-        if (bh_b < 0) bh_b = bh;  // head (third coordinate) of the streamed operand
+                                                    int njobs, const HeadRef& hb, int n1 = -1, int s1 = 1) {
         if (n1 < 0) {
             n1 = ctl->nblk;
             s1 = 1;
         }
         mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
-        tma_load_3d(smem_u32(smem_a), map_a, 0, a_row0, bh, smem_u32(&ctl->full_a));
+        tma_load_3d(smem_u32(smem_a), map_a, 0, ha.c1(a_row0), ha.c2(a_row0), smem_u32(&ctl->full_a));
         int issued = 0;
         for (int n = 0; n < njobs; ++n) {
             const int s = n % NSTAGE;
@@ -217,8 +217,8 @@ struct Pipe {
             if (!wait_bounded(smem_u32(&ctl->empty_b[s]), ph ^ 1u, &ctl->abort_flag, wc)) break;
             const int e = n < n1 ? n * s1 : n - n1;
             mbar_arrive_expect_tx(smem_u32(&ctl->full_b[s]), BLK_BYTES);
-            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, (int)(blk_list[e] & ~FULL_BLOCK) * BLK, bh_b,
-                        smem_u32(&ctl->full_b[s]));
+            const int row = (int)(blk_list[e] & ~FULL_BLOCK) * BLK;
+            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, hb.c1(row), hb.c2(row), smem_u32(&ctl->full_b[s]));
             ++issued;
         }
         if (aborted(ctl)) {

@@ -444,13 +444,13 @@ __device__ __forceinline__ float block_max(float a, float* red) {
 template <bool GEN>
 __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                                           const __nv_bfloat16* __restrict__ V, const uint32_t* bits, float* sbuf,
-                                          float* red, int bh, int bhk, int i, int L, int causal, int window, float scale,
-                                          float am1, int nallow, void* O, int out_f32, float* tau) {
+                                          float* red, const HeadRef& hq, const HeadRef& hkv, int bh, int i, int L,
+                                          int causal, int window, float scale, float am1, int nallow, void* O,
+                                          int out_f32, float* tau) {
     const int tid = threadIdx.x;
     float* qf = red + 64;  // 64 floats (red[0..63] holds reduction partials)
-    const size_t head = (size_t)bh * L * HEAD_DIM, kv_head = (size_t)bhk * L * HEAD_DIM;
     __syncthreads();
-    if (tid < HEAD_DIM) qf[tid] = __bfloat162float(Q[head + (size_t)i * HEAD_DIM + tid]);
+    if (tid < HEAD_DIM) qf[tid] = __bfloat162float(Q[hq.row(i) * HEAD_DIM + tid]);
     __syncthreads();
     int lo, hi;
     row_key_range(i, L, causal, window, lo, hi);
@@ -460,7 +460,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         const int j = lo + e;
         float s = -INFINITY;
         if ((bits[j >> 5] >> (j & 31)) & 1u) {
-            const uint4* kr = reinterpret_cast<const uint4*>(K + kv_head + (size_t)j * HEAD_DIM);
+            const uint4* kr = reinterpret_cast<const uint4*>(K + hkv.row(j) * HEAD_DIM);
             float acc = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -606,7 +606,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
                 const float h = 0.5f * (s - t);
                 p = h * h;
             }
-            acc = fmaf(p, __bfloat162float(V[kv_head + (size_t)(lo + e) * HEAD_DIM + d]), acc);
+            acc = fmaf(p, __bfloat162float(V[hkv.row(lo + e) * HEAD_DIM + d]), acc);
         }
     }
     __syncthreads();
@@ -616,7 +616,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         float o = 0.f;
 #pragma unroll
         for (int p = 0; p < PH; ++p) o += red[tid + p * HEAD_DIM];
-        const size_t oi = head + (size_t)i * HEAD_DIM + tid;
+        const size_t oi = hq.row(i) * HEAD_DIM + tid;
         if (out_f32) reinterpret_cast<float*>(O)[oi] = o;
         else reinterpret_cast<__nv_bfloat16*>(O)[oi] = __float2bfloat16_rn(o);
         if (tid == 0) tau[(size_t)bh * L + i] = GEN ? m + t * ex : t;
@@ -631,11 +631,12 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
 __device__ __forceinline__ int half_block(int p, int m, int mA) { return m < mA ? 2 * (p + 2 * m) : p + 2 * (m - mA); }
 
 __device__ __noinline__ void produce_half(PipeCtl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
-                                          const CUtensorMap* map_b, int bh, int bhk, int a_row0, const uint16_t* blk_list,
-                                          uint8_t* smem_a, uint8_t* smem_b, int p, int mA, int mB) {
+                                          const CUtensorMap* map_b, const HeadRef& ha, const HeadRef& hb, int a_row0,
+                                          const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b, int p, int mA,
+                                          int mB) {
     if (p == 0) {
         mbar_arrive_expect_tx(smem_u32(&ctl->full_a), TILE_BYTES);
-        tma_load_3d(smem_u32(smem_a), map_a, 0, a_row0, bh, smem_u32(&ctl->full_a));
+        tma_load_3d(smem_u32(smem_a), map_a, 0, ha.c1(a_row0), ha.c2(a_row0), smem_u32(&ctl->full_a));
     }
     int issued = 0;
     for (int m = 0; m < mA + mB; ++m) {
@@ -643,8 +644,8 @@ __device__ __noinline__ void produce_half(PipeCtl* ctl, const WaitCfg& wc, const
         const uint32_t ph = (uint32_t)(m >> 1) & 1u;
         if (!wait_bounded(smem_u32(&ctl->empty_b[st]), ph ^ 1u, &ctl->abort_flag, wc)) break;
         mbar_arrive_expect_tx(smem_u32(&ctl->full_b[st]), BLK_BYTES);
-        tma_load_3d(smem_u32(smem_b + st * BLK_BYTES), map_b, 0, (int)(blk_list[half_block(p, m, mA)] & ~FULL_BLOCK) * BLK,
-                    bhk, smem_u32(&ctl->full_b[st]));
+        const int row = (int)(blk_list[half_block(p, m, mA)] & ~FULL_BLOCK) * BLK;
+        tma_load_3d(smem_u32(smem_b + st * BLK_BYTES), map_b, 0, hb.c1(row), hb.c2(row), smem_u32(&ctl->full_b[st]));
         ++issued;
     }
     if (P::aborted(ctl)) {
@@ -710,10 +711,14 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int L = args.L;
     const int tile = blockIdx.x, bh = blockIdx.y;
     const int b = bh / args.H;
-    const int bhk = kv_head_of(bh, args.H, args.Hkv);  // K/V head
+    const int bhk = kv_head_of(bh, args.H, args.Hkv);  // K/V head (b * Hkv + index)
+    const HeadRef hq{args.layout, b, bh - b * args.H, args.H, L};          // rows of Q and O
+    const HeadRef hkv{args.layout, b, bhk - b * args.Hkv, args.Hkv, L};    // rows of K and V
     const int i0 = tile * TILE;
     const WaitCfg wc{args.status, args.timeout_ns};
-    const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(args.V) + (size_t)bhk * L * HEAD_DIM;
+    // V row j of this head at Vh + j * vstep
+    const __nv_bfloat16* Vh = reinterpret_cast<const __nv_bfloat16*>(args.V) + hkv.row(0) * HEAD_DIM;
+    const size_t vstep = hkv.step() * HEAD_DIM;
 
     if (tid == 0) {
         mbar_init(smem_u32(vbar), 1);
@@ -766,9 +771,9 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const int p = warp == WARP_PRODUCER ? 0 : 1;
         if (lane == 0) {
             if (resident) {
-                if (p == 0) P::producer(ctl, wc, &map_q, &map_k, bh, i0, blk_list, smem_a, smem_b, njobs, -1, 1, bhk);
+                if (p == 0) P::producer(ctl, wc, &map_q, &map_k, hq, i0, blk_list, smem_a, smem_b, njobs, hkv);
             } else {
-                produce_half(ctl, wc, &map_q, &map_k, bh, bhk, i0, blk_list, smem_a, smem_b, p, p ? mA1 : mA0, p ? mB1 : mB0);
+                produce_half(ctl, wc, &map_q, &map_k, hq, hkv, i0, blk_list, smem_a, smem_b, p, p ? mA1 : mA0, p ? mB1 : mB0);
             }
         }
         __syncwarp();
@@ -870,7 +875,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         if (nc < CAPW) {
                             pcv[nc * TILE + r] = staged(stage, slot, q);
                             pcj[nc * TILE + r] = (uint16_t)(jc + q);
-                            if (!resident) prefetch_l2(Vh + (size_t)(jc + q) * HEAD_DIM);
+                            if (!resident) prefetch_l2(Vh + (size_t)(jc + q) * vstep);
                         }
                         ++nc;
                     } while (hits);
@@ -904,9 +909,10 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     // V blocks of a resident tile into the (now idle) ring, overlapping phase 2
     if (warp == WARP_PRODUCER && lane == 0 && v_staged) {
         mbar_arrive_expect_tx(smem_u32(vbar), (uint32_t)(nblk * BLK_BYTES));
-        for (int s = 0; s < nblk; ++s)
-            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), &map_v, 0, (int)(blk_list[s] & ~FULL_BLOCK) * BLK, bhk,
-                        smem_u32(vbar));
+        for (int s = 0; s < nblk; ++s) {
+            const int row = (int)(blk_list[s] & ~FULL_BLOCK) * BLK;
+            tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), &map_v, 0, hkv.c1(row), hkv.c2(row), smem_u32(vbar));
+        }
     }
 
     // ---------------- phase 2: tau per row, two threads per row (one per partition)
@@ -1044,7 +1050,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     for (int u = 0; u < 2; ++u) {
                         const int ee = e + u < ns ? e + u : e;
                         const int sl = ee < n0 ? ee : CAPW + (ee - n0);
-                        const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)cj[sl * TILE + r] * HEAD_DIM) + 4 * h;
+                        const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)cj[sl * TILE + r] * vstep) + 4 * h;
                         pw[u] = e + u < ns ? (GEN ? pow_pos(cv[sl * TILE + r], ex) : cv[sl * TILE + r]) : 0.f;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) x[u][c] = __ldg(src + c);
@@ -1055,7 +1061,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         for (int c = 0; c < 4; ++c) fma_bf16x8(acc[c], pw[u], x[u][c]);
                 }
             }
-            const size_t oi = ((size_t)bh * L + i) * HEAD_DIM + 32 * h;
+            const size_t oi = hq.row(i) * HEAD_DIM + 32 * h;
             if (out.out_f32) {
                 float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out.O) + oi);
 #pragma unroll
@@ -1088,9 +1094,9 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 mask &= mask - 1;
                 fallback_row<GEN>(reinterpret_cast<const __nv_bfloat16*>(args.Q),
                                   reinterpret_cast<const __nv_bfloat16*>(args.K),
-                                  reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, bh, bhk, i0 + rr,
-                                  L, args.causal, args.window, scale, am1, rows[rr].nallow + rows[TILE + rr].nallow,
-                                  out.O, out.out_f32, out.tau);
+                                  reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, hq, hkv, bh,
+                                  i0 + rr, L, args.causal, args.window, scale, am1,
+                                  rows[rr].nallow + rows[TILE + rr].nallow, out.O, out.out_f32, out.tau);
             }
         }
     }
@@ -1109,11 +1115,11 @@ size_t fwd_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
-    cudaError_t e = make_tile_map(&mq, a.Q, a.B * a.H, a.L, TILE);
+    cudaError_t e = make_tile_map(&mq, a.Q, a.layout, a.B, a.H, a.L, TILE);
     if (e != cudaSuccess) return e;
-    e = make_tile_map(&mk, a.K, a.B * a.Hkv, a.L, BLK);
+    e = make_tile_map(&mk, a.K, a.layout, a.B, a.Hkv, a.L, BLK);
     if (e != cudaSuccess) return e;
-    e = make_tile_map(&mv, a.V, a.B * a.Hkv, a.L, BLK);
+    e = make_tile_map(&mv, a.V, a.layout, a.B, a.Hkv, a.L, BLK);
     if (e != cudaSuccess) return e;
     const bool gen = generic_alpha(a);
     const void* kfn = gen ? reinterpret_cast<const void*>(entmax_fwd_kernel<true>)

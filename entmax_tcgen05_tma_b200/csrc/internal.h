@@ -21,6 +21,23 @@ struct AttnArgs {
     int Hkv;                 // key/value heads (H % Hkv == 0); query head h of batch b reads KV head
                              // b * Hkv + h / (H / Hkv) -- grouped-query attention when Hkv < H
     float am1;               // alpha - 1 in (0, 1]: p = max(0, am1 (S - tau))^(1 / am1); 0.5 is 1.5-entmax
+    int layout;              // 0: Q, K, V, O, dO, dQ, dK, dV are [B, heads, L, 64]; 1: [B, L, heads, 64]
+};
+
+// One head of a [B, nh, L, 64] (layout 0) or [B, L, nh, 64] (layout 1) tensor: its memory rows
+// (units of 64 elements) and the TMA coordinates of a box of its rows.  Layout 0 maps are
+// (d, L, B*nh) with boxes (64, rows, 1) at (0, row, b*nh + hh); layout 1 maps are (d, nh, B*L)
+// with boxes (64, 1, rows) at (0, hh, b*L + row).  Either box lands in shared memory as `rows`
+// consecutive 128-byte rows.  A layout-1 box that runs past row L of its batch reads the next
+// batch's rows (or the zero fill after the last batch): the kernels mask rows and keys >= L.
+struct HeadRef {
+    int layout, b, hh, nh, L;
+    __host__ __device__ __forceinline__ int c1(int row) const { return layout ? hh : row; }
+    __host__ __device__ __forceinline__ int c2(int row) const { return layout ? b * L + row : b * nh + hh; }
+    __host__ __device__ __forceinline__ size_t row(int i) const {
+        return layout ? ((size_t)b * L + i) * nh + hh : ((size_t)b * nh + hh) * L + i;
+    }
+    __host__ __device__ __forceinline__ size_t step() const { return layout ? (size_t)nh : 1; }
 };
 
 // alpha = 1.5 runs the specialised kernels (closed-form tau finish, p = h^2); any other alpha the
@@ -77,7 +94,7 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
                              cudaStream_t stream);
 
 // Tensor map over a [B*H, L, 64] bf16 tensor, boxes of box_rows rows, 128-byte swizzle.
-cudaError_t make_tile_map(CUtensorMap* map, const void* base, int BH, int L, int box_rows);
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B, int nh, int L, int box_rows);
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
 cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);

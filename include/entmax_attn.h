@@ -21,8 +21,8 @@
  * Masked keys are excluded, not filled with a large negative value.  A row with no allowed
  * key gets O_i = 0, tau_i = +inf and zero gradients.
  *
- * Layout: Q, K, V, dO, O, dQ, dK, dV are contiguous row-major [B, H, L, D] tensors; tau is
- * [B, H, L]; key_mask is [B, L] bytes.  D must be 64.  All pointers are DEVICE pointers owned
+ * Layout: Q, K, V, dO, O, dQ, dK, dV are contiguous row-major [B, H, L, D] tensors (the _ex entry
+ * points also take [B, L, H, D]: entmax_layout); tau is [B, H, L]; key_mask is [B, L] bytes.  D must be 64.  All pointers are DEVICE pointers owned
  * by the caller; the library keeps no reference after a call returns.  Every call is
  * asynchronous on `stream` (0 = the legacy default stream).
  *
@@ -60,6 +60,15 @@ typedef enum {
     ENTMAX_BF16 = 0,
     ENTMAX_F32 = 1
 } entmax_dtype;
+
+/* Memory layout of Q, K, V, O, dO, dQ, dK, dV for the _ex entry points (every other entry point
+ * takes ENTMAX_LAYOUT_BHLD).  BLHD is the [B, L, heads, 64] tensor that the attention layer of page
+ * "svd-sst2-roberta-adasplash" (section 3, the reshape-and-transpose step) views as [B, heads, L, 64]:
+ * passing it directly avoids a transposing copy.  tau is [B, H, L] in both. */
+typedef enum {
+    ENTMAX_LAYOUT_BHLD = 0, /* [B, heads, L, 64], rows of one head contiguous */
+    ENTMAX_LAYOUT_BLHD = 1  /* [B, L, heads, 64], heads of one position contiguous */
+} entmax_layout;
 
 /*
  * Forward pass.
@@ -187,17 +196,20 @@ ENTMAX_API int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const voi
  *              the same alpha, Q, K, masks and scale.  Each saved entry holds b_ij = a (S_ij - tau_i)
  *              (sqrt(p_ij) at alpha = 1.5).
  *   tau        fp32 [B, H, L], score units for every alpha (+inf for a row with no allowed key).
+ *   layout     ENTMAX_LAYOUT_BHLD or ENTMAX_LAYOUT_BLHD (else ENTMAX_ERR_ARG), for all of Q, K, V,
+ *              O, dO, dQ, dK, dV alike (K, V, dK, dV with H_kv heads).  The saved supports do not
+ *              depend on it.
  * Other arguments, layouts and errors: as entmax_attn_fwd / _fwd_train / _bwd_saved and their _gqa
  * forms.
  */
 ENTMAX_API int entmax_attn_fwd_ex(const void* Q, const void* K, const void* V, int in_dtype,
                                   const uint8_t* key_mask, int causal, int window, float scale, float alpha,
-                                  int B, int H, int H_kv, int L, int D,
+                                  int B, int H, int H_kv, int L, int D, int layout,
                                   void* O, int out_dtype, float* tau,
                                   void* saved, size_t saved_bytes, cudaStream_t stream);
 ENTMAX_API int entmax_attn_bwd_saved_ex(const void* Q, const void* K, const void* V, int in_dtype,
                                         const uint8_t* key_mask, int causal, int window, float scale,
-                                        float alpha, int B, int H, int H_kv, int L, int D,
+                                        float alpha, int B, int H, int H_kv, int L, int D, int layout,
                                         const float* tau, const void* saved, size_t saved_bytes,
                                         const void* dO, float* dQ, float* dK, float* dV,
                                         void* workspace, size_t ws_bytes, cudaStream_t stream);

@@ -181,14 +181,14 @@ def test_binding_rejects_bad_kv_head_count():
         E.entmax_attn_fwd_gqa(q, k, k)
 
 
-def _ex_calls(alpha, B=1, H=2, Hkv=2, in_dtype=0, saved=P, saved_bytes=None):
+def _ex_calls(alpha, B=1, H=2, Hkv=2, in_dtype=0, saved=P, saved_bytes=None, layout=0):
     R = max(B * H * 64, 1)
     need = E.entmax_attn_saved_bytes(1, 1, R) if saved_bytes is None else saved_bytes
     ws = E.entmax_attn_bwd_saved_workspace_size(1, 1, R)
-    f = E.lib.entmax_attn_fwd_ex(P, P, P, in_dtype, None, 0, 0, 0.125, alpha, B, H, Hkv, 64, 64, P, 0, P, saved,
-                                 need, None)
-    b = E.lib.entmax_attn_bwd_saved_ex(P, P, P, in_dtype, None, 0, 0, 0.125, alpha, B, H, Hkv, 64, 64, P, P, need,
-                                       P, P, P, P, P, ws, None)
+    f = E.lib.entmax_attn_fwd_ex(P, P, P, in_dtype, None, 0, 0, 0.125, alpha, B, H, Hkv, 64, 64, layout, P, 0, P,
+                                 saved, need, None)
+    b = E.lib.entmax_attn_bwd_saved_ex(P, P, P, in_dtype, None, 0, 0, 0.125, alpha, B, H, Hkv, 64, 64, layout, P, P,
+                                       need, P, P, P, P, P, ws, None)
     return f, b
 
 
@@ -224,3 +224,23 @@ def test_binding_rejects_bad_alpha_before_the_library():
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         E.entmax_attn_fwd_ex(q, q, q, alpha=1.5)  # CPU tensors are refused first
+
+
+@pytest.mark.parametrize("layout", [-1, 2, 7])
+def test_layout_argument_checks(layout):
+    assert _ex_calls(1.5, layout=layout) == (E.ENTMAX_ERR_ARG, E.ENTMAX_ERR_ARG)
+    assert _ex_calls(1.75, B=0, layout=1) == (E.ENTMAX_OK, E.ENTMAX_OK)
+
+
+def test_binding_layout_detection():
+    import torch
+
+    from entmax_tcgen05_tma_b200 import _binding as bnd
+
+    x = torch.zeros(2, 5, 3, 64)  # [B, L, H, D] memory
+    assert bnd._layout_of(x.transpose(1, 2)) == E.ENTMAX_LAYOUT_BLHD
+    assert bnd._layout_of(torch.zeros(2, 3, 5, 64)) == E.ENTMAX_LAYOUT_BHLD
+    with pytest.raises(ValueError):
+        bnd._layout_of(torch.zeros(2, 3, 64, 5).transpose(2, 3))  # d not innermost
+    y = bnd._empty((2, 3, 5, 64), torch.float32, "cpu", E.ENTMAX_LAYOUT_BLHD)
+    assert y.shape == (2, 3, 5, 64) and y.transpose(1, 2).is_contiguous()
