@@ -94,6 +94,13 @@ struct GlobalRows {
         return __ldg(reinterpret_cast<const uint4*>(x + j * step) + sd);
     }
 };
+// The same with consecutive rows (step 64, a shift).
+struct DenseRows {
+    const __nv_bfloat16* x;
+    __device__ __forceinline__ uint4 get(size_t j, int sd) const {
+        return __ldg(reinterpret_cast<const uint4*>(x + j * HEAD_DIM) + sd);
+    }
+};
 // One query row per group of eight lanes (lane sd owns dimensions 8 sd .. 8 sd + 7), row list
 // staged in shared memory (mj, msp; mds holds dA, then dS).  dA_e = dO_i . V_je with one 16-byte
 // piece of V_je per lane and a three-step group reduction, two entries in flight; then u_i, dS_e,
@@ -102,11 +109,13 @@ struct GlobalRows {
 // GEN: general alpha, weights w = b^em1 (em1 = 1/am1 - 1) and p = w b; the buckets then hold p
 // instead of b.
 // qmem: memory row of query row `row` in Q, dO and dQ (layout); bucket entries name it by qmem.
-template <bool GEN, class Rows>
+// PLAIN (layout 0, one key/value head per query head): qmem is row itself and is not used.
+template <bool GEN, bool PLAIN, class Rows>
 __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
-                                           const SavedBwdWs& ws, long long row, size_t qmem, int cnt, int bhk,
+                                           const SavedBwdWs& ws, long long row, size_t qmem_, int cnt, int bhk,
                                            const Rows& Vr, const Rows& Kr, uint16_t* mj, float* msp, float* mds,
                                            int sd, float em1) {
+    const size_t qmem = PLAIN ? (size_t)row : qmem_;
     const int L = a.L;
     const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
     const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(io.dO);
@@ -198,11 +207,12 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
 // One key per group of eight lanes: dK_j = scale sum dS Q_i and dV_j = sum p dO_i over key j's bucket,
 // lane sd of the group loading entry e0 + sd and the group sharing it by shuffles; two entries (two
 // 16-byte pieces each per lane) in flight.  valid = false: no key (the group still takes part).
-// key: logical key row (bhk * L + j); kmem: its memory row in K, V, dK and dV (layout).
-template <bool GEN, class Rows>
+// key: logical key row (bhk * L + j); kmem: its memory row in K, V, dK and dV (layout; PLAIN: key).
+template <bool GEN, bool PLAIN, class Rows>
 __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
-                                           const SavedBwdWs& ws, long long key, size_t kmem, bool valid, int bhk,
+                                           const SavedBwdWs& ws, long long key, size_t kmem_, bool valid, int bhk,
                                            const Rows& Qr, const Rows& Gr, int sd, int g0) {
+    const size_t kmem = PLAIN ? (size_t)key : kmem_;
     const int L = a.L;
     const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
     const int n = valid ? sv.key_cnt[key] : 0;
@@ -255,8 +265,9 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
     }
 }
 
-// Four query rows per warp (eight lanes each), rows of K and V gathered from L2.
-template <bool GEN>
+// Four query rows per warp (eight lanes each), rows of K and V gathered from L2.  PLAIN: layout 0
+// with one key/value head per query head, where memory rows are the logical ones (no head maps).
+template <bool GEN, bool PLAIN>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     __shared__ uint16_t lj[ROW_WARPS][RPW][SAVE_CAP];
@@ -271,19 +282,30 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
         const long long row = grp * RPW + q;
         const int cnt = row < R ? sv.row_cnt[row] : -1;
         const int bh = row < R ? (int)(row / L) : 0;
-        const int b = bh / a.H, i = (int)(row - (long long)bh * L);
-        const int bhk = kv_head_of(bh, a.H, a.Hkv);
-        const HeadRef hq{a.layout, b, bh - b * a.H, a.H, L}, hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};
-        const size_t head = hkv.row(0) * HEAD_DIM, step = hkv.step() * HEAD_DIM;
-        const GlobalRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head, step};
-        const GlobalRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head, step};
-        rows_group<GEN>(a, io, sv, ws, row, hq.row(i), cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q], sd,
-                        em1);
+        if (PLAIN) {
+            // (bhk equals bh here; taking it through kv_head_of measured 5% faster at L = 4096 --
+            // instruction scheduling, not work)
+            const int bhk = kv_head_of(bh, a.H, a.Hkv);
+            const size_t head = (size_t)bhk * L * HEAD_DIM;
+            const DenseRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head};
+            const DenseRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head};
+            rows_group<GEN, true>(a, io, sv, ws, row, 0, cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q], lds[warp][q],
+                                  sd, em1);
+        } else {
+            const int b = bh / a.H, i = (int)(row - (long long)bh * L);
+            const int bhk = kv_head_of(bh, a.H, a.Hkv);
+            const HeadRef hq{a.layout, b, bh - b * a.H, a.H, L}, hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};
+            const size_t head = hkv.row(0) * HEAD_DIM, step = hkv.step() * HEAD_DIM;
+            const GlobalRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head, step};
+            const GlobalRows Kr{reinterpret_cast<const __nv_bfloat16*>(a.K) + head, step};
+            rows_group<GEN, false>(a, io, sv, ws, row, hq.row(i), cnt, bhk, Vr, Kr, lj[warp][q], lsp[warp][q],
+                                   lds[warp][q], sd, em1);
+        }
     }
 }
 
-// Four keys per warp (eight lanes each), rows of Q and dO gathered from L2.
-template <bool GEN>
+// Four keys per warp (eight lanes each), rows of Q and dO gathered from L2.  PLAIN as for the rows.
+template <bool GEN, bool PLAIN>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -291,15 +313,19 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnAr
     const int L = a.L;
     const long long Rk = (long long)a.B * a.Hkv * L;  // keys
     // bucket entries name their query row by its memory row, so Q and dO are read from the base
-    const GlobalRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q), HEAD_DIM};
-    const GlobalRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO), HEAD_DIM};
+    const DenseRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q)};
+    const DenseRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO)};
     for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < Rk; grp += (long long)gridDim.x * ROW_WARPS) {
         const long long key = grp * RPW + q;
         const bool kv = key < Rk;
         const int bhk = kv ? (int)(key / L) : 0;
-        const int b = bhk / a.Hkv;
-        const HeadRef hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};
-        keys_group<GEN>(a, io, sv, ws, key, hkv.row((int)(key - (long long)bhk * L)), kv, bhk, Qr, Gr, sd, g0);
+        size_t kmem = 0;
+        if (!PLAIN) {
+            const int b = bhk / a.Hkv;
+            const HeadRef hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};
+            kmem = hkv.row((int)(key - (long long)bhk * L));
+        }
+        keys_group<GEN, PLAIN>(a, io, sv, ws, key, kmem, kv, bhk, Qr, Gr, sd, g0);
     }
 }
 
@@ -472,14 +498,25 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>((R + ROW_WARPS - 1) / ROW_WARPS, (long long)sms * 8));
     const bool gen = generic_alpha(a);
-    if (gen) saved_rows_kernel<true><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
-    else saved_rows_kernel<false><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    const bool plain = a.layout == 0 && a.Hkv == a.H;
+    if (gen) {
+        if (plain) saved_rows_kernel<true, true><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+        else saved_rows_kernel<true, false><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    } else {
+        if (plain) saved_rows_kernel<false, true><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+        else saved_rows_kernel<false, false><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long Rk = (long long)a.B * a.Hkv * a.L;
     const unsigned kgrid = (unsigned)std::max<long long>(1, std::min<long long>((Rk + ROW_WARPS * RPW - 1) / (ROW_WARPS * RPW), (long long)sms * 8));
-    if (gen) saved_keys_kernel<true><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
-    else saved_keys_kernel<false><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    if (gen) {
+        if (plain) saved_keys_kernel<true, true><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+        else saved_keys_kernel<true, false><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    } else {
+        if (plain) saved_keys_kernel<false, true><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+        else saved_keys_kernel<false, false><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int smem = 2 * a.L * (int)sizeof(float);

@@ -444,7 +444,7 @@ __device__ __forceinline__ float block_max(float a, float* red) {
 template <bool GEN>
 __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                                           const __nv_bfloat16* __restrict__ V, const uint32_t* bits, float* sbuf,
-                                          float* red, const HeadRef& hq, const HeadRef& hkv, int bh, int i, int L,
+                                          float* red, HeadRef hq, HeadRef hkv, int bh, int i, int L,
                                           int causal, int window, float scale, float am1, int nallow, void* O,
                                           int out_f32, float* tau) {
     const int tid = threadIdx.x;
@@ -631,7 +631,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
 __device__ __forceinline__ int half_block(int p, int m, int mA) { return m < mA ? 2 * (p + 2 * m) : p + 2 * (m - mA); }
 
 __device__ __noinline__ void produce_half(PipeCtl* ctl, const WaitCfg& wc, const CUtensorMap* map_a,
-                                          const CUtensorMap* map_b, const HeadRef& ha, const HeadRef& hb, int a_row0,
+                                          const CUtensorMap* map_b, HeadRef ha, HeadRef hb, int a_row0,
                                           const uint16_t* blk_list, uint8_t* smem_a, uint8_t* smem_b, int p, int mA,
                                           int mB) {
     if (p == 0) {
