@@ -987,21 +987,30 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             // this thread's partition of the support: cv <- p_ij (alpha 1.5) or b_ij = y - t (general
             // alpha; p = b^ex), cj <- j (in place)
             int sn = 0;
-            for (int k = 0; k < nh; ++k) {
-                const float xv = fmaf(scale, pcv[k * TILE + r], -ms);
+            auto keep = [&](float c, uint16_t j) {
+                const float xv = fmaf(scale, c, -ms);
                 if (GEN) {
                     const float b = am1 * xv - tau_x;
                     if (b > 0.f) {
                         pcv[sn * TILE + r] = b;
-                        pcj[sn * TILE + r] = pcj[k * TILE + r];
+                        pcj[sn * TILE + r] = j;
                         ++sn;
                     }
                 } else if (xv > tau_x) {
                     const float hh = 0.5f * (xv - tau_x);
                     pcv[sn * TILE + r] = hh * hh;
-                    pcj[sn * TILE + r] = pcj[k * TILE + r];
+                    pcj[sn * TILE + r] = j;
                     ++sn;
                 }
+            };
+            // two entries per step, both read before either is written back (writes go to slots
+            // sn <= k, never past the entries still to be read)
+            for (int k = 0; k < nh; k += 2) {
+                const bool two = k + 1 < nh;
+                const float c0 = pcv[k * TILE + r], c1 = two ? pcv[(k + 1) * TILE + r] : -INFINITY;
+                const uint16_t j0 = pcj[k * TILE + r], j1 = two ? pcj[(k + 1) * TILE + r] : (uint16_t)0;
+                keep(c0, j0);
+                keep(c1, j1);
             }
             supp_cnt[h * TILE + r] = sn;
             if (h == 0) out.tau[(size_t)bh * L + i] = GEN ? ms + tau_x * ex : ms + tau_x;
@@ -1028,17 +1037,30 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 for (int k = 0; k < 8; ++k) acc[c][k] = 0.f;
             const int ns = n0 + n1;
             if (v_staged) {
-                for (int e = 0; e < ns; ++e) {
-                    const int sl = e < n0 ? e : CAPW + (e - n0);
-                    const int j = cj[sl * TILE + r];
-                    const float p = GEN ? pow_pos(cv[sl * TILE + r], ex) : cv[sl * TILE + r];
-                    // 128-byte swizzled V block in ring slot vslot[j / BLK]: 16-byte chunk c of row
-                    // `row` sits at chunk position c ^ (row & 7)
-                    const uint32_t row = (uint32_t)j & (BLK - 1);
-                    const uint8_t* base = smem_b + vslot[j / BLK] * BLK_BYTES + row * 128u;
+                // two support entries per step (their shared-memory reads overlap; a missing second
+                // entry repeats the first with weight 0)
+                for (int e = 0; e < ns; e += 2) {
+                    uint4 x[2][4];
+                    float pw[2];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        fma_bf16x8(acc[c], p, *reinterpret_cast<const uint4*>(base + ((((uint32_t)(4 * h + c)) ^ (row & 7u)) << 4)));
+                    for (int u = 0; u < 2; ++u) {
+                        const int ee = e + u < ns ? e + u : e;
+                        const int sl = ee < n0 ? ee : CAPW + (ee - n0);
+                        const int j = cj[sl * TILE + r];
+                        const float c = cv[sl * TILE + r];
+                        pw[u] = e + u < ns ? (GEN ? pow_pos(c, ex) : c) : 0.f;
+                        // 128-byte swizzled V block in ring slot vslot[j / BLK]: 16-byte chunk q of
+                        // row `row` sits at chunk position q ^ (row & 7)
+                        const uint32_t row = (uint32_t)j & (BLK - 1);
+                        const uint8_t* base = smem_b + vslot[j / BLK] * BLK_BYTES + row * 128u;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            x[u][q] = *reinterpret_cast<const uint4*>(base + ((((uint32_t)(4 * h + q)) ^ (row & 7u)) << 4));
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) fma_bf16x8(acc[q], pw[u], x[u][q]);
                 }
             } else {
                 // V rows from L2, two support entries per step (eight 16-byte loads in flight; a missing
