@@ -109,7 +109,7 @@ struct DenseRows {
 // GEN: general alpha, weights w = b^em1 (em1 = 1/am1 - 1) and p = w b; the buckets then hold p
 // instead of b.
 // qmem: memory row of query row `row` in Q, dO and dQ (layout); bucket entries name it by qmem.
-// PLAIN (layout 0, one key/value head per query head): qmem is row itself and is not used.
+// PLAIN (layout 0): qmem is row itself and is not used.
 template <bool GEN, bool PLAIN, class Rows>
 __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
                                            const SavedBwdWs& ws, long long row, size_t qmem_, int cnt, int bhk,
@@ -207,11 +207,15 @@ __device__ __forceinline__ void rows_group(const AttnArgs& a, const BwdIO& io, c
 // One key per group of eight lanes: dK_j = scale sum dS Q_i and dV_j = sum p dO_i over key j's bucket,
 // lane sd of the group loading entry e0 + sd and the group sharing it by shuffles; two entries (two
 // 16-byte pieces each per lane) in flight.  valid = false: no key (the group still takes part).
-// key: logical key row (bhk * L + j); kmem: its memory row in K, V, dK and dV (layout; PLAIN: key).
-template <bool GEN, bool PLAIN, class Rows>
+// key: logical key row (bhk * L + j); kmem: its memory row in K, V, dK and dV (layout; PLAIN, i.e.
+// layout 0: key).
+// SPLIT groups of eight lanes share one key (grouped-query heads make its bucket SPLIT-fold longer):
+// group `sub` takes every SPLIT-th run of eight entries, and the partial sums are added across the
+// groups (lane groups 8q .. 8q + 7 with q = key slot * SPLIT + sub) before group 0 writes.
+template <bool GEN, bool PLAIN, int SPLIT, class Rows>
 __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv,
                                            const SavedBwdWs& ws, long long key, size_t kmem_, bool valid, int bhk,
-                                           const Rows& Qr, const Rows& Gr, int sd, int g0) {
+                                           const Rows& Qr, const Rows& Gr, int sd, int g0, int sub) {
     const size_t kmem = PLAIN ? (size_t)key : kmem_;
     const int L = a.L;
     const size_t cap = (size_t)(a.H / a.Hkv) * L * SAVE_CAP;  // bucket entries of one KV head
@@ -221,7 +225,10 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
     float ak[8], av[8];
 #pragma unroll
     for (int d = 0; d < 8; ++d) ak[d] = av[d] = 0.f;
-    for (int e0 = 0; e0 < maxn; e0 += 8) {
+    // every group runs the same number of steps (the shuffles below take all 32 lanes); group sub
+    // reads entries e0 + 8 sub .. e0 + 8 sub + 7 of each step
+    for (int e00 = 0; e00 < maxn; e00 += 8 * SPLIT) {
+        const int e0 = e00 + 8 * sub;
         const bool mine = e0 + sd < n;
         const uint32_t ei = mine ? ws.bucket_i[b0 + e0 + sd] : 0u;
         const float esp = mine ? ws.bucket_sp[b0 + e0 + sd] : 0.f;
@@ -255,7 +262,15 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
             }
         }
     }
-    if (valid) {
+#pragma unroll
+    for (int o = 8; o < 8 * SPLIT; o <<= 1) {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+            ak[d] += __shfl_xor_sync(0xffffffffu, ak[d], o);
+            av[d] += __shfl_xor_sync(0xffffffffu, av[d], o);
+        }
+    }
+    if (valid && sub == 0) {
         float4* dk = reinterpret_cast<float4*>(io.dK + kmem * HEAD_DIM + 8 * sd);
         float4* dv4 = reinterpret_cast<float4*>(io.dV + kmem * HEAD_DIM + 8 * sd);
         dk[0] = make_float4(a.scale * ak[0], a.scale * ak[1], a.scale * ak[2], a.scale * ak[3]);
@@ -265,8 +280,8 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
     }
 }
 
-// Four query rows per warp (eight lanes each), rows of K and V gathered from L2.  PLAIN: layout 0
-// with one key/value head per query head, where memory rows are the logical ones (no head maps).
+// Four query rows per warp (eight lanes each), rows of K and V gathered from L2.  PLAIN: layout 0,
+// where memory rows are the logical row ids and rows of one head are consecutive.
 template <bool GEN, bool PLAIN>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
@@ -283,8 +298,6 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
         const int cnt = row < R ? sv.row_cnt[row] : -1;
         const int bh = row < R ? (int)(row / L) : 0;
         if (PLAIN) {
-            // (bhk equals bh here; taking it through kv_head_of measured 5% faster at L = 4096 --
-            // instruction scheduling, not work)
             const int bhk = kv_head_of(bh, a.H, a.Hkv);
             const size_t head = (size_t)bhk * L * HEAD_DIM;
             const DenseRows Vr{reinterpret_cast<const __nv_bfloat16*>(a.V) + head};
@@ -304,19 +317,23 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnAr
     }
 }
 
-// Four keys per warp (eight lanes each), rows of Q and dO gathered from L2.  PLAIN as for the rows.
-template <bool GEN, bool PLAIN>
+// 4 / SPLIT keys per warp (8 SPLIT lanes each), rows of Q and dO gathered from L2.  PLAIN as for
+// the rows.
+template <bool GEN, bool PLAIN, int SPLIT>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
+    static_assert(SPLIT == 1 || SPLIT == 2 || SPLIT == 4, "lane groups per key");
+    constexpr int KPW = RPW / SPLIT;  // keys per warp
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = lane >> 3, sd = lane & 7, g0 = lane & ~7;
+    const int kq = q / SPLIT, sub = q % SPLIT;
     const int L = a.L;
     const long long Rk = (long long)a.B * a.Hkv * L;  // keys
     // bucket entries name their query row by its memory row, so Q and dO are read from the base
     const DenseRows Qr{reinterpret_cast<const __nv_bfloat16*>(a.Q)};
     const DenseRows Gr{reinterpret_cast<const __nv_bfloat16*>(io.dO)};
-    for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * RPW < Rk; grp += (long long)gridDim.x * ROW_WARPS) {
-        const long long key = grp * RPW + q;
+    for (long long grp = (long long)blockIdx.x * ROW_WARPS + warp; grp * KPW < Rk; grp += (long long)gridDim.x * ROW_WARPS) {
+        const long long key = grp * KPW + kq;
         const bool kv = key < Rk;
         const int bhk = kv ? (int)(key / L) : 0;
         size_t kmem = 0;
@@ -325,7 +342,7 @@ __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnAr
             const HeadRef hkv{a.layout, b, bhk - b * a.Hkv, a.Hkv, L};
             kmem = hkv.row((int)(key - (long long)bhk * L));
         }
-        keys_group<GEN, PLAIN>(a, io, sv, ws, key, kmem, kv, bhk, Qr, Gr, sd, g0);
+        keys_group<GEN, PLAIN, SPLIT>(a, io, sv, ws, key, kmem, kv, bhk, Qr, Gr, sd, g0, sub);
     }
 }
 
@@ -498,7 +515,7 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>((R + ROW_WARPS - 1) / ROW_WARPS, (long long)sms * 8));
     const bool gen = generic_alpha(a);
-    const bool plain = a.layout == 0 && a.Hkv == a.H;
+    const bool plain = a.layout == 0;  // memory rows = logical row ids
     if (gen) {
         if (plain) saved_rows_kernel<true, true><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
         else saved_rows_kernel<true, false><<<grid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
@@ -509,14 +526,18 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long Rk = (long long)a.B * a.Hkv * a.L;
-    const unsigned kgrid = (unsigned)std::max<long long>(1, std::min<long long>((Rk + ROW_WARPS * RPW - 1) / (ROW_WARPS * RPW), (long long)sms * 8));
-    if (gen) {
-        if (plain) saved_keys_kernel<true, true><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
-        else saved_keys_kernel<true, false><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
-    } else {
-        if (plain) saved_keys_kernel<false, true><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
-        else saved_keys_kernel<false, false><<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
-    }
+    // lane groups per key: grouped-query buckets hold H / H_kv query heads' entries
+    const int rep_heads = a.H / a.Hkv, split = rep_heads >= 4 ? 4 : rep_heads >= 2 ? 2 : 1;
+    const long long kwarps = (Rk * split + RPW - 1) / RPW;
+    const unsigned kgrid = (unsigned)std::max<long long>(1, std::min<long long>((kwarps + ROW_WARPS - 1) / ROW_WARPS, (long long)sms * 8));
+    // one instantiation per (generic alpha, layout 0, lane groups per key)
+    using KeysFn = void (*)(const AttnArgs, const BwdIO, const SavedSupport, const SavedBwdWs);
+    static const KeysFn keys_fns[2][2][3] = {
+        {{saved_keys_kernel<false, false, 1>, saved_keys_kernel<false, false, 2>, saved_keys_kernel<false, false, 4>},
+         {saved_keys_kernel<false, true, 1>, saved_keys_kernel<false, true, 2>, saved_keys_kernel<false, true, 4>}},
+        {{saved_keys_kernel<true, false, 1>, saved_keys_kernel<true, false, 2>, saved_keys_kernel<true, false, 4>},
+         {saved_keys_kernel<true, true, 1>, saved_keys_kernel<true, true, 2>, saved_keys_kernel<true, true, 4>}}};
+    keys_fns[gen][plain][split == 4 ? 2 : split - 1]<<<kgrid, ROW_WARPS * 32, 0, stream>>>(a, io, sv, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int smem = 2 * a.L * (int)sizeof(float);
