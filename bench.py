@@ -18,9 +18,10 @@ value = total work of all ranks / max step time over ranks ("scaling": "weak").
 
 --impl reference times the fp64 CPU oracle on the host cores (bounded sample per step).
 
-Variants (side measurements, not the headline line): --alpha A runs alpha-entmax for A in (1, 2]
-and --hkv N grouped-query attention with N key/value heads, both through entmax_attn_fwd_ex /
-entmax_attn_bwd_saved_ex; the dense-equivalent FLOP count is unchanged (it counts query heads).
+Variants (side measurements, not the headline line): --alpha A runs alpha-entmax for A in (1, 2],
+--hkv N grouped-query attention with N key/value heads and --blhd keeps Q, K, V, dO (and the
+outputs) in [B, L, H, 64] memory, all through entmax_attn_fwd_ex / entmax_attn_bwd_saved_ex; the
+dense-equivalent FLOP count is unchanged (it counts query heads).
 """
 from __future__ import annotations
 
@@ -204,20 +205,22 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
 
     w = bench_workload(args)
     alpha = args.alpha
-    variant = alpha != 1.5 or w.kv_heads != w.H  # the _ex entry points
+    variant = alpha != 1.5 or w.kv_heads != w.H or args.blhd  # the _ex entry points
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     inp = make_inputs(w)
     pairs = allowed_pairs(w, inp["key_mask"])
     flops = dense_equiv_flops(w, pairs)
-    Q, K, V, dO = (inp[k].to(dev) for k in ("Q", "K", "V", "dO"))
+    # --blhd: the same values held in [B, L, H, 64] memory, passed as transpose(1, 2) views
+    lay = (lambda x: x.transpose(1, 2).contiguous().transpose(1, 2)) if args.blhd else (lambda x: x)
+    Q, K, V, dO = (lay(inp[k].to(dev)) for k in ("Q", "K", "V", "dO"))
     km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
     B, H, L, D = w.B, w.H, w.L, w.D
     Hkv = w.kv_heads
-    O = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
+    O = lay(torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev))
     tau = torch.empty((B, H, L), dtype=torch.float32, device=dev)
-    dQ = torch.empty((B, H, L, D), dtype=torch.float32, device=dev)
-    dK, dV = (torch.empty((B, Hkv, L, D), dtype=torch.float32, device=dev) for _ in range(2))
+    dQ = lay(torch.empty((B, H, L, D), dtype=torch.float32, device=dev))
+    dK, dV = (lay(torch.empty((B, Hkv, L, D), dtype=torch.float32, device=dev)) for _ in range(2))
     saved = torch.empty((E.entmax_attn_saved_bytes(B, H, L, D),), dtype=torch.uint8, device=dev)
     ws = torch.empty((E.entmax_attn_bwd_saved_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
@@ -283,12 +286,20 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     host_in = {k: inp[k].pin_memory() for k in ("Q", "K", "V", "dO")}
+    if args.blhd:  # host tensors in [B, L, H, 64] memory too
+        host_in = {k: v.transpose(1, 2).contiguous().pin_memory().transpose(1, 2) for k, v in host_in.items()}
     host_km = None if inp["key_mask"] is None else inp["key_mask"].pin_memory()
-    host_out = {"O": torch.empty(O.shape, dtype=O.dtype).pin_memory(),
+    def host_empty(shape, dtype):  # pinned, in the device tensors' memory layout
+        if args.blhd:
+            b_, h_, l_, d_ = shape
+            return torch.empty((b_, l_, h_, d_), dtype=dtype).pin_memory().transpose(1, 2)
+        return torch.empty(shape, dtype=dtype).pin_memory()
+
+    host_out = {"O": host_empty(O.shape, O.dtype),
                 "tau": torch.empty(tau.shape, dtype=tau.dtype).pin_memory()}
     if w.backward:
         for name in ("dQ", "dK", "dV"):
-            host_out[name] = torch.empty((B, H if name == "dQ" else Hkv, L, D), dtype=torch.float32).pin_memory()
+            host_out[name] = host_empty((B, H if name == "dQ" else Hkv, L, D), torch.float32)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + (
         0 if host_km is None else host_km.numel())
     if not w.backward:
@@ -395,7 +406,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "l2": "flushed between timed steps (256 MiB write, outside the step events)",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
-        "variant": {"alpha": alpha, "H_kv": Hkv} if variant else None,
+        "variant": {"alpha": alpha, "H_kv": Hkv, "layout": "BLHD" if args.blhd else "BHLD"} if variant else None,
         "fwd_ms": round(fwd_mean, 4),
         "bwd_ms": round(bwd_mean, 4),
         "step_ms_median": round(statistics.median(step_ms), 4),
@@ -502,6 +513,7 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--alpha", type=float, default=1.5, help="alpha-entmax variant, alpha in (1, 2]")
     ap.add_argument("--hkv", type=int, default=0, help="grouped-query variant: key/value heads")
+    ap.add_argument("--blhd", action="store_true", help="variant: tensors in [B, L, H, 64] memory")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
