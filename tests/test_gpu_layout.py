@@ -103,3 +103,43 @@ def test_blhd_autograd_views():
     assert torch.equal(O.float(), O2.float())
     for a, b in zip(x, y):
         assert torch.allclose(a.grad.transpose(1, 2).float(), b.grad.float(), atol=1e-2, rtol=1e-2)
+
+
+def test_variants_at_the_size_limits():
+    """L = 16384 (the longest sequence) with sparsemax, two query heads on one key/value head and
+    [B, L, H, 64] memory, causal window 32: sampled rows forward, the whole key/value head backward."""
+    B, H, Hkv, L = 1, 2, 1, 16384
+    w = Workload(0, "limits", B, H, L, 64, 1 / 8, True, 32, H_kv=Hkv)
+    inp = make_inputs(w, seed=54)
+    d = inputs_f64(inp, False)
+    Q, K, V, dO = (_blhd(inp[k].to(DEV)) for k in ("Q", "K", "V", "dO"))
+    O, tau, g = _run(Q, K, V, dO, None, w, 2.0)
+    rng = np.random.default_rng(54)
+    ids = np.unique(np.concatenate([rng.integers(0, B * H * L, size=96), [0, 31, 32, L - 1, L, 2 * L - 1]]))
+    O_ref, tau_ref = orc.attn_fwd_rows_gqa(d["Q"], d["K"], d["V"], ids, None, True, 32, 1 / 8, alpha=2.0)
+    assert np.max(np.abs(to64(O).reshape(-1, 64)[ids] - O_ref)) <= O_TOL
+    assert np.max(np.abs(to64(tau).reshape(-1)[ids] - tau_ref)) <= 1e-3
+    refs = orc.attn_bwd_gqa(d["Q"], d["K"], d["V"], d["dO"], None, True, 32, 1 / 8, alpha=2.0)
+    for x, r in zip(g, refs):
+        assert np.max(np.abs(to64(x) - r)) <= GRAD_TOL
+
+
+def test_blhd_at_the_head_limit():
+    """B * H = 65535 heads of two positions in [B, L, H, 64] memory (H = 3), key padding down to one
+    key: the tensor maps' third dimension is B * L = 43690 positions."""
+    B, H, L = 21845, 3, 2
+    w = Workload(0, "head-limit", B, H, L, 64, 1 / 8, len_range=(1, 2))
+    inp = make_inputs(w, seed=55)
+    d = inputs_f64(inp, False)
+    km_np = inp["key_mask"].numpy()
+    Q, K, V, dO = (_blhd(inp[k].to(DEV)) for k in ("Q", "K", "V", "dO"))
+    km = inp["key_mask"].to(DEV)
+    O, tau, g = _run(Q, K, V, dO, km, w, 1.5)
+    ids = np.array(sorted({0, 1, 2, 5, B * H * L - 1, B * H * L - 2} | set(range(70000, 70030))), dtype=np.int64)
+    O_ref, tau_ref = orc.attn_fwd_rows(d["Q"], d["K"], d["V"], ids, km_np, False, 0, 1 / 8)
+    assert np.max(np.abs(to64(O).reshape(-1, 64)[ids] - O_ref)) <= O_TOL
+    assert np.max(np.abs(to64(tau).reshape(-1)[ids] - tau_ref)) <= 1e-3
+    heads = [0, 1, 40000, B * H - 1]
+    rQ, rK, rV = orc.attn_bwd_heads(d["Q"], d["K"], d["V"], d["dO"], heads, km_np, False, 0, 1 / 8)
+    for x, r in zip(g, (rQ, rK, rV)):
+        assert np.max(np.abs(to64(x).reshape(-1, L, 64)[heads] - r)) <= GRAD_TOL
