@@ -67,3 +67,27 @@ def test_single_process_helpers_need_no_process_group():
     bench.dist_barrier(1)
     assert bench.dist_max(3.5, 1, torch.device("cpu")) == 3.5
     assert bench.aggregate_value(2e12, 1, 1000.0) == pytest.approx(2.0)
+
+
+def test_allowed_pairs_by_brute_force():
+    """bench.py's dense-equivalent FLOP count rests on the number of (query, key) pairs the masks
+    allow: checked against a direct count over every pair."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    from entmax_tcgen05_tma_b200.workloads import Workload
+
+    for causal, window, lens in ((False, 0, None), (False, 0, (3, 17)), (True, 0, None), (True, 5, (4, 17))):
+        w = Workload(0, "pairs", 3, 2, 17, 64, 0.125, causal, window, lens)
+        km = None
+        if lens is not None:
+            km = torch.zeros(3, 17, dtype=torch.uint8)
+            for b, n in enumerate((lens[0], 9, lens[1])):
+                km[b, :n] = 1
+        want = 0
+        for b in range(3):
+            for i in range(17):
+                for j in range(17):
+                    ok = (km is None or km[b, j] == 1) and (not causal or j <= i) and (window == 0 or j >= i - window + 1)
+                    want += int(ok)
+        assert bench.allowed_pairs(w, km) == want * 2
+        assert bench.dense_equiv_flops(w, want * 2) == 14.0 * 64 * want * 2
