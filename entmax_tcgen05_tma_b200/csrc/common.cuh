@@ -279,21 +279,6 @@ struct Pipe {
         return ctl->tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((n % NBUF) * BLK + c * 32);
     }
 
-    // Reads the 32-column chunks of score block n one at a time (for kernels with enough epilogue
-    // warps per SM sub-partition to hide the TMEM load latency) and calls f(v, c) for chunk c.  The
-    // buffer goes back to the MMA warp once its last chunk is in registers.
-    template <class F>
-    static __device__ __forceinline__ void for_each_chunk_single(Ctl* ctl, int n, F&& f) {
-#pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
-            float v[32];
-            tmem_ld32(taddr(ctl, n, c), v);
-            tmem_wait_ld(v);
-            if (c == CHUNKS - 1) release_scores(ctl, n);
-            f(v, c);
-        }
-    }
-
     // Reads the 32-column chunks of score block n (the next chunk's load in flight while f runs)
     // and calls f(v, c) for chunk c.  With kRelease the buffer goes back to the MMA warp once its
     // last chunk is in registers; without, it stays readable for a later pass.
@@ -397,21 +382,6 @@ __device__ __forceinline__ float staged(const float* stage, int slot, int k) {
     return stage[slot * 32 + ((((k >> 2) ^ (slot & 7))) << 2) + (k & 3)];
 }
 
-// Half-chunk variants (16 values: chunk values [16 half, 16 half + 16)).
-__device__ __forceinline__ void stage_half(float* stage, int slot, const float (&v)[32], int half) {
-    float* row = stage + slot * 16;
-    const int sw = slot & 3;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const int b = 16 * half + 4 * c;
-        *reinterpret_cast<float4*>(row + ((c ^ sw) << 2)) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
-    }
-}
-
-__device__ __forceinline__ float staged_half(const float* stage, int slot, int k16) {
-    return stage[slot * 16 + ((((k16 >> 2) ^ (slot & 3))) << 2) + (k16 & 3)];
-}
-
 // b^e for b > 0 (0 for b <= 0), as 2^(e log2 b) with the hardware base-2 approximations
 // lg2.approx and ex2.approx (close to fp32 precision; the result's relative error grows with
 // |e log2 b|).
@@ -425,31 +395,10 @@ __device__ __forceinline__ float pow_pos(float b, float e) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// acc += sum over list slots e in [e0, e1) of w[e] * X[j[e]][2 lane .. 2 lane + 1], where the
-// slot arrays are [slot][TILE] with column `col`.  Loads go out eight rows at a time so a warp
-// keeps eight independent global reads in flight.
-__device__ __forceinline__ void gather_accumulate(const __nv_bfloat16* __restrict__ X, const uint16_t* cj,
-                                                  const float* cw, int col, int e0, int e1, int lane, float& acc0,
-                                                  float& acc1) {
-    for (int e = e0; e < e1; e += 8) {
-        uint32_t x[8];
-        float w[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const bool ok = e + u < e1;
-            const int j = ok ? (int)cj[(e + u) * TILE + col] : 0;
-            w[u] = ok ? cw[(e + u) * TILE + col] : 0.f;
-            x[u] = ok ? __ldg(reinterpret_cast<const uint32_t*>(X + (size_t)j * HEAD_DIM) + lane) : 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            acc0 = fmaf(w[u], bf16lo(x[u]), acc0);
-            acc1 = fmaf(w[u], bf16hi(x[u]), acc1);
-        }
-    }
-}
-
-// Two lists at once (columns ca, cb), so a warp keeps sixteen gathered rows in flight.
+// a += sum over list slots e in [ea0, ea1) of w[e] * X[j[e]][2 lane .. 2 lane + 1] for the list in
+// column ca of the [slot][TILE] arrays cj (key index) and cw (weight), and b likewise for column cb;
+// the two lists go together, eight slots each per step, so a warp keeps sixteen gathered rows in
+// flight.
 __device__ __forceinline__ void gather_accumulate2(const __nv_bfloat16* __restrict__ X, const uint16_t* cj,
                                                    const float* cw, int ca, int ea0, int ea1, int cb, int eb0,
                                                    int eb1, int lane, float& a0, float& a1, float& b0, float& b1) {
