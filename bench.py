@@ -225,10 +225,14 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     ws = torch.empty((E.entmax_attn_bwd_saved_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 1 + (4 if w.backward else 0)
+    recompute = args.bwd == "recompute"  # entmax_attn_fwd + entmax_attn_bwd (scores recomputed)
+    rws = torch.empty((max(E.entmax_attn_bwd_workspace_size(B, H, L, D), 1),), dtype=torch.uint8, device=dev)
+    launches_per_step = 1 + ((2 if recompute else 4) if w.backward else 0)
 
     def fwd_call():
-        if variant:
+        if recompute:
+            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+        elif variant:
             E.entmax_attn_fwd_ex(Q, K, V, km, w.causal, w.window, w.scale, alpha=alpha, save=w.backward, O=O, tau=tau,
                                  saved=saved if w.backward else None)
         elif w.backward:
@@ -237,7 +241,9 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
 
     def bwd_call():
-        if variant:
+        if recompute:
+            E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV, workspace=rws)
+        elif variant:
             E.entmax_attn_bwd_saved_ex(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale, alpha=alpha, dQ=dQ,
                                        dK=dK, dV=dV, workspace=ws)
         else:
@@ -327,7 +333,10 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         Vd = hin["V"].to(dev, non_blocking=True)
         kmd = None if host_km is None else host_km[b0:b1].to(dev, non_blocking=True)
         sv_buf, ws_buf = e2e_saved[k], e2e_ws[k]
-        if variant:
+        if recompute:
+            Oo, to = E.entmax_attn_fwd(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale)
+            sv = None
+        elif variant:
             r = E.entmax_attn_fwd_ex(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale, alpha=alpha, save=w.backward,
                                      saved=sv_buf if w.backward else None)
             Oo, to, sv = r if w.backward else (r[0], r[1], None)
@@ -339,7 +348,9 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         host_out["tau"][b0:b1].copy_(to, non_blocking=True)
         if w.backward:
             dOd = hin["dO"].to(dev, non_blocking=True)
-            if variant:
+            if recompute:
+                g = E.entmax_attn_bwd(Qd, Kd, Vd, to, dOd, kmd, w.causal, w.window, w.scale)
+            elif variant:
                 g = E.entmax_attn_bwd_saved_ex(Qd, Kd, Vd, to, sv, dOd, kmd, w.causal, w.window, w.scale, alpha=alpha,
                                                workspace=ws_buf)
             else:
@@ -388,7 +399,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     # saved support: a count and a (u16 key, fp32 sqrt p) pair per entry
     kv_rows = B * Hkv * L
     fwd_alg_bytes = rows * D * 2 + 2.0 * kv_rows * D * 2 + rows * D * 2 + rows * 4
-    if w.backward:
+    if w.backward and not recompute:
         fwd_alg_bytes += rows * 4 + supp_pairs * 6
     fwd_mean = statistics.mean(fwd_ms)
     bwd_mean = statistics.mean(bwd_ms) if w.backward else 0.0
@@ -435,6 +446,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
         "variant": {"alpha": alpha, "H_kv": Hkv, "layout": "BLHD" if args.blhd else "BHLD"} if variant else None,
+        "backward": "entmax_attn_bwd (scores recomputed)" if recompute else "entmax_attn_bwd_saved (saved supports)",
         "fwd_ms": round(fwd_mean, 4),
         "bwd_ms": round(bwd_mean, 4),
         "step_ms_median": round(statistics.median(step_ms), 4),
@@ -543,11 +555,15 @@ def main() -> int:
     ap.add_argument("--alpha", type=float, default=1.5, help="alpha-entmax variant, alpha in (1, 2]")
     ap.add_argument("--hkv", type=int, default=0, help="grouped-query variant: key/value heads")
     ap.add_argument("--blhd", action="store_true", help="variant: tensors in [B, L, H, 64] memory")
+    ap.add_argument("--bwd", default="saved", choices=["saved", "recompute"],
+                    help="backward path: from the forward's saved supports, or entmax_attn_bwd (scores recomputed)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if not 1.0 < args.alpha <= 2.0:
         ap.error("--alpha must lie in (1, 2]")
+    if args.bwd == "recompute" and (args.alpha != 1.5 or args.hkv or args.blhd):
+        ap.error("--bwd recompute takes the plain path only (alpha 1.5, H_kv = H, [B, H, L, 64])")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
