@@ -185,8 +185,9 @@ ENTMAX_API int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const voi
  * and the backward uses the Jacobian w_i (delta_ij - w_j / sum_k w_k), w = p^(2 - alpha).
  *   alpha      in (1, 2]; alpha = 1 (softmax, dense supports) returns ENTMAX_ERR_UNSUPPORTED, any
  *              other value (or NaN) ENTMAX_ERR_ARG.  alpha = 1.5 runs exactly the kernels of the
- *              entry points above; other values run variants whose tau solve ends with Newton's
- *              method on the settled support instead of the closed form.  Supports grow as alpha
+ *              entry points above; other values run variants whose tau solve is Newton's method
+ *              from the bracket's lower end (bisection as the backstop) instead of bisection with a
+ *              closed-form finish.  Supports grow as alpha
  *              approaches 1: rows with more candidates than the kernels list are recomputed on CUDA
  *              cores, so small alpha - 1 is correct but slow.
  *   H_kv       key/value heads as in the _gqa calls (H_kv = H: plain multi-head attention).
