@@ -69,6 +69,21 @@ def dense_equiv_flops(w: Workload, pairs: int) -> float:
     return (14.0 if w.backward else 4.0) * w.D * pairs
 
 
+def min_hbm_bytes(w: Workload, key_mask) -> float:
+    """Bytes a step must move at least, each tensor once: the forward reads Q and the K, V rows of
+    valid keys and writes O (bf16) and tau; the backward reads Q, K, V (valid rows), dO and tau and
+    writes dQ, dK, dV (fp32)."""
+    D, in_b = w.D, (4 if w.fp32_inputs else 2)
+    rows = w.B * w.H * w.L
+    valid_keys = w.B * w.L if key_mask is None else int(key_mask.to(torch.int64).sum())
+    kv_rows = valid_keys * w.kv_heads
+    fwd = rows * D * in_b + 2 * kv_rows * D * in_b + rows * D * 2 + rows * 4
+    if not w.backward:
+        return float(fwd)
+    bwd = 2 * rows * D * in_b + 2 * kv_rows * D * in_b + rows * 4 + rows * D * 4 + 2 * w.B * w.kv_heads * w.L * D * 4
+    return float(fwd + bwd)
+
+
 def workload_desc(w: Workload) -> str:
     s = "%s: B=%d H=%d L=%d d=%d scale=%g" % (w.name, w.B, w.H, w.L, w.D, w.scale)
     if w.len_range:
@@ -142,9 +157,19 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: int = 64, alpha: float = 1.5) -> dict:
-    """Time the fp64 oracle (as it stands) on whole heads of the workload until ~budget_s."""
+def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: int = 64, alpha: float = 1.5,
+                    threads: int = 0) -> dict:
+    """Time the fp64 oracle (as it stands) on whole heads of the workload until ~budget_s; threads > 0
+    limits its OpenMP threads for the call."""
     from oracle import oracle as orc
+
+    if threads > 0:
+        before = orc.num_threads()
+        orc.set_num_threads(threads)
+        try:
+            return oracle_baseline(w, inp, budget_s, max_heads, alpha)
+        finally:
+            orc.set_num_threads(before)
 
     f64 = {k: inp[k].to(torch.float64).numpy() for k in ("Q", "K", "V", "dO")}
     if w.kv_heads != w.H:  # grouped heads: the oracle's repeat of K and V (outside the timed loop)
@@ -423,6 +448,14 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         if t.get("kernel") == "entmax_fwd_kernel" and t.get("source_hash") == source_hash():
             roof["traffic"] = t["bytes_per_launch"]
 
+    # the whole step against its roofline time: max(dense-equivalent FLOPs / bf16 peak, minimum HBM
+    # bytes / HBM peak), as a fraction of the measured step time
+    step_bytes = min_hbm_bytes(w, km)
+    t_flop, t_byte = flops / (peaks["bf16_tflops"] * 1e12), step_bytes / (peaks["hbm_gbs"] * 1e9)
+    step_roof = {"bound": "tensor" if t_flop >= t_byte else "hbm", "time_us": round(1e6 * max(t_flop, t_byte), 2),
+                 "frac": round(1e3 * max(t_flop, t_byte) / ms_per_step, 4), "min_hbm_bytes": step_bytes,
+                 "peaks": "bf16 %.1f TFLOP/s, HBM %.1f GB/s (%s)" % (peaks["bf16_tflops"], peaks["hbm_gbs"],
+                                                                  peaks["source"])}
     value = aggregate_value(flops, world, ms_per_step)
     out = {
         "metric": METRIC,
@@ -442,6 +475,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "workload_id": w.wid,
             "allowed_pairs": pairs,
             "dense_equiv_gflop_per_step": flops / 1e9,
+            "dense_equiv_gflop_full_L2": dense_equiv_flops(w, w.B * w.H * w.L * w.L) / 1e9,
             "l2": "flushed between timed steps (256 MiB write, outside the step events)",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
@@ -453,6 +487,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "wall_ms_per_step_incl_flush": round(wall * 1e3 / args.steps, 4),
         "sparsity": round(sparsity, 4),
         "roofline": roof,
+        "step_roofline": step_roof,
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -462,6 +497,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     if world == 1 and not args.no_cpu_baseline:
         cb = oracle_baseline(w, inp, budget_s=args.cpu_seconds, alpha=alpha)
         out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        cb1 = oracle_baseline(w, inp, budget_s=args.cpu_seconds / 3, max_heads=8, alpha=alpha, threads=1)
+        out["cpu_baseline_1thread"] = {k: cb1[k] for k in ("value", "unit", "cores", "kind", "sample")}
     return out
 
 

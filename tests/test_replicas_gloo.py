@@ -91,3 +91,19 @@ def test_allowed_pairs_by_brute_force():
                     want += int(ok)
         assert bench.allowed_pairs(w, km) == want * 2
         assert bench.dense_equiv_flops(w, want * 2) == 14.0 * 64 * want * 2
+
+
+def test_min_hbm_bytes_counts_each_tensor_once():
+    sys.path.insert(0, str(ROOT))
+    import bench
+    from entmax_tcgen05_tma_b200.workloads import Workload
+
+    w = Workload(0, "bytes", 2, 3, 10, 64, 0.125, len_range=(4, 10), H_kv=1)
+    km = torch.zeros(2, 10, dtype=torch.uint8)
+    km[0, :4] = 1
+    km[1, :7] = 1
+    rows, kv_rows = 2 * 3 * 10, (4 + 7) * 1
+    fwd = rows * 64 * 2 + 2 * kv_rows * 64 * 2 + rows * 64 * 2 + rows * 4
+    bwd = 2 * rows * 64 * 2 + 2 * kv_rows * 64 * 2 + rows * 4 + rows * 64 * 4 + 2 * 2 * 1 * 10 * 64 * 4
+    assert bench.min_hbm_bytes(w, km) == fwd + bwd
+    assert bench.min_hbm_bytes(w.with_shape(backward=False), km) == fwd
