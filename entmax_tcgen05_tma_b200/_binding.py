@@ -49,6 +49,9 @@ EXPORTED = (
 
 
 class EntmaxError(RuntimeError):
+    """A library call returned a negative status (``status``); the message names the call, the
+    status and, for ENTMAX_ERR_CUDA, the CUDA error code."""
+
     def __init__(self, status: int, what: str):
         self.status = status
         msg = "%s failed: %s (%d)" % (what, strerror(status), status)
@@ -121,10 +124,12 @@ lib = _LazyLibrary()
 
 
 def strerror(status: int) -> str:
+    """Static description of a status code."""
     return lib.entmax_attn_strerror(int(status)).decode()
 
 
 def version() -> int:
+    """Library version, major * 10000 + minor * 100 + patch."""
     return lib.entmax_attn_version()
 
 
@@ -252,6 +257,7 @@ def entmax_attn_fwd_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=No
 
 
 def entmax_attn_bwd_workspace_size(B: int, H: int, L: int, D: int = 64) -> int:
+    """Bytes of device workspace entmax_attn_bwd needs (one float per query row, rounded up)."""
     return int(lib.entmax_attn_bwd_workspace_size(B, H, L, D))
 
 
@@ -315,10 +321,12 @@ def entmax_attn_bwd_noalloc(Q, K, V, tau, dO, key_mask=None, causal=False, windo
 
 
 def entmax_attn_saved_bytes(B: int, H: int, L: int, D: int = 64) -> int:
+    """Bytes of the buffer the training forward saves the supports into (H: query heads)."""
     return int(lib.entmax_attn_saved_bytes(B, H, L, D))
 
 
 def entmax_attn_bwd_saved_workspace_size(B: int, H: int, L: int, D: int = 64) -> int:
+    """Bytes of device workspace the saved-support backward needs (H: query heads)."""
     return int(lib.entmax_attn_bwd_saved_workspace_size(B, H, L, D))
 
 
@@ -458,10 +466,12 @@ def entmax_attn_device_status(stream=None) -> int:
 
 
 def entmax_attn_set_wait_timeout_ns(ns: int) -> None:
+    """Bound on each device-side wait for later launches, in nanoseconds (0: the default, 2 s)."""
     lib.entmax_attn_set_wait_timeout_ns(int(ns))
 
 
 def entmax_attn_last_cuda_error() -> int:
+    """cudaError_t value of the most recent failed CUDA call inside the library (0 if none)."""
     return int(lib.entmax_attn_last_cuda_error())
 
 
