@@ -219,7 +219,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
     if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
     if (!O || !tau) return ENTMAX_ERR_ARG;
-    if (!aligned(O, 8) || !aligned(tau, 4)) return ENTMAX_ERR_ARG;
+    if (!aligned(O, 16) || !aligned(tau, 4)) return ENTMAX_ERR_ARG;
     int* status = nullptr;
     rc = record(status_ptr(&status));
     if (rc) return rc;
@@ -329,7 +329,7 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     if (out_dtype != ENTMAX_BF16 && out_dtype != ENTMAX_F32) return ENTMAX_ERR_ARG;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
     if (!O || !tau) return ENTMAX_ERR_ARG;
-    if (!aligned(O, 8) || !aligned(tau, 4)) return ENTMAX_ERR_ARG;
+    if (!aligned(O, 16) || !aligned(tau, 4)) return ENTMAX_ERR_ARG;
     const long long R = (long long)B * H * L;
     if (!saved || saved_bytes < saved_support_bytes(R)) return ENTMAX_ERR_WORKSPACE;
     if (!aligned(saved, 256)) return ENTMAX_ERR_ARG;
@@ -370,7 +370,7 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     if (rc) return rc;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
     if (!tau || !dO || !dQ || !dK || !dV) return ENTMAX_ERR_ARG;
-    if (!aligned(dO, 16) || !aligned(dQ, 8) || !aligned(dK, 8) || !aligned(dV, 8) || !aligned(tau, 4))
+    if (!aligned(dO, 16) || !aligned(dQ, 16) || !aligned(dK, 16) || !aligned(dV, 16) || !aligned(tau, 4))
         return ENTMAX_ERR_ARG;
     const long long R = (long long)B * H * L;
     if (!saved || saved_bytes < saved_support_bytes(R)) return ENTMAX_ERR_WORKSPACE;

@@ -78,7 +78,7 @@ typedef enum {
  *   key_mask  [B,L] uint8, 1 = valid key; NULL = all valid.
  *   causal    0/1.   window: keys per row including the query (0 = off; > 0 needs causal).
  *   scale     > 0, multiplies Q.K (1/sqrt(D) on the pages' encoders).
- *   O         [B,H,L,D] in `out_dtype` (bf16 or fp32), 8-byte aligned.
+ *   O         [B,H,L,D] in `out_dtype` (bf16 or fp32), 16-byte aligned (16-byte stores).
  *   tau       [B,H,L] fp32, the threshold in score units: A_ij = max(0,(S_ij - tau_i)/2)^2.
  *             Needed by the backward pass.
  * Returns ENTMAX_OK once the work is queued on `stream`.  B, H or L equal to 0 is a no-op.
@@ -126,6 +126,8 @@ ENTMAX_API int entmax_attn_bwd(const void* Q, const void* K, const void* V, int 
  *              entmax_attn_fwd_train and read by entmax_attn_bwd_saved for the same Q, K, masks and
  *              scale; owned by the caller.
  *   workspace  device buffer of entmax_attn_bwd_saved_workspace_size(B,H,L,D) bytes, 256-byte aligned.
+ *   O (training forward) and dQ, dK, dV (this backward): 16-byte aligned (16-byte stores); the
+ *   other arguments as in entmax_attn_fwd / entmax_attn_bwd.
  * dK and dV are summed in an order that depends on scheduling (last-bit differences between runs);
  * dQ, O and tau are deterministic.
  */

@@ -86,6 +86,7 @@ def _bwd(**kw):
     (dict(tau=None), E.ENTMAX_ERR_ARG),
     (dict(K=P + 8), E.ENTMAX_ERR_ARG),
     (dict(O=P + 4), E.ENTMAX_ERR_ARG),
+    (dict(O=P + 8), E.ENTMAX_ERR_ARG),  # 16-byte stores
     (dict(B=-1), E.ENTMAX_ERR_ARG),
     (dict(B=0), E.ENTMAX_OK),
     (dict(L=0, Q=None, K=None, V=None, O=None, tau=None), E.ENTMAX_OK),
@@ -143,6 +144,11 @@ def test_training_path_argument_checks():
     nb = list(bargs)
     nb[16] = P + 4
     assert b(*nb) == E.ENTMAX_ERR_ARG
+    for k in (16, 17, 18):  # dQ, dK, dV take 16-byte stores
+        nb = list(bargs)
+        nb[k] = P + 8
+        assert b(*nb) == E.ENTMAX_ERR_ARG
+    assert f(*args[:12], P + 8, *args[13:]) == E.ENTMAX_ERR_ARG  # O of the training forward
 
 
 def _gqa_calls(H, Hkv, in_dtype=0, B=1, L=64, D=64):
