@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <atomic>
 #include <mutex>
 #include "../../include/entmax_attn.h"
 #include "common.cuh"
@@ -17,8 +18,12 @@ namespace {
 __device__ int g_device_status;  // ENTMAX_OK or the first device-side error since the last read
 
 constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;
-unsigned long long g_timeout_ns = DEFAULT_TIMEOUT_NS;
-int g_last_cuda_error = 0;
+// process-wide settings and the last error: calls may come from several host threads
+std::atomic<unsigned long long> g_timeout_ns{DEFAULT_TIMEOUT_NS};
+std::atomic<int> g_last_cuda_error{0};
+
+unsigned long long timeout_ns() { return g_timeout_ns.load(std::memory_order_relaxed); }
+
 constexpr int MAX_DEVICES = 64;
 int* g_status_ptr[MAX_DEVICES] = {};
 std::mutex g_mu;
@@ -27,7 +32,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int record(cudaError_t e) {
     if (e == cudaSuccess) return ENTMAX_OK;
-    g_last_cuda_error = (int)e;
+    g_last_cuda_error.store((int)e, std::memory_order_relaxed);
     return ENTMAX_ERR_CUDA;
 }
 
@@ -110,14 +115,15 @@ cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, cudaStream
 }
 
 cudaError_t ensure_smem_attr(const void* func, int bytes, int slot) {
-    static bool done[8][MAX_DEVICES] = {};
+    static std::atomic<bool> done[8][MAX_DEVICES] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= MAX_DEVICES || slot < 0 || slot >= 8) return cudaErrorInvalidValue;
-    if (done[slot][dev]) return cudaSuccess;
+    if (done[slot][dev].load(std::memory_order_acquire)) return cudaSuccess;
+    // setting the attribute twice (two threads racing here) is harmless
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) done[slot][dev] = true;
+    if (e == cudaSuccess) done[slot][dev].store(true, std::memory_order_release);
     return e;
 }
 
@@ -166,9 +172,11 @@ const char* entmax_attn_strerror(int status) {
     }
 }
 
-int entmax_attn_last_cuda_error(void) { return g_last_cuda_error; }
+int entmax_attn_last_cuda_error(void) { return g_last_cuda_error.load(std::memory_order_relaxed); }
 
-void entmax_attn_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns = ns ? ns : DEFAULT_TIMEOUT_NS; }
+void entmax_attn_set_wait_timeout_ns(unsigned long long ns) {
+    g_timeout_ns.store(ns ? ns : DEFAULT_TIMEOUT_NS, std::memory_order_relaxed);
+}
 
 int entmax_attn_device_status(cudaStream_t stream) {
     int* p = nullptr;
@@ -225,7 +233,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f, layout};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, alpha - 1.f, layout};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -279,7 +287,7 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f, 0};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), H, 0.5f, 0};
     BwdIO io{tau, dO, dQ, dK, dV, static_cast<float*>(workspace)};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -342,7 +350,7 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f, layout};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, alpha - 1.f, layout};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -380,7 +388,7 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(status_ptr(&status));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, Hkv, alpha - 1.f, layout};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, alpha - 1.f, layout};
     BwdIO io{tau, dO, dQ, dK, dV, nullptr};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -502,7 +510,7 @@ extern "C" int entmax_attn_bwd_noalloc(const void* Q, const void* K, const void*
     float* scratch = nullptr;
     rc = record(noalloc_scratch(&scratch));
     if (rc) return rc;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, g_timeout_ns, H, 0.5f, 0};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), H, 0.5f, 0};
     BwdIO io{tau, dO, dQ, dK, dV, scratch};
     return record(launch_bwd(a, io, stream));
 }
