@@ -22,9 +22,14 @@
  * key gets O_i = 0, tau_i = +inf and zero gradients.
  *
  * Layout: Q, K, V, dO, O, dQ, dK, dV are contiguous row-major [B, H, L, D] tensors (the _ex entry
- * points also take [B, L, H, D]: entmax_layout); tau is [B, H, L]; key_mask is [B, L] bytes.  D must be 64.  All pointers are DEVICE pointers owned
- * by the caller; the library keeps no reference after a call returns.  Every call is
- * asynchronous on `stream` (0 = the legacy default stream).
+ * points also take [B, L, H, D]: entmax_layout); tau is [B, H, L]; key_mask is [B, L] bytes.
+ * D must be 64.  All pointers are DEVICE pointers owned by the caller; the library keeps no
+ * reference after a call returns.  Every call is asynchronous on `stream` (0 = the legacy
+ * default stream) and works on the calling thread's current device.
+ *
+ * Host threads: any entry point may be called from several threads at once.  The wait bound
+ * (entmax_attn_set_wait_timeout_ns), the last CUDA error and each device's status word are
+ * shared by the whole process.
  *
  * Errors: arguments are checked on the host before any launch; a bad argument returns a
  * negative status and launches nothing.  Problems found on the device (a bounded wait that
