@@ -250,3 +250,25 @@ def test_binding_layout_detection():
         bnd._layout_of(torch.zeros(2, 3, 64, 5).transpose(2, 3))  # d not innermost
     y = bnd._empty((2, 3, 5, 64), torch.float32, "cpu", E.ENTMAX_LAYOUT_BLHD)
     assert y.shape == (2, 3, 5, 64) and y.transpose(1, 2).is_contiguous()
+
+
+def test_missing_library_fails_loudly():
+    """No CPU path stands behind the binding: without the built library every call raises."""
+    import subprocess
+    import sys
+
+    code = (
+        "from pathlib import Path\n"
+        "import entmax_tcgen05_tma_b200._binding as B\n"
+        "B.LIB_PATH = Path('/nonexistent/libentmax_attn.so')\n"
+        "for f in (B.version, lambda: B.strerror(0), lambda: B.entmax_attn_bwd_workspace_size(1, 1, 64)):\n"
+        "    try:\n"
+        "        f()\n"
+        "    except ImportError as e:\n"
+        "        assert 'not built' in str(e)\n"
+        "    else:\n"
+        "        raise SystemExit('call succeeded without the library')\n"
+        "print('raised')\n"
+    )
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT, timeout=300)
+    assert r.returncode == 0 and "raised" in r.stdout, r.stdout + r.stderr
