@@ -1,6 +1,6 @@
 """Shared helpers for the GPU-vs-oracle parity tests.
 
-Tolerances (fixed by the spec of the hot path; the same numbers appear in the design doc):
+Tolerances (fixed by the specification of the hot path):
   * O:      max |O_gpu - O_ref| <= 1e-2  (fp32 output); bf16 output adds its own rounding,
             half a bf16 ulp = 2^-9 |O_ref| relative.
   * tau:    |tau_gpu - tau_ref| <= 1e-3
