@@ -538,7 +538,7 @@ def run_reference(args) -> dict:
         "metric": METRIC,
         "value": round(value, 6),
         "unit": "TFLOP/s",
-        "n_gpus": 0,
+        "n_gpus": args.gpus,  # the launch's N; the oracle itself runs on host cores only
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(1e3 * dense_equiv_flops(w, pairs) / (value * 1e12), 3),
@@ -549,7 +549,7 @@ def run_reference(args) -> dict:
         "data": "synthetic (seeded i.i.d. N(0,1), bf16-rounded)",
         "config": {"workload": workload_desc(w), "workload_id": w.wid,
                    "note": "each step times the fp64 CPU oracle on a bounded sample of whole heads; "
-                           "ms_per_step extrapolates to the full workload"},
+                           "ms_per_step extrapolates to the full workload; no GPU is used"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
                          "sample": "%d steps, each %s" % (args.steps, per[-1]["sample"])},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
