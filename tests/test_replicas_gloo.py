@@ -107,3 +107,24 @@ def test_min_hbm_bytes_counts_each_tensor_once():
     bwd = 2 * rows * 64 * 2 + 2 * kv_rows * 64 * 2 + rows * 4 + rows * 64 * 4 + 2 * 2 * 1 * 10 * 64 * 4
     assert bench.min_hbm_bytes(w, km) == fwd + bwd
     assert bench.min_hbm_bytes(w.with_shape(backward=False), km) == fwd
+
+
+def test_reference_arm_under_torchrun_prints_one_line():
+    """`bench.py --impl reference` launched as two ranks: rank 0 alone times the oracle and prints
+    the one JSON line (with the launch's n_gpus), the other rank exits 0 without work."""
+    import json
+    import subprocess
+
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), str(ROOT / "bench.py"),
+           "--gpus", "2", "--impl", "reference", "--workload", "2", "--steps", "1", "--warmup", "3",
+           "--ref-step-seconds", "0.5"]
+    r = subprocess.run(cmd, capture_output=True, text=True, cwd=ROOT, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["n_gpus"] == 2 and out["steps"] == 1 and out["warmup"] == 3
+    assert out["value"] > 0 and out["e2e"]["value"] == out["value"]
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["cpu_baseline"]["kind"] == "oracle"
+    assert out["config"]["workload_id"] == 2
