@@ -143,3 +143,30 @@ def test_blhd_at_the_head_limit():
     rQ, rK, rV = orc.attn_bwd_heads(d["Q"], d["K"], d["V"], d["dO"], heads, km_np, False, 0, 1 / 8)
     for x, r in zip(g, (rQ, rK, rV)):
         assert np.max(np.abs(to64(x).reshape(-1, L, 64)[heads] - r)) <= GRAD_TOL
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25])
+def test_fully_masked_batch_in_every_variant(alpha):
+    """A batch whose keys are all padding, in [B, L, H, 64] memory with grouped heads: its rows have
+    no allowed key, so O = 0, tau = +inf and every gradient of that batch is 0; the other batch
+    against the oracle."""
+    B, H, Hkv, L = 2, 4, 2, 200
+    w = Workload(0, "masked", B, H, L, 64, 1 / 8, H_kv=Hkv)
+    inp = make_inputs(w, seed=56)
+    km_np = np.ones((B, L), dtype=np.uint8)
+    km_np[1] = 0
+    km_np[0, 150:] = 0
+    d = inputs_f64(inp, False)
+    Q, K, V, dO = (_blhd(inp[k].to(DEV)) for k in ("Q", "K", "V", "dO"))
+    km = torch.from_numpy(km_np).to(DEV)
+    O, tau, g = _run(Q, K, V, dO, km, w, alpha)
+    assert torch.all(O[1] == 0) and torch.all(torch.isinf(tau[1])) and torch.all(tau[1] > 0)
+    for x in g:
+        assert torch.all(x[1] == 0)
+    O_ref, tau_ref = orc.attn_fwd_gqa(d["Q"], d["K"], d["V"], km_np, False, 0, 1 / 8, alpha=alpha)
+    assert np.array_equal(np.isfinite(to64(tau)), np.isfinite(tau_ref))
+    assert np.max(np.abs(to64(O) - O_ref)) <= O_TOL
+    assert np.max(np.abs(to64(tau)[0] - tau_ref[0])) <= 1e-3
+    refs = orc.attn_bwd_gqa(d["Q"], d["K"], d["V"], d["dO"], km_np, False, 0, 1 / 8, alpha=alpha)
+    for x, r in zip(g, refs):
+        assert np.max(np.abs(to64(x) - r)) <= GRAD_TOL
