@@ -6,7 +6,6 @@ scratch is a fixed array inside the library.  Its gradients must match entmax_at
 gradient tolerance of the parity tests, on two calls in a row (the second sees the array as the
 first left it).  This file is collected last on purpose, and passes alone in a fresh process too.
 """
-import numpy as np
 import pytest
 import torch
 
