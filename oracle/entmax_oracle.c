@@ -395,7 +395,6 @@ void eo_attn_bwd_heads(const double* Q, const double* K, const double* V,
     for (int hh = 0; hh < nheads; ++hh) {
         long long bh = bh_ids[hh];
         int b = (int)(bh / H);
-        int h = (int)(bh % H);
         size_t head = (size_t)bh * per_head;
         double* dQh = dQ + (size_t)hh * per_head;
         double* dKh = dK + (size_t)hh * per_head;
