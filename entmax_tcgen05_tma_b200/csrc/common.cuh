@@ -75,6 +75,10 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ masks
+// The allowed keys of query i follow page "svd-sst2-roberta-adasplash", section 3 ("Structural
+// Masking Stage"): the padding mask of the key's batch row, the causal mask (j <= i) and the
+// causal local window (j >= i - window + 1).  Masked keys are left out of the row, not filled
+// with a large negative score.
 // Bitmap of valid keys of batch row b: bit j set iff j < L and key_mask[b, j] != 0 (or no mask).
 // All threads of the CTA participate.
 __device__ __forceinline__ void build_key_bitmap(uint32_t* bits, const uint8_t* key_mask, int b, int L) {
