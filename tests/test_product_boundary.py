@@ -1,6 +1,8 @@
-"""The product path never reaches the oracle: no module of the package imports it, and the oracle's
-compiled library is not among the package's own files.  bench.py may use it only in its CPU-baseline
-and reference legs (functions whose names say so)."""
+"""The product path and the oracle stay apart.
+
+No module of the package imports the oracle or names its compiled library, and the oracle imports
+nothing of the package and includes none of its headers.  bench.py may use the oracle only in its
+CPU-baseline and reference legs (functions whose names say so)."""
 import ast
 from pathlib import Path
 
@@ -45,3 +47,14 @@ def test_bench_uses_the_oracle_only_in_its_baseline_legs():
         mods = [a.name for a in node.names] if isinstance(node, ast.Import) else [node.module or ""]
         assert not any(m.split(".")[0] == "oracle" for m in mods), "module-level oracle import in bench.py"
     assert users and users <= {"oracle_baseline", "run_reference"}, users
+
+
+def test_oracle_never_imports_the_package():
+    for f in sorted((ROOT / "oracle").glob("*.py")):
+        for _, name in _imports(f):
+            assert name.split(".")[0] != "entmax_tcgen05_tma_b200", (f, name)
+    for f in sorted((ROOT / "oracle").glob("*.c")):
+        text = f.read_text()
+        for line in text.splitlines():
+            if line.startswith("#include"):
+                assert "<" in line and "entmax_attn" not in line, (f, line)
