@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
     ENTMAX_OK = 0,
     ENTMAX_ERR_ARG = -1,          /* null pointer, bad size, bad dtype, misaligned pointer, scale <= 0 */
-    ENTMAX_ERR_UNSUPPORTED = -2,  /* D != 64, L > 16384, B*H > 65535, window without causal */
+    ENTMAX_ERR_UNSUPPORTED = -2,  /* D != 64, L > 16384, B*H > 65535, window without causal, alpha = 1 */
     ENTMAX_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed (see entmax_attn_last_cuda_error) */
     ENTMAX_ERR_TIMEOUT = -4,      /* a device-side bounded wait expired */
     ENTMAX_ERR_WORKSPACE = -5     /* workspace missing or smaller than entmax_attn_bwd_workspace_size */
