@@ -199,6 +199,38 @@ def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: i
             "seconds": dt, "heads": heads, "full_job_seconds_est": dt * full_pairs / max(1, sum(pairs_per_head))}
 
 
+def host_link_rates(dev, stream, nbytes: int = 1 << 28, reps: int = 5) -> dict:
+    """Pinned host-to-device and device-to-host copy rates (GB/s) of this GPU's host link, one
+    direction at a time, timed with CUDA events on `stream`: the ceiling of the end-to-end copies.
+    Runs outside every timed region; any failure is reported instead of the rates."""
+    try:
+        h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+        d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        rates = {}
+        with torch.cuda.stream(stream):
+            for name, dst, src in (("h2d_gbs", d, h), ("d2h_gbs", h, d)):
+                dst.copy_(src, non_blocking=True)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    dst.copy_(src, non_blocking=True)
+                e1.record(stream)
+                e1.synchronize()
+                rates[name] = round(nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9, 2)
+        return rates
+    except Exception as exc:  # a measurement aid only: never fail the bench line for it
+        return {"error": repr(exc)[:200]}
+
+
+def link_bound(rates: dict, h2d_bytes: int, d2h_bytes: int, e2e_ms: float) -> dict:
+    """The end-to-end step against its copy time: the two directions run on separate copy engines,
+    so the bound is the slower direction's bytes over its measured rate."""
+    if "h2d_gbs" not in rates or "d2h_gbs" not in rates:
+        return dict(rates)
+    bound_ms = 1e3 * max(h2d_bytes / (rates["h2d_gbs"] * 1e9), d2h_bytes / (rates["d2h_gbs"] * 1e9))
+    return {**rates, "copy_bound_ms": round(bound_ms, 4), "frac": round(bound_ms / e2e_ms, 4)}
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def measured_sparsity(w: Workload, Q, K, tau, km) -> float:
     """Fraction of allowed pairs with A = 0 (scores recomputed in fp32 with torch, outside the timed
@@ -409,6 +441,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     e2e_ms = dist_max(e0.elapsed_time(e1), world, dev) / e2e_steps
     if E.entmax_attn_device_status() != 0:
         raise RuntimeError("device status after the end-to-end steps")
+    link = host_link_rates(dev, stream)
 
     if rank != 0:
         return None
@@ -490,7 +523,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "chunks": "%d chunks of whole sequences on 2 streams (copies overlap kernels)" % nchunk},
+                "chunks": "%d chunks of whole sequences on 2 streams (copies overlap kernels)" % nchunk,
+                "host_link": link_bound(link, h2d, d2h, e2e_ms)},
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -128,3 +128,24 @@ def test_reference_arm_under_torchrun_prints_one_line():
     assert out["value"] > 0 and out["e2e"]["value"] == out["value"]
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["cpu_baseline"]["kind"] == "oracle"
     assert out["config"]["workload_id"] == 2
+
+
+def test_link_bound_takes_the_slower_direction():
+    import bench
+
+    r = bench.link_bound({"h2d_gbs": 50.0, "d2h_gbs": 40.0}, 100_000_000, 200_000_000, 10.0)
+    # 100 MB at 50 GB/s = 2 ms in, 200 MB at 40 GB/s = 5 ms out: the step cannot beat 5 ms
+    assert r["copy_bound_ms"] == pytest.approx(5.0) and r["frac"] == pytest.approx(0.5)
+    assert r["h2d_gbs"] == 50.0 and r["d2h_gbs"] == 40.0
+    r = bench.link_bound({"h2d_gbs": 10.0, "d2h_gbs": 40.0}, 100_000_000, 200_000_000, 20.0)
+    assert r["copy_bound_ms"] == pytest.approx(10.0) and r["frac"] == pytest.approx(0.5)
+    assert bench.link_bound({"error": "x"}, 1, 1, 1.0) == {"error": "x"}
+
+
+def test_link_rates_report_failure_instead_of_raising():
+    import bench
+
+    if torch.cuda.is_available():
+        pytest.skip("checks the failure path, which needs a machine without a GPU")
+    r = bench.host_link_rates(torch.device("cpu"), None, nbytes=1 << 10, reps=1)
+    assert set(r) == {"error"}
