@@ -225,7 +225,7 @@ def host_link_rates(dev, stream, nbytes: int = 1 << 28, reps: int = 5) -> dict:
 def link_bound(rates: dict, h2d_bytes: int, d2h_bytes: int, e2e_ms: float) -> dict:
     """The end-to-end step against its copy time: the two directions run on separate copy engines,
     so the bound is the slower direction's bytes over its measured rate."""
-    if "h2d_gbs" not in rates or "d2h_gbs" not in rates:
+    if not (rates.get("h2d_gbs", 0) > 0 and rates.get("d2h_gbs", 0) > 0 and e2e_ms > 0):
         return dict(rates)
     bound_ms = 1e3 * max(h2d_bytes / (rates["h2d_gbs"] * 1e9), d2h_bytes / (rates["d2h_gbs"] * 1e9))
     return {**rates, "copy_bound_ms": round(bound_ms, 4), "frac": round(bound_ms / e2e_ms, 4)}

@@ -149,3 +149,10 @@ def test_link_rates_report_failure_instead_of_raising():
         pytest.skip("checks the failure path, which needs a machine without a GPU")
     r = bench.host_link_rates(torch.device("cpu"), None, nbytes=1 << 10, reps=1)
     assert set(r) == {"error"}
+
+
+def test_link_bound_never_divides_by_zero():
+    import bench
+
+    assert bench.link_bound({"h2d_gbs": 0.0, "d2h_gbs": 40.0}, 1, 1, 1.0) == {"h2d_gbs": 0.0, "d2h_gbs": 40.0}
+    assert "copy_bound_ms" not in bench.link_bound({"h2d_gbs": 1.0, "d2h_gbs": 1.0}, 1, 1, 0.0)
