@@ -256,96 +256,182 @@ def measured_sparsity(w: Workload, Q, K, tau, km) -> float:
     return zeros / max(1, allowed)
 
 
+class _Flush:
+    """Evicts L2 between timed steps, outside the step's events: a 256 MiB write (larger than the
+    126 MB L2), then a 256 MiB read of a second buffer, so L2 is left holding clean lines and the
+    timed kernels neither hit on their inputs nor write back the flush's dirty lines."""
+
+    def __init__(self, dev):
+        self.w = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+        self.r = torch.ones((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self, k: int) -> None:
+        self.w.fill_(float(k))
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
+class _Prepared:
+    """Device-resident inputs, outputs and the step's library calls for one workload."""
+
+    def __init__(self, args, w: Workload, dev):
+        import entmax_tcgen05_tma_b200 as E
+
+        self.E, self.w, self.dev = E, w, dev
+        alpha = args.alpha
+        self.variant = variant = alpha != 1.5 or w.kv_heads != w.H or args.blhd  # the _ex entry points
+        self.recompute = recompute = args.bwd == "recompute"  # entmax_attn_fwd + entmax_attn_bwd
+        self.inp = inp = make_inputs(w)
+        self.pairs = allowed_pairs(w, inp["key_mask"])
+        self.flops = dense_equiv_flops(w, self.pairs)
+        # --blhd: the same values held in [B, L, H, 64] memory, passed as transpose(1, 2) views
+        lay = (lambda x: x.transpose(1, 2).contiguous().transpose(1, 2)) if args.blhd else (lambda x: x)
+        self.Q, self.K, self.V, self.dO = (lay(inp[k].to(dev)) for k in ("Q", "K", "V", "dO"))
+        self.km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
+        B, H, L, D = w.B, w.H, w.L, w.D
+        Hkv = w.kv_heads
+        self.O = lay(torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev))
+        self.tau = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+        self.dQ = lay(torch.empty((B, H, L, D), dtype=torch.float32, device=dev))
+        self.dK, self.dV = (lay(torch.empty((B, Hkv, L, D), dtype=torch.float32, device=dev)) for _ in range(2))
+        self.saved = torch.empty((E.entmax_attn_saved_bytes(B, H, L, D),), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty((E.entmax_attn_bwd_saved_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
+        self.rws = torch.empty((max(E.entmax_attn_bwd_workspace_size(B, H, L, D), 1),), dtype=torch.uint8,
+                               device=dev)
+        self.alpha = alpha
+
+    def fwd_call(self):
+        E, w = self.E, self.w
+        Q, K, V, km, O, tau = self.Q, self.K, self.V, self.km, self.O, self.tau
+        if self.recompute:
+            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+        elif self.variant:
+            E.entmax_attn_fwd_ex(Q, K, V, km, w.causal, w.window, w.scale, alpha=self.alpha, save=w.backward, O=O,
+                                 tau=tau, saved=self.saved if w.backward else None)
+        elif w.backward:
+            E.entmax_attn_fwd_train(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau, saved=self.saved)
+        else:
+            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
+
+    def bwd_call(self):
+        E, w = self.E, self.w
+        Q, K, V, km, tau, dO = self.Q, self.K, self.V, self.km, self.tau, self.dO
+        if self.recompute:
+            E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, dQ=self.dQ, dK=self.dK, dV=self.dV,
+                              workspace=self.rws)
+        elif self.variant:
+            E.entmax_attn_bwd_saved_ex(Q, K, V, tau, self.saved, dO, km, w.causal, w.window, w.scale,
+                                       alpha=self.alpha, dQ=self.dQ, dK=self.dK, dV=self.dV, workspace=self.ws)
+        else:
+            E.entmax_attn_bwd_saved(Q, K, V, tau, self.saved, dO, km, w.causal, w.window, w.scale, dQ=self.dQ,
+                                    dK=self.dK, dV=self.dV, workspace=self.ws)
+
+    def step(self):
+        self.fwd_call()
+        if self.w.backward:
+            self.bwd_call()
+
+
+def launches_per_step(w: Workload, recompute: bool) -> int:
+    """The library's kernel launches in one step: the forward kernel, then the backward's kernels
+    (saved supports: key scan, rows, keys and the exact pass for unsaved rows; recompute: rows and
+    keys)."""
+    if not w.backward:
+        return 1
+    return 1 + (2 if recompute else 4)
+
+
+def time_device(prep: _Prepared, flush: _Flush, steps: int, warmup: int, world: int) -> dict:
+    """W warm-up steps, then `steps` timed steps: L2 evicted before each (outside the events), CUDA
+    events on the launching stream around the forward and the backward, clocks sampled during the
+    timed region.  Per-step lists in ms; `total_ms` is the max over ranks."""
+    E, dev, w = prep.E, prep.dev, prep.w
+    stream = torch.cuda.current_stream(dev)
+    for k in range(warmup):
+        flush(k)
+        prep.step()
+    torch.cuda.synchronize(dev)
+    st = E.entmax_attn_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after warm-up" % st)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        wall0 = time.perf_counter()
+        for k in range(steps):
+            flush(k)
+            ev[k][0].record(stream)
+            prep.fwd_call()
+            ev[k][1].record(stream)
+            if w.backward:
+                prep.bwd_call()
+            ev[k][2].record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    dist_barrier(world)
+    st = E.entmax_attn_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after the timed steps" % st)
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    return {"fwd_ms": [a.elapsed_time(b) for a, b, _ in ev], "bwd_ms": [b.elapsed_time(c) for _, b, c in ev],
+            "step_ms": step_ms, "total_ms": dist_max(sum(step_ms), world, dev), "wall_s": wall,
+            "clocks": clk.summary()}
+
+
+def step_roofline(w: Workload, km, flops: float, ms_per_step: float, peaks: dict) -> dict:
+    """The whole step against its roofline time: max(dense-equivalent FLOPs / bf16 burst peak,
+    minimum HBM bytes / HBM peak), as a fraction of the measured step time."""
+    step_bytes = min_hbm_bytes(w, km)
+    t_flop, t_byte = flops / (peaks["bf16_tflops"] * 1e12), step_bytes / (peaks["hbm_gbs"] * 1e9)
+    return {"bound": "tensor" if t_flop >= t_byte else "hbm", "time_us": round(1e6 * max(t_flop, t_byte), 2),
+            "frac": round(1e3 * max(t_flop, t_byte) / ms_per_step, 4), "min_hbm_bytes": step_bytes,
+            "peaks": "bf16 %.1f TFLOP/s (burst), HBM %.1f GB/s (%s)" % (peaks["bf16_tflops"], peaks["hbm_gbs"],
+                                                                     peaks["source"])}
+
+
+def extra_workload(args, wid: int, dev, world: int, flush: _Flush, peaks: dict) -> dict:
+    """Another fwd+bwd workload timed in the same process and the same way as the headline line
+    (same library calls, L2 eviction, events, warm-up and step count)."""
+    w = WORKLOADS[wid]
+    prep = _Prepared(args, w, dev)
+    t = time_device(prep, flush, args.steps, args.warmup, world)
+    ms = t["total_ms"] / args.steps
+    sparsity = measured_sparsity(w, prep.Q, prep.K, prep.tau, prep.km)
+    out = {"workload": workload_desc(w), "steps": args.steps, "warmup": args.warmup,
+           "value": round(aggregate_value(prep.flops, world, ms), 3), "unit": "TFLOP/s",
+           "ms_per_step": round(ms, 4), "fwd_ms": round(statistics.mean(t["fwd_ms"]), 4),
+           "bwd_ms": round(statistics.mean(t["bwd_ms"]), 4) if w.backward else 0.0,
+           "step_ms_median": round(statistics.median(t["step_ms"]), 4),
+           "dense_equiv_gflop_per_step": prep.flops / 1e9, "allowed_pairs": prep.pairs,
+           "sparsity": round(sparsity, 4), "step_roofline": step_roofline(w, prep.km, prep.flops, ms, peaks),
+           "gpu_launches": launches_per_step(w, prep.recompute) * args.steps, "clocks": t["clocks"]}
+    del prep
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args, rank: int, world: int) -> dict | None:
     import entmax_tcgen05_tma_b200 as E
 
     w = bench_workload(args)
     alpha = args.alpha
-    variant = alpha != 1.5 or w.kv_heads != w.H or args.blhd  # the _ex entry points
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    inp = make_inputs(w)
-    pairs = allowed_pairs(w, inp["key_mask"])
-    flops = dense_equiv_flops(w, pairs)
-    # --blhd: the same values held in [B, L, H, 64] memory, passed as transpose(1, 2) views
-    lay = (lambda x: x.transpose(1, 2).contiguous().transpose(1, 2)) if args.blhd else (lambda x: x)
-    Q, K, V, dO = (lay(inp[k].to(dev)) for k in ("Q", "K", "V", "dO"))
-    km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
+    prep = _Prepared(args, w, dev)
+    variant, recompute = prep.variant, prep.recompute
+    inp, pairs, flops = prep.inp, prep.pairs, prep.flops
+    Q, K, tau, km = prep.Q, prep.K, prep.tau, prep.km
     B, H, L, D = w.B, w.H, w.L, w.D
     Hkv = w.kv_heads
-    O = lay(torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev))
-    tau = torch.empty((B, H, L), dtype=torch.float32, device=dev)
-    dQ = lay(torch.empty((B, H, L, D), dtype=torch.float32, device=dev))
-    dK, dV = (lay(torch.empty((B, Hkv, L, D), dtype=torch.float32, device=dev)) for _ in range(2))
-    saved = torch.empty((E.entmax_attn_saved_bytes(B, H, L, D),), dtype=torch.uint8, device=dev)
-    ws = torch.empty((E.entmax_attn_bwd_saved_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
-    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device=dev)
+    O = prep.O
     stream = torch.cuda.current_stream(dev)
-    recompute = args.bwd == "recompute"  # entmax_attn_fwd + entmax_attn_bwd (scores recomputed)
-    rws = torch.empty((max(E.entmax_attn_bwd_workspace_size(B, H, L, D), 1),), dtype=torch.uint8, device=dev)
-    launches_per_step = 1 + ((2 if recompute else 4) if w.backward else 0)
+    flush = _Flush(dev)
 
-    def fwd_call():
-        if recompute:
-            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
-        elif variant:
-            E.entmax_attn_fwd_ex(Q, K, V, km, w.causal, w.window, w.scale, alpha=alpha, save=w.backward, O=O, tau=tau,
-                                 saved=saved if w.backward else None)
-        elif w.backward:
-            E.entmax_attn_fwd_train(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau, saved=saved)
-        else:
-            E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale, O=O, tau=tau)
-
-    def bwd_call():
-        if recompute:
-            E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV, workspace=rws)
-        elif variant:
-            E.entmax_attn_bwd_saved_ex(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale, alpha=alpha, dQ=dQ,
-                                       dK=dK, dV=dV, workspace=ws)
-        else:
-            E.entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, km, w.causal, w.window, w.scale, dQ=dQ, dK=dK, dV=dV,
-                                    workspace=ws)
-
-    def step():
-        fwd_call()
-        if w.backward:
-            bwd_call()
-
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        step()
-    torch.cuda.synchronize(dev)
-    st = E.entmax_attn_device_status()
-    if st != 0:
-        raise RuntimeError("device status %d after warm-up" % st)
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    dist_barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clk:
-        wall0 = time.perf_counter()
-        for k in range(args.steps):
-            flush.fill_(float(k))  # evict L2 between steps (outside the timed events)
-            ev[k][0].record(stream)
-            fwd_call()
-            ev[k][1].record(stream)
-            if w.backward:
-                bwd_call()
-            ev[k][2].record(stream)
-        torch.cuda.synchronize(dev)
-        wall = time.perf_counter() - wall0
-    dist_barrier(world)
-    clocks = clk.summary()
-    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
-    bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
-    step_ms = [a.elapsed_time(c) for a, _, c in ev]
-    total_ms = sum(step_ms)
-    total_ms = dist_max(total_ms, world, dev)
-    st = E.entmax_attn_device_status()
-    if st != 0:
-        raise RuntimeError("device status %d after the timed steps" % st)
-
+    t = time_device(prep, flush, args.steps, args.warmup, world)
+    fwd_ms, bwd_ms, step_ms, total_ms = t["fwd_ms"], t["bwd_ms"], t["step_ms"], t["total_ms"]
+    clocks, wall = t["clocks"], t["wall_s"]
     # ---- end to end through the public API, host buffers, copies inside the timed region
     host_in = {k: inp[k].pin_memory() for k in ("Q", "K", "V", "dO")}
     if args.blhd:  # host tensors in [B, L, H, 64] memory too
@@ -443,6 +529,13 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         raise RuntimeError("device status after the end-to-end steps")
     link = host_link_rates(dev, stream)
 
+    # the other fwd+bwd workloads the bf16-roofline target covers (L >= 512), timed the same way on
+    # every rank (their timing takes the same barriers and max over ranks)
+    extras = {}
+    if not args.no_extra and not variant and not recompute and args.workload == 4:
+        peaks = load_peaks()
+        extras = {str(k): extra_workload(args, k, dev, world, flush, peaks) for k in (3, 5)}
+
     if rank != 0:
         return None
 
@@ -461,12 +554,14 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     fwd_mean = statistics.mean(fwd_ms)
     bwd_mean = statistics.mean(bwd_ms) if w.backward else 0.0
     ms_per_step = total_ms / args.steps
-    t_tensor = fwd_alg_flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    # the forward kernel runs for well under a millisecond inside a sub-millisecond step: the burst
+    # bf16 figure is its tensor peak
+    t_tensor = fwd_alg_flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = fwd_alg_bytes / (peaks["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
         roof = {"kernel": "entmax_fwd_kernel", "bound": "tensor",
-                "achieved": fwd_alg_flops / (fwd_mean * 1e-3) / 1e12, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "peak_source": "%s bf16 sustained (MEASURED_PEAKS.json)" % peaks["source"]}
+                "achieved": fwd_alg_flops / (fwd_mean * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks["source"]}
     else:
         roof = {"kernel": "entmax_fwd_kernel", "bound": "hbm",
                 "achieved": fwd_alg_bytes / (fwd_mean * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
@@ -480,14 +575,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         if t.get("kernel") == "entmax_fwd_kernel" and t.get("source_hash") == source_hash():
             roof["traffic"] = t["bytes_per_launch"]
 
-    # the whole step against its roofline time: max(dense-equivalent FLOPs / bf16 peak, minimum HBM
-    # bytes / HBM peak), as a fraction of the measured step time
-    step_bytes = min_hbm_bytes(w, km)
-    t_flop, t_byte = flops / (peaks["bf16_tflops"] * 1e12), step_bytes / (peaks["hbm_gbs"] * 1e9)
-    step_roof = {"bound": "tensor" if t_flop >= t_byte else "hbm", "time_us": round(1e6 * max(t_flop, t_byte), 2),
-                 "frac": round(1e3 * max(t_flop, t_byte) / ms_per_step, 4), "min_hbm_bytes": step_bytes,
-                 "peaks": "bf16 %.1f TFLOP/s, HBM %.1f GB/s (%s)" % (peaks["bf16_tflops"], peaks["hbm_gbs"],
-                                                                  peaks["source"])}
+    step_roof = step_roofline(w, km, flops, ms_per_step, peaks)
     value = aggregate_value(flops, world, ms_per_step)
     out = {
         "metric": METRIC,
@@ -508,7 +596,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "allowed_pairs": pairs,
             "dense_equiv_gflop_per_step": flops / 1e9,
             "dense_equiv_gflop_full_L2": dense_equiv_flops(w, w.B * w.H * w.L * w.L) / 1e9,
-            "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+            "l2": "evicted before each timed step, outside its events: 256 MiB written, then another 256 MiB read "
+                  "(L2 left holding clean lines)",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
         "variant": {"alpha": alpha, "H_kv": Hkv, "layout": "BLHD" if args.blhd else "BHLD"} if variant else None,
@@ -520,13 +609,15 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "sparsity": round(sparsity, 4),
         "roofline": roof,
         "step_roofline": step_roof,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step(w, recompute) * args.steps,
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "chunks": "%d chunks of whole sequences on 2 streams (copies overlap kernels)" % nchunk,
                 "host_link": link_bound(link, h2d, d2h, e2e_ms)},
         "clocks": clocks,
     }
+    if extras:
+        out["workloads"] = extras
     if world == 1 and not args.no_cpu_baseline:
         cb = oracle_baseline(w, inp, budget_s=args.cpu_seconds, alpha=alpha)
         out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
@@ -622,6 +713,8 @@ def main() -> int:
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the selected workload (the default workload-4 line also times 3 and 5)")
     ap.add_argument("--alpha", type=float, default=1.5, help="alpha-entmax variant, alpha in (1, 2]")
     ap.add_argument("--hkv", type=int, default=0, help="grouped-query variant: key/value heads")
     ap.add_argument("--blhd", action="store_true", help="variant: tensors in [B, L, H, 64] memory")

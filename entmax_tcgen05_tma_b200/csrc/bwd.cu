@@ -292,6 +292,17 @@ __device__ __forceinline__ void setup_cta(const Smem& sm, const CUtensorMap* ma,
 __device__ __forceinline__ void finish_cta(const Smem& sm) {
     tc_fence_before();
     __syncthreads();
+    // Past this barrier no thread waits, so the abort flag is final (uniform).  After an abort every
+    // TMA load and MMA issued must complete before the CTA frees TMEM and its shared memory.
+    if (P::aborted(sm.ctl)) {
+        const int warp = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) {
+            if (warp == WARP_PRODUCER) P::drain_loads(sm.ctl);
+            if (warp == WARP_MMA) P::drain_mma(sm.ctl);
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if ((threadIdx.x >> 5) == WARP_PRODUCER) {
         tc_fence_after();
         tmem_dealloc(sm.ctl->tmem_base, TMEM_COLS);

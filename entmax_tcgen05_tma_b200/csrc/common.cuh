@@ -13,8 +13,12 @@
 //   producer warp        : TMEM allocation / release
 //
 // Every wait is bounded: on timeout the CTA records ENTMAX_ERR_TIMEOUT in the device status
-// word, raises a CTA-local abort flag that all roles poll, waits (again bounded) for its own
-// TMA loads and MMAs in flight, releases TMEM and returns.
+// word and raises a CTA-local abort flag that all roles poll; every role then stops and the CTA
+// meets at its teardown barrier.  Past that barrier no thread waits on anything else, so the flag
+// is final: if it is set, the producer thread waits (again bounded) for every TMA load it issued
+// and the MMA thread for its last commit (drain_loads / drain_mma), and only then is TMEM released
+// and the CTA returns.  A role that finished issuing before another role timed out still has its
+// copies drained this way.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -49,19 +53,21 @@ static __device__ __noinline__ void raise_timeout(int* abort_flag, const WaitCfg
     if (wc.status) atomicExch(wc.status, STATUS_TIMEOUT);
 }
 
+constexpr uint32_t POLL_SUSPEND_NS = 256;  // longest suspension inside one poll of a bounded wait
+
 // Bounded wait on an mbarrier phase.  Returns false if the CTA aborted (this wait timed out,
-// or another role already raised the abort flag).
+// or another role already raised the abort flag).  Each poll after the first suspends the thread
+// for at most POLL_SUSPEND_NS, and the abort flag and the clock are checked after every failed
+// poll, so a wait gives up within about POLL_SUSPEND_NS of its bound.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, int* abort_flag, const WaitCfg& wc) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 127u) == 0) {
-            if (flag_set(abort_flag)) return false;
-            if (globaltimer_ns() - t0 > wc.timeout_ns) {
-                raise_timeout(abort_flag, wc);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_hint(bar, parity, POLL_SUSPEND_NS)) return true;
+        if (flag_set(abort_flag)) return false;
+        if (globaltimer_ns() - t0 > wc.timeout_ns) {
+            raise_timeout(abort_flag, wc);
+            return false;
         }
     }
 }
@@ -69,7 +75,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, int*
 // Wait used only while draining after an abort: ignores the abort flag, fixed bound.
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_hint(bar, parity, POLL_SUSPEND_NS)) {
         if (globaltimer_ns() - t0 > TEARDOWN_TIMEOUT_NS) return;
     }
 }
@@ -148,6 +154,8 @@ struct Pipe {
         uint32_t tmem_base;
         int abort_flag;
         int nblk;                      // streamed blocks this CTA visits
+        int nload[2];                  // B-block loads issued (per producer/MMA pair)
+        int nmma[2];                   // score blocks whose MMAs were issued (per pair)
         int pad_;
     };
 
@@ -166,7 +174,25 @@ struct Pipe {
             mbar_init(smem_u32(&ctl->s_empty[b]), empty_arrivals);
         }
         ctl->abort_flag = 0;
+        ctl->nload[0] = ctl->nload[1] = 0;
+        ctl->nmma[0] = ctl->nmma[1] = 0;
         fence_barrier_init();
+    }
+
+    // Teardown after an abort, run by the producer thread past the CTA's teardown barrier: waits
+    // (bounded) for the A tile and the last NSTAGE B loads -- every earlier load was waited on by
+    // the MMA thread before it reused the stage.
+    static __device__ __forceinline__ void drain_loads(Ctl* ctl) {
+        wait_drain(smem_u32(&ctl->full_a), 0);
+        const int n1 = ctl->nload[0];
+        for (int n = max(0, n1 - NSTAGE); n < n1; ++n)
+            wait_drain(smem_u32(&ctl->full_b[n % NSTAGE]), (uint32_t)(n / NSTAGE) & 1u);
+    }
+
+    // Teardown after an abort, run by the MMA thread: its last commit covers every MMA it issued.
+    static __device__ __forceinline__ void drain_mma(Ctl* ctl) {
+        const int n = ctl->nmma[0] - 1;
+        if (n >= 0) wait_drain(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u);
     }
 
     // Streamed blocks a query tile (rows [i0, i_last]) visits: blocks kb in [klo/BLK, khi/BLK]
@@ -225,12 +251,7 @@ struct Pipe {
             tma_load_3d(smem_u32(smem_b + s * BLK_BYTES), map_b, 0, hb.c1(row), hb.c2(row), smem_u32(&ctl->full_b[s]));
             ++issued;
         }
-        if (aborted(ctl)) {
-            // drain: every load issued must land before the CTA's shared memory is released
-            wait_drain(smem_u32(&ctl->full_a), 0);
-            for (int n = max(0, issued - NSTAGE); n < issued; ++n)
-                wait_drain(smem_u32(&ctl->full_b[n % NSTAGE]), (uint32_t)(n / NSTAGE) & 1u);
-        }
+        ctl->nload[0] = issued;  // drained at teardown if the CTA aborts (drain_loads)
     }
 
     // MMA issuer (one thread).
@@ -257,10 +278,7 @@ struct Pipe {
                 ++issued;
             }
         }
-        if (aborted(ctl) && issued > 0) {
-            const int n = issued - 1;  // the last commit covers every earlier MMA
-            wait_drain(smem_u32(&ctl->s_full[n % NBUF]), (uint32_t)(n / NBUF) & 1u);
-        }
+        ctl->nmma[0] = issued;  // drained at teardown if the CTA aborts (drain_mma)
     }
 
     // Epilogue side: wait for the score buffer of streamed block n; false on abort.

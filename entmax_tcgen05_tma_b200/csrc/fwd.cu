@@ -648,12 +648,22 @@ __device__ __noinline__ void produce_half(PipeCtl* ctl, const WaitCfg& wc, const
         tma_load_3d(smem_u32(smem_b + st * BLK_BYTES), map_b, 0, hb.c1(row), hb.c2(row), smem_u32(&ctl->full_b[st]));
         ++issued;
     }
-    if (P::aborted(ctl)) {
-        // drain: every copy issued must land before the CTA's shared memory is released
-        if (p == 0) wait_drain(smem_u32(&ctl->full_a), 0);
-        for (int m = max(0, issued - 2); m < issued; ++m)
-            wait_drain(smem_u32(&ctl->full_b[2 * p + (m & 1)]), (uint32_t)(m >> 1) & 1u);
+    ctl->nload[p] = issued;  // drained at teardown if the CTA aborts (drain_half)
+}
+
+// Teardown after an abort (past the CTA's teardown barrier), streamed tile, pipeline p: the producer
+// thread waits for the A tile (pipeline 0) and its last two K loads; the MMA thread for its last
+// commit, which covers every MMA it issued.
+__device__ __noinline__ void drain_half(PipeCtl* ctl, int p, bool mma_thread) {
+    if (mma_thread) {
+        const int m = ctl->nmma[p] - 1;
+        if (m >= 0) wait_drain(smem_u32(&ctl->s_full[p + 2 * (m & 1)]), (uint32_t)(m >> 1) & 1u);
+        return;
     }
+    if (p == 0) wait_drain(smem_u32(&ctl->full_a), 0);
+    const int n = ctl->nload[p];
+    for (int m = max(0, n - 2); m < n; ++m)
+        wait_drain(smem_u32(&ctl->full_b[2 * p + (m & 1)]), (uint32_t)(m >> 1) & 1u);
 }
 
 __device__ __noinline__ void mma_half(PipeCtl* ctl, const WaitCfg& wc, const uint8_t* smem_a, const uint8_t* smem_b,
@@ -679,10 +689,7 @@ __device__ __noinline__ void mma_half(PipeCtl* ctl, const WaitCfg& wc, const uin
             ++issued;
         }
     }
-    if (P::aborted(ctl) && issued > 0) {
-        const int m = issued - 1;  // the last commit covers every earlier MMA of this thread
-        wait_drain(smem_u32(&ctl->s_full[p + 2 * (m & 1)]), (uint32_t)(m >> 1) & 1u);
-    }
+    ctl->nmma[p] = issued;  // drained at teardown if the CTA aborts (drain_half)
 }
 
 template <bool GEN>
@@ -1125,6 +1132,22 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
+    // Past this barrier no thread waits, so the abort flag is final (uniform).  After an abort every
+    // TMA load and MMA issued must complete before the CTA frees TMEM and its shared memory.
+    if (P::aborted(ctl)) {
+        if (lane == 0) {
+            if (resident) {
+                if (warp == WARP_PRODUCER) P::drain_loads(ctl);
+                if (warp == WARP_MMA) P::drain_mma(ctl);
+            } else if (warp == WARP_PRODUCER || warp == WARP_PRODUCER2) {
+                drain_half(ctl, warp == WARP_PRODUCER ? 0 : 1, false);
+            } else if (warp == WARP_MMA || warp == WARP_MMA2) {
+                drain_half(ctl, warp == WARP_MMA ? 0 : 1, true);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == WARP_PRODUCER) {
         tc_fence_after();
         tmem_dealloc(ctl->tmem_base, TMEM_COLS);

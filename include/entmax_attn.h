@@ -31,6 +31,12 @@
  * (entmax_attn_set_wait_timeout_ns), the last CUDA error and each device's status word are
  * shared by the whole process.
  *
+ * Contexts: the first call on a device looks up, once, the device addresses of the library's own
+ * device variables (the status word; the scratch array of entmax_attn_bwd_noalloc) in that
+ * device's primary context and keeps them for the life of the process.  Destroying or resetting
+ * the primary context (cudaDeviceReset, cuDevicePrimaryCtxReset) invalidates them: do not call
+ * the library on that device again in the same process after such a reset.
+ *
  * Errors: arguments are checked on the host before any launch; a bad argument returns a
  * negative status and launches nothing.  Problems found on the device (a bounded wait that
  * timed out) are recorded in a device status word; entmax_attn_device_status() reads it.
