@@ -332,12 +332,20 @@ class _Prepared:
             self.bwd_call()
 
 
-def launches_per_step(w: Workload, recompute: bool) -> int:
+def tensor_core_backward(w: Workload, alpha: float = 1.5) -> bool:
+    """Whether the library runs the backward on its tensor-core kernels (dq, dkdv): alpha 1.5 with
+    L <= 512 or a causal window of at most 128 keys (the library's own dispatch rule)."""
+    return alpha == 1.5 and (w.L <= 512 or (w.causal and 0 < w.window <= 128))
+
+
+def launches_per_step(w: Workload, recompute: bool, alpha: float = 1.5) -> int:
     """The library's kernel launches in one step: the forward kernel, then the backward's kernels
-    (saved supports: key scan, rows, keys and the exact pass for unsaved rows; recompute: rows and
-    keys)."""
+    (tensor-core configurations: dq and dkdv; otherwise saved supports: key scan, rows, keys and the
+    exact pass for unsaved rows, or, recomputing the scores: rows and keys)."""
     if not w.backward:
         return 1
+    if tensor_core_backward(w, alpha):
+        return 3
     return 1 + (2 if recompute else 4)
 
 
@@ -406,7 +414,7 @@ def extra_workload(args, wid: int, dev, world: int, flush: _Flush, peaks: dict) 
            "step_ms_median": round(statistics.median(t["step_ms"]), 4),
            "dense_equiv_gflop_per_step": prep.flops / 1e9, "allowed_pairs": prep.pairs,
            "sparsity": round(sparsity, 4), "step_roofline": step_roofline(w, prep.km, prep.flops, ms, peaks),
-           "gpu_launches": launches_per_step(w, prep.recompute) * args.steps, "clocks": t["clocks"]}
+           "gpu_launches": launches_per_step(w, prep.recompute, args.alpha) * args.steps, "clocks": t["clocks"]}
     del prep
     torch.cuda.empty_cache()
     return out
@@ -601,7 +609,9 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
         "variant": {"alpha": alpha, "H_kv": Hkv, "layout": "BLHD" if args.blhd else "BHLD"} if variant else None,
-        "backward": "entmax_attn_bwd (scores recomputed)" if recompute else "entmax_attn_bwd_saved (saved supports)",
+        "backward": ("entmax_attn_bwd" if recompute else "entmax_attn_bwd_saved") + (
+            " (tensor-core kernels: scores recomputed, every product on tcgen05)" if tensor_core_backward(w, alpha)
+            else " (scores recomputed)" if recompute else " (saved supports)"),
         "fwd_ms": round(fwd_mean, 4),
         "bwd_ms": round(bwd_mean, 4),
         "step_ms_median": round(statistics.median(step_ms), 4),
@@ -609,7 +619,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "sparsity": round(sparsity, 4),
         "roofline": roof,
         "step_roofline": step_roof,
-        "gpu_launches": launches_per_step(w, recompute) * args.steps,
+        "gpu_launches": launches_per_step(w, recompute, alpha) * args.steps,
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "chunks": "%d chunks of whole sequences on 2 streams (copies overlap kernels)" % nchunk,

@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     EntmaxAttention,
     EntmaxError,
     entmax_attn_bwd,
+    entmax_attn_bwd_aux,
     entmax_attn_bwd_noalloc,
     entmax_attn_bwd_saved,
     entmax_attn_bwd_saved_ex,
@@ -30,6 +31,7 @@ from ._binding import (  # noqa: F401
     entmax_attn_bwd_workspace_size,
     entmax_attn_device_status,
     entmax_attn_fwd,
+    entmax_attn_fwd_aux,
     entmax_attn_fwd_ex,
     entmax_attn_fwd_gqa,
     entmax_attn_fwd_train,

@@ -31,6 +31,8 @@ EXPORTED = (
     "entmax_attn_bwd_workspace_size",
     "entmax_attn_bwd",
     "entmax_attn_bwd_noalloc",
+    "entmax_attn_fwd_aux",
+    "entmax_attn_bwd_aux",
     "entmax_attn_saved_bytes",
     "entmax_attn_bwd_saved_workspace_size",
     "entmax_attn_fwd_train",
@@ -74,6 +76,11 @@ def _load_library() -> ctypes.CDLL:
     lib.entmax_attn_bwd.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.entmax_attn_bwd_noalloc.restype = i
     lib.entmax_attn_bwd_noalloc.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp]
+    lib.entmax_attn_fwd_aux.restype = i
+    lib.entmax_attn_fwd_aux.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, i, vp, vp, vp, vp]
+    lib.entmax_attn_bwd_aux.restype = i
+    lib.entmax_attn_bwd_aux.argtypes = [vp, vp, vp, i, vp, i, i, f, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                        vp]
     lib.entmax_attn_saved_bytes.restype = sz
     lib.entmax_attn_saved_bytes.argtypes = [i, i, i, i]
     lib.entmax_attn_bwd_saved_workspace_size.restype = sz
@@ -317,6 +324,68 @@ def entmax_attn_bwd_noalloc(Q, K, V, tau, dO, key_mask=None, causal=False, windo
                                      outs[1].data_ptr(), outs[2].data_ptr(), _stream_handle(stream))
     if st != ENTMAX_OK:
         raise EntmaxError(st, "entmax_attn_bwd_noalloc")
+    return tuple(outs)
+
+
+def entmax_attn_fwd_aux(Q, K, V, key_mask=None, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
+                        O=None, tau=None, Otil=None, rsum=None, stream=None):
+    """Forward pass that also returns the auxiliary rows: Otil [B,H,L,64] fp32 (sum_j sqrt(p_ij) V_j)
+    and rsum [B,H,L] fp32 (sum_j sqrt(p_ij)).  Returns (O, tau, Otil, rsum)."""
+    B, H, L, D = Q.shape
+    _check_input("Q", Q, (B, H, L, D))
+    _check_input("K", K, (B, H, L, D), Q.dtype)
+    _check_input("V", V, (B, H, L, D), Q.dtype)
+    if scale is None:
+        scale = D ** -0.5
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be bfloat16 or float32")
+    outs = []
+    for name, t, shape, dt in (("O", O, (B, H, L, D), out_dtype), ("tau", tau, (B, H, L), torch.float32),
+                               ("Otil", Otil, (B, H, L, D), torch.float32), ("rsum", rsum, (B, H, L), torch.float32)):
+        if t is None:
+            t = torch.empty(shape, dtype=dt, device=Q.device)
+        else:
+            _check_input(name, t, shape, dt)
+        outs.append(t)
+    st = lib.entmax_attn_fwd_aux(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
+                                 _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale), B,
+                                 H, L, D, outs[0].data_ptr(), ENTMAX_F32 if out_dtype == torch.float32 else ENTMAX_BF16,
+                                 outs[1].data_ptr(), outs[2].data_ptr(), outs[3].data_ptr(), _stream_handle(stream))
+    if st != ENTMAX_OK:
+        raise EntmaxError(st, "entmax_attn_fwd_aux")
+    return tuple(outs)
+
+
+def entmax_attn_bwd_aux(Q, K, V, tau, Otil, rsum, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None,
+                        dK=None, dV=None, workspace=None, stream=None):
+    """Backward pass taking the auxiliary rows of entmax_attn_fwd_aux.  Returns (dQ, dK, dV) fp32."""
+    B, H, L, D = Q.shape
+    _check_input("Q", Q, (B, H, L, D))
+    _check_input("K", K, (B, H, L, D), Q.dtype)
+    _check_input("V", V, (B, H, L, D), Q.dtype)
+    _check_input("dO", dO, (B, H, L, D), Q.dtype)
+    _check_input("tau", tau, (B, H, L), torch.float32)
+    _check_input("Otil", Otil, (B, H, L, D), torch.float32)
+    _check_input("rsum", rsum, (B, H, L), torch.float32)
+    if scale is None:
+        scale = D ** -0.5
+    outs = []
+    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        if t is None:
+            t = torch.empty((B, H, L, D), dtype=torch.float32, device=Q.device)
+        else:
+            _check_input(name, t, (B, H, L, D), torch.float32)
+        outs.append(t)
+    ws_bytes = entmax_attn_bwd_workspace_size(B, H, L, D)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=Q.device)
+    st = lib.entmax_attn_bwd_aux(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),
+                                 _mask_ptr(key_mask, B, L, Q.device), int(bool(causal)), int(window), float(scale), B,
+                                 H, L, D, tau.data_ptr(), Otil.data_ptr(), rsum.data_ptr(), dO.data_ptr(),
+                                 outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != ENTMAX_OK:
+        raise EntmaxError(st, "entmax_attn_bwd_aux")
     return tuple(outs)
 
 

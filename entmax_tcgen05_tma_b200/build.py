@@ -14,7 +14,7 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libentmax_attn.so"
-SOURCES = ["abi.cu", "fwd.cu", "bwd.cu", "bwd_saved.cu"]
+SOURCES = ["abi.cu", "fwd.cu", "bwd.cu", "bwd_saved.cu", "bwd_dense.cu"]
 DEPS = SOURCES + ["common.cuh", "ptx.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -115,14 +115,17 @@ cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, cudaStream
 }
 
 cudaError_t ensure_smem_attr(const void* func, int bytes, int slot) {
-    static std::atomic<bool> done[8][MAX_DEVICES] = {};
+    constexpr int SLOTS = 16;
+    static std::atomic<bool> done[SLOTS][MAX_DEVICES] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= MAX_DEVICES || slot < 0 || slot >= 8) return cudaErrorInvalidValue;
+    if (dev < 0 || dev >= MAX_DEVICES || slot < 0 || slot >= SLOTS) return cudaErrorInvalidValue;
     if (done[slot][dev].load(std::memory_order_acquire)) return cudaSuccess;
-    // setting the attribute twice (two threads racing here) is harmless
+    // setting the attributes twice (two threads racing here) is harmless
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // the whole unified L1/shared array as shared memory, so kernels sized for two CTAs per SM get two
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e == cudaSuccess) done[slot][dev].store(true, std::memory_order_release);
     return e;
 }
@@ -216,7 +219,7 @@ int check_alpha(float alpha) {
 
 int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
              int window, float scale, float alpha, int B, int H, int Hkv, int L, int D, int layout, void* O,
-             int out_dtype, float* tau, cudaStream_t stream) {
+             int out_dtype, float* tau, cudaStream_t stream, float* otil = nullptr, float* rsum = nullptr) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
     rc = check_alpha(alpha);
@@ -244,7 +247,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
         a.K = dst[1];
         a.V = dst[2];
     }
-    FwdOut o{O, out_dtype == ENTMAX_F32, tau, SavedSupport{}};
+    FwdOut o{O, out_dtype == ENTMAX_F32, tau, SavedSupport{}, otil, rsum};
     return record(launch_fwd(a, o, stream));
 }
 }  // namespace
@@ -271,9 +274,13 @@ size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D) {
     return (((size_t)B * H * L * sizeof(float)) + 255) & ~size_t(255);
 }
 
-int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
-                    int window, float scale, int B, int H, int L, int D, const float* tau, const void* dO, float* dQ,
-                    float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+int bwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+             int window, float scale, int B, int H, int L, int D, const float* tau, const void* dO, float* dQ,
+             float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream,
+             const float* otil = nullptr, const float* rsum = nullptr) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
     if (B == 0 || H == 0 || L == 0) return ENTMAX_OK;
@@ -288,7 +295,7 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
     AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), H, 0.5f, 0};
-    BwdIO io{tau, dO, dQ, dK, dV, static_cast<float*>(workspace)};
+    BwdIO io{tau, dO, dQ, dK, dV, static_cast<float*>(workspace), otil, rsum};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[4] = {Q, K, V, dO};
@@ -300,7 +307,36 @@ int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, c
         a.V = dst[2];
         io.dO = dst[3];
     }
-    return record(launch_bwd(a, io, stream));
+    // the tensor-core kernels store gradient rows 16 bytes at a time
+    const bool dense = dense_bwd(a) && aligned(dQ, 16) && aligned(dK, 16) && aligned(dV, 16);
+    return record(dense ? launch_bwd_dense(a, io, stream) : launch_bwd(a, io, stream));
+}
+}  // namespace
+
+extern "C" {
+
+int entmax_attn_bwd(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
+                    int window, float scale, int B, int H, int L, int D, const float* tau, const void* dO, float* dQ,
+                    float* dK, float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    return bwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, L, D, tau, dO, dQ, dK, dV, workspace,
+                    ws_bytes, stream);
+}
+
+int entmax_attn_fwd_aux(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                        int causal, int window, float scale, int B, int H, int L, int D, void* O, int out_dtype,
+                        float* tau, float* Otil, float* rsum, cudaStream_t stream) {
+    if (B > 0 && H > 0 && L > 0 && (!Otil || !rsum || !aligned(Otil, 16) || !aligned(rsum, 4))) return ENTMAX_ERR_ARG;
+    return fwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, 1.5f, B, H, H, L, D, 0, O, out_dtype, tau,
+                    stream, Otil, rsum);
+}
+
+int entmax_attn_bwd_aux(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask,
+                        int causal, int window, float scale, int B, int H, int L, int D, const float* tau,
+                        const float* Otil, const float* rsum, const void* dO, float* dQ, float* dK, float* dV,
+                        void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (B > 0 && H > 0 && L > 0 && (!Otil || !rsum || !aligned(Otil, 16) || !aligned(rsum, 4))) return ENTMAX_ERR_ARG;
+    return bwd_impl(Q, K, V, in_dtype, key_mask, causal, window, scale, B, H, L, D, tau, dO, dQ, dK, dV, workspace,
+                    ws_bytes, stream, Otil, rsum);
 }
 
 }  // extern "C"
@@ -344,13 +380,18 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     int* status = nullptr;
     rc = record(status_ptr(&status));
     if (rc) return rc;
-    const SavedSupport sv = carve_saved(saved, R);
-    rc = record(cudaMemsetAsync(sv.key_cnt, 0, sizeof(int) * (size_t)R, stream));
-    if (rc) return rc;
-    rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
-    if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
     AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, alpha - 1.f, layout};
+    // the tensor-core backward recomputes the scores and reads no support lists: none are saved
+    // (it derives u_i in a pass of its own, which costs less than writing the auxiliary rows here)
+    const bool save = !dense_bwd(a);
+    const SavedSupport sv = save ? carve_saved(saved, R) : SavedSupport{};
+    if (save) {
+        rc = record(cudaMemsetAsync(sv.key_cnt, 0, sizeof(int) * (size_t)R, stream));
+        if (rc) return rc;
+        rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
+        if (rc) return rc;
+    }
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -401,8 +442,12 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
         a.V = dst[2];
         io.dO = dst[3];
     }
-    return record(launch_bwd_saved(a, io, carve_saved(const_cast<void*>(saved), R), carve_saved_bwd_ws(workspace, R),
-                                   stream));
+    const SavedBwdWs ws = carve_saved_bwd_ws(workspace, R);
+    if (dense_bwd(a)) {
+        io.u = reinterpret_cast<float*>(ws.key_off);  // R floats of the workspace hold u
+        return record(launch_bwd_dense(a, io, stream));
+    }
+    return record(launch_bwd_saved(a, io, carve_saved(const_cast<void*>(saved), R), ws, stream));
 }
 }  // namespace
 
@@ -512,5 +557,7 @@ extern "C" int entmax_attn_bwd_noalloc(const void* Q, const void* K, const void*
     if (rc) return rc;
     AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), H, 0.5f, 0};
     BwdIO io{tau, dO, dQ, dK, dV, scratch};
-    return record(launch_bwd(a, io, stream));
+    // the tensor-core kernels store gradient rows 16 bytes at a time
+    const bool dense = dense_bwd(a) && aligned(dQ, 16) && aligned(dK, 16) && aligned(dV, 16);
+    return record(dense ? launch_bwd_dense(a, io, stream) : launch_bwd(a, io, stream));
 }

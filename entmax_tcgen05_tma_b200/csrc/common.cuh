@@ -53,19 +53,27 @@ static __device__ __noinline__ void raise_timeout(int* abort_flag, const WaitCfg
     if (wc.status) atomicExch(wc.status, STATUS_TIMEOUT);
 }
 
-constexpr uint32_t POLL_SUSPEND_NS = 256;  // longest suspension inside one poll of a bounded wait
+constexpr uint32_t POLL_SUSPEND_NS = 1000;  // longest suspension inside one poll of a wait
 
 // Bounded wait on an mbarrier phase.  Returns false if the CTA aborted (this wait timed out,
-// or another role already raised the abort flag).  Each poll after the first suspends the thread
-// for at most POLL_SUSPEND_NS, and the abort flag and the clock are checked after every failed
-// poll, so a wait gives up within about POLL_SUSPEND_NS of its bound.
+// or another role already raised the abort flag).  After a first non-suspending test the thread
+// waits inside mbarrier.try_wait, suspended (taking no issue slots from the warps that work) until
+// the phase completes or POLL_SUSPEND_NS pass, and checks the abort flag and the elapsed time
+// after every poll that returns without the phase.
+// Elapsed time: the global timer, or half the SM cycles elapsed if that is larger (the SM clock
+// runs below 2 GHz, so cycles / 2 never overstates the nanoseconds), since the global timer may
+// advance in steps coarser than a short bound.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, int* abort_flag, const WaitCfg& wc) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    const long long c0 = clock64();
+    // a bound shorter than a few polls gets short polls, so it is seen
+    const uint32_t hint = wc.timeout_ns < 4ull * POLL_SUSPEND_NS ? 20u : POLL_SUSPEND_NS;
     for (;;) {
-        if (mbar_try_wait_hint(bar, parity, POLL_SUSPEND_NS)) return true;
+        if (mbar_try_wait_hint(bar, parity, hint)) return true;
         if (flag_set(abort_flag)) return false;
-        if (globaltimer_ns() - t0 > wc.timeout_ns) {
+        const uint64_t dt = globaltimer_ns() - t0, dc = (uint64_t)(clock64() - c0) >> 1;
+        if ((dt > dc ? dt : dc) > wc.timeout_ns) {
             raise_timeout(abort_flag, wc);
             return false;
         }
@@ -412,6 +420,59 @@ __device__ __forceinline__ float pow_pos(float b, float e) {
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(b));
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(e * l));
     return b > 0.f ? r : 0.f;
+}
+
+// ------------------------------------------------------------ packed fp32 pairs (sm_100 f32x2)
+// Two fp32 values in one 64-bit register pair: lane x in the low half, y in the high half.  The
+// f32x2 arithmetic instructions round each lane as their scalar forms do.
+__device__ __forceinline__ uint64_t f2pack(float x, float y) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& x, float& y) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// max(v, 0) lane by lane
+__device__ __forceinline__ uint64_t f2relu(uint64_t v) {
+    float x, y;
+    f2unpack(v, x, y);
+    return f2pack(fmaxf(x, 0.f), fmaxf(y, 0.f));
+}
+
+// A pair of fp32 values as two bf16 pairs hi + lo (x = hi + lo to about 16 significant bits): hi
+// keeps each value's top 16 bits (truncation, exact in fp32), lo = bf16(x - hi) rounded to nearest
+// even.  Lane x goes to the low bf16 of each word, lane y to the high one.
+__device__ __forceinline__ void f2split(uint64_t v, uint32_t& hi, uint32_t& lo) {
+    float x, y;
+    f2unpack(v, x, y);
+    const uint32_t xt = __float_as_uint(x) & 0xffff0000u, yt = __float_as_uint(y) & 0xffff0000u;
+    hi = __byte_perm(xt, yt, 0x7632);  // {x_hi16, y_hi16}
+    const uint64_t r = f2sub(v, f2pack(__uint_as_float(xt), __uint_as_float(yt)));
+    float rx, ry;
+    f2unpack(r, rx, ry);
+    __nv_bfloat162 b = __floats2bfloat162_rn(rx, ry);
+    lo = *reinterpret_cast<uint32_t*>(&b);
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

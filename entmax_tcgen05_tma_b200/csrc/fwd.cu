@@ -372,7 +372,7 @@ __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float w, const uint4
     }
 }
 
-// Writes row r's support (both partitions, p_ij in cv; b_ij for general alpha) to the saved lists as
+// Writes row r's support (both partitions, h_ij = sqrt(p_ij) in cv; b_ij for general alpha) to the saved lists as
 // (j, b_ij), b_ij = am1 (S_ij - tau_i) scaled (= sqrt(p_ij) at alpha 1.5), and
 // counts each key once per row that holds it.  Run by the row's two threads (h = 0, 1) after phase 2;
 // rows redone on CUDA cores (mode 2) or with more than SAVE_CAP entries are marked unsaved.
@@ -397,8 +397,8 @@ __device__ __forceinline__ void save_row_support(const SavedSupport& sv, const f
     for (int e = 0; e < n; ++e) {
         const int j = cj[(slot0 + e) * TILE + r];
         sv.row_j[row * SAVE_CAP + base + e] = (uint16_t)j;
-        const float c = cv[(slot0 + e) * TILE + r];  // p (alpha 1.5) or b = am1 (x - tau) (generic)
-        sv.row_sp[row * SAVE_CAP + base + e] = GEN ? c : sqrtf(c);
+        // h = sqrt(p) (alpha 1.5) or b = am1 (x - tau) (generic): saved as is
+        sv.row_sp[row * SAVE_CAP + base + e] = cv[(slot0 + e) * TILE + r];
         atomicAdd(sv.key_cnt + key_row0 + j, 1);
     }
 }
@@ -446,7 +446,7 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
                                           const __nv_bfloat16* __restrict__ V, const uint32_t* bits, float* sbuf,
                                           float* red, HeadRef hq, HeadRef hkv, int bh, int i, int L,
                                           int causal, int window, float scale, float am1, int nallow, void* O,
-                                          int out_f32, float* tau) {
+                                          int out_f32, float* tau, float* otil, float* rsum) {
     const int tid = threadIdx.x;
     float* qf = red + 64;  // 64 floats (red[0..63] holds reduction partials)
     __syncthreads();
@@ -592,21 +592,26 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
     } else {
         t = 0.5f * (blo + bhi);
     }
-    // O_i: thread -> (dimension d, key phase ph)
+    // O_i (and, alpha 1.5 with otil, Otil_i = sum h_ij V_j and r_i = sum h_ij): thread -> (dimension d,
+    // key phase ph)
     constexpr int PH = NUM_THREADS / HEAD_DIM;
     const int d = tid % HEAD_DIM, ph = tid / HEAD_DIM;
-    float acc = 0.f;
+    const bool aux = !GEN && otil != nullptr;
+    float acc = 0.f, acc2 = 0.f, hsum = 0.f;
     for (int e = ph; e < span; e += PH) {
         const float s = unit(sbuf[e]);
         if (s > t) {
-            float p;
+            float p, hv = 0.f;
             if (GEN) {
                 p = pow_pos(s - t, ex);
             } else {
-                const float h = 0.5f * (s - t);
-                p = h * h;
+                hv = 0.5f * (s - t);
+                p = hv * hv;
             }
-            acc = fmaf(p, __bfloat162float(V[hkv.row(lo + e) * HEAD_DIM + d]), acc);
+            const float v = __bfloat162float(V[hkv.row(lo + e) * HEAD_DIM + d]);
+            acc = fmaf(p, v, acc);
+            acc2 = fmaf(hv, v, acc2);
+            hsum += hv;
         }
     }
     __syncthreads();
@@ -620,6 +625,27 @@ __device__ __noinline__ void fallback_row(const __nv_bfloat16* __restrict__ Q, c
         if (out_f32) reinterpret_cast<float*>(O)[oi] = o;
         else reinterpret_cast<__nv_bfloat16*>(O)[oi] = __float2bfloat16_rn(o);
         if (tid == 0) tau[(size_t)bh * L + i] = GEN ? m + t * ex : t;
+    }
+    if (aux) {  // uniform across the CTA
+        __syncthreads();
+        red[tid] = acc2;
+        __syncthreads();
+        if (tid < HEAD_DIM) {
+            float o = 0.f;
+#pragma unroll
+            for (int p = 0; p < PH; ++p) o += red[tid + p * HEAD_DIM];
+            otil[((size_t)bh * L + i) * HEAD_DIM + tid] = o;
+        }
+        // every (dimension, phase) thread summed h over its phase's keys: the d = 0 threads hold r_i
+        __syncthreads();
+        red[tid] = d == 0 ? hsum : 0.f;
+        __syncthreads();
+        if (tid == 0) {
+            float rs = 0.f;
+#pragma unroll
+            for (int p = 0; p < PH; ++p) rs += red[p * HEAD_DIM];
+            rsum[(size_t)bh * L + i] = rs;
+        }
     }
     __syncthreads();
 }
@@ -991,8 +1017,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
             }
         }
         if (mode == 0) {
-            // this thread's partition of the support: cv <- p_ij (alpha 1.5) or b_ij = y - t (general
-            // alpha; p = b^ex), cj <- j (in place)
+            // this thread's partition of the support: cv <- h_ij = sqrt(p_ij) (alpha 1.5) or
+            // b_ij = y - t (general alpha; p = b^ex), cj <- j (in place)
             int sn = 0;
             auto keep = [&](float c, uint16_t j) {
                 const float xv = fmaf(scale, c, -ms);
@@ -1005,7 +1031,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     }
                 } else if (xv > tau_x) {
                     const float hh = 0.5f * (xv - tau_x);
-                    pcv[sn * TILE + r] = hh * hh;
+                    pcv[sn * TILE + r] = hh;  // h = sqrt(p)
                     pcj[sn * TILE + r] = j;
                     ++sn;
                 }
@@ -1055,7 +1081,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         const int sl = ee < n0 ? ee : CAPW + (ee - n0);
                         const int j = cj[sl * TILE + r];
                         const float c = cv[sl * TILE + r];
-                        pw[u] = e + u < ns ? (GEN ? pow_pos(c, ex) : c) : 0.f;
+                        pw[u] = e + u < ns ? (GEN ? pow_pos(c, ex) : c * c) : 0.f;
                         // 128-byte swizzled V block in ring slot vslot[j / BLK]: 16-byte chunk q of
                         // row `row` sits at chunk position q ^ (row & 7)
                         const uint32_t row = (uint32_t)j & (BLK - 1);
@@ -1080,7 +1106,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         const int ee = e + u < ns ? e + u : e;
                         const int sl = ee < n0 ? ee : CAPW + (ee - n0);
                         const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)cj[sl * TILE + r] * vstep) + 4 * h;
-                        pw[u] = e + u < ns ? (GEN ? pow_pos(cv[sl * TILE + r], ex) : cv[sl * TILE + r]) : 0.f;
+                        const float c = cv[sl * TILE + r];
+                        pw[u] = e + u < ns ? (GEN ? pow_pos(c, ex) : c * c) : 0.f;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) x[u][c] = __ldg(src + c);
                     }
@@ -1108,6 +1135,43 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                     dst[c] = *reinterpret_cast<const uint4*>(hv);
                 }
             }
+            if (!GEN && out.otil) {
+                // auxiliary row (alpha 1.5): Otil_i = sum_j h_ij V_j and r_i = sum_j h_ij over the same
+                // support, in a second walk over it (the V rows are hot)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) acc[c][k] = 0.f;
+                float rs = 0.f;
+                for (int e = 0; e < ns; ++e) {
+                    const int sl = e < n0 ? e : CAPW + (e - n0);
+                    const int j = cj[sl * TILE + r];
+                    const float w = cv[sl * TILE + r];
+                    rs += w;
+                    uint4 x[4];
+                    if (v_staged) {
+                        const uint32_t row = (uint32_t)j & (BLK - 1);
+                        const uint8_t* base = smem_b + vslot[j / BLK] * BLK_BYTES + row * 128u;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            x[q] = *reinterpret_cast<const uint4*>(base + ((((uint32_t)(4 * h + q)) ^ (row & 7u)) << 4));
+                    } else {
+                        const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)j * vstep) + 4 * h;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) x[q] = __ldg(src + q);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) fma_bf16x8(acc[q], w, x[q]);
+                }
+                const size_t row = (size_t)bh * L + i;
+                float4* dst = reinterpret_cast<float4*>(out.otil + row * HEAD_DIM + 32 * h);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    dst[2 * c] = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+                    dst[2 * c + 1] = make_float4(acc[c][4], acc[c][5], acc[c][6], acc[c][7]);
+                }
+                if (h == 0) out.rsum[row] = rs;
+            }
         }
     }
     __syncthreads();
@@ -1125,7 +1189,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                                   reinterpret_cast<const __nv_bfloat16*>(args.K),
                                   reinterpret_cast<const __nv_bfloat16*>(args.V), bits, scratch, red, hq, hkv, bh,
                                   i0 + rr, L, args.causal, args.window, scale, am1,
-                                  rows[rr].nallow + rows[TILE + rr].nallow, out.O, out.out_f32, out.tau);
+                                  rows[rr].nallow + rows[TILE + rr].nallow, out.O, out.out_f32, out.tau,
+                                  out.otil, out.rsum);
             }
         }
     }

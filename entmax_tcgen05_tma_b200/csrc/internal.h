@@ -63,6 +63,8 @@ struct FwdOut {
     int out_f32;
     float* tau;              // [B,H,L]
     SavedSupport save;       // row_cnt == nullptr: nothing saved
+    float* otil;             // optional (alpha 1.5): [B*H*L][64] sum_j sqrt(p_ij) V_j, logical row order
+    float* rsum;             // optional with otil: [B*H*L] sum_j sqrt(p_ij)
 };
 
 // Carves a caller buffer of entmax_attn_saved_bytes() into its arrays.
@@ -78,6 +80,8 @@ struct BwdIO {
     float* dK;
     float* dV;
     float* u;                // workspace [B,H,L]: u_i = sum_j sqrt(p_ij) dA_ij / sum_j sqrt(p_ij)
+    const float* otil;       // optional [B*H*L][64]: the forward's sum_j sqrt(p_ij) V_j (logical row order)
+    const float* rsum;       // optional [B*H*L]: the forward's sum_j sqrt(p_ij); with otil, u_i = dO_i . otil_i / rsum_i
 };
 
 // Workspace of the support-list backward.
@@ -98,6 +102,17 @@ cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B,
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
 cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
+
+// The tensor-core backward (bwd_dense.cu) serves rows whose allowed keys span few key blocks:
+// sequences of at most 512 keys, or causal windows of at most 128 keys.  There a 128 x 64 tile of
+// (query, key) pairs costs less as tcgen05 products than as gathers over its support.  alpha 1.5
+// only.  Every backward entry point dispatches on this, and the training forward saves no support
+// lists when it holds (the tensor-core backward does not read them).
+__host__ __device__ __forceinline__ bool dense_bwd(const AttnArgs& a) {
+    return a.am1 == 0.5f && (a.L <= 512 || (a.causal && a.window > 0 && a.window <= 128));
+}
+// dq kernel (writes io.u, one float per query row, and dQ), then dkdv kernel (dK, dV).
+cudaError_t launch_bwd_dense(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, cudaStream_t stream);
 
 // Raises a kernel's dynamic shared-memory limit once per (kernel slot, device).
@@ -106,5 +121,7 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, int slot);
 size_t fwd_smem_bytes();
 size_t bwd_rows_smem_bytes();
 size_t bwd_keys_smem_bytes();
+size_t dense_dq_smem_bytes();
+size_t dense_dkdv_smem_bytes();
 
 }  // namespace entmax

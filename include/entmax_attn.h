@@ -126,6 +126,34 @@ ENTMAX_API int entmax_attn_bwd(const void* Q, const void* K, const void* V, int 
                     void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Auxiliary rows of the forward pass, for the backward's row scalar (page "svd-sst2-roberta-adasplash",
+ * section 2.4: u_i = sum_j sqrt(A_ij) dA_ij / sum_j sqrt(A_ij) with dA_ij = dO_i . V_j; since dA is
+ * linear in V, u_i = dO_i . Otil_i / r_i).  entmax_attn_fwd_aux computes exactly what entmax_attn_fwd
+ * computes and also, for every query row,
+ *   Otil   [B,H,L,D] fp32, Otil_i = sum_j sqrt(A_ij) V_j, rows in [B,H,L] order, 16-byte aligned,
+ *   rsum   [B,H,L] fp32,   r_i = sum_j sqrt(A_ij)  (0 for a row with no allowed key),
+ * both caller-owned device buffers, fully written.  entmax_attn_bwd_aux computes exactly what
+ * entmax_attn_bwd computes, taking u_i from these rows instead of deriving it: on the tensor-core
+ * configurations (L <= 512, or a causal window of at most 128 keys) that removes a pass over the
+ * scores.  Elsewhere the rows are checked but not needed (the support gathers form u_i on the way).
+ *   Otil, rsum   from entmax_attn_fwd_aux with the same Q, K, V, masks and scale.
+ *   workspace    as for entmax_attn_bwd (entmax_attn_bwd_workspace_size bytes).
+ * Other arguments and errors: as entmax_attn_fwd / entmax_attn_bwd; a null or misaligned Otil or rsum
+ * returns ENTMAX_ERR_ARG.
+ */
+ENTMAX_API int entmax_attn_fwd_aux(const void* Q, const void* K, const void* V, int in_dtype,
+                                   const uint8_t* key_mask, int causal, int window, float scale,
+                                   int B, int H, int L, int D,
+                                   void* O, int out_dtype, float* tau, float* Otil, float* rsum,
+                                   cudaStream_t stream);
+ENTMAX_API int entmax_attn_bwd_aux(const void* Q, const void* K, const void* V, int in_dtype,
+                                   const uint8_t* key_mask, int causal, int window, float scale,
+                                   int B, int H, int L, int D,
+                                   const float* tau, const float* Otil, const float* rsum, const void* dO,
+                                   float* dQ, float* dK, float* dV,
+                                   void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Training path.  entmax_attn_fwd_train computes exactly what entmax_attn_fwd computes and also saves
  * each row's support {(j, sqrt(A_ij)) : A_ij > 0} (up to 64 entries per row; rows with more, and rows
  * the forward had to redo exactly on CUDA cores, are marked and recomputed by the backward) plus, per
@@ -139,8 +167,10 @@ ENTMAX_API int entmax_attn_bwd(const void* Q, const void* K, const void* V, int 
  *   workspace  device buffer of entmax_attn_bwd_saved_workspace_size(B,H,L,D) bytes, 256-byte aligned.
  *   O (training forward) and dQ, dK, dV (this backward): 16-byte aligned (16-byte stores); the
  *   other arguments as in entmax_attn_fwd / entmax_attn_bwd.
- * dK and dV are summed in an order that depends on scheduling (last-bit differences between runs);
- * dQ, O and tau are deterministic.
+ * On the tensor-core configurations (L <= 512, or a causal window of at most 128 keys, at alpha 1.5)
+ * the backward recomputes the scores on tcgen05 and reads nothing from `saved` but its size; every
+ * output is then the same bit for bit from run to run.  Elsewhere dK and dV are summed in an order
+ * that depends on scheduling (last-bit differences between runs); dQ, O and tau are deterministic.
  */
 ENTMAX_API size_t entmax_attn_saved_bytes(int B, int H, int L, int D);
 ENTMAX_API size_t entmax_attn_bwd_saved_workspace_size(int B, int H, int L, int D);

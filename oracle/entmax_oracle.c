@@ -364,6 +364,61 @@ void eo_attn_fwd_rows(const double* Q, const double* K, const double* V,
     }
 }
 
+/* Auxiliary rows of the backward's row scalar (page "svd-sst2-roberta-adasplash", section 2.4, the   */
+/* closed-form Jacobian: u_i = sum_j sqrt(p_ij) dA_ij / sum_j sqrt(p_ij)), alpha = 1.5: for each listed   */
+/* row, Otil_i = sum_j sqrt(p_ij) V_j and r_i = sum_j sqrt(p_ij), with p from the exact tau (sort).       */
+/* Otil_rows is [nrows, D], r_rows [nrows]; a row with no allowed key gets zeros.                       */
+void eo_attn_aux_rows(const double* Q, const double* K, const double* V,
+                      const unsigned char* key_mask, int causal, int window, double scale,
+                      int B, int H, int L, int D, const long long* row_ids, long long nrows,
+                      double* Otil_rows, double* r_rows)
+{
+    (void)B;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)L);
+        double* p = (double*)malloc(sizeof(double) * (size_t)L);
+        int* idx = (int*)malloc(sizeof(int) * (size_t)L);
+#pragma omp for schedule(dynamic, 16)
+        for (long long r = 0; r < nrows; ++r) {
+            long long id = row_ids[r];
+            int i = (int)(id % L);
+            long long bh = id / L;
+            int h = (int)(bh % H);
+            int b = (int)(bh / H);
+            const size_t head = ((size_t)b * H + h) * (size_t)L * D;
+            const double* q = Q + head + (size_t)i * D;
+            double* out = Otil_rows + (size_t)r * D;
+            int n = 0;
+            for (int j = 0; j < L; ++j) {
+                if (!allowed(key_mask, b, L, causal, window, i, j)) continue;
+                const double* k = K + head + (size_t)j * D;
+                double acc = 0.0;
+                for (int t = 0; t < D; ++t) acc += q[t] * k[t];
+                s[n] = scale * acc;
+                idx[n] = j;
+                ++n;
+            }
+            for (int t = 0; t < D; ++t) out[t] = 0.0;
+            r_rows[r] = 0.0;
+            if (n == 0) continue;
+            double tau;
+            eo_tau_sort(s, n, &tau);
+            eo_entmax15(s, n, tau, p);
+            for (int e = 0; e < n; ++e) {
+                if (p[e] == 0.0) continue;
+                const double w = sqrt(p[e]);
+                const double* v = V + head + (size_t)idx[e] * D;
+                for (int t = 0; t < D; ++t) out[t] += w * v[t];
+                r_rows[r] += w;
+            }
+        }
+        free(s);
+        free(p);
+        free(idx);
+    }
+}
+
 /* Full forward: O [B,H,L,D], tau [B,H,L]. */
 void eo_attn_fwd(const double* Q, const double* K, const double* V,
                  const unsigned char* key_mask, int causal, int window, double scale, double alpha,

@@ -72,6 +72,9 @@ def _load():
         lib.eo_attn_fwd.argtypes = [_dp, _dp, _dp, _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                     ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, _dp, _dp]
+        lib.eo_attn_aux_rows.argtypes = [_dp, _dp, _dp, _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i64p,
+                                         ctypes.c_longlong, _dp, _dp]
         lib.eo_attn_bwd_heads.argtypes = [_dp, _dp, _dp, _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                           ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           _dp, _i64p, ctypes.c_int, _dp, _dp, _dp]
@@ -242,6 +245,21 @@ def attn_fwd_rows(Q, K, V, row_ids, key_mask=None, causal=False, window=0, scale
                              _alpha_arg(alpha), B, H, L, D, ids.ctypes.data_as(_i64p), ids.size,
                              0 if tau_method == "sort" else 1, int(n_iter), _d(O), _d(tau))
     return O, tau
+
+
+def attn_aux_rows(Q, K, V, row_ids, key_mask=None, causal=False, window=0, scale=0.125):
+    """Auxiliary rows (1.5-entmax) of selected rows: Otil_i = sum_j sqrt(p_ij) V_j and
+    r_i = sum_j sqrt(p_ij), the factors of the backward's row scalar u_i = dO_i . Otil_i / r_i (page
+    "svd-sst2-roberta-adasplash", section 2.4).  Returns (Otil_rows [n, D], r_rows [n])."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    B, H, L, D = Q.shape
+    m, mp = _mask_arg(key_mask, B, L)
+    ids = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64))
+    Ot = np.empty((ids.size, D), dtype=np.float64)
+    r = np.empty((ids.size,), dtype=np.float64)
+    _load().eo_attn_aux_rows(_d(Q), _d(K), _d(V), mp, int(bool(causal)), int(window), float(scale), B, H, L, D,
+                             ids.ctypes.data_as(_i64p), ids.size, _d(Ot), _d(r))
+    return Ot, r
 
 
 def attn_bwd_heads(Q, K, V, dO, bh_ids, key_mask=None, causal=False, window=0, scale=0.125, alpha=1.5):

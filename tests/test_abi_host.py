@@ -113,6 +113,38 @@ def test_bwd_argument_checks(kw, code):
     assert _bwd(**kw) == code
 
 
+def _fwd_aux(**kw):
+    a = dict(Q=P, K=P, V=P, in_dtype=0, mask=None, causal=0, window=0, scale=0.125, B=1, H=1, L=64, D=64,
+             O=P, out_dtype=0, tau=P, Otil=P, rsum=P, stream=None)
+    a.update(kw)
+    return E.lib.entmax_attn_fwd_aux(a["Q"], a["K"], a["V"], a["in_dtype"], a["mask"], a["causal"], a["window"],
+                                     a["scale"], a["B"], a["H"], a["L"], a["D"], a["O"], a["out_dtype"], a["tau"],
+                                     a["Otil"], a["rsum"], a["stream"])
+
+
+def _bwd_aux(**kw):
+    a = dict(Q=P, K=P, V=P, in_dtype=0, mask=None, causal=0, window=0, scale=0.125, B=1, H=1, L=64, D=64, tau=P,
+             Otil=P, rsum=P, dO=P, dQ=P, dK=P, dV=P, ws=P, ws_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return E.lib.entmax_attn_bwd_aux(a["Q"], a["K"], a["V"], a["in_dtype"], a["mask"], a["causal"], a["window"],
+                                     a["scale"], a["B"], a["H"], a["L"], a["D"], a["tau"], a["Otil"], a["rsum"],
+                                     a["dO"], a["dQ"], a["dK"], a["dV"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("call", [_fwd_aux, _bwd_aux])
+@pytest.mark.parametrize("kw,code", [
+    (dict(Otil=None), E.ENTMAX_ERR_ARG),
+    (dict(rsum=None), E.ENTMAX_ERR_ARG),
+    (dict(Otil=P + 8), E.ENTMAX_ERR_ARG),
+    (dict(rsum=P + 2), E.ENTMAX_ERR_ARG),
+    (dict(D=32), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(window=8), E.ENTMAX_ERR_UNSUPPORTED),
+    (dict(B=0, Otil=None, rsum=None), E.ENTMAX_OK),
+])
+def test_aux_argument_checks(call, kw, code):
+    assert call(**kw) == code
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
 

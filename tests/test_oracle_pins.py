@@ -588,3 +588,83 @@ def test_alpha_attention_backward_matches_finite_differences(alpha):
         if done == 2:
             break
     assert done >= 1
+
+
+# ------------------------------------------------------- auxiliary rows
+def test_aux_rows_uniform_and_one_hot():
+    """Otil_i = sum_j sqrt(p_ij) V_j, r_i = sum_j sqrt(p_ij).  Q = 0: p = 1/n on the allowed keys, so
+    r = sqrt(n) and Otil = (sum of the allowed V rows) / sqrt(n).  A key far above the rest: p is
+    one-hot, r = 1 and Otil = that key's V row."""
+    B, H, L, D = 2, 2, 24, 8
+    _, K, V, _ = _rand_qkv(31, B, H, L, D)
+    Q = np.zeros_like(K)
+    mask = np.zeros((B, L), np.uint8)
+    mask[0, :24] = 1
+    mask[1, :9] = 1
+    ids = np.arange(B * H * L)
+    Ot, r = orc.attn_aux_rows(Q, K, V, ids, mask, scale=0.125)
+    for rid in ids:
+        b, h, i = rid // (H * L), (rid // L) % H, rid % L
+        n = int(mask[b].sum())
+        assert r[rid] == pytest.approx(math.sqrt(n), abs=1e-12)
+        np.testing.assert_allclose(Ot[rid], V[b, h, :n].sum(axis=0) / math.sqrt(n), atol=1e-12)
+    Q2 = np.zeros((1, 1, 8, 4))
+    K2 = np.zeros((1, 1, 8, 4))
+    V2 = np.arange(32, dtype=float).reshape(1, 1, 8, 4)
+    Q2[0, 0, :, 0] = 1.0
+    K2[0, 0, 3, 0] = 10.0
+    Ot2, r2 = orc.attn_aux_rows(Q2, K2, V2, np.arange(8), None, scale=1.0)
+    np.testing.assert_allclose(r2, 1.0, atol=1e-15)
+    np.testing.assert_allclose(Ot2, np.broadcast_to(V2[0, 0, 3], (8, 4)), atol=1e-15)
+    # a row with no allowed key
+    m0 = np.zeros((1, 8), np.uint8)
+    Ot3, r3 = orc.attn_aux_rows(Q2, K2, V2, [0, 5], m0, scale=1.0)
+    assert np.all(Ot3 == 0) and np.all(r3 == 0)
+
+
+def test_aux_rows_by_kkt_bruteforce():
+    """Tiny heads: tau of every row by enumerating supports (KKT), then sqrt(p) = (s - tau)/2 on the
+    support and the two sums written out."""
+    rng = np.random.default_rng(32)
+    for trial in range(20):
+        L, D = int(rng.integers(1, 5)), int(rng.integers(1, 5))
+        Q = rng.normal(0, 1.5, (1, 1, L, D))
+        K = rng.normal(0, 1.5, (1, 1, L, D))
+        V = rng.normal(0, 1.0, (1, 1, L, D))
+        Ot, r = orc.attn_aux_rows(Q, K, V, np.arange(L), None, scale=0.7)
+        for i in range(L):
+            s = 0.7 * (K[0, 0] @ Q[0, 0, i])
+            tau = _kkt_bruteforce(s)[0]
+            w = np.where(s > tau, (s - tau) / 2.0, 0.0)
+            assert r[i] == pytest.approx(w.sum(), abs=1e-10)
+            np.testing.assert_allclose(Ot[i], w @ V[0, 0], atol=1e-10)
+
+
+def test_aux_rows_give_the_score_gradient():
+    """The backward's row scalar from the auxiliary rows, u_i = dO_i . Otil_i / r_i, against central
+    finite differences of <dO_i, O_i> in the scores: on the support, d<dO_i, O_i>/ds_j =
+    sqrt(p_j) (dO_i . V_j - u_i) (section 2.4), so u_i = dO_i . V_j - (FD_j / sqrt(p_j))."""
+    rng = np.random.default_rng(33)
+    L, D = 12, 6
+    Q = rng.normal(0, 1.0, (1, 1, L, D))
+    K = rng.normal(0, 1.0, (1, 1, L, D))
+    V = rng.normal(0, 1.0, (1, 1, L, D))
+    dO = rng.normal(0, 1.0, (L, D))
+    scale = 1.3
+    Ot, r = orc.attn_aux_rows(Q, K, V, np.arange(L), None, scale=scale)
+    checked = 0
+    for i in range(L):
+        s = scale * (K[0, 0] @ Q[0, 0, i])
+        p = orc.entmax15(s)
+        u = dO[i] @ Ot[i] / r[i]
+        tau = orc.tau_sort(s)[0]
+        if np.min(np.abs(s - tau)) < 1e-3:
+            continue  # a kink: skip
+        h = 1e-6
+        for j in np.nonzero(p > 0)[0]:
+            e = np.zeros(L)
+            e[j] = h
+            fd = (dO[i] @ (orc.entmax15(s + e) @ V[0, 0]) - dO[i] @ (orc.entmax15(s - e) @ V[0, 0])) / (2 * h)
+            assert dO[i] @ V[0, 0, j] - fd / math.sqrt(p[j]) == pytest.approx(u, abs=1e-5)
+            checked += 1
+    assert checked > 10
