@@ -17,6 +17,9 @@
  *   backward: closed-form Jacobian of section 2.4,
  *     dL/dS_j = 1[j in S] sqrt(p_j) (g_j - sum_k sqrt(p_k) g_k / sum_k sqrt(p_k))
  *
+ * alpha = 1 is softmax (the pages' branch for |alpha - 1| < 1e-4 in the same
+ * routine): p_ij = exp(S_ij - tau_i), tau_i = log sum_j exp(S_ij).
+ *
  * General alpha in (1, 2] (the pages' alpha-entmax by bisection, page
  * "svd-sst2-roberta-adasplash", section 4, the entmax_bisect routine): with
  * a = alpha - 1, p_ij = max(0, a (S_ij - tau_i))^(1/a), sum_j p_ij = 1 (tau in
@@ -271,10 +274,38 @@ void eo_entmax_alpha_jvp(const double* p, const double* g, int n, double alpha, 
     for (int j = 0; j < n; ++j) ds[j] = p[j] > 0.0 ? pow(p[j], 2.0 - alpha) * (g[j] - u) : 0.0;
 }
 
-/* tau and p of one row for any alpha: the closed form (alpha = 1.5, sort)  */
-/* or the converged bisection; tau_method 1 = the pages' n_iter halvings.   */
+/* ------------------------------------------------------------------------ */
+/* alpha = 1: softmax.  The pages' alpha-entmax routine takes this branch     */
+/* when |alpha - 1| < 1e-4 (page "svd-sst2-roberta-adasplash", section 4,     */
+/* entmax_bisect), and it is the alpha -> 1 limit of alpha-entmax.           */
+/*   p_i = exp(s_i - tau),  tau = log sum_k exp(s_k),                        */
+/* so tau plays the threshold's role (p = exp(s - tau) sums to 1).  tau is   */
+/* written as m + log sum_k exp(s_k - m), m = max_k s_k, so that no term     */
+/* overflows.  The Jacobian is the alpha-entmax one with w = p^(2-1) = p:    */
+/* ds_j = p_j (g_j - sum_k p_k g_k), which eo_entmax_alpha_jvp computes at   */
+/* alpha = 1 (there sum_k w_k = 1).                                          */
+/* ------------------------------------------------------------------------ */
+double eo_tau_softmax(const double* s, int n)
+{
+    if (n <= 0) return INFINITY;
+    double m = s[0];
+    for (int i = 1; i < n; ++i) if (s[i] > m) m = s[i];
+    double acc = 0.0;
+    for (int i = 0; i < n; ++i) acc += exp(s[i] - m);
+    return m + log(acc);
+}
+
+void eo_softmax(const double* s, int n, double tau, double* p)
+{
+    for (int i = 0; i < n; ++i) p[i] = exp(s[i] - tau);
+}
+
+/* tau and p of one row for any alpha: softmax (alpha = 1), the closed form */
+/* (alpha = 1.5, sort) or the converged bisection; tau_method 1 = the pages' */
+/* n_iter halvings (alpha > 1).                                             */
 static double row_tau(const double* s, int n, double alpha, int tau_method, int n_iter)
 {
+    if (alpha == 1.0) return eo_tau_softmax(s, n);
     if (alpha == 1.5) {
         double tau;
         if (tau_method == 0) eo_tau_sort(s, n, &tau);
@@ -287,7 +318,8 @@ static double row_tau(const double* s, int n, double alpha, int tau_method, int 
 
 static void row_probs(const double* s, int n, double tau, double alpha, double* p)
 {
-    if (alpha == 1.5) eo_entmax15(s, n, tau, p);
+    if (alpha == 1.0) eo_softmax(s, n, tau, p);
+    else if (alpha == 1.5) eo_entmax15(s, n, tau, p);
     else eo_entmax_alpha(s, n, tau, alpha, p);
 }
 

@@ -86,6 +86,9 @@ def _load():
         lib.eo_tau_alpha_bisect.argtypes = [_dp, ctypes.c_int, ctypes.c_double, ctypes.c_int]
         lib.eo_entmax_alpha.argtypes = [_dp, ctypes.c_int, ctypes.c_double, ctypes.c_double, _dp]
         lib.eo_entmax_alpha_jvp.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_double, _dp]
+        lib.eo_tau_softmax.restype = ctypes.c_double
+        lib.eo_tau_softmax.argtypes = [_dp, ctypes.c_int]
+        lib.eo_softmax.argtypes = [_dp, ctypes.c_int, ctypes.c_double, _dp]
         lib.eo_num_threads.restype = ctypes.c_int
         lib.eo_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -203,8 +206,25 @@ def entmax_alpha_jvp(p, gvec, alpha: float) -> np.ndarray:
     return ds
 
 
+def tau_softmax(s) -> float:
+    """alpha = 1 (softmax): tau = log sum_k exp(s_k), so that p = exp(s - tau) sums to 1 (the pages'
+    branch for |alpha - 1| < 1e-4, page "svd-sst2-roberta-adasplash", section 4, entmax_bisect)."""
+    s = _f64(s)
+    return _load().eo_tau_softmax(_d(s), s.size)
+
+
+def softmax(s, tau: float | None = None) -> np.ndarray:
+    """p = exp(s - tau), tau from tau_softmax unless given."""
+    s = _f64(s)
+    if tau is None:
+        tau = tau_softmax(s)
+    p = np.empty_like(s)
+    _load().eo_softmax(_d(s), s.size, float(tau), _d(p))
+    return p
+
+
 # --------------------------------------------------------------------------
-# attention (alpha = 1.5 unless given; other alpha in (1, 2] use tau_alpha)
+# attention (alpha = 1.5 unless given; other alpha in (1, 2] use tau_alpha, alpha = 1 is softmax)
 # --------------------------------------------------------------------------
 def _mask_arg(key_mask, B, L):
     if key_mask is None:
@@ -215,8 +235,8 @@ def _mask_arg(key_mask, B, L):
 
 def _alpha_arg(alpha) -> float:
     a = float(alpha)
-    if not (1.0 < a <= 2.0):
-        raise ValueError("alpha must lie in (1, 2], got %r" % alpha)
+    if not (a == 1.0 or 1.0 < a <= 2.0):
+        raise ValueError("alpha must be 1 (softmax) or lie in (1, 2], got %r" % alpha)
     return a
 
 

@@ -590,6 +590,133 @@ def test_alpha_attention_backward_matches_finite_differences(alpha):
     assert done >= 1
 
 
+# ------------------------------------------------------------ alpha = 1 (softmax)
+# The pages' alpha-entmax routine returns softmax when |alpha - 1| < 1e-4 (page
+# "svd-sst2-roberta-adasplash", section 4, entmax_bisect): p = exp(s - tau), tau = log sum exp(s).
+def test_softmax_closed_forms():
+    # n equal scores c: p = 1/n, tau = c + log n
+    for n, c in ((1, 0.3), (5, -2.0), (64, 7.5)):
+        s = np.full(n, c)
+        assert orc.tau_softmax(s) == pytest.approx(c + math.log(n), abs=1e-13)
+        np.testing.assert_allclose(orc.softmax(s), np.full(n, 1.0 / n), atol=1e-14)
+    # two scores: the logistic function of their gap
+    for a, b in ((0.0, 1.0), (3.0, -2.5), (1000.0, 999.0)):
+        s = np.array([a, b])
+        assert orc.softmax(s)[0] == pytest.approx(1.0 / (1.0 + math.exp(b - a)), abs=1e-13)
+        assert orc.tau_softmax(s) == pytest.approx(max(a, b) + math.log1p(math.exp(-abs(a - b))), abs=1e-12)
+    # a shift moves tau by the same amount and leaves p alone
+    for s in _rows(51, 40, nmin=1, nmax=30):
+        assert orc.tau_softmax(s + 4.25) == pytest.approx(orc.tau_softmax(s) + 4.25, abs=1e-12)
+        np.testing.assert_allclose(orc.softmax(s + 4.25), orc.softmax(s), atol=1e-14)
+    assert orc.tau_softmax(np.array([])) == math.inf
+
+
+def test_softmax_is_the_gibbs_argmax():
+    """softmax(s) = argmax over the simplex of p.s - sum p log p, and the maximum is log sum exp(s)
+    (the alpha -> 1 member of the entropy family whose alpha = 1.5 case is section 2.1)."""
+    rng = np.random.default_rng(52)
+    for _ in range(12):
+        n = int(rng.integers(2, 8))
+        s = rng.normal(0, 1.5, size=n)
+
+        def neg(p):
+            q = np.clip(p, 1e-300, None)
+            return -(p @ s - np.sum(q * np.log(q)))
+
+        cons = ({"type": "eq", "fun": lambda p: np.sum(p) - 1.0},)
+        res = optimize.minimize(neg, np.full(n, 1.0 / n), method="SLSQP", bounds=[(0.0, 1.0)] * n,
+                                constraints=cons, options={"ftol": 1e-14, "maxiter": 500})
+        np.testing.assert_allclose(orc.softmax(s), res.x, atol=2e-4)
+        assert -res.fun == pytest.approx(orc.tau_softmax(s), abs=1e-8)
+
+
+def test_softmax_is_the_alpha_one_limit():
+    """alpha-entmax (pinned on its own above) tends to softmax as alpha -> 1+, the gap shrinking with
+    alpha - 1."""
+    for s in _rows(53, 10, nmin=2, nmax=12, spread=(0.3, 1.5)):
+        sm = orc.softmax(s)
+        errs = [np.max(np.abs(orc.entmax_alpha(s, 1.0 + e) - sm)) for e in (1e-1, 1e-2, 1e-3)]
+        assert errs[0] > errs[1] > errs[2] and errs[2] < 2e-3
+
+
+def test_softmax_jvp_matches_finite_differences():
+    """The Jacobian-vector product at alpha = 1 (w = p) against central differences of softmax."""
+    rng = np.random.default_rng(54)
+    for _ in range(20):
+        n = int(rng.integers(1, 10))
+        s = rng.normal(0, 2.0, size=n)
+        gv = rng.normal(size=n)
+        h = 1e-6
+        J = np.empty((n, n))
+        for j in range(n):
+            e = np.zeros(n)
+            e[j] = h
+            J[:, j] = (orc.softmax(s + e) - orc.softmax(s - e)) / (2 * h)
+        ds = orc.entmax_alpha_jvp(orc.softmax(s), gv, 1.0)
+        np.testing.assert_allclose(ds, J.T @ gv, atol=2e-8)
+
+
+def test_softmax_attention_special_cases():
+    """alpha = 1 attention: Q = 0 gives every allowed key weight 1/n (O = mean of the allowed V rows,
+    tau = log n); causal row 0 sees key 0 alone (O = V_0, tau = S_00); a fully padded batch gives
+    O = 0, tau = +inf; one key far above the rest takes all the weight."""
+    B, H, L, D = 2, 2, 20, 8
+    _, K, V, _ = _rand_qkv(55, B, H, L, D)
+    Q = np.zeros_like(K)
+    mask = np.ones((B, L), np.uint8)
+    mask[1, 13:] = 0
+    mask[1, 2] = 0
+    O, tau = orc.attn_fwd(Q, K, V, mask, False, 0, 0.125, alpha=1.0)
+    for b in range(B):
+        keep = mask[b].astype(bool)
+        for h in range(H):
+            np.testing.assert_allclose(O[b, h], np.broadcast_to(V[b, h][keep].mean(0), (L, D)), atol=1e-13)
+            np.testing.assert_allclose(tau[b, h], math.log(keep.sum()), atol=1e-13)
+    Q, K, V, _ = _rand_qkv(56, B, H, L, D)
+    O, tau = orc.attn_fwd(Q, K, V, None, True, 0, 0.3, alpha=1.0)
+    np.testing.assert_allclose(O[:, :, 0], V[:, :, 0], atol=1e-13)
+    np.testing.assert_allclose(tau[:, :, 0], 0.3 * np.einsum("bhd,bhd->bh", Q[:, :, 0], K[:, :, 0]), atol=1e-12)
+    mask = np.ones((B, L), np.uint8)
+    mask[0] = 0
+    O, tau = orc.attn_fwd(Q, K, V, mask, False, 0, 0.3, alpha=1.0)
+    assert np.all(O[0] == 0) and np.all(np.isinf(tau[0]))
+    # key 5 aligned with every query and far longer than the others
+    K2 = K.copy()
+    K2[:, :, 5] = 60.0 * Q.mean(axis=2)
+    O, _ = orc.attn_fwd(Q, K2, V, None, False, 0, 1.0, alpha=1.0)
+    S = np.einsum("bhid,bhjd->bhij", Q, K2)
+    gap = S[:, :, :, 5] - np.delete(S, 5, axis=3).max(axis=3)
+    rows = gap > 40.0
+    assert rows.sum() > 10
+    err = np.abs(O - V[:, :, 5:6, :])[rows]
+    assert err.max() < 1e-12
+
+
+def test_softmax_attention_backward_matches_finite_differences():
+    """dQ, dK, dV at alpha = 1 against central differences of <dO, O>, with a causal window and a
+    padded key."""
+    B, H, L, D = 1, 2, 7, 4
+    scale = 0.7
+    Q, K, V, dO = _rand_qkv(57, B, H, L, D)
+    mask = np.ones((B, L), np.uint8)
+    mask[0, 3] = 0
+    args = (mask, True, 4, scale)
+    dQ, dK, dV = orc.attn_bwd(Q, K, V, dO, *args, alpha=1.0)
+    eps = 1e-6
+    for X, dX in ((Q, dQ), (K, dK), (V, dV)):
+        num = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            old = X[idx]
+            X[idx] = old + eps
+            Lp = np.sum(dO * orc.attn_fwd(Q, K, V, *args, alpha=1.0)[0])
+            X[idx] = old - eps
+            Lm = np.sum(dO * orc.attn_fwd(Q, K, V, *args, alpha=1.0)[0])
+            X[idx] = old
+            num[idx] = (Lp - Lm) / (2 * eps)
+        np.testing.assert_allclose(dX, num, atol=3e-7)
+    assert np.all(dK[0, :, 3] == 0) and np.all(dV[0, :, 3] == 0)
+
+
 # ------------------------------------------------------- auxiliary rows
 def test_aux_rows_uniform_and_one_hot():
     """Otil_i = sum_j sqrt(p_ij) V_j, r_i = sum_j sqrt(p_ij).  Q = 0: p = 1/n on the allowed keys, so
