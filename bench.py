@@ -274,11 +274,11 @@ class _Flush:
 class _Prepared:
     """Device-resident inputs, outputs and the step's library calls for one workload."""
 
-    def __init__(self, args, w: Workload, dev):
+    def __init__(self, args, w: Workload, dev, alpha: float | None = None):
         import entmax_tcgen05_tma_b200 as E
 
         self.E, self.w, self.dev = E, w, dev
-        alpha = args.alpha
+        alpha = args.alpha if alpha is None else alpha
         self.variant = variant = alpha != 1.5 or w.kv_heads != w.H or args.blhd  # the _ex entry points
         self.recompute = recompute = args.bwd == "recompute"  # entmax_attn_fwd + entmax_attn_bwd
         self.inp = inp = make_inputs(w)
@@ -333,9 +333,10 @@ class _Prepared:
 
 
 def tensor_core_backward(w: Workload, alpha: float = 1.5) -> bool:
-    """Whether the library runs the backward on its tensor-core kernels (dq, dkdv): alpha 1.5 with
-    L <= 512 or a causal window of at most 128 keys (the library's own dispatch rule)."""
-    return alpha == 1.5 and (w.L <= 512 or (w.causal and 0 < w.window <= 128))
+    """Whether the library runs the backward on its tensor-core kernels (dq, dkdv): softmax (alpha 1)
+    always, alpha 1.5 with L <= 512 or a causal window of at most 128 keys (the library's own
+    dispatch rule)."""
+    return alpha == 1.0 or (alpha == 1.5 and (w.L <= 512 or (w.causal and 0 < w.window <= 128)))
 
 
 def launches_per_step(w: Workload, recompute: bool, alpha: float = 1.5) -> int:
@@ -399,22 +400,33 @@ def step_roofline(w: Workload, km, flops: float, ms_per_step: float, peaks: dict
                                                                      peaks["source"])}
 
 
-def extra_workload(args, wid: int, dev, world: int, flush: _Flush, peaks: dict) -> dict:
+def extra_workload(args, w: Workload, dev, world: int, flush: _Flush, peaks: dict, alpha: float = 1.5) -> dict:
     """Another fwd+bwd workload timed in the same process and the same way as the headline line
     (same library calls, L2 eviction, events, warm-up and step count)."""
-    w = WORKLOADS[wid]
-    prep = _Prepared(args, w, dev)
+    prep = _Prepared(args, w, dev, alpha)
     t = time_device(prep, flush, args.steps, args.warmup, world)
     ms = t["total_ms"] / args.steps
-    sparsity = measured_sparsity(w, prep.Q, prep.K, prep.tau, prep.km)
-    out = {"workload": workload_desc(w), "steps": args.steps, "warmup": args.warmup,
+    # softmax keeps every allowed pair (no zeros to count)
+    sparsity = 0.0 if alpha == 1.0 else measured_sparsity(w, prep.Q, prep.K, prep.tau, prep.km)
+    out = {"workload": workload_desc(w), "alpha": alpha, "steps": args.steps, "warmup": args.warmup,
            "value": round(aggregate_value(prep.flops, world, ms), 3), "unit": "TFLOP/s",
            "ms_per_step": round(ms, 4), "fwd_ms": round(statistics.mean(t["fwd_ms"]), 4),
            "bwd_ms": round(statistics.mean(t["bwd_ms"]), 4) if w.backward else 0.0,
            "step_ms_median": round(statistics.median(t["step_ms"]), 4),
            "dense_equiv_gflop_per_step": prep.flops / 1e9, "allowed_pairs": prep.pairs,
            "sparsity": round(sparsity, 4), "step_roofline": step_roofline(w, prep.km, prep.flops, ms, peaks),
-           "gpu_launches": launches_per_step(w, prep.recompute, args.alpha) * args.steps, "clocks": t["clocks"]}
+           "gpu_launches": launches_per_step(w, prep.recompute, alpha) * args.steps, "clocks": t["clocks"]}
+    if alpha == 1.0:
+        # softmax forward kernel: its algorithmic work is the dense 4 d P of S = Q K^T and P V (every
+        # allowed pair is in the support); the tensor core issues 8 d P (S twice, P as two bf16 parts)
+        fwd_ms = statistics.mean(t["fwd_ms"])
+        alg = 4.0 * w.D * prep.pairs
+        out["roofline"] = {"kernel": "softmax_fwd_kernel", "bound": "tensor",
+                           "achieved": alg / (fwd_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                           "unit": "TFLOP/s", "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks["source"],
+                           "algorithmic_flops_per_launch": alg, "issued_mma_flops_per_launch": 2.0 * alg,
+                           "traffic": None}
+        out["roofline"]["frac"] = out["roofline"]["achieved"] / out["roofline"]["peak"]
     del prep
     torch.cuda.empty_cache()
     return out
@@ -542,14 +554,16 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     extras = {}
     if not args.no_extra and not variant and not recompute and args.workload == 4:
         peaks = load_peaks()
-        extras = {str(k): extra_workload(args, k, dev, world, flush, peaks) for k in (3, 5)}
+        extras = {str(k): extra_workload(args, WORKLOADS[k], dev, world, flush, peaks) for k in (3, 5)}
+        # softmax attention (alpha = 1, the pages' alpha -> 1 branch) on the headline shape
+        extras["softmax_4"] = extra_workload(args, WORKLOADS[4], dev, world, flush, peaks, alpha=1.0)
 
     if rank != 0:
         return None
 
     # ---- dominant kernel roofline (forward kernel: one launch per entmax_attn_fwd call)
     peaks = load_peaks()
-    sparsity = measured_sparsity(w, Q, K, tau, km)
+    sparsity = 0.0 if alpha == 1.0 else measured_sparsity(w, Q, K, tau, km)
     supp_pairs = (1.0 - sparsity) * pairs
     fwd_alg_flops = 2.0 * D * pairs + 2.0 * D * supp_pairs
     rows = B * H * L
@@ -557,7 +571,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     # saved support: a count and a (u16 key, fp32 sqrt p) pair per entry
     kv_rows = B * Hkv * L
     fwd_alg_bytes = rows * D * 2 + 2.0 * kv_rows * D * 2 + rows * D * 2 + rows * 4
-    if w.backward and not recompute:
+    if w.backward and not recompute and not tensor_core_backward(w, alpha):
         fwd_alg_bytes += rows * 4 + supp_pairs * 6
     fwd_mean = statistics.mean(fwd_ms)
     bwd_mean = statistics.mean(bwd_ms) if w.backward else 0.0
@@ -566,12 +580,13 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     # bf16 figure is its tensor peak
     t_tensor = fwd_alg_flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = fwd_alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    fwd_kernel = "softmax_fwd_kernel" if alpha == 1.0 else "entmax_fwd_kernel"
     if t_tensor >= t_hbm:
-        roof = {"kernel": "entmax_fwd_kernel", "bound": "tensor",
+        roof = {"kernel": fwd_kernel, "bound": "tensor",
                 "achieved": fwd_alg_flops / (fwd_mean * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks["source"]}
     else:
-        roof = {"kernel": "entmax_fwd_kernel", "bound": "hbm",
+        roof = {"kernel": fwd_kernel, "bound": "hbm",
                 "achieved": fwd_alg_bytes / (fwd_mean * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks["source"]}
     roof.update({"traffic": None, "algorithmic_flops_per_launch": fwd_alg_flops,
@@ -725,7 +740,7 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="time only the selected workload (the default workload-4 line also times 3 and 5)")
-    ap.add_argument("--alpha", type=float, default=1.5, help="alpha-entmax variant, alpha in (1, 2]")
+    ap.add_argument("--alpha", type=float, default=1.5, help="alpha-entmax variant, alpha in [1, 2] (1: softmax)")
     ap.add_argument("--hkv", type=int, default=0, help="grouped-query variant: key/value heads")
     ap.add_argument("--blhd", action="store_true", help="variant: tensors in [B, L, H, 64] memory")
     ap.add_argument("--bwd", default="saved", choices=["saved", "recompute"],

@@ -511,7 +511,8 @@ def entmax_attn_bwd_saved_gqa(Q, K, V, tau, saved, dO, key_mask=None, causal=Fal
 
 def entmax_attn_fwd_ex(Q, K, V, key_mask=None, causal=False, window=0, scale=None, alpha=1.5, save=False,
                        out_dtype=torch.bfloat16, O=None, tau=None, saved=None, stream=None):
-    """alpha-entmax forward, alpha in (1, 2]; K and V may have fewer heads than Q (H % H_kv == 0).
+    """alpha-entmax forward, alpha in [1, 2] (|alpha - 1| < 1e-4: softmax, tau = log sum exp of the
+    row's scores); K and V may have fewer heads than Q (H % H_kv == 0).
 
     Q, K, V are [B,H,L,64] tensors: contiguous, or all three the transpose(1, 2) views of contiguous
     [B,L,H,64] tensors (then O is returned in that layout too).  Returns (O, tau) or, with

@@ -29,6 +29,20 @@ int* g_status_ptr[MAX_DEVICES] = {};
 std::mutex g_mu;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+
+// Driver entry point `name` (version `ver`) through the runtime, once; under g_mu.
+template <class F>
+cudaError_t driver_fn(F* out, const char* name, int ver) {
+    if (*out) return cudaSuccess;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion(name, &fn, ver, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    *out = reinterpret_cast<F>(fn);
+    return cudaSuccess;
+}
 
 int record(cudaError_t e) {
     if (e == cudaSuccess) return ENTMAX_OK;
@@ -36,11 +50,30 @@ int record(cudaError_t e) {
     return ENTMAX_ERR_CUDA;
 }
 
+// The calling thread's device, with a context current on it.  The tensor-map encoder (a driver call
+// outside the runtime) needs a current context, and a host thread that has not used CUDA yet -- a new
+// thread, or a framework's autograd worker whose first CUDA work is a call here -- has none until
+// the runtime makes one current on its first stream operation.  So when no context is current, the
+// device's primary context is made current (cudaSetDevice); a context the caller made current is
+// left as it is.
+cudaError_t current_device(int* dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return e;
+    if (*dev < 0 || *dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        e = driver_fn(&g_ctx_current, "cuCtxGetCurrent", 4000);
+    }
+    if (e != cudaSuccess) return e;
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) == CUDA_SUCCESS && ctx) return cudaSuccess;
+    return cudaSetDevice(*dev);
+}
+
 cudaError_t status_ptr(int** out) {
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = current_device(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_status_ptr[dev]) {
         void* p = nullptr;
@@ -133,14 +166,8 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, int slot) {
 cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B, int nh, int L, int box_rows) {
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_encode) {
-            void* fn = nullptr;
-            cudaDriverEntryPointQueryResult q;
-            cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
-            if (e != cudaSuccess) return e;
-            if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
-            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-        }
+        cudaError_t e = driver_fn(&g_encode, "cuTensorMapEncodeTiled", 12000);
+        if (e != cudaSuccess) return e;
     }
     // layout 0 [B, nh, L, 64]: (d, L, B*nh); layout 1 [B, L, nh, 64]: (d, nh, B*L) -- see HeadRef
     const cuuint64_t row_bytes = (cuuint64_t)HEAD_DIM * 2;
@@ -152,7 +179,8 @@ cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B,
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+    if (r == CUDA_SUCCESS) return cudaSuccess;
+    return r == CUDA_ERROR_INVALID_CONTEXT ? cudaErrorDeviceUninitialized : cudaErrorInvalidValue;
 }
 
 }  // namespace entmax
@@ -209,11 +237,16 @@ int check_kv_heads(int H, int Hkv, int in_dtype) {
     return ENTMAX_OK;
 }
 
-// alpha of alpha-entmax: (1, 2].  alpha = 1 is softmax attention, which this library does not
-// compute (its supports are dense).
-int check_alpha(float alpha) {
-    if (alpha == 1.f) return ENTMAX_ERR_UNSUPPORTED;
+// alpha of alpha-entmax: [1, 2].  Like the pages' entmax_bisect routine (page
+// "svd-sst2-roberta-adasplash", section 4), |alpha - 1| < 1e-4 means softmax; am1 (alpha - 1) is then
+// exactly 0, the kernels' softmax flag.
+int check_alpha(float alpha, float* am1) {
+    if (fabsf(alpha - 1.f) < 1e-4f) {
+        *am1 = 0.f;
+        return ENTMAX_OK;
+    }
     if (!(alpha > 1.f && alpha <= 2.f)) return ENTMAX_ERR_ARG;
+    *am1 = alpha - 1.f;
     return ENTMAX_OK;
 }
 
@@ -222,7 +255,8 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
              int out_dtype, float* tau, cudaStream_t stream, float* otil = nullptr, float* rsum = nullptr) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
-    rc = check_alpha(alpha);
+    float am1 = 0.5f;
+    rc = check_alpha(alpha, &am1);
     if (rc) return rc;
     if (layout != ENTMAX_LAYOUT_BHLD && layout != ENTMAX_LAYOUT_BLHD) return ENTMAX_ERR_ARG;
     rc = check_kv_heads(H, Hkv, in_dtype);
@@ -236,7 +270,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
     if (rc) return rc;
 
     const size_t n = (size_t)B * H * L * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, alpha - 1.f, layout};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, am1, layout};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[3] = {Q, K, V};
@@ -248,7 +282,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
         a.V = dst[2];
     }
     FwdOut o{O, out_dtype == ENTMAX_F32, tau, SavedSupport{}, otil, rsum};
-    return record(launch_fwd(a, o, stream));
+    return record(softmax_alpha(a) ? launch_fwd_softmax(a, o, stream) : launch_fwd(a, o, stream));
 }
 }  // namespace
 
@@ -365,7 +399,8 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
                    int out_dtype, float* tau, void* saved, size_t saved_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
-    rc = check_alpha(alpha);
+    float am1 = 0.5f;
+    rc = check_alpha(alpha, &am1);
     if (rc) return rc;
     if (layout != ENTMAX_LAYOUT_BHLD && layout != ENTMAX_LAYOUT_BLHD) return ENTMAX_ERR_ARG;
     rc = check_kv_heads(H, Hkv, in_dtype);
@@ -381,7 +416,7 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(status_ptr(&status));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, alpha - 1.f, layout};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, am1, layout};
     // the tensor-core backward recomputes the scores and reads no support lists: none are saved
     // (it derives u_i in a pass of its own, which costs less than writing the auxiliary rows here)
     const bool save = !dense_bwd(a);
@@ -403,7 +438,7 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
         a.V = dst[2];
     }
     FwdOut o{O, out_dtype == ENTMAX_F32, tau, sv};
-    return record(launch_fwd(a, o, stream));
+    return record(softmax_alpha(a) ? launch_fwd_softmax(a, o, stream) : launch_fwd(a, o, stream));
 }
 
 int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
@@ -412,7 +447,8 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
                    float* dV, void* workspace, size_t ws_bytes, cudaStream_t stream) {
     int rc = check_common(Q, K, V, in_dtype, causal, window, scale, B, H, L, D);
     if (rc) return rc;
-    rc = check_alpha(alpha);
+    float am1 = 0.5f;
+    rc = check_alpha(alpha, &am1);
     if (rc) return rc;
     if (layout != ENTMAX_LAYOUT_BHLD && layout != ENTMAX_LAYOUT_BLHD) return ENTMAX_ERR_ARG;
     rc = check_kv_heads(H, Hkv, in_dtype);
@@ -429,7 +465,7 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     rc = record(status_ptr(&status));
     if (rc) return rc;
     const size_t n = (size_t)R * HEAD_DIM;
-    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, alpha - 1.f, layout};
+    AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, am1, layout};
     BwdIO io{tau, dO, dQ, dK, dV, nullptr};
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
@@ -521,9 +557,8 @@ float* g_noalloc_ptr[MAX_DEVICES] = {};
 // may not use the array's symbol as an address); the lookup allocates nothing.
 cudaError_t noalloc_scratch(float** out) {
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = current_device(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_noalloc_ptr[dev]) {
         void* p = nullptr;

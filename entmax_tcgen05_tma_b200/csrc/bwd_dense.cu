@@ -1,5 +1,6 @@
-// bwd_dense.cu -- backward pass of 1.5-entmax attention with every contraction on tcgen05, for
-// rows whose allowed keys span few key blocks (short sequences, causal windows).
+// bwd_dense.cu -- backward pass with every contraction on tcgen05: 1.5-entmax attention on rows
+// whose allowed keys span few key blocks (short sequences, causal windows), and softmax attention
+// (alpha = 1, dense supports) at every length.
 //
 // Closed-form Jacobian of page "svd-sst2-roberta-adasplash", section 2.4 (model card
 // "roberta-base-adasplash", section 2): with h_ij = sqrt(p_ij) = max(0, (S_ij - tau_i)/2),
@@ -19,6 +20,9 @@
 //  * dkdv kernel (key-major, one CTA per 128 keys, 64-query blocks over every query head that
 //    reads the key/value head):
 //      S^T = K Q^T, dA^T = V dO^T;  P^T = h^2, dS^T as above;  dV += P^T dO,  dK += dS^T Q  (hi + lo)
+// Softmax (the pages' alpha = 1 branch, page "svd-sst2-roberta-adasplash", section 4) has the same
+// Jacobian with h replaced by p = exp(S - tau) (tau = log sum_j exp(S_ij)) and P = p: both kernels
+// take it as a template flag that changes only the weight of a score (dense.cuh, weight2).
 // The dq kernel runs first: the dkdv kernel reads its u.  dS and P enter the tensor core as two
 // bf16 parts each (x = hi + lo to about 16 significant bits), so dQ, dK and dV carry fp32-level
 // accuracy (one bf16 part would leave errors of order 1e-2 in sums over a few hundred terms).  No
@@ -34,20 +38,14 @@
 // MMAs at teardown (common.cuh).
 #include <cuda_bf16.h>
 #include <math.h>
-#include "common.cuh"
+#include "dense.cuh"
 #include "internal.h"
 
 namespace entmax {
 namespace {
 
-constexpr int THREADS = 320;
-constexpr int NUM_EPI = 256;          // epilogue threads: two per tile row
-constexpr int W_PROD = 8, W_MMA = 9;
-constexpr int TMEM_COLS_D = 256;
-constexpr int BK = 64;                // keys (dq kernel) or queries (dkdv kernel) per streamed block
-constexpr int HB = BK / 2;            // columns of a block per epilogue thread
-constexpr int SUB = 16;               // columns an epilogue thread holds at a time
-constexpr int BLK_ROW_BYTES = BK * HEAD_DIM * 2;   // 8 KiB: one streamed [64][64] bf16 block
+using namespace dense;
+
 // TMEM set: columns [0, 64) score tile, [64, 128) dA tile.  Epilogue half g reads columns
 // [32 g, 32 g + 32) of each, 16 at a time, and writes the bf16 parts of those 16 back over them:
 // the hi part (8 packed columns) first, then the lo part.  A product's K step k (block columns
@@ -87,7 +85,7 @@ constexpr int NSK = 4;                               // input ring stages
 constexpr int KO_K = 0;                              // K tile [128][64], SW128
 constexpr int KO_V = KO_K + TILE_BYTES;              // V tile
 constexpr int KO_RING = KO_V + TILE_BYTES;           // NSK x (Q block, dO block)
-constexpr int KO_CU = KO_RING + NSK * 2 * BLK_ROW_BYTES;  // per epilogue warp: float [2][32]: -tau/2, u of its 32 queries
+constexpr int KO_CU = KO_RING + NSK * 2 * BLK_ROW_BYTES;  // per epilogue warp: float [2][32]: woffset(tau), u of its 32 queries
 constexpr int KO_CTL = KO_CU + (NUM_EPI / 32) * 2 * HB * 4;
 
 struct DkCtl {
@@ -108,48 +106,8 @@ constexpr int K_SMEM_BYTES = KO_CTL + (int)sizeof(DkCtl) + 1024;
 static_assert(KO_RING % 1024 == 0, "operand alignment");
 static_assert(K_SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
 
-using QPipe = Pipe<BK, 2, 2, 1>;  // only its block-list builder (64-key blocks)
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// Bounded wait whose outcome the whole warp shares.
-__device__ __forceinline__ bool warp_wait_d(uint32_t bar, uint32_t parity, int* abort_flag, const WaitCfg& wc) {
-    return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, wc));
-}
-
-// Named barrier over the 8 epilogue warps (id 1; 0 is __syncthreads).
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(NUM_EPI) : "memory"); }
-
-// Zeroes lane x (y) of a pair unless bit k (k + 1) of vm is set.
-__device__ __forceinline__ uint64_t f2mask(uint64_t v, uint32_t vm, int k) {
-    float x, y;
-    f2unpack(v, x, y);
-    return f2pack(((vm >> k) & 1u) ? x : 0.f, ((vm >> (k + 1)) & 1u) ? y : 0.f);
-}
-
-// MMA thread: commit to `bar` (phase parity `par`) and remember it as the last commit.
-__device__ __forceinline__ void commit_to(uint64_t* bar, uint32_t par, uint32_t* last_bar, uint32_t* last_par) {
-    tc_commit(smem_u32(bar));
-    *last_bar = smem_u32(bar);
-    *last_par = par;
-}
-
-// Teardown after an abort, past the CTA's teardown barrier: the producer thread waits for the
-// fixed tiles and its last ns streamed loads, the MMA thread for its last commit.
-__device__ __forceinline__ void drain_dense(uint64_t* full_a, uint64_t* full, int ns, int nload, uint32_t last_bar,
-                                            uint32_t last_par, int warp, int lane) {
-    if (lane != 0) return;
-    if (warp == W_PROD) {
-        wait_drain(smem_u32(full_a), 0);
-        for (int m = max(0, nload - ns); m < nload; ++m) wait_drain(smem_u32(&full[m % ns]), (uint32_t)(m / ns) & 1u);
-    }
-    if (warp == W_MMA && last_bar) wait_drain(last_bar, last_par);
-}
-
 // ================================================================== dq kernel
-template <bool kPass1>
+template <bool kPass1, bool kSoftmax>
 __global__ void __launch_bounds__(THREADS, 2)
 dense_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
                 const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
@@ -202,7 +160,7 @@ dense_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int i_last = min(i0 + TILE - 1, L - 1);
         const int klo = a.window > 0 ? max(0, i0 - a.window + 1) : 0;
         const int khi = a.causal ? i_last : L - 1;
-        const int nb = QPipe::build_block_list(blk, bits, klo, khi, i0, i_last, a.causal, a.window);
+        const int nb = BlockList::build_block_list(blk, bits, klo, khi, i0, i_last, a.causal, a.window);
         if (lane == 0) ctl->nblk = nb;
     }
     tc_fence_before();
@@ -290,7 +248,7 @@ dense_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         int rlo, rhi;
         row_key_range(i, L, a.causal, a.window, rlo, rhi);
         const float tau_i = i < L ? io.tau[(size_t)bh * L + i] : INFINITY;
-        const float hs = 0.5f * a.scale, hc = -0.5f * tau_i;  // h = max(0, hs * raw score + hc)
+        const float hs = wslope<kSoftmax>(a.scale), hc = woffset<kSoftmax>(tau_i);  // weight of a raw score pair
         const uint64_t hs2 = f2pack(hs, hs), hc2 = f2pack(hc, hc);
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t trow = tmem + lane_base + (uint32_t)(HB * g);
@@ -329,7 +287,7 @@ dense_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     read_sub(c, sv, av);
 #pragma unroll
                     for (int k = 0; k < SUB; k += 2) {
-                        const uint64_t h2 = f2mask(f2relu(f2fma(f2pack(sv[k], sv[k + 1]), hs2, hc2)), vm, SUB * c + k);
+                        const uint64_t h2 = f2mask(weight2<kSoftmax>(f2pack(sv[k], sv[k + 1]), hs2, hc2), vm, SUB * c + k);
                         sh2 = f2add(sh2, h2);
                         sw2 = f2fma(h2, f2pack(av[k], av[k + 1]), sw2);
                     }
@@ -409,7 +367,7 @@ dense_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 uint32_t hi[SUB / 2], lo[SUB / 2];
 #pragma unroll
                 for (int k = 0; k < SUB; k += 2) {
-                    uint64_t h2 = f2relu(f2fma(f2pack(sv[k], sv[k + 1]), hs2, hc2));
+                    uint64_t h2 = weight2<kSoftmax>(f2pack(sv[k], sv[k + 1]), hs2, hc2);
                     if (masked) h2 = f2mask(h2, vm, SUB * c + k);
                     f2split(f2mul(h2, f2sub(f2pack(av[k], av[k + 1]), u2)), hi[k >> 1], lo[k >> 1]);
                 }
@@ -464,6 +422,7 @@ dense_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 }
 
 // ================================================================== dkdv kernel
+template <bool kSoftmax>
 __global__ void __launch_bounds__(THREADS, 2)
 dense_dkdv_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                   const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
@@ -601,12 +560,12 @@ dense_dkdv_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
         const bool key_ok = my_key_ok;
         int cq_lo, cq_hi;
         col_query_range(j, L, a.causal, a.window, cq_lo, cq_hi);
-        const float hs = 0.5f * a.scale;
+        const float hs = wslope<kSoftmax>(a.scale);
         const uint64_t hs2 = f2pack(hs, hs);
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t trow = tmem + lane_base + (uint32_t)(HB * g);
-        float* cu = cu_all + warp * 2 * HB;  // this warp's copy: [0, 32) -tau/2, [32, 64) u of its 32 queries
-        // lane l fetches, for job m, -tau/2 and u of query 32 g + l of the block (-inf / 0 past L: no
+        float* cu = cu_all + warp * 2 * HB;  // this warp's copy: [0, 32) woffset(tau), [32, 64) u of its 32 queries
+        // lane l fetches, for job m, woffset(tau) and u of query 32 g + l of the block (-inf / 0 past L: no
         // such query row)
         auto fetch = [&](int m, float& c, float& uu) {
             c = -INFINITY;
@@ -615,7 +574,7 @@ dense_dkdv_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                 const int gq = m / nbq, q = (qb0 + m - gq * nbq) * BK + HB * g + lane;
                 if (q < L) {
                     const size_t row = (size_t)(b * a.H + hk * rep + gq) * L + q;
-                    c = -0.5f * io.tau[row];
+                    c = woffset<kSoftmax>(io.tau[row]);
                     uu = io.u[row];
                 }
             }
@@ -624,7 +583,7 @@ dense_dkdv_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
         fetch(0, c_next, u_next);
         bool live = true;
         for (int m = 0; m < njobs && live; ++m) {
-            // stage this job's (-tau/2, u) for the warp; start fetching the next job's
+            // stage this job's (woffset(tau), u) for the warp; start fetching the next job's
             __syncwarp();
             cu[lane] = c_next;
             cu[HB + lane] = u_next;
@@ -636,8 +595,8 @@ dense_dkdv_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
             // every pair of the block allowed for every key of the tile: no per-pair mask
             const bool full = (!a.causal || q0 >= j_last) && (a.window == 0 || q0 + BK - 1 <= j0 + a.window - 1);
             const uint32_t vm = !key_ok ? 0u : full ? 0xffffffffu : range_bits(q0 + HB * g, cq_lo, cq_hi);
-            // P^T = h^2 and dS^T = h (dA^T - u) for 16 columns, split into bf16 parts and written back
-            // over the S^T and dA^T columns this thread just read
+            // P^T (h^2, or p for softmax) and dS^T = w (dA^T - u) for 16 columns, split into bf16 parts
+            // and written back over the S^T and dA^T columns this thread just read
             auto pds_sub = [&](int c, bool masked) {
                 float sv[SUB], av[SUB];
                 tmem_ld16(trow + SUB * c, sv);
@@ -654,9 +613,9 @@ dense_dkdv_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_consta
                         const int k = 4 * k4 + 2 * e;
                         const uint64_t c2 = e ? f2pack(c4.z, c4.w) : f2pack(c4.x, c4.y);
                         const uint64_t uu2 = e ? f2pack(u4.z, u4.w) : f2pack(u4.x, u4.y);
-                        uint64_t h2 = f2relu(f2fma(f2pack(sv[k], sv[k + 1]), hs2, c2));
+                        uint64_t h2 = weight2<kSoftmax>(f2pack(sv[k], sv[k + 1]), hs2, c2);
                         if (masked) h2 = f2mask(h2, vm, SUB * c + k);
-                        f2split(f2mul(h2, h2), ph[k >> 1], pl[k >> 1]);
+                        f2split(kSoftmax ? h2 : f2mul(h2, h2), ph[k >> 1], pl[k >> 1]);
                         f2split(f2mul(h2, f2sub(f2pack(av[k], av[k + 1]), uu2)), hi[k >> 1], lo[k >> 1]);
                     }
                 }
@@ -728,15 +687,19 @@ cudaError_t launch_bwd_dense(const AttnArgs& a, const BwdIO& io, cudaStream_t st
     if (e == cudaSuccess) e = make_tile_map(&mk, a.K, a.layout, a.B, a.Hkv, a.L, BK);
     if (e == cudaSuccess) e = make_tile_map(&mv, a.V, a.layout, a.B, a.Hkv, a.L, BK);
     if (e != cudaSuccess) return e;
-    // without the forward's auxiliary rows the dq kernel first derives u from a pass over the blocks
-    const bool pass1 = io.otil == nullptr || io.rsum == nullptr;
-    const void* fq = pass1 ? reinterpret_cast<const void*>(dense_dq_kernel<true>)
-                           : reinterpret_cast<const void*>(dense_dq_kernel<false>);
-    e = ensure_smem_attr(fq, Q_SMEM_BYTES, pass1 ? 6 : 8);
+    // without the forward's auxiliary rows (1.5-entmax only) the dq kernel first derives u from a
+    // pass over the blocks
+    const bool sm = softmax_alpha(a);
+    const bool pass1 = sm || io.otil == nullptr || io.rsum == nullptr;
+    const void* fq = sm ? reinterpret_cast<const void*>(dense_dq_kernel<true, true>)
+                     : pass1 ? reinterpret_cast<const void*>(dense_dq_kernel<true, false>)
+                             : reinterpret_cast<const void*>(dense_dq_kernel<false, false>);
+    e = ensure_smem_attr(fq, Q_SMEM_BYTES, sm ? 9 : pass1 ? 6 : 8);
     if (e != cudaSuccess) return e;
     dim3 gq((a.L + TILE - 1) / TILE, a.B * a.H);
-    if (pass1) dense_dq_kernel<true><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
-    else dense_dq_kernel<false><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
+    if (sm) dense_dq_kernel<true, true><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
+    else if (pass1) dense_dq_kernel<true, false><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
+    else dense_dq_kernel<false, false><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -746,11 +709,13 @@ cudaError_t launch_bwd_dense(const AttnArgs& a, const BwdIO& io, cudaStream_t st
     if (e == cudaSuccess) e = make_tile_map(&kq, a.Q, a.layout, a.B, a.H, a.L, BK);
     if (e == cudaSuccess) e = make_tile_map(&kdo, dO, a.layout, a.B, a.H, a.L, BK);
     if (e != cudaSuccess) return e;
-    const void* fk = reinterpret_cast<const void*>(dense_dkdv_kernel);
-    e = ensure_smem_attr(fk, K_SMEM_BYTES, 7);
+    const void* fk = sm ? reinterpret_cast<const void*>(dense_dkdv_kernel<true>)
+                        : reinterpret_cast<const void*>(dense_dkdv_kernel<false>);
+    e = ensure_smem_attr(fk, K_SMEM_BYTES, sm ? 10 : 7);
     if (e != cudaSuccess) return e;
     dim3 gk((a.L + TILE - 1) / TILE, a.B * a.Hkv);
-    dense_dkdv_kernel<<<gk, THREADS, K_SMEM_BYTES, stream>>>(kk, kv, kq, kdo, a, io);
+    if (sm) dense_dkdv_kernel<true><<<gk, THREADS, K_SMEM_BYTES, stream>>>(kk, kv, kq, kdo, a, io);
+    else dense_dkdv_kernel<false><<<gk, THREADS, K_SMEM_BYTES, stream>>>(kk, kv, kq, kdo, a, io);
     return cudaGetLastError();
 }
 

@@ -20,7 +20,8 @@ struct AttnArgs {
     unsigned long long timeout_ns;
     int Hkv;                 // key/value heads (H % Hkv == 0); query head h of batch b reads KV head
                              // b * Hkv + h / (H / Hkv) -- grouped-query attention when Hkv < H
-    float am1;               // alpha - 1 in (0, 1]: p = max(0, am1 (S - tau))^(1 / am1); 0.5 is 1.5-entmax
+    float am1;               // alpha - 1 in (0, 1]: p = max(0, am1 (S - tau))^(1 / am1); 0.5 is 1.5-entmax.
+                             // 0: softmax, p = exp(S - tau) with tau = log sum_j exp(S_ij)
     int layout;              // 0: Q, K, V, O, dO, dQ, dK, dV are [B, heads, L, 64]; 1: [B, L, heads, 64]
 };
 
@@ -40,8 +41,10 @@ struct HeadRef {
     __host__ __device__ __forceinline__ size_t step() const { return layout ? (size_t)nh : 1; }
 };
 
-// alpha = 1.5 runs the specialised kernels (closed-form tau finish, p = h^2); any other alpha the
-// generic ones.
+// alpha = 1.5 runs the specialised kernels (closed-form tau finish, p = h^2); any other alpha in
+// (1, 2] the generic ones; alpha = 1 (softmax) the tensor-core kernels of fwd_softmax.cu and
+// bwd_dense.cu.
+__host__ __device__ __forceinline__ bool softmax_alpha(const AttnArgs& a) { return a.am1 == 0.f; }
 __host__ __device__ __forceinline__ bool generic_alpha(const AttnArgs& a) { return a.am1 != 0.5f; }
 
 // Key/value head of query head bh = b * H + h.
@@ -101,15 +104,17 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
 cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B, int nh, int L, int box_rows);
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
+// Softmax forward (fwd_softmax.cu): writes O and tau = log sum_j exp(S_ij); o.save and o.otil unused.
+cudaError_t launch_fwd_softmax(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
 cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
 
-// The tensor-core backward (bwd_dense.cu) serves rows whose allowed keys span few key blocks:
-// sequences of at most 512 keys, or causal windows of at most 128 keys.  There a 128 x 64 tile of
-// (query, key) pairs costs less as tcgen05 products than as gathers over its support.  alpha 1.5
-// only.  Every backward entry point dispatches on this, and the training forward saves no support
-// lists when it holds (the tensor-core backward does not read them).
+// The tensor-core backward (bwd_dense.cu) serves 1.5-entmax rows whose allowed keys span few key
+// blocks -- sequences of at most 512 keys, or causal windows of at most 128 keys: there a 128 x 64
+// tile of (query, key) pairs costs less as tcgen05 products than as gathers over its support -- and
+// softmax (dense supports) at every length.  Every backward entry point dispatches on this, and the
+// training forward saves no support lists when it holds (the tensor-core backward does not read them).
 __host__ __device__ __forceinline__ bool dense_bwd(const AttnArgs& a) {
-    return a.am1 == 0.5f && (a.L <= 512 || (a.causal && a.window > 0 && a.window <= 128));
+    return softmax_alpha(a) || (a.am1 == 0.5f && (a.L <= 512 || (a.causal && a.window > 0 && a.window <= 128)));
 }
 // dq kernel (writes io.u, one float per query row, and dQ), then dkdv kernel (dK, dV).
 cudaError_t launch_bwd_dense(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
@@ -123,5 +128,6 @@ size_t bwd_rows_smem_bytes();
 size_t bwd_keys_smem_bytes();
 size_t dense_dq_smem_bytes();
 size_t dense_dkdv_smem_bytes();
+size_t softmax_fwd_smem_bytes();
 
 }  // namespace entmax

@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
     ENTMAX_OK = 0,
     ENTMAX_ERR_ARG = -1,          /* null pointer, bad size, bad dtype, misaligned pointer, scale <= 0 */
-    ENTMAX_ERR_UNSUPPORTED = -2,  /* D != 64, L > 16384, B*H > 65535, window without causal, alpha = 1 */
+    ENTMAX_ERR_UNSUPPORTED = -2,  /* D != 64, L > 16384, B*H > 65535, window without causal */
     ENTMAX_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed (see entmax_attn_last_cuda_error) */
     ENTMAX_ERR_TIMEOUT = -4,      /* a device-side bounded wait expired */
     ENTMAX_ERR_WORKSPACE = -5     /* workspace missing or smaller than entmax_attn_bwd_workspace_size */
@@ -220,19 +220,26 @@ ENTMAX_API int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const voi
                                          void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
- * alpha-entmax attention for any alpha in (1, 2] (page "svd-sst2-roberta-adasplash", section 4: the
+ * alpha-entmax attention for any alpha in [1, 2] (page "svd-sst2-roberta-adasplash", section 4: the
  * attention layer's entmax_bisect routine solves sum_j max(0, (alpha-1) s_j - tau')^(1/(alpha-1)) = 1
- * by bisection for alpha in (1, 2]; alpha = 1.5 is the 1.5-entmax of every other entry point, alpha =
- * 2 is sparsemax).  With a = alpha - 1 and tau in score units (tau' = a tau):
+ * by bisection for alpha in (1, 2] and returns softmax for |alpha - 1| < 1e-4; alpha = 1.5 is the
+ * 1.5-entmax of every other entry point, alpha = 2 is sparsemax).  For alpha in (1, 2], with
+ * a = alpha - 1 and tau in score units (tau' = a tau):
  *   p_ij = max(0, a (S_ij - tau_i))^(1/a),  sum_j p_ij = 1,  O_i = sum_j p_ij V_j,
  * and the backward uses the Jacobian w_i (delta_ij - w_j / sum_k w_k), w = p^(2 - alpha).
- *   alpha      in (1, 2]; alpha = 1 (softmax, dense supports) returns ENTMAX_ERR_UNSUPPORTED, any
- *              other value (or NaN) ENTMAX_ERR_ARG.  alpha = 1.5 runs exactly the kernels of the
- *              entry points above; other values run variants whose tau solve is Newton's method
- *              from the bracket's lower end (bisection as the backstop) instead of bisection with a
- *              closed-form finish.  Supports grow as alpha
- *              approaches 1: rows with more candidates than the kernels list are recomputed on CUDA
- *              cores, so small alpha - 1 is correct but slow.
+ *   alpha      in [1, 2]; any other value (or NaN) returns ENTMAX_ERR_ARG.  alpha = 1.5 runs exactly
+ *              the kernels of the entry points above; other values in (1, 2] run variants whose tau
+ *              solve is Newton's method from the bracket's lower end (bisection as the backstop)
+ *              instead of bisection with a closed-form finish.  Supports grow as alpha approaches 1:
+ *              rows with more candidates than the kernels list are recomputed on CUDA cores, so
+ *              small alpha - 1 is correct but slow.
+ *              Softmax: like the pages' routine, |alpha - 1| < 1e-4 computes softmax attention,
+ *              p_ij = exp(S_ij - tau_i) with tau_i = log sum_j exp(S_ij) over the allowed keys (the
+ *              alpha -> 1 limit; every allowed key is in the support).  Its forward and backward run
+ *              every product on the tensor cores (two passes over the key blocks in the forward:
+ *              tau first, then O); the training forward saves no supports (saved is still checked
+ *              for size and alignment, and nothing is written to it) and the backward recomputes
+ *              the scores.  Its gradients are the same bit for bit from run to run.
  *   H_kv       key/value heads as in the _gqa calls (H_kv = H: plain multi-head attention).
  *   saved      entmax_attn_fwd_ex: NULL with saved_bytes = 0 computes the forward only
  *              (entmax_attn_fwd / _gqa); otherwise the training forward (entmax_attn_fwd_train /

@@ -50,7 +50,8 @@ def allowed_matrix(L, causal, window, mask_row):
 
 def check_rows(Qd, Kd, row_ids, tau_gpu_rows, tau_ref_rows, key_mask, causal, window, scale, H, L, alpha=1.5):
     """Simplex and support checks for the listed rows, in fp64 from the GPU's tau
-    (p = max(0, (alpha-1)(s - tau))^(1/(alpha-1)); alpha 1.5: ((s - tau)/2)^2)."""
+    (p = max(0, (alpha-1)(s - tau))^(1/(alpha-1)); alpha 1.5: ((s - tau)/2)^2; alpha 1: softmax,
+    p = exp(s - tau), every allowed key in the support)."""
     a1 = alpha - 1.0
     worst_sum = 0.0
     for r, rid in enumerate(row_ids):
@@ -65,6 +66,9 @@ def check_rows(Qd, Kd, row_ids, tau_gpu_rows, tau_ref_rows, key_mask, causal, wi
         s = scale * (Kd[b, h][a] @ Qd[b, h, i])
         tg, tr = tau_gpu_rows[r], tau_ref_rows[r]
         assert abs(tg - tr) <= TAU_TOL, (rid, tg, tr)
+        if alpha == 1.0:
+            worst_sum = max(worst_sum, abs(np.exp(s - tg).sum() - 1.0))
+            continue
         p = np.clip(a1 * (s - tg), 0, None) ** (1.0 / a1)
         worst_sum = max(worst_sum, abs(p.sum() - 1.0))
         differ = (s > tg) != (s > tr)

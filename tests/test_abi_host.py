@@ -231,7 +231,7 @@ def _ex_calls(alpha, B=1, H=2, Hkv=2, in_dtype=0, saved=P, saved_bytes=None, lay
 
 
 @pytest.mark.parametrize("alpha,code", [
-    (1.0, E.ENTMAX_ERR_UNSUPPORTED),  # softmax
+    (0.9998, E.ENTMAX_ERR_ARG),  # below the softmax band |alpha - 1| < 1e-4
     (0.5, E.ENTMAX_ERR_ARG),
     (2.0001, E.ENTMAX_ERR_ARG),
     (float("nan"), E.ENTMAX_ERR_ARG),
@@ -246,6 +246,10 @@ def test_ex_entry_points_validate_before_launch():
     # valid alpha, empty batch: a no-op
     assert _ex_calls(1.75, B=0) == (E.ENTMAX_OK, E.ENTMAX_OK)
     assert _ex_calls(2.0, B=0) == (E.ENTMAX_OK, E.ENTMAX_OK)
+    # softmax: alpha = 1 and the band around it (the pages' |alpha - 1| < 1e-4)
+    for a in (1.0, 0.99995, 1.00005):
+        assert _ex_calls(a, B=0) == (E.ENTMAX_OK, E.ENTMAX_OK)
+        assert _ex_calls(a, H=4, Hkv=3) == (E.ENTMAX_ERR_ARG, E.ENTMAX_ERR_ARG)
     # grouped heads are checked as in the _gqa calls
     assert _ex_calls(1.25, H=4, Hkv=3) == (E.ENTMAX_ERR_ARG, E.ENTMAX_ERR_ARG)
     assert _ex_calls(1.25, H=4, Hkv=2, in_dtype=1) == (E.ENTMAX_ERR_UNSUPPORTED, E.ENTMAX_ERR_UNSUPPORTED)

@@ -55,10 +55,10 @@ int main(void) {
     EXPECT(entmax_attn_bwd(FAKE, FAKE, FAKE, ENTMAX_BF16, NULL, 0, 0, 0.125f, 1, 1, 64, 64, tau, FAKE,
                            (float*)FAKE, (float*)FAKE, (float*)FAKE, NULL, 0, (cudaStream_t)0)
            == ENTMAX_ERR_WORKSPACE);
-    /* alpha = 1 (softmax) is outside the method; alpha > 2 is a bad argument */
-    EXPECT(entmax_attn_fwd_ex(FAKE, FAKE, FAKE, ENTMAX_BF16, NULL, 0, 0, 0.125f, 1.0f, 1, 2, 1, 64, 64,
+    /* alpha below 1 (the softmax band is |alpha - 1| < 1e-4) or above 2 is a bad argument */
+    EXPECT(entmax_attn_fwd_ex(FAKE, FAKE, FAKE, ENTMAX_BF16, NULL, 0, 0, 0.125f, 0.999f, 1, 2, 1, 64, 64,
                               ENTMAX_LAYOUT_BHLD, FAKE, ENTMAX_BF16, tau, NULL, 0, (cudaStream_t)0)
-           == ENTMAX_ERR_UNSUPPORTED);
+           == ENTMAX_ERR_ARG);
     EXPECT(entmax_attn_fwd_ex(FAKE, FAKE, FAKE, ENTMAX_BF16, NULL, 0, 0, 0.125f, 2.5f, 1, 2, 1, 64, 64,
                               ENTMAX_LAYOUT_BHLD, FAKE, ENTMAX_BF16, tau, NULL, 0, (cudaStream_t)0)
            == ENTMAX_ERR_ARG);
