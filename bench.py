@@ -552,7 +552,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     # the other fwd+bwd workloads the bf16-roofline target covers (L >= 512), timed the same way on
     # every rank (their timing takes the same barriers and max over ranks)
     extras = {}
-    if not args.no_extra and not variant and not recompute and args.workload == 4:
+    if not args.no_extra and not variant and not recompute and not w.fp32_inputs and args.workload == 4:
         peaks = load_peaks()
         extras = {str(k): extra_workload(args, WORKLOADS[k], dev, world, flush, peaks) for k in (3, 5)}
         # softmax attention (alpha = 1, the pages' alpha -> 1 branch) on the headline shape
@@ -623,7 +623,9 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                   "(L2 left holding clean lines)",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
-        "variant": {"alpha": alpha, "H_kv": Hkv, "layout": "BLHD" if args.blhd else "BHLD"} if variant else None,
+        "variant": {"alpha": alpha, "H_kv": Hkv, "layout": "BLHD" if args.blhd else "BHLD",
+                    "inputs": "fp32 (rounded to bf16 on the device)" if w.fp32_inputs else "bf16"}
+        if variant or w.fp32_inputs else None,
         "backward": ("entmax_attn_bwd" if recompute else "entmax_attn_bwd_saved") + (
             " (tensor-core kernels: scores recomputed, every product on tcgen05)" if tensor_core_backward(w, alpha)
             else " (scores recomputed)" if recompute else " (saved supports)"),
@@ -666,6 +668,8 @@ def bench_workload(args) -> Workload:
         if args.hkv < 1 or w.H % args.hkv:
             raise SystemExit("--hkv must divide the workload's %d heads" % w.H)
         w = w.with_shape(H_kv=args.hkv)
+    if getattr(args, "fp32_inputs", False):
+        w = w.with_shape(fp32_inputs=True)
     return w
 
 
@@ -743,6 +747,8 @@ def main() -> int:
     ap.add_argument("--alpha", type=float, default=1.5, help="alpha-entmax variant, alpha in [1, 2] (1: softmax)")
     ap.add_argument("--hkv", type=int, default=0, help="grouped-query variant: key/value heads")
     ap.add_argument("--blhd", action="store_true", help="variant: tensors in [B, L, H, 64] memory")
+    ap.add_argument("--fp32-inputs", action="store_true",
+                    help="variant: Q, K, V, dO given as fp32 (the library rounds them to bf16 on the device)")
     ap.add_argument("--bwd", default="saved", choices=["saved", "recompute"],
                     help="backward path: from the forward's saved supports, or entmax_attn_bwd (scores recomputed)")
     args = ap.parse_args()
