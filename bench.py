@@ -427,6 +427,11 @@ def extra_workload(args, w: Workload, dev, world: int, flush: _Flush, peaks: dic
                            "algorithmic_flops_per_launch": alg, "issued_mma_flops_per_launch": 2.0 * alg,
                            "traffic": None}
         out["roofline"]["frac"] = out["roofline"]["achieved"] / out["roofline"]["peak"]
+        tr = ROOT / "profiles" / "traffic_softmax_workload%d.txt" % w.wid
+        if tr.exists() and w.H == w.kv_heads and not args.blhd:
+            t = json.loads(tr.read_text())
+            if t.get("kernel") == "softmax_fwd_kernel" and t.get("source_hash") == source_hash("softmax_fwd_kernel"):
+                out["roofline"]["traffic"] = t["bytes_per_launch"]
     del prep
     torch.cuda.empty_cache()
     return out
@@ -595,7 +600,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     tr = ROOT / "profiles" / ("traffic_workload%d.txt" % w.wid)
     if tr.exists() and not variant:
         t = json.loads(tr.read_text())
-        if t.get("kernel") == "entmax_fwd_kernel" and t.get("source_hash") == source_hash():
+        if t.get("kernel") == fwd_kernel and t.get("source_hash") == source_hash(fwd_kernel):
             roof["traffic"] = t["bytes_per_launch"]
 
     step_roof = step_roofline(w, km, flops, ms_per_step, peaks)
@@ -653,11 +658,22 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     return out
 
 
-def source_hash() -> str:
+# The source files each profiled kernel is built from: a committed traffic figure counts only while
+# the hash of its kernel's files is the one it was captured at.
+KERNEL_SOURCES = {
+    "entmax_fwd_kernel": ("fwd.cu", "common.cuh", "ptx.cuh", "internal.h"),
+    "softmax_fwd_kernel": ("fwd_softmax.cu", "dense.cuh", "common.cuh", "ptx.cuh", "internal.h"),
+}
+
+
+def source_hash(kernel: str | None = None) -> str:
+    """sha256 (16 hex digits) of the kernel's source files, or of every file under csrc/."""
     import hashlib
 
+    csrc = ROOT / "entmax_tcgen05_tma_b200" / "csrc"
+    files = [csrc / f for f in KERNEL_SOURCES[kernel]] if kernel else sorted(csrc.glob("*"))
     h = hashlib.sha256()
-    for p in sorted((ROOT / "entmax_tcgen05_tma_b200" / "csrc").glob("*")):
+    for p in files:
         h.update(p.read_bytes())
     return h.hexdigest()[:16]
 
@@ -754,8 +770,8 @@ def main() -> int:
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if not 1.0 < args.alpha <= 2.0:
-        ap.error("--alpha must lie in (1, 2]")
+    if not (args.alpha == 1.0 or 1.0 < args.alpha <= 2.0):
+        ap.error("--alpha must be 1 (softmax) or lie in (1, 2]")
     if args.bwd == "recompute" and (args.alpha != 1.5 or args.hkv or args.blhd):
         ap.error("--bwd recompute takes the plain path only (alpha 1.5, H_kv = H, [B, H, L, 64])")
 

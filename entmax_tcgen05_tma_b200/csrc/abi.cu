@@ -438,7 +438,13 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
         a.V = dst[2];
     }
     FwdOut o{O, out_dtype == ENTMAX_F32, tau, sv};
-    return record(softmax_alpha(a) ? launch_fwd_softmax(a, o, stream) : launch_fwd(a, o, stream));
+    if (softmax_alpha(a)) {
+        // the saved buffer holds O in fp32, the softmax backward's auxiliary row (u_i = dO_i . O_i)
+        static_assert(SAVE_CAP * 6 >= HEAD_DIM * 4, "the saved buffer holds an fp32 row of O");
+        o.otil = static_cast<float*>(saved);
+        return record(launch_fwd_softmax(a, o, stream));
+    }
+    return record(launch_fwd(a, o, stream));
 }
 
 int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,
@@ -481,6 +487,7 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     const SavedBwdWs ws = carve_saved_bwd_ws(workspace, R);
     if (dense_bwd(a)) {
         io.u = reinterpret_cast<float*>(ws.key_off);  // R floats of the workspace hold u
+        if (softmax_alpha(a)) io.otil = static_cast<const float*>(saved);  // the forward's fp32 O
         return record(launch_bwd_dense(a, io, stream));
     }
     return record(launch_bwd_saved(a, io, carve_saved(const_cast<void*>(saved), R), ws, stream));

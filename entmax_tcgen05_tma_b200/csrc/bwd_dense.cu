@@ -347,7 +347,7 @@ dense_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (g == 0) red[TILE + r] = dot + red[r];
             epi_bar();
             if (i < L) {
-                const float rs = io.rsum[row];
+                const float rs = kSoftmax ? 1.f : io.rsum[row];  // softmax: sum_j p_ij = 1
                 u = rs > 0.f ? red[TILE + r] / rs : 0.f;
                 if (g == 0) io.u[row] = u;
             }
@@ -687,19 +687,25 @@ cudaError_t launch_bwd_dense(const AttnArgs& a, const BwdIO& io, cudaStream_t st
     if (e == cudaSuccess) e = make_tile_map(&mk, a.K, a.layout, a.B, a.Hkv, a.L, BK);
     if (e == cudaSuccess) e = make_tile_map(&mv, a.V, a.layout, a.B, a.Hkv, a.L, BK);
     if (e != cudaSuccess) return e;
-    // without the forward's auxiliary rows (1.5-entmax only) the dq kernel first derives u from a
-    // pass over the blocks
+    // without the forward's auxiliary rows the dq kernel first derives u from a pass over the blocks
+    // (1.5-entmax); softmax always has them: its auxiliary row is the forward's fp32 O, row sum 1
     const bool sm = softmax_alpha(a);
-    const bool pass1 = sm || io.otil == nullptr || io.rsum == nullptr;
-    const void* fq = sm ? reinterpret_cast<const void*>(dense_dq_kernel<true, true>)
-                     : pass1 ? reinterpret_cast<const void*>(dense_dq_kernel<true, false>)
-                             : reinterpret_cast<const void*>(dense_dq_kernel<false, false>);
-    e = ensure_smem_attr(fq, Q_SMEM_BYTES, sm ? 9 : pass1 ? 6 : 8);
-    if (e != cudaSuccess) return e;
+    const bool pass1 = io.otil == nullptr || (!sm && io.rsum == nullptr);
     dim3 gq((a.L + TILE - 1) / TILE, a.B * a.H);
-    if (sm) dense_dq_kernel<true, true><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
-    else if (pass1) dense_dq_kernel<true, false><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
-    else dense_dq_kernel<false, false><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
+    if (sm) {
+        if (pass1) return cudaErrorInvalidValue;  // every softmax backward has the forward's fp32 O
+        const void* fq = reinterpret_cast<const void*>(dense_dq_kernel<false, true>);
+        e = ensure_smem_attr(fq, Q_SMEM_BYTES, 9);
+        if (e != cudaSuccess) return e;
+        dense_dq_kernel<false, true><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
+    } else {
+        const void* fq = pass1 ? reinterpret_cast<const void*>(dense_dq_kernel<true, false>)
+                               : reinterpret_cast<const void*>(dense_dq_kernel<false, false>);
+        e = ensure_smem_attr(fq, Q_SMEM_BYTES, pass1 ? 6 : 8);
+        if (e != cudaSuccess) return e;
+        if (pass1) dense_dq_kernel<true, false><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
+        else dense_dq_kernel<false, false><<<gq, THREADS, Q_SMEM_BYTES, stream>>>(mq, mdo, mk, mv, a, io);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 

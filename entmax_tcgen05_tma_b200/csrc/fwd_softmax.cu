@@ -15,7 +15,9 @@
 // pair costs one exponential.  p~ enters the product as two bf16 parts (p~ = hi + lo to about 16
 // significant bits), so O carries fp32-level accuracy.  Two TMEM sets (block n and n + 1's
 // scores) let the MMA warp issue the next S while the epilogue works on the current one.  Roles and
-// the TMEM part layout: dense.cuh.  A row with no allowed key gets O = 0 and tau = +inf.  Every wait
+// the TMEM part layout: dense.cuh.  A row with no allowed key gets O = 0 and tau = +inf.  The
+// training forward also writes O in fp32: the backward's row scalar u_i = sum_j p_ij dA_ij is then
+// dO_i . O_i, a row dot instead of a pass over the key blocks.  Every wait
 // is bounded; an abort drains the CTA's own loads and MMAs at teardown.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -293,6 +295,11 @@ softmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             for (int k = 0; k < 32; ++k) v[k] = 0.f;
         }
         if (i < L && (have || (nb == 0 && live))) {
+            if (out.otil) {  // the backward's auxiliary row: sum_j p_ij V_j = O_i, in fp32
+                float4* dst = reinterpret_cast<float4*>(out.otil + ((size_t)bh * L + i) * HEAD_DIM + 32 * g);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            }
             if (out.out_f32) {
                 float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out.O) + orow);
 #pragma unroll

@@ -66,8 +66,9 @@ struct FwdOut {
     int out_f32;
     float* tau;              // [B,H,L]
     SavedSupport save;       // row_cnt == nullptr: nothing saved
-    float* otil;             // optional (alpha 1.5): [B*H*L][64] sum_j sqrt(p_ij) V_j, logical row order
-    float* rsum;             // optional with otil: [B*H*L] sum_j sqrt(p_ij)
+    float* otil;             // optional: [B*H*L][64] sum_j w_ij V_j, logical row order, w the Jacobian's
+                             // weight (sqrt(p) at alpha 1.5; p for softmax, where otil is the fp32 O)
+    float* rsum;             // optional with otil at alpha 1.5: [B*H*L] sum_j sqrt(p_ij) (softmax: 1, not written)
 };
 
 // Carves a caller buffer of entmax_attn_saved_bytes() into its arrays.
@@ -83,8 +84,9 @@ struct BwdIO {
     float* dK;
     float* dV;
     float* u;                // workspace [B,H,L]: u_i = sum_j sqrt(p_ij) dA_ij / sum_j sqrt(p_ij)
-    const float* otil;       // optional [B*H*L][64]: the forward's sum_j sqrt(p_ij) V_j (logical row order)
-    const float* rsum;       // optional [B*H*L]: the forward's sum_j sqrt(p_ij); with otil, u_i = dO_i . otil_i / rsum_i
+    const float* otil;       // optional [B*H*L][64]: the forward's sum_j w_ij V_j (logical row order)
+    const float* rsum;       // optional [B*H*L]: the forward's sum_j w_ij; with otil, u_i = dO_i . otil_i / rsum_i
+                             // (softmax: rsum = 1, passed as null)
 };
 
 // Workspace of the support-list backward.
@@ -104,7 +106,8 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
 cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B, int nh, int L, int box_rows);
 
 cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
-// Softmax forward (fwd_softmax.cu): writes O and tau = log sum_j exp(S_ij); o.save and o.otil unused.
+// Softmax forward (fwd_softmax.cu): writes O and tau = log sum_j exp(S_ij), and O in fp32 into o.otil
+// when given; o.save and o.rsum unused.
 cudaError_t launch_fwd_softmax(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
 cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
 

@@ -237,9 +237,10 @@ ENTMAX_API int entmax_attn_bwd_saved_gqa(const void* Q, const void* K, const voi
  *              p_ij = exp(S_ij - tau_i) with tau_i = log sum_j exp(S_ij) over the allowed keys (the
  *              alpha -> 1 limit; every allowed key is in the support).  Its forward and backward run
  *              every product on the tensor cores (two passes over the key blocks in the forward:
- *              tau first, then O); the training forward saves no supports (saved is still checked
- *              for size and alignment, and nothing is written to it) and the backward recomputes
- *              the scores.  Its gradients are the same bit for bit from run to run.
+ *              the row max, then O and tau); the training forward saves no supports but writes O in
+ *              fp32 into saved ([B*H*L][64], logical row order), from which the backward forms
+ *              u_i = sum_j p_ij dA_ij as the row dot dO_i . O_i; the backward recomputes the scores.
+ *              Its gradients are the same bit for bit from run to run.
  *   H_kv       key/value heads as in the _gqa calls (H_kv = H: plain multi-head attention).
  *   saved      entmax_attn_fwd_ex: NULL with saved_bytes = 0 computes the forward only
  *              (entmax_attn_fwd / _gqa); otherwise the training forward (entmax_attn_fwd_train /
