@@ -427,7 +427,7 @@ def extra_workload(args, w: Workload, dev, world: int, flush: _Flush, peaks: dic
                            "algorithmic_flops_per_launch": alg, "issued_mma_flops_per_launch": 2.0 * alg,
                            "traffic": None}
         out["roofline"]["frac"] = out["roofline"]["achieved"] / out["roofline"]["peak"]
-        tr = ROOT / "profiles" / "traffic_softmax_workload%d.txt" % w.wid
+        tr = ROOT / "profiles" / ("traffic_softmax_workload%d.txt" % w.wid)
         if tr.exists() and w.H == w.kv_heads and not args.blhd:
             t = json.loads(tr.read_text())
             if t.get("kernel") == "softmax_fwd_kernel" and t.get("source_hash") == source_hash("softmax_fwd_kernel"):
@@ -661,7 +661,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
 # The source files each profiled kernel is built from: a committed traffic figure counts only while
 # the hash of its kernel's files is the one it was captured at.
 KERNEL_SOURCES = {
-    "entmax_fwd_kernel": ("fwd.cu", "common.cuh", "ptx.cuh", "internal.h"),
+    "entmax_fwd_kernel": ("fwd.cu", "tau15.cuh", "common.cuh", "ptx.cuh", "internal.h"),
     "softmax_fwd_kernel": ("fwd_softmax.cu", "dense.cuh", "common.cuh", "ptx.cuh", "internal.h"),
 }
 
