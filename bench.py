@@ -335,7 +335,7 @@ class _Prepared:
 def tensor_core_backward(w: Workload, alpha: float = 1.5) -> bool:
     """Whether the library runs the backward on its tensor-core kernels (dq, dkdv): softmax (alpha 1)
     always, alpha 1.5 with L <= 512 or a causal window of at most 128 keys (the library's own
-    dispatch rule)."""
+    dispatch rule; alpha 1.5's forward then runs its tensor-core kernel too)."""
     return alpha == 1.0 or (alpha == 1.5 and (w.L <= 512 or (w.causal and 0 < w.window <= 128)))
 
 
@@ -585,7 +585,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     # bf16 figure is its tensor peak
     t_tensor = fwd_alg_flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = fwd_alg_bytes / (peaks["hbm_gbs"] * 1e9)
-    fwd_kernel = "softmax_fwd_kernel" if alpha == 1.0 else "entmax_fwd_kernel"
+    fwd_kernel = ("softmax_fwd_kernel" if alpha == 1.0 else
+                  "entmax_dense_fwd_kernel" if alpha == 1.5 and tensor_core_backward(w, alpha) else "entmax_fwd_kernel")
     if t_tensor >= t_hbm:
         roof = {"kernel": fwd_kernel, "bound": "tensor",
                 "achieved": fwd_alg_flops / (fwd_mean * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
@@ -663,6 +664,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
 KERNEL_SOURCES = {
     "entmax_fwd_kernel": ("fwd.cu", "tau15.cuh", "common.cuh", "ptx.cuh", "internal.h"),
     "softmax_fwd_kernel": ("fwd_softmax.cu", "dense.cuh", "common.cuh", "ptx.cuh", "internal.h"),
+    "entmax_dense_fwd_kernel": ("fwd_dense.cu", "tau15.cuh", "dense.cuh", "common.cuh", "ptx.cuh", "internal.h"),
 }
 
 

@@ -14,8 +14,8 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libentmax_attn.so"
-SOURCES = ["abi.cu", "fwd.cu", "fwd_softmax.cu", "bwd.cu", "bwd_saved.cu", "bwd_dense.cu"]
-DEPS = SOURCES + ["common.cuh", "dense.cuh", "ptx.cuh", "internal.h"]
+SOURCES = ["abi.cu", "fwd.cu", "fwd_dense.cu", "fwd_softmax.cu", "bwd.cu", "bwd_saved.cu", "bwd_dense.cu"]
+DEPS = SOURCES + ["common.cuh", "dense.cuh", "tau15.cuh", "ptx.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -282,7 +282,10 @@ int fwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
         a.V = dst[2];
     }
     FwdOut o{O, out_dtype == ENTMAX_F32, tau, SavedSupport{}, otil, rsum};
-    return record(softmax_alpha(a) ? launch_fwd_softmax(a, o, stream) : launch_fwd(a, o, stream));
+    if (softmax_alpha(a)) return record(launch_fwd_softmax(a, o, stream));
+    // the auxiliary rows come from the gather forward alone
+    if (dense_fwd(a) && !otil) return record(launch_fwd_dense(a, o, stream));
+    return record(launch_fwd(a, o, stream));
 }
 }  // namespace
 
@@ -444,7 +447,7 @@ int fwd_train_impl(const void* Q, const void* K, const void* V, int in_dtype, co
         o.otil = static_cast<float*>(saved);
         return record(launch_fwd_softmax(a, o, stream));
     }
-    return record(launch_fwd(a, o, stream));
+    return record(dense_fwd(a) ? launch_fwd_dense(a, o, stream) : launch_fwd(a, o, stream));
 }
 
 int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, const uint8_t* key_mask, int causal,

@@ -26,6 +26,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 #include "common.cuh"
+#include "tau15.cuh"
 #include "internal.h"
 
 namespace entmax {
@@ -82,27 +83,6 @@ struct __align__(16) RowOut {
     int ovf;
     int pad_;
 };
-// Exact threshold (raw units: sum (v - t)^2 = c4 over the kept values) of the set {a0..a3}
-// (a0 >= a1 >= a2 >= a3, missing values -inf), lowered by a rounding margin.  Any subset of a
-// row gives a lower bound of the row's tau: adding scores can only raise the threshold.
-__device__ __forceinline__ float top4_bound(float a0, float a1, float a2, float a3, float c4) {
-    const float z[4] = {a0, a1, a2, a3};
-    const float inv[4] = {1.f, 0.5f, 1.f / 3.f, 0.25f};
-    float sum = 0.f, sq = 0.f, bound = a0 - sqrtf(c4);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        sum += z[k];
-        sq = fmaf(z[k], z[k], sq);
-        const float mu = sum * inv[k];
-        const float delta = fmaf(c4 - sq, inv[k], mu * mu);
-        if (delta >= 0.f) {
-            const float tk = mu - sqrtf(delta);
-            if (tk <= z[k]) bound = tk;
-        }
-    }
-    return bound - 1e-5f * sqrtf(c4);
-}
-
 // General alpha (am1 = alpha - 1, p = max(0, am1 (x - tau))^(1/am1) in scaled units x = scale S):
 // lower bound (raw units) of the row's tau from the four largest chunk maxima z0 >= .. >= z3 (scores
 // of the row; missing values -inf).  Any subset's threshold is at most the row's.  Start: at
@@ -133,23 +113,6 @@ __device__ __forceinline__ float gen_bound(float a0, float a1, float a2, float a
     b = fmaxf(b, a0 + t / c);
     return b - 1e-5f * wk[0];
 }
-
-__device__ __forceinline__ void top4_insert(float v, float& a0, float& a1, float& a2, float& a3) {
-    if (v > a3) {
-        if (v > a2) {
-            a3 = a2;
-            if (v > a1) {
-                a2 = a1;
-                if (v > a0) { a1 = a0; a0 = v; } else { a1 = v; }
-            } else {
-                a2 = v;
-            }
-        } else {
-            a3 = v;
-        }
-    }
-}
-
 
 // Named barrier over the 8 epilogue warps (id 3; 0 is __syncthreads).
 __device__ __forceinline__ void epi_sync() {
@@ -195,75 +158,6 @@ __device__ __forceinline__ void for_half_block(const PipeCtl* ctl, int n, int ha
     tmem_wait_ld(vb);
     f(va, 2 * half);
     f(vb, 2 * half + 1);
-}
-
-// tau of one row in shifted scaled units (x = scale * S - scale * m, so the row max is 0), from the
-// row's candidates (both partitions, partition 0 first) split evenly over a lane pair: lane h holds
-// entries h, h + 2, ... (NC registers, -inf where unused).
-// Bisection of [lo, hi], a sub-bracket of [-2, -2/sqrt(n)] that still holds the root (the caller's
-// bounds: g(lo) >= 1, g(hi) <= 1; g(-2) >= 1 from the max alone, g(-2/sqrt n) <= 1); every four
-// halvings the warp stops if no lane pair has a candidate strictly inside its bracket: the support
-// is then fixed and the closed-form root on it is exact.  Returns tau_x.
-template <int NC>
-__device__ __forceinline__ float solve_tau(const float* lcv, int r, int h, int nh, int n0, float scale, float ms,
-                                           float lo, float hi) {
-    float x[NC];
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-        const int e = 2 * k + h;  // entry e of the row's two lists, partition 0's n0 entries first
-        x[k] = k < nh ? fmaf(scale, lcv[(e < n0 ? e : CAPW + (e - n0)) * TILE + r], -ms) : -INFINITY;
-    }
-    bool settled = false;
-    for (int it = 0; it < 25; ++it) {
-        const float mid = 0.5f * (lo + hi);
-        float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
-#pragma unroll
-        for (int k = 0; k < NC; k += 4) {
-            const float d0 = fmaxf(x[k] - mid, 0.f), d1 = fmaxf(x[k + 1] - mid, 0.f);
-            const float d2 = fmaxf(x[k + 2] - mid, 0.f), d3 = fmaxf(x[k + 3] - mid, 0.f);
-            g0 = fmaf(d0, d0, g0);
-            g1 = fmaf(d1, d1, g1);
-            g2 = fmaf(d2, d2, g2);
-            g3 = fmaf(d3, d3, g3);
-        }
-        float gs = (g0 + g1) + (g2 + g3);
-        gs += __shfl_xor_sync(0xffffffffu, gs, 1);
-        if (0.25f * gs > 1.f) lo = mid;
-        else hi = mid;
-        if ((it & 3) == 3 || it == 24) {
-            int und = 0;
-#pragma unroll
-            for (int k = 0; k < NC; ++k) und += (x[k] > lo && x[k] < hi) ? 1 : 0;
-            und += __shfl_xor_sync(0xffffffffu, und, 1);
-            settled = und == 0;
-            if (__all_sync(0xffffffffu, settled)) break;
-        }
-    }
-    // closed-form root of sum_S (x - tau)^2 = 4 on S = {x > final midpoint}
-    const float mid = 0.5f * (lo + hi);
-    float K = 0.f, S1 = 0.f, S2 = 0.f;
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-        if (x[k] > mid) {
-            K += 1.f;
-            S1 += x[k];
-            S2 = fmaf(x[k], x[k], S2);
-        }
-    }
-    K += __shfl_xor_sync(0xffffffffu, K, 1);
-    S1 += __shfl_xor_sync(0xffffffffu, S1, 1);
-    S2 += __shfl_xor_sync(0xffffffffu, S2, 1);
-    float tau_x = mid;
-    if (K > 0.f) {
-        const float mu = S1 / K;
-        const float var = fmaxf(S2 / K - mu * mu, 0.f);
-        const float tc = mu - sqrtf(fmaxf(4.f / K - var, 0.f));
-        // with the support settled the root lies in the bracket (clamp only absorbs rounding);
-        // otherwise keep it only if it does
-        if (settled) tau_x = fminf(fmaxf(tc, lo), hi);
-        else if (tc >= lo && tc <= hi) tau_x = tc;
-    }
-    return tau_x;
 }
 
 // General alpha: tau of one row in units y = am1 (scale S - ms) (row max 0, every p term is
@@ -1006,14 +900,14 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         } else {
             switch ((nmax + 7) >> 3) {
                 case 0:
-                case 1: tau_x = solve_tau<8>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-                case 2: tau_x = solve_tau<16>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-                case 3: tau_x = solve_tau<24>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-                case 4: tau_x = solve_tau<32>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-                case 5: tau_x = solve_tau<40>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-                case 6: tau_x = solve_tau<48>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-                case 7: tau_x = solve_tau<56>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
-                default: tau_x = solve_tau<CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 1: tau_x = solve_tau<8, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 2: tau_x = solve_tau<16, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 3: tau_x = solve_tau<24, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 4: tau_x = solve_tau<32, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 5: tau_x = solve_tau<40, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 6: tau_x = solve_tau<48, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                case 7: tau_x = solve_tau<56, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
+                default: tau_x = solve_tau<CAPW, CAPW>(cv, r, h, ns, s0.n, scale, ms, lo, hi); break;
             }
         }
         if (mode == 0) {

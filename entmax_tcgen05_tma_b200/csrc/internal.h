@@ -119,6 +119,10 @@ cudaError_t launch_bwd(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
 __host__ __device__ __forceinline__ bool dense_bwd(const AttnArgs& a) {
     return softmax_alpha(a) || (a.am1 == 0.5f && (a.L <= 512 || (a.causal && a.window > 0 && a.window <= 128)));
 }
+// The tensor-core forward of 1.5-entmax (fwd_dense.cu) serves the same configurations; the gather
+// forward (fwd.cu) keeps the auxiliary rows and the support lists, which it alone writes.
+__host__ __device__ __forceinline__ bool dense_fwd(const AttnArgs& a) { return a.am1 == 0.5f && dense_bwd(a); }
+cudaError_t launch_fwd_dense(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
 // dq kernel (writes io.u, one float per query row, and dQ), then dkdv kernel (dK, dV).
 cudaError_t launch_bwd_dense(const AttnArgs& a, const BwdIO& io, cudaStream_t stream);
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, cudaStream_t stream);
@@ -132,5 +136,6 @@ size_t bwd_keys_smem_bytes();
 size_t dense_dq_smem_bytes();
 size_t dense_dkdv_smem_bytes();
 size_t softmax_fwd_smem_bytes();
+size_t dense_fwd_smem_bytes();
 
 }  // namespace entmax

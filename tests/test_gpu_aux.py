@@ -3,7 +3,8 @@
 
 Otil_i = sum_j sqrt(p_ij) V_j and r_i = sum_j sqrt(p_ij) give the backward's row scalar
 u_i = dO_i . Otil_i / r_i (page "svd-sst2-roberta-adasplash", section 2.4).  The forward's O and tau
-must be exactly those of entmax_attn_fwd; Otil and r are compared with the oracle's attn_aux_rows,
+must be those of entmax_attn_fwd (bit for bit where both run the gather forward, to 1e-4 where
+entmax_attn_fwd runs the tensor-core one); Otil and r are compared with the oracle's attn_aux_rows,
 the gradients with its attn_bwd.  Shapes cover the tensor-core configurations (L <= 512, causal
 windows) and the others, ragged tails, padding down to one key and a fully padded batch.
 """
@@ -49,7 +50,14 @@ def test_aux_rows_and_backward(B, H, L, scale, causal, window, lens):
     O, tau, Ot, rs = E.entmax_attn_fwd_aux(Q, K, V, kmd, causal, window, scale, out_dtype=torch.float32)
     O2, tau2 = E.entmax_attn_fwd(Q, K, V, kmd, causal, window, scale, out_dtype=torch.float32)
     assert E.entmax_attn_device_status() == 0
-    assert torch.equal(O, O2) and torch.equal(tau, tau2)
+    if L <= 512 or (causal and 0 < window <= 128):
+        # entmax_attn_fwd runs the tensor-core forward here, the auxiliary rows the gather forward:
+        # the same O and tau up to the order of their sums
+        assert torch.allclose(O, O2, atol=1e-4, rtol=0) and torch.allclose(tau, tau2, atol=1e-4, rtol=0)
+    else:
+        assert torch.equal(O, O2) and torch.equal(tau, tau2)
+    O_ref, tau_ref = orc.attn_fwd(d["Q"], d["K"], d["V"], km, causal, window, scale)
+    assert np.max(np.abs(to64(O) - O_ref)) <= O_TOL
     ids = np.arange(B * H * L)
     Ot_ref, r_ref = orc.attn_aux_rows(d["Q"], d["K"], d["V"], ids, km, causal, window, scale)
     assert np.max(np.abs(to64(Ot).reshape(-1, 64) - Ot_ref)) <= O_TOL
