@@ -14,8 +14,10 @@
 //            support -- go to the row's two candidate lists in shared memory (one per half row);
 //   tau:     two lanes per row, candidates in registers (tau15.cuh: halvings of a sub-bracket of the
 //            pages' bracket that still holds the root, stop once the support is fixed, exact
-//            closed-form finish); a row with more candidates than its lists hold gets tau from all
-//            of its scores on CUDA cores (one warp per row, the same solve over 32 lanes);
+//            closed-form finish); candidates past a full list go to a spill area
+//            shared by the CTA, and a row that used it is solved by a whole warp (the bisection over
+//            32 lanes); only if the spill area overflows, tau comes from all of the row's scores,
+//            recomputed on CUDA cores;
 //   pass 3:  S again; P = [(S - tau)/2]_+^2 as bf16 hi + lo parts written back over the S columns
 //            (tcgen05.st); O += P_hi V + P_lo V, A read from TMEM, the V block (M/N-major) from
 //            shared memory;
@@ -40,14 +42,17 @@ constexpr int NSD = 3;                               // input ring stages
 constexpr int CAPD = 32;                             // candidates per row and half
 constexpr int DO_Q = 0;                              // Q tile [128][64] bf16, SW128
 constexpr int DO_RING = DO_Q + TILE_BYTES;           // NSD x (K block, V block)
-constexpr int DO_CV = DO_RING + NSD * 2 * BLK_ROW_BYTES;  // float [2][CAPD][TILE] candidate lists
-constexpr int DO_BITS = DO_CV + 2 * CAPD * TILE * 4; // u32 [MASK_WORDS] valid keys
+constexpr int DO_CV = DO_RING + NSD * 2 * BLK_ROW_BYTES;  // float [2][CAPD + 1][TILE] candidate lists
+constexpr int DO_BITS = DO_CV + 2 * (CAPD + 1) * TILE * 4;  // u32 [MASK_WORDS] valid keys
 constexpr int DO_BLK = DO_BITS + MASK_WORDS * 4;     // u16 [MAX_L / BK] key blocks
 constexpr int DO_TOP = DO_BLK + (MAX_L / BK) * 2;    // float4 [2][TILE] each half's four largest chunk maxima
 constexpr int DO_CNT = DO_TOP + 2 * TILE * 16;       // int [2][TILE] each half's candidate count
 constexpr int DO_ROW = DO_CNT + 2 * TILE * 4;        // float [2][TILE] the row's cut t; -tau/2
 constexpr int DO_OVF = DO_ROW + 2 * TILE * 4;        // u32 [TILE / 32] rows whose lists overflowed
-constexpr int DO_CTL = DO_OVF + 16;
+constexpr int NSP = 512;                             // spill entries: candidates past a full list
+constexpr int DO_SPV = DO_OVF + 16;                  // float [NSP] spilled candidate values
+constexpr int DO_SPR = DO_SPV + NSP * 4;             // u8 [NSP] their rows
+constexpr int DO_CTL = DO_SPR + NSP;
 
 struct FdCtl {
     uint64_t full_q;          // Q tile landed
@@ -61,6 +66,7 @@ struct FdCtl {
     int abort_flag;
     int nblk;
     int nload;
+    int nspill;               // spill entries claimed (may exceed NSP: then the spill area overflowed)
     uint32_t last_bar;
     uint32_t last_par;
 };
@@ -70,6 +76,63 @@ static_assert(DO_TOP % 16 == 0 && DO_CTL % 8 == 0, "alignment");
 static_assert(D_SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
 constexpr int FB_NPL = 16;                           // a fallback row's scores per lane: 512 keys at most
 static_assert(FB_NPL * 32 >= 512 && 3 * 64 >= 128 + 63, "a dense row has at most 512 allowed keys");
+
+// The hits of a 32-value chunk (bit 31 - k <-> value k) past the first `skip` into the CTA's spill
+// area, tagged with their row.  Out of line: it runs only when a row's list is full.
+__device__ __noinline__ void spill_hits(const float (&v)[32], uint32_t hits, int skip, int r, int* nspill,
+                                        float* spv, uint8_t* spr) {
+    for (int k = 0; k < 32; ++k) {
+        if (!((hits >> (31 - k)) & 1u)) continue;
+        if (skip > 0) {
+            --skip;
+            continue;
+        }
+        const int q = atomicAdd(nspill, 1);
+        if (q < NSP) {
+            spv[q] = v[k];
+            spr[q] = (uint8_t)r;
+        }
+    }
+}
+
+// tau (score units) of a row whose lists overflowed, from its candidates: the full lists plus its
+// entries of the spill area, gathered into a warp's registers (lane l takes list entries l, l + 32
+// and spill slots l + 32 q) and solved over 32 lanes.  t_cut: the cut the candidates passed.  Out
+// of line: it runs only for such rows.
+__device__ __noinline__ float solve_spilled_row(const float* cv, const int* cnt, const float* spv, const uint8_t* spr,
+                                                int nsp, int rr, float t_cut, float scale, int lane) {
+    const int m0 = min(cnt[rr], CAPD), m1 = min(cnt[TILE + rr], CAPD);
+    float y[2 + NSP / 32];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const int e = lane + 32 * c;
+        y[c] = e < m0 ? cv[e * TILE + rr] : (e - m0 < m1 ? cv[(CAPD + 1 + e - m0) * TILE + rr] : -INFINITY);
+    }
+#pragma unroll
+    for (int c = 0; c < NSP / 32; ++c) {
+        const int q = lane + 32 * c;
+        y[2 + c] = (q < nsp && spr[q] == rr) ? spv[q] : -INFINITY;
+    }
+    float mx = -INFINITY;
+    int na = 0;
+#pragma unroll
+    for (int c = 0; c < 2 + NSP / 32; ++c) {
+        mx = fmaxf(mx, y[c]);
+        na += y[c] > -INFINITY ? 1 : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        na += __shfl_xor_sync(0xffffffffu, na, o);
+    }
+    const float ms = scale * mx;
+#pragma unroll
+    for (int c = 0; c < 2 + NSP / 32; ++c) y[c] = fmaf(scale, y[c], -ms);  // -inf stays -inf
+    // the candidates are the scores above the cut: a superset of the support
+    const float hi = -2.f / sqrtf((float)max(na, 1));
+    const float lo = fminf(fmaxf(-2.f, fmaf(scale, t_cut, -ms)), hi);
+    return ms + solve_tau_warp<2 + NSP / 32>(y, lo, hi);
+}
 
 __device__ __forceinline__ float bfl(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bfh(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -88,6 +151,8 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
     int* cnt = reinterpret_cast<int*>(smem + DO_CNT);
     float* rowv = reinterpret_cast<float*>(smem + DO_ROW);
     uint32_t* ovf = reinterpret_cast<uint32_t*>(smem + DO_OVF);
+    float* spv = reinterpret_cast<float*>(smem + DO_SPV);
+    uint8_t* spr = smem + DO_SPR;
     FdCtl* ctl = reinterpret_cast<FdCtl*>(smem + DO_CTL);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -112,6 +177,7 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
         mbar_init(smem_u32(&ctl->acc_done), 1);
         ctl->abort_flag = 0;
         ctl->nload = 0;
+        ctl->nspill = 0;
         ctl->last_bar = 0;
         ctl->last_par = 0;
         fence_barrier_init();
@@ -277,7 +343,7 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
         if (g == 0) rowv[r] = t;
 
         // ---- pass 2: candidates s > t into this half's list
-        float* lst = cv + g * CAPD * TILE + r;
+        float* lst = cv + g * (CAPD + 1) * TILE + r;
         int nc = 0;
         for (int n = 0; n < nb && live; ++n) {
             float v[32];
@@ -285,13 +351,15 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
             if (!live) break;
             const uint32_t hits = hit_bits(v, t) & __brev(allowed(n));  // bit 31 - k <-> value k
             if (__any_sync(0xffffffffu, hits != 0u)) {
+                // branch-free append: every value goes to the next free slot (slot CAPD, past the
+                // list, takes the writes of a full list) and the count moves on a hit only
+                const int nc0 = nc;
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
-                    if (hits & (0x80000000u >> k)) {
-                        if (nc < CAPD) lst[nc * TILE] = v[k];
-                        ++nc;
-                    }
+                    lst[min(nc, CAPD) * TILE] = v[k];
+                    nc += (int)((hits >> (31 - k)) & 1u);
                 }
+                if (nc > CAPD) spill_hits(v, hits, max(0, CAPD - nc0), r, &ctl->nspill, spv, spr);  // rare
             }
         }
         cnt[g * TILE + r] = nc;
@@ -310,7 +378,7 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
             float cmax = -INFINITY;
             for (int k = 0; k < ns; ++k) {
                 const int e = 2 * k + h;
-                cmax = fmaxf(cmax, cv[(e < n0 ? e : CAPD + (e - n0)) * TILE + rr]);
+                cmax = fmaxf(cmax, cv[(e < n0 ? e : CAPD + 1 + (e - n0)) * TILE + rr]);
             }
             cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
             const float ms = scale * cmax;
@@ -321,10 +389,10 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
             const float lo = fminf(fmaxf(-2.f, fmaf(scale, tcut, -ms)), hi);
             const int nmax = __reduce_max_sync(0xffffffffu, ns);
             float tau_x;
-            if (nmax <= 8) tau_x = solve_tau<8, CAPD>(cv, rr, h, ns, n0, scale, ms, lo, hi);
-            else if (nmax <= 16) tau_x = solve_tau<16, CAPD>(cv, rr, h, ns, n0, scale, ms, lo, hi);
-            else if (nmax <= 24) tau_x = solve_tau<24, CAPD>(cv, rr, h, ns, n0, scale, ms, lo, hi);
-            else tau_x = solve_tau<CAPD, CAPD>(cv, rr, h, ns, n0, scale, ms, lo, hi);
+            if (nmax <= 8) tau_x = solve_tau<8, CAPD + 1>(cv, rr, h, ns, n0, scale, ms, lo, hi);
+            else if (nmax <= 16) tau_x = solve_tau<16, CAPD + 1>(cv, rr, h, ns, n0, scale, ms, lo, hi);
+            else if (nmax <= 24) tau_x = solve_tau<24, CAPD + 1>(cv, rr, h, ns, n0, scale, ms, lo, hi);
+            else tau_x = solve_tau<CAPD, CAPD + 1>(cv, rr, h, ns, n0, scale, ms, lo, hi);
             // a row with no allowed key (or past L): tau = +inf, so that every weight below is 0
             const float tau = solve ? ms + tau_x : INFINITY;
             if (h == 0 && !over) {
@@ -333,11 +401,15 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
             }
         }
 
-        // ---- rows whose lists overflowed: tau from all of the row's scores, one warp per row
+        // ---- rows whose lists overflowed, one warp per row.  Their candidates are the full lists plus
+        // their entries of the spill area: gathered into the warp's registers (lane l takes list
+        // entries l, l + 32 and spill slots l + 32 q), then solved as above over 32 lanes.  Only if the
+        // spill area itself overflowed, tau comes from all of the row's scores, recomputed on CUDA cores.
         {
             uint32_t wm[TILE / 32];
 #pragma unroll
             for (int q = 0; q < TILE / 32; ++q) wm[q] = ovf[q];
+            const int nsp = ctl->nspill;
             int seen = 0;
             for (int q = 0; q < TILE / 32; ++q) {
                 while (wm[q] && live) {
@@ -345,6 +417,14 @@ entmax_dense_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_
                     wm[q] &= wm[q] - 1u;
                     if ((seen++ & 7) != warp) continue;
                     const int ii = i0 + rr;
+                    if (nsp <= NSP) {
+                        const float tau = solve_spilled_row(cv, cnt, spv, spr, nsp, rr, rowv[rr], scale, lane);
+                        if (lane == 0) {
+                            rowv[TILE + rr] = -0.5f * tau;
+                            out.tau[(size_t)bh * L + ii] = tau;
+                        }
+                        continue;
+                    }
                     int lo_k, hi_k;
                     row_key_range(ii, L, a.causal, a.window, lo_k, hi_k);
                     // Q row from the swizzled tile: 16-byte chunk c of row rr at rr*128 + ((c ^ (rr & 7)) << 4)

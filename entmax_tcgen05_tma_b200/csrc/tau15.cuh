@@ -117,22 +117,34 @@ __device__ __forceinline__ float solve_tau(const float* lcv, int r, int h, int n
     return tau_x;
 }
 
+// Sum of a fixed-point value over the 32 lanes of a warp.
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 // tau of one row whose values x (scaled, shifted so that the row max is 0; -inf where unused) are
 // spread over the 32 lanes of a warp, NPL per lane: the same bisection of [lo, hi] with the
-// every-four-halvings stop and the closed-form finish as solve_tau, with warp-wide sums.
+// every-four-halvings stop and the closed-form finish as solve_tau, with warp-wide sums.  The sums
+// are taken in 64-bit fixed point (2^-40 units; every term lies in [-4, 4] on the bracket, which is
+// inside [-2, 0]): integer addition is associative, so the result does not depend on which lane
+// holds which value.
 template <int NPL>
 __device__ __forceinline__ float solve_tau_warp(const float (&x)[NPL], float lo, float hi) {
+    constexpr float FX = 1099511627776.f;  // 2^40
+    constexpr long long FOUR = 4ll << 40;
     bool settled = false;
     for (int it = 0; it < 25; ++it) {
         const float mid = 0.5f * (lo + hi);
-        float g = 0.f;
+        long long g = 0;
 #pragma unroll
         for (int k = 0; k < NPL; ++k) {
             const float d = fmaxf(x[k] - mid, 0.f);
-            g = fmaf(d, d, g);
+            g += __float2ll_rn(d * d * FX);
         }
-        g = warp_sum(g);
-        if (0.25f * g > 1.f) lo = mid;
+        g = warp_sum_ll(g);
+        if (g > FOUR) lo = mid;
         else hi = mid;
         if ((it & 3) == 3 || it == 24) {
             int und = 0;
@@ -143,23 +155,24 @@ __device__ __forceinline__ float solve_tau_warp(const float (&x)[NPL], float lo,
         }
     }
     const float mid = 0.5f * (lo + hi);
-    float K = 0.f, S1 = 0.f, S2 = 0.f;
+    long long K = 0, S1 = 0, S2 = 0;
 #pragma unroll
     for (int k = 0; k < NPL; ++k) {
         if (x[k] > mid) {
-            K += 1.f;
-            S1 += x[k];
-            S2 = fmaf(x[k], x[k], S2);
+            K += 1;
+            S1 += __float2ll_rn(x[k] * FX);
+            S2 += __float2ll_rn(x[k] * x[k] * FX);
         }
     }
-    K = warp_sum(K);
-    S1 = warp_sum(S1);
-    S2 = warp_sum(S2);
+    K = warp_sum_ll(K);
+    S1 = warp_sum_ll(S1);
+    S2 = warp_sum_ll(S2);
     float tau_x = mid;
-    if (K > 0.f) {
-        const float mu = S1 / K;
-        const float var = fmaxf(S2 / K - mu * mu, 0.f);
-        const float tc = mu - sqrtf(fmaxf(4.f / K - var, 0.f));
+    if (K > 0) {
+        const double kd = (double)K, s1 = (double)S1 / (double)FX, s2 = (double)S2 / (double)FX;
+        const float mu = (float)(s1 / kd);
+        const float var = fmaxf((float)(s2 / kd) - mu * mu, 0.f);
+        const float tc = mu - sqrtf(fmaxf(4.f / (float)K - var, 0.f));
         if (settled) tau_x = fminf(fmaxf(tc, lo), hi);
         else if (tc >= lo && tc <= hi) tau_x = tc;
     }

@@ -200,6 +200,33 @@ def test_uniform_rows_take_the_exact_redo_path(L):
         assert np.max(np.abs(to64(g) - r)) <= GRAD_TOL
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_past_the_candidate_lists(causal):
+    """Rows whose candidates do not fit the tensor-core forward's lists (32 per half row): a zero query
+    row ties every allowed key, so all of them are candidates.  Tile 0 of head 0 has two such rows
+    and tile 1 of head 0 one: their extra candidates fit the CTA's spill area, and a warp solves each
+    row from its lists and its spill entries.  Tile 0 of head 1 has eight: without the causal mask
+    (256 candidates a row) they overflow the spill area and tau comes from the rows' scores
+    recomputed on CUDA cores; with it (about 100 a row) they fit.  Everything is compared with the
+    oracle."""
+    w = Workload(0, "spill", 1, 2, 256, 64, 1 / 8, causal=causal)
+    inp = make_inputs(w, seed=13)
+    Q = inp["Q"]
+    for h, rows in ((0, (90, 117, 200)), (1, range(100, 108))):
+        for r in rows:
+            Q[0, h, r].zero_()
+    d = inputs_f64(inp, False)
+    O, tau, dev = _gpu_fwd(inp, w)
+    O_ref, tau_ref = orc.attn_fwd(d["Q"], d["K"], d["V"], None, causal, 0, w.scale)
+    assert np.max(np.abs(to64(O) - O_ref)) <= O_TOL
+    check_rows(d["Q"], d["K"], np.arange(2 * 256), to64(tau).reshape(-1), tau_ref.reshape(-1), None, causal, 0,
+               w.scale, 2, 256)
+    dQ, dK, dV = _gpu_bwd(dev, tau, inp["dO"], w)
+    refs = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], None, causal, 0, w.scale)
+    for g, r in zip((dQ, dK, dV), refs):
+        assert np.max(np.abs(to64(g) - r)) <= GRAD_TOL
+
+
 def test_one_hot_rows():
     """A key aligned with every query and far above the rest takes all the weight."""
     w = Workload(0, "onehot", 1, 1, 256, 64, 1.0)
