@@ -200,12 +200,15 @@ def oracle_baseline(w: Workload, inp: dict, budget_s: float = 12.0, max_heads: i
 
 
 def host_link_rates(dev, stream, nbytes: int = 1 << 28, reps: int = 5) -> dict:
-    """Pinned host-to-device and device-to-host copy rates (GB/s) of this GPU's host link, one
-    direction at a time, timed with CUDA events on `stream`: the ceiling of the end-to-end copies.
-    Runs outside every timed region; any failure is reported instead of the rates."""
+    """Pinned copy rates (GB/s) of this GPU's host link, timed with CUDA events: host-to-device and
+    device-to-host one direction at a time, then both at once on two streams ("duplex_gbs", bytes
+    of both directions over the time both took) -- the ceilings of the end-to-end copies.  Runs
+    outside every timed region; any failure is reported instead of the rates."""
     try:
         h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
         d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        h2 = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+        d2 = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         rates = {}
         with torch.cuda.stream(stream):
             for name, dst, src in (("h2d_gbs", d, h), ("d2h_gbs", h, d)):
@@ -217,17 +220,34 @@ def host_link_rates(dev, stream, nbytes: int = 1 << 28, reps: int = 5) -> dict:
                 e1.record(stream)
                 e1.synchronize()
                 rates[name] = round(nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9, 2)
+        other = torch.cuda.Stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        other.wait_event(e0)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                d.copy_(h, non_blocking=True)
+        with torch.cuda.stream(other):
+            for _ in range(reps):
+                h2.copy_(d2, non_blocking=True)
+        stream.wait_stream(other)
+        e1.record(stream)
+        e1.synchronize()
+        rates["duplex_gbs"] = round(2 * nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9, 2)
         return rates
     except Exception as exc:  # a measurement aid only: never fail the bench line for it
         return {"error": repr(exc)[:200]}
 
 
 def link_bound(rates: dict, h2d_bytes: int, d2h_bytes: int, e2e_ms: float) -> dict:
-    """The end-to-end step against its copy time: the two directions run on separate copy engines,
-    so the bound is the slower direction's bytes over its measured rate."""
+    """The end-to-end step against its copy time: each direction's bytes over its own rate, and the
+    bytes of both over the rate the link sustains with both directions busy; the bound is the
+    largest of the three."""
     if not (rates.get("h2d_gbs", 0) > 0 and rates.get("d2h_gbs", 0) > 0 and e2e_ms > 0):
         return dict(rates)
     bound_ms = 1e3 * max(h2d_bytes / (rates["h2d_gbs"] * 1e9), d2h_bytes / (rates["d2h_gbs"] * 1e9))
+    if rates.get("duplex_gbs", 0) > 0:
+        bound_ms = max(bound_ms, 1e3 * (h2d_bytes + d2h_bytes) / (rates["duplex_gbs"] * 1e9))
     return {**rates, "copy_bound_ms": round(bound_ms, 4), "frac": round(bound_ms / e2e_ms, 4)}
 
 
@@ -479,22 +499,33 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         h2d -= host_in["dO"].numel() * host_in["dO"].element_size()
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     e2e_steps = max(3, min(args.steps, 20))
-    # The step's batch in up to four chunks of whole sequences, alternating over two streams: each
-    # chunk's host-to-device copies, its calls and its device-to-host copies are queued on its
-    # stream, so one chunk's copies overlap another's kernels (the two copy directions run on
-    # separate engines).  Every byte of the step still crosses PCIe inside the timed region.
-    nchunk = min(w.B, 4)
-    cuts = [w.B * c // nchunk for c in range(nchunk + 1)]
-    chunks = [(cuts[c], cuts[c + 1]) for c in range(nchunk)]
+    # The step's batch in chunks, alternating over two streams: each chunk's host-to-device copies,
+    # its calls and its device-to-host copies are queued on its stream, so one chunk's copies
+    # overlap another's kernels (the two copy directions run on separate engines), and only the
+    # first chunk's inputs and the last chunk's outputs cross PCIe with nothing beside them.  A chunk
+    # is a run of whole sequences or, with fewer sequences than chunks, a group of heads of one
+    # sequence (contiguous in [B, H, L, 64] memory; plain heads only).  Every byte of the step still
+    # crosses PCIe inside the timed region.
+    target = max(1, args.e2e_chunks)
+    if w.B >= target or Hkv != H or args.blhd:
+        nb_ = min(w.B, target)
+        cuts = [w.B * c // nb_ for c in range(nb_ + 1)]
+        chunks = [(cuts[c], cuts[c + 1], 0, H) for c in range(nb_)]
+    else:
+        ng = min(H, -(-target // w.B))
+        hc = [H * g // ng for g in range(ng + 1)]
+        chunks = [(b, b + 1, hc[g], hc[g + 1]) for b in range(w.B) for g in range(ng)]
+    nchunk = len(chunks)
     e2e_streams = [torch.cuda.Stream(dev) for _ in range(2)]
-    bmax = max(b1 - b0 for b0, b1 in chunks)
-    e2e_saved = [torch.empty((E.entmax_attn_saved_bytes(bmax, H, L, D),), dtype=torch.uint8, device=dev)
+    bmax = max(c[1] - c[0] for c in chunks)
+    hmax = max(c[3] - c[2] for c in chunks)
+    e2e_saved = [torch.empty((E.entmax_attn_saved_bytes(bmax, hmax, L, D),), dtype=torch.uint8, device=dev)
                  for _ in e2e_streams]
-    e2e_ws = [torch.empty((E.entmax_attn_bwd_saved_workspace_size(bmax, H, L, D),), dtype=torch.uint8, device=dev)
-              for _ in e2e_streams]
+    e2e_ws = [torch.empty((E.entmax_attn_bwd_saved_workspace_size(bmax, hmax, L, D),), dtype=torch.uint8,
+                          device=dev) for _ in e2e_streams]
 
-    def e2e_chunk(b0, b1, k):
-        hin = {n: t[b0:b1] for n, t in host_in.items()}
+    def e2e_chunk(b0, b1, h0, h1, k):
+        hin = {n: (t[b0:b1] if (h0, h1) == (0, H) else t[b0:b1, h0:h1]) for n, t in host_in.items()}
         Qd = hin["Q"].to(dev, non_blocking=True)
         Kd = hin["K"].to(dev, non_blocking=True)
         Vd = hin["V"].to(dev, non_blocking=True)
@@ -511,8 +542,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             Oo, to, sv = E.entmax_attn_fwd_train(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale, saved=sv_buf)
         else:
             Oo, to = E.entmax_attn_fwd(Qd, Kd, Vd, kmd, w.causal, w.window, w.scale)
-        host_out["O"][b0:b1].copy_(Oo, non_blocking=True)
-        host_out["tau"][b0:b1].copy_(to, non_blocking=True)
+        host_out["O"][b0:b1, h0:h1].copy_(Oo, non_blocking=True)
+        host_out["tau"][b0:b1, h0:h1].copy_(to, non_blocking=True)
         if w.backward:
             dOd = hin["dO"].to(dev, non_blocking=True)
             if recompute:
@@ -524,15 +555,15 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                 g = E.entmax_attn_bwd_saved(Qd, Kd, Vd, to, sv, dOd, kmd, w.causal, w.window, w.scale,
                                             workspace=ws_buf)
             for name, t in zip(("dQ", "dK", "dV"), g):
-                host_out[name][b0:b1].copy_(t, non_blocking=True)
+                host_out[name][b0:b1, h0:h1].copy_(t, non_blocking=True)
 
     def e2e_step(start_event):
         for k, s in enumerate(e2e_streams):
             s.wait_event(start_event)
-        for c, (b0, b1) in enumerate(chunks):
+        for c, (b0, b1, h0, h1) in enumerate(chunks):
             k = c % len(e2e_streams)
             with torch.cuda.stream(e2e_streams[k]):
-                e2e_chunk(b0, b1, k)
+                e2e_chunk(b0, b1, h0, h1, k)
         for s in e2e_streams:
             stream.wait_stream(s)
 
@@ -645,7 +676,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "gpu_launches": launches_per_step(w, recompute, alpha) * args.steps,
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "chunks": "%d chunks of whole sequences on 2 streams (copies overlap kernels)" % nchunk,
+                "chunks": "%d chunks (%s) on 2 streams (copies overlap kernels)" % (
+                    nchunk, "whole sequences" if chunks[0][2:] == (0, H) else "head groups of one sequence"),
                 "host_link": link_bound(link, h2d, d2h, e2e_ms)},
         "clocks": clocks,
     }
@@ -767,6 +799,8 @@ def main() -> int:
     ap.add_argument("--blhd", action="store_true", help="variant: tensors in [B, L, H, 64] memory")
     ap.add_argument("--fp32-inputs", action="store_true",
                     help="variant: Q, K, V, dO given as fp32 (the library rounds them to bf16 on the device)")
+    ap.add_argument("--e2e-chunks", type=int, default=4,
+                    help="end-to-end step: chunks of the batch whose copies overlap other chunks' kernels")
     ap.add_argument("--bwd", default="saved", choices=["saved", "recompute"],
                     help="backward path: from the forward's saved supports, or entmax_attn_bwd (scores recomputed)")
     args = ap.parse_args()

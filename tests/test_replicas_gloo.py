@@ -140,6 +140,12 @@ def test_link_bound_takes_the_slower_direction():
     r = bench.link_bound({"h2d_gbs": 10.0, "d2h_gbs": 40.0}, 100_000_000, 200_000_000, 20.0)
     assert r["copy_bound_ms"] == pytest.approx(10.0) and r["frac"] == pytest.approx(0.5)
     assert bench.link_bound({"error": "x"}, 1, 1, 1.0) == {"error": "x"}
+    # both directions at once at 50 GB/s in total: 300 MB take 6 ms, above either direction alone
+    r = bench.link_bound({"h2d_gbs": 50.0, "d2h_gbs": 40.0, "duplex_gbs": 50.0}, 100_000_000, 200_000_000, 12.0)
+    assert r["copy_bound_ms"] == pytest.approx(6.0) and r["frac"] == pytest.approx(0.5)
+    # a full-duplex link leaves the slower direction as the bound
+    r = bench.link_bound({"h2d_gbs": 50.0, "d2h_gbs": 40.0, "duplex_gbs": 90.0}, 100_000_000, 200_000_000, 10.0)
+    assert r["copy_bound_ms"] == pytest.approx(5.0)
 
 
 def test_link_rates_report_failure_instead_of_raising():
