@@ -64,19 +64,25 @@ __device__ __forceinline__ float solve_tau(const float* lcv, int r, int h, int n
         const int e = 2 * k + h;  // entry e of the row's two lists, partition 0's n0 entries first
         x[k] = k < nh ? fmaf(scale, lcv[(e < n0 ? e : CAPW + (e - n0)) * TILE + r], -ms) : -INFINITY;
     }
+    // the candidates as packed pairs: a halving costs a packed subtraction, two maxima and a packed
+    // fma per pair
+    uint64_t x2[NC / 2];
+#pragma unroll
+    for (int k = 0; k < NC; k += 2) x2[k >> 1] = f2pack(x[k], x[k + 1]);
     bool settled = false;
     for (int it = 0; it < 25; ++it) {
         const float mid = 0.5f * (lo + hi);
-        float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
+        const uint64_t mid2 = f2pack(mid, mid);
+        uint64_t ga = 0, gb = 0;
 #pragma unroll
-        for (int k = 0; k < NC; k += 4) {
-            const float d0 = fmaxf(x[k] - mid, 0.f), d1 = fmaxf(x[k + 1] - mid, 0.f);
-            const float d2 = fmaxf(x[k + 2] - mid, 0.f), d3 = fmaxf(x[k + 3] - mid, 0.f);
-            g0 = fmaf(d0, d0, g0);
-            g1 = fmaf(d1, d1, g1);
-            g2 = fmaf(d2, d2, g2);
-            g3 = fmaf(d3, d3, g3);
+        for (int k = 0; k < NC / 2; k += 2) {
+            const uint64_t da = f2relu(f2sub(x2[k], mid2)), db = f2relu(f2sub(x2[k + 1], mid2));
+            ga = f2fma(da, da, ga);
+            gb = f2fma(db, db, gb);
         }
+        float g0, g1, g2, g3;
+        f2unpack(ga, g0, g1);
+        f2unpack(gb, g2, g3);
         float gs = (g0 + g1) + (g2 + g3);
         gs += __shfl_xor_sync(0xffffffffu, gs, 1);
         if (0.25f * gs > 1.f) lo = mid;
