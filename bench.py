@@ -361,13 +361,14 @@ def tensor_core_backward(w: Workload, alpha: float = 1.5) -> bool:
 
 def launches_per_step(w: Workload, recompute: bool, alpha: float = 1.5) -> int:
     """The library's kernel launches in one step: the forward kernel, then the backward's kernels
-    (tensor-core configurations: dq and dkdv; otherwise saved supports: key scan, rows, keys and the
-    exact pass for unsaved rows, or, recomputing the scores: rows and keys)."""
+    (tensor-core configurations: dq and dkdv; otherwise the support-list backward: key scan, rows,
+    keys and the exact pass for unsaved rows -- which entmax_attn_bwd, given its full workspace,
+    precedes by the training forward that rebuilds the supports)."""
     if not w.backward:
         return 1
     if tensor_core_backward(w, alpha):
         return 3
-    return 1 + (2 if recompute else 4)
+    return 1 + (5 if recompute else 4)
 
 
 def time_device(prep: _Prepared, flush: _Flush, steps: int, warmup: int, world: int) -> dict:
@@ -665,7 +666,8 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         if variant or w.fp32_inputs else None,
         "backward": ("entmax_attn_bwd" if recompute else "entmax_attn_bwd_saved") + (
             " (tensor-core kernels: scores recomputed, every product on tcgen05)" if tensor_core_backward(w, alpha)
-            else " (scores recomputed)" if recompute else " (saved supports)"),
+            else " (supports rebuilt by the training forward, then the support-list backward)" if recompute
+            else " (saved supports)"),
         "fwd_ms": round(fwd_mean, 4),
         "bwd_ms": round(bwd_mean, 4),
         "step_ms_median": round(statistics.median(step_ms), 4),

@@ -2,7 +2,8 @@
 
 Multi-head attention whose softmax is replaced by Tsallis 1.5-entmax: per query row,
 tau solves sum_j max(0, (S_ij - tau)/2)^2 = 1 by bisection, A = max(0, (S - tau)/2)^2 has exact
-zeros, O = A V; the backward pass uses the closed-form Jacobian.  The work runs in hand-written
+zeros, O = A V; the backward pass uses the closed-form Jacobian.  The _ex entry points take any
+alpha in [1, 2] (alpha within 1e-4 of 1: softmax).  The work runs in hand-written
 sm_100a kernels (tcgen05 tensor cores, TMEM, TMA) behind the C ABI in include/entmax_attn.h;
 this package is its thin Python binding.
 """
@@ -21,6 +22,7 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     EntmaxAttention,
     EntmaxError,
+    bwd_min_workspace_size,
     entmax_attn_bwd,
     entmax_attn_bwd_aux,
     entmax_attn_bwd_noalloc,

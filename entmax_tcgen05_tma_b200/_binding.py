@@ -264,8 +264,15 @@ def entmax_attn_fwd_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=No
 
 
 def entmax_attn_bwd_workspace_size(B: int, H: int, L: int, D: int = 64) -> int:
-    """Bytes of device workspace entmax_attn_bwd needs (one float per query row, rounded up)."""
+    """Bytes of device workspace for entmax_attn_bwd's fastest path (long rows rebuild the forward's
+    supports in it); the minimum it accepts is bwd_min_workspace_size."""
     return int(lib.entmax_attn_bwd_workspace_size(B, H, L, D))
+
+
+def bwd_min_workspace_size(B: int, H: int, L: int) -> int:
+    """The smallest workspace entmax_attn_bwd and entmax_attn_bwd_aux accept: one float per query
+    row, rounded up to 256 bytes."""
+    return (B * H * L * 4 + 255) // 256 * 256
 
 
 def entmax_attn_bwd(Q, K, V, tau, dO, key_mask=None, causal=False, window=0, scale=None, dQ=None, dK=None,
@@ -376,7 +383,7 @@ def entmax_attn_bwd_aux(Q, K, V, tau, Otil, rsum, dO, key_mask=None, causal=Fals
         else:
             _check_input(name, t, (B, H, L, D), torch.float32)
         outs.append(t)
-    ws_bytes = entmax_attn_bwd_workspace_size(B, H, L, D)
+    ws_bytes = bwd_min_workspace_size(B, H, L)  # the auxiliary rows' path needs the minimum only
     if workspace is None:
         workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=Q.device)
     st = lib.entmax_attn_bwd_aux(Q.data_ptr(), K.data_ptr(), V.data_ptr(), _dtype_code(Q),

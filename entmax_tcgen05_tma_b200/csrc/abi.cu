@@ -93,6 +93,18 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16*
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+size_t align256b(size_t n) { return (n + 255) & ~size_t(255); }
+
+// entmax_attn_bwd's workspace: the minimum holds one float per row (the row scalar u_i); with
+// room for the forward's outputs and saved supports and the saved backward's buckets, rows that
+// are not on the tensor-core path rebuild the supports with the training forward and take the
+// support-list backward.
+size_t bwd_min_ws_bytes(long long R) { return align256b((size_t)R * sizeof(float)); }
+size_t bwd_rebuild_ws_bytes(long long R) {
+    return align256b((size_t)R * HEAD_DIM * 2) + align256b((size_t)R * 4) + saved_support_bytes(R) +
+           saved_bwd_ws_bytes(R);
+}
+
 int check_common(const void* Q, const void* K, const void* V, int in_dtype, int causal, int window, float scale,
                  int B, int H, int L, int D) {
     if (B < 0 || H < 0 || L < 0) return ENTMAX_ERR_ARG;
@@ -308,7 +320,9 @@ int entmax_attn_fwd_gqa(const void* Q, const void* K, const void* V, int in_dtyp
 size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D) {
     (void)D;
     if (B <= 0 || H <= 0 || L <= 0) return 0;
-    return (((size_t)B * H * L * sizeof(float)) + 255) & ~size_t(255);
+    const long long R = (long long)B * H * L;
+    // rows of at most 512 keys always take the tensor-core backward, which needs the minimum only
+    return L <= 512 ? bwd_min_ws_bytes(R) : std::max(bwd_min_ws_bytes(R), bwd_rebuild_ws_bytes(R));
 }
 
 }  // extern "C"
@@ -324,7 +338,8 @@ int bwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
     if (!tau || !dO || !dQ || !dK || !dV) return ENTMAX_ERR_ARG;
     if (!aligned(dO, 16) || !aligned(dQ, 8) || !aligned(dK, 8) || !aligned(dV, 8) || !aligned(tau, 4))
         return ENTMAX_ERR_ARG;
-    if (!workspace || ws_bytes < entmax_attn_bwd_workspace_size(B, H, L, D)) return ENTMAX_ERR_WORKSPACE;
+    const long long R = (long long)B * H * L;
+    if (!workspace || ws_bytes < bwd_min_ws_bytes(R)) return ENTMAX_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return ENTMAX_ERR_ARG;
     int* status = nullptr;
     rc = record(status_ptr(&status));
@@ -344,9 +359,32 @@ int bwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
         a.V = dst[2];
         io.dO = dst[3];
     }
-    // the tensor-core kernels store gradient rows 16 bytes at a time
-    const bool dense = dense_bwd(a) && aligned(dQ, 16) && aligned(dK, 16) && aligned(dV, 16);
-    return record(dense ? launch_bwd_dense(a, io, stream) : launch_bwd(a, io, stream));
+    // the tensor-core kernels and the support-list backward store gradient rows 16 bytes at a time
+    const bool g16 = aligned(dQ, 16) && aligned(dK, 16) && aligned(dV, 16);
+    if (dense_bwd(a) && g16) return record(launch_bwd_dense(a, io, stream));
+    if (!otil && g16 && ws_bytes >= bwd_rebuild_ws_bytes(R) && aligned(workspace, 256)) {
+        // Rebuild the forward's supports: the training forward (deterministic, so its tau is the
+        // caller's bit for bit) into scratch O, tau and support lists, then the support-list backward.
+        uint8_t* p = static_cast<uint8_t*>(workspace);
+        void* o_s = p;
+        p += align256b((size_t)R * HEAD_DIM * 2);
+        float* tau_s = reinterpret_cast<float*>(p);
+        p += align256b((size_t)R * 4);
+        const SavedSupport sv = carve_saved(p, R);
+        p += saved_support_bytes(R);
+        rc = record(cudaMemsetAsync(sv.key_cnt, 0, sizeof(int) * (size_t)R, stream));
+        if (rc) return rc;
+        rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
+        if (rc) return rc;
+        FwdOut o{o_s, 0, tau_s, sv};
+        rc = record(launch_fwd(a, o, stream));
+        if (rc) return rc;
+        io.tau = tau_s;
+        io.u = nullptr;
+        io.guard = status;  // if that forward gave up, its lists hold anything: the backward does nothing
+        return record(launch_bwd_saved(a, io, sv, carve_saved_bwd_ws(p, R), stream));
+    }
+    return record(launch_bwd(a, io, stream));
 }
 }  // namespace
 

@@ -31,8 +31,13 @@ namespace {
 
 constexpr int ROW_WARPS = 8;  // warps per CTA of the rows / keys kernels
 
+// Whether the support-list backward must do nothing: the forward that wrote its lists in the same
+// call gave up (a recorded device error), so the lists may hold anything.
+__device__ __forceinline__ bool guarded(const int* guard) { return guard && *(volatile const int*)guard != 0; }
+
 __global__ void __launch_bounds__(1024) key_scan_kernel(const int* __restrict__ key_cnt, int* __restrict__ key_off,
-                                                        int* __restrict__ key_cur, int L) {
+                                                        int* __restrict__ key_cur, int L, const int* guard) {
+    if (guarded(guard)) return;
     __shared__ int wsum[32];
     const size_t base = (size_t)blockIdx.x * L;
     const int per = (L + 1023) / 1024;
@@ -285,6 +290,7 @@ __device__ __forceinline__ void keys_group(const AttnArgs& a, const BwdIO& io, c
 template <bool GEN, bool PLAIN>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
+    if (guarded(io.guard)) return;
     __shared__ uint16_t lj[ROW_WARPS][RPW][SAVE_CAP];
     __shared__ float lsp[ROW_WARPS][RPW][SAVE_CAP];
     __shared__ float lds[ROW_WARPS][RPW][SAVE_CAP];  // dA, then dS
@@ -323,6 +329,7 @@ template <bool GEN, bool PLAIN, int SPLIT>
 __global__ void __launch_bounds__(ROW_WARPS * 32) saved_keys_kernel(const AttnArgs a, const BwdIO io,
                                                                     const SavedSupport sv, const SavedBwdWs ws) {
     static_assert(SPLIT == 1 || SPLIT == 2 || SPLIT == 4, "lane groups per key");
+    if (guarded(io.guard)) return;
     constexpr int KPW = RPW / SPLIT;  // keys per warp
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = lane >> 3, sd = lane & 7, g0 = lane & ~7;
@@ -381,6 +388,7 @@ __device__ __forceinline__ float dot64_f32(const float* a, const __nv_bfloat16* 
 template <bool GEN>
 __global__ void __launch_bounds__(UNSAVED_THREADS) unsaved_rows_kernel(const AttnArgs a, const BwdIO io,
                                                                       const SavedSupport sv) {
+    if (guarded(io.guard)) return;
     extern __shared__ float sbuf[];  // [L]: b_ij = am1 (S_ij - tau_i) (sqrt(p_ij) at alpha 1.5); [L, 2L): dA_ij
     const float am1 = a.am1, em1 = 1.f / am1 - 1.f;
     __shared__ float red[UNSAVED_THREADS];
@@ -507,7 +515,7 @@ SavedBwdWs carve_saved_bwd_ws(void* base, long long R) {
 cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupport& sv, const SavedBwdWs& ws,
                              cudaStream_t stream) {
     const long long R = (long long)a.B * a.H * a.L;
-    key_scan_kernel<<<a.B * a.Hkv, 1024, 0, stream>>>(sv.key_cnt, ws.key_off, ws.key_cur, a.L);
+    key_scan_kernel<<<a.B * a.Hkv, 1024, 0, stream>>>(sv.key_cnt, ws.key_off, ws.key_cur, a.L, io.guard);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;

@@ -87,6 +87,8 @@ struct BwdIO {
     const float* otil;       // optional [B*H*L][64]: the forward's sum_j w_ij V_j (logical row order)
     const float* rsum;       // optional [B*H*L]: the forward's sum_j w_ij; with otil, u_i = dO_i . otil_i / rsum_i
                              // (softmax: rsum = 1, passed as null)
+    const int* guard;        // optional (support-list backward): the device status word; when it is set
+                             // (the forward that wrote the lists gave up), the kernels do nothing
 };
 
 // Workspace of the support-list backward.

@@ -17,6 +17,7 @@ from entmax_tcgen05_tma_b200 import (
     entmax_attn_fwd,
     entmax_attn_fwd_train,
 )
+import entmax_tcgen05_tma_b200 as E
 from entmax_tcgen05_tma_b200.workloads import WORKLOADS, Workload, make_inputs
 from oracle import oracle as orc
 from tests.gpu_helpers import GRAD_TOL, O_TOL, assert_bf16_is_rounded, check_rows, inputs_f64, to64
@@ -225,6 +226,29 @@ def test_rows_past_the_candidate_lists(causal):
     refs = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], None, causal, 0, w.scale)
     for g, r in zip((dQ, dK, dV), refs):
         assert np.max(np.abs(to64(g) - r)) <= GRAD_TOL
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_recompute_backward_both_workspaces(causal):
+    """Long rows through entmax_attn_bwd: with the full workspace the supports are rebuilt by the
+    training forward and the support-list backward runs; with the minimum one float per row the
+    recompute kernels run.  Both against the oracle, and against each other."""
+    w = Workload(0, "recompute", 2, 2, 900, 64, 1 / 8, causal=causal, len_range=(500, 900))
+    inp = make_inputs(w, seed=29)
+    d = inputs_f64(inp, False)
+    km = _mask_np(inp)
+    O, tau, dev = _gpu_fwd(inp, w)
+    Q, K, V, kmd = dev
+    dO = inp["dO"].to(DEV)
+    full = entmax_attn_bwd(Q, K, V, tau, dO, kmd, causal, 0, w.scale)
+    ws = torch.empty(E.bwd_min_workspace_size(w.B, w.H, w.L), dtype=torch.uint8, device=DEV)
+    small = entmax_attn_bwd(Q, K, V, tau, dO, kmd, causal, 0, w.scale, workspace=ws)
+    assert entmax_attn_device_status() == 0
+    refs = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], km, causal, 0, w.scale)
+    for name, a, b, r in zip(("dQ", "dK", "dV"), full, small, refs):
+        assert np.max(np.abs(to64(a) - r)) <= GRAD_TOL, name
+        assert np.max(np.abs(to64(b) - r)) <= GRAD_TOL, name
+        assert torch.allclose(a, b, atol=1e-4, rtol=0), (name, float((a - b).abs().max()))
 
 
 def test_one_hot_rows():

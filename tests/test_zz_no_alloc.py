@@ -25,7 +25,10 @@ def _run(w: Workload, seed: int):
     Q, K, V, dO = (inp[k].cuda() for k in ("Q", "K", "V", "dO"))
     km = None if inp["key_mask"] is None else inp["key_mask"].cuda()
     O, tau = E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale)
-    ref = E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale)
+    # the minimum workspace: entmax_attn_bwd then runs the kernels the allocation-free entry point
+    # runs at every length (with the full workspace, long rows rebuild the forward's supports)
+    ws = torch.empty(E.bwd_min_workspace_size(w.B, w.H, w.L), dtype=torch.uint8, device="cuda")
+    ref = E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, workspace=ws)
     got = E.entmax_attn_bwd_noalloc(Q, K, V, tau, dO, km, w.causal, w.window, w.scale)
     assert E.entmax_attn_device_status() == 0
     for a, b in zip(ref, got):
@@ -36,7 +39,9 @@ def _run(w: Workload, seed: int):
 def test_noalloc_matches_workspace_backward_twice():
     big = Workload(0, "noalloc-1", 1, 4, 520, 64, 1 / 8, causal=True, window=32)
     small = Workload(0, "noalloc-2", 2, 3, 300, 64, 1 / 8, len_range=(100, 300))
+    long = Workload(0, "noalloc-3", 1, 2, 700, 64, 1 / 8)  # long rows: the recompute kernels
     assert big.B * big.H * big.L > small.B * small.H * small.L
+    _run(long, seed=23)
     _run(big, seed=22)
     # the second, smaller call: the array still holds the first call's values past its rows
     inp, got = _run(small, seed=21)
