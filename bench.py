@@ -300,7 +300,9 @@ class _Prepared:
         self.E, self.w, self.dev = E, w, dev
         alpha = args.alpha if alpha is None else alpha
         self.variant = variant = alpha != 1.5 or w.kv_heads != w.H or args.blhd  # the _ex entry points
-        self.recompute = recompute = args.bwd == "recompute"  # entmax_attn_fwd + entmax_attn_bwd
+        # entmax_attn_fwd + entmax_attn_bwd: with its full workspace, or with the minimum (one float per
+        # row), which runs the recompute kernels at long rows
+        self.recompute = recompute = args.bwd in ("recompute", "recompute-min")
         self.inp = inp = make_inputs(w)
         self.pairs = allowed_pairs(w, inp["key_mask"])
         self.flops = dense_equiv_flops(w, self.pairs)
@@ -316,8 +318,9 @@ class _Prepared:
         self.dK, self.dV = (lay(torch.empty((B, Hkv, L, D), dtype=torch.float32, device=dev)) for _ in range(2))
         self.saved = torch.empty((E.entmax_attn_saved_bytes(B, H, L, D),), dtype=torch.uint8, device=dev)
         self.ws = torch.empty((E.entmax_attn_bwd_saved_workspace_size(B, H, L, D),), dtype=torch.uint8, device=dev)
-        self.rws = torch.empty((max(E.entmax_attn_bwd_workspace_size(B, H, L, D), 1),), dtype=torch.uint8,
-                               device=dev)
+        rws = E.bwd_min_workspace_size(B, H, L) if args.bwd == "recompute-min" else \
+            E.entmax_attn_bwd_workspace_size(B, H, L, D)
+        self.rws = torch.empty((max(rws, 1),), dtype=torch.uint8, device=dev)
         self.alpha = alpha
 
     def fwd_call(self):
@@ -359,16 +362,19 @@ def tensor_core_backward(w: Workload, alpha: float = 1.5) -> bool:
     return alpha == 1.0 or (alpha == 1.5 and (w.L <= 512 or (w.causal and 0 < w.window <= 128)))
 
 
-def launches_per_step(w: Workload, recompute: bool, alpha: float = 1.5) -> int:
+def launches_per_step(w: Workload, recompute: bool, alpha: float = 1.5, minimum: bool = False) -> int:
     """The library's kernel launches in one step: the forward kernel, then the backward's kernels
     (tensor-core configurations: dq and dkdv; otherwise the support-list backward: key scan, rows,
     keys and the exact pass for unsaved rows -- which entmax_attn_bwd, given its full workspace,
-    precedes by the training forward that rebuilds the supports)."""
+    precedes by the training forward that rebuilds the supports; with the minimum workspace its
+    recompute kernels, rows and keys)."""
     if not w.backward:
         return 1
     if tensor_core_backward(w, alpha):
         return 3
-    return 1 + (5 if recompute else 4)
+    if recompute:
+        return 1 + (2 if minimum else 5)
+    return 1 + 4
 
 
 def time_device(prep: _Prepared, flush: _Flush, steps: int, warmup: int, world: int) -> dict:
@@ -524,6 +530,9 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                  for _ in e2e_streams]
     e2e_ws = [torch.empty((E.entmax_attn_bwd_saved_workspace_size(bmax, hmax, L, D),), dtype=torch.uint8,
                           device=dev) for _ in e2e_streams]
+    rws_bytes = (E.bwd_min_workspace_size(bmax, hmax, L) if args.bwd == "recompute-min"
+                 else E.entmax_attn_bwd_workspace_size(bmax, hmax, L, D)) if recompute else 1
+    e2e_rws = [torch.empty((max(rws_bytes, 1),), dtype=torch.uint8, device=dev) for _ in e2e_streams]
 
     def e2e_chunk(b0, b1, h0, h1, k):
         hin = {n: (t[b0:b1] if (h0, h1) == (0, H) else t[b0:b1, h0:h1]) for n, t in host_in.items()}
@@ -548,7 +557,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         if w.backward:
             dOd = hin["dO"].to(dev, non_blocking=True)
             if recompute:
-                g = E.entmax_attn_bwd(Qd, Kd, Vd, to, dOd, kmd, w.causal, w.window, w.scale)
+                g = E.entmax_attn_bwd(Qd, Kd, Vd, to, dOd, kmd, w.causal, w.window, w.scale, workspace=e2e_rws[k])
             elif variant:
                 g = E.entmax_attn_bwd_saved_ex(Qd, Kd, Vd, to, sv, dOd, kmd, w.causal, w.window, w.scale, alpha=alpha,
                                                workspace=ws_buf)
@@ -666,6 +675,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         if variant or w.fp32_inputs else None,
         "backward": ("entmax_attn_bwd" if recompute else "entmax_attn_bwd_saved") + (
             " (tensor-core kernels: scores recomputed, every product on tcgen05)" if tensor_core_backward(w, alpha)
+            else " (recompute kernels: minimum workspace)" if args.bwd == "recompute-min"
             else " (supports rebuilt by the training forward, then the support-list backward)" if recompute
             else " (saved supports)"),
         "fwd_ms": round(fwd_mean, 4),
@@ -675,7 +685,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "sparsity": round(sparsity, 4),
         "roofline": roof,
         "step_roofline": step_roof,
-        "gpu_launches": launches_per_step(w, recompute, alpha) * args.steps,
+        "gpu_launches": launches_per_step(w, recompute, alpha, args.bwd == "recompute-min") * args.steps,
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "chunks": "%d chunks (%s) on 2 streams (copies overlap kernels)" % (
@@ -803,14 +813,15 @@ def main() -> int:
                     help="variant: Q, K, V, dO given as fp32 (the library rounds them to bf16 on the device)")
     ap.add_argument("--e2e-chunks", type=int, default=4,
                     help="end-to-end step: chunks of the batch whose copies overlap other chunks' kernels")
-    ap.add_argument("--bwd", default="saved", choices=["saved", "recompute"],
-                    help="backward path: from the forward's saved supports, or entmax_attn_bwd (scores recomputed)")
+    ap.add_argument("--bwd", default="saved", choices=["saved", "recompute", "recompute-min"],
+                    help="backward path: from the forward's saved supports, or entmax_attn_bwd with its full "
+                         "workspace (long rows rebuild the supports) or with the minimum one (recompute kernels)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if not (args.alpha == 1.0 or 1.0 < args.alpha <= 2.0):
         ap.error("--alpha must be 1 (softmax) or lie in (1, 2]")
-    if args.bwd == "recompute" and (args.alpha != 1.5 or args.hkv or args.blhd):
+    if args.bwd != "saved" and (args.alpha != 1.5 or args.hkv or args.blhd):
         ap.error("--bwd recompute takes the plain path only (alpha 1.5, H_kv = H, [B, H, L, 64])")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
