@@ -514,6 +514,7 @@ int bwd_saved_impl(const void* Q, const void* K, const void* V, int in_dtype, co
     const size_t n = (size_t)R * HEAD_DIM;
     AttnArgs a{Q, K, V, key_mask, B, H, L, causal, window, scale, status, timeout_ns(), Hkv, am1, layout};
     BwdIO io{tau, dO, dQ, dK, dV, nullptr};
+    io.guard = status;  // a recorded device error (a forward that gave up): its lists are not read
     Bf16Copies tmp;
     if (in_dtype == ENTMAX_F32) {
         const void* src[4] = {Q, K, V, dO};

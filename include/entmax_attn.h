@@ -182,6 +182,10 @@ ENTMAX_API int entmax_attn_bwd_aux(const void* Q, const void* K, const void* V, 
  * the backward recomputes the scores on tcgen05 and reads nothing from `saved` but its size; every
  * output is then the same bit for bit from run to run.  Elsewhere dK and dV are summed in an order
  * that depends on scheduling (last-bit differences between runs); dQ, O and tau are deterministic.
+ * A training forward that reported a device error (ENTMAX_ERR_TIMEOUT) left `saved` invalid: do not
+ * pass it to the backward.  While such an error is recorded and not yet read, the support-list
+ * backward does nothing (it does not read lists that may be half-written) and dQ, dK, dV are left
+ * unwritten.
  */
 ENTMAX_API size_t entmax_attn_saved_bytes(int B, int H, int L, int D);
 ENTMAX_API size_t entmax_attn_bwd_saved_workspace_size(int B, int H, int L, int D);

@@ -49,3 +49,28 @@ def test_forced_timeout_then_recovery(L, causal):
     for name, g, r in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (rQ, rK, rV)):
         err = np.max(np.abs(to64(g).reshape(w.B * w.H, L, 64)[heads] - r))
         assert err <= GRAD_TOL, (name, err)
+
+
+def test_saved_backward_after_a_forward_that_gave_up():
+    """A training forward whose waits give up leaves its support lists half-written.  While that
+    error is recorded (not yet read), the support-list backward reads none of them: the call returns,
+    the status still reports the timeout, and the context works afterwards."""
+    w = Workload(0, "timeout-train", 1, 2, 1000, 64, 1 / 8)
+    inp = make_inputs(w, seed=73)
+    Q, K, V, dO = (inp[k].cuda() for k in ("Q", "K", "V", "dO"))
+    assert E.entmax_attn_device_status() == 0
+    try:
+        E.entmax_attn_set_wait_timeout_ns(1)
+        O, tau, saved = E.entmax_attn_fwd_train(Q, K, V, None, False, 0, w.scale)
+    finally:
+        E.entmax_attn_set_wait_timeout_ns(0)
+    E.entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, None, False, 0, w.scale)
+    assert E.entmax_attn_device_status() == E.ENTMAX_ERR_TIMEOUT
+    torch.cuda.synchronize()
+    O, tau, saved = E.entmax_attn_fwd_train(Q, K, V, None, False, 0, w.scale)
+    grads = E.entmax_attn_bwd_saved(Q, K, V, tau, saved, dO, None, False, 0, w.scale)
+    assert E.entmax_attn_device_status() == 0
+    d = inputs_f64(inp, False)
+    refs = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], None, False, 0, w.scale)
+    for name, g, r in zip(("dQ", "dK", "dV"), grads, refs):
+        assert np.max(np.abs(to64(g) - r)) <= GRAD_TOL, name
