@@ -366,8 +366,8 @@ def launches_per_step(w: Workload, recompute: bool, alpha: float = 1.5, minimum:
     """The library's kernel launches in one step: the forward kernel, then the backward's kernels
     (tensor-core configurations: dq and dkdv; otherwise the support-list backward: key scan, rows,
     keys and the exact pass for unsaved rows -- which entmax_attn_bwd, given its full workspace,
-    precedes by the training forward that rebuilds the supports; with the minimum workspace its
-    recompute kernels, rows and keys)."""
+    precedes by the support extraction that lists each row's support from tau; with the minimum
+    workspace its recompute kernels, rows and keys)."""
     if not w.backward:
         return 1
     if tensor_core_backward(w, alpha):
@@ -676,7 +676,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "backward": ("entmax_attn_bwd" if recompute else "entmax_attn_bwd_saved") + (
             " (tensor-core kernels: scores recomputed, every product on tcgen05)" if tensor_core_backward(w, alpha)
             else " (recompute kernels: minimum workspace)" if args.bwd == "recompute-min"
-            else " (supports rebuilt by the training forward, then the support-list backward)" if recompute
+            else " (supports listed from tau by one score pass, then the support-list backward)" if recompute
             else " (saved supports)"),
         "fwd_ms": round(fwd_mean, 4),
         "bwd_ms": round(bwd_mean, 4),
@@ -815,7 +815,7 @@ def main() -> int:
                     help="end-to-end step: chunks of the batch whose copies overlap other chunks' kernels")
     ap.add_argument("--bwd", default="saved", choices=["saved", "recompute", "recompute-min"],
                     help="backward path: from the forward's saved supports, or entmax_attn_bwd with its full "
-                         "workspace (long rows rebuild the supports) or with the minimum one (recompute kernels)")
+                         "workspace (long rows list their supports from tau) or with the minimum one (recompute kernels)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

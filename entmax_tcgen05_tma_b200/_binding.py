@@ -264,8 +264,8 @@ def entmax_attn_fwd_gqa(Q, K, V, key_mask=None, causal=False, window=0, scale=No
 
 
 def entmax_attn_bwd_workspace_size(B: int, H: int, L: int, D: int = 64) -> int:
-    """Bytes of device workspace for entmax_attn_bwd's fastest path (long rows rebuild the forward's
-    supports in it); the minimum it accepts is bwd_min_workspace_size."""
+    """Bytes of device workspace for entmax_attn_bwd's fastest path (long rows list their supports
+    from tau in it); the minimum it accepts is bwd_min_workspace_size."""
     return int(lib.entmax_attn_bwd_workspace_size(B, H, L, D))
 
 

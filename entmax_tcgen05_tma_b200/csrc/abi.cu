@@ -96,14 +96,11 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 size_t align256b(size_t n) { return (n + 255) & ~size_t(255); }
 
 // entmax_attn_bwd's workspace: the minimum holds one float per row (the row scalar u_i); with
-// room for the forward's outputs and saved supports and the saved backward's buckets, rows that
-// are not on the tensor-core path rebuild the supports with the training forward and take the
-// support-list backward.
+// room for the saved supports and the saved backward's buckets, rows that are not on the
+// tensor-core path rebuild their supports from tau (support extraction) and take the support-list
+// backward.
 size_t bwd_min_ws_bytes(long long R) { return align256b((size_t)R * sizeof(float)); }
-size_t bwd_rebuild_ws_bytes(long long R) {
-    return align256b((size_t)R * HEAD_DIM * 2) + align256b((size_t)R * 4) + saved_support_bytes(R) +
-           saved_bwd_ws_bytes(R);
-}
+size_t bwd_rebuild_ws_bytes(long long R) { return saved_support_bytes(R) + saved_bwd_ws_bytes(R); }
 
 int check_common(const void* Q, const void* K, const void* V, int in_dtype, int causal, int window, float scale,
                  int B, int H, int L, int D) {
@@ -363,25 +360,20 @@ int bwd_impl(const void* Q, const void* K, const void* V, int in_dtype, const ui
     const bool g16 = aligned(dQ, 16) && aligned(dK, 16) && aligned(dV, 16);
     if (dense_bwd(a) && g16) return record(launch_bwd_dense(a, io, stream));
     if (!otil && g16 && ws_bytes >= bwd_rebuild_ws_bytes(R) && aligned(workspace, 256)) {
-        // Rebuild the forward's supports: the training forward (deterministic, so its tau is the
-        // caller's bit for bit) into scratch O, tau and support lists, then the support-list backward.
+        // Rebuild the forward's supports from the caller's tau: one score pass on the tensor cores,
+        // cut at tau_i, lists each row's support into the workspace; then the support-list backward.
         uint8_t* p = static_cast<uint8_t*>(workspace);
-        void* o_s = p;
-        p += align256b((size_t)R * HEAD_DIM * 2);
-        float* tau_s = reinterpret_cast<float*>(p);
-        p += align256b((size_t)R * 4);
         const SavedSupport sv = carve_saved(p, R);
         p += saved_support_bytes(R);
         rc = record(cudaMemsetAsync(sv.key_cnt, 0, sizeof(int) * (size_t)R, stream));
         if (rc) return rc;
         rc = record(cudaMemsetAsync(sv.unsaved_cnt, 0, sizeof(int), stream));
         if (rc) return rc;
-        FwdOut o{o_s, 0, tau_s, sv};
-        rc = record(launch_fwd(a, o, stream));
+        FwdOut o{nullptr, 0, const_cast<float*>(tau), sv};  // tau is only read in extraction
+        rc = record(launch_fwd(a, o, stream, true));
         if (rc) return rc;
-        io.tau = tau_s;
         io.u = nullptr;
-        io.guard = status;  // if that forward gave up, its lists hold anything: the backward does nothing
+        io.guard = status;  // if the extraction gave up, its lists hold anything: the backward does nothing
         return record(launch_bwd_saved(a, io, sv, carve_saved_bwd_ws(p, R), stream));
     }
     return record(launch_bwd(a, io, stream));

@@ -23,6 +23,11 @@
 //     streamed tiles gather them from L2 (prefetched when the candidate was listed).
 //  4. Rows with more candidates than a list holds are redone exactly by the whole CTA on CUDA
 //     cores (scores into shared memory, bisection with block reductions).
+//
+// Support extraction (the XT instantiation, for the backward that is given tau alone): pass B alone,
+// cut at the given tau_i instead of a lower bound, lists the row's support directly; its entries
+// are written as saved supports (phase 2's save step) and nothing else runs: no pass A, no tau
+// solve, no O.
 #include <cuda_bf16.h>
 #include <math.h>
 #include "common.cuh"
@@ -612,7 +617,7 @@ __device__ __noinline__ void mma_half(PipeCtl* ctl, const WaitCfg& wc, const uin
     ctl->nmma[p] = issued;  // drained at teardown if the CTA aborts (drain_half)
 }
 
-template <bool GEN>
+template <bool GEN, bool XT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const AttnArgs args, const FwdOut out) {
@@ -687,8 +692,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     const int nblk = ctl->nblk;
     const bool resident = nblk <= NBUF;
     // Streamed tiles run pass A on every other listed block only (any subset of a row bounds tau
-    // from below); pass B visits them all.
-    const int nA = resident ? nblk : (nblk + 1) / 2;
+    // from below); pass B visits them all.  Extraction runs pass B alone.
+    const int nA = XT ? 0 : resident ? nblk : (nblk + 1) / 2;
     const int njobs = resident ? nblk : nA + nblk;
 
     // per-warpgroup job counts of a streamed tile: pass-A blocks 2k (k < nA, k = g mod 2), then
@@ -746,7 +751,8 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 a0 = fmaxf(a0, cm);
             };
         };
-        if (resident) {
+        if (XT) {
+        } else if (resident) {
             for (int n = 0; n < nblk; ++n) {
                 if (live) live = warp_wait(smem_u32(&ctl->s_full[n]), 0u, &ctl->abort_flag, wc);
                 tc_fence_after();
@@ -762,15 +768,15 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 if (live) P::for_each_chunk(ctl, buf, pass_a(half_block(g, m, mA)));
             }
         }
-        {
-            RowOut& mine = rows[g * TILE + r];
-            mine.a0 = a0;
-            mine.a1 = a1;
-            mine.a2 = a2;
-            mine.a3 = a3;
-        }
-        epi_sync();
-        {
+        if (!XT) {
+            {
+                RowOut& mine = rows[g * TILE + r];
+                mine.a0 = a0;
+                mine.a1 = a1;
+                mine.a2 = a2;
+                mine.a3 = a3;
+            }
+            epi_sync();
             const RowOut& other = rows[(g ^ 1) * TILE + r];
             top4_insert(other.a0, a0, a1, a2, a3);
             top4_insert(other.a1, a0, a1, a2, a3);
@@ -779,20 +785,32 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         // scores at or below t are outside the support: the largest chunk maximum seen minus 2
         // (scaled), raised to the exact threshold of the four largest chunk maxima seen (any
-        // subset's threshold is at most tau)
-        const float t = GEN ? gen_bound(a0, a1, a2, a3, wk, am1, ex, scale)
-                            : fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
+        // subset's threshold is at most tau).  Extraction: the given tau_i over the scale, lowered
+        // by 2^-20 of itself so that no raw score whose scaled value exceeds tau_i is cut (the
+        // exact test S_ij > tau_i follows on the listed candidates); an infinite tau_i (a row with
+        // no allowed key) cuts everything.
+        float t;
+        if (XT) {
+            t = i < L ? out.tau[(size_t)bh * L + i] / scale : INFINITY;
+            if (isfinite(t)) t -= fabsf(t) * 0x1p-20f;
+        } else {
+            t = GEN ? gen_bound(a0, a1, a2, a3, wk, am1, ex, scale)
+                    : fmaxf(a0 - two_over_scale, top4_bound(a0, a1, a2, a3, c4));
+        }
 
         // ---------------- pass B: candidates s > m - 2 (scaled) into this warpgroup's partition
         float* pcv = cv + g * CAPW * TILE;
         uint16_t* pcj = cj + g * CAPW * TILE;
         int nc = 0;
         auto pass_b = [&](int e) {
-            const int j0 = (int)(blk_list[e] & ~FULL_BLOCK) * BLK;
-            return [&, e, j0](const float (&cur)[32], int c) {
+            const uint16_t ent = blk_list[e];
+            const int j0 = (int)(ent & ~FULL_BLOCK) * BLK;
+            const bool full = (ent & FULL_BLOCK) && i < L;
+            return [&, j0, full](const float (&cur)[32], int c) {
                 const int jc = j0 + c * 32;
-                const uint32_t vm = allowed(e, jc);
-                nallow += __popc(vm);
+                const uint32_t vm = full ? 0xffffffffu
+                                         : (jc < L && i < L) ? (bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
+                if (!XT) nallow += __popc(vm);  // extraction: a row with no allowed key has no hit
                 uint32_t hits = hit_bits(cur, t) & __brev(vm);
                 if (hits) {
                     stage_chunk(stage, slot, cur);
@@ -802,7 +820,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                         if (nc < CAPW) {
                             pcv[nc * TILE + r] = staged(stage, slot, q);
                             pcj[nc * TILE + r] = (uint16_t)(jc + q);
-                            if (!resident) prefetch_l2(Vh + (size_t)(jc + q) * vstep);
+                            if (!XT && !resident) prefetch_l2(Vh + (size_t)(jc + q) * vstep);
                         }
                         ++nc;
                     } while (hits);
@@ -811,8 +829,13 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         };
         if (resident) {
             tc_fence_after();
-            if (live) {
-                for (int n = 0; n < nblk; ++n) for_half_block(ctl, n, g, pass_b(n));
+            for (int n = 0; n < nblk && live; ++n) {
+                if (XT) {  // no pass A waited on the blocks
+                    live = warp_wait(smem_u32(&ctl->s_full[n]), 0u, &ctl->abort_flag, wc);
+                    tc_fence_after();
+                    if (!live) break;
+                }
+                for_half_block(ctl, n, g, pass_b(n));
             }
         } else {
             const int mA = g ? mA1 : mA0, mB = g ? mB1 : mB0;
@@ -831,7 +854,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const bool aborted = P::aborted(ctl);
-    const bool v_staged = resident && !aborted;
+    const bool v_staged = !XT && resident && !aborted;
 
     // V blocks of a resident tile into the (now idle) ring, overlapping phase 2
     if (warp == WARP_PRODUCER && lane == 0 && v_staged) {
@@ -842,8 +865,37 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
     }
 
+    // ---------------- extraction: the support is every candidate with S_ij > tau_i; written as
+    // phase 2 writes it (a row past a partition's list is marked unsaved), two threads per row
+    if (XT && !aborted && tid < NUM_EPI) {
+        const int r = (warp << 4) | (lane >> 1), h = lane & 1;
+        const int i = i0 + r;
+        const RowOut s0 = rows[r], s1 = rows[TILE + r];
+        int mode = 0;  // 0: listed (none when no key is allowed), 2: unsaved (a partition overflowed), 3: no row
+        if (i >= L) mode = 3;
+        else if (s0.ovf | s1.ovf) mode = 2;
+        const int nh = mode == 0 ? (h == 0 ? s0.n : s1.n) : 0;
+        float* pcv = cv + h * CAPW * TILE;
+        uint16_t* pcj = cj + h * CAPW * TILE;
+        const float tau_i = nh > 0 ? out.tau[(size_t)bh * L + i] : 0.f;
+        int sn = 0;
+        for (int k = 0; k < nh; ++k) {
+            const float d = fmaf(scale, pcv[k * TILE + r], -tau_i);  // S_ij - tau_i (scaled)
+            const uint16_t j = pcj[k * TILE + r];
+            if (d > 0.f) {
+                // h_ij = sqrt(p_ij) (alpha 1.5) or b_ij = am1 (S_ij - tau_i) (general alpha)
+                pcv[sn * TILE + r] = GEN ? am1 * d : 0.5f * d;
+                pcj[sn * TILE + r] = j;
+                ++sn;
+            }
+        }
+        supp_cnt[h * TILE + r] = sn;
+        __syncwarp();
+        save_row_support<GEN>(out.save, cv, cj, supp_cnt, r, h, mode, (size_t)bh * L, (size_t)bhk * L, i, L);
+    }
+
     // ---------------- phase 2: tau per row, two threads per row (one per partition)
-    if (!aborted && tid < NUM_EPI) {
+    if (!XT && !aborted && tid < NUM_EPI) {
         const int r = (warp << 4) | (lane >> 1), h = lane & 1;
         const int i = i0 + r;
         const RowOut s0 = rows[r], s1 = rows[TILE + r];
@@ -1073,7 +1125,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     if (v_staged && warp == WARP_PRODUCER && lane == 0 && P::aborted(ctl)) wait_drain(smem_u32(vbar), 0u);
 
     // ---------------- phase 4: exact redo of overflowed rows
-    if (!P::aborted(ctl)) {
+    if (!XT && !P::aborted(ctl)) {
         for (int wd = 0; wd < TILE / 32; ++wd) {
             uint32_t mask = redo[wd];  // uniform across the CTA
             while (mask) {
@@ -1117,7 +1169,7 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 
 size_t fwd_smem_bytes() { return SMEM_BYTES; }
 
-cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream) {
+cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream, bool extract) {
     CUtensorMap mq, mk, mv;
     cudaError_t e = make_tile_map(&mq, a.Q, a.layout, a.B, a.H, a.L, TILE);
     if (e != cudaSuccess) return e;
@@ -1125,14 +1177,17 @@ cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     e = make_tile_map(&mv, a.V, a.layout, a.B, a.Hkv, a.L, BLK);
     if (e != cudaSuccess) return e;
+    using Fn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const AttnArgs, const FwdOut);
+    // [extract][generic alpha]; shared-memory attribute slots 0, 4 (forward), 12, 14 (extraction)
+    static const Fn fns[2][2] = {{entmax_fwd_kernel<false, false>, entmax_fwd_kernel<true, false>},
+                                 {entmax_fwd_kernel<false, true>, entmax_fwd_kernel<true, true>}};
+    static const int slots[2][2] = {{0, 4}, {12, 14}};
     const bool gen = generic_alpha(a);
-    const void* kfn = gen ? reinterpret_cast<const void*>(entmax_fwd_kernel<true>)
-                          : reinterpret_cast<const void*>(entmax_fwd_kernel<false>);
-    e = ensure_smem_attr(kfn, SMEM_BYTES, gen ? 4 : 0);
+    const Fn f = fns[extract][gen];
+    e = ensure_smem_attr(reinterpret_cast<const void*>(f), SMEM_BYTES, slots[extract][gen]);
     if (e != cudaSuccess) return e;
     dim3 grid((a.L + TILE - 1) / TILE, a.B * a.H);
-    if (gen) entmax_fwd_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, a, o);
-    else entmax_fwd_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, a, o);
+    f<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, a, o);
     return cudaGetLastError();
 }
 

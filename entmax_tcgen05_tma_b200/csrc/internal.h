@@ -107,7 +107,9 @@ cudaError_t launch_bwd_saved(const AttnArgs& a, const BwdIO& io, const SavedSupp
 // Tensor map over a [B*H, L, 64] bf16 tensor, boxes of box_rows rows, 128-byte swizzle.
 cudaError_t make_tile_map(CUtensorMap* map, const void* base, int layout, int B, int nh, int L, int box_rows);
 
-cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);
+// Gather forward (fwd.cu).  extract: support extraction for a backward given tau alone -- o.tau is
+// read (the caller's tau), o.save receives the support lists, o.O, o.otil and o.rsum are unused.
+cudaError_t launch_fwd(const AttnArgs& a, const FwdOut& o, cudaStream_t stream, bool extract = false);
 // Softmax forward (fwd_softmax.cu): writes O and tau = log sum_j exp(S_ij), and O in fp32 into o.otil
 // when given; o.save and o.rsum unused.
 cudaError_t launch_fwd_softmax(const AttnArgs& a, const FwdOut& o, cudaStream_t stream);

@@ -102,11 +102,11 @@ ENTMAX_API int entmax_attn_fwd(const void* Q, const void* K, const void* V, int 
 /* Bytes of device workspace for entmax_attn_bwd's fastest path; 0 when B, H or L is 0.
  * The minimum entmax_attn_bwd accepts is one float per query row (the row scalar u_i passed from
  * the dQ kernel to the dK/dV kernel), rounded up to 256 bytes, and that is what this returns for
- * L <= 512 (every such row takes the tensor-core backward).  For L > 512 it returns room for the
- * forward's outputs, its saved supports and the support-list backward's buckets (about 1.2 KB per
- * query row): given that much, 256-byte aligned, rows off the tensor-core path rebuild the supports
- * with the training forward and take the support-list backward instead of recomputing each row's
- * support on CUDA cores (at workload 4, B = 4, H = 12, L = 4096: about 0.8 ms instead of 1.6). */
+ * L <= 512 (every such row takes the tensor-core backward).  For L > 512 it returns room for
+ * support lists and the support-list backward's buckets (about 1.1 KB per query row): given that
+ * much, 256-byte aligned, rows off the tensor-core path rebuild their supports from tau in one
+ * score pass on the tensor cores (support extraction) and take the support-list backward, instead
+ * of recomputing each row's support on CUDA cores in every kernel of the backward. */
 ENTMAX_API size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D);
 
 /*
@@ -121,11 +121,10 @@ ENTMAX_API size_t entmax_attn_bwd_workspace_size(int B, int H, int L, int D);
  *   workspace    device buffer of at least one float per query row (rounded up to 256 bytes),
  *                16-byte aligned, owned by the caller; its contents need no initialisation.  With
  *                entmax_attn_bwd_workspace_size(B,H,L,D) bytes, 256-byte aligned, long rows take the
- *                faster path described there: the supports (and tau, bit for bit the forward's)
- *                are recomputed by the training forward into the workspace; the caller's tau then
- *                serves only the tensor-core rows.  On that path a device error recorded before or
- *                during the call (see entmax_attn_device_status) leaves dQ, dK, dV unwritten: the
- *                support lists of a forward that gave up are not read.
+ *                faster path described there: each row's support {j : S_ij > tau_i} is listed
+ *                into the workspace from the caller's tau.  On that path a device error recorded
+ *                before or during the call (see entmax_attn_device_status) leaves dQ, dK, dV
+ *                unwritten: the support lists of an extraction that gave up are not read.
  * fp32 inputs additionally use stream-ordered temporaries (cudaMallocAsync) for their bf16
  * copies; bf16 inputs allocate nothing.
  */

@@ -251,6 +251,39 @@ def test_recompute_backward_both_workspaces(causal):
         assert torch.allclose(a, b, atol=1e-4, rtol=0), (name, float((a - b).abs().max()))
 
 
+EXTRACT_CASES = [
+    # B, H, L, scale, causal, window, len_range: streamed tiles with padding; causal; a causal
+    # window of 200 keys (tiles of at most three key blocks, scored once); near-uniform rows whose
+    # supports overflow the lists (every row takes the unsaved-row kernel)
+    (2, 2, 1100, 1 / 8, False, 0, (600, 1100)),
+    (1, 3, 900, 2 / 8, True, 0, None),
+    (2, 2, 1000, 1 / 8, True, 200, None),
+    (1, 2, 700, 1e-3, False, 0, None),
+]
+
+
+@pytest.mark.parametrize("B,H,L,scale,causal,window,lens", EXTRACT_CASES)
+def test_support_extraction_backward(B, H, L, scale, causal, window, lens):
+    """entmax_attn_bwd with its full workspace lists each row's support from the caller's tau (one
+    score pass cut at tau_i) and runs the support-list backward.  Against the oracle, and against
+    the training path (entmax_attn_fwd_train + entmax_attn_bwd_saved), whose lists hold the same
+    supports: the two differ only by the rounding of sqrt(p_ij) (one fused step from tau against
+    the forward's two from the row max) and by the atomic order of the dK, dV sums."""
+    w = Workload(0, "extract", B, H, L, 64, scale, causal, window, lens)
+    inp = make_inputs(w, seed=41 + L + window)
+    d = inputs_f64(inp, False)
+    km = _mask_np(inp)
+    O, tau, dev = _gpu_fwd(inp, w)
+    got = _gpu_bwd(dev, tau, inp["dO"], w)
+    _, tau_t, saved = _gpu_train(inp, w)
+    assert torch.equal(tau, tau_t)
+    refs = orc.attn_bwd(d["Q"], d["K"], d["V"], d["dO"], km, causal, window, w.scale)
+    for name, a, b, r in zip(("dQ", "dK", "dV"), got, saved, refs):
+        assert np.max(np.abs(to64(a) - r)) <= GRAD_TOL, name
+        bound = 1e-5 * max(1.0, float(b.abs().max()))
+        assert float((a - b).abs().max()) <= bound, (name, float((a - b).abs().max()))
+
+
 def test_one_hot_rows():
     """A key aligned with every query and far above the rest takes all the weight."""
     w = Workload(0, "onehot", 1, 1, 256, 64, 1.0)

@@ -26,7 +26,7 @@ def _run(w: Workload, seed: int):
     km = None if inp["key_mask"] is None else inp["key_mask"].cuda()
     O, tau = E.entmax_attn_fwd(Q, K, V, km, w.causal, w.window, w.scale)
     # the minimum workspace: entmax_attn_bwd then runs the kernels the allocation-free entry point
-    # runs at every length (with the full workspace, long rows rebuild the forward's supports)
+    # runs at every length (with the full workspace, long rows list their supports from tau)
     ws = torch.empty(E.bwd_min_workspace_size(w.B, w.H, w.L), dtype=torch.uint8, device="cuda")
     ref = E.entmax_attn_bwd(Q, K, V, tau, dO, km, w.causal, w.window, w.scale, workspace=ws)
     got = E.entmax_attn_bwd_noalloc(Q, K, V, tau, dO, km, w.causal, w.window, w.scale)
