@@ -153,6 +153,21 @@ __device__ __forceinline__ float masked_max(const float (&v)[32], uint32_t vm) {
     return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
+// v[q] for a thread-dependent q in [0, 32): a tree of selects on the bits of q, 16 + 8 + 4 + 2 + 1 of them
+// (no indexed register access, no shared memory).
+__device__ __forceinline__ float pick32(const float (&v)[32], int q) {
+    float a[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) a[k] = (q & 16) ? v[16 + k] : v[k];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = (q & 8) ? a[8 + k] : a[k];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = (q & 4) ? a[4 + k] : a[k];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) a[k] = (q & 2) ? a[2 + k] : a[k];
+    return (q & 1) ? a[1] : a[0];
+}
+
 // Reads chunks 2 half and 2 half + 1 of the (resident) score buffer of block n and calls f(v, c).
 template <class F>
 __device__ __forceinline__ void for_half_block(const PipeCtl* ctl, int n, int half, F&& f) {
@@ -812,7 +827,19 @@ entmax_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                                          : (jc < L && i < L) ? (bits[jc >> 5] & range_bits(jc, rlo, rhi)) : 0u;
                 if (!XT) nallow += __popc(vm);  // extraction: a row with no allowed key has no hit
                 uint32_t hits = hit_bits(cur, t) & __brev(vm);
-                if (hits) {
+                if (XT) {
+                    // the support is sparse (about one hit per chunk that has one): each hit's score
+                    // is picked from registers, with no staging of the chunk through shared memory
+                    while (hits) {
+                        const int q = __clz(hits);
+                        hits &= ~(0x80000000u >> q);
+                        if (nc < CAPW) {
+                            pcv[nc * TILE + r] = pick32(cur, q);
+                            pcj[nc * TILE + r] = (uint16_t)(jc + q);
+                        }
+                        ++nc;
+                    }
+                } else if (hits) {
                     stage_chunk(stage, slot, cur);
                     do {
                         const int q = __clz(hits);
