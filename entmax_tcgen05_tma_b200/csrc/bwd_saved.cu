@@ -7,8 +7,9 @@
 // General alpha (p = b^(1/am1), b = am1 (S - tau), am1 = alpha - 1; the pages' entmax_bisect
 // routine): the Jacobian has the same form with the weight w_ij = p_ij^(2 - alpha) = b^(1/am1 - 1) in
 // place of sp_ij (at alpha 1.5, w = b = sqrt(p)).  The saved lists hold b_ij in both cases.
-// The supports {(j, b_ij)} come from the training forward instead of a recomputed score pass, so
-// no QK^T is formed again: the work is proportional to the number of support entries.
+// The supports {(j, b_ij)} come from the training forward (or, for a backward given tau alone, from
+// the support extraction of fwd.cu), so these kernels form no QK^T: their work is proportional to
+// the number of support entries.
 //
 //  1. key_scan:   per head, exclusive scan of the per-key support counts -> bucket offsets.
 //  2. rows:       four query rows per warp, eight lanes per row (each lane owns eight dimensions, so

@@ -43,6 +43,16 @@ def test_workspace_size():
     assert E.entmax_attn_bwd_workspace_size(0, 12, 128) == 0
     n = E.entmax_attn_bwd_workspace_size(4, 12, 4096)
     assert n >= 4 * 12 * 4096 * 4 and n % 256 == 0
+    # rows of at most 512 keys take the tensor-core backward: the minimum (one float per row) is all
+    # it asks for; longer rows get room for the support lists (the saved buffer) and the
+    # support-list backward's buckets
+    for B, H, L in ((2, 3, 1), (4, 12, 512), (1, 1, 300)):
+        assert E.entmax_attn_bwd_workspace_size(B, H, L) == E.bwd_min_workspace_size(B, H, L)
+    for B, H, L in ((4, 12, 4096), (1, 2, 513), (3, 5, 16384)):
+        full = E.entmax_attn_bwd_workspace_size(B, H, L)
+        assert full >= E.entmax_attn_saved_bytes(B, H, L) + E.entmax_attn_bwd_saved_workspace_size(B, H, L)
+        assert full > E.bwd_min_workspace_size(B, H, L) and full % 256 == 0
+        assert full < 1300 * B * H * L  # about 1.1 KB per query row
 
 
 P = 0x10000  # fake, 16-byte aligned device address: never dereferenced by these calls
