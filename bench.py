@@ -603,6 +603,16 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         extras = {str(k): extra_workload(args, WORKLOADS[k], dev, world, flush, peaks) for k in (3, 5)}
         # softmax attention (alpha = 1, the pages' alpha -> 1 branch) on the headline shape
         extras["softmax_4"] = extra_workload(args, WORKLOADS[4], dev, world, flush, peaks, alpha=1.0)
+        # the backward from tau alone on the headline shape: entmax_attn_bwd with its full workspace
+        # (support extraction, then the support-list backward), after entmax_attn_fwd
+        try:
+            rec = extra_workload(argparse.Namespace(**{**vars(args), "bwd": "recompute"}), WORKLOADS[4], dev, world,
+                                 flush, peaks)
+            rec["backward"] = "entmax_attn_bwd, full workspace (support extraction, then the support-list backward)"
+            rec["bwd_vs_saved"] = round(rec["bwd_ms"] / statistics.mean(bwd_ms), 3)
+        except Exception as exc:  # recorded, not fatal: the headline line still prints
+            rec = {"error": "%s: %s" % (type(exc).__name__, exc)}
+        extras["recompute_bwd_4"] = rec
 
     if rank != 0:
         return None
